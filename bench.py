@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the beam-decode hot path; prints ONE JSON line.
+
+A step is one whole beam decode of a batch: xgr_begin, then for every decode
+step s: staged attention (xgr_decode_step), the valid-path mask
+(xgr_build_mask) and the masked top-K with rewiring (xgr_beam_select).  The
+default workload is the 128x128 candidate pool (8 requests, 1024-token
+prompts, beam width = top-K = 128, 3 steps, Hq=16, Hkv=4, D=128, V=8192, 1M
+valid 3-token items), logits-mode scores.
+
+metric: beam-candidates/s = sum over decode steps of (requests x live beams x K)
+        per second of device time (L2 flushed before every timed step).
+--impl reference: the CPU oracle timed on the host cores, same metric.
+Multi-GPU (torchrun): every rank decodes its own batch (weak scaling, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "beam-candidates/s per decode step"
+UNIT = "candidates/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="xgr", choices=["xgr", "reference"])
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--scores", default="logits", choices=["logits", "logprob"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w, scores):
+    return {
+        "workload": f"{w.name}: B={w.B} requests, prompt {w.prompt[0]}-{w.prompt[1]} tokens, "
+                    f"BW={w.BW}, top-K={w.K}, {w.S} steps, Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, "
+                    f"V={w.V}, {w.n_items} valid items",
+        "scores": scores,
+        "l2": "flushed (256 MiB write) before every timed step; step time from CUDA events",
+    }
+
+
+def candidates_per_decode(w):
+    return sum(w.candidates_per_step(s) for s in range(w.S))
+
+
+# ---------------------------------------------------------------- clocks
+
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = [l.strip().split(", ") for l in open(self.f.name) if l.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = max(mx, float(r[1]))
+                for n, v in zip(names, r[3:7]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_decode_sample(w, items, sorted_items, requests, scores_mode):
+    """One full oracle decode of the given requests; returns (seconds, candidates)."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    u16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    mode = "logprob" if scores_mode == "logprob" else "logits"
+    inputs = []
+    for s in range(w.S):
+        q, kn, vn = workloads.step_qkv(w, s, "cpu")
+        sc = (workloads.step_logprobs if mode == "logprob" else workloads.step_logits)(w, s, "cpu")
+        inputs.append((q, kn, vn, sc.numpy()))
+    kvs = {r: workloads.shared_kv(w, w.shared_id(r), "cpu") for r in requests}
+    t0 = time.perf_counter()
+    cands = 0
+    for r in requests:
+        dec = oracle.BeamDecode(sorted_items, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V, mode=mode)
+        k, v = kvs[r]
+        dec.begin(u16(k), u16(v))
+        for s in range(w.S):
+            q, kn, vn, sc = inputs[s]
+            cands += dec.n_live * w.K
+            dec.attention(s, q[r], kn[r], vn[r])
+            m = dec.mask(s)
+            dec.select(s, sc[r], m)
+    return time.perf_counter() - t0, cands
+
+
+def cpu_baseline(w, items, scores_mode, budget_s=20.0):
+    import oracle
+    si = oracle.SortedItems(items, w.V)
+    secs, cands = oracle_decode_sample(w, items, si, [0], scores_mode)
+    reqs = [0]
+    r = 1
+    while secs < budget_s / 2 and r < w.B:          # grow the sample while it stays short
+        t, c = oracle_decode_sample(w, items, si, [r], scores_mode)
+        secs += t
+        cands += c
+        reqs.append(r)
+        r += 1
+    return {"value": cands / secs, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"full {w.S}-step decode of {len(reqs)} of {w.B} requests "
+                      f"({cands} candidates in {secs:.2f} s)"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import workloads
+    items = workloads.items(w)
+    si = oracle.SortedItems(items, w.V)
+    for _ in range(args.warmup):
+        oracle_decode_sample(w, items, si, [0], args.scores)
+    secs, cands = 0.0, 0
+    for i in range(args.steps):
+        t, c = oracle_decode_sample(w, items, si, [i % w.B], args.scores)
+        secs += t
+        cands += c
+    value = cands / secs
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": workload_config(w, args.scores),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: full {w.S}-step decode of one request"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def algorithmic(w, s, logits_mode, nnz_step):
+    """Required bytes / flops of the attention and the selection of step s >= 1."""
+    B, BW, Hq, Hkv, D, V = w.B, w.BW, w.Hq, w.Hkv, w.D, w.V
+    P = sum(int(x) for x in __import__("workloads").prompt_lengths(w)) / w.n_shared
+    att_bytes = (2 * B * Hkv * P * D * 2            # shared K,V read once per request
+                 + 2 * B * BW * Hkv * s * D * 2     # distinct earlier unshared tokens
+                 + 2 * B * BW * Hkv * D * 2 * 2     # this step's k/v: read + append
+                 + 2 * B * BW * Hq * D * 2          # q read + O write
+                 + B * BW * Hq * 4)                 # LSE
+    att_flops = 4.0 * B * BW * Hq * D * (P + s + 1)
+    sel_bytes = (B * BW * V * 4 if logits_mode else nnz_step * 4) + nnz_step * 4 + B * BW * 16
+    return att_bytes, att_flops, sel_bytes
+
+
+def run_gpu(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import workloads
+    from shared_prefix_decode_xattention_b200 import xgr
+    from shared_prefix_decode_xattention_b200.session import Session, config_for
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(dev))
+
+    items = workloads.items(w)
+    logits_mode = args.scores == "logits"
+    flags = xgr.XGR_SCORES_LOGITS if logits_mode else xgr.XGR_SCORES_LOGPROB
+    sess = Session(config_for(w), dev)
+    sess.build_trie(items)
+    for r in range(w.B):
+        k, v = workloads.shared_kv(w, w.shared_id(r), dev)
+        sess.prefill(r, w.shared_id(r), k, v)
+    del k, v
+    inputs = []
+    for s in range(w.S):
+        q, kn, vn = workloads.step_qkv(w, s, dev)
+        sc = (workloads.step_logits if logits_mode else workloads.step_logprobs)(w, s, dev)
+        inputs.append((q, kn, vn, sc))
+    out = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=dev)
+    par = torch.empty((w.B, w.BW), dtype=torch.int32, device=dev)
+    tok = torch.empty_like(par)
+    cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
+    nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sess.begin(w.B, stream)   # plan once (setup)
+    torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def decode(timers=None, inp=inputs, host=None):
+        sess.begin(w.B, stream)
+        for s in range(w.S):
+            q, kn, vn, sc = inp[s]
+            if host is not None:                      # end-to-end: host -> device inputs
+                hq, hk, hv, hs = host[s]
+                q.copy_(hq, non_blocking=True)
+                kn.copy_(hk, non_blocking=True)
+                vn.copy_(hv, non_blocking=True)
+                sc.copy_(hs, non_blocking=True)
+            if timers is not None and s >= 1:
+                timers["att"][-1][s][0].record(stream)
+            sess.decode_step(s, q, kn, vn, out, lse, stream)
+            if timers is not None and s >= 1:
+                timers["att"][-1][s][1].record(stream)
+            m = sess.build_mask(s, stream)
+            if timers is not None and s >= 1:
+                timers["sel"][-1][s][0].record(stream)
+            sess.beam_select(s, sc, flags, m, par, tok, cum, nout, stream)
+            if timers is not None and s >= 1:
+                timers["sel"][-1][s][1].record(stream)
+            if host is not None:
+                hp, ht, hc, hn = host[w.S + s]
+                hp.copy_(par, non_blocking=True)
+                ht.copy_(tok, non_blocking=True)
+                hc.copy_(cum, non_blocking=True)
+                hn.copy_(nout, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        decode()
+    torch.cuda.synchronize()
+    if sess.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    # timed region
+    timers = {"att": [], "sel": []}
+    starts, ends = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
+    clk = Clocks(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        timers["att"].append({s: (ev(), ev()) for s in range(1, w.S)})
+        timers["sel"].append({s: (ev(), ev()) for s in range(1, w.S)})
+        starts[i].record(stream)
+        decode(timers)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.stop() if clk else None
+    total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    att_ms = [t[s][0].elapsed_time(t[s][1]) for t in timers["att"] for s in t]
+    sel_ms = [t[s][0].elapsed_time(t[s][1]) for t in timers["sel"] for s in t]
+    n_live = nout.cpu().numpy()
+    cands = candidates_per_decode(w) * args.steps * world
+    value = cands / (total_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host = []
+        h2d = d2h = 0
+        for s in range(w.S):
+            hs = [t.cpu().pin_memory() for t in inputs[s]]
+            host.append(hs)
+            h2d += sum(t.numel() * t.element_size() for t in hs)
+        for s in range(w.S):
+            hs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (par, tok, cum, nout)]
+            host.append(hs)
+            d2h += sum(t.numel() * t.element_size() for t in hs)
+        dev_in = [tuple(torch.empty_like(t) for t in inputs[s]) for s in range(w.S)]
+        for _ in range(2):
+            decode(inp=dev_in, host=host)
+        torch.cuda.synchronize()
+        e_s, e_e = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            e_s[i].record(stream)
+            decode(inp=dev_in, host=host)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e))
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": cands / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    status = sess.device_status()
+
+    # ---- roofline of the dominant call (attention vs selection at steps >= 1)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    tf = peaks.get("bf16_tflops", 1590.0)
+    src = "of measured" if peaks else "of fallback"
+    # nnz of the sparse masks: expected children per beam (measured once on host)
+    nnz_step = int(round(w.B * w.BW * min(w.V, w.n_items / w.V))) if w.V else 0
+    att_bytes, att_flops, sel_bytes = algorithmic(w, 1, logits_mode, nnz_step)
+    att_avg = statistics.mean(att_ms) / 1e3
+    sel_avg = statistics.mean(sel_ms) / 1e3
+    if att_avg >= sel_avg:
+        achieved = att_flops / att_avg / 1e12
+        roof = {"kernel": "xgr_decode_step (staged attention, steps >= 1)", "bound": "tensor",
+                "achieved": achieved, "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
+                "peak_source": f"bf16_tflops burst {src}", "traffic": None,
+                "algorithmic_per_launch": att_flops, "launch_ms": att_avg * 1e3,
+                "hbm_gbs_required_bytes": att_bytes / att_avg / 1e9}
+    else:
+        achieved = sel_bytes / sel_avg / 1e9
+        roof = {"kernel": "xgr_beam_select (steps >= 1)", "bound": "hbm", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": f"hbm_gbs {src}", "traffic": None,
+                "algorithmic_per_launch": sel_bytes, "launch_ms": sel_avg * 1e3}
+
+    launches_per_decode = 1 + sum((2) + (0 if s == 0 else 2) + 2 for s in range(w.S))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w, args.scores), global_batch=w.B * world,
+                           parallelism=f"dp{world}" if world > 1 else "single"),
+            "roofline": roof,
+            "step_breakdown_ms": {"attention_step_ge1": att_avg * 1e3,
+                                  "select_step_ge1": sel_avg * 1e3},
+            "gpu_launches": launches_per_decode * args.steps,
+            "device_status": status, "n_live_last": int(n_live.min()) if n_live.size else 0}
+    if e2e:
+        line["e2e"] = e2e
+    if clocks:
+        line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, items, args.scores)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    sess.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    import workloads
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

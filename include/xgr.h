@@ -1,0 +1,215 @@
+/*
+ * xgr.h -- C ABI of the B200 beam-decode hot path (libxgr.so).
+ *
+ * What the library computes, per the xGR page ("xGR: Efficient Generative
+ * Recommendation Serving at Scale"):
+ *   2.1 xAttention  The KV cache is split in two.  The Shared part holds the
+ *                   prompt (user history), computed once at prefill and read
+ *                   once per request for all beams.  The Unshared part holds
+ *                   only the tokens generated at each decode step, managed
+ *                   token by token (no block padding, no block copy when
+ *                   beams fork).  Attention runs in three stages: Shared and
+ *                   Unshared each produce local scores with max/sum
+ *                   statistics; a Merging stage combines them by online
+ *                   softmax.  The Unshared cache is updated in place through
+ *                   direct indices, without write-before-read hazards.
+ *   2.2 xBeam       Candidates are filtered by masks built from a pre-built
+ *                   vocabulary of valid items: dense, pre-generated masks for
+ *                   the first step, sparse masks afterwards.  The top
+ *                   candidates are chosen with early termination (a global
+ *                   threshold cuts every beam's sorted candidate list).
+ * The same split-KV attention serves prefix-homogeneous LLM batches (several
+ * requests sharing one prompt prefix plus a private suffix), the batching the
+ * Feather page argues for ("Requests of the same feather must flock
+ * together", "Methodology").
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller allocates every device buffer, including the one
+ *    workspace handed to xgr_create; the library allocates no device memory.
+ *    The context (host struct) is owned by the library and freed by
+ *    xgr_destroy.
+ *  - Pointers named d_* are device pointers, h_* host pointers.  Device
+ *    pointers must be 16-byte aligned.  bf16 means IEEE bfloat16 bits.
+ *  - Streams: hot calls (xgr_decode_step, xgr_build_mask, xgr_beam_select,
+ *    xgr_begin when its plan is unchanged, xgr_get_sequences) only enqueue
+ *    kernels on the given stream; they never synchronise the host.  Setup
+ *    calls (xgr_create, xgr_build_trie, xgr_prefill_kv, xgr_begin after a
+ *    prefill) may synchronise.  xgr_device_status synchronises.
+ *  - Errors: host-side validation returns a negative xgr_status at once and
+ *    enqueues nothing.  Faults found on the device (an index out of range, a
+ *    NaN score, a capacity overflow, a token outside the vocabulary) never
+ *    trap: the kernel records a code in the device status word, skips the
+ *    faulty element and carries on; xgr_device_status reports it.
+ *  - Row layout: request r, beam b lives at row r * BW + b of every
+ *    [B][BW]... array; beams b >= n_live(r) are dead: their attention output
+ *    is 0 with LSE -inf, their selection slots hold parent -1, token -1,
+ *    cum -inf.
+ */
+#ifndef XGR_H_
+#define XGR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *xgr_stream_t;
+
+typedef struct xgr_ctx xgr_ctx;
+typedef int32_t xgr_status;
+
+enum {
+    XGR_OK = 0,
+    XGR_ERR_ARG = -1,           /* null/misaligned pointer, unknown flag or kind */
+    XGR_ERR_SHAPE = -2,         /* a size inconsistent with the config */
+    XGR_ERR_CAPACITY = -3,      /* more than a capacity fixed at xgr_create */
+    XGR_ERR_STATE = -4,         /* call out of order (e.g. step != current step) */
+    XGR_ERR_CUDA = -5,          /* a CUDA runtime call failed */
+    XGR_ERR_DEVICE = -6,        /* the device status word was non-zero */
+    XGR_ERR_UNIMPLEMENTED = -7  /* configuration not supported by this build */
+};
+
+/* Device status word bits (xgr_device_status). */
+enum {
+    XGR_DEV_NAN = 1,            /* NaN among the scores or cumulative scores read */
+    XGR_DEV_INDEX = 2,          /* ancestry slot / trie node out of range */
+    XGR_DEV_MASK = 4,           /* a mask token that is not a child in the trie, or >= V */
+    XGR_DEV_CAPACITY = 8        /* mask rows exceeded the CSR capacity */
+};
+
+/* Score input of xgr_beam_select. */
+enum {
+    XGR_SCORES_LOGPROB = 0,     /* fp32 log-probs; score = fp32(cum + lp), bit-exact contract */
+    XGR_SCORES_LOGITS = 1       /* fp32 logits; lp = logit - logsumexp(row) over the full vocabulary */
+};
+
+/* KV kinds of xgr_prefill_kv. */
+enum {
+    XGR_KV_SHARED = 0,          /* prompt / shared prefix, stored once per shared id */
+    XGR_KV_SUFFIX = 1           /* a request's private prefix continuation (beam width 1 use) */
+};
+
+enum { XGR_MASK_DENSE = 0, XGR_MASK_CSR = 1 };
+
+typedef struct {
+    int32_t max_requests;   /* B: requests per batch */
+    int32_t max_shared;     /* number of shared ids (distinct prompt prefixes) */
+    int64_t kv_tokens;      /* capacity of the prompt KV store, in tokens (all ids and suffixes) */
+    int32_t beam_width;     /* BW (1..1024) */
+    int32_t top_k;          /* K >= BW: candidates kept per beam before the global cut */
+    int32_t steps;          /* S decode steps == item length (1..8) */
+    int32_t n_q_heads;      /* Hq */
+    int32_t n_kv_heads;     /* Hkv, divides Hq (query head h reads kv head h / (Hq/Hkv)) */
+    int32_t head_dim;       /* D: 64 or 128 */
+    int32_t vocab;          /* V: tokens per level (0: no selection, attention only) */
+    int64_t max_items;      /* trie capacity, items */
+    int32_t max_fanout;     /* bound on the children of any node below the root (0: V) */
+    int32_t max_partials;   /* partial-attention slots per row for split-K (0: 8) */
+} xgr_config;
+
+/* A mask as produced by xgr_build_mask: views into the workspace, valid until
+ * the next xgr_build_mask.  Dense: bits[w] bit j set <=> token 32w+j valid
+ * (shared by every live beam of step 0).  CSR: the valid next tokens of row
+ * r*BW+b are cols[row_ptr[row] .. row_ptr[row+1]), ascending; row_ptr lives
+ * on the device, so nnz = row_ptr[n_rows] is known to kernels only. */
+typedef struct {
+    int32_t kind;
+    int32_t step;
+    const uint32_t *bits;
+    int32_t n_words;
+    int32_t n_rows;
+    const int32_t *row_ptr;
+    const int32_t *cols;
+    int64_t cols_capacity;
+} xgr_mask;
+
+/* Bytes of device workspace a context with this config needs (256-byte
+ * aligned regions: prompt KV store, Unshared pool, beam state, trie, masks,
+ * selection and split-K scratch).  Returns XGR_ERR_ARG / XGR_ERR_SHAPE for an
+ * invalid config. */
+xgr_status xgr_workspace_bytes(const xgr_config *cfg, size_t *bytes);
+
+/* Creates a context over a caller-owned device workspace of at least
+ * xgr_workspace_bytes bytes (256-byte aligned), on the current device.
+ * The workspace must outlive the context. */
+xgr_status xgr_create(const xgr_config *cfg, void *d_workspace, size_t bytes, xgr_ctx **out);
+xgr_status xgr_destroy(xgr_ctx *ctx);
+const char *xgr_status_string(xgr_status s);
+
+/* Builds the item trie (xGR 2.2 "Valid-path constraint") from h_items
+ * [n_items][item_len] int32 (host; any order; duplicates are merged), and the
+ * pre-generated dense mask of step 0.  item_len must equal cfg.steps; tokens
+ * must lie in [0, V).  Synchronous (setup).  XGR_ERR_CAPACITY when n_items >
+ * max_items or a node below the root has more than max_fanout children. */
+xgr_status xgr_build_trie(xgr_ctx *ctx, const int32_t *h_items, int64_t n_items, int32_t item_len);
+
+/* Loads prompt KV (xGR 2.1 "Separate KV cache": computed once at prefill).
+ * d_k, d_v: bf16 [Hkv][len][D] (device).  Copied into the library's store;
+ * the caller may free them after the call returns (the copy is complete on
+ * return: this call synchronises the stream).
+ *  kind XGR_KV_SHARED: links request -> shared_id; when d_k is non-null it
+ *    (re)loads that id's prefix, when null the id must already be loaded.
+ *  kind XGR_KV_SUFFIX: loads request's private suffix (shared_id ignored).
+ * XGR_ERR_CAPACITY when the store (kv_tokens) is full. */
+xgr_status xgr_prefill_kv(xgr_ctx *ctx, int32_t request, int32_t shared_id,
+                          const void *d_k, const void *d_v, int32_t len, int32_t kind,
+                          xgr_stream_t stream);
+
+/* Forgets every prefilled prefix and suffix (the store is reused). */
+xgr_status xgr_reset_kv(xgr_ctx *ctx);
+
+/* Starts a beam decode of requests 0..n_requests-1: one live beam per request
+ * with cumulative score 0 at the trie root.  Re-plans the attention work when
+ * KV was prefilled since the last plan (then it synchronises). */
+xgr_status xgr_begin(xgr_ctx *ctx, int32_t n_requests, xgr_stream_t stream);
+
+/* Staged attention of decode step `step` (xGR 2.1), for every live beam:
+ *   d_q     bf16 [B][BW][Hq][D]   this step's queries (rows of dead beams ignored)
+ *   d_k_new bf16 [B][BW][Hkv][D]  this step's keys of each live beam's fed token,
+ *   d_v_new bf16 [B][BW][Hkv][D]  appended to the Unshared pool at slot (step, b)
+ *   d_out   bf16 [B][BW][Hq][D]   softmax(q K^T / sqrt(D)) V over the beam's
+ *                                  shared prompt (+ suffix) and its own step+1
+ *                                  Unshared tokens
+ *   d_lse   fp32 [B][BW][Hq]      natural-log log-sum-exp of the scaled scores
+ * B is n_requests of xgr_begin.  step must be the current step. */
+xgr_status xgr_decode_step(xgr_ctx *ctx, int32_t step, const void *d_q, const void *d_k_new,
+                           const void *d_v_new, void *d_out, float *d_lse, xgr_stream_t stream);
+
+/* Valid-path mask of step `step` (xGR 2.2 "Hybrid dense/sparse storage"):
+ * step 0 returns the pre-generated dense bitset (no kernel); later steps
+ * write one CSR row per beam (the sorted valid next tokens of its trie node).
+ * Fills *out with views into the workspace. */
+xgr_status xgr_build_mask(xgr_ctx *ctx, int32_t step, xgr_mask *out, xgr_stream_t stream);
+
+/* Masked top-K beam selection with in-place rewiring (xGR 2.2 "Early sort
+ * termination", 2.1 "In-place updates"):
+ *   d_scores fp32 [B][BW][V]  log-probs or logits (flags); rows of dead beams
+ *                             are not read
+ *   mask                      as returned by xgr_build_mask for this step
+ *   d_parent, d_token int32 [B][BW], d_cum fp32 [B][BW], d_n_out int32 [B]:
+ *     the new beams in rank order (slot = rank): higher score first, then
+ *     lower parent, then lower token.  Score = fp32(cum[parent] + lp).
+ * Each beam first keeps its top-K valid candidates; the best BW of their
+ * union survive.  The context's ancestry (Unshared slot of every earlier
+ * step), trie node, token history and cumulative score are rewired in place
+ * to the new beams, and the current step advances. */
+xgr_status xgr_beam_select(xgr_ctx *ctx, int32_t step, const float *d_scores, int32_t flags,
+                           const xgr_mask *mask, int32_t *d_parent, int32_t *d_token,
+                           float *d_cum, int32_t *d_n_out, xgr_stream_t stream);
+
+/* Tokens chosen so far by each current beam: d_seq int32 [B][BW][S]; entries
+ * past the decoded steps and rows of dead beams are -1. */
+xgr_status xgr_get_sequences(xgr_ctx *ctx, int32_t *d_seq, xgr_stream_t stream);
+
+/* Synchronises `stream`, returns the device status word in *host_code (0 when
+ * clean) and clears it.  Returns XGR_ERR_DEVICE when the word was non-zero. */
+xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XGR_H_ */

@@ -50,7 +50,7 @@ def lib():
         i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         L.orc_attend.argtypes = [i32, i32, P, i32, P, P, f64, P, P]
         L.orc_decode_attention.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, i32, P, P, i32,
-                                           P, P, P, i32, P, P]
+                                           P, P, P, i32, P, i32, P, P]
         L.orc_next_tokens_scan.argtypes = [P, i64, i32, i32, P, i32, P]
         L.orc_sort_items.argtypes = [P, i64, i32]
         L.orc_sort_items.restype = None
@@ -110,15 +110,18 @@ def attend(q, k, v, scale: Optional[float] = None):
     return out, lse
 
 
-def decode_attention(q, ks, vs, kpool, vpool, anc, s: int, n_live: int, kx=None, vx=None):
+def decode_attention(q, ks, vs, kpool, vpool, anc, s: int, n_live: int, kx=None, vx=None,
+                     beams=None):
     """Attention of one request at step s over shared prompt + optional suffix +
     the beams' own Unshared tokens (see xgr_oracle.c).
 
     q [BW][Hq][D]; ks, vs [Hkv][P][D]; kx, vx [Hkv][X][D] or None;
     kpool, vpool [S'][BW][Hkv][D] (S' > s); anc int32 [BW][>s].
-    Returns out fp64 [BW][Hq][D], lse fp64 [BW][Hq]."""
+    beams: optional list of beam ids to compute (q then holds only those rows).
+    Returns out fp64 [n][Hq][D], lse fp64 [n][Hq] (n = BW or len(beams))."""
     q, ks, vs, kpool, vpool = _u16(q), _u16(ks), _u16(vs), _u16(kpool), _u16(vpool)
-    BW, Hq, D = q.shape
+    BW = kpool.shape[1]
+    _, Hq, D = q.shape
     Hkv, P, _ = ks.shape
     if kx is None:
         kx = np.zeros((Hkv, 0, D), np.uint16)
@@ -127,11 +130,15 @@ def decode_attention(q, ks, vs, kpool, vpool, anc, s: int, n_live: int, kx=None,
     X = kx.shape[1]
     anc = np.ascontiguousarray(anc, dtype=np.int32)
     assert kpool.shape[1:] == (BW, Hkv, D) and kpool.shape[0] > s
-    out = np.zeros((BW, Hq, D), np.float64)
-    lse = np.zeros((BW, Hq), np.float64)
+    ids = None if beams is None else np.ascontiguousarray(beams, dtype=np.int32)
+    n = BW if ids is None else len(ids)
+    assert q.shape[0] == n
+    out = np.zeros((n, Hq, D), np.float64)
+    lse = np.zeros((n, Hq), np.float64)
     rc = lib().orc_decode_attention(BW, Hq, Hkv, D, s, n_live, _p(q), _p(ks), _p(vs), P,
                                     _p(kx), _p(vx), X, _p(kpool), _p(vpool), _p(anc),
-                                    anc.shape[1], _p(out), _p(lse))
+                                    anc.shape[1], None if ids is None else _p(ids),
+                                    0 if ids is None else n, _p(out), _p(lse))
     if rc:
         raise RuntimeError(f"orc_decode_attention failed: {rc}")
     return out, lse
@@ -305,12 +312,16 @@ class BeamDecode:
         self.kpool = np.zeros((S, BW, self.Hkv, self.D), np.uint16)
         self.vpool = np.zeros((S, BW, self.Hkv, self.D), np.uint16)
 
-    def attention(self, s: int, q, k_new, v_new):
-        """Append this step's k/v at slot (s, b) of the Unshared pool, then attend."""
+    def attention(self, s: int, q, k_new, v_new, beams=None):
+        """Append this step's k/v at slot (s, b) of the Unshared pool, then attend
+        (all beams, or only the listed ones)."""
         self.kpool[s] = _u16(k_new)
         self.vpool[s] = _u16(v_new)
-        return decode_attention(q, self.ks, self.vs, self.kpool, self.vpool, self.anc, s,
-                                self.n_live, self.kx, self.vx)
+        qq = _u16(q)
+        if beams is not None:
+            qq = np.ascontiguousarray(qq[np.asarray(beams)])
+        return decode_attention(qq, self.ks, self.vs, self.kpool, self.vpool, self.anc, s,
+                                self.n_live, self.kx, self.vx, beams=beams)
 
     def mask(self, s: int):
         """Step 0: dense bitset of valid first tokens.  Step >= 1: CSR rows over

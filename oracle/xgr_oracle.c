@@ -125,6 +125,8 @@ int orc_attend(int n_q, int D, const uint16_t *q, int n, const uint16_t *k,
  * Layouts (bf16 bits): q [BW][Hq][D]; ks, vs [Hkv][P][D]; kx, vx [Hkv][X][D];
  * kpool, vpool [S][BW][Hkv][D]; anc[b * anc_stride + i].
  * Output rows of beams b >= n_live are dead: O = 0, LSE = -inf.
+ * beam_ids (optional): compute only these n_ids beams; output row i (and
+ * query row i of q) then belongs to beam beam_ids[i].  NULL: all BW beams.
  */
 int orc_decode_attention(int BW, int Hq, int Hkv, int D, int s, int n_live,
                          const uint16_t *q,
@@ -132,18 +134,24 @@ int orc_decode_attention(int BW, int Hq, int Hkv, int D, int s, int n_live,
                          const uint16_t *kx, const uint16_t *vx, int X,
                          const uint16_t *kpool, const uint16_t *vpool,
                          const int32_t *anc, int anc_stride,
+                         const int32_t *beam_ids, int n_ids,
                          double *out, double *lse)
 {
+    const int n_beams = beam_ids ? n_ids : BW;
     const int G = Hq / Hkv;
     const double scale = 1.0 / sqrt((double)D);
     const int n = P + X + s + 1;
     int err = ORC_OK;
 
-    for (int b = 0; b < n_live; ++b)
+    for (int bi = 0; bi < n_beams; ++bi) {
+        const int b = beam_ids ? beam_ids[bi] : bi;
+        if (b < 0 || b >= BW) return ORC_ERR_INDEX;
+        if (b >= n_live) continue;
         for (int i = 0; i <= s; ++i) {
             int slot = anc[(size_t)b * anc_stride + i];
             if (slot < 0 || slot >= BW) err = ORC_ERR_INDEX;
         }
+    }
     if (err) return err;
 
 #pragma omp parallel
@@ -152,8 +160,9 @@ int orc_decode_attention(int BW, int Hq, int Hkv, int D, int s, int n_live,
         const uint16_t **vr = malloc(sizeof(*vr) * (size_t)n);
         double *sc = malloc(sizeof(double) * (size_t)n);
 #pragma omp for schedule(dynamic, 4)
-        for (int row = 0; row < BW * Hq; ++row) {
-            const int b = row / Hq, h = row % Hq, g = h / G;
+        for (int row = 0; row < n_beams * Hq; ++row) {
+            const int bi = row / Hq, h = row % Hq, g = h / G;
+            const int b = beam_ids ? beam_ids[bi] : bi;
             double *o = out + (size_t)row * D;
             if (b >= n_live) {
                 for (int d = 0; d < D; ++d) o[d] = 0.0;

@@ -1,0 +1,80 @@
+// kernels.h -- argument blocks and launchers of the device kernels (internal).
+#pragma once
+
+#include "common.cuh"
+
+namespace xgr {
+
+// Shared stage, few rows per work item (SIMT).
+struct SmallArgs {
+    const WorkItem *items;
+    const int32_t *members;
+    const __nv_bfloat16 *q;        // [B][BW][Hq][D]
+    const __nv_bfloat16 *kstore;   // [Hkv][kv_tokens][D]
+    const __nv_bfloat16 *vstore;
+    int64_t kv_tokens;
+    Dims dims;
+    int nb;                        // beams per request of the plan (1 at step 0, BW after)
+    const int32_t *n_live;
+    Partials part;
+};
+cudaError_t launch_attn_small(const SmallArgs &a, int n_items, cudaStream_t st);
+
+// Unshared stage + Merging stage (+ append of this step's k/v).
+struct MergeArgs {
+    const __nv_bfloat16 *q;        // [B][BW][Hq][D]
+    const __nv_bfloat16 *k_new;    // [B][BW][Hkv][D]
+    const __nv_bfloat16 *v_new;
+    __nv_bfloat16 *pool_k;         // [S][Bcap][BW][Hkv][D]
+    __nv_bfloat16 *pool_v;
+    __nv_bfloat16 *out;            // [B][BW][Hq][D]
+    float *lse;                    // [B][BW][Hq]
+    BeamState st;
+    Dims dims;
+    int Bcap;
+    int step;
+    const int32_t *n_slots;        // [B] partial slots of each request
+    Partials part;
+};
+cudaError_t launch_attn_merge(const MergeArgs &a, cudaStream_t st);
+
+// Beam state reset of xgr_begin.
+cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, cudaStream_t s);
+
+// Sparse masks of steps >= 1: one CSR row per beam.
+struct MaskArgs {
+    BeamState st;
+    TrieView trie;
+    Dims dims;
+    int step;
+    int32_t *row_ptr;   // [B*BW + 1]
+    int32_t *cols;      // [cap]
+    int64_t cap;
+};
+cudaError_t launch_build_mask(const MaskArgs &a, cudaStream_t s);
+
+// Beam selection + in-place rewiring.
+struct SelectArgs {
+    BeamState st;
+    TrieView trie;
+    Dims dims;
+    int step;
+    int logits;                 // XGR_SCORES_LOGITS
+    const float *scores;        // [B][BW][V]
+    int dense;                  // mask kind
+    const uint32_t *bits;
+    const int32_t *row_ptr;
+    const int32_t *cols;
+    float *row_lse;             // [Bcap][BW] scratch
+    uint64_t *lists;            // [Bcap][BW][K] per-beam sorted candidates
+    int32_t *counts;            // [Bcap][BW]
+    int32_t *parent;            // outputs [B][BW]
+    int32_t *token;
+    float *cum_out;
+    int32_t *n_out;             // [B]
+};
+cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
+
+cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);
+
+}  // namespace xgr

@@ -1,0 +1,186 @@
+"""Test-side driver: run the CUDA path (through the C ABI) and the oracle on the
+same seeded inputs, step by step, and compare.
+
+Tolerances (attention): max-abs 2e-2, relative L2 5e-3 over the compared rows,
+|dLSE| 1e-3 -- bf16 K/V/Q with fp32 accumulation against fp64.  Masks and the
+log-prob selection are compared bit for bit.  Logits-mode selection is
+compared tie-aware: a difference is allowed only between candidates whose
+fp64 oracle scores are within 1e-4.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+import oracle
+import workloads
+from shared_prefix_decode_xattention_b200 import xgr
+from shared_prefix_decode_xattention_b200.session import Session, config_for
+
+ATOL_O = 2e-2
+RL2_O = 5e-3
+ATOL_LSE = 1e-3
+TIE_EPS = 1e-4
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclasses.dataclass
+class StepOut:
+    out: torch.Tensor
+    lse: torch.Tensor
+    mask: tuple
+    parent: Optional[np.ndarray] = None
+    token: Optional[np.ndarray] = None
+    cum: Optional[np.ndarray] = None
+    n_out: Optional[np.ndarray] = None
+
+
+class GpuRun:
+    """One decode of workload w on cuda:0 through the C ABI."""
+
+    def __init__(self, w, items=None, device="cuda", max_partials=0):
+        self.w, self.device = w, device
+        self.sess = Session(config_for(w, max_partials=max_partials), device)
+        if w.V:
+            self.sess.build_trie(items)
+        self.kv = {}
+        for sid in range(w.n_shared):
+            members = [r for r in range(w.B) if w.shared_id(r) == sid]
+            if not members:
+                continue
+            k, v = workloads.shared_kv(w, sid, device)
+            self.kv[("s", sid)] = (k, v)
+            self.sess.prefill(members[0], sid, k, v)
+            for r in members[1:]:
+                self.sess.link(r, sid)
+        if w.suffix[1]:
+            for r in range(w.B):
+                k, v = workloads.suffix_kv(w, r, device)
+                self.kv[("x", r)] = (k, v)
+                self.sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+        self.sess.begin(w.B)
+
+    def step(self, s, q, kn, vn, scores=None, flags=xgr.XGR_SCORES_LOGPROB) -> StepOut:
+        w = self.w
+        out = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=self.device)
+        lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=self.device)
+        self.sess.decode_step(s, q, kn, vn, out, lse)
+        if not w.V:
+            return StepOut(out, lse, None)
+        m = self.sess.build_mask(s)
+        if m.kind == xgr.XGR_MASK_DENSE:
+            bits = torch.empty(m.n_words, dtype=torch.int32, device=self.device)
+            torch.cuda.synchronize()
+            _copy_dev(bits, m.bits, m.n_words * 4, self.sess)
+            mask = ("dense", bits.cpu().numpy().view(np.uint32).copy())
+        else:
+            n_rows = m.n_rows
+            rp = torch.empty(n_rows + 1, dtype=torch.int32, device=self.device)
+            _copy_dev(rp, m.row_ptr, (n_rows + 1) * 4, self.sess)
+            rpn = rp.cpu().numpy()
+            nnz = int(rpn[-1])
+            cols = torch.empty(max(nnz, 1), dtype=torch.int32, device=self.device)
+            if nnz:
+                _copy_dev(cols, m.cols, nnz * 4, self.sess)
+            mask = ("csr", (rpn.astype(np.int64), cols.cpu().numpy()[:nnz].copy()))
+        parent = torch.empty((w.B, w.BW), dtype=torch.int32, device=self.device)
+        token = torch.empty_like(parent)
+        cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=self.device)
+        n_out = torch.empty((w.B,), dtype=torch.int32, device=self.device)
+        self.sess.beam_select(s, scores, flags, m, parent, token, cum, n_out)
+        torch.cuda.synchronize()
+        return StepOut(out, lse, mask, parent.cpu().numpy(), token.cpu().numpy(),
+                       cum.cpu().numpy(), n_out.cpu().numpy())
+
+    def sequences(self) -> np.ndarray:
+        w = self.w
+        seq = torch.empty((w.B, w.BW, w.S), dtype=torch.int32, device=self.device)
+        self.sess.sequences(seq)
+        torch.cuda.synchronize()
+        return seq.cpu().numpy()
+
+    def status(self) -> int:
+        return self.sess.device_status()
+
+
+def _copy_dev(dst: torch.Tensor, src_ptr: int, nbytes: int, sess: Session):
+    """Copy a library-owned view (a pointer into the session's workspace tensor)."""
+    off = src_ptr - sess.workspace.data_ptr()
+    assert 0 <= off and off + nbytes <= sess.nbytes
+    dst.view(torch.uint8)[:nbytes].copy_(sess.workspace[off:off + nbytes])
+
+
+def oracle_request(w, sorted_items, run: GpuRun, r: int, mode="logprob"):
+    """Oracle beam decode of request r with the same prompt/suffix KV as the GPU run."""
+    ks, vs = run.kv[("s", w.shared_id(r))]
+    kx = vx = None
+    if ("x", r) in run.kv:
+        kx, vx = run.kv[("x", r)]
+        kx, vx = u16(kx), u16(vx)
+    dec = oracle.BeamDecode(sorted_items, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V, mode=mode)
+    dec.begin(u16(ks), u16(vs), kx, vx)
+    return dec
+
+
+def compare_attention(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: np.ndarray,
+                      lse_ref: np.ndarray, live: np.ndarray, what=""):
+    """o_gpu [n][Hq][D] bf16, lse_gpu [n][Hq]; o_ref, lse_ref fp64; live bool [n]."""
+    og = o_gpu.float().cpu().numpy().astype(np.float64)
+    lg = lse_gpu.cpu().numpy().astype(np.float64)
+    if (~live).any():
+        assert np.all(og[~live] == 0), f"{what}: dead rows not zero"
+        assert np.all(np.isneginf(lg[~live])), f"{what}: dead LSE not -inf"
+    if live.any():
+        a, b = og[live], o_ref[live]
+        err = np.abs(a - b).max()
+        rl2 = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
+        lerr = np.abs(lg[live] - lse_ref[live]).max()
+        assert err <= ATOL_O, f"{what}: max-abs {err}"
+        assert rl2 <= RL2_O, f"{what}: rel-L2 {rl2}"
+        assert lerr <= ATOL_LSE, f"{what}: LSE {lerr}"
+        return err, rl2, lerr
+    return 0.0, 0.0, 0.0
+
+
+def compare_mask(gpu_mask, ora_mask, r: int, BW: int, what=""):
+    kind, data = gpu_mask
+    okind, odata = ora_mask
+    assert kind == okind, what
+    if kind == "dense":
+        assert np.array_equal(data, odata), f"{what}: dense mask differs"
+        return
+    rp, cols = data
+    orp, ocols = odata
+    for b in range(BW):
+        row = r * BW + b
+        g = cols[rp[row]:rp[row + 1]]
+        o = ocols[orp[b]:orp[b + 1]]
+        assert np.array_equal(g, o), f"{what}: mask row {row} differs"
+
+
+def compare_select_exact(so: StepOut, r: int, parent, token, cum, n, what=""):
+    assert so.n_out[r] == n, f"{what}: n_out {so.n_out[r]} vs {n}"
+    assert np.array_equal(so.parent[r], parent), f"{what}: parent differs"
+    assert np.array_equal(so.token[r], token), f"{what}: token differs"
+    assert so.cum[r].tobytes() == np.asarray(cum, np.float32).tobytes(), f"{what}: cum differs"
+
+
+def compare_select_tie_aware(so: StepOut, r: int, dec, scores_r: np.ndarray, mask, s: int,
+                             what=""):
+    """Logits mode: the GPU's chosen set may differ from the oracle's only among
+    candidates whose fp64 scores are within TIE_EPS; cum within TIE_EPS."""
+    row_ptr, cols = dec._rows(s, mask)
+    pr, tk, cm, n, _ = oracle.select_logits(dec.cum, scores_r, row_ptr, cols, dec.BW, dec.n_live)
+    assert so.n_out[r] == n, what
+    gp, gt = so.parent[r][:n], so.token[r][:n]
+    gk = oracle.logits_keys(dec.cum, scores_r, list(zip(gp.tolist(), gt.tolist())))
+    # the GPU's k-th choice has the oracle's k-th best score up to near-ties
+    assert np.all(np.abs(np.sort(gk)[::-1] - cm[:n]) <= TIE_EPS), f"{what}: selection differs"
+    assert np.all(np.abs(so.cum[r][:n].astype(np.float64) - gk) <= TIE_EPS), f"{what}: cum"
+    return gp, gt, n

@@ -1,0 +1,185 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle, step by
+step, on the same seeded inputs, for every workload shape.
+
+Workloads 1, 2 and 4 are compared in full; 3 and 5 on sampled requests (every
+selection of the request, a deterministic sample of beams for attention).
+Attention within max-abs 2e-2 / rel-L2 5e-3 / LSE 1e-3; masks and log-prob
+selections bit-exact; logits-mode selections tie-aware (1e-4).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from harness import (GpuRun, compare_attention, compare_mask, compare_select_exact,
+                     compare_select_tie_aware, oracle_request)
+from shared_prefix_decode_xattention_b200 import xgr
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_beams(n_live, k, seed):
+    if k is None or n_live <= k:
+        return None
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(n_live, size=k, replace=False)).astype(np.int32)
+
+
+def decode_and_compare(w, mode="logprob", requests=None, beams_per_step=None, items=None,
+                       max_partials=0, scores_fn=None):
+    items = workloads.items(w) if items is None else items
+    si = oracle.SortedItems(items, w.V) if w.V else None
+    run = GpuRun(w, items, max_partials=max_partials)
+    reqs = list(range(w.B)) if requests is None else list(requests)
+    decs = {r: oracle_request(w, si, run, r, mode) for r in reqs}
+    flags = xgr.XGR_SCORES_LOGPROB if mode == "logprob" else xgr.XGR_SCORES_LOGITS
+    worst = [0.0, 0.0, 0.0]
+    for s in range(w.S):
+        q, kn, vn = workloads.step_qkv(w, s, "cuda")
+        scores = None
+        if w.V:
+            if scores_fn is not None:
+                scores = scores_fn(s)
+            elif mode == "logprob":
+                scores = workloads.step_logprobs(w, s, "cuda")
+            else:
+                scores = workloads.step_logits(w, s, "cuda")
+        so = run.step(s, q, kn, vn, scores, flags)
+        qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
+        sc = scores.cpu().numpy() if scores is not None else None
+        for r in reqs:
+            dec = decs[r]
+            beams = _sample_beams(dec.n_live, beams_per_step, 1000 * s + r)
+            o_ref, l_ref = dec.attention(s, qc[r], knc[r], vnc[r], beams)
+            ids = np.arange(w.BW) if beams is None else beams
+            live = ids < dec.n_live
+            errs = compare_attention(so.out[r][torch.as_tensor(ids).long()],
+                                     so.lse[r][torch.as_tensor(ids).long()], o_ref, l_ref, live,
+                                     f"step {s} request {r}")
+            worst = [max(a, b) for a, b in zip(worst, errs)]
+            if not w.V:
+                continue
+            om = dec.mask(s)
+            compare_mask(so.mask, om, r, w.BW, f"step {s} request {r}")
+            if mode == "logprob":
+                p, t, c, n = dec.select(s, sc[r], om)
+                compare_select_exact(so, r, p, t, c, n, f"step {s} request {r}")
+            else:
+                compare_select_tie_aware(so, r, dec, sc[r], om, s, f"step {s} request {r}")
+                dec.select(s, sc[r], om, force=(so.parent[r], so.token[r], so.n_out[r]))
+    if w.V:
+        seq = run.sequences()
+        item_set = {tuple(x) for x in items.tolist()}
+        for r in reqs:
+            dec = decs[r]
+            assert np.array_equal(seq[r], dec.paths), f"sequences of request {r}"
+            for b in range(dec.n_live):
+                assert tuple(seq[r, b].tolist()) in item_set
+    assert run.status() == 0
+    run.sess.close()
+    return worst
+
+
+def test_workload1_logprob_full():
+    decode_and_compare(workloads.WORKLOADS[1])
+
+
+def test_workload1_logits_tie_aware():
+    decode_and_compare(workloads.WORKLOADS[1], mode="logits")
+
+
+def test_workload2_logprob_full():
+    decode_and_compare(workloads.WORKLOADS[2])
+
+
+def test_workload2_logits_sampled():
+    decode_and_compare(workloads.WORKLOADS[2], mode="logits", requests=[0, 5],
+                       beams_per_step=16)
+
+
+def test_workload3_sampled():
+    decode_and_compare(workloads.WORKLOADS[3], requests=[0, 13, 22, 31], beams_per_step=12)
+
+
+def test_workload4_homogeneous():
+    decode_and_compare(workloads.WORKLOADS[4])
+
+
+def test_workload4_heterogeneous_sampled():
+    w = workloads.heterogeneous(workloads.WORKLOADS[4])
+    decode_and_compare(w, requests=[0, 9, 17, 30, 41, 50, 58, 63])
+
+
+def test_workload5_sampled():
+    decode_and_compare(workloads.WORKLOADS[5], requests=[0, 41, 90, 127], beams_per_step=8)
+
+
+# ------------------------------------------------------------------ edges
+
+def test_ragged_prompts_and_split_k():
+    """Prompt lengths that are not multiples of any tile (1 .. 700 tokens), and
+    several requests per shared prefix so split-K partials are merged."""
+    w = workloads.small(workloads.WORKLOADS[1], wid=101, B=6, prompt=(1, 700), BW=8, K=9,
+                        Hq=8, Hkv=2, D=128)
+    decode_and_compare(w)
+    w2 = workloads.small(workloads.WORKLOADS[4], wid=102, B=8, groups=2, prompt=(1000, 1000),
+                         suffix=(1, 300), Hq=16, Hkv=4)
+    decode_and_compare(w2, max_partials=6)
+
+
+def test_fewer_candidates_than_beams():
+    """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
+    w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
+    decode_and_compare(w)
+
+
+def test_all_scores_tied_fallback_path():
+    """Every score equal: the ordering falls to parent then token, and the
+    survivors of the threshold exceed the sort buffer (exact radix fallback)."""
+    w = workloads.small(workloads.WORKLOADS[2], wid=104, B=2)
+    tie = lambda s: torch.full((w.B, w.BW, w.V), -9.0, device="cuda")
+    decode_and_compare(w, scores_fn=tie, beams_per_step=4)
+
+
+def test_nan_score_sets_device_status():
+    w = workloads.WORKLOADS[1]
+    items = workloads.items(w)
+    run = GpuRun(w, items)
+    q, kn, vn = workloads.step_qkv(w, 0, "cuda")
+    lp = workloads.step_logprobs(w, 0, "cuda")
+    lp[0, 0, int(items[0, 0])] = float("nan")
+    run.step(0, q, kn, vn, lp)
+    assert run.status() & xgr.XGR_DEV_NAN
+    assert run.status() == 0   # cleared by the read
+
+
+def test_abi_call_order_and_arguments():
+    w = workloads.WORKLOADS[1]
+    items = workloads.items(w)
+    run = GpuRun(w, items)
+    q, kn, vn = workloads.step_qkv(w, 0, "cuda")
+    out = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device="cuda")
+    with pytest.raises(xgr.XgrError) as e:
+        run.sess.decode_step(1, q, kn, vn, out, lse)           # step 1 before step 0
+    assert e.value.status == xgr.XGR_ERR_STATE
+    with pytest.raises(xgr.XgrError) as e:
+        run.sess.decode_step(0, q.data_ptr() + 2, kn, vn, out, lse)   # misaligned
+    assert e.value.status == xgr.XGR_ERR_ARG
+    with pytest.raises(xgr.XgrError) as e:
+        xgr.xgr_build_trie(run.sess.ctx, items[:, :2])         # wrong item length
+    assert e.value.status == xgr.XGR_ERR_SHAPE
+    big = torch.zeros((w.Hkv, 10_000, w.D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(xgr.XgrError) as e:
+        run.sess.prefill(0, 0, big, big)                      # store too small
+    assert e.value.status == xgr.XGR_ERR_CAPACITY
+    m = run.sess.build_mask(0)
+    p = torch.empty((w.B, w.BW), dtype=torch.int32, device="cuda")
+    c = torch.empty((w.B, w.BW), dtype=torch.float32, device="cuda")
+    n = torch.empty((w.B,), dtype=torch.int32, device="cuda")
+    lp = workloads.step_logprobs(w, 0, "cuda")
+    with pytest.raises(xgr.XgrError) as e:
+        run.sess.beam_select(0, lp, 7, m, p, p.clone(), c, n)   # unknown flag
+    assert e.value.status == xgr.XGR_ERR_ARG
+    assert run.status() == 0

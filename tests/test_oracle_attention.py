@@ -161,3 +161,13 @@ def test_split_merge_equals_unsplit(orc):
             mo, ml = _merge(parts)
             assert np.allclose(mo[0], out[b, h], atol=1e-12)
             assert abs(ml[0] - lse[b, h]) < 1e-12
+
+
+def test_beam_subset_equals_full(orc):
+    c = _decode_case(50, X=7, n_live=3)
+    full, full_lse = orc.decode_attention(c["q"], c["ks"], c["vs"], c["kp"], c["vp"], c["anc"],
+                                          c["s"], c["n_live"], c["kx"], c["vx"])
+    ids = [2, 0, 3]
+    sub, sub_lse = orc.decode_attention(c["q"][ids], c["ks"], c["vs"], c["kp"], c["vp"], c["anc"],
+                                        c["s"], c["n_live"], c["kx"], c["vx"], beams=ids)
+    assert np.array_equal(sub, full[ids]) and np.array_equal(sub_lse, full_lse[ids])
