@@ -77,7 +77,8 @@ enum {
     XGR_DEV_NAN = 1,            /* NaN among the scores or cumulative scores read */
     XGR_DEV_INDEX = 2,          /* ancestry slot / trie node out of range */
     XGR_DEV_MASK = 4,           /* a mask token that is not a child in the trie, or >= V */
-    XGR_DEV_CAPACITY = 8        /* mask rows exceeded the CSR capacity */
+    XGR_DEV_CAPACITY = 8,       /* mask rows exceeded the CSR capacity */
+    XGR_DEV_TIMEOUT = 16        /* a bounded on-chip wait gave up (the CTA unwound, results invalid) */
 };
 
 /* Score input of xgr_beam_select. */

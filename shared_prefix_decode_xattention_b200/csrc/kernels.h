@@ -1,6 +1,8 @@
 // kernels.h -- argument blocks and launchers of the device kernels (internal).
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace xgr {
@@ -19,6 +21,23 @@ struct SmallArgs {
     Partials part;
 };
 cudaError_t launch_attn_small(const SmallArgs &a, int n_items, cudaStream_t st);
+
+// Shared stage on the tensor cores: 128-row tiles, D = 128, TMA-fed K/V.
+struct TcArgs {
+    const WorkItem *items;
+    const int32_t *members;
+    const __nv_bfloat16 *q;        // [B][BW][Hq][D]
+    int64_t kv_tokens;
+    Dims dims;
+    int nb;
+    const int32_t *n_live;
+    Partials part;
+    int32_t *status;
+};
+// 2-D tensor map over a [rows][128] bf16 store, 64 x 128 boxes, 128-byte swizzle.
+cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows);
+cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const TcArgs &a,
+                           int n_items, cudaStream_t st);
 
 // Unshared stage + Merging stage (+ append of this step's k/v).
 struct MergeArgs {

@@ -107,6 +107,7 @@ xgr_status check_config(const xgr_config *c) {
     if (!c) return XGR_ERR_ARG;
     if (c->max_requests < 1 || c->max_shared < 0 || c->kv_tokens < 0) return XGR_ERR_SHAPE;
     if (c->kv_tokens >= (1ll << 31)) return XGR_ERR_SHAPE;
+    if (c->n_kv_heads >= 1 && (int64_t)c->n_kv_heads * c->kv_tokens >= (1ll << 31)) return XGR_ERR_SHAPE;
     if (c->beam_width < 1 || c->beam_width > 1024) return XGR_ERR_SHAPE;
     if (c->steps < 1 || c->steps > kMaxSteps) return XGR_ERR_SHAPE;
     if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) return XGR_ERR_SHAPE;
@@ -144,7 +145,10 @@ struct xgr_ctx {
     std::vector<int64_t> suf_off, suf_len;
     bool plan_dirty = true;
     int planned_B = -1;
-    int n_plan_items[2] = {0, 0};
+    int n_small[2] = {0, 0};   // small-row work items of each plan (then n_tc[] tensor-core ones)
+    int n_tc[2] = {0, 0};
+    bool has_tc = false;       // tensor-core Shared stage available (D = 128, tensor maps built)
+    CUtensorMap tmk, tmv;
     // decode state
     bool begun = false;
     int cur_step = 0;
@@ -187,24 +191,53 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     for (auto &sg : segs)
         for (int r : sg.members) nseg[r]++;
 
-    int64_t base = 0;
-    for (auto &sg : segs) {
-        const int64_t rows = (int64_t)sg.members.size() * nb * G;
-        base += (rows + kSmallRows - 1) / kSmallRows * cf.n_kv_heads;
-    }
-    const int64_t target = 4ll * c->num_sms;
-    const int64_t f = base > 0 ? std::max<int64_t>(1, (target + base - 1) / base) : 1;
+    // kind of every segment: tensor-core tiles of 128 rows when it has more
+    // than kSmallRows rows (and D = 128), else the small-row kernel
+    auto rows_of = [&](const Seg &sg) { return (int64_t)sg.members.size() * nb * G; };
+    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > kSmallRows; };
+    // split factor per kind: the fewest waves x keys per item (+ a fixed
+    // per-item overhead in key units), over the resident CTAs of the GPU
+    auto pick_split = [&](bool tc) {
+        int64_t base = 0, keys = 0, nseg_k = 0;
+        for (auto &sg : segs) {
+            if (is_tc(sg) != tc) continue;
+            const int64_t R = tc ? kTcRows : kSmallRows;
+            base += (rows_of(sg) + R - 1) / R * cf.n_kv_heads;
+            keys += sg.len;
+            ++nseg_k;
+        }
+        if (!nseg_k) return (int64_t)1;
+        const double L = (double)keys / nseg_k;
+        const int64_t cap = tc ? c->num_sms : 2ll * c->num_sms;
+        const double over = tc ? 384.0 : 128.0;
+        int64_t best = 1;
+        double best_cost = 1e300;
+        for (int64_t f = 1; f <= c->L.slots; ++f) {
+            if (f > 1 && L / f < kMinChunk) break;
+            const double waves = (double)((base * f + cap - 1) / cap);
+            const double cost = waves * (L / f + over);
+            if (cost < best_cost * 0.999) {
+                best_cost = cost;
+                best = f;
+            }
+        }
+        return best;
+    };
+    const int64_t f_tc = pick_split(true), f_small = pick_split(false);
 
-    std::vector<WorkItem> items;
+    std::vector<WorkItem> items_small, items_tc;
     std::vector<int32_t> members;
     std::vector<int32_t> nslots(B, 0);
     for (auto &sg : segs) {
-        const int64_t rows = (int64_t)sg.members.size() * nb * G;
-        const int64_t tiles = (rows + kSmallRows - 1) / kSmallRows;
+        const bool tc = is_tc(sg);
+        const int64_t R = tc ? kTcRows : kSmallRows;
+        const int64_t rows = rows_of(sg);
+        const int64_t tiles = (rows + R - 1) / R;
         int max_seg = 1;
         for (int r : sg.members) max_seg = std::max(max_seg, nseg[r]);
         const int64_t slot_cap = std::max(1, c->L.slots / max_seg);
-        int64_t splits = std::min<int64_t>({f, slot_cap, (sg.len + kMinChunk - 1) / kMinChunk});
+        int64_t splits = std::min<int64_t>({tc ? f_tc : f_small, slot_cap,
+                                            (sg.len + kMinChunk - 1) / kMinChunk});
         splits = std::max<int64_t>(1, splits);
         int64_t chunk = (sg.len + splits - 1) / splits;
         chunk = (chunk + 127) / 128 * 128;
@@ -214,6 +247,7 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         if (slot0 + splits > c->L.slots) return XGR_ERR_CAPACITY;
         const int member_off = (int)members.size();
         for (int r : sg.members) members.push_back(r);
+        auto &dst = tc ? items_tc : items_small;
         for (int g = 0; g < cf.n_kv_heads; ++g)
             for (int64_t sp = 0; sp < splits; ++sp)
                 for (int64_t t = 0; t < tiles; ++t) {
@@ -224,13 +258,15 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
                     it.g = g;
                     it.member_off = member_off;
                     it.n_members = (int32_t)sg.members.size();
-                    it.row_begin = (int32_t)(t * kSmallRows);
-                    it.n_rows = (int32_t)std::min<int64_t>(kSmallRows, rows - t * kSmallRows);
+                    it.row_begin = (int32_t)(t * R);
+                    it.n_rows = (int32_t)std::min<int64_t>(R, rows - t * R);
                     it.slot = (int32_t)(slot0 + sp);
-                    items.push_back(it);
+                    dst.push_back(it);
                 }
         for (int r : sg.members) nslots[r] = (int32_t)(slot0 + splits);
     }
+    std::vector<WorkItem> items(items_small);
+    items.insert(items.end(), items_tc.begin(), items_tc.end());
     if ((int64_t)items.size() > c->L.item_cap || (int64_t)members.size() > c->L.member_cap)
         return XGR_ERR_CAPACITY;
     if (!items.empty() &&
@@ -244,7 +280,8 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     if (cudaMemcpy(c->at<int32_t>(c->L.plan_nslots[which]), nslots.data(), (size_t)B * 4,
                    cudaMemcpyHostToDevice) != cudaSuccess)
         return XGR_ERR_CUDA;
-    c->n_plan_items[which] = (int)items.size();
+    c->n_small[which] = (int)items_small.size();
+    c->n_tc[which] = (int)items_tc.size();
     return XGR_OK;
 }
 
@@ -308,9 +345,20 @@ xgr_status xgr_create(const xgr_config *cfg, void *d_workspace, size_t bytes, xg
     c->suf_off.assign(cfg->max_requests, 0);
     c->suf_len.assign(cfg->max_requests, 0);
     std::memset(&c->trie, 0, sizeof(c->trie));
-    if (cudaMemset(c->st.status, 0, 16) != cudaSuccess) {
+    // the store starts as zeros so that key rows read past the end of a segment
+    // (a tile's tail, masked out of the softmax) are always finite
+    const size_t store_bytes = (size_t)2 * cfg->n_kv_heads * cfg->kv_tokens * cfg->head_dim;
+    if (cudaMemset(c->st.status, 0, 16) != cudaSuccess ||
+        (store_bytes && (cudaMemset(c->at<uint8_t>(L.kstore), 0, store_bytes) != cudaSuccess ||
+                         cudaMemset(c->at<uint8_t>(L.vstore), 0, store_bytes) != cudaSuccess)) ||
+        cudaDeviceSynchronize() != cudaSuccess) {
         delete c;
         return XGR_ERR_CUDA;
+    }
+    if (cfg->head_dim == 128 && cfg->kv_tokens > 0) {
+        const int64_t rows = (int64_t)cfg->n_kv_heads * cfg->kv_tokens;
+        c->has_tc = make_kv_tensor_map(&c->tmk, c->at<void>(L.kstore), rows) == cudaSuccess &&
+                    make_kv_tensor_map(&c->tmv, c->at<void>(L.vstore), rows) == cudaSuccess;
     }
     *out = c;
     return XGR_OK;
@@ -487,7 +535,21 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
     sa.nb = (which == 0) ? 1 : c->cfg.beam_width;
     sa.n_live = c->st.n_live;
     sa.part = partials_of(c);
-    if (launch_attn_small(sa, c->n_plan_items[which], s) != cudaSuccess) return XGR_ERR_CUDA;
+    if (launch_attn_small(sa, c->n_small[which], s) != cudaSuccess) return XGR_ERR_CUDA;
+    if (c->n_tc[which] > 0) {
+        TcArgs ta;
+        ta.items = sa.items + c->n_small[which];
+        ta.members = sa.members;
+        ta.q = sa.q;
+        ta.kv_tokens = sa.kv_tokens;
+        ta.dims = sa.dims;
+        ta.nb = sa.nb;
+        ta.n_live = sa.n_live;
+        ta.part = sa.part;
+        ta.status = c->st.status;
+        if (launch_attn_tc(c->tmk, c->tmv, ta, c->n_tc[which], s) != cudaSuccess)
+            return XGR_ERR_CUDA;
+    }
     MergeArgs ma;
     ma.q = sa.q;
     ma.k_new = static_cast<const __nv_bfloat16 *>(d_k_new);
