@@ -52,6 +52,7 @@ def workload_config(w, scores):
                     f"V={w.V}, {w.n_items} valid items",
         "scores": scores,
         "l2": "flushed (256 MiB write) before every timed step; step time from CUDA events",
+        "execution": "each decode replayed as one CUDA graph (per-phase graphs for the breakdown)",
     }
 
 
@@ -236,47 +237,64 @@ def run_gpu(args, w):
     cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
     nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-    sess.begin(w.B, stream)   # plan once (setup)
+    sess.begin(w.B)   # plan once (setup)
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream
 
-    def decode(timers=None, inp=inputs, host=None):
-        sess.begin(w.B, stream)
-        for s in range(w.S):
-            q, kn, vn, sc = inp[s]
-            if host is not None:                      # end-to-end: host -> device inputs
-                hq, hk, hv, hs = host[s]
-                q.copy_(hq, non_blocking=True)
-                kn.copy_(hk, non_blocking=True)
-                vn.copy_(hv, non_blocking=True)
-                sc.copy_(hs, non_blocking=True)
-            if timers is not None and s >= 1:
-                timers["att"][-1][s][0].record(stream)
-            sess.decode_step(s, q, kn, vn, out, lse, stream)
-            if timers is not None and s >= 1:
-                timers["att"][-1][s][1].record(stream)
-            m = sess.build_mask(s, stream)
-            if timers is not None and s >= 1:
-                timers["sel"][-1][s][0].record(stream)
-            sess.beam_select(s, sc, flags, m, par, tok, cum, nout, stream)
-            if timers is not None and s >= 1:
-                timers["sel"][-1][s][1].record(stream)
-            if host is not None:
-                hp, ht, hc, hn = host[w.S + s]
-                hp.copy_(par, non_blocking=True)
-                ht.copy_(tok, non_blocking=True)
-                hc.copy_(cum, non_blocking=True)
-                hn.copy_(nout, non_blocking=True)
+    # One decode = phases: [begin + step 0] then, for s >= 1, [attention s] and
+    # [mask + selection s].  Each phase is enqueued on the current stream (the
+    # capture stream while a CUDA graph is recorded); with `host`, the step's
+    # inputs come from pinned host memory and its outputs go back to it.
+    def enqueue_att(s, inp, host):
+        q, kn, vn, sc = inp[s]
+        if host is not None:
+            for d, h in zip(inp[s], host[s]):
+                d.copy_(h, non_blocking=True)
+        sess.decode_step(s, q, kn, vn, out, lse, cur())
 
-    for _ in range(max(args.warmup, 3)):
-        decode()
+    def enqueue_sel(s, inp, host):
+        m = sess.build_mask(s, cur())
+        sess.beam_select(s, inp[s][3], flags, m, par, tok, cum, nout, cur())
+        if host is not None:
+            for h, d in zip(host[w.S + s], (par, tok, cum, nout)):
+                h.copy_(d, non_blocking=True)
+
+    def enqueue_head(inp, host):
+        sess.begin(w.B, cur())
+        enqueue_att(0, inp, host)
+        enqueue_sel(0, inp, host)
+
+    def enqueue_decode(inp=inputs, host=None):
+        enqueue_head(inp, host)
+        for s in range(1, w.S):
+            enqueue_att(s, inp, host)
+            enqueue_sel(s, inp, host)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    for _ in range(max(args.warmup, 3)):   # eager warm-up (plans, attributes)
+        enqueue_decode()
     torch.cuda.synchronize()
     if sess.device_status() != 0:
         raise RuntimeError("device status set during warm-up")
-    # timed region
-    timers = {"att": [], "sel": []}
+    # the graph-based execution of the pages' system level: a whole decode is one graph
+    g_decode = capture(lambda: enqueue_decode())
+    g_phase = [capture(lambda: enqueue_head(inputs, None))]
+    for s in range(1, w.S):
+        g_phase.append(capture(lambda s=s: enqueue_att(s, inputs, None)))
+        g_phase.append(capture(lambda s=s: enqueue_sel(s, inputs, None)))
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        g_decode.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K whole-decode graph replays, L2 flushed before each
     starts, ends = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
     clk = Clocks(local) if rank == 0 else None
     if world > 1:
@@ -284,11 +302,9 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.zero_()
-        timers["att"].append({s: (ev(), ev()) for s in range(1, w.S)})
-        timers["sel"].append({s: (ev(), ev()) for s in range(1, w.S)})
-        starts[i].record(stream)
-        decode(timers)
-        ends[i].record(stream)
+        starts[i].record()
+        g_decode.replay()
+        ends[i].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -298,13 +314,24 @@ def run_gpu(args, w):
         t = torch.tensor([total_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    att_ms = [t[s][0].elapsed_time(t[s][1]) for t in timers["att"] for s in t]
-    sel_ms = [t[s][0].elapsed_time(t[s][1]) for t in timers["sel"] for s in t]
     n_live = nout.cpu().numpy()
     cands = candidates_per_decode(w) * args.steps * world
     value = cands / (total_ms / 1e3)
 
-    # ---- end to end through the C ABI with host buffers
+    # ---- per-phase device time (same decode, one graph per phase, events between)
+    att_ms, sel_ms = [], []
+    for i in range(args.steps):
+        flush.zero_()
+        evs = [ev() for _ in range(len(g_phase) + 1)]
+        evs[0].record()
+        for k, g in enumerate(g_phase):
+            g.replay()
+            evs[k + 1].record()
+        torch.cuda.synchronize()
+        for k in range(1, len(g_phase)):
+            (att_ms if k % 2 == 1 else sel_ms).append(evs[k].elapsed_time(evs[k + 1]))
+
+    # ---- end to end through the C ABI with host buffers (copies inside the graph)
     e2e = None
     if not args.no_e2e:
         host = []
@@ -318,15 +345,17 @@ def run_gpu(args, w):
             host.append(hs)
             d2h += sum(t.numel() * t.element_size() for t in hs)
         dev_in = [tuple(torch.empty_like(t) for t in inputs[s]) for s in range(w.S)]
-        for _ in range(2):
-            decode(inp=dev_in, host=host)
+        enqueue_decode(dev_in, host)
+        torch.cuda.synchronize()
+        g_e2e = capture(lambda: enqueue_decode(dev_in, host))
+        g_e2e.replay()
         torch.cuda.synchronize()
         e_s, e_e = [ev() for _ in range(args.steps)], [ev() for _ in range(args.steps)]
         for i in range(args.steps):
             flush.zero_()
-            e_s[i].record(stream)
-            decode(inp=dev_in, host=host)
-            e_e[i].record(stream)
+            e_s[i].record()
+            g_e2e.replay()
+            e_e[i].record()
         torch.cuda.synchronize()
         e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e))
         if world > 1:
@@ -335,6 +364,7 @@ def run_gpu(args, w):
             e_ms = float(t.item())
         e2e = {"value": cands / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
+        del g_e2e
 
     status = sess.device_status()
 
@@ -386,6 +416,7 @@ def run_gpu(args, w):
         line["cpu_baseline"] = cpu_baseline(w, items, args.scores)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del g_decode, g_phase
     sess.close()
     if world > 1:
         dist.barrier()

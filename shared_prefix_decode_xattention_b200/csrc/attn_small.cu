@@ -194,9 +194,13 @@ __global__ void __launch_bounds__(kThreads) attn_small_kernel(SmallArgs a) {
 template <int D>
 cudaError_t launch_small_impl(const SmallArgs &a, int n_items, cudaStream_t st) {
     const size_t smem = sizeof(SmallSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(attn_small_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+    static bool attr = false;   // set once, on the first (uncaptured) launch
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(attn_small_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
     attn_small_kernel<D><<<n_items, kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

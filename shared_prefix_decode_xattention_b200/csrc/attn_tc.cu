@@ -340,12 +340,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + sbuf * 128 + q4 * 32, s + q4 * 32);
             tmem_wait_ld();
             const int nvalid = min(kBlockN, n_keys - j * kBlockN);
-            float mx = -INFINITY;
+            // row max over the raw scores (the scale is positive), 8 independent chains
+            float mxp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 128; ++c) {
-                s[c] = (c < nvalid) ? s[c] * cscale : -INFINITY;
-                mx = fmaxf(mx, s[c]);
+                if (c >= nvalid) s[c] = -INFINITY;
+                mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
             }
+            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * cscale;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + 8.f) {
@@ -353,15 +358,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 rescale = j > 0;
                 m_used = mx;
             }
-            float sum = 0.f;
+            const float neg_m = -m_used;
+            float sp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
             uint32_t packed[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                const float p0 = exp2f(s[2 * c] - m_used), p1 = exp2f(s[2 * c + 1] - m_used);
-                sum += p0 + p1;
+                const float p0 = exp2f(fmaf(s[2 * c], cscale, neg_m));
+                const float p1 = exp2f(fmaf(s[2 * c + 1], cscale, neg_m));
+                sp[c & 7] += p0 + p1;
                 __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                 packed[c] = *reinterpret_cast<uint32_t *>(&h);
             }
+            const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
             l = l * alpha + sum;
             if (j >= 2) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + sbuf), ((j - 2) >> 1) & 1, abort));

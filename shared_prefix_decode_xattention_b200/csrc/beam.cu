@@ -554,9 +554,13 @@ cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = select_request_smem(a.dims);
-    e = cudaFuncSetAttribute(select_request_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
+    static size_t attr = 0;   // largest size set so far (set outside graph capture in practice)
+    if (smem > attr) {
+        e = cudaFuncSetAttribute(select_request_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = smem;
+    }
     select_request_kernel<<<a.dims.B, kReqThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
