@@ -209,6 +209,35 @@ xgr_status xgr_get_sequences(xgr_ctx *ctx, int32_t *d_seq, xgr_stream_t stream);
  * clean) and clears it.  Returns XGR_ERR_DEVICE when the word was non-zero. */
 xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_code);
 
+/* Masked beam top-K for callers that cannot allocate device memory.  The
+ * pages have no counterpart of this call: it exists for code that may not
+ * call cudaMalloc or create a workspace (a host framework that owns every
+ * device byte, a plugin that must not allocate after start-up).  It needs no
+ * context and writes no beam state: given
+ *   d_scores  fp32 [B][BW][V]   log-probs or logits (flags, as xgr_beam_select)
+ *   d_cum     fp32 [B][BW]      cumulative score of each live beam
+ *   d_n_live  int32 [B]         live beams per request
+ *   the mask: d_bits (dense, uint32 [ceil(V/32)], first step: only beam 0 of
+ *             each request is read) or, when d_bits is NULL, the CSR rows
+ *             d_row_ptr [B*BW+1] / d_cols (as built by xgr_build_mask)
+ * it writes d_parent, d_token, d_cum_out [B][BW] and d_n_out [B] exactly as
+ * xgr_beam_select does (same order, same tie-break, same bits).
+ * Allocation: none.  Its scratch is one static device array of 8 MiB per GPU
+ * (held by every GPU that loads the library until the process exits); a call
+ * needs B*BW*(8*K + 8) bytes of it and returns XGR_ERR_CAPACITY beyond that.
+ * The first call on a device looks the array up (cudaGetSymbolAddress) and
+ * sets a kernel attribute, so make that first call before any stream capture.
+ * All calls share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller.  NaN scores and out-of-range mask tokens are
+ * skipped, as in the context path, but not reported.  Host-side argument
+ * errors return XGR_ERR_ARG / XGR_ERR_SHAPE; nothing is enqueued then. */
+xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_width, int32_t top_k,
+                                 int32_t vocab, const float *d_scores, int32_t flags,
+                                 const float *d_cum, const int32_t *d_n_live,
+                                 const uint32_t *d_bits, const int32_t *d_row_ptr,
+                                 const int32_t *d_cols, int32_t *d_parent, int32_t *d_token,
+                                 float *d_cum_out, int32_t *d_n_out, xgr_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

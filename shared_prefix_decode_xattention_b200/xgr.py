@@ -111,6 +111,7 @@ def lib():
         "xgr_beam_select": [P, i32, P, i32, ctypes.POINTER(xgr_mask), P, P, P, P, P],
         "xgr_get_sequences": [P, P, P],
         "xgr_device_status": [P, P, ctypes.POINTER(i32)],
+        "xgr_beam_topk_noalloc": [i32, i32, i32, i32, P, i32, P, P, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -213,6 +214,16 @@ def xgr_device_status(ctx: int, stream=None) -> int:
     if st not in (XGR_OK, XGR_ERR_DEVICE):
         raise XgrError("xgr_device_status", st)
     return code.value
+
+
+def xgr_beam_topk_noalloc(n_requests: int, beam_width: int, top_k: int, vocab: int, scores,
+                          flags: int, cum, n_live, bits, row_ptr, cols, parent, token, cum_out,
+                          n_out, stream=None) -> None:
+    """Masked top-K without a context or any allocation (see include/xgr.h)."""
+    _check("xgr_beam_topk_noalloc", lib().xgr_beam_topk_noalloc(
+        n_requests, beam_width, top_k, vocab, _ptr(scores), flags, _ptr(cum), _ptr(n_live),
+        _ptr(bits), _ptr(row_ptr), _ptr(cols), _ptr(parent), _ptr(token), _ptr(cum_out),
+        _ptr(n_out), _stream(stream)))
 
 
 def make_config(**kw) -> xgr_config:
