@@ -67,7 +67,6 @@ __global__ void __launch_bounds__(kWarps * 32) attn_merge_kernel(MergeArgs a) {
     const int s = a.step;
     const int64_t beam_row = (int64_t)r * dm.BW + b;
     const int64_t gid0 = beam_row * dm.Hq + (int64_t)g * G;   // row of query head g*G
-
     if (b >= a.st.n_live[r]) {   // dead beam: O = 0, LSE = -inf
 #pragma unroll
         for (int hg = 0; hg < G; ++hg) {
@@ -77,6 +76,8 @@ __global__ void __launch_bounds__(kWarps * 32) attn_merge_kernel(MergeArgs a) {
         }
         return;
     }
+    const int n_slots = a.n_slots[r];
+    if (n_slots < 0) return;   // the tensor-core kernel already finished this live beam
 
     // append this step's token of the beam at Unshared slot (s, b)
     const int64_t kv_off = (beam_row * dm.Hkv + g) * D;
@@ -151,7 +152,6 @@ __global__ void __launch_bounds__(kWarps * 32) attn_merge_kernel(MergeArgs a) {
     (void)n_tok;
 
     // ---- Merging stage: fold in every Shared-stage partial (online softmax)
-    const int n_slots = a.n_slots[r];
     for (int p = 0; p < n_slots; ++p) {
 #pragma unroll
         for (int hg = 0; hg < G; ++hg) {

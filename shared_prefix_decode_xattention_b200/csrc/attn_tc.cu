@@ -34,22 +34,29 @@ namespace xgr {
 
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;              // producer warp, MMA warp, 2 softmax warpgroups
+constexpr int kSoftmaxThreads = 256;
 constexpr int kBlockN = 128;                 // keys per chunk
+constexpr int kKStages = 3;                  // K chunks in flight
+constexpr int kVStages = 2;                  // V chunks in flight
 constexpr uint32_t kHalf = 16384;            // one 128-row x 64-column bf16 sub-tile
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 bf16
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTile;            // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTile;
-constexpr uint32_t kOffP = kOffV + 2 * kTile;  // 2 buffers
-constexpr uint32_t kOffBar = kOffP + 2 * kTile;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // barriers + alignment slack
+constexpr uint32_t kOffK = kTile;
+constexpr uint32_t kOffV = kOffK + kKStages * kTile;
+constexpr uint32_t kOffP = kOffV + kVStages * kTile;
+constexpr uint32_t kOffBar = kOffP + kTile;
+constexpr uint32_t kOffMisc = kOffBar + 256;  // TMEM address, abort flag
+constexpr uint32_t kOffRed = kOffMisc + 16;   // row-max exchange [2 parity][2 halves][128 rows]
+constexpr uint32_t kSmemUsed = kOffRed + 2048;
+constexpr uint32_t kSmemBytes = 232448;       // the sm_100 per-block maximum
+constexpr uint32_t kSmemSpare = kSmemBytes - kSmemUsed;   // room to realign the window
 constexpr uint32_t kTmemCols = 512;          // S0 [0,128) S1 [128,256) O [256,384)
 constexpr uint32_t kSpinLimit = 1u << 22;
 
 // barrier slots (8 bytes each) after kOffBar
-enum { B_KFULL = 0, B_VFULL = 2, B_KEMPTY = 4, B_VEMPTY = 6, B_SFULL = 8, B_PFULL = 10,
-       B_PVDONE = 12, B_QFULL = 14, B_DRAIN = 15, B_COUNT = 16 };
+enum { B_KFULL = 0, B_KEMPTY = 3, B_VFULL = 6, B_VEMPTY = 8, B_SFULL = 10, B_PFULL = 12,
+       B_PVDONE = 13, B_QFULL = 14, B_DRAIN = 15, B_XCH = 16, B_COUNT = 17 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -185,76 +192,155 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int c) {
     return (uint32_t)(c >> 3) * kHalf + (uint32_t)row * 128u + (uint32_t)(((c & 7) ^ (row & 7)) << 4);
 }
 
+__device__ __forceinline__ float ex2(float x) {   // 2^x, one MUFU op; tiny results flush to 0
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// query row `row` of a work item -> (request, beam, query head, global row, live)
+struct RowInfo {
+    int r, b, hg;
+    int64_t gid;
+    bool valid, live;
+};
+__device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it, int row) {
+    RowInfo ri{0, 0, 0, 0, false, false};
+    if (row < it.n_rows) {
+        const int G = a.dims.G;
+        const int i = it.row_begin + row;
+        const int member = i / (a.nb * G);
+        ri.b = (i / G) % a.nb;
+        ri.hg = i % G;
+        ri.r = a.members[it.member_off + member];
+        ri.gid = ((int64_t)ri.r * a.dims.BW + ri.b) * a.dims.Hq + it.g * G + ri.hg;
+        ri.valid = true;
+    }
+    return ri;
+}
+
+// 10 warps: the register file is split over the 4 schedulers (16K registers each) and 3 of
+// the 10 warps share one, so a thread may use at most 168 registers
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    TcArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ uint32_t tmem_holder;
-    __shared__ int abort_flag;
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > kSmemSpare) {   // the dynamic window is expected 1024-aligned; never trap
+        if (threadIdx.x == 0) set_status(a.status, XGR_DEV_TIMEOUT);
+        return;
+    }
+    uint8_t *base = smem_raw + pad;
     const uint32_t sb = smem_u32(base);
     const uint32_t bar0 = sb + kOffBar;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + kOffMisc);
+    int *abort_flag = reinterpret_cast<int *>(base + kOffMisc + 4);
+    float *red = reinterpret_cast<float *>(base + kOffRed);   // [2 parity][2 halves][128 rows]
 
     const WorkItem it = a.items[blockIdx.x];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int n_keys = it.key_end - it.key_begin;
     const int nchunks = (n_keys + kBlockN - 1) / kBlockN;
+    const bool final_item = (it.flags & 1) != 0;
+    volatile int *abort = abort_flag;
+    const int y0 = it.g * (int)a.kv_tokens + it.kv_off + it.key_begin;
+    // producer lanes: lane 0 streams K chunks, lane 1 V chunks, each on its own ring
+    auto issue_k = [&](int j) {
+        const int st = j % kKStages;
+        mbar_expect_tx(bar(B_KFULL + st), kTile);
+        tma_load_2d(sb + kOffK + st * kTile, &tmk, 0, y0 + j * kBlockN, bar(B_KFULL + st));
+        tma_load_2d(sb + kOffK + st * kTile + kHalf, &tmk, 64, y0 + j * kBlockN, bar(B_KFULL + st));
+    };
+    auto issue_v = [&](int j) {
+        const int st = j % kVStages;
+        mbar_expect_tx(bar(B_VFULL + st), kTile);
+        tma_load_2d(sb + kOffV + st * kTile, &tmv, 0, y0 + j * kBlockN, bar(B_VFULL + st));
+        tma_load_2d(sb + kOffV + st * kTile + kHalf, &tmv, 64, y0 + j * kBlockN, bar(B_VFULL + st));
+    };
 
-    if (tid == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(B_KFULL + s), 1);
-            mbar_init(bar(B_VFULL + s), 1);
-            mbar_init(bar(B_KEMPTY + s), 1);
-            mbar_init(bar(B_VEMPTY + s), 1);
-            mbar_init(bar(B_SFULL + s), 1);
-            mbar_init(bar(B_PFULL + s), 128);
-            mbar_init(bar(B_PVDONE + s), 1);
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < kKStages; ++s) {
+                mbar_init(bar(B_KFULL + s), 1);
+                mbar_init(bar(B_KEMPTY + s), 1);
+            }
+            for (int s = 0; s < kVStages; ++s) {
+                mbar_init(bar(B_VFULL + s), 1);
+                mbar_init(bar(B_VEMPTY + s), 1);
+            }
+            for (int s = 0; s < 2; ++s) mbar_init(bar(B_SFULL + s), 1);
+            mbar_init(bar(B_PFULL), kSoftmaxThreads);
+            mbar_init(bar(B_PVDONE), 1);
+            mbar_init(bar(B_QFULL), kSoftmaxThreads);
+            mbar_init(bar(B_DRAIN), 1);
+            mbar_init(bar(B_XCH), kSoftmaxThreads / 2);
+            *abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
-        mbar_init(bar(B_QFULL), 128);
-        mbar_init(bar(B_DRAIN), 1);
-        abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        __syncwarp();
+        // the first chunks start streaming before the block-wide setup barrier
+        if (lane == 0)
+            for (int j = 0; j < min(nchunks, kKStages); ++j) issue_k(j);
+        if (lane == 1)
+            for (int j = 0; j < min(nchunks, kVStages); ++j) issue_v(j);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(&tmem_holder)),
+                         smem_u32(tmem_holder)),
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // softmax threads stage the Q tile meanwhile: 16 consecutive threads read one
+    // 256-byte row (coalesced) and write it in the swizzled K-major layout
+    if (warp >= 2) {
+        const int ts = tid - 64;
+        uint4 qv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = ts + kSoftmaxThreads * k;
+            const RowInfo qi = row_info(a, it, idx >> 4);
+            qv[k] = qi.valid ? reinterpret_cast<const uint4 *>(a.q + qi.gid * 128)[idx & 15]
+                             : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = ts + kSoftmaxThreads * k;
+            *reinterpret_cast<uint4 *>(base + kOffQ + sw128_off(idx >> 4, idx & 15)) = qv[k];
+        }
+    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    const uint32_t tmem = tmem_holder;
-    volatile int *abort = &abort_flag;
+    const uint32_t tmem = *tmem_holder;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ producers
         if (lane == 0) {
-            const int y0 = it.g * (int)a.kv_tokens + it.kv_off + it.key_begin;
-            int nk[2] = {0, 0}, nv[2] = {0, 0};   // loads issued per stage
-            for (int j = 0; j < nchunks; ++j) {
-                const int st = j & 1;
-                const int y = y0 + j * kBlockN;
-                if (j >= 2 && !mbar_wait(bar(B_KEMPTY + st), ((j - 2) >> 1) & 1, abort)) break;
-                mbar_expect_tx(bar(B_KFULL + st), kTile);
-                tma_load_2d(sb + kOffK + st * kTile, &tmk, 0, y, bar(B_KFULL + st));
-                tma_load_2d(sb + kOffK + st * kTile + kHalf, &tmk, 64, y, bar(B_KFULL + st));
-                ++nk[st];
-                if (j >= 2 && !mbar_wait(bar(B_VEMPTY + st), ((j - 2) >> 1) & 1, abort)) break;
-                mbar_expect_tx(bar(B_VFULL + st), kTile);
-                tma_load_2d(sb + kOffV + st * kTile, &tmv, 0, y, bar(B_VFULL + st));
-                tma_load_2d(sb + kOffV + st * kTile + kHalf, &tmv, 64, y, bar(B_VFULL + st));
-                ++nv[st];
+            int n_issued = min(nchunks, kKStages);
+            for (int j = kKStages; j < nchunks; ++j) {
+                if (!mbar_wait(bar(B_KEMPTY + j % kKStages), ((j / kKStages) - 1) & 1, abort)) break;
+                issue_k(j);
+                ++n_issued;
             }
-            if (*abort) {   // let the copies in flight land before the CTA exits
-                for (int st = 0; st < 2; ++st) {
-                    if (nk[st]) mbar_wait(bar(B_KFULL + st), (nk[st] - 1) & 1, nullptr);
-                    if (nv[st]) mbar_wait(bar(B_VFULL + st), (nv[st] - 1) & 1, nullptr);
-                }
+            if (*abort)   // let the copies in flight land before the CTA exits
+                for (int j = max(0, n_issued - kKStages); j < n_issued; ++j)
+                    mbar_wait(bar(B_KFULL + j % kKStages), (j / kKStages) & 1, nullptr);
+        } else if (lane == 1) {
+            int n_issued = min(nchunks, kVStages);
+            for (int j = kVStages; j < nchunks; ++j) {
+                if (!mbar_wait(bar(B_VEMPTY + j % kVStages), ((j / kVStages) - 1) & 1, abort)) break;
+                issue_v(j);
+                ++n_issued;
             }
+            if (*abort)
+                for (int j = max(0, n_issued - kVStages); j < n_issued; ++j)
+                    mbar_wait(bar(B_VFULL + j % kVStages), (j / kVStages) & 1, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -263,26 +349,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
             bool ok = mbar_wait(bar(B_QFULL), 0, abort);
             for (int j = 0; ok && j <= nchunks; ++j) {
-                if (j < nchunks) {
-                    const int st = j & 1;
-                    if (!mbar_wait(bar(B_KFULL + st), (j >> 1) & 1, abort)) break;
+                if (j < nchunks) {   // S_j = Q K_j^T into TMEM buffer j % 2
+                    const int st = j % kKStages;
+                    if (!mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) break;
                     fence_after_sync();
                     const uint32_t kq = sb + kOffQ, kk = sb + kOffK + st * kTile;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                        umma_bf16(tmem + (uint32_t)st * 128u, umma_desc(kq + off, 16, 1024),
+                        umma_bf16(tmem + (uint32_t)(j & 1) * 128u, umma_desc(kq + off, 16, 1024),
                                   umma_desc(kk + off, 16, 1024), idS, k > 0);
                     }
-                    umma_commit(bar(B_SFULL + st));
+                    umma_commit(bar(B_SFULL + (j & 1)));
                     umma_commit(bar(B_KEMPTY + st));
                 }
-                if (j >= 1) {
-                    const int jp = j - 1, sp = jp & 1;
-                    if (!mbar_wait(bar(B_PFULL + sp), (jp >> 1) & 1, abort)) break;
-                    if (!mbar_wait(bar(B_VFULL + sp), (jp >> 1) & 1, abort)) break;
+                if (j >= 1) {        // O += P_{j-1} V_{j-1}
+                    const int jp = j - 1, sv = jp % kVStages;
+                    if (!mbar_wait(bar(B_PFULL), jp & 1, abort)) break;
+                    if (!mbar_wait(bar(B_VFULL + sv), (jp / kVStages) & 1, abort)) break;
                     fence_after_sync();
-                    const uint32_t kp = sb + kOffP + sp * kTile, kv = sb + kOffV + sp * kTile;
+                    const uint32_t kp = sb + kOffP, kv = sb + kOffV + sv * kTile;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t offp = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
@@ -290,8 +376,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                   umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
                                   (jp > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(bar(B_PVDONE + sp));
-                    umma_commit(bar(B_VEMPTY + sp));
+                    umma_commit(bar(B_PVDONE));
+                    umma_commit(bar(B_VEMPTY + sv));
                 }
             }
             if (*abort) {   // every MMA issued so far must finish before TMEM is freed
@@ -300,128 +386,228 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax rows
+        // ------------------------------------------------------------ softmax
+        // thread (row, half): TMEM lane `row`, S columns [64*half, 64*half + 64);
+        // the two halves swap their partial row max through shared memory
+        const int half = (warp - 2) >> 2;
         const int row = 32 * (warp & 3) + lane;
-        const Dims dm = a.dims;
-        const int G = dm.G;
-        int64_t gid = -1;
-        bool live = false;
-        if (row < it.n_rows) {
-            const int i = it.row_begin + row;
-            const int member = i / (a.nb * G);
-            const int b = (i / G) % a.nb;
-            const int hg = i % G;
-            const int r = a.members[it.member_off + member];
-            gid = ((int64_t)r * dm.BW + b) * dm.Hq + it.g * G + hg;
-            live = b < a.n_live[r];
-        }
-        // Q row -> shared memory (canonical swizzled K-major layout)
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (live ? gid : 0) * 128);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint4 u = live ? src[c] : make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(base + kOffQ + sw128_off(row, c)) = u;
-            }
-            fence_async_smem();
-            mbar_arrive(bar(B_QFULL));
-        }
+        fence_async_smem();
+        mbar_arrive(bar(B_QFULL));
+
+        const RowInfo ri = row_info(a, it, row);
+        const bool live = ri.valid && ri.b < a.n_live[ri.r];
         const float cscale = kLog2e * rsqrtf(128.f);
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t col0 = (uint32_t)(64 * half);
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nchunks && ok; ++j) {
+        // Every softmax warp executes exactly one exchange barrier per chunk, even
+        // after an abort, so the named barrier can never deadlock.
+        for (int j = 0; j < nchunks; ++j) {
             const int sbuf = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + sbuf), (j >> 1) & 1, abort));
-            if (!ok) break;
-            fence_after_sync();
-            float s[128];
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + sbuf), (j >> 1) & 1, abort));
+            float s[64];
+            float mine = -INFINITY;
+            if (ok) {
+                fence_after_sync();
+                tmem_ld32(tmem + lane_base + sbuf * 128 + col0, s);
+                tmem_ld32(tmem + lane_base + sbuf * 128 + col0 + 32, s + 32);
+                tmem_wait_ld();
+                const int nvalid = n_keys - j * kBlockN - (int)col0;
+                float mxp[8];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + lane_base + sbuf * 128 + q4 * 32, s + q4 * 32);
-            tmem_wait_ld();
-            const int nvalid = min(kBlockN, n_keys - j * kBlockN);
-            // row max over the raw scores (the scale is positive), 8 independent chains
-            float mxp[8];
+                for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                if (c >= nvalid) s[c] = -INFINITY;
-                mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
+                for (int c = 0; c < 64; ++c) {
+                    if (c >= nvalid) s[c] = -INFINITY;
+                    mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
+                }
+                mine = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+                red[(sbuf * 2 + half) * 128 + row] = mine;
             }
-            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * cscale;
+            named_sync(1, kSoftmaxThreads);
+            if (!ok) continue;
+            const float mx = fmaxf(mine, red[(sbuf * 2 + (half ^ 1)) * 128 + row]) * cscale;
             float alpha = 1.f;
             bool rescale = false;
-            if (mx > m_used + 8.f) {
-                alpha = exp2f(m_used - mx);
+            if (mx > m_used + 8.f) {   // lazy rescaling: keep the old max unless it grew by 2^8
+                alpha = ex2(m_used - mx);
                 rescale = j > 0;
                 m_used = mx;
             }
+            // P buffer free and O complete up to chunk j-1 once P V of chunk j-1 is done
+            if (j >= 1) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE), (j - 1) & 1, abort));
+                if (!ok) continue;
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                fence_after_sync();
+                const float f = rescale ? alpha : 1.f;
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_base + 256 + col0 + q2 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= f;
+                    tmem_st32(tmem + lane_base + 256 + col0 + q2 * 32, o);
+                }
+                tmem_wait_st();
+            }
+            // exponentials, row sum and P (bf16), 8 columns (one 16-byte chunk) at a time
             const float neg_m = -m_used;
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-            uint32_t packed[64];
+            uint8_t *pb = base + kOffP;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float p0 = exp2f(fmaf(s[2 * c], cscale, neg_m));
-                const float p1 = exp2f(fmaf(s[2 * c + 1], cscale, neg_m));
-                sp[c & 7] += p0 + p1;
-                __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                packed[c] = *reinterpret_cast<uint32_t *>(&h);
-            }
-            const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-            l = l * alpha + sum;
-            if (j >= 2) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + sbuf), ((j - 2) >> 1) & 1, abort));
-                if (!ok) break;
-            }
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O must hold every P V product up to chunk j-1 before it is rescaled
-                const int jp = j - 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + (jp & 1)), (jp >> 1) & 1, abort));
-                if (!ok) break;
-                fence_after_sync();
-                const float f = rescale ? alpha : 1.f;
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w4[4];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float o[32];
-                    tmem_ld32(tmem + lane_base + 256 + q4 * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= f;
-                    tmem_st32(tmem + lane_base + 256 + q4 * 32, o);
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = ex2(fmaf(s[8 * c + 2 * e], cscale, neg_m));
+                    const float p1 = ex2(fmaf(s[8 * c + 2 * e + 1], cscale, neg_m));
+                    sp[(2 * e) & 7] += p0;
+                    sp[(2 * e + 1) & 7] += p1;
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    w4[e] = *reinterpret_cast<uint32_t *>(&h);
                 }
-                tmem_wait_st();
+                *reinterpret_cast<uint4 *>(pb + sw128_off(row, 8 * half + c)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            uint8_t *pb = base + kOffP + sbuf * kTile;
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-                *reinterpret_cast<uint4 *>(pb + sw128_off(row, c)) =
-                    make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+            l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
             fence_async_smem();
             fence_before_sync();
-            mbar_arrive(bar(B_PFULL + sbuf));
+            mbar_arrive(bar(B_PFULL));
         }
-        if (ok && nchunks > 0) {
-            const int jl = nchunks - 1;
-            if (__all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + (jl & 1)), (jl >> 1) & 1, abort))) {
-                fence_after_sync();
-                float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + (live ? gid : 0)) * 128;
+        if (ok && nchunks > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE), (nchunks - 1) & 1, abort));
+        if (ok) {
+            fence_after_sync();
+            // half 1 hands its partial row sum to half 0 (P buffers are free now)
+            float *xl = reinterpret_cast<float *>(base + kOffP);
+            if (half == 1) {
+                xl[row] = l;
+                mbar_arrive(bar(B_XCH));
+            } else {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH), 0, abort));
+            }
+            if (ok && !final_item) {
+                float o[64];
+                tmem_ld32(tmem + lane_base + 256 + col0, o);
+                tmem_ld32(tmem + lane_base + 256 + col0 + 32, o + 32);
+                tmem_wait_ld();
+                if (live) {
+                    float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + col0;
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4)
+                        *reinterpret_cast<float4 *>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+                    if (half == 0)
+                        a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(m_used, l + xl[row]);
+                }
+            } else if (ok && half == 0) {
+                // ---- fused Unshared stage + Merging stage + output for the whole row
+                // (the item covers its request's only KV segment): the beam's own
+                // tokens of steps 0..s, read through its direct indices
+                const Dims dm = a.dims;
+                const int s_now = a.step;
+                const float l_row = l + xl[row];
+                const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
+                const int64_t kvo = (beam_row * dm.Hkv + it.g) * 128;
+                const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+                const int64_t pool_req = (int64_t)ri.r * dm.BW * dm.Hkv * 128;
+                const __nv_bfloat16 *kp[kMaxSteps], *vp[kMaxSteps];
+                float sc[kMaxSteps];
+                const int n_tok = s_now + 1;
+                for (int i = 0; i < n_tok; ++i) {
+                    int slot = ri.b;
+                    if (i < s_now) slot = live ? a.st.anc[beam_row * dm.S + i] : 0;
+                    kp[i] = vp[i] = nullptr;
+                    if (slot < 0 || slot >= dm.BW) {
+                        if (live) set_status(a.status, XGR_DEV_INDEX);
+                        continue;
+                    }
+                    if (i == s_now) {
+                        kp[i] = a.k_new + kvo;
+                        vp[i] = a.v_new + kvo;
+                    } else {
+                        const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot * dm.Hkv + it.g) * 128;
+                        kp[i] = a.pool_k + o2;
+                        vp[i] = a.pool_v + o2;
+                    }
+                }
+                float m_new = m_used;
+                for (int i = 0; i < n_tok; ++i) {
+                    float acc = 0.f;
+                    if (live && kp[i]) {
+#pragma unroll 4
+                        for (int c = 0; c < 16; ++c) {
+                            float qf[8], kf[8];
+                            unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, c)), qf);
+                            unpack8(reinterpret_cast<const uint4 *>(kp[i])[c], kf);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
+                        }
+                    }
+                    sc[i] = kp[i] ? acc * cscale : -INFINITY;
+                    m_new = fmaxf(m_new, sc[i]);
+                }
+                const float a_s = ex2(m_used - m_new);
+                float l_new = l_row * a_s;
+                float pw[kMaxSteps];
+                for (int i = 0; i < n_tok; ++i) {
+                    pw[i] = kp[i] ? ex2(sc[i] - m_new) : 0.f;
+                    l_new += pw[i];
+                }
+                const float inv = live ? 1.f / l_new : 0.f;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     float o[32];
                     tmem_ld32(tmem + lane_base + 256 + q4 * 32, o);
                     tmem_wait_ld();
-                    if (live) {
+                    if (!ri.valid) continue;
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(dst + q4 * 32 + e) =
-                                make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+                    for (int e = 0; e < 32; ++e) o[e] = live ? o[e] * a_s : 0.f;
+                    if (live) {
+                        for (int i = 0; i < n_tok; ++i) {
+                            if (!vp[i]) continue;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                float vf[8];
+                                unpack8(reinterpret_cast<const uint4 *>(vp[i] + q4 * 32)[c], vf);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw[i], vf[e], o[8 * c + e]);
+                            }
+                        }
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + q4 * 32);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(o[8 * c + 2 * e] * inv,
+                                                                     o[8 * c + 2 * e + 1] * inv);
+                            w4[e] = *reinterpret_cast<uint32_t *>(&h);
+                        }
+                        dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
                 }
-                if (live) a.part.ml[(int64_t)it.slot * a.part.rows + gid] = make_float2(m_used, l);
+                if (ri.valid) a.lse[ri.gid] = live ? (m_new + __log2f(l_new)) * kLn2 : -INFINITY;
+                // append this step's k and v at Unshared slot (s, b), once per kv head
+                if (live && ri.hg == 0) {
+                    const int64_t dsto = s_now * pool_step + pool_req + ((int64_t)ri.b * dm.Hkv + it.g) * 128;
+                    uint4 *dk = reinterpret_cast<uint4 *>(a.pool_k + dsto);
+                    uint4 *dv = reinterpret_cast<uint4 *>(a.pool_v + dsto);
+                    const uint4 *sk = reinterpret_cast<const uint4 *>(a.k_new + kvo);
+                    const uint4 *sv = reinterpret_cast<const uint4 *>(a.v_new + kvo);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        dk[c] = sk[c];
+                        dv[c] = sv[c];
+                    }
+                }
             }
         }
     }
@@ -467,6 +653,14 @@ cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.maxThreadsPerBlock < kTcThreads) {
+            debug_log("attn_tc: %d registers/thread allow only %d threads per block", fa.numRegs,
+                      fa.maxThreadsPerBlock);
+            return cudaErrorLaunchOutOfResources;
+        }
         attr = true;
     }
     attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, a);

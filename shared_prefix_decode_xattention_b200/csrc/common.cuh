@@ -4,7 +4,10 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stdarg.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include "../../include/xgr.h"
 
@@ -56,7 +59,9 @@ struct WorkItem {
     int32_t row_begin;   // first segment row of this item
     int32_t n_rows;      // rows of this item
     int32_t slot;        // partial slot this item writes for its rows
-    int32_t pad[3];
+    int32_t flags;       // bit 0: final -- the item covers its requests' only KV segment
+                         // whole, so it also runs the Unshared and Merging stages
+    int32_t pad[2];
 };
 static_assert(sizeof(WorkItem) == 48, "WorkItem layout");
 
@@ -67,6 +72,18 @@ struct Partials {
     float2 *ml;      // [slots][rows]
     int64_t rows;    // B*BW*Hq of the workspace capacity
 };
+
+// Host-side diagnostics on stderr, only when the environment sets XGR_DEBUG.
+inline void debug_log(const char *fmt, ...) {
+    static const bool on = getenv("XGR_DEBUG") != nullptr;
+    if (!on) return;
+    va_list ap;
+    va_start(ap, fmt);
+    fprintf(stderr, "[xgr] ");
+    vfprintf(stderr, fmt, ap);
+    fprintf(stderr, "\n");
+    va_end(ap);
+}
 
 __device__ __forceinline__ void set_status(int32_t *status, int32_t bit) {
     atomicOr(status, bit);

@@ -33,6 +33,16 @@ struct TcArgs {
     const int32_t *n_live;
     Partials part;
     int32_t *status;
+    // fused epilogue of final items (Unshared stage, Merging stage, append)
+    const __nv_bfloat16 *k_new;    // [B][BW][Hkv][D]
+    const __nv_bfloat16 *v_new;
+    __nv_bfloat16 *pool_k;         // [S][Bcap][BW][Hkv][D]
+    __nv_bfloat16 *pool_v;
+    __nv_bfloat16 *out;            // [B][BW][Hq][D]
+    float *lse;                    // [B][BW][Hq]
+    BeamState st;
+    int Bcap;
+    int step;
 };
 // 2-D tensor map over a [rows][128] bf16 store, 64 x 128 boxes, 128-byte swizzle.
 cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows);
@@ -52,7 +62,7 @@ struct MergeArgs {
     Dims dims;
     int Bcap;
     int step;
-    const int32_t *n_slots;        // [B] partial slots of each request
+    const int32_t *n_slots;        // [B] partial slots of each request; -1: done by a fused item
     Partials part;
 };
 cudaError_t launch_attn_merge(const MergeArgs &a, cudaStream_t st);

@@ -147,6 +147,7 @@ struct xgr_ctx {
     int planned_B = -1;
     int n_small[2] = {0, 0};   // small-row work items of each plan (then n_tc[] tensor-core ones)
     int n_tc[2] = {0, 0};
+    int n_unfused[2] = {0, 0};   // requests the merge kernel still has to finish
     bool has_tc = false;       // tensor-core Shared stage available (D = 128, tensor maps built)
     CUtensorMap tmk, tmv;
     // decode state
@@ -191,10 +192,11 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     for (auto &sg : segs)
         for (int r : sg.members) nseg[r]++;
 
-    // kind of every segment: tensor-core tiles of 128 rows when it has more
-    // than kSmallRows rows (and D = 128), else the small-row kernel
+    // kind of every segment: tensor-core tiles of 128 rows whenever D = 128
+    // (few rows waste tensor work but the stage then streams K/V at HBM speed),
+    // else the small-row kernel
     auto rows_of = [&](const Seg &sg) { return (int64_t)sg.members.size() * nb * G; };
-    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > kSmallRows; };
+    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > 0; };
     // split factor per kind: the fewest waves x keys per item (+ a fixed
     // per-item overhead in key units), over the resident CTAs of the GPU
     auto pick_split = [&](bool tc) {
@@ -228,6 +230,7 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     std::vector<WorkItem> items_small, items_tc;
     std::vector<int32_t> members;
     std::vector<int32_t> nslots(B, 0);
+    std::vector<char> fused(B, 0);
     for (auto &sg : segs) {
         const bool tc = is_tc(sg);
         const int64_t R = tc ? kTcRows : kSmallRows;
@@ -248,6 +251,11 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         const int member_off = (int)members.size();
         for (int r : sg.members) members.push_back(r);
         auto &dst = tc ? items_tc : items_small;
+        // a final item runs the Unshared and Merging stages itself: no split and
+        // no other segment for any of its requests
+        const bool final_seg = tc && splits == 1 && max_seg == 1;
+        if (final_seg)
+            for (int r : sg.members) fused[r] = 1;
         for (int g = 0; g < cf.n_kv_heads; ++g)
             for (int64_t sp = 0; sp < splits; ++sp)
                 for (int64_t t = 0; t < tiles; ++t) {
@@ -261,12 +269,18 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
                     it.row_begin = (int32_t)(t * R);
                     it.n_rows = (int32_t)std::min<int64_t>(R, rows - t * R);
                     it.slot = (int32_t)(slot0 + sp);
+                    it.flags = final_seg ? 1 : 0;
                     dst.push_back(it);
                 }
         for (int r : sg.members) nslots[r] = (int32_t)(slot0 + splits);
     }
     std::vector<WorkItem> items(items_small);
     items.insert(items.end(), items_tc.begin(), items_tc.end());
+    int unfused = 0;
+    for (int r = 0; r < B; ++r) {
+        if (fused[r]) nslots[r] = -1;   // the merge kernel skips this request
+        else ++unfused;
+    }
     if ((int64_t)items.size() > c->L.item_cap || (int64_t)members.size() > c->L.member_cap)
         return XGR_ERR_CAPACITY;
     if (!items.empty() &&
@@ -282,6 +296,7 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         return XGR_ERR_CUDA;
     c->n_small[which] = (int)items_small.size();
     c->n_tc[which] = (int)items_tc.size();
+    c->n_unfused[which] = unfused;
     return XGR_OK;
 }
 
@@ -535,7 +550,13 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
     sa.nb = (which == 0) ? 1 : c->cfg.beam_width;
     sa.n_live = c->st.n_live;
     sa.part = partials_of(c);
-    if (launch_attn_small(sa, c->n_small[which], s) != cudaSuccess) return XGR_ERR_CUDA;
+    {
+        const cudaError_t e = launch_attn_small(sa, c->n_small[which], s);
+        if (e != cudaSuccess) {
+            debug_log("decode_step: small-row launch failed: %s", cudaGetErrorString(e));
+            return XGR_ERR_CUDA;
+        }
+    }
     if (c->n_tc[which] > 0) {
         TcArgs ta;
         ta.items = sa.items + c->n_small[which];
@@ -547,8 +568,26 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
         ta.n_live = sa.n_live;
         ta.part = sa.part;
         ta.status = c->st.status;
-        if (launch_attn_tc(c->tmk, c->tmv, ta, c->n_tc[which], s) != cudaSuccess)
+        ta.k_new = static_cast<const __nv_bfloat16 *>(d_k_new);
+        ta.v_new = static_cast<const __nv_bfloat16 *>(d_v_new);
+        ta.pool_k = c->at<__nv_bfloat16>(c->L.pool_k);
+        ta.pool_v = c->at<__nv_bfloat16>(c->L.pool_v);
+        ta.out = static_cast<__nv_bfloat16 *>(d_out);
+        ta.lse = d_lse;
+        ta.st = c->st;
+        ta.Bcap = c->cfg.max_requests;
+        ta.step = step;
+        const cudaError_t e = launch_attn_tc(c->tmk, c->tmv, ta, c->n_tc[which], s);
+        if (e != cudaSuccess) {
+            debug_log("decode_step: tensor-core launch failed: %s", cudaGetErrorString(e));
             return XGR_ERR_CUDA;
+        }
+    }
+    // the merge kernel also writes the rows of dead beams; at step 0 only beam 0
+    // of each request is covered by Shared-stage work items
+    if (c->n_unfused[which] == 0 && (which == 1 || c->cfg.beam_width == 1)) {
+        if (c->cfg.vocab == 0) c->cur_step = step + 1;
+        return XGR_OK;
     }
     MergeArgs ma;
     ma.q = sa.q;
@@ -564,7 +603,13 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
     ma.step = step;
     ma.n_slots = c->at<int32_t>(c->L.plan_nslots[which]);
     ma.part = sa.part;
-    if (launch_attn_merge(ma, s) != cudaSuccess) return XGR_ERR_CUDA;
+    {
+        const cudaError_t e = launch_attn_merge(ma, s);
+        if (e != cudaSuccess) {
+            debug_log("decode_step: merge launch failed: %s", cudaGetErrorString(e));
+            return XGR_ERR_CUDA;
+        }
+    }
     if (c->cfg.vocab == 0) c->cur_step = step + 1;   // attention-only: no selection step
     return XGR_OK;
 }
