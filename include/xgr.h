@@ -224,9 +224,10 @@ xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_co
  * xgr_beam_select does (same order, same tie-break, same bits).
  * Allocation: none.  Its scratch is one static device array of 8 MiB per GPU
  * (held by every GPU that loads the library until the process exits); a call
- * needs B*BW*(8*K + 8) bytes of it and returns XGR_ERR_CAPACITY beyond that.
+ * needs about 36 bytes per beam row (B*BW rows, up to about 233 000 rows) and
+ * returns XGR_ERR_CAPACITY beyond that.
  * The first call on a device looks the array up (cudaGetSymbolAddress) and
- * sets a kernel attribute, so make that first call before any stream capture.
+ * may set a kernel attribute, so make that first call before any stream capture.
  * All calls share the array: calls that overlap on the GPU race and must be
  * serialised by the caller.  NaN scores and out-of-range mask tokens are
  * skipped, as in the context path, but not reported.  Host-side argument

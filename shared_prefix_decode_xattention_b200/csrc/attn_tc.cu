@@ -56,7 +56,7 @@ constexpr uint32_t kSpinLimit = 1u << 22;
 
 // barrier slots (8 bytes each) after kOffBar
 enum { B_KFULL = 0, B_KEMPTY = 3, B_VFULL = 6, B_VEMPTY = 8, B_SFULL = 10, B_PFULL = 12,
-       B_PVDONE = 13, B_QFULL = 14, B_DRAIN = 15, B_XCH = 16, B_COUNT = 17 };
+       B_PVDONE = 13, B_QFULL = 14, B_DRAIN = 15, B_XCH = 16, B_COUNT = 18 };   // B_XCH: 2 halves
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar(B_QFULL), kSoftmaxThreads);
             mbar_init(bar(B_DRAIN), 1);
             mbar_init(bar(B_XCH), kSoftmaxThreads / 2);
+            mbar_init(bar(B_XCH + 1), kSoftmaxThreads / 2);
             *abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const uint32_t offp = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
                         umma_bf16(tmem + 256u, umma_desc(kp + offp, 16, 1024),
                                   umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
-                                  (jp > 0 || k > 0) ? 1u : 0u);
+                                  (jp > 0 || k > 0 || final_item) ? 1u : 0u);
                     }
                     umma_commit(bar(B_PVDONE));
                     umma_commit(bar(B_VEMPTY + sv));
@@ -401,6 +402,98 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t col0 = (uint32_t)(64 * half);
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
+        const Dims dm = a.dims;
+        const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
+        const int64_t kvo = (beam_row * dm.Hkv + it.g) * 128;
+        const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+        const int64_t pool_req = (int64_t)ri.r * dm.BW * dm.Hkv * 128;
+        if (final_item) {
+            // ---- Unshared stage first (the item covers its requests' only KV
+            // segment): the beam's own tokens of steps 0..s, read through its
+            // direct indices, seed the online softmax -- their max, their sum (on
+            // half 0) and their weighted values in the TMEM O accumulator.
+            const int s_now = a.step;
+            const int n_tok = s_now + 1;
+            const __nv_bfloat16 *kp[kMaxSteps], *vp[kMaxSteps];
+            for (int i = 0; i < n_tok; ++i) {
+                kp[i] = vp[i] = nullptr;
+                if (!live) continue;
+                const int slot = (i == s_now) ? ri.b : a.st.anc[beam_row * dm.S + i];
+                if (slot < 0 || slot >= dm.BW) {
+                    set_status(a.status, XGR_DEV_INDEX);
+                    continue;
+                }
+                if (i == s_now) {
+                    kp[i] = a.k_new + kvo;
+                    vp[i] = a.v_new + kvo;
+                } else {
+                    const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot * dm.Hkv + it.g) * 128;
+                    kp[i] = a.pool_k + o2;
+                    vp[i] = a.pool_v + o2;
+                }
+            }
+            float qf[64];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)), qf + 8 * c);
+            float *xd = reinterpret_cast<float *>(base + kOffP);   // [2 halves][kMaxSteps][128]
+            for (int i = 0; i < n_tok; ++i) {
+                float acc = 0.f;
+                if (kp[i]) {
+                    uint4 kv[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) kv[c] = reinterpret_cast<const uint4 *>(kp[i] + col0)[c];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float kf[8];
+                        unpack8(kv[c], kf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc = fmaf(qf[8 * c + e], kf[e], acc);
+                    }
+                }
+                xd[(half * kMaxSteps + i) * 128 + row] = acc;
+            }
+            named_sync(1, kSoftmaxThreads);
+            float sc[kMaxSteps];
+            float m_u = -INFINITY;
+            for (int i = 0; i < n_tok; ++i) {
+                sc[i] = kp[i] ? (xd[i * 128 + row] + xd[(kMaxSteps + i) * 128 + row]) * cscale : -INFINITY;
+                m_u = fmaxf(m_u, sc[i]);
+            }
+            named_sync(1, kSoftmaxThreads);   // the exchange area is reused by P afterwards
+            float o[64];
+#pragma unroll
+            for (int e = 0; e < 64; ++e) o[e] = 0.f;
+            float l_u = 0.f;
+            for (int i = 0; i < n_tok; ++i) {
+                if (!vp[i]) continue;
+                const float pw = ex2(sc[i] - m_u);
+                l_u += pw;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float vf[8];
+                    unpack8(reinterpret_cast<const uint4 *>(vp[i] + col0)[c], vf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw, vf[e], o[8 * c + e]);
+                }
+            }
+            tmem_st32(tmem + lane_base + 256 + col0, o);
+            tmem_st32(tmem + lane_base + 256 + col0 + 32, o + 32);
+            tmem_wait_st();
+            if (live) {
+                m_used = m_u;
+                l = half == 0 ? l_u : 0.f;   // the row sum is split over the halves
+            }
+            // append this step's k (half 0) and v (half 1) at Unshared slot (s, b), once per kv head
+            if (live && ri.hg == 0) {
+                const __nv_bfloat16 *src = (half == 0 ? a.k_new : a.v_new) + kvo;
+                __nv_bfloat16 *dst = (half == 0 ? a.pool_k : a.pool_v) + s_now * pool_step + pool_req +
+                                     ((int64_t)ri.b * dm.Hkv + it.g) * 128;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    reinterpret_cast<uint4 *>(dst)[c] = reinterpret_cast<const uint4 *>(src)[c];
+            }
+        }
         // Every softmax warp executes exactly one exchange barrier per chunk, even
         // after an abort, so the named barrier can never deadlock.
         for (int j = 0; j < nchunks; ++j) {
@@ -433,7 +526,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool rescale = false;
             if (mx > m_used + 8.f) {   // lazy rescaling: keep the old max unless it grew by 2^8
                 alpha = ex2(m_used - mx);
-                rescale = j > 0;
+                rescale = j > 0 || final_item;   // O holds the Unshared stage in final items
                 m_used = mx;
             }
             // P buffer free and O complete up to chunk j-1 once P V of chunk j-1 is done
@@ -485,128 +578,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE), (nchunks - 1) & 1, abort));
         if (ok) {
             fence_after_sync();
-            // half 1 hands its partial row sum to half 0 (P buffers are free now)
+            // the halves swap their partial row sums (P buffer is free now)
             float *xl = reinterpret_cast<float *>(base + kOffP);
-            if (half == 1) {
-                xl[row] = l;
-                mbar_arrive(bar(B_XCH));
-            } else {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH), 0, abort));
-            }
-            if (ok && !final_item) {
+            xl[half * 128 + row] = l;
+            mbar_arrive(bar(B_XCH + half));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH + (half ^ 1)), 0, abort));
+            const float l_row = l + xl[(half ^ 1) * 128 + row];
+            if (ok) {
                 float o[64];
                 tmem_ld32(tmem + lane_base + 256 + col0, o);
                 tmem_ld32(tmem + lane_base + 256 + col0 + 32, o + 32);
                 tmem_wait_ld();
-                if (live) {
-                    float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + col0;
-#pragma unroll
-                    for (int e = 0; e < 64; e += 4)
-                        *reinterpret_cast<float4 *>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
-                    if (half == 0)
-                        a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(m_used, l + xl[row]);
-                }
-            } else if (ok && half == 0) {
-                // ---- fused Unshared stage + Merging stage + output for the whole row
-                // (the item covers its request's only KV segment): the beam's own
-                // tokens of steps 0..s, read through its direct indices
-                const Dims dm = a.dims;
-                const int s_now = a.step;
-                const float l_row = l + xl[row];
-                const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
-                const int64_t kvo = (beam_row * dm.Hkv + it.g) * 128;
-                const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
-                const int64_t pool_req = (int64_t)ri.r * dm.BW * dm.Hkv * 128;
-                const __nv_bfloat16 *kp[kMaxSteps], *vp[kMaxSteps];
-                float sc[kMaxSteps];
-                const int n_tok = s_now + 1;
-                for (int i = 0; i < n_tok; ++i) {
-                    int slot = ri.b;
-                    if (i < s_now) slot = live ? a.st.anc[beam_row * dm.S + i] : 0;
-                    kp[i] = vp[i] = nullptr;
-                    if (slot < 0 || slot >= dm.BW) {
-                        if (live) set_status(a.status, XGR_DEV_INDEX);
-                        continue;
-                    }
-                    if (i == s_now) {
-                        kp[i] = a.k_new + kvo;
-                        vp[i] = a.v_new + kvo;
-                    } else {
-                        const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot * dm.Hkv + it.g) * 128;
-                        kp[i] = a.pool_k + o2;
-                        vp[i] = a.pool_v + o2;
-                    }
-                }
-                float m_new = m_used;
-                for (int i = 0; i < n_tok; ++i) {
-                    float acc = 0.f;
-                    if (live && kp[i]) {
-#pragma unroll 4
-                        for (int c = 0; c < 16; ++c) {
-                            float qf[8], kf[8];
-                            unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, c)), qf);
-                            unpack8(reinterpret_cast<const uint4 *>(kp[i])[c], kf);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
-                        }
-                    }
-                    sc[i] = kp[i] ? acc * cscale : -INFINITY;
-                    m_new = fmaxf(m_new, sc[i]);
-                }
-                const float a_s = ex2(m_used - m_new);
-                float l_new = l_row * a_s;
-                float pw[kMaxSteps];
-                for (int i = 0; i < n_tok; ++i) {
-                    pw[i] = kp[i] ? ex2(sc[i] - m_new) : 0.f;
-                    l_new += pw[i];
-                }
-                const float inv = live ? 1.f / l_new : 0.f;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float o[32];
-                    tmem_ld32(tmem + lane_base + 256 + q4 * 32, o);
-                    tmem_wait_ld();
-                    if (!ri.valid) continue;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = live ? o[e] * a_s : 0.f;
+                if (!final_item) {
                     if (live) {
-                        for (int i = 0; i < n_tok; ++i) {
-                            if (!vp[i]) continue;
+                        float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + col0;
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                float vf[8];
-                                unpack8(reinterpret_cast<const uint4 *>(vp[i] + q4 * 32)[c], vf);
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw[i], vf[e], o[8 * c + e]);
-                            }
-                        }
+                        for (int e = 0; e < 64; e += 4)
+                            *reinterpret_cast<float4 *>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+                        if (half == 0)
+                            a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(m_used, l_row);
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + q4 * 32);
+                } else if (ri.valid) {
+                    // final: O / l in bf16, LSE = m + log2(l) in natural log; dead rows 0 / -inf
+                    const float inv = live ? 1.f / l_row : 0.f;
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + col0);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t w4[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(o[8 * c + 2 * e] * inv,
-                                                                     o[8 * c + 2 * e + 1] * inv);
+                            const float v0 = live ? o[8 * c + 2 * e] * inv : 0.f;
+                            const float v1 = live ? o[8 * c + 2 * e + 1] * inv : 0.f;
+                            __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
                             w4[e] = *reinterpret_cast<uint32_t *>(&h);
                         }
                         dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     }
-                }
-                if (ri.valid) a.lse[ri.gid] = live ? (m_new + __log2f(l_new)) * kLn2 : -INFINITY;
-                // append this step's k and v at Unshared slot (s, b), once per kv head
-                if (live && ri.hg == 0) {
-                    const int64_t dsto = s_now * pool_step + pool_req + ((int64_t)ri.b * dm.Hkv + it.g) * 128;
-                    uint4 *dk = reinterpret_cast<uint4 *>(a.pool_k + dsto);
-                    uint4 *dv = reinterpret_cast<uint4 *>(a.pool_v + dsto);
-                    const uint4 *sk = reinterpret_cast<const uint4 *>(a.k_new + kvo);
-                    const uint4 *sv = reinterpret_cast<const uint4 *>(a.v_new + kvo);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        dk[c] = sk[c];
-                        dv[c] = sv[c];
-                    }
+                    if (half == 0) a.lse[ri.gid] = live ? (m_used + __log2f(l_row)) * kLn2 : -INFINITY;
                 }
             }
         }

@@ -58,39 +58,74 @@ __device__ __forceinline__ int row_children(const MaskArgs &a, int64_t row) {
     return a.trie.ptr[a.step][node + 1] - a.trie.ptr[a.step][node];
 }
 
-constexpr int kScanThreads = 1024;
+constexpr int kMaskThreads = 1024;
 
-// One CTA: children count of every beam row, exclusive scan -> row_ptr.
-__global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(MaskArgs a) {
-    __shared__ int64_t part[kScanThreads];
+// block-wide exclusive scan of one value per thread (1024 threads); returns the
+// exclusive prefix of this thread and writes the block total to *total
+__device__ int64_t block_exclusive_scan(int64_t v, int64_t *warp_tot, int64_t *total) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int64_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int64_t w = warp_tot[lane];
+        int64_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        warp_tot[lane] = wi - w;   // exclusive prefix of each warp
+        if (lane == 31) *total = wi;
+    }
+    __syncthreads();
+    return warp_tot[warp] + incl - v;
+}
+
+// The CSR mask in two kernels.  mask_scan_kernel (one CTA): each thread owns a
+// contiguous chunk of rows, loads their trie nodes and child ranges in
+// independent batches, and a block scan turns the counts into row_ptr.
+// mask_copy_kernel: one warp per row copies the node's sorted children.
+__global__ void __launch_bounds__(kMaskThreads) mask_scan_kernel(MaskArgs a) {
+    __shared__ int64_t warp_tot[32];
+    __shared__ int64_t tot;
     const int64_t n_rows = (int64_t)a.dims.B * a.dims.BW;
     const int tid = threadIdx.x;
-    const int64_t chunk = (n_rows + kScanThreads - 1) / kScanThreads;
-    const int64_t lo = min(n_rows, tid * chunk), hi = min(n_rows, lo + chunk);
+    const int64_t chunk = (n_rows + kMaskThreads - 1) / kMaskThreads;
+    const int64_t lo = min(n_rows, (int64_t)tid * chunk), hi = min(n_rows, lo + chunk);
+    constexpr int U = 8;
     int64_t sum = 0;
-    for (int64_t row = lo; row < hi; ++row) sum += row_children(a, row);
-    part[tid] = sum;
-    __syncthreads();
-    for (int o = 1; o < kScanThreads; o <<= 1) {   // inclusive Hillis-Steele scan
-        int64_t v = (tid >= o) ? part[tid - o] : 0;
-        __syncthreads();
-        part[tid] += v;
-        __syncthreads();
+    for (int64_t r0 = lo; r0 < hi; r0 += U) {
+        int c[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) c[u] = (r0 + u < hi) ? row_children(a, r0 + u) : 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) sum += c[u];
     }
-    int64_t off = part[tid] - sum;
-    const int64_t total = part[kScanThreads - 1];
-    for (int64_t row = lo; row < hi; ++row) {
-        a.row_ptr[row] = (int32_t)min(off, a.cap);
-        off += row_children(a, row);
+    const int64_t ex = block_exclusive_scan(sum, warp_tot, &tot);
+    int64_t off = ex;
+    for (int64_t r0 = lo; r0 < hi; r0 += U) {
+        int c[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) c[u] = (r0 + u < hi) ? row_children(a, r0 + u) : 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (r0 + u < hi) a.row_ptr[r0 + u] = (int32_t)min(off, a.cap);
+            off += c[u];
+        }
     }
     if (tid == 0) {
-        a.row_ptr[n_rows] = (int32_t)min(total, a.cap);
-        if (total > a.cap) set_status(a.st.status, XGR_DEV_CAPACITY);
+        a.row_ptr[n_rows] = (int32_t)min(tot, a.cap);
+        if (tot > a.cap) set_status(a.st.status, XGR_DEV_CAPACITY);
     }
 }
 
-// One warp per beam row: copy the node's sorted children into the CSR row.
-__global__ void mask_fill_kernel(MaskArgs a) {
+__global__ void mask_copy_kernel(MaskArgs a) {
     const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     const int64_t n_rows = (int64_t)a.dims.B * a.dims.BW;
@@ -103,12 +138,6 @@ __global__ void mask_fill_kernel(MaskArgs a) {
 }
 
 // ------------------------------------------------------------------ sorting helpers
-
-__device__ __forceinline__ int pow2_ceil(int n) {
-    int p = 1;
-    while (p < n) p <<= 1;
-    return p;
-}
 
 // Ascending bitonic sort of n (a power of two) keys in shared memory.
 __device__ void block_sort(uint64_t *buf, int n) {
@@ -168,148 +197,230 @@ __device__ void radix_select(const Cand &cand, int64_t E, int want, int *hist, i
     }
 }
 
-// ------------------------------------------------------------------ per-beam candidates
+// ------------------------------------------------------------------ selection
+//
+// Kernel 1 (row statistics): per live beam, the row log-sum-exp over the full
+// vocabulary (logits mode; one online pass, 16-byte loads) and the beam's best
+// kSampleK candidate keys.
+// Kernel 2 (select): per request, tau = the BW-th best key of the beams'
+// samples.  The samples are real candidates, so at least BW candidates rank at
+// or above tau and the BW winners all do: one pass keeps the candidates at or
+// above tau (usually a few hundred), sorts them and takes the first BW.  When
+// the survivors overflow shared memory (or the sample is too small) an exact
+// radix select over all candidates takes over.  With K >= BW the per-beam
+// top-K cut never removes a winner, so the flat top-BW computed here equals
+// the two-stage selection.
 
-constexpr int kRowThreads = 256;
-constexpr int kMaxK = 1024;
-
-struct RowCand {
-    const float *x;
-    const uint32_t *bits;
-    const int32_t *cols;
-    int32_t *status;
-    float cum, lse;
-    int dense, logits, V, b;
-    __device__ bool operator()(int64_t e, uint64_t &key) const {
-        int t;
-        if (dense) {
-            t = (int)e;
-            if (!((bits[t >> 5] >> (t & 31)) & 1u)) return false;
-        } else {
-            t = cols[e];
-            if (t < 0 || t >= V) {
-                set_status(status, XGR_DEV_MASK);
-                return false;
-            }
-        }
-        float lp = x[t];
-        if (logits) lp = lp - lse;
-        float k = cum + lp;   // one fp32 add: the score of (beam b, token t)
-        if (isnan(k)) {
-            set_status(status, XGR_DEV_NAN);
-            return false;
-        }
-        if (k == 0.f) k = 0.f;   // -0.0 -> +0.0
-        key = ((uint64_t)score_to_desc_bits(k) << 32) | (uint32_t)(b * V + t);
-        return true;
-    }
-};
-
-// One CTA per live beam row: (logits mode) the row's log-sum-exp over the
-// whole vocabulary, then the beam's top-K valid candidates, sorted.
-__global__ void __launch_bounds__(kRowThreads) select_row_kernel(SelectArgs a, int rows_per_req) {
-    __shared__ uint64_t buf[kMaxK];
-    __shared__ int hist[256];
-    __shared__ int sc[4];
-    __shared__ float red[kRowThreads / 32];
-    const Dims dm = a.dims;
-    const int r = blockIdx.x / rows_per_req, b = blockIdx.x % rows_per_req;
-    const int64_t row = (int64_t)r * dm.BW + b;
-    const int tid = threadIdx.x;
-    if (b >= a.st.n_live[r]) {
-        if (tid == 0) a.counts[row] = 0;
-        return;
-    }
-    const float *x = a.scores + row * dm.V;
-    const float cum = a.st.cum[row];
-
-    float lse = 0.f;
-    if (a.logits) {
-        float mx = -INFINITY;
-        int nan = 0;
-        for (int t = tid; t < dm.V; t += kRowThreads) {
-            const float v = x[t];
-            nan |= isnan(v);
-            mx = fmaxf(mx, v);
-        }
-        if (nan) set_status(a.st.status, XGR_DEV_NAN);
-        mx = warp_max(mx);
-        if (tid % 32 == 0) red[tid / 32] = mx;
-        __syncthreads();
-        mx = red[0];
-        for (int w = 1; w < kRowThreads / 32; ++w) mx = fmaxf(mx, red[w]);
-        __syncthreads();
-        float sum = 0.f;
-        for (int t = tid; t < dm.V; t += kRowThreads) sum += expf(x[t] - mx);
-        sum = warp_sum(sum);
-        if (tid % 32 == 0) red[tid / 32] = sum;
-        __syncthreads();
-        sum = 0.f;
-        for (int w = 0; w < kRowThreads / 32; ++w) sum += red[w];
-        lse = mx + logf(sum);
-        if (tid == 0) a.row_lse[row] = lse;
-    }
-
-    RowCand cand;
-    cand.x = x;
-    cand.bits = a.bits;
-    cand.status = a.st.status;
-    cand.cum = cum;
-    cand.lse = lse;
-    cand.dense = a.dense;
-    cand.logits = a.logits;
-    cand.V = dm.V;
-    cand.b = b;
-    int64_t E;
-    if (a.dense) {
-        cand.cols = nullptr;
-        E = dm.V;
-    } else {
-        const int beg = a.row_ptr[row];
-        cand.cols = a.cols + beg;
-        E = a.row_ptr[row + 1] - beg;
-    }
-
-    // number of valid candidates
-    if (tid == 0) sc[3] = 0;
-    __syncthreads();
-    int mine = 0;
-    for (int64_t e = tid; e < E; e += kRowThreads) {
-        uint64_t key;
-        mine += cand(e, key) ? 1 : 0;
-    }
-    atomicAdd(&sc[3], mine);
-    __syncthreads();
-    const int c = sc[3];
-    __syncthreads();
-
-    uint64_t prefix = ~0ull, mask = 0;
-    if (c > dm.K) radix_select(cand, E, dm.K, hist, sc, prefix, mask);
-    const int n_sel = min(c, dm.K);
-
-    if (tid == 0) sc[3] = 0;
-    __syncthreads();
-    for (int64_t e = tid; e < E; e += kRowThreads) {
-        uint64_t key;
-        if (cand(e, key) && (key & mask) <= prefix) {
-            const int pos = atomicAdd(&sc[3], 1);
-            if (pos < kMaxK) buf[pos] = key;
-        }
-    }
-    __syncthreads();
-    const int P = pow2_ceil(max(n_sel, 1));
-    for (int i = n_sel + tid; i < P; i += kRowThreads) buf[i] = kNoKey;
-    __syncthreads();
-    block_sort(buf, P);
-    uint64_t *dst = a.lists + row * dm.K;
-    for (int i = tid; i < n_sel; i += kRowThreads) dst[i] = buf[i];
-    if (tid == 0) a.counts[row] = n_sel;
+__device__ __forceinline__ void cswap(uint64_t &x, uint64_t &y) {
+    const uint64_t lo = x < y ? x : y, hi = x < y ? y : x;
+    x = lo;
+    y = hi;
 }
 
-// ------------------------------------------------------------------ per-request select + rewire
+__device__ __forceinline__ void top4_insert(uint64_t (&t)[kSampleK], uint64_t key) {
+    if (key >= t[3]) return;
+    t[3] = key;
+    cswap(t[2], t[3]);
+    cswap(t[1], t[2]);
+    cswap(t[0], t[1]);
+}
 
-constexpr int kReqThreads = 512;
-constexpr int kSurvCap = 4096;
+// the 4 smallest keys of two ascending 4-lists, ascending (bitonic merge)
+__device__ __forceinline__ void top4_merge(uint64_t (&t)[kSampleK], const uint64_t (&u)[kSampleK]) {
+    uint64_t m0 = t[0] < u[3] ? t[0] : u[3], m1 = t[1] < u[2] ? t[1] : u[2];
+    uint64_t m2 = t[2] < u[1] ? t[2] : u[1], m3 = t[3] < u[0] ? t[3] : u[0];
+    cswap(m0, m2);
+    cswap(m1, m3);
+    cswap(m0, m1);
+    cswap(m2, m3);
+    t[0] = m0; t[1] = m1; t[2] = m2; t[3] = m3;
+}
+
+__device__ __forceinline__ void top4_warp(uint64_t (&t)[kSampleK]) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        uint64_t u[kSampleK];
+#pragma unroll
+        for (int i = 0; i < kSampleK; ++i) u[i] = __shfl_xor_sync(0xffffffffu, t[i], o);
+        top4_merge(t, u);
+    }
+}
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// online (max, sum of 2^((x - max) log2 e)) of one value into (m, s)
+__device__ __forceinline__ void lse_add(float &m, float &s, float v) {
+    if (v > m) {
+        s = s * ex2f((m - v) * kLog2e) + 1.f;
+        m = v;
+    } else if (v != -INFINITY) {
+        s += ex2f((v - m) * kLog2e);
+    }
+}
+__device__ __forceinline__ void lse_combine(float &m, float &s, float m2, float s2) {
+    if (m2 > m) {
+        s = s * ex2f((m - m2) * kLog2e) + s2;
+        m = m2;
+    } else if (m2 != -INFINITY) {
+        s += s2 * ex2f((m2 - m) * kLog2e);
+    }
+}
+
+// key of (beam b, token t): one fp32 add of the beam's cumulative score and
+// the token's log-prob; -0.0 is canonical +0.0; NaN is reported and skipped
+__device__ __forceinline__ bool make_key(float cum, float lp, int b, int t, int V, int32_t *status,
+                                         uint64_t &key) {
+    float k = cum + lp;
+    if (isnan(k)) {
+        set_status(status, XGR_DEV_NAN);
+        return false;
+    }
+    if (k == 0.f) k = 0.f;
+    key = ((uint64_t)score_to_desc_bits(k) << 32) | (uint32_t)(b * V + t);
+    return true;
+}
+
+constexpr int kStatThreads = 256;
+
+// cta_per_row = 1 (dense first step): one CTA per request (its single live beam);
+// otherwise one warp per beam row.
+__global__ void __launch_bounds__(kStatThreads, 1) row_stats_kernel(SelectArgs a, int cta_per_row) {
+    __shared__ float red_m[kStatThreads / 32], red_s[kStatThreads / 32];
+    __shared__ uint64_t red_k[kStatThreads / 32][kSampleK];
+    const Dims dm = a.dims;
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int r, b, t0, stride;
+    if (cta_per_row) {
+        r = blockIdx.x;
+        b = 0;
+        t0 = threadIdx.x;
+        stride = kStatThreads;
+    } else {
+        const int64_t gw = (int64_t)blockIdx.x * (kStatThreads / 32) + warp;
+        if (gw >= (int64_t)dm.B * dm.BW) return;
+        r = (int)(gw / dm.BW);
+        b = (int)(gw % dm.BW);
+        t0 = lane;
+        stride = 32;
+    }
+    if (b >= a.n_live[r]) return;
+    const int64_t row = (int64_t)r * dm.BW + b;
+    const float *x = a.scores + row * dm.V;
+    float lse = 0.f;
+    if (a.logits) {
+        float m = -INFINITY, s = 0.f;
+        bool nan = false;
+        if ((dm.V & 3) == 0) {
+            // 16 independent 16-byte loads in flight per thread
+            const float4 *x4 = reinterpret_cast<const float4 *>(x);
+            const int n4 = dm.V / 4;
+            constexpr int U = 16;
+            for (int i0 = t0; i0 < n4; i0 += U * stride) {
+                float4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = i0 + u * stride;
+                    v[u] = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    nan |= isnan(v[u].x) | isnan(v[u].y) | isnan(v[u].z) | isnan(v[u].w);
+                    const float cm = fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w));
+                    if (cm > m) {
+                        s *= ex2f((m - cm) * kLog2e);
+                        m = cm;
+                    }
+                    if (cm != -INFINITY) {
+                        s += ex2f((v[u].x - m) * kLog2e) + ex2f((v[u].y - m) * kLog2e) +
+                             ex2f((v[u].z - m) * kLog2e) + ex2f((v[u].w - m) * kLog2e);
+                    }
+                }
+            }
+        } else {
+            for (int i = t0; i < dm.V; i += stride) {
+                nan |= isnan(x[i]);
+                lse_add(m, s, x[i]);
+            }
+        }
+        if (nan) set_status(a.status, XGR_DEV_NAN);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            lse_combine(m, s, m2, s2);
+        }
+        if (cta_per_row) {
+            if (lane == 0) {
+                red_m[warp] = m;
+                red_s[warp] = s;
+            }
+            __syncthreads();
+            m = red_m[0];
+            s = red_s[0];
+            for (int w = 1; w < kStatThreads / 32; ++w) lse_combine(m, s, red_m[w], red_s[w]);
+        }
+        lse = m + logf(s);
+    }
+    const float cum = a.cum[row];
+    uint64_t t[kSampleK] = {kNoKey, kNoKey, kNoKey, kNoKey};
+    if (a.dense) {
+        for (int tok = t0; tok < dm.V; tok += stride) {
+            if (!((a.bits[tok >> 5] >> (tok & 31)) & 1u)) continue;
+            float lp = x[tok];
+            if (a.logits) lp -= lse;
+            uint64_t key;
+            if (make_key(cum, lp, b, tok, dm.V, a.status, key)) top4_insert(t, key);
+        }
+    } else {
+        // batches of 8 entries per thread: the token and score loads overlap
+        const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
+        constexpr int U = 8;
+        for (int e0 = beg + t0; e0 < end; e0 += U * stride) {
+            int tk[U];
+            float lv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * stride;
+                tk[u] = e < end ? a.cols[e] : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * stride;
+                if (e < end && (tk[u] < 0 || tk[u] >= dm.V)) set_status(a.status, XGR_DEV_MASK);
+                lv[u] = (tk[u] >= 0 && tk[u] < dm.V) ? x[tk[u]] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (tk[u] < 0 || tk[u] >= dm.V) continue;
+                float lp = lv[u];
+                if (a.logits) lp -= lse;
+                uint64_t key;
+                if (make_key(cum, lp, b, tk[u], dm.V, a.status, key)) top4_insert(t, key);
+            }
+        }
+    }
+    top4_warp(t);
+    if (cta_per_row) {
+        if (lane == 0)
+            for (int i = 0; i < kSampleK; ++i) red_k[warp][i] = t[i];
+        __syncthreads();
+        if (warp == 0) {
+            for (int i = 0; i < kSampleK; ++i) t[i] = lane < kStatThreads / 32 ? red_k[lane][i] : kNoKey;
+            top4_warp(t);
+        }
+    }
+    if ((cta_per_row ? threadIdx.x : lane) == 0) {
+        for (int i = 0; i < kSampleK; ++i) a.sample[row * kSampleK + i] = t[i];
+        a.row_lse[row] = lse;
+    }
+}
+
+constexpr int kSelThreads = 1024;
+constexpr int kSurvCap = 4096;   // survivors kept in shared memory
+constexpr int kRankCap = 2048;   // sets up to this size are ordered by rank counting
 
 __device__ int find_child(const TrieView &tr, int level, int node, int t) {
     if (level >= tr.levels || node < 0 || node >= tr.n_nodes[level]) return -1;
@@ -323,145 +434,267 @@ __device__ int find_child(const TrieView &tr, int level, int node, int t) {
     return (lo < end && tr.tok[level][lo] == t) ? lo : -1;
 }
 
-struct ListCand {   // the surviving prefixes of every beam's sorted list, flattened
-    const uint64_t *lists;
-    const int *off;   // [n+1] exclusive offsets of survivors per beam
-    int n, K;
+// the candidates of one request as a flat index space: the dense first step
+// enumerates tokens of beam 0; later steps enumerate the CSR entries of the
+// live beams (rp = per-beam offsets relative to the request's first entry)
+struct ReqCand {
+    const float *x;          // scores of the request's first row
+    const uint32_t *bits;
+    const int32_t *cols;     // CSR entries of the request's first row
+    const int *rp;           // [n+1] in shared memory
+    const float *cum, *lse;  // [n] in shared memory
+    int32_t *status;
+    int n, dense, logits, V;
     __device__ bool operator()(int64_t e, uint64_t &key) const {
-        int lo = 0, hi = n;   // beam b with off[b] <= e < off[b+1]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (off[mid] <= e) lo = mid; else hi = mid;
+        int b, t;
+        if (dense) {
+            b = 0;
+            t = (int)e;
+            if (!((bits[t >> 5] >> (t & 31)) & 1u)) return false;
+        } else {
+            int lo = 0, hi = n;   // beam b with rp[b] <= e < rp[b+1]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (rp[mid] <= e) lo = mid; else hi = mid;
+            }
+            b = lo;
+            t = cols[e];
+            if (t < 0 || t >= V) return false;
         }
-        key = lists[(int64_t)lo * K + (e - off[lo])];
-        return true;
+        float lp = x[(int64_t)b * V + t];
+        if (logits) lp -= lse[b];
+        return make_key(cum[b], lp, b, t, V, status, key);
     }
 };
 
-// dst[e] = the e-th entry of the concatenated heads of the beams' lists, the
-// head of beam b being its first off[b+1]-off[b] entries.
-__device__ void gather_flat(uint64_t *dst, const uint64_t *lists, const int *off, int n, int K,
-                            int total) {
-    const ListCand lc{lists, off, n, K};
-    for (int e = threadIdx.x; e < total; e += blockDim.x) {
-        uint64_t key;
-        lc(e, key);
-        dst[e] = key;
-    }
+// ascending bitonic sort of (key, payload) pairs, n a power of two
+__device__ void block_sort_pairs(uint64_t *k, int *v, int n) {
+    for (int kk = 2; kk <= n; kk <<= 1)
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint64_t x = k[i], y = k[ixj];
+                    if ((x > y) == ((i & kk) == 0)) {
+                        k[i] = y;
+                        k[ixj] = x;
+                        const int t = v[i];
+                        v[i] = v[ixj];
+                        v[ixj] = t;
+                    }
+                }
+            }
+            __syncthreads();
+        }
 }
 
-__global__ void __launch_bounds__(kReqThreads) select_request_kernel(SelectArgs a) {
+size_t select_smem(const Dims &dm) {
+    return (size_t)kSurvCap * 12 + (size_t)kSampleK * dm.BW * 8 + (size_t)(dm.BW + 1) * 4 +
+           (size_t)dm.BW * 8 + (size_t)dm.BW * 12 + (size_t)dm.BW * dm.S * 8 + (size_t)dm.BW * 4 + 64;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const Dims dm = a.dims;
     const int BW = dm.BW, S = dm.S;
-    const int sample_cap = pow2_ceil(2 * BW);
-    uint64_t *sample = reinterpret_cast<uint64_t *>(smem_raw);
-    uint64_t *surv = sample + sample_cap;
-    int *off = reinterpret_cast<int *>(surv + kSurvCap);     // [BW+1]
-    int *cnt_s = off + (BW + 1);                              // [BW]
-    int *st_anc = cnt_s + BW;                                 // [BW*S]
-    int *st_seq = st_anc + BW * S;                            // [BW*S]
-    int *st_node = st_seq + BW * S;                           // [BW]
+    uint64_t *surv = reinterpret_cast<uint64_t *>(smem_raw);    // [kSurvCap]
+    uint64_t *samp = surv + kSurvCap;                           // [kSampleK*BW]
+    uint64_t *win_k = samp + kSampleK * BW;                     // [BW]
+    int *surv_e = reinterpret_cast<int *>(win_k + BW);          // [kSurvCap] entry of each survivor
+    int *win_e = surv_e + kSurvCap;                             // [BW]
+    int *rp = win_e + BW;                                       // [BW+1]
+    float *cum_s = reinterpret_cast<float *>(rp + BW + 1);      // [BW]
+    float *lse_s = cum_s + BW;                                  // [BW]
+    int *st_anc = reinterpret_cast<int *>(lse_s + BW);          // [BW*S]
+    int *st_seq = st_anc + BW * S;                              // [BW*S]
+    int *st_node = st_seq + BW * S;                             // [BW]
     __shared__ int hist[256];
     __shared__ int sc[4];
+    __shared__ int cnt;
+    __shared__ unsigned long long tau_s;
 
-    const int r = blockIdx.x;
-    const int tid = threadIdx.x;
-    const int n = a.st.n_live[r];
-    const uint64_t *L = a.lists + (int64_t)r * BW * dm.K;
-    const int32_t *cnt = a.counts + (int64_t)r * BW;
+    const int r = blockIdx.x, tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int64_t rb = (int64_t)r * BW;
+    int n = a.n_live[r];
+    if (a.dense) n = min(n, 1);   // the dense first step scores beam 0 only
 
-    for (int b = tid; b < BW; b += kReqThreads) cnt_s[b] = (b < n) ? cnt[b] : 0;
+    // ---- per-request tables in shared memory
+    for (int b = tid; b < n; b += kSelThreads) {
+        cum_s[b] = a.cum[rb + b];
+        lse_s[b] = a.logits ? a.row_lse[rb + b] : 0.f;
+    }
+    int64_t base = 0;
+    if (!a.dense) {
+        base = a.row_ptr[rb];
+        for (int b = tid; b <= n; b += kSelThreads) rp[b] = a.row_ptr[rb + b] - (int)base;
+    }
+    const int ns = n * kSampleK;
+    for (int i = tid; i < ns; i += kSelThreads) samp[i] = a.sample[rb * kSampleK + i];
+    if (tid == 0) {
+        cnt = 0;
+        tau_s = kNoKey;
+    }
     __syncthreads();
 
-    // exclusive scan helper over cnt-like values (serial on one warp; BW <= 1024)
-    auto scan_into_off = [&](auto value_of) {
-        if (tid < 32) {
-            int carry = 0;
-            for (int base = 0; base < BW; base += 32) {
-                const int b = base + tid;
-                int v = (b < BW) ? value_of(b) : 0;
-                int incl = v;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    int t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (tid >= o) incl += t;
+    // ---- threshold: the sample key of rank BW-1 (keys are unique; padding is kNoKey)
+    if (ns >= BW) {
+        if (ns <= kRankCap) {
+            for (int i = tid; i < ns; i += kSelThreads) {
+                const uint64_t k = samp[i];
+                if (k == kNoKey) continue;
+                int rank = 0;
+                for (int j = 0; j < ns; ++j) rank += samp[j] < k;
+                if (rank == BW - 1) tau_s = k;
+            }
+        } else {
+            int P = 1;
+            while (P < ns) P <<= 1;
+            // sort in the survivors buffer (P <= 4 * 1024 = kSurvCap)
+            for (int i = tid; i < P; i += kSelThreads) surv[i] = i < ns ? samp[i] : kNoKey;
+            __syncthreads();
+            block_sort(surv, P);
+            if (tid == 0) tau_s = surv[BW - 1];
+        }
+    }
+    __syncthreads();
+    const uint64_t tau = tau_s;
+    const int64_t E = a.dense ? (n > 0 ? dm.V : 0) : rp[n];
+    int total = 0;   // candidates of the request
+    if (a.dense) {
+        if (n > 0)
+            for (int w = tid; w < (dm.V + 31) / 32; w += kSelThreads) total += __popc(a.bits[w]);
+        atomicAdd(&cnt, total);
+        __syncthreads();
+        total = cnt;
+        __syncthreads();
+        if (tid == 0) cnt = 0;
+        __syncthreads();
+    } else {
+        total = (int)E;
+    }
+    const int want = min(BW, total);
+    const float *xr = a.scores + rb * dm.V;
+
+    // ---- survivors: the candidates ranked at or above tau, with their entry index
+    int T = kSurvCap + 1;
+    if (tau != kNoKey || total <= kSurvCap) {
+        if (a.dense) {
+            for (int t = tid; t < (n > 0 ? dm.V : 0); t += kSelThreads) {
+                if (!((a.bits[t >> 5] >> (t & 31)) & 1u)) continue;
+                float lp = xr[t];
+                if (a.logits) lp -= lse_s[0];
+                uint64_t key;
+                if (make_key(cum_s[0], lp, 0, t, dm.V, a.status, key) && key <= tau) {
+                    const int pos = atomicAdd(&cnt, 1);
+                    if (pos < kSurvCap) {
+                        surv[pos] = key;
+                        surv_e[pos] = t;
+                    }
                 }
-                if (b < BW) off[b] = carry + incl - v;
-                carry += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (tid == 0) off[BW] = carry;
+        } else {
+            // one warp per beam; 4 entries per lane in flight
+            const int32_t *cr = a.cols + base;
+            for (int b = warp; b < n; b += kSelThreads / 32) {
+                const int e_beg = rp[b], e_end = rp[b + 1];
+                const float cb = cum_s[b], lb = lse_s[b];
+                const float *xb = xr + (int64_t)b * dm.V;
+                for (int e0 = e_beg + lane; e0 < e_end; e0 += 4 * 32) {
+                    int tk[4];
+                    float xv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = e0 + 32 * u;
+                        tk[u] = e < e_end ? cr[e] : -1;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) xv[u] = (tk[u] >= 0 && tk[u] < dm.V) ? xb[tk[u]] : 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (tk[u] < 0 || tk[u] >= dm.V) continue;
+                        float lp = xv[u];
+                        if (a.logits) lp -= lb;
+                        uint64_t key;
+                        if (make_key(cb, lp, b, tk[u], dm.V, a.status, key) && key <= tau) {
+                            const int pos = atomicAdd(&cnt, 1);
+                            if (pos < kSurvCap) {
+                                surv[pos] = key;
+                                surv_e[pos] = e0 + 32 * u;
+                            }
+                        }
+                    }
+                }
+            }
         }
         __syncthreads();
-    };
-
-    // ---- total candidates, and a sample of the head of every beam's list
-    scan_into_off([&](int b) { return cnt_s[b]; });
-    const int total = off[BW];
-    const int n_out = min(BW, total);
-    __syncthreads();
-    const int cs = n > 0 ? (BW + n - 1) / n : 0;
-    scan_into_off([&](int b) { return min(cs, cnt_s[b]); });
-    const int S0 = off[BW];
-    gather_flat(sample, L, off, n, dm.K, S0);
-    __syncthreads();
-    uint64_t tau = kNoKey;
-    if (S0 >= BW) {   // the BW-th best of the sample bounds the BW-th best overall
-        const int P = pow2_ceil(S0);
-        for (int i = S0 + tid; i < P; i += kReqThreads) sample[i] = kNoKey;
+        T = cnt;
         __syncthreads();
-        block_sort(sample, P);
-        tau = sample[BW - 1];
     }
-    __syncthreads();
-
-    // ---- survivors: the prefix of each beam's sorted list at or above the threshold
-    for (int b = tid; b < BW; b += kReqThreads) {
-        int lo = 0, hi = cnt_s[b];
-        const uint64_t *lb = L + (int64_t)b * dm.K;
-        while (lo < hi) {   // upper bound of tau
-            const int mid = (lo + hi) >> 1;
-            if (lb[mid] <= tau) lo = mid + 1; else hi = mid;
-        }
-        st_node[b] = lo;    // temporarily: survivors of beam b
-    }
-    __syncthreads();
-    scan_into_off([&](int b) { return st_node[b]; });
-    const int T = off[BW];
-
-    int n_sel;
-    if (T <= kSurvCap) {
-        gather_flat(surv, L, off, n, dm.K, T);
-        n_sel = T;
-    } else {   // rare: too many survivors -> exact radix select of the best BW
-        ListCand lc{L, off, n, dm.K};
-        uint64_t prefix, mask;
-        radix_select(lc, T, n_out, hist, sc, prefix, mask);
-        if (tid == 0) sc[3] = 0;
+    if (T > kSurvCap) {   // exact radix select of the best `want` over all candidates
+        ReqCand cand;
+        cand.x = xr;
+        cand.bits = a.bits;
+        cand.cols = a.dense ? nullptr : a.cols + base;
+        cand.rp = rp;
+        cand.cum = cum_s;
+        cand.lse = lse_s;
+        cand.status = a.status;
+        cand.n = n;
+        cand.dense = a.dense;
+        cand.logits = a.logits;
+        cand.V = dm.V;
+        uint64_t prefix = ~0ull, mask = 0;
+        if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
+        if (tid == 0) cnt = 0;
         __syncthreads();
-        for (int64_t e = tid; e < T; e += kReqThreads) {
+        for (int64_t e = tid; e < E; e += kSelThreads) {
             uint64_t key;
-            lc(e, key);
-            if ((key & mask) <= prefix) {
-                const int pos = atomicAdd(&sc[3], 1);
-                if (pos < kSurvCap) surv[pos] = key;
+            if (cand(e, key) && (key & mask) <= prefix) {
+                const int pos = atomicAdd(&cnt, 1);
+                if (pos < kSurvCap) {
+                    surv[pos] = key;
+                    surv_e[pos] = (int)e;
+                }
             }
         }
-        n_sel = n_out;
+        __syncthreads();
+        T = min(cnt, kSurvCap);
+        __syncthreads();
+    }
+    const int n_win = min(want, T);   // fewer only if some counted candidates were invalid
+
+    // ---- the winners in rank order
+    if (T <= kRankCap) {
+        for (int i = tid; i < T; i += kSelThreads) {
+            const uint64_t k = surv[i];
+            int rank = 0;
+            for (int j = 0; j < T; ++j) rank += surv[j] < k;
+            if (rank < n_win) {
+                win_k[rank] = k;
+                win_e[rank] = surv_e[i];
+            }
+        }
+    } else {
+        int PT = 1;
+        while (PT < T) PT <<= 1;
+        for (int i = T + tid; i < PT; i += kSelThreads) {
+            surv[i] = kNoKey;
+            surv_e[i] = -1;
+        }
+        __syncthreads();
+        block_sort_pairs(surv, surv_e, PT);
+        for (int i = tid; i < n_win; i += kSelThreads) {
+            win_k[i] = surv[i];
+            win_e[i] = surv_e[i];
+        }
     }
     __syncthreads();
-    {
-        const int P = pow2_ceil(max(n_sel, 1));
-        for (int i = n_sel + tid; i < P; i += kReqThreads) surv[i] = kNoKey;
-        __syncthreads();
-        block_sort(surv, P);
-    }
 
     // ---- outputs in rank order
-    for (int i = tid; i < BW; i += kReqThreads) {
-        const int64_t o = (int64_t)r * BW + i;
-        if (i < n_out) {
-            const uint64_t key = surv[i];
+    for (int i = tid; i < BW; i += kSelThreads) {
+        const int64_t o = rb + i;
+        if (i < n_win) {
+            const uint64_t key = win_k[i];
             const uint32_t lo = (uint32_t)key;
             a.parent[o] = (int32_t)(lo / (uint32_t)dm.V);
             a.token[o] = (int32_t)(lo % (uint32_t)dm.V);
@@ -472,21 +705,21 @@ __global__ void __launch_bounds__(kReqThreads) select_request_kernel(SelectArgs 
             a.cum_out[o] = -INFINITY;
         }
     }
-    if (tid == 0) a.n_out[r] = n_out;
+    if (tid == 0) a.n_out[r] = n_win;
+    if (!a.rewire) return;
 
     // ---- in-place rewiring: stage every old row first, then write
-    const int64_t rb = (int64_t)r * BW;
-    for (int i = tid; i < n * S; i += kReqThreads) {
+    for (int i = tid; i < n * S; i += kSelThreads) {
         st_anc[i] = a.st.anc[rb * S + i];
         st_seq[i] = a.st.seq[rb * S + i];
     }
-    for (int b = tid; b < n; b += kReqThreads) st_node[b] = a.st.node[rb + b];
+    for (int b = tid; b < n; b += kSelThreads) st_node[b] = a.st.node[rb + b];
     __syncthreads();
     const int s = a.step;
-    for (int nb = tid; nb < BW; nb += kReqThreads) {
+    for (int nb = tid; nb < BW; nb += kSelThreads) {
         const int64_t o = rb + nb;
-        if (nb < n_out) {
-            const uint64_t key = surv[nb];
+        if (nb < n_win) {
+            const uint64_t key = win_k[nb];
             const uint32_t lo = (uint32_t)key;
             const int p = (int)(lo / (uint32_t)dm.V), t = (int)(lo % (uint32_t)dm.V);
             for (int i = 0; i < S; ++i) {
@@ -503,8 +736,17 @@ __global__ void __launch_bounds__(kReqThreads) select_request_kernel(SelectArgs 
                 a.st.anc[o * S + i] = av;
                 a.st.seq[o * S + i] = sv;
             }
-            const int child = find_child(a.trie, s, st_node[p], t);
-            if (child < 0) set_status(a.st.status, XGR_DEV_MASK);
+            // trie child: the mask row of parent p lists its children in trie
+            // order, so the entry index locates the child directly
+            int child = -1;
+            const int node = st_node[p];
+            if (a.dense) {
+                child = find_child(a.trie, s, node, t);
+            } else if (s < a.trie.levels && node >= 0 && node < a.trie.n_nodes[s]) {
+                const int c = a.trie.ptr[s][node] + (win_e[nb] - rp[p]);
+                if (c < a.trie.ptr[s][node + 1] && a.trie.tok[s][c] == t) child = c;
+            }
+            if (child < 0) set_status(a.status, XGR_DEV_MASK);
             a.st.node[o] = child;
             a.st.cum[o] = desc_bits_to_score((uint32_t)(key >> 32));
         } else {
@@ -517,7 +759,7 @@ __global__ void __launch_bounds__(kReqThreads) select_request_kernel(SelectArgs 
         }
     }
     __syncthreads();
-    if (tid == 0) a.st.n_live[r] = n_out;
+    if (tid == 0) a.st.n_live[r] = n_win;
 }
 
 __global__ void get_sequences_kernel(BeamState st, Dims dm, int32_t *seq) {
@@ -527,13 +769,6 @@ __global__ void get_sequences_kernel(BeamState st, Dims dm, int32_t *seq) {
 
 }  // namespace
 
-size_t select_request_smem(const Dims &dm) {
-    int sample_cap = 1;
-    while (sample_cap < 2 * dm.BW) sample_cap <<= 1;
-    return (size_t)(sample_cap + kSurvCap) * 8 + (size_t)(dm.BW + 1 + dm.BW) * 4 +
-           (size_t)dm.BW * dm.S * 8 + (size_t)dm.BW * 4;
-}
-
 cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, cudaStream_t s) {
     const int64_t n = (int64_t)Bcap * dm.BW;
     begin_kernel<<<(int)((n + 255) / 256), 256, 0, s>>>(st, dm, Bcap, all_live);
@@ -541,27 +776,37 @@ cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, cudaStre
 }
 
 cudaError_t launch_build_mask(const MaskArgs &a, cudaStream_t s) {
-    mask_scan_kernel<<<1, kScanThreads, 0, s>>>(a);
     const int64_t rows = (int64_t)a.dims.B * a.dims.BW;
-    mask_fill_kernel<<<(int)((rows * 32 + 255) / 256), 256, 0, s>>>(a);
+    mask_scan_kernel<<<1, kMaskThreads, 0, s>>>(a);
+    mask_copy_kernel<<<(int)((rows * 32 + 255) / 256), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
+size_t select_sample_offset(int64_t rows) { return ((size_t)rows * 4 + 255) & ~(size_t)255; }
+size_t select_scratch_bytes(int64_t rows) {
+    return select_sample_offset(rows) + (size_t)rows * 8 * kSampleK;
+}
+
 cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s) {
-    if (a.dims.K > kMaxK) return cudaErrorInvalidValue;
-    const int rows_per_req = (a.step == 0) ? 1 : a.dims.BW;
-    select_row_kernel<<<a.dims.B * rows_per_req, kRowThreads, 0, s>>>(a, rows_per_req);
+    if (a.dims.BW > 1024) return cudaErrorInvalidValue;
+    if (a.dense) {
+        row_stats_kernel<<<a.dims.B, kStatThreads, 0, s>>>(a, 1);
+    } else {
+        const int64_t rows = (int64_t)a.dims.B * a.dims.BW;
+        const int per_cta = kStatThreads / 32;
+        row_stats_kernel<<<(int)((rows + per_cta - 1) / per_cta), kStatThreads, 0, s>>>(a, 0);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t smem = select_request_smem(a.dims);
+    const size_t smem = select_smem(a.dims);
     static size_t attr = 0;   // largest size set so far (set outside graph capture in practice)
     if (smem > attr) {
-        e = cudaFuncSetAttribute(select_request_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
         attr = smem;
     }
-    select_request_kernel<<<a.dims.B, kReqThreads, smem, s>>>(a);
+    select_kernel<<<a.dims.B, kSelThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -82,26 +82,34 @@ struct MaskArgs {
 };
 cudaError_t launch_build_mask(const MaskArgs &a, cudaStream_t s);
 
-// Beam selection + in-place rewiring.
+// Beam selection (+ in-place rewiring of the context's beam state).
 struct SelectArgs {
+    const float *cum;           // [B][BW] cumulative scores before this step
+    const int32_t *n_live;      // [B] live beams before this step
+    int32_t *status;            // device status word
+    int rewire;                 // 1: rewrite st (anc, seq, node, cum, n_live) in place
     BeamState st;
     TrieView trie;
     Dims dims;
     int step;
     int logits;                 // XGR_SCORES_LOGITS
     const float *scores;        // [B][BW][V]
-    int dense;                  // mask kind
+    int dense;                  // mask kind (dense: only beam 0 of each request is read)
     const uint32_t *bits;
     const int32_t *row_ptr;
     const int32_t *cols;
-    float *row_lse;             // [Bcap][BW] scratch
-    uint64_t *lists;            // [Bcap][BW][K] per-beam sorted candidates
-    int32_t *counts;            // [Bcap][BW]
+    float *row_lse;             // [B][BW] scratch
+    uint64_t *sample;           // [B][BW][kSampleK] scratch: each beam's best keys
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
     float *cum_out;
     int32_t *n_out;             // [B]
 };
+constexpr int kSampleK = 4;     // best keys per beam kept for the threshold sample
+// scratch of the selection for `rows` beam rows: row_lse [rows] f32 at offset 0,
+// sample [rows][kSampleK] u64 at select_sample_offset(rows)
+size_t select_scratch_bytes(int64_t rows);
+size_t select_sample_offset(int64_t rows);
 cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
 
 cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);

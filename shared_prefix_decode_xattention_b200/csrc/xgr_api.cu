@@ -46,7 +46,7 @@ struct Layout {
     int64_t trie_level_cap;    // ints per level in each of trie_ptr / trie_tok
     size_t mask_row_ptr, mask_cols;
     int64_t mask_cap;
-    size_t row_lse, lists, counts;
+    size_t select_scratch;
     size_t part_o, part_ml;
     int slots;
     size_t plan_items[2], plan_members[2], plan_nslots[2];
@@ -81,13 +81,11 @@ void make_layout(const xgr_config &c, Layout &L) {
         L.mask_cap = B * BW * (int64_t)fanout_cap(c);
         L.mask_row_ptr = take(4 * (B * BW + 1));
         L.mask_cols = take(4 * L.mask_cap);
-        L.row_lse = take(4 * B * BW);
-        L.lists = take(8 * B * BW * (int64_t)c.top_k);
-        L.counts = take(4 * B * BW);
+        L.select_scratch = take(select_scratch_bytes(B * BW));
     } else {
         L.trie_level_cap = 0;
         L.trie_ptr = L.trie_tok = L.root_bits = L.mask_row_ptr = L.mask_cols = 0;
-        L.row_lse = L.lists = L.counts = 0;
+        L.select_scratch = 0;
         L.mask_cap = 0;
     }
     L.slots = partial_slots(c);
@@ -658,6 +656,10 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
                   : (mask->kind != XGR_MASK_CSR || !mask->row_ptr || !mask->cols))
         return XGR_ERR_ARG;
     SelectArgs a;
+    a.cum = c->st.cum;
+    a.n_live = c->st.n_live;
+    a.status = c->st.status;
+    a.rewire = 1;
     a.st = c->st;
     a.trie = c->trie;
     a.dims = c->dims;
@@ -668,9 +670,10 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.bits = mask->bits;
     a.row_ptr = mask->row_ptr;
     a.cols = mask->cols;
-    a.row_lse = c->at<float>(c->L.row_lse);
-    a.lists = c->at<uint64_t>(c->L.lists);
-    a.counts = c->at<int32_t>(c->L.counts);
+    a.row_lse = c->at<float>(c->L.select_scratch);
+    a.sample = reinterpret_cast<uint64_t *>(
+        c->at<uint8_t>(c->L.select_scratch) +
+        select_sample_offset((int64_t)c->cfg.max_requests * c->cfg.beam_width));
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum;
