@@ -197,6 +197,51 @@ def algorithmic(w, s, logits_mode, nnz_step):
     return att_bytes, att_flops, sel_bytes
 
 
+def decode_required_bytes(w, logits_mode, nnz):
+    """Bytes one decode must move at least: per step, every prompt and suffix
+    K/V once, each live beam's earlier Unshared k/v, this step's k/v (read and
+    appended), q and O and LSE, the score rows the selection needs (full rows
+    of the live beams with logits, the masked entries with log-probs), the
+    mask (bitset, or CSR row pointers + entries + the trie tokens copied) and
+    the selection's outputs."""
+    B, BW, Hq, Hkv, D, V = w.B, w.BW, w.Hq, w.Hkv, w.D, w.V
+    import workloads
+    kv_tokens = int(workloads.prompt_lengths(w).sum()) + int(workloads.suffix_lengths(w).sum())
+    shared = 2 * Hkv * D * 2 * kv_tokens          # every prompt / suffix K and V once per step
+    total = 0
+    for s in range(w.S):
+        live = B * (1 if (s == 0 and V) else BW)
+        b = shared
+        b += 2 * live * Hkv * s * D * 2            # earlier Unshared k/v
+        b += 2 * live * Hkv * D * 2 * 2            # this step's k/v: read + append
+        b += 2 * live * Hq * D * 2 + live * Hq * 4  # q, O, LSE
+        if V:
+            if s == 0:
+                b += B * V * 4 + (V + 7) // 8      # beam 0's score row, bitset
+            else:
+                b += (live * V * 4 if logits_mode else nnz[s] * 4)
+                b += (B * BW + 1) * 4 + nnz[s] * 4 * 2   # row_ptr, cols written, trie tokens read
+            b += B * BW * 16                       # parent, token, cum, n_out
+        total += b
+    return total
+
+
+def graph_kernel_nodes(g) -> int:
+    """Kernel nodes of a captured CUDA graph: the library kernels one decode launches."""
+    from cuda.bindings import runtime as rt
+    graph = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    count = 0
+    for nd in nodes[:n]:
+        err, kind = rt.cudaGraphNodeGetType(nd)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        count += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    return count
+
+
 def run_gpu(args, w):
     import numpy as np
     import torch
@@ -247,16 +292,24 @@ def run_gpu(args, w):
     # [mask + selection s].  Each phase is enqueued on the current stream (the
     # capture stream while a CUDA graph is recorded); with `host`, the step's
     # inputs come from pinned host memory and its outputs go back to it.
+    # The valid-path mask of step s depends only on the beam state the previous
+    # selection left, so it is built on a side stream while the attention runs.
+    side = torch.cuda.Stream(device=dev)
+    masks = [None] * w.S
+
     def enqueue_att(s, inp, host):
         q, kn, vn, sc = inp[s]
+        side.wait_stream(cur())
+        with torch.cuda.stream(side):
+            masks[s] = sess.build_mask(s, side)
         if host is not None:
             for d, h in zip(inp[s], host[s]):
                 d.copy_(h, non_blocking=True)
         sess.decode_step(s, q, kn, vn, out, lse, cur())
+        cur().wait_stream(side)
 
     def enqueue_sel(s, inp, host):
-        m = sess.build_mask(s, cur())
-        sess.beam_select(s, inp[s][3], flags, m, par, tok, cum, nout, cur())
+        sess.beam_select(s, inp[s][3], flags, masks[s], par, tok, cum, nout, cur())
         if host is not None:
             for h, d in zip(host[w.S + s], (par, tok, cum, nout)):
                 h.copy_(d, non_blocking=True)
@@ -272,19 +325,32 @@ def run_gpu(args, w):
             enqueue_att(s, inp, host)
             enqueue_sel(s, inp, host)
 
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
+    def capture(fn, keep=False):
+        g = torch.cuda.CUDAGraph(keep_graph=keep)
         with torch.cuda.graph(g):
             fn()
+        if keep:
+            g.instantiate()
         return g
 
     for _ in range(max(args.warmup, 3)):   # eager warm-up (plans, attributes)
         enqueue_decode()
     torch.cuda.synchronize()
+    # CSR entries of every step (one eager decode, read back after each mask)
+    nnz = []
+    sess.begin(w.B, cur())
+    for s in range(w.S):
+        enqueue_att(s, inputs, None)
+        m = masks[s]
+        torch.cuda.synchronize()
+        nnz.append(sess.mask_entries(m) if m.kind == xgr.XGR_MASK_CSR else 0)
+        enqueue_sel(s, inputs, None)
+    torch.cuda.synchronize()
     if sess.device_status() != 0:
         raise RuntimeError("device status set during warm-up")
     # the graph-based execution of the pages' system level: a whole decode is one graph
-    g_decode = capture(lambda: enqueue_decode())
+    g_decode = capture(lambda: enqueue_decode(), keep=True)
+    launches_per_decode = graph_kernel_nodes(g_decode)
     g_phase = [capture(lambda: enqueue_head(inputs, None))]
     for s in range(1, w.S):
         g_phase.append(capture(lambda s=s: enqueue_att(s, inputs, None)))
@@ -377,9 +443,10 @@ def run_gpu(args, w):
     hbm = peaks.get("hbm_gbs", 6650.0)
     tf = peaks.get("bf16_tflops", 1590.0)
     src = "of measured" if peaks else "of fallback"
-    # nnz of the sparse masks: expected children per beam (measured once on host)
-    nnz_step = int(round(w.B * w.BW * min(w.V, w.n_items / w.V))) if w.V else 0
+    nnz_step = nnz[1] if w.S > 1 else 0   # CSR entries of step 1 (measured above)
     att_bytes, att_flops, sel_bytes = algorithmic(w, 1, logits_mode, nnz_step)
+    required = decode_required_bytes(w, logits_mode, nnz)
+    dec_gbs = required / (total_ms / args.steps / 1e3) / 1e9
     att_avg = statistics.mean(att_ms) / 1e3
     sel_avg = statistics.mean(sel_ms) / 1e3
     if att_avg >= sel_avg:
@@ -396,7 +463,6 @@ def run_gpu(args, w):
                 "peak_source": f"hbm_gbs {src}", "traffic": None,
                 "algorithmic_per_launch": sel_bytes, "launch_ms": sel_avg * 1e3}
 
-    launches_per_decode = 1 + sum((2) + (0 if s == 0 else 2) + 2 for s in range(w.S))
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -404,8 +470,12 @@ def run_gpu(args, w):
             "config": dict(workload_config(w, args.scores), global_batch=w.B * world,
                            parallelism=f"dp{world}" if world > 1 else "single"),
             "roofline": roof,
-            "step_breakdown_ms": {"attention_step_ge1": att_avg * 1e3,
+            "step_breakdown_ms": {"attention_with_mask_step_ge1": att_avg * 1e3,
                                   "select_step_ge1": sel_avg * 1e3},
+            "decode_hbm": {"required_bytes_per_decode": required, "achieved_gbs": dec_gbs,
+                           "peak_gbs": hbm, "frac": dec_gbs / hbm,
+                           "note": "whole decode (all steps, every kernel) against the copy "
+                                   f"bandwidth {src}"},
             "gpu_launches": launches_per_decode * args.steps,
             "device_status": status, "n_live_last": int(n_live.min()) if n_live.size else 0}
     if e2e:

@@ -186,7 +186,8 @@ xgr_status xgr_decode_step(xgr_ctx *ctx, int32_t step, const void *d_q, const vo
 xgr_status xgr_build_mask(xgr_ctx *ctx, int32_t step, xgr_mask *out, xgr_stream_t stream);
 
 /* Masked top-K beam selection with in-place rewiring (xGR 2.2 "Early sort
- * termination", 2.1 "In-place updates"):
+ * termination", 2.1 "In-place updates").  Vocabularies up to 32768 tokens
+ * (xgr_create returns XGR_ERR_UNIMPLEMENTED above):
  *   d_scores fp32 [B][BW][V]  log-probs or logits (flags); rows of dead beams
  *                             are not read
  *   mask                      as returned by xgr_build_mask for this step
@@ -223,9 +224,14 @@ xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_co
  * it writes d_parent, d_token, d_cum_out [B][BW] and d_n_out [B] exactly as
  * xgr_beam_select does (same order, same tie-break, same bits).
  * Allocation: none.  Its scratch is one static device array of 8 MiB per GPU
- * (held by every GPU that loads the library until the process exits); a call
- * needs about 36 bytes per beam row (B*BW rows, up to about 233 000 rows) and
- * returns XGR_ERR_CAPACITY beyond that.
+ * (held by every GPU that loads the library until the process exits).  After
+ * about 12 bytes per beam row, the rest is shared by the requests as a key
+ * buffer (8 bytes per CSR entry) plus a survivor buffer (12 bytes per entry,
+ * half as many); a call returns XGR_ERR_CAPACITY unless every request gets
+ * room for max(V, 8*BW, 4096) entries (e.g. 8 requests x 128 beams over
+ * V = 8192 get about 74000).  A request with more CSR entries than its share
+ * is still selected exactly, on a slower path.  V above 32768 returns
+ * XGR_ERR_UNIMPLEMENTED (a score row is staged whole in shared memory).
  * The first call on a device looks the array up (cudaGetSymbolAddress) and
  * may set a kernel attribute, so make that first call before any stream capture.
  * All calls share the array: calls that overlap on the GPU race and must be

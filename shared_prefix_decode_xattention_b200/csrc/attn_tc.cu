@@ -11,22 +11,30 @@
 // the tensor cores here.
 //
 // One CTA per work item (kv head, 128-row tile, key range):
-//   warp 0      TMA producer: K and V chunks of 128 keys (two 64-column
-//               128-byte-swizzled boxes each), double-buffered, K and V on
-//               separate barriers so the next K streams in while P V runs;
+//   warp 0      TMA producer: Q, then K and V chunks of 128 keys (two 64-column
+//               128-byte-swizzled boxes each) on separate two-stage rings;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_j = Q K_j^T into one of two TMEM buffers, then
-//               O += P_{j-1} V_{j-1} into the TMEM O accumulator;
-//   warps 2-5   one query row per thread: read S_j from TMEM, running max
-//               (lazy rescaling: O is rescaled only when the max grows by more
-//               than 2^8), exponentials, row sums, P_j (bf16) into shared
-//               memory in the canonical 128-byte-swizzled K-major layout;
-//               finally read O from TMEM and write the partial (O, m, l).
+//               S_j = Q K_j^T into TMEM buffer j % 2, O_{j%2} += P_j V_j;
+//   warps 2-9   two softmax warpgroups; warpgroup h owns the chunks j with
+//               j % 2 == h, one query row per thread: it reads S_j from TMEM,
+//               keeps the running max and sum of its own accumulator O_h (lazy
+//               rescaling: O_h is rescaled only when the max grows by more than
+//               2^8), and writes P_j (bf16) into its own shared-memory buffer in
+//               the canonical 128-byte-swizzled K-major layout.  The two
+//               warpgroups never wait for each other inside the loop, so one's
+//               exponentials overlap the other's row maxima and TMEM traffic;
+//               at the end they swap (m, l) and merge O_0 and O_1 into the
+//               partial (O, m, l) or, for a request's only segment, the output.
+// In a request's only KV segment ("final" items) the Unshared and Merging
+// stages run here too: before the loop the softmax threads gather the beam's
+// own tokens (direct indices into the token-granular pool), seed O_0 and its
+// (m, l) with them, and append this step's k / v to the pool.
 // Every wait on an mbarrier is bounded; on time-out the CTA records
 // XGR_DEV_TIMEOUT in the status word and unwinds (no trap, no hang).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,61 +44,32 @@ namespace {
 
 constexpr int kTcThreads = 320;              // producer warp, MMA warp, 2 softmax warpgroups
 constexpr int kSoftmaxThreads = 256;
+constexpr int kGroupThreads = 128;           // one softmax warpgroup: one query row per thread
 constexpr int kBlockN = 128;                 // keys per chunk
-constexpr int kKStages = 3;                  // K chunks in flight
+constexpr int kKStages = 2;                  // K chunks in flight
 constexpr int kVStages = 2;                  // V chunks in flight
 constexpr uint32_t kHalf = 16384;            // one 128-row x 64-column bf16 sub-tile
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
-constexpr uint32_t kOffP = kOffV + kVStages * kTile;
-constexpr uint32_t kOffBar = kOffP + kTile;
+constexpr uint32_t kOffP = kOffV + kVStages * kTile;   // P of warpgroup 0, then of warpgroup 1
+constexpr uint32_t kOffBar = kOffP + 2 * kTile;
 constexpr uint32_t kOffMisc = kOffBar + 256;  // TMEM address, abort flag
-constexpr uint32_t kOffRed = kOffMisc + 16;   // row-max exchange [2 parity][2 halves][128 rows]
-constexpr uint32_t kSmemUsed = kOffRed + 2048;
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = 232448;       // the sm_100 per-block maximum
 constexpr uint32_t kSmemSpare = kSmemBytes - kSmemUsed;   // room to realign the window
-constexpr uint32_t kTmemCols = 512;          // S0 [0,128) S1 [128,256) O [256,384)
-constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kTmemCols = 512;          // S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512)
 
-// barrier slots (8 bytes each) after kOffBar
-enum { B_KFULL = 0, B_KEMPTY = 3, B_VFULL = 6, B_VEMPTY = 8, B_SFULL = 10, B_PFULL = 12,
-       B_PVDONE = 13, B_QFULL = 14, B_DRAIN = 15, B_XCH = 16, B_COUNT = 18 };   // B_XCH: 2 halves
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Bounded wait for the completion of the phase with the given parity.  Gives
-// up early when another role has aborted (abort != nullptr and set); on its
-// own time-out it sets the abort flag.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.b32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if (abort && (it & 255) == 255 && *abort) return false;
-    }
-    if (abort) *abort = 1;
-    return false;
-}
+// barrier slots (8 bytes each) after kOffBar; SFULL, PFULL, PVDONE and XCH have one
+// slot per warpgroup
+enum { B_KFULL = 0, B_KEMPTY = 2, B_VFULL = 4, B_VEMPTY = 6, B_SFULL = 8, B_PFULL = 10,
+       B_PVDONE = 12, B_QFULL = 14, B_DONE = 15, B_XCH = 16, B_PRO = 18, B_SFREE = 19,
+       B_COUNT = 21 };
+// B_SFREE: a warpgroup has read all of S_j (its TMEM buffer may take S_{j+2});
+// B_DONE: every MMA has completed; B_XCH: the warpgroups' (m, l) exchange;
+// B_PRO: the Unshared prologue's loads have returned
+static_assert(B_COUNT * 8 <= 256, "barrier area");
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {
@@ -98,6 +77,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
 
@@ -216,7 +204,7 @@ __device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it,
         const int member = i / (a.nb * G);
         ri.b = (i / G) % a.nb;
         ri.hg = i % G;
-        ri.r = a.members[it.member_off + member];
+        ri.r = it.n_members == 1 ? it.r0 : a.members[it.member_off + member];
         ri.gid = ((int64_t)ri.r * a.dims.BW + ri.b) * a.dims.Hq + it.g * G + ri.hg;
         ri.valid = true;
     }
@@ -227,7 +215,7 @@ __device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it,
 // the 10 warps share one, so a thread may use at most 168 registers
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                   TcArgs a) {
+                   const __grid_constant__ CUtensorMap tmq, TcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
     if (pad > kSmemSpare) {   // the dynamic window is expected 1024-aligned; never trap
@@ -240,13 +228,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + kOffMisc);
     int *abort_flag = reinterpret_cast<int *>(base + kOffMisc + 4);
-    float *red = reinterpret_cast<float *>(base + kOffRed);   // [2 parity][2 halves][128 rows]
 
     const WorkItem it = a.items[blockIdx.x];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int n_keys = it.key_end - it.key_begin;
     const int nchunks = (n_keys + kBlockN - 1) / kBlockN;
     const bool final_item = (it.flags & 1) != 0;
+    const bool q_tma = (it.flags & 2) != 0;   // the Q tile is one TMA box
     volatile int *abort = abort_flag;
     const int y0 = it.g * (int)a.kv_tokens + it.kv_off + it.key_begin;
     // producer lanes: lane 0 streams K chunks, lane 1 V chunks, each on its own ring
@@ -273,21 +261,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_init(bar(B_VFULL + s), 1);
                 mbar_init(bar(B_VEMPTY + s), 1);
             }
-            for (int s = 0; s < 2; ++s) mbar_init(bar(B_SFULL + s), 1);
-            mbar_init(bar(B_PFULL), kSoftmaxThreads);
-            mbar_init(bar(B_PVDONE), 1);
-            mbar_init(bar(B_QFULL), kSoftmaxThreads);
-            mbar_init(bar(B_DRAIN), 1);
-            mbar_init(bar(B_XCH), kSoftmaxThreads / 2);
-            mbar_init(bar(B_XCH + 1), kSoftmaxThreads / 2);
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(bar(B_SFULL + h), 1);
+                mbar_init(bar(B_PFULL + h), kGroupThreads);
+                mbar_init(bar(B_PVDONE + h), 1);
+                mbar_init(bar(B_XCH + h), kGroupThreads);
+                mbar_init(bar(B_SFREE + h), kGroupThreads);
+            }
+            mbar_init(bar(B_QFULL), q_tma ? 1 : kSoftmaxThreads);
+            mbar_init(bar(B_DONE), 1);
+            mbar_init(bar(B_PRO), kSoftmaxThreads);
             *abort_flag = 0;
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            fence_mbar_init();
         }
         __syncwarp();
-        // the first chunks start streaming before the block-wide setup barrier
+        // Q and the first chunks start streaming before the block-wide setup barrier
+        if (lane == 0 && q_tma) {
+            const int G = a.dims.G;
+            const int z = it.r0 * a.dims.BW + it.row_begin / G;
+            mbar_expect_tx(bar(B_QFULL), kTile);
+            tma_load_3d(sb + kOffQ, &tmq, 0, it.g * G, z, bar(B_QFULL));
+            tma_load_3d(sb + kOffQ + kHalf, &tmq, 64, it.g * G, z, bar(B_QFULL));
+        }
+        // In final items only Q and the first K chunk go out now: the rest of the
+        // K/V fill waits until the Unshared prologue's scattered loads have
+        // returned, so that those do not queue behind megabytes of streaming.
         if (lane == 0)
-            for (int j = 0; j < min(nchunks, kKStages); ++j) issue_k(j);
-        if (lane == 1)
+            for (int j = 0; j < min(nchunks, final_item ? 1 : kKStages); ++j) issue_k(j);
+        if (lane == 1 && !final_item)
             for (int j = 0; j < min(nchunks, kVStages); ++j) issue_v(j);
     }
     if (warp == 1) {
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // softmax threads stage the Q tile meanwhile: 16 consecutive threads read one
     // 256-byte row (coalesced) and write it in the swizzled K-major layout
-    if (warp >= 2) {
+    if (warp >= 2 && !q_tma) {
         const int ts = tid - 64;
         uint4 qv[8];
 #pragma unroll
@@ -323,8 +324,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producers
         if (lane == 0) {
-            int n_issued = min(nchunks, kKStages);
-            for (int j = kKStages; j < nchunks; ++j) {
+            int n_issued = min(nchunks, final_item ? 1 : kKStages);
+            if (final_item && n_issued < min(nchunks, kKStages) && mbar_wait(bar(B_PRO), 0, abort))
+                for (; n_issued < min(nchunks, kKStages); ++n_issued) issue_k(n_issued);
+            for (int j = kKStages; j < nchunks && n_issued == j; ++j) {
                 if (!mbar_wait(bar(B_KEMPTY + j % kKStages), ((j / kKStages) - 1) & 1, abort)) break;
                 issue_k(j);
                 ++n_issued;
@@ -333,8 +336,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = max(0, n_issued - kKStages); j < n_issued; ++j)
                     mbar_wait(bar(B_KFULL + j % kKStages), (j / kKStages) & 1, nullptr);
         } else if (lane == 1) {
-            int n_issued = min(nchunks, kVStages);
-            for (int j = kVStages; j < nchunks; ++j) {
+            int n_issued = final_item ? 0 : min(nchunks, kVStages);
+            if (final_item && nchunks > 0 && mbar_wait(bar(B_PRO), 0, abort))
+                for (; n_issued < min(nchunks, kVStages); ++n_issued) issue_v(n_issued);
+            for (int j = kVStages; j < nchunks && n_issued == j; ++j) {
                 if (!mbar_wait(bar(B_VEMPTY + j % kVStages), ((j / kVStages) - 1) & 1, abort)) break;
                 issue_v(j);
                 ++n_issued;
@@ -345,81 +350,108 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Chunk j belongs to warpgroup h = j % 2: S_j goes to TMEM buffer h, P_j
+        // comes from P buffer h, and P_j V_j accumulates into O_h.  Order of
+        // issue: S_0, S_1, then for each j: S_{j+2} as soon as warpgroup h has
+        // read S_j, then P_j V_j once P_j is written.
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
+            auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T
+                const int st = j % kKStages;
+                if (!mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) return false;
+                fence_after_sync();
+                const uint32_t kq = sb + kOffQ, kk = sb + kOffK + st * kTile;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
+                    umma_bf16(tmem + (uint32_t)(j & 1) * 128u, umma_desc(kq + off, 16, 1024),
+                              umma_desc(kk + off, 16, 1024), idS, k > 0);
+                }
+                umma_commit(bar(B_SFULL + (j & 1)));
+                umma_commit(bar(B_KEMPTY + st));
+                return true;
+            };
             bool ok = mbar_wait(bar(B_QFULL), 0, abort);
-            for (int j = 0; ok && j <= nchunks; ++j) {
-                if (j < nchunks) {   // S_j = Q K_j^T into TMEM buffer j % 2
-                    const int st = j % kKStages;
-                    if (!mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) break;
-                    fence_after_sync();
-                    const uint32_t kq = sb + kOffQ, kk = sb + kOffK + st * kTile;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                        umma_bf16(tmem + (uint32_t)(j & 1) * 128u, umma_desc(kq + off, 16, 1024),
-                                  umma_desc(kk + off, 16, 1024), idS, k > 0);
-                    }
-                    umma_commit(bar(B_SFULL + (j & 1)));
-                    umma_commit(bar(B_KEMPTY + st));
+            for (int j = 0; ok && j < min(nchunks, 2); ++j) ok = issue_s(j);
+            for (int j = 0; ok && j < nchunks; ++j) {   // S_{j+2}, then O_h += P_j V_j
+                const int h = j & 1, sv = j % kVStages;
+                if (j + 2 < nchunks) {
+                    if (!mbar_wait(bar(B_SFREE + h), (j >> 1) & 1, abort)) break;
+                    if (!issue_s(j + 2)) break;
                 }
-                if (j >= 1) {        // O += P_{j-1} V_{j-1}
-                    const int jp = j - 1, sv = jp % kVStages;
-                    if (!mbar_wait(bar(B_PFULL), jp & 1, abort)) break;
-                    if (!mbar_wait(bar(B_VFULL + sv), (jp / kVStages) & 1, abort)) break;
-                    fence_after_sync();
-                    const uint32_t kp = sb + kOffP, kv = sb + kOffV + sv * kTile;
+                if (!mbar_wait(bar(B_PFULL + h), (j >> 1) & 1, abort)) break;
+                if (!mbar_wait(bar(B_VFULL + sv), (j / kVStages) & 1, abort)) break;
+                fence_after_sync();
+                const uint32_t kp = sb + kOffP + (uint32_t)h * kTile, kv = sb + kOffV + sv * kTile;
+                // O_0 starts from the Unshared stage in final items
+                const bool acc0 = j >= 2 || (j == 0 && final_item);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t offp = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                        umma_bf16(tmem + 256u, umma_desc(kp + offp, 16, 1024),
-                                  umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
-                                  (jp > 0 || k > 0 || final_item) ? 1u : 0u);
-                    }
-                    umma_commit(bar(B_PVDONE));
-                    umma_commit(bar(B_VEMPTY + sv));
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t offp = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
+                    umma_bf16(tmem + 256u + (uint32_t)h * 128u, umma_desc(kp + offp, 16, 1024),
+                              umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
+                              (k > 0 || acc0) ? 1u : 0u);
                 }
+                umma_commit(bar(B_PVDONE + h));
+                umma_commit(bar(B_VEMPTY + sv));
             }
-            if (*abort) {   // every MMA issued so far must finish before TMEM is freed
-                umma_commit(bar(B_DRAIN));
-                mbar_wait(bar(B_DRAIN), 0, nullptr);
-            }
+            // arrives once every MMA issued above has completed (TMEM final / free)
+            umma_commit(bar(B_DONE));
+            if (*abort) mbar_wait(bar(B_DONE), 0, nullptr);
         }
     } else {
         // ------------------------------------------------------------ softmax
-        // thread (row, half): TMEM lane `row`, S columns [64*half, 64*half + 64);
-        // the two halves swap their partial row max through shared memory
+        // Warpgroup `half` owns the chunks j with j % 2 == half, whole rows: thread
+        // `row` reads TMEM lane `row` of S buffer `half`, keeps the running max and
+        // sum of accumulator O_half and writes row `row` of P buffer `half`.  The
+        // two warpgroups never wait for each other inside the loop; their
+        // (m, l, O) are merged at the end.  In the Unshared prologue thread
+        // (row, half) handles head-dim columns [64*half, 64*half + 64).
         const int half = (warp - 2) >> 2;
         const int row = 32 * (warp & 3) + lane;
-        fence_async_smem();
-        mbar_arrive(bar(B_QFULL));
+        bool ok = true;
+        if (!q_tma) {
+            fence_async_smem();
+            mbar_arrive(bar(B_QFULL));
+        }
 
         const RowInfo ri = row_info(a, it, row);
-        const bool live = ri.valid && ri.b < a.n_live[ri.r];
         const float cscale = kLog2e * rsqrtf(128.f);
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
         const uint32_t col0 = (uint32_t)(64 * half);
-        float m_used = -INFINITY, l = 0.f;
-        bool ok = true;
+        float m_used = -INFINITY, l = 0.f;   // running max / sum of O_half
         const Dims dm = a.dims;
         const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
         const int64_t kvo = (beam_row * dm.Hkv + it.g) * 128;
         const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
         const int64_t pool_req = (int64_t)ri.r * dm.BW * dm.Hkv * 128;
+        const int s_now = a.step;
+        const int n_tok = s_now + 1;
+        // the beam's ancestry slots are read together with n_live, while Q is in flight
+        int slot[kMaxSteps];
+        if (final_item) {
+#pragma unroll
+            for (int i = 0; i < kMaxSteps; ++i)
+                slot[i] = (ri.valid && i < s_now) ? a.st.anc[beam_row * dm.S + i] : ri.b;
+        }
+        const bool live = ri.valid && ri.b < a.n_live[ri.r];
+        float sc[kMaxSteps];   // scaled scores of the beam's own tokens (final items)
         if (final_item) {
             // ---- Unshared stage first (the item covers its requests' only KV
             // segment): the beam's own tokens of steps 0..s, read through its
-            // direct indices, seed the online softmax -- their max, their sum (on
-            // half 0) and their weighted values in the TMEM O accumulator.
-            const int s_now = a.step;
-            const int n_tok = s_now + 1;
+            // direct indices, seed the online softmax -- their max, their sum (half
+            // 0) and their weighted values in the TMEM O accumulator -- so the
+            // main loop merges the two stages as it goes.  Row hg = 0 of each beam
+            // also appends this step's k/v (already in registers) at Unshared slot
+            // (s, b).
+            const bool appender = live && ri.hg == 0;
             const __nv_bfloat16 *kp[kMaxSteps], *vp[kMaxSteps];
-            for (int i = 0; i < n_tok; ++i) {
+#pragma unroll
+            for (int i = 0; i < kMaxSteps; ++i) {
                 kp[i] = vp[i] = nullptr;
-                if (!live) continue;
-                const int slot = (i == s_now) ? ri.b : a.st.anc[beam_row * dm.S + i];
-                if (slot < 0 || slot >= dm.BW) {
+                if (!live || i >= n_tok) continue;
+                if (slot[i] < 0 || slot[i] >= dm.BW) {
                     set_status(a.status, XGR_DEV_INDEX);
                     continue;
                 }
@@ -427,194 +459,255 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     kp[i] = a.k_new + kvo;
                     vp[i] = a.v_new + kvo;
                 } else {
-                    const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot * dm.Hkv + it.g) * 128;
+                    const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot[i] * dm.Hkv + it.g) * 128;
                     kp[i] = a.pool_k + o2;
                     vp[i] = a.pool_v + o2;
                 }
+                if (i >= 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(kp[i] + col0));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(vp[i] + col0));
             }
-            float qf[64];
+            __nv_bfloat16 *const k_app = a.pool_k + s_now * pool_step + kvo + col0;
+            __nv_bfloat16 *const v_app = a.pool_v + s_now * pool_step + kvo + col0;
+            // the first two k rows load while Q is still in flight
+            uint4 k0[8], k1[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)), qf + 8 * c);
+            for (int c = 0; c < 8; ++c) {
+                k0[c] = kp[0] ? reinterpret_cast<const uint4 *>(kp[0] + col0)[c] : make_uint4(0, 0, 0, 0);
+                k1[c] = (1 < n_tok && kp[1]) ? reinterpret_cast<const uint4 *>(kp[1] + col0)[c]
+                                             : make_uint4(0, 0, 0, 0);
+            }
+            if (q_tma)   // the prologue reads Q from shared memory
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort));
             float *xd = reinterpret_cast<float *>(base + kOffP);   // [2 halves][kMaxSteps][128]
-            for (int i = 0; i < n_tok; ++i) {
-                float acc = 0.f;
-                if (kp[i]) {
-                    uint4 kv[8];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) kv[c] = reinterpret_cast<const uint4 *>(kp[i] + col0)[c];
+            for (int i = 0; i < kMaxSteps; i += 2) {
+                if (i >= n_tok) break;
+                if (i > 0) {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        float kf[8];
-                        unpack8(kv[c], kf);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) acc = fmaf(qf[8 * c + e], kf[e], acc);
+                        k0[c] = kp[i] ? reinterpret_cast<const uint4 *>(kp[i] + col0)[c] : make_uint4(0, 0, 0, 0);
+                        k1[c] = (i + 1 < n_tok && kp[i + 1])
+                                    ? reinterpret_cast<const uint4 *>(kp[i + 1] + col0)[c]
+                                    : make_uint4(0, 0, 0, 0);
                     }
                 }
-                xd[(half * kMaxSteps + i) * 128 + row] = acc;
+                if (appender && i == s_now) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(k_app)[c] = k0[c];
+                }
+                if (appender && i + 1 == s_now) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(k_app)[c] = k1[c];
+                }
+                float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {   // q (bf16, swizzled K-major) read 8 columns at a time
+                    float qf[8], f0[8], f1[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)), qf);
+                    unpack8(k0[c], f0);
+                    unpack8(k1[c], f1);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        acc0 = fmaf(qf[e], f0[e], acc0);
+                        acc1 = fmaf(qf[e], f1[e], acc1);
+                    }
+                }
+                xd[(half * kMaxSteps + i) * 128 + row] = acc0;
+                if (i + 1 < n_tok) xd[(half * kMaxSteps + i + 1) * 128 + row] = acc1;
             }
             named_sync(1, kSoftmaxThreads);
-            float sc[kMaxSteps];
             float m_u = -INFINITY;
-            for (int i = 0; i < n_tok; ++i) {
-                sc[i] = kp[i] ? (xd[i * 128 + row] + xd[(kMaxSteps + i) * 128 + row]) * cscale : -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kMaxSteps; ++i) {
+                sc[i] = (i < n_tok && kp[i]) ? (xd[i * 128 + row] + xd[(kMaxSteps + i) * 128 + row]) * cscale
+                                             : -INFINITY;
                 m_u = fmaxf(m_u, sc[i]);
             }
             named_sync(1, kSoftmaxThreads);   // the exchange area is reused by P afterwards
+            float l_u = 0.f;
             float o[64];
 #pragma unroll
             for (int e = 0; e < 64; ++e) o[e] = 0.f;
-            float l_u = 0.f;
-            for (int i = 0; i < n_tok; ++i) {
-                if (!vp[i]) continue;
+#pragma unroll
+            for (int i = 0; i < kMaxSteps; ++i) {
+                if (i >= n_tok || sc[i] == -INFINITY) continue;
                 const float pw = ex2(sc[i] - m_u);
                 l_u += pw;
+                uint4 vv[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) vv[c] = reinterpret_cast<const uint4 *>(vp[i] + col0)[c];
+                if (appender && i == s_now) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(v_app)[c] = vv[c];
+                }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     float vf[8];
-                    unpack8(reinterpret_cast<const uint4 *>(vp[i] + col0)[c], vf);
+                    unpack8(vv[c], vf);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw, vf[e], o[8 * c + e]);
                 }
             }
+            mbar_arrive(bar(B_PRO));   // the scattered loads are in: the K/V fill may start
+            // the Unshared stage seeds the O accumulator, the running max and (half 0) sum
             tmem_st32(tmem + lane_base + 256 + col0, o);
             tmem_st32(tmem + lane_base + 256 + col0 + 32, o + 32);
             tmem_wait_st();
-            if (live) {
+            if (live && half == 0) {   // O_0 holds the Unshared stage
                 m_used = m_u;
-                l = half == 0 ? l_u : 0.f;   // the row sum is split over the halves
-            }
-            // append this step's k (half 0) and v (half 1) at Unshared slot (s, b), once per kv head
-            if (live && ri.hg == 0) {
-                const __nv_bfloat16 *src = (half == 0 ? a.k_new : a.v_new) + kvo;
-                __nv_bfloat16 *dst = (half == 0 ? a.pool_k : a.pool_v) + s_now * pool_step + pool_req +
-                                     ((int64_t)ri.b * dm.Hkv + it.g) * 128;
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    reinterpret_cast<uint4 *>(dst)[c] = reinterpret_cast<const uint4 *>(src)[c];
+                l = l_u;
             }
         }
-        // Every softmax warp executes exactly one exchange barrier per chunk, even
-        // after an abort, so the named barrier can never deadlock.
-        for (int j = 0; j < nchunks; ++j) {
-            const int sbuf = j & 1;
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + sbuf), (j >> 1) & 1, abort));
-            float s[64];
-            float mine = -INFINITY;
-            if (ok) {
-                fence_after_sync();
-                tmem_ld32(tmem + lane_base + sbuf * 128 + col0, s);
-                tmem_ld32(tmem + lane_base + sbuf * 128 + col0 + 32, s + 32);
+        const uint32_t s_col = (uint32_t)half * 128u;          // S buffer of this warpgroup
+        const uint32_t o_col = 256u + (uint32_t)half * 128u;   // its O accumulator
+        uint8_t *pb = base + kOffP + (uint32_t)half * kTile;   // its P buffer
+        for (int j = half, jj = 0; ok && j < nchunks; j += 2, ++jj) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + half), jj & 1, abort));
+            if (!ok) break;
+            fence_after_sync();
+            const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
+            // pass 1: the row max over the chunk's 128 scores
+            float mxp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                float sv[64];
+                tmem_ld32(tmem + lane_base + s_col + 64 * q2, sv);
+                tmem_ld32(tmem + lane_base + s_col + 64 * q2 + 32, sv + 32);
                 tmem_wait_ld();
-                const int nvalid = n_keys - j * kBlockN - (int)col0;
-                float mxp[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    if (c >= nvalid) s[c] = -INFINITY;
-                    mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
-                }
-                mine = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-                red[(sbuf * 2 + half) * 128 + row] = mine;
+                for (int c = 0; c < 64; ++c)
+                    if (64 * q2 + c < nvalid) mxp[c & 7] = fmaxf(mxp[c & 7], sv[c]);
             }
-            named_sync(1, kSoftmaxThreads);
-            if (!ok) continue;
-            const float mx = fmaxf(mine, red[(sbuf * 2 + (half ^ 1)) * 128 + row]) * cscale;
+            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * cscale;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + 8.f) {   // lazy rescaling: keep the old max unless it grew by 2^8
                 alpha = ex2(m_used - mx);
-                rescale = j > 0 || final_item;   // O holds the Unshared stage in final items
+                rescale = jj > 0 || (half == 0 && final_item);   // O_half already holds data
                 m_used = mx;
             }
-            // P buffer free and O complete up to chunk j-1 once P V of chunk j-1 is done
-            if (j >= 1) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE), (j - 1) & 1, abort));
-                if (!ok) continue;
+            // P V of this warpgroup's previous chunk has read P_half and written O_half
+            if (jj > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + half), (jj - 1) & 1, abort));
+                if (!ok) break;
             }
             if (__any_sync(0xffffffffu, rescale)) {
                 fence_after_sync();
                 const float f = rescale ? alpha : 1.f;
 #pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
+                for (int q2 = 0; q2 < 4; ++q2) {
                     float o[32];
-                    tmem_ld32(tmem + lane_base + 256 + col0 + q2 * 32, o);
+                    tmem_ld32(tmem + lane_base + o_col + q2 * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] *= f;
-                    tmem_st32(tmem + lane_base + 256 + col0 + q2 * 32, o);
+                    tmem_st32(tmem + lane_base + o_col + q2 * 32, o);
                 }
                 tmem_wait_st();
             }
-            // exponentials, row sum and P (bf16), 8 columns (one 16-byte chunk) at a time
+            // pass 2: exponentials, row sum and P (bf16), 8 columns (16 bytes) at a time
             const float neg_m = -m_used;
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-            uint8_t *pb = base + kOffP;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2(fmaf(s[8 * c + 2 * e], cscale, neg_m));
-                    const float p1 = ex2(fmaf(s[8 * c + 2 * e + 1], cscale, neg_m));
-                    sp[(2 * e) & 7] += p0;
-                    sp[(2 * e + 1) & 7] += p1;
-                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                    w4[e] = *reinterpret_cast<uint32_t *>(&h);
+            for (int q2 = 0; q2 < 2; ++q2) {
+                float sv[64];
+                tmem_ld32(tmem + lane_base + s_col + 64 * q2, sv);
+                tmem_ld32(tmem + lane_base + s_col + 64 * q2 + 32, sv + 32);
+                tmem_wait_ld();
+                if (q2 == 1) {   // S_j fully read: its buffer may take S_{j+2}
+                    fence_before_sync();
+                    mbar_arrive(bar(B_SFREE + half));
                 }
-                *reinterpret_cast<uint4 *>(pb + sw128_off(row, 8 * half + c)) =
-                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int cc = 64 * q2 + 8 * c + 2 * e;
+                        const float p0 =
+                            cc < nvalid ? ex2(fmaf(sv[8 * c + 2 * e], cscale, neg_m)) : 0.f;
+                        const float p1 =
+                            cc + 1 < nvalid ? ex2(fmaf(sv[8 * c + 2 * e + 1], cscale, neg_m)) : 0.f;
+                        sp[(2 * e) & 7] += p0;
+                        sp[(2 * e + 1) & 7] += p1;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        w4[e] = *reinterpret_cast<uint32_t *>(&h2);
+                    }
+                    *reinterpret_cast<uint4 *>(pb + sw128_off(row, 8 * q2 + c)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
             }
             l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
             fence_async_smem();
             fence_before_sync();
-            mbar_arrive(bar(B_PFULL));
+            mbar_arrive(bar(B_PFULL + half));
         }
-        if (ok && nchunks > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE), (nchunks - 1) & 1, abort));
+        // every MMA done: O_0 and O_1 are final, the P buffers free
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort));
         if (ok) {
             fence_after_sync();
-            // the halves swap their partial row sums (P buffer is free now)
-            float *xl = reinterpret_cast<float *>(base + kOffP);
-            xl[half * 128 + row] = l;
+            // the warpgroups swap (m, l); thread (row, half) then merges head-dim
+            // columns [64*half, 64*half + 64) of O_0 and O_1
+            float2 *xl = reinterpret_cast<float2 *>(base + kOffP);   // [2][128]
+            xl[half * 128 + row] = make_float2(m_used, l);
             mbar_arrive(bar(B_XCH + half));
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH + (half ^ 1)), 0, abort));
-            const float l_row = l + xl[(half ^ 1) * 128 + row];
+            const float2 other = xl[(half ^ 1) * 128 + row];
+            const float m0 = half == 0 ? m_used : other.x, l0 = half == 0 ? l : other.y;
+            const float m1 = half == 0 ? other.x : m_used, l1 = half == 0 ? other.y : l;
+            const float M = fmaxf(m0, m1);
+            // an accumulator that never received a chunk (m = -inf) holds no data
+            const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+            const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+            const float l_row = l0 * f0 + l1 * f1;
             if (ok) {
-                float o[64];
-                tmem_ld32(tmem + lane_base + 256 + col0, o);
-                tmem_ld32(tmem + lane_base + 256 + col0 + 32, o + 32);
-                tmem_wait_ld();
-                if (!final_item) {
-                    if (live) {
-                        float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + col0;
 #pragma unroll
-                        for (int e = 0; e < 64; e += 4)
-                            *reinterpret_cast<float4 *>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
-                        if (half == 0)
-                            a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(m_used, l_row);
-                    }
-                } else if (ri.valid) {
-                    // final: O / l in bf16, LSE = m + log2(l) in natural log; dead rows 0 / -inf
-                    const float inv = live ? 1.f / l_row : 0.f;
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + col0);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float o[32], o1[32];
+                    tmem_ld32(tmem + lane_base + 256 + col0 + 32 * q2, o);
+                    tmem_ld32(tmem + lane_base + 384 + col0 + 32 * q2, o1);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t w4[4];
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = (f0 != 0.f ? o[e] * f0 : 0.f) + (f1 != 0.f ? o1[e] * f1 : 0.f);
+                    const uint32_t c0 = col0 + 32 * q2;
+                    if (!final_item) {
+                        if (live) {
+                            float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + c0;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float v0 = live ? o[8 * c + 2 * e] * inv : 0.f;
-                            const float v1 = live ? o[8 * c + 2 * e + 1] * inv : 0.f;
-                            __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                            w4[e] = *reinterpret_cast<uint32_t *>(&h);
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4 *>(dst + e) =
+                                    make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
                         }
-                        dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    } else if (ri.valid) {
+                        // final: O / l in bf16; dead rows 0
+                        const float inv = live ? 1.f / l_row : 0.f;
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + c0);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float v0 = live ? o[8 * c + 2 * e] * inv : 0.f;
+                                const float v1 = live ? o[8 * c + 2 * e + 1] * inv : 0.f;
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                                w4[e] = *reinterpret_cast<uint32_t *>(&h2);
+                            }
+                            dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
                     }
-                    if (half == 0) a.lse[ri.gid] = live ? (m_used + __log2f(l_row)) * kLn2 : -INFINITY;
+                }
+                if (half == 0) {
+                    if (!final_item) {
+                        if (live) a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(M, l_row);
+                    } else if (ri.valid) {   // LSE = m + log2(l) in natural log; dead rows -inf
+                        a.lse[ri.gid] = live ? (M + __log2f(l_row)) * kLn2 : -INFINITY;
+                    }
                 }
             }
         }
@@ -633,15 +726,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 }  // namespace
 
-cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows) {
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
         cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return nullptr;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    return encode;
+}
+
+cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {128, (cuuint64_t)rows};
     cuuint64_t strides[1] = {128 * 2};
     cuuint32_t box[2] = {64, 128};
@@ -652,8 +751,21 @@ cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows)
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const TcArgs &a,
-                           int n_items, cudaStream_t st) {
+cudaError_t make_q_tensor_map(CUtensorMap *map, const void *q, int64_t beam_rows, int Hq, int G) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {128, (cuuint64_t)Hq, (cuuint64_t)beam_rows};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)Hq * 128 * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+                           const TcArgs &a, int n_items, cudaStream_t st) {
     if (n_items <= 0) return cudaSuccess;
     static bool attr = false;
     if (!attr) {
@@ -671,7 +783,7 @@ cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const
         }
         attr = true;
     }
-    attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, a);
+    attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
     return cudaGetLastError();
 }
 

@@ -60,8 +60,10 @@ struct WorkItem {
     int32_t n_rows;      // rows of this item
     int32_t slot;        // partial slot this item writes for its rows
     int32_t flags;       // bit 0: final -- the item covers its requests' only KV segment
-                         // whole, so it also runs the Unshared and Merging stages
-    int32_t pad[2];
+                         // whole, so it also runs the Unshared and Merging stages;
+                         // bit 1: its query rows form one TMA box (a single request)
+    int32_t r0;          // the item's first member request
+    int32_t pad;
 };
 static_assert(sizeof(WorkItem) == 48, "WorkItem layout");
 

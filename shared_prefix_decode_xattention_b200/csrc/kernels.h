@@ -46,8 +46,10 @@ struct TcArgs {
 };
 // 2-D tensor map over a [rows][128] bf16 store, 64 x 128 boxes, 128-byte swizzle.
 cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows);
-cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const TcArgs &a,
-                           int n_items, cudaStream_t st);
+// 3-D tensor map over q [beam rows][Hq][128] bf16 with boxes 64 x G x (128 / G)
+cudaError_t make_q_tensor_map(CUtensorMap *map, const void *q, int64_t beam_rows, int Hq, int G);
+cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+                           const TcArgs &a, int n_items, cudaStream_t st);
 
 // Unshared stage + Merging stage (+ append of this step's k/v).
 struct MergeArgs {
@@ -68,7 +70,9 @@ struct MergeArgs {
 cudaError_t launch_attn_merge(const MergeArgs &a, cudaStream_t st);
 
 // Beam state reset of xgr_begin.
-cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, cudaStream_t s);
+// mask_sync: the mask builder's look-back words [Bcap] and ticket, zeroed here
+cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync,
+                         cudaStream_t s);
 
 // Sparse masks of steps >= 1: one CSR row per beam.
 struct MaskArgs {
@@ -79,8 +83,11 @@ struct MaskArgs {
     int32_t *row_ptr;   // [B*BW + 1]
     int32_t *cols;      // [cap]
     int64_t cap;
+    uint64_t *flags;    // [Bcap] published request totals (zero between calls)
+    uint32_t *ticket;   // [2]: CTAs done, CTAs started (zero between calls)
 };
-cudaError_t launch_build_mask(const MaskArgs &a, cudaStream_t s);
+// parts: CTAs per request that share the copy of its children
+cudaError_t launch_build_mask(const MaskArgs &a, int parts, cudaStream_t s);
 
 // Beam selection (+ in-place rewiring of the context's beam state).
 struct SelectArgs {
@@ -98,18 +105,33 @@ struct SelectArgs {
     const uint32_t *bits;
     const int32_t *row_ptr;
     const int32_t *cols;
-    float *row_lse;             // [B][BW] scratch
-    uint64_t *sample;           // [B][BW][kSampleK] scratch: each beam's best keys
+    int64_t max_entries;        // expected largest CSR entry count of one request (sizes the pick grid)
+    // scratch (select_scratch_carve)
+    float *row_lse;             // [B][BW]
+    uint64_t *best;             // [B][BW] each beam's best candidate key
+    int32_t *surv_cnt;          // [B] survivors appended
+    uint32_t *ticket;           // [B] pick CTAs done (reset by the rows kernel)
+    uint64_t *keys;             // [B][key_cap] key of each CSR entry (relative to the request)
+    int64_t key_cap;
+    uint64_t *surv_key;         // [B][surv_cap] candidates at or above the threshold
+    int32_t *surv_e;            // [B][surv_cap] their entry
+    int64_t surv_cap;
+    int pick_parts;             // set by the launcher
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
     float *cum_out;
     int32_t *n_out;             // [B]
 };
-constexpr int kSampleK = 4;     // best keys per beam kept for the threshold sample
-// scratch of the selection for `rows` beam rows: row_lse [rows] f32 at offset 0,
-// sample [rows][kSampleK] u64 at select_sample_offset(rows)
-size_t select_scratch_bytes(int64_t rows);
-size_t select_sample_offset(int64_t rows);
+// Largest vocabulary of the selection: a score row is staged whole in shared memory.
+constexpr int kSelectMaxVocab = 32768;
+// Scratch of the selection for B requests of BW beams: row_lse and best per
+// beam row, surv_cnt and ticket per request, keys [B][key_cap] (a request's
+// CSR entries beyond key_cap take the exact fallback over the scores) and the
+// survivor buffer [B][surv_cap] (more survivors: exact selection over the keys).
+// Everything in it is written by the same call before it is read.
+size_t select_scratch_bytes(int B, int BW, int64_t key_cap, int64_t surv_cap);
+void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, int64_t surv_cap,
+                          SelectArgs &a);
 cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
 
 cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);

@@ -1,0 +1,886 @@
+// select.cu -- masked beam Top-K with a global threshold (early termination)
+// and the in-place rewiring of the beam state.
+//
+// xGR page ("xGR: Efficient Generative Recommendation Serving at Scale"):
+//  2.2 "Valid-path constraint" / "Hybrid dense/sparse storage": candidates
+//      come only from the valid-item vocabulary -- a dense bitset of first
+//      tokens at step 0, sparse rows (each beam's sorted trie children) later.
+//      "Early sort termination": the page orders each beam's candidates and
+//      cuts every list at a global min-heap threshold.  Here the threshold tau
+//      is the worst of the live beams' best keys: with all BW beams live these
+//      are BW real candidates, so every one of the BW winners ranks at or
+//      above tau, and only the candidates at or above it ("survivors") reach
+//      the exact selection.
+//  2.1 "In-place updates": the beam state (ancestry slots, trie node, token
+//      history, cumulative score) is rewritten in place; every row a new beam
+//      reads is staged in shared memory before any row is written.
+//
+// Keys: 64-bit integers whose ascending order is the rank order (higher fp32
+// score, then lower parent beam, then lower token), so every comparison is an
+// exact integer comparison and ties resolve identically everywhere.
+//
+// Two shapes of work:
+//  * dense mask (one live beam per request): select_dense_kernel, one CTA per
+//    request, stages the beam's score row in shared memory with one bulk copy,
+//    takes its log-sum-exp (logits) and selects the best BW tokens there; the
+//    keys are recomputed from shared memory in every radix pass.
+//  * sparse (CSR) masks: select_rows_kernel, one CTA per beam row, stages the
+//    row (logits mode) with one bulk copy while it reads the row's CSR
+//    entries, and writes each entry's key beside its CSR position plus the
+//    row's best key; select_pick_kernel, a few CTAs per request, reduces tau
+//    from the best keys, filters its slices of the request's keys and appends
+//    the survivors; the last CTA of the request to finish (an atomic ticket
+//    that the rows kernel resets) runs the exact selection, the ordering, the
+//    outputs and the rewiring.
+#include <algorithm>
+
+#include "async.cuh"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace xgr {
+
+namespace {
+
+constexpr int kDenseThreads = 1024;
+constexpr int kRowThreads = 256;
+constexpr int kPickThreads = 512;
+constexpr int kPickKeys = 4096;    // keys one pick CTA filters per slice (8 per thread)
+constexpr int kSmemSurv = 4096;    // survivors selected in shared memory
+constexpr int kMaxPickParts = 16;
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// (m, s) pairs: s = sum of 2^((x - m) log2 e) over the values seen
+__device__ __forceinline__ void lse_combine(float &m, float &s, float m2, float s2) {
+    if (m2 > m) {
+        s = s * ex2f((m - m2) * kLog2e) + s2;
+        m = m2;
+    } else if (m2 != -INFINITY) {
+        s += s2 * ex2f((m2 - m) * kLog2e);
+    }
+}
+
+// key of (beam b, token t): one fp32 add of the beam's cumulative score and
+// the token's log-prob; -0.0 is canonical +0.0; NaN is reported and skipped
+__device__ __forceinline__ bool make_key(float cum, float lp, int b, int t, int V, int32_t *status,
+                                         uint64_t &key) {
+    float k = cum + lp;
+    if (isnan(k)) {
+        set_status(status, XGR_DEV_NAN);
+        return false;
+    }
+    if (k == 0.f) k = 0.f;
+    key = ((uint64_t)score_to_desc_bits(k) << 32) | (uint32_t)(b * V + t);
+    return true;
+}
+
+__device__ __forceinline__ uint64_t warp_min_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t u = __shfl_xor_sync(0xffffffffu, v, o);
+        v = u < v ? u : v;
+    }
+    return v;
+}
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t u = __shfl_xor_sync(0xffffffffu, v, o);
+        v = u > v ? u : v;
+    }
+    return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// block-wide reductions; every thread gets the result; red holds 32 entries
+__device__ uint64_t block_min_u64(uint64_t v, uint64_t *red) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    v = warp_min_u64(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    v = warp_min_u64(lane < nw ? red[lane] : kNoKey);
+    __syncthreads();
+    return v;
+}
+__device__ uint64_t block_max_u64(uint64_t v, uint64_t *red) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    v = warp_max_u64(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    v = warp_max_u64(lane < nw ? red[lane] : 0);
+    __syncthreads();
+    return v;
+}
+__device__ int block_sum_int(int v, int *red) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    v = warp_sum_int(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    v = warp_sum_int(lane < nw ? red[lane] : 0);
+    __syncthreads();
+    return v;
+}
+// block-wide exclusive scan of one int per thread; *total gets the block sum
+__device__ int block_exclusive_scan_int(int v, int *warp_tot, int *total) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int wt = lane < nw ? warp_tot[lane] : 0, wi = wt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += t;
+    }
+    const int before = __shfl_sync(0xffffffffu, wi - wt, warp);   // warps before this one
+    *total = __shfl_sync(0xffffffffu, wi, 31);
+    __syncthreads();
+    return before + incl - v;
+}
+
+// log-sum-exp of the values x[i], i = threadIdx.x (mod blockDim.x), i < n, in
+// shared memory; reports NaN; red holds 64 floats
+__device__ float block_lse(const float *x, int n, float *red, int32_t *status) {
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
+    float m = -INFINITY, s = 0.f;
+    bool nan = false;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * blockDim.x;
+            v[u] = i < n ? x[i] : -INFINITY;
+            nan |= isnan(v[u]);
+        }
+        const float cm = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+        if (cm > m) {
+            s *= ex2f((m - cm) * kLog2e);
+            m = cm;
+        }
+        if (cm != -INFINITY)
+            s += (ex2f((v[0] - m) * kLog2e) + ex2f((v[1] - m) * kLog2e)) +
+                 (ex2f((v[2] - m) * kLog2e) + ex2f((v[3] - m) * kLog2e));
+    }
+    if (nan) set_status(status, XGR_DEV_NAN);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_combine(m, s, m2, s2);
+    }
+    if (lane == 0) {
+        red[warp] = m;
+        red[32 + warp] = s;
+    }
+    __syncthreads();
+    m = red[0];
+    s = red[32];
+    for (int w = 1; w < nw; ++w) lse_combine(m, s, red[w], red[32 + w]);
+    __syncthreads();
+    return m + logf(s);
+}
+
+// Exact block-wide radix select over E candidates given by `cand(e, key)`
+// (false for a non-candidate).  Keys are unique.  On return exactly `want`
+// candidates satisfy (key & mask) <= prefix (want <= number of candidates).
+// hist: 256 ints of shared memory; sc: 3 shared ints.  The bucket holding the
+// want-th key is found by a one-warp scan of the 256 bins.
+template <class Cand>
+__device__ void radix_select(const Cand &cand, int64_t E, int want, int *hist, int *sc,
+                             uint64_t &prefix, uint64_t &mask) {
+    prefix = 0;
+    mask = 0;
+    int k_rem = want;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int64_t e = threadIdx.x; e < E; e += blockDim.x) {
+            uint64_t key;
+            if (cand(e, key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            int h[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                h[i] = hist[lane * 8 + i];
+                sum += h[i];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            int acc = incl - sum;   // keys in the bins before this lane's 8
+            // the lane whose range crosses k_rem owns the bucket
+            if (acc < k_rem && acc + sum >= k_rem) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (acc + h[i] >= k_rem) {
+                        sc[0] = lane * 8 + i;
+                        sc[1] = h[i] - (k_rem - acc);   // 0 <=> the whole bucket is taken
+                        sc[2] = k_rem - acc;
+                        break;
+                    }
+                    acc += h[i];
+                }
+            }
+        }
+        __syncthreads();
+        const int d = sc[0], surplus = sc[1];
+        k_rem = sc[2];
+        prefix |= (uint64_t)d << shift;
+        mask |= 0xFFull << shift;
+        __syncthreads();
+        if (surplus == 0) break;
+    }
+}
+
+// ---- candidate spaces
+
+// the dense first step: token t of beam 0, score row staged in shared memory
+struct DenseCand {
+    const float *x;
+    const uint32_t *bits;
+    float cum, lse;
+    int V, logits;
+    int32_t *status;
+    __device__ bool operator()(int64_t e, uint64_t &key) const {
+        const int t = (int)e;
+        if (!((bits[t >> 5] >> (t & 31)) & 1u)) return false;
+        float lp = x[t];
+        if (logits) lp -= lse;
+        return make_key(cum, lp, 0, t, V, status, key);
+    }
+};
+
+// survivor keys in shared memory (kGlobal = false) or, written by other CTAs
+// of the same launch, in global memory (read through L2)
+template <bool kGlobal>
+struct ListCand {
+    const uint64_t *k;
+    __device__ bool operator()(int64_t e, uint64_t &key) const {
+        key = kGlobal ? __ldcg(k + e) : k[e];
+        return true;
+    }
+};
+
+// the request's key buffer, restricted to the survivors of tau
+struct KeyCand {
+    const uint64_t *k;
+    uint64_t tau;
+    __device__ bool operator()(int64_t e, uint64_t &key) const {
+        key = __ldcg(k + e);
+        return key != kNoKey && key <= tau;
+    }
+};
+
+// every CSR entry of the request's live beams, keys recomputed from the scores
+// (rp = per-beam entry offsets relative to the request's first entry)
+struct ReqCand {
+    const float *x;          // scores of the request's first row
+    const int32_t *cols;     // CSR entries of the request's first row
+    const int *rp;           // [n+1] in shared memory
+    const float *cum, *lse;  // [n] in shared memory
+    int32_t *status;
+    int n, logits, V;
+    __device__ bool operator()(int64_t e, uint64_t &key) const {
+        int lo = 0, hi = n;   // beam b with rp[b] <= e < rp[b+1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (rp[mid] <= e) lo = mid; else hi = mid;
+        }
+        const int b = lo, t = cols[e];
+        if (t < 0 || t >= V) return false;
+        float lp = x[(int64_t)b * V + t];
+        if (logits) lp -= lse[b];
+        return make_key(cum[b], lp, b, t, V, status, key);
+    }
+};
+
+__device__ int find_child(const TrieView &tr, int level, int node, int t) {
+    if (level >= tr.levels || node < 0 || node >= tr.n_nodes[level]) return -1;
+    int lo = tr.ptr[level][node];
+    const int end = tr.ptr[level][node + 1];
+    int hi = end;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (tr.tok[level][mid] < t) lo = mid + 1; else hi = mid;
+    }
+    return (lo < end && tr.tok[level][lo] == t) ? lo : -1;
+}
+
+// ---- shared memory of the finishing CTA (carved from dynamic shared memory)
+
+struct FinishSmem {
+    uint64_t *win_k;   // [BW] winners (unordered)
+    int *win_e;        // [BW] their entry: CSR entry relative to the request (sparse) or token
+    int *rank;         // [BW]
+    int *rp;           // [BW+1] sparse: entry offset of each live beam
+    int *st_node;      // [n_stage] staged old rows (rewiring)
+    int *st_anc;       // [n_stage*S]
+    int *st_seq;       // [n_stage*S]
+    int *cb, *ce;      // [n_stage] sparse: child range of each staged row's trie node
+    uint32_t *root;    // dense: [nw] root-children bitset, [nw] prefix popcounts
+    int *cnt;          // winners appended
+};
+
+__host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// n_stage: old rows staged for the rewiring (the live beams: BW, or 1 for a dense step)
+__host__ __device__ inline size_t finish_bytes(int BW, int n_stage, int S, int nw_root) {
+    return al16((size_t)BW * 8) + 2 * al16((size_t)BW * 4) + al16((size_t)(BW + 1) * 4) +
+           3 * al16((size_t)n_stage * 4) + 2 * al16((size_t)n_stage * S * 4) + al16((size_t)nw_root * 8) +
+           16;
+}
+
+__device__ FinishSmem carve_finish(uint8_t *p, int BW, int n_stage, int S, int nw_root) {
+    FinishSmem f;
+    f.win_k = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)BW * 8);
+    f.win_e = reinterpret_cast<int *>(p);
+    p += al16((size_t)BW * 4);
+    f.rank = reinterpret_cast<int *>(p);
+    p += al16((size_t)BW * 4);
+    f.rp = reinterpret_cast<int *>(p);
+    p += al16((size_t)(BW + 1) * 4);
+    f.st_node = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * 4);
+    f.st_anc = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * S * 4);
+    f.st_seq = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * S * 4);
+    f.cb = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * 4);
+    f.ce = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * 4);
+    f.root = reinterpret_cast<uint32_t *>(p);
+    p += al16((size_t)nw_root * 8);
+    f.cnt = reinterpret_cast<int *>(p);
+    return f;
+}
+
+// stage the request's old beam rows (n live beams) for the rewiring
+__device__ void stage_rows(const SelectArgs &a, int64_t rb, int n, const FinishSmem &f) {
+    const int S = a.dims.S;
+    for (int i = threadIdx.x; i < n * S; i += blockDim.x) {
+        f.st_anc[i] = a.st.anc[rb * S + i];
+        f.st_seq[i] = a.st.seq[rb * S + i];
+    }
+    for (int b = threadIdx.x; b < n; b += blockDim.x) f.st_node[b] = a.st.node[rb + b];
+}
+
+// child range of every staged row's trie node (sparse steps; after stage_rows)
+__device__ void stage_children(const SelectArgs &a, int n, const FinishSmem &f) {
+    const int s = a.step;
+    for (int b = threadIdx.x; b < n; b += blockDim.x) {
+        const int node = f.st_node[b];
+        const bool ok = s < a.trie.levels && node >= 0 && node < a.trie.n_nodes[s];
+        f.cb[b] = ok ? a.trie.ptr[s][node] : -1;
+        f.ce[b] = ok ? a.trie.ptr[s][node + 1] : -1;
+    }
+}
+
+// append the winners among the candidates [0, E) of `cand` ((key & mask) <= prefix)
+template <class Cand, class Entry>
+__device__ void collect(const Cand &cand, int64_t E, uint64_t prefix, uint64_t mask, int BW,
+                        const Entry &entry, const FinishSmem &f) {
+    for (int64_t e = threadIdx.x; e < E; e += blockDim.x) {
+        uint64_t key;
+        if (cand(e, key) && (key & mask) <= prefix) {
+            const int pos = atomicAdd(f.cnt, 1);
+            if (pos < BW) {
+                f.win_k[pos] = key;
+                f.win_e[pos] = entry(e);
+            }
+        }
+    }
+}
+
+// Rank the n_win winners (unique keys; a winner's rank is its number of better
+// winners, counted by one warp per winner), write the outputs in rank order
+// and, when a.rewire, rewrite the request's beam state in place.  The caller
+// has staged the old rows (stage_rows) and rp / root.
+__device__ void finish_request(const SelectArgs &a, int r, int n_win, const FinishSmem &f) {
+    const Dims dm = a.dims;
+    const int BW = dm.BW, S = dm.S, V = dm.V;
+    const int64_t rb = (int64_t)r * BW;
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+    for (int i = warp; i < n_win; i += nwarps) {
+        const uint64_t k = f.win_k[i];
+        int c = 0;
+        for (int j = lane; j < n_win; j += 32) c += f.win_k[j] < k;
+        c = warp_sum_int(c);
+        if (lane == 0) f.rank[i] = c;
+    }
+    __syncthreads();
+    const int s = a.step;
+    for (int i = threadIdx.x; i < BW; i += blockDim.x) {
+        if (i < n_win) {
+            const int nb = f.rank[i];
+            const int64_t o = rb + nb;
+            const uint64_t key = f.win_k[i];
+            const uint32_t lo = (uint32_t)key;
+            const int p = (int)(lo / (uint32_t)V), t = (int)(lo % (uint32_t)V);
+            const float sc = desc_bits_to_score((uint32_t)(key >> 32));
+            a.parent[o] = p;
+            a.token[o] = t;
+            a.cum_out[o] = sc;
+            if (!a.rewire) continue;
+            for (int j = 0; j < S; ++j) {
+                int av = -1, sv = -1;
+                if (j < s) {
+                    av = f.st_anc[p * S + j];
+                    sv = f.st_seq[p * S + j];
+                } else if (j == s) {
+                    av = p;    // the parent's own token of step s sits at slot (s, p)
+                    sv = t;
+                } else if (j == s + 1) {
+                    av = nb;   // the new beam's token of step s+1 will sit at slot (s+1, nb)
+                }
+                a.st.anc[o * S + j] = av;
+                a.st.seq[o * S + j] = sv;
+            }
+            // the trie child of the parent's node through token t
+            int child = -1;
+            const int node = f.st_node[p];
+            if (a.dense) {
+                if (s == 0 && node == 0 && a.trie.levels > 0 && a.trie.root_bits) {
+                    // the root's children in trie order are its bitset in token order
+                    const int nw = (V + 31) / 32;
+                    const uint32_t w = f.root[t >> 5], bit = 1u << (t & 31);
+                    if (w & bit) child = (int)f.root[nw + (t >> 5)] + __popc(w & (bit - 1u));
+                } else {
+                    child = find_child(a.trie, s, node, t);
+                }
+            } else if (f.cb[p] >= 0) {
+                // the mask row of parent p lists its children in trie order, so
+                // the entry index locates the child directly
+                const int c = f.cb[p] + (f.win_e[i] - f.rp[p]);
+                if (c < f.ce[p] && a.trie.tok[s][c] == t) child = c;
+            }
+            if (child < 0) set_status(a.status, XGR_DEV_MASK);
+            a.st.node[o] = child;
+            a.st.cum[o] = sc;
+        } else {
+            const int64_t o = rb + i;
+            a.parent[o] = -1;
+            a.token[o] = -1;
+            a.cum_out[o] = -INFINITY;
+            if (!a.rewire) continue;
+            for (int j = 0; j < S; ++j) {
+                a.st.anc[o * S + j] = -1;
+                a.st.seq[o * S + j] = -1;
+            }
+            a.st.node[o] = -1;
+            a.st.cum[o] = -INFINITY;
+        }
+    }
+    if (threadIdx.x == 0) {
+        a.n_out[r] = n_win;
+        if (a.rewire) a.st.n_live[r] = n_win;
+    }
+}
+
+// ------------------------------------------------------------------ dense step
+
+__host__ __device__ inline size_t dense_x_bytes(int V) { return al16((size_t)V * 4); }
+__host__ __device__ inline size_t dense_bits_bytes(int V) { return al16((size_t)((V + 31) / 32) * 4); }
+
+size_t dense_smem(const Dims &dm) {
+    return dense_x_bytes(dm.V) + dense_bits_bytes(dm.V) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32);
+}
+
+__global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bar_mem;
+    __shared__ float red_f[64];
+    __shared__ int red_i[32];
+    __shared__ int hist[256];
+    __shared__ int sc[4];
+    const Dims dm = a.dims;
+    const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32;
+    const int r = blockIdx.x, tid = threadIdx.x;
+    const int64_t rb = (int64_t)r * BW;
+    float *x = reinterpret_cast<float *>(smem);
+    uint32_t *bits = reinterpret_cast<uint32_t *>(smem + dense_x_bytes(V));
+    const FinishSmem f = carve_finish(smem + dense_x_bytes(V) + dense_bits_bytes(V), BW, 1, dm.S, nw);
+    const float *xg = a.scores + rb * V;   // beam 0 of request r
+    const uint32_t bar = smem_u32(&bar_mem);
+    const bool bulk = (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
+    if (tid == 0) {
+        *f.cnt = 0;
+        if (bulk) {
+            mbar_init(bar, 1);
+            fence_mbar_init();
+            mbar_expect_tx(bar, (uint32_t)V * 4u);
+            bulk_g2s(smem_u32(x), xg, (uint32_t)V * 4u, bar);
+        }
+    }
+    const int n = min(a.n_live[r], 1);
+    const float cum = a.cum[rb];
+    for (int w = tid; w < nw; w += blockDim.x) bits[w] = a.bits[w];
+    if (a.rewire) {
+        stage_rows(a, rb, n, f);
+        // root children: bitset and exclusive prefix popcounts (trie order = token order)
+        if (a.trie.root_bits) {
+            int c = 0;
+            for (int w = tid; w < nw; w += blockDim.x) {   // nw <= blockDim.x (V <= 32768)
+                const uint32_t v = a.trie.root_bits[w];
+                f.root[w] = v;
+                c = __popc(v);
+            }
+            // block exclusive scan of one count per thread
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid % 32 >= o) incl += t;
+            }
+            if (tid % 32 == 31) red_i[tid / 32] = incl;
+            __syncthreads();
+            if (tid < 32) {
+                const int wv = red_i[tid];
+                int wi = wv;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int t = __shfl_up_sync(0xffffffffu, wi, o);
+                    if (tid >= o) wi += t;
+                }
+                red_i[tid] = wi - wv;
+            }
+            __syncthreads();
+            if (tid < nw) f.root[nw + tid] = (uint32_t)(red_i[tid / 32] + incl - c);
+            __syncthreads();
+        }
+    }
+    if (!bulk)
+        for (int i = tid; i < V; i += blockDim.x) x[i] = xg[i];
+    __syncthreads();
+    if (bulk && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
+    float lse = 0.f;
+    if (a.logits && n > 0) lse = block_lse(x, V, red_f, a.status);
+    int c = 0;   // candidates: mask bits below V
+    for (int w = tid; w < nw; w += blockDim.x)
+        c += __popc(bits[w] & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u));
+    const int total = n > 0 ? block_sum_int(c, red_i) : 0;
+    const int want = min(BW, total);
+    DenseCand cand{x, bits, cum, lse, V, a.logits, a.status};
+    const int64_t E = n > 0 ? V : 0;
+    uint64_t prefix = ~0ull, mask = 0;
+    if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
+    collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    __syncthreads();
+    finish_request(a, r, min(*f.cnt, want), f);
+}
+
+// ------------------------------------------------------------------ sparse steps
+
+__global__ void __launch_bounds__(kRowThreads) select_rows_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bar_mem;
+    __shared__ float red_f[64];
+    __shared__ uint64_t red_k[32];
+    const Dims dm = a.dims;
+    const int V = dm.V;
+    const int64_t row = blockIdx.x;
+    const int r = (int)(row / dm.BW), b = (int)(row % dm.BW);
+    const int64_t rb = (int64_t)r * dm.BW;
+    const int tid = threadIdx.x;
+    float *x = reinterpret_cast<float *>(smem);
+    const float *xg = a.scores + row * V;
+    const uint32_t bar = smem_u32(&bar_mem);
+    // logits mode needs the whole row (its log-sum-exp); it is staged in shared
+    // memory with one bulk copy while the CSR entries are read
+    const bool stage = a.logits;
+    const bool bulk = stage && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
+    if (tid == 0 && bulk) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar, (uint32_t)V * 4u);
+        bulk_g2s(smem_u32(x), xg, (uint32_t)V * 4u, bar);
+    }
+    const int n = a.n_live[r];
+    const int base = a.row_ptr[rb];
+    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
+    const float cum = a.cum[row];
+    if (b == 0 && tid == 0) {   // the pick kernel counts from 0
+        a.surv_cnt[r] = 0;
+        a.ticket[r] = 0;
+    }
+    const bool live = b < n;
+    // the row's entries, up to 4 per thread per batch: tokens first
+    constexpr int U = 4;
+    const int n_e = max(0, end - beg);
+    int tk[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int j = tid + u * kRowThreads;
+        tk[u] = (live && j < n_e) ? a.cols[beg + j] : -1;
+    }
+    if (stage && !bulk)
+        for (int i = tid; i < V; i += kRowThreads) x[i] = xg[i];
+    __syncthreads();
+    if (bulk && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
+    float lse = 0.f;
+    if (stage && live) lse = block_lse(x, V, red_f, a.status);
+    uint64_t *keys = a.keys + (int64_t)r * a.key_cap - base;   // keys[e] for CSR entry e
+    const int64_t kend = (int64_t)base + a.key_cap;
+    uint64_t best = kNoKey;
+    for (int j0 = 0; j0 < n_e; j0 += U * kRowThreads) {
+        if (j0 > 0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + tid + u * kRowThreads;
+                tk[u] = (live && j < n_e) ? a.cols[beg + j] : -1;
+            }
+        }
+        float lv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = j0 + tid + u * kRowThreads;
+            const bool ok = live && j < n_e && tk[u] >= 0 && tk[u] < V;
+            if (live && j < n_e && !ok) set_status(a.status, XGR_DEV_MASK);
+            lv[u] = ok ? (stage ? x[tk[u]] : xg[tk[u]]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int j = j0 + tid + u * kRowThreads;
+            if (j >= n_e) continue;
+            uint64_t key = kNoKey;
+            if (live && tk[u] >= 0 && tk[u] < V) {
+                float lp = lv[u];
+                if (a.logits) lp -= lse;
+                uint64_t k2;
+                if (make_key(cum, lp, b, tk[u], V, a.status, k2)) key = k2;
+            }
+            const int64_t e = (int64_t)beg + j;
+            if (e >= base && e < kend) keys[e] = key;
+            best = key < best ? key : best;
+        }
+    }
+    best = block_min_u64(best, red_k);
+    if (tid == 0) {
+        a.best[row] = best;
+        a.row_lse[row] = lse;
+    }
+}
+
+size_t pick_smem(const Dims &dm) {
+    return (size_t)kSmemSurv * 12 + finish_bytes(dm.BW, dm.BW, dm.S, 0) + al16((size_t)dm.BW * 8);
+}
+
+__global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t red_k[32];
+    __shared__ int hist[256];
+    __shared__ int sc[4];
+    __shared__ int last;
+    __shared__ int scan_w[32];
+    __shared__ int slice_base;
+    const Dims dm = a.dims;
+    const int BW = dm.BW, P = a.pick_parts;
+    const int r = blockIdx.x / P, part = blockIdx.x % P;
+    const int tid = threadIdx.x;
+    const int64_t rb = (int64_t)r * BW;
+    const int n = a.n_live[r];
+    const int base = a.row_ptr[rb];
+    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;   // dead rows' entries hold kNoKey
+    // tau: the worst of the live beams' best keys, when all BW beams are live
+    uint64_t worst = 0;
+    for (int b = tid; b < BW; b += kPickThreads) {
+        const uint64_t k = a.best[rb + b];
+        if (b < n) worst = k > worst ? k : worst;
+    }
+    worst = block_max_u64(worst, red_k);
+    const uint64_t tau = n == BW ? worst : kNoKey;
+    const bool fits = E <= a.key_cap;
+    const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
+    uint64_t *sk_g = a.surv_key + (int64_t)r * a.surv_cap;
+    int32_t *se_g = a.surv_e + (int64_t)r * a.surv_cap;
+    if (fits) {
+        // survivors of each slice: a block scan of the per-thread counts, one
+        // atomic per slice for the slice's place in the request's buffer
+        constexpr int U = kPickKeys / kPickThreads;
+        for (int64_t s0 = (int64_t)part * kPickKeys; s0 < E; s0 += (int64_t)P * kPickKeys) {
+            uint64_t k[U];
+            int c = 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t e = s0 + tid + u * kPickThreads;
+                k[u] = e < E ? __ldcg(keys + e) : kNoKey;
+                c += k[u] != kNoKey && k[u] <= tau;
+            }
+            int n_slice;
+            int pos = block_exclusive_scan_int(c, scan_w, &n_slice);
+            if (tid == 0) slice_base = n_slice ? atomicAdd(&a.surv_cnt[r], n_slice) : 0;
+            __syncthreads();
+            pos += slice_base;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (k[u] == kNoKey || k[u] > tau) continue;
+                if (pos < a.surv_cap) {
+                    sk_g[pos] = k[u];
+                    se_g[pos] = (int32_t)(s0 + tid + u * kPickThreads);
+                }
+                ++pos;
+            }
+            __syncthreads();   // slice_base is reused
+        }
+    }
+    // the last CTA of the request to finish its slices takes the selection
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(&a.ticket[r], 1u) == (unsigned)(P - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+
+    uint64_t *sk = reinterpret_cast<uint64_t *>(smem);
+    int *se = reinterpret_cast<int *>(smem + (size_t)kSmemSurv * 8);
+    uint8_t *fin = smem + (size_t)kSmemSurv * 12;
+    const FinishSmem f = carve_finish(fin, BW, BW, dm.S, 0);
+    float *cum_s = reinterpret_cast<float *>(fin + finish_bytes(BW, BW, dm.S, 0));
+    float *lse_s = cum_s + BW;
+    const int T = __ldcg(&a.surv_cnt[r]);
+    if (tid == 0) *f.cnt = 0;
+    for (int b = tid; b <= n; b += kPickThreads) f.rp[b] = a.row_ptr[rb + b] - base;
+    if (a.rewire) stage_rows(a, rb, n, f);
+    if (!fits)
+        for (int b = tid; b < n; b += kPickThreads) {
+            cum_s[b] = a.cum[rb + b];
+            lse_s[b] = a.logits ? a.row_lse[rb + b] : 0.f;
+        }
+    __syncthreads();
+    // the survivors and the parents' child ranges load together
+    const bool in_smem = fits && T <= kSmemSurv;
+    if (in_smem) {
+        for (int i = tid; i < T; i += kPickThreads) {
+            sk[i] = __ldcg(sk_g + i);
+            se[i] = __ldcg(se_g + i);
+        }
+    }
+    if (a.rewire) stage_children(a, n, f);
+    __syncthreads();
+    uint64_t prefix = ~0ull, mask = 0;
+    int want;
+    if (fits) {
+        // every winner survived tau; T >= BW whenever tau cuts anything
+        want = min(BW, T);
+        if (in_smem) {
+            const ListCand<false> cand{sk};
+            if (want < T) radix_select(cand, T, want, hist, sc, prefix, mask);
+            collect(cand, T, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
+        } else if (T <= a.surv_cap) {
+            const ListCand<true> cand{sk_g};
+            if (want < T) radix_select(cand, T, want, hist, sc, prefix, mask);
+            collect(cand, T, prefix, mask, BW, [&](int64_t i) { return __ldcg(se_g + i); }, f);
+        } else {
+            const KeyCand cand{keys, tau};
+            if (want < T) radix_select(cand, E, want, hist, sc, prefix, mask);
+            collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+        }
+    } else {
+        // the key buffer overflowed: exact selection over every candidate
+        ReqCand cand;
+        cand.x = a.scores + rb * dm.V;
+        cand.cols = a.cols + base;
+        cand.rp = f.rp;
+        cand.cum = cum_s;
+        cand.lse = lse_s;
+        cand.status = a.status;
+        cand.n = n;
+        cand.logits = a.logits;
+        cand.V = dm.V;
+        const int total = f.rp[n];
+        want = min(BW, total);
+        if (want < total) radix_select(cand, total, want, hist, sc, prefix, mask);
+        collect(cand, total, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    }
+    __syncthreads();
+    finish_request(a, r, min(*f.cnt, want), f);
+}
+
+template <class K>
+cudaError_t ensure_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t select_scratch_bytes(int B, int BW, int64_t key_cap, int64_t surv_cap) {
+    const size_t rows = (size_t)B * BW;
+    return al256(rows * 4) + al256(rows * 8) + al256((size_t)B * 4) + al256((size_t)B * 4) +
+           al256((size_t)B * key_cap * 8) + al256((size_t)B * surv_cap * 8) +
+           al256((size_t)B * surv_cap * 4);
+}
+
+void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, int64_t surv_cap,
+                          SelectArgs &a) {
+    const size_t rows = (size_t)B * BW;
+    a.row_lse = reinterpret_cast<float *>(base);
+    base += al256(rows * 4);
+    a.best = reinterpret_cast<uint64_t *>(base);
+    base += al256(rows * 8);
+    a.surv_cnt = reinterpret_cast<int32_t *>(base);
+    base += al256((size_t)B * 4);
+    a.ticket = reinterpret_cast<uint32_t *>(base);
+    base += al256((size_t)B * 4);
+    a.keys = reinterpret_cast<uint64_t *>(base);
+    base += al256((size_t)B * key_cap * 8);
+    a.surv_key = reinterpret_cast<uint64_t *>(base);
+    base += al256((size_t)B * surv_cap * 8);
+    a.surv_e = reinterpret_cast<int32_t *>(base);
+    a.key_cap = key_cap;
+    a.surv_cap = surv_cap;
+}
+
+cudaError_t launch_beam_select(const SelectArgs &a_in, cudaStream_t s) {
+    SelectArgs a = a_in;
+    const Dims &dm = a.dims;
+    if (dm.BW > 1024 || dm.V > kSelectMaxVocab || dm.V < 1) return cudaErrorInvalidValue;
+    if (a.dense) {
+        const size_t smem = dense_smem(dm);
+        cudaError_t e = ensure_smem(select_dense_kernel, smem);
+        if (e != cudaSuccess) return e;
+        select_dense_kernel<<<dm.B, kDenseThreads, smem, s>>>(a);
+        return cudaGetLastError();
+    }
+    {
+        const size_t smem = a.logits ? dense_x_bytes(dm.V) : 0;
+        cudaError_t e = ensure_smem(select_rows_kernel, smem);
+        if (e != cudaSuccess) return e;
+        select_rows_kernel<<<dm.B * dm.BW, kRowThreads, smem, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    int64_t parts = (std::min<int64_t>(a.max_entries, a.key_cap) + kPickKeys - 1) / kPickKeys;
+    a.pick_parts = (int)std::max<int64_t>(1, std::min<int64_t>(parts, kMaxPickParts));
+    const size_t smem = pick_smem(dm);
+    cudaError_t e = ensure_smem(select_pick_kernel, smem);
+    if (e != cudaSuccess) return e;
+    select_pick_kernel<<<dm.B * a.pick_parts, kPickThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace xgr

@@ -11,15 +11,17 @@
 // beam counts and the mask, and gets parent / token / cum / n_out back.
 //
 // It runs the very same selection kernels as xgr_beam_select (without the
-// rewiring).  Their scratch (each beam's row log-sum-exp and best keys) lives in
-// one file-scope device array of kScratchBytes; every
-// GPU that loads the library holds that array until the process exits.  All
+// rewiring).  Their scratch (each beam's row log-sum-exp and best key, and each
+// request's key and survivor buffers) lives in one file-scope device array of
+// kScratchBytes; every GPU that loads the library holds that array until the
+// process exits.  All
 // calls share it, so calls that overlap on the GPU (two streams, two threads)
 // race on it and must be serialised by the caller.  The array keeps the last
 // call's contents; everything a call reads from it is written by that same
 // call first.  Device faults (NaN scores, out-of-vocabulary mask tokens) are
 // skipped as in the context path but not reported -- use the context path
 // (xgr_device_status) to diagnose them.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -29,7 +31,7 @@ namespace xgr {
 
 namespace {
 
-constexpr size_t kScratchBytes = 8u << 20;   // 8 MiB: status word + row LSE + samples
+constexpr size_t kScratchBytes = 8u << 20;   // 8 MiB: status word + selection scratch
 constexpr size_t kStatusBytes = 256;
 constexpr int kMaxDevices = 64;
 
@@ -79,8 +81,16 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     if (n_requests < 1 || beam_width < 1 || beam_width > 1024 || top_k < beam_width ||
         top_k > 1024 || vocab < 1 || (int64_t)beam_width * vocab >= (1ll << 32))
         return XGR_ERR_SHAPE;
-    const int64_t rows = (int64_t)n_requests * beam_width;
-    if (kStatusBytes + select_scratch_bytes(rows) > kScratchBytes)
+    if (vocab > kSelectMaxVocab) return XGR_ERR_UNIMPLEMENTED;
+    // what the fixed array leaves after the per-row scratch goes to the key
+    // buffer (8 bytes a CSR entry) and the survivors (12 bytes, half as many)
+    const size_t fixed = kStatusBytes + select_scratch_bytes(n_requests, beam_width, 0, 0) + 1024;
+    if (fixed >= kScratchBytes) return XGR_ERR_CAPACITY;
+    const int64_t key_cap = (int64_t)((kScratchBytes - fixed) / ((size_t)n_requests * 14)) & ~31ll;
+    const int64_t surv_cap = key_cap / 2;
+    const int64_t need = std::max<int64_t>({(int64_t)vocab, 8ll * beam_width, 4096});
+    if (key_cap < need ||
+        kStatusBytes + select_scratch_bytes(n_requests, beam_width, key_cap, surv_cap) > kScratchBytes)
         return XGR_ERR_CAPACITY;   // beyond the fixed 8 MiB scratch
     void *scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return XGR_ERR_CUDA;
@@ -98,8 +108,8 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     a.bits = d_bits;
     a.row_ptr = d_row_ptr;
     a.cols = d_cols;
-    a.row_lse = reinterpret_cast<float *>(sc + kStatusBytes);
-    a.sample = reinterpret_cast<uint64_t *>(sc + kStatusBytes + select_sample_offset(rows));
+    a.max_entries = key_cap;
+    select_scratch_carve(sc + kStatusBytes, n_requests, beam_width, key_cap, surv_cap, a);
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum_out;

@@ -16,6 +16,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMinChunk = 256;     // fewest keys per split-K work item
+constexpr int64_t kSurvCap = 65536;   // selection survivors per request (more: exact path over the keys)
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -44,9 +45,10 @@ struct Layout {
     size_t kstore, vstore, pool_k, pool_v;
     size_t trie_ptr, trie_tok, root_bits;
     int64_t trie_level_cap;    // ints per level in each of trie_ptr / trie_tok
-    size_t mask_row_ptr, mask_cols;
+    size_t mask_row_ptr, mask_cols, mask_sync;
     int64_t mask_cap;
     size_t select_scratch;
+    int64_t key_cap, surv_cap;   // selection keys / survivors per request
     size_t part_o, part_ml;
     int slots;
     size_t plan_items[2], plan_members[2], plan_nslots[2];
@@ -80,13 +82,17 @@ void make_layout(const xgr_config &c, Layout &L) {
         L.root_bits = take(4 * ((c.vocab + 31) / 32));
         L.mask_cap = B * BW * (int64_t)fanout_cap(c);
         L.mask_row_ptr = take(4 * (B * BW + 1));
+        L.mask_sync = take(8 * (B + 1));   // look-back words, then the two ticket words
         L.mask_cols = take(4 * L.mask_cap);
-        L.select_scratch = take(select_scratch_bytes(B * BW));
+        L.key_cap = BW * (int64_t)fanout_cap(c);
+        L.surv_cap = std::min<int64_t>(L.key_cap, kSurvCap);
+        L.select_scratch = take(select_scratch_bytes((int)B, (int)BW, L.key_cap, L.surv_cap));
     } else {
         L.trie_level_cap = 0;
-        L.trie_ptr = L.trie_tok = L.root_bits = L.mask_row_ptr = L.mask_cols = 0;
+        L.trie_ptr = L.trie_tok = L.root_bits = L.mask_row_ptr = L.mask_cols = L.mask_sync = 0;
         L.select_scratch = 0;
         L.mask_cap = 0;
+        L.key_cap = L.surv_cap = 0;
     }
     L.slots = partial_slots(c);
     L.part_o = take(4 * (size_t)L.slots * partial_rows(c) * D);
@@ -118,6 +124,7 @@ xgr_status check_config(const xgr_config *c) {
         if (c->top_k < c->beam_width || c->top_k > 1024) return XGR_ERR_SHAPE;
         if ((int64_t)c->beam_width * c->vocab >= (1ll << 32)) return XGR_ERR_SHAPE;
         if (c->max_items < 1) return XGR_ERR_SHAPE;
+        if (c->vocab > kSelectMaxVocab) return XGR_ERR_UNIMPLEMENTED;
     }
     if ((int64_t)c->max_requests * c->beam_width * c->n_q_heads >= (1ll << 31)) return XGR_ERR_SHAPE;
     return XGR_OK;
@@ -136,6 +143,7 @@ struct xgr_ctx {
     BeamState st;
     TrieView trie;
     bool has_trie = false;
+    int level_fanout[kMaxSteps] = {};   // most children of one node of each trie level
     // prompt KV store bookkeeping (host)
     int64_t kv_used = 0;
     std::vector<int64_t> sid_off, sid_len;
@@ -267,7 +275,8 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
                     it.row_begin = (int32_t)(t * R);
                     it.n_rows = (int32_t)std::min<int64_t>(R, rows - t * R);
                     it.slot = (int32_t)(slot0 + sp);
-                    it.flags = final_seg ? 1 : 0;
+                    it.flags = (final_seg ? 1 : 0) | (sg.members.size() == 1 ? 2 : 0);
+                    it.r0 = sg.members[0];
                     dst.push_back(it);
                 }
         for (int r : sg.members) nslots[r] = (int32_t)(slot0 + splits);
@@ -440,6 +449,7 @@ xgr_status xgr_build_trie(xgr_ctx *c, const int32_t *h_items, int64_t n_items, i
             return XGR_ERR_CUDA;
         tv.ptr[l] = dptr;
         tv.tok[l] = dtok;
+        c->level_fanout[l] = max_children;
         tv.n_nodes[l + 1] = (int32_t)tok.size();
         if (l == 0) {
             std::vector<uint32_t> bits((cf.vocab + 31) / 32, 0u);
@@ -521,6 +531,7 @@ xgr_status xgr_begin(xgr_ctx *c, int32_t n_requests, xgr_stream_t stream) {
     }
     c->dims.B = n_requests;
     if (launch_begin(c->st, c->dims, c->cfg.max_requests, c->cfg.vocab == 0,
+                     c->cfg.vocab > 0 ? c->at<uint64_t>(c->L.mask_sync) : nullptr,
                      (cudaStream_t)stream) != cudaSuccess)
         return XGR_ERR_CUDA;
     c->begun = true;
@@ -575,7 +586,15 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
         ta.st = c->st;
         ta.Bcap = c->cfg.max_requests;
         ta.step = step;
-        const cudaError_t e = launch_attn_tc(c->tmk, c->tmv, ta, c->n_tc[which], s);
+        // Q tiles of single-request items are one TMA box: D x (query heads of
+        // one kv head) x (128 / G beams) over q viewed as [B*BW][Hq][D]
+        CUtensorMap tmq;
+        if (make_q_tensor_map(&tmq, d_q, (int64_t)c->dims.B * c->cfg.beam_width, c->cfg.n_q_heads,
+                              c->dims.G) != cudaSuccess) {
+            debug_log("decode_step: q tensor map failed");
+            return XGR_ERR_CUDA;
+        }
+        const cudaError_t e = launch_attn_tc(c->tmk, c->tmv, tmq, ta, c->n_tc[which], s);
         if (e != cudaSuccess) {
             debug_log("decode_step: tensor-core launch failed: %s", cudaGetErrorString(e));
             return XGR_ERR_CUDA;
@@ -633,7 +652,12 @@ xgr_status xgr_build_mask(xgr_ctx *c, int32_t step, xgr_mask *out, xgr_stream_t 
     ma.row_ptr = c->at<int32_t>(c->L.mask_row_ptr);
     ma.cols = c->at<int32_t>(c->L.mask_cols);
     ma.cap = c->L.mask_cap;
-    if (launch_build_mask(ma, (cudaStream_t)stream) != cudaSuccess) return XGR_ERR_CUDA;
+    ma.flags = c->at<uint64_t>(c->L.mask_sync);
+    ma.ticket = reinterpret_cast<uint32_t *>(ma.flags + c->cfg.max_requests);
+    // CTAs per request sharing the copy: about 16K entries each
+    const int64_t entries = (int64_t)c->cfg.beam_width * c->level_fanout[step];
+    const int parts = (int)std::min<int64_t>(16, std::max<int64_t>(1, (entries + 16383) / 16384));
+    if (launch_build_mask(ma, parts, (cudaStream_t)stream) != cudaSuccess) return XGR_ERR_CUDA;
     out->kind = XGR_MASK_CSR;
     out->row_ptr = ma.row_ptr;
     out->cols = ma.cols;
@@ -670,10 +694,9 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.bits = mask->bits;
     a.row_ptr = mask->row_ptr;
     a.cols = mask->cols;
-    a.row_lse = c->at<float>(c->L.select_scratch);
-    a.sample = reinterpret_cast<uint64_t *>(
-        c->at<uint8_t>(c->L.select_scratch) +
-        select_sample_offset((int64_t)c->cfg.max_requests * c->cfg.beam_width));
+    a.max_entries = step == 0 ? c->cfg.vocab : (int64_t)c->cfg.beam_width * c->level_fanout[step];
+    select_scratch_carve(c->at<uint8_t>(c->L.select_scratch), c->cfg.max_requests,
+                         c->cfg.beam_width, c->L.key_cap, c->L.surv_cap, a);
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum;

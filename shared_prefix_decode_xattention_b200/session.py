@@ -56,6 +56,13 @@ class Session:
     def build_mask(self, step, stream=None) -> xgr.xgr_mask:
         return xgr.xgr_build_mask(self.ctx, step, stream)
 
+    def mask_entries(self, mask: xgr.xgr_mask) -> int:
+        """CSR entries of a mask built in this workspace (reads row_ptr[n_rows]; synchronises)."""
+        import torch
+        off = mask.row_ptr + 4 * mask.n_rows - self.workspace.data_ptr()
+        assert 0 <= off and off + 4 <= self.nbytes
+        return int(self.workspace[off:off + 4].view(torch.int32).item())
+
     def beam_select(self, step, scores, flags, mask, parent, token, cum, n_out, stream=None):
         xgr.xgr_beam_select(self.ctx, step, scores, flags, mask, parent, token, cum, n_out, stream)
 
