@@ -213,6 +213,9 @@ __device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it,
 
 // 10 warps: the register file is split over the 4 schedulers (16K registers each) and 3 of
 // the 10 warps share one, so a thread may use at most 168 registers
+// NT: the most Unshared tokens (step + 1) the prologue handles; one instance per
+// step range keeps the unrolled prologue (and the instruction footprint) small
+template <int NT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const __grid_constant__ CUtensorMap tmq, TcArgs a) {
@@ -429,14 +432,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int s_now = a.step;
         const int n_tok = s_now + 1;
         // the beam's ancestry slots are read together with n_live, while Q is in flight
-        int slot[kMaxSteps];
+        int slot[NT];
         if (final_item) {
 #pragma unroll
-            for (int i = 0; i < kMaxSteps; ++i)
+            for (int i = 0; i < NT; ++i)
                 slot[i] = (ri.valid && i < s_now) ? a.st.anc[beam_row * dm.S + i] : ri.b;
         }
         const bool live = ri.valid && ri.b < a.n_live[ri.r];
-        float sc[kMaxSteps];   // scaled scores of the beam's own tokens (final items)
+        float sc[NT];   // scaled scores of the beam's own tokens (final items)
         if (final_item) {
             // ---- Unshared stage first (the item covers its requests' only KV
             // segment): the beam's own tokens of steps 0..s, read through its
@@ -446,9 +449,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // also appends this step's k/v (already in registers) at Unshared slot
             // (s, b).
             const bool appender = live && ri.hg == 0;
-            const __nv_bfloat16 *kp[kMaxSteps], *vp[kMaxSteps];
+            const __nv_bfloat16 *kp[NT], *vp[NT];
 #pragma unroll
-            for (int i = 0; i < kMaxSteps; ++i) {
+            for (int i = 0; i < NT; ++i) {
                 kp[i] = vp[i] = nullptr;
                 if (!live || i >= n_tok) continue;
                 if (slot[i] < 0 || slot[i] >= dm.BW) {
@@ -478,9 +481,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (q_tma)   // the prologue reads Q from shared memory
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort));
-            float *xd = reinterpret_cast<float *>(base + kOffP);   // [2 halves][kMaxSteps][128]
+            float *xd = reinterpret_cast<float *>(base + kOffP);   // [2 halves][NT][128]
 #pragma unroll
-            for (int i = 0; i < kMaxSteps; i += 2) {
+            for (int i = 0; i < NT; i += 2) {
                 if (i >= n_tok) break;
                 if (i > 0) {
 #pragma unroll
@@ -512,14 +515,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         acc1 = fmaf(qf[e], f1[e], acc1);
                     }
                 }
-                xd[(half * kMaxSteps + i) * 128 + row] = acc0;
-                if (i + 1 < n_tok) xd[(half * kMaxSteps + i + 1) * 128 + row] = acc1;
+                xd[(half * NT + i) * 128 + row] = acc0;
+                if (i + 1 < n_tok) xd[(half * NT + i + 1) * 128 + row] = acc1;
             }
             named_sync(1, kSoftmaxThreads);
             float m_u = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < kMaxSteps; ++i) {
-                sc[i] = (i < n_tok && kp[i]) ? (xd[i * 128 + row] + xd[(kMaxSteps + i) * 128 + row]) * cscale
+            for (int i = 0; i < NT; ++i) {
+                sc[i] = (i < n_tok && kp[i]) ? (xd[i * 128 + row] + xd[(NT + i) * 128 + row]) * cscale
                                              : -INFINITY;
                 m_u = fmaxf(m_u, sc[i]);
             }
@@ -529,7 +532,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int e = 0; e < 64; ++e) o[e] = 0.f;
 #pragma unroll
-            for (int i = 0; i < kMaxSteps; ++i) {
+            for (int i = 0; i < NT; ++i) {
                 if (i >= n_tok || sc[i] == -INFINITY) continue;
                 const float pw = ex2(sc[i] - m_u);
                 l_u += pw;
@@ -566,20 +569,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok) break;
             fence_after_sync();
             const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
-            // pass 1: the row max over the chunk's 128 scores
+            // the chunk's 128 scores in one TMEM read; S_j's buffer is then free for S_{j+2}
+            float sv[128];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) tmem_ld32(tmem + lane_base + s_col + 32 * q2, sv + 32 * q2);
+            tmem_wait_ld();
+            fence_before_sync();
+            mbar_arrive(bar(B_SFREE + half));
+            if (nvalid < kBlockN) {   // the range's last chunk: keys past its end do not count
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= nvalid) sv[c] = -INFINITY;
+            }
             float mxp[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+            for (int e = 0; e < 8; ++e) mxp[e] = sv[e];
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float sv[64];
-                tmem_ld32(tmem + lane_base + s_col + 64 * q2, sv);
-                tmem_ld32(tmem + lane_base + s_col + 64 * q2 + 32, sv + 32);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (64 * q2 + c < nvalid) mxp[c & 7] = fmaxf(mxp[c & 7], sv[c]);
-            }
+            for (int c = 8; c < 128; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], sv[c]);
             const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
                                    fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * cscale;
             float alpha = 1.f;
@@ -594,10 +600,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + half), (jj - 1) & 1, abort));
                 if (!ok) break;
             }
-            if (__any_sync(0xffffffffu, rescale)) {
+            // exponentials, row sum and P (bf16), 8 columns (16 bytes) at a time
+            const float neg_m = -m_used;
+            float sp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = ex2(fmaf(sv[8 * c + 2 * e], cscale, neg_m));
+                    const float p1 = ex2(fmaf(sv[8 * c + 2 * e + 1], cscale, neg_m));
+                    sp[(2 * e) & 7] += p0;
+                    sp[(2 * e + 1) & 7] += p1;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    w4[e] = *reinterpret_cast<uint32_t *>(&h2);
+                }
+                *reinterpret_cast<uint4 *>(pb + sw128_off(row, c)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            if (__any_sync(0xffffffffu, rescale)) {   // O_half *= alpha before P_j V_j adds in
                 fence_after_sync();
                 const float f = rescale ? alpha : 1.f;
-#pragma unroll
+#pragma unroll 1
                 for (int q2 = 0; q2 < 4; ++q2) {
                     float o[32];
                     tmem_ld32(tmem + lane_base + o_col + q2 * 32, o);
@@ -607,40 +632,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_st32(tmem + lane_base + o_col + q2 * 32, o);
                 }
                 tmem_wait_st();
-            }
-            // pass 2: exponentials, row sum and P (bf16), 8 columns (16 bytes) at a time
-            const float neg_m = -m_used;
-            float sp[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float sv[64];
-                tmem_ld32(tmem + lane_base + s_col + 64 * q2, sv);
-                tmem_ld32(tmem + lane_base + s_col + 64 * q2 + 32, sv + 32);
-                tmem_wait_ld();
-                if (q2 == 1) {   // S_j fully read: its buffer may take S_{j+2}
-                    fence_before_sync();
-                    mbar_arrive(bar(B_SFREE + half));
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int cc = 64 * q2 + 8 * c + 2 * e;
-                        const float p0 =
-                            cc < nvalid ? ex2(fmaf(sv[8 * c + 2 * e], cscale, neg_m)) : 0.f;
-                        const float p1 =
-                            cc + 1 < nvalid ? ex2(fmaf(sv[8 * c + 2 * e + 1], cscale, neg_m)) : 0.f;
-                        sp[(2 * e) & 7] += p0;
-                        sp[(2 * e + 1) & 7] += p1;
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                        w4[e] = *reinterpret_cast<uint32_t *>(&h2);
-                    }
-                    *reinterpret_cast<uint4 *>(pb + sw128_off(row, 8 * q2 + c)) =
-                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
             }
             l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
             fence_async_smem();
@@ -666,7 +657,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
             const float l_row = l0 * f0 + l1 * f1;
             if (ok) {
-#pragma unroll
+#pragma unroll 1
                 for (int q2 = 0; q2 < 2; ++q2) {
                     float o[32], o1[32];
                     tmem_ld32(tmem + lane_base + 256 + col0 + 32 * q2, o);
@@ -764,17 +755,19 @@ cudaError_t make_q_tensor_map(CUtensorMap *map, const void *q, int64_t beam_rows
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
-                           const TcArgs &a, int n_items, cudaStream_t st) {
-    if (n_items <= 0) return cudaSuccess;
+namespace {
+
+template <int NT>
+cudaError_t launch_nt(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+                      const TcArgs &a, int n_items, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
+        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<NT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
+        e = cudaFuncGetAttributes(&fa, attn_tc_kernel<NT>);
         if (e != cudaSuccess) return e;
         if (fa.maxThreadsPerBlock < kTcThreads) {
             debug_log("attn_tc: %d registers/thread allow only %d threads per block", fa.numRegs,
@@ -783,8 +776,20 @@ cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const
         }
         attr = true;
     }
-    attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
+    attn_tc_kernel<NT><<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+                           const TcArgs &a, int n_items, cudaStream_t st) {
+    if (n_items <= 0) return cudaSuccess;
+    const int n_tok = a.step + 1;   // Unshared tokens of a beam at this step
+    if (n_tok <= 2) return launch_nt<2>(tmk, tmv, tmq, a, n_items, st);
+    if (n_tok <= 4) return launch_nt<4>(tmk, tmv, tmq, a, n_items, st);
+    if (n_tok <= kMaxSteps) return launch_nt<kMaxSteps>(tmk, tmv, tmq, a, n_items, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace xgr

@@ -117,6 +117,7 @@ struct SelectArgs {
     int32_t *surv_e;            // [B][surv_cap] their entry
     int64_t surv_cap;
     int pick_parts;             // set by the launcher
+    int num_sms;                // SMs of the device (sizes the persistent row kernel)
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
     float *cum_out;

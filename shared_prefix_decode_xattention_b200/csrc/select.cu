@@ -43,7 +43,6 @@ namespace xgr {
 namespace {
 
 constexpr int kDenseThreads = 1024;
-constexpr int kRowThreads = 256;
 constexpr int kPickThreads = 512;
 constexpr int kPickKeys = 4096;    // keys one pick CTA filters per slice (8 per thread)
 constexpr int kSmemSurv = 4096;    // survivors selected in shared memory
@@ -53,16 +52,6 @@ __device__ __forceinline__ float ex2f(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// (m, s) pairs: s = sum of 2^((x - m) log2 e) over the values seen
-__device__ __forceinline__ void lse_combine(float &m, float &s, float m2, float s2) {
-    if (m2 > m) {
-        s = s * ex2f((m - m2) * kLog2e) + s2;
-        m = m2;
-    } else if (m2 != -INFINITY) {
-        s += s2 * ex2f((m2 - m) * kLog2e);
-    }
 }
 
 // key of (beam b, token t): one fp32 add of the beam's cumulative score and
@@ -152,102 +141,189 @@ __device__ int block_exclusive_scan_int(int v, int *warp_tot, int *total) {
     return before + incl - v;
 }
 
-// log-sum-exp of the values x[i], i = threadIdx.x (mod blockDim.x), i < n, in
-// shared memory; reports NaN; red holds 64 floats
-__device__ float block_lse(const float *x, int n, float *red, int32_t *status) {
-    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nw = blockDim.x / 32;
-    float m = -INFINITY, s = 0.f;
+// A set of threads that reduce together: the whole block (barrier 0) or a
+// group of warps with its own named barrier.
+struct Group {
+    int bar, n, t;   // barrier id (0: __syncthreads), threads, this thread's index in the group
+    __device__ __forceinline__ void sync() const {
+        if (bar == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(n) : "memory");
+    }
+};
+__device__ __forceinline__ Group whole_block() { return Group{0, (int)blockDim.x, (int)threadIdx.x}; }
+
+// log-sum-exp of the values x[i], i < n, in shared memory, over a group: the
+// row max first, then the sum of exponentials, each reduced without
+// branches; reports NaN.  red: 33 floats of shared memory for the group.
+__device__ float group_lse(const float *x, int n, float *red, int32_t *status, const Group &g) {
+    const int lane = g.t % 32, w = g.t / 32, nw = g.n / 32;
+    float m = -INFINITY;
     bool nan = false;
-    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
-        float v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * blockDim.x;
-            v[u] = i < n ? x[i] : -INFINITY;
-            nan |= isnan(v[u]);
-        }
-        const float cm = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-        if (cm > m) {
-            s *= ex2f((m - cm) * kLog2e);
-            m = cm;
-        }
-        if (cm != -INFINITY)
-            s += (ex2f((v[0] - m) * kLog2e) + ex2f((v[1] - m) * kLog2e)) +
-                 (ex2f((v[2] - m) * kLog2e) + ex2f((v[3] - m) * kLog2e));
+    for (int i = g.t; i < n; i += g.n) {
+        const float v = x[i];
+        nan |= isnan(v);
+        m = fmaxf(m, v);
     }
     if (nan) set_status(status, XGR_DEV_NAN);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_combine(m, s, m2, s2);
-    }
-    if (lane == 0) {
-        red[warp] = m;
-        red[32 + warp] = s;
-    }
-    __syncthreads();
+    m = warp_max(m);
+    if (lane == 0) red[w] = m;
+    g.sync();
     m = red[0];
-    s = red[32];
-    for (int w = 1; w < nw; ++w) lse_combine(m, s, red[w], red[32 + w]);
-    __syncthreads();
+    for (int k = 1; k < nw; ++k) m = fmaxf(m, red[k]);
+    g.sync();   // red is reused
+    float s = 0.f;
+    if (m != -INFINITY) {
+        const float mk = m * kLog2e;
+        for (int i = g.t; i < n; i += g.n) s += ex2f(fmaf(x[i], kLog2e, -mk));
+    }
+    s = warp_sum(s);
+    if (lane == 0) red[w] = s;
+    g.sync();
+    s = red[0];
+    for (int k = 1; k < nw; ++k) s += red[k];
+    g.sync();
     return m + logf(s);
+}
+__device__ float block_lse(const float *x, int n, float *red, int32_t *status) {
+    return group_lse(x, n, red, status, whole_block());
+}
+__device__ uint64_t group_min_u64(uint64_t v, uint64_t *red, const Group &g) {
+    const int lane = g.t % 32, w = g.t / 32, nw = g.n / 32;
+    v = warp_min_u64(v);
+    if (lane == 0) red[w] = v;
+    g.sync();
+    v = red[0];
+    for (int k = 1; k < nw; ++k) v = red[k] < v ? red[k] : v;
+    g.sync();
+    return v;
+}
+
+// One radix pass's bucket search over the digit of `width` bits at `shift`:
+// the bin holding the k_rem-th key, by a one-warp scan of the 256-bin
+// histogram.  Returns whether the digit is resolved exactly (the bin's keys are
+// all taken); updates prefix, mask and k_rem.
+__device__ __forceinline__ bool radix_bucket(const int *hist, int *sc, int shift, int width, int &k_rem,
+                                             uint64_t &prefix, uint64_t &mask) {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int h[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            h[i] = hist[lane * 8 + i];
+            sum += h[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int acc = incl - sum;   // keys in the bins before this lane's 8
+        // the lane whose range crosses k_rem owns the bucket
+        if (acc < k_rem && acc + sum >= k_rem) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (acc + h[i] >= k_rem) {
+                    sc[0] = lane * 8 + i;
+                    sc[1] = h[i] - (k_rem - acc);   // 0 <=> the whole bucket is taken
+                    sc[2] = k_rem - acc;
+                    break;
+                }
+                acc += h[i];
+            }
+        }
+    }
+    __syncthreads();
+    const int d = sc[0], surplus = sc[1];
+    k_rem = sc[2];
+    prefix |= (uint64_t)d << shift;
+    mask |= ((1ull << width) - 1ull) << shift;
+    __syncthreads();
+    return surplus == 0;
+}
+
+// add one key (if `in`) to its bin; lanes whose keys share a bin add them with
+// one atomic (keys cluster in few bins in the leading digits).  All lanes call it.
+__device__ __forceinline__ void hist_add(int *hist, bool in, uint64_t key, int shift) {
+    const int bin = in ? (int)((key >> shift) & 255) : 256;
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (in && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
 }
 
 // Exact block-wide radix select over E candidates given by `cand(e, key)`
 // (false for a non-candidate).  Keys are unique.  On return exactly `want`
 // candidates satisfy (key & mask) <= prefix (want <= number of candidates).
-// hist: 256 ints of shared memory; sc: 3 shared ints.  The bucket holding the
-// want-th key is found by a one-warp scan of the 256 bins.
+// hist: 256 ints of shared memory; sc: 3 shared ints.
 template <class Cand>
 __device__ void radix_select(const Cand &cand, int64_t E, int want, int *hist, int *sc,
                              uint64_t &prefix, uint64_t &mask) {
     prefix = 0;
     mask = 0;
     int k_rem = want;
+    const int64_t E_up = (E + blockDim.x - 1) / blockDim.x * blockDim.x;   // same trip count for all
     for (int shift = 56; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        for (int64_t e = threadIdx.x; e < E; e += blockDim.x) {
-            uint64_t key;
-            if (cand(e, key) && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        for (int64_t e = threadIdx.x; e < E_up; e += blockDim.x) {
+            uint64_t key = 0;
+            const bool in = e < E && cand(e, key) && (key & mask) == prefix;
+            hist_add(hist, in, key, shift);
         }
         __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            int h[8], sum = 0;
+        if (radix_bucket(hist, sc, shift, 8, k_rem, prefix, mask)) break;
+    }
+}
+
+// The same over keys held in registers (KPT per thread, kNoKey for none) plus
+// an optional tail of n_tail keys in shared memory.  The digits start at the
+// highest bit where the smallest and largest key differ (the bits above are
+// common to all keys), so the first histogram already spreads the keys over
+// many bins and plain shared-memory atomics do not pile onto one counter.
+// red: 32 u64 of shared memory.
+template <int KPT>
+__device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist, int *sc,
+                                  uint64_t *red, uint64_t &prefix, uint64_t &mask,
+                                  const uint64_t *tail = nullptr, int n_tail = 0) {
+    uint64_t lo = kNoKey, hi = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                h[i] = hist[lane * 8 + i];
-                sum += h[i];
-            }
-            int incl = sum;
+    for (int u = 0; u < KPT; ++u)
+        if (k[u] != kNoKey) {
+            lo = k[u] < lo ? k[u] : lo;
+            hi = k[u] > hi ? k[u] : hi;
+        }
+    for (int i = threadIdx.x; i < n_tail; i += blockDim.x)
+        if (tail[i] != kNoKey) {
+            lo = tail[i] < lo ? tail[i] : lo;
+            hi = tail[i] > hi ? tail[i] : hi;
+        }
+    lo = block_min_u64(lo, red);
+    hi = block_max_u64(hi, red);
+    const uint64_t diff = lo ^ hi;
+    if (diff == 0) {   // one distinct key (keys are unique: one candidate)
+        prefix = lo;
+        mask = ~0ull;
+        return;
+    }
+    // digits of 8 bits from the highest differing bit down (the last may be narrower)
+    int pos = 64 - __clzll((long long)diff);   // bits [pos, 64) are common to every key
+    mask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
+    prefix = lo & mask;
+    int k_rem = want;
+    while (pos > 0) {
+        const int shift = pos > 8 ? pos - 8 : 0, width = pos - shift;
+        const uint64_t dmask = (1ull << width) - 1ull;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            int acc = incl - sum;   // keys in the bins before this lane's 8
-            // the lane whose range crosses k_rem owns the bucket
-            if (acc < k_rem && acc + sum >= k_rem) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (acc + h[i] >= k_rem) {
-                        sc[0] = lane * 8 + i;
-                        sc[1] = h[i] - (k_rem - acc);   // 0 <=> the whole bucket is taken
-                        sc[2] = k_rem - acc;
-                        break;
-                    }
-                    acc += h[i];
-                }
-            }
+        for (int u = 0; u < KPT; ++u)
+            if (k[u] != kNoKey && (k[u] & mask) == prefix) atomicAdd(&hist[(k[u] >> shift) & dmask], 1);
+        for (int i = threadIdx.x; i < n_tail; i += blockDim.x) {
+            const uint64_t key = tail[i];
+            if (key != kNoKey && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
         }
         __syncthreads();
-        const int d = sc[0], surplus = sc[1];
-        k_rem = sc[2];
-        prefix |= (uint64_t)d << shift;
-        mask |= 0xFFull << shift;
-        __syncthreads();
-        if (surplus == 0) break;
+        if (radix_bucket(hist, sc, shift, width, k_rem, prefix, mask)) break;
+        pos = shift;
     }
 }
 
@@ -412,6 +488,22 @@ __device__ void collect(const Cand &cand, int64_t E, uint64_t prefix, uint64_t m
     }
 }
 
+// the same for keys held in registers (KPT per thread; entry(u) names key u's entry)
+template <int KPT, class Entry>
+__device__ void collect_regs(const uint64_t (&k)[KPT], uint64_t prefix, uint64_t mask, int BW,
+                             const Entry &entry, const FinishSmem &f) {
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+        if (k[u] != kNoKey && (k[u] & mask) <= prefix) {
+            const int pos = atomicAdd(f.cnt, 1);
+            if (pos < BW) {
+                f.win_k[pos] = k[u];
+                f.win_e[pos] = entry(u);
+            }
+        }
+    }
+}
+
 // Rank the n_win winners (unique keys; a winner's rank is its number of better
 // winners, counted by one warp per winner), write the outputs in rank order
 // and, when a.rewire, rewrite the request's beam state in place.  The caller
@@ -421,6 +513,26 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
     const int BW = dm.BW, S = dm.S, V = dm.V;
     const int64_t rb = (int64_t)r * BW;
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32, nwarps = blockDim.x / 32;
+    const int s = a.step;
+    // sparse rewiring: each winner's trie child and the check of its token load
+    // while the winners are ranked (winners i = threadIdx.x + u * blockDim.x)
+    constexpr int kWinPerThread = 2;   // BW <= 1024 <= 2 * blockDim.x
+    int child_c[kWinPerThread], child_t[kWinPerThread];
+#pragma unroll
+    for (int u = 0; u < kWinPerThread; ++u) {
+        const int i = threadIdx.x + u * blockDim.x;
+        child_c[u] = -1;
+        child_t[u] = -1;
+        if (!a.rewire || a.dense || i >= n_win) continue;
+        const uint32_t lo = (uint32_t)f.win_k[i];
+        const int p = (int)(lo / (uint32_t)V);
+        if (f.cb[p] < 0) continue;
+        const int c = f.cb[p] + (f.win_e[i] - f.rp[p]);
+        if (c < f.ce[p]) {
+            child_c[u] = c;
+            child_t[u] = a.trie.tok[s][c];
+        }
+    }
     for (int i = warp; i < n_win; i += nwarps) {
         const uint64_t k = f.win_k[i];
         int c = 0;
@@ -428,8 +540,13 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
         c = warp_sum_int(c);
         if (lane == 0) f.rank[i] = c;
     }
-    __syncthreads();
-    const int s = a.step;
+#pragma unroll
+    for (int u = 0; u < kWinPerThread; ++u) {   // the checked child of winner i, in rank
+        const int i = threadIdx.x + u * blockDim.x;
+        if (i < n_win && !a.dense && a.rewire)
+            f.win_e[i] = (child_c[u] >= 0 && child_t[u] == (int)((uint32_t)f.win_k[i] % (uint32_t)V)) ? child_c[u] : -1;
+    }
+    __syncthreads();   // every rank is written
     for (int i = threadIdx.x; i < BW; i += blockDim.x) {
         if (i < n_win) {
             const int nb = f.rank[i];
@@ -468,11 +585,10 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
                 } else {
                     child = find_child(a.trie, s, node, t);
                 }
-            } else if (f.cb[p] >= 0) {
+            } else {
                 // the mask row of parent p lists its children in trie order, so
-                // the entry index locates the child directly
-                const int c = f.cb[p] + (f.win_e[i] - f.rp[p]);
-                if (c < f.ce[p] && a.trie.tok[s][c] == t) child = c;
+                // the entry index located the child (checked above)
+                child = f.win_e[i];
             }
             if (child < 0) set_status(a.status, XGR_DEV_MASK);
             a.st.node[o] = child;
@@ -509,8 +625,9 @@ size_t dense_smem(const Dims &dm) {
 __global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bar_mem;
-    __shared__ float red_f[64];
+    __shared__ float red_f[72];
     __shared__ int red_i[32];
+    __shared__ uint64_t red_k[32];
     __shared__ int hist[256];
     __shared__ int sc[4];
     const Dims dm = a.dims;
@@ -583,101 +700,190 @@ __global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectAr
     DenseCand cand{x, bits, cum, lse, V, a.logits, a.status};
     const int64_t E = n > 0 ? V : 0;
     uint64_t prefix = ~0ull, mask = 0;
-    if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
-    collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    if (V <= 8 * kDenseThreads) {   // every key computed once, held in registers
+        uint64_t kr[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = tid + u * kDenseThreads;
+            uint64_t key = kNoKey;
+            kr[u] = (t < E && cand(t, key)) ? key : kNoKey;
+        }
+        if (want < total) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask);
+        collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kDenseThreads; }, f);
+    } else {
+        if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
+        collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    }
     __syncthreads();
     finish_request(a, r, min(*f.cnt, want), f);
 }
 
 // ------------------------------------------------------------------ sparse steps
 
-__global__ void __launch_bounds__(kRowThreads) select_rows_kernel(SelectArgs a) {
+// One persistent CTA per SM takes a contiguous block of beam rows.  It reads
+// the metadata of a window of its rows (row pointers, cumulative scores, live
+// counts) in one round trip and the window's CSR tokens -- one contiguous range
+// -- in another (log-prob mode: then the tokens' scores), all into shared
+// memory.  In logits mode the score rows stream through nbuf slots by bulk
+// copies issued nbuf rows ahead, so the HBM traffic overlaps the work on
+// earlier rows.  Four groups of warps work on four rows at a time.  Per row:
+// the log-sum-exp (logits), each entry's key beside its CSR position, the
+// row's best key.
+constexpr int kRowsThreads = 1024;
+constexpr int kRowsGroups = 4;                       // rows in work at once
+constexpr int kRowsGroup = kRowsThreads / kRowsGroups;
+constexpr int kRowsMaxBuf = 8;
+constexpr int kRowsWin = 256;     // rows per metadata window
+constexpr int kRowsTok = 8192;    // CSR entries staged per window (a longer row reads the rest in place)
+
+__host__ __device__ inline size_t rows_fixed_bytes(bool logits) {
+    return (size_t)kRowsTok * 4 * (logits ? 1 : 2) + (size_t)(kRowsWin + 1) * 4 + (size_t)kRowsWin * 12;
+}
+
+__global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs a, int nbuf) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t bar_mem;
-    __shared__ float red_f[64];
-    __shared__ uint64_t red_k[32];
+    __shared__ uint64_t full[kRowsMaxBuf];
+    __shared__ int slot_row[kRowsMaxBuf];   // the row (index in the block) whose copy a slot holds
+    __shared__ float red_f[36 * kRowsGroups];
+    __shared__ uint64_t red_k[8 * kRowsGroups];
+    __shared__ int win_end;
     const Dims dm = a.dims;
-    const int V = dm.V;
-    const int64_t row = blockIdx.x;
-    const int r = (int)(row / dm.BW), b = (int)(row % dm.BW);
-    const int64_t rb = (int64_t)r * dm.BW;
-    const int tid = threadIdx.x;
-    float *x = reinterpret_cast<float *>(smem);
-    const float *xg = a.scores + row * V;
-    const uint32_t bar = smem_u32(&bar_mem);
-    // logits mode needs the whole row (its log-sum-exp); it is staged in shared
-    // memory with one bulk copy while the CSR entries are read
-    const bool stage = a.logits;
-    const bool bulk = stage && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
-    if (tid == 0 && bulk) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
+    const int V = dm.V, BW = dm.BW, tid = threadIdx.x;
+    const int64_t n_rows = (int64_t)dm.B * BW;
+    const int64_t per = (n_rows + gridDim.x - 1) / gridDim.x;
+    const int64_t r0 = (int64_t)blockIdx.x * per, r1 = min(n_rows, r0 + per);
+    const bool stage = a.logits;   // logits: whole rows (their log-sum-exp)
+    const bool bulk = stage && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
+    const size_t xb = stage ? al16((size_t)V * 4) : 0;
+    uint8_t *p = smem + nbuf * xb;
+    int *tok = reinterpret_cast<int *>(p);
+    p += (size_t)kRowsTok * 4;
+    float *val = reinterpret_cast<float *>(p);   // log-prob mode only
+    if (!stage) p += (size_t)kRowsTok * 4;
+    int *rp = reinterpret_cast<int *>(p);        // [kRowsWin + 1]
+    p += (size_t)(kRowsWin + 1) * 4;
+    float *cum_w = reinterpret_cast<float *>(p);  // [kRowsWin]
+    int *nl_w = reinterpret_cast<int *>(cum_w + kRowsWin);   // [kRowsWin] live beams of the row's request
+    int *base_w = nl_w + kRowsWin;                           // [kRowsWin] first entry of the row's request
+    auto x_of = [&](int64_t row) { return reinterpret_cast<float *>(smem + ((row - r0) % nbuf) * xb); };
+    auto issue = [&](int64_t row) {   // one thread: the bulk copy of a row into its slot
+        const uint32_t bar = smem_u32(&full[(row - r0) % nbuf]);
+        reinterpret_cast<volatile int *>(slot_row)[(row - r0) % nbuf] = (int)(row - r0);
         mbar_expect_tx(bar, (uint32_t)V * 4u);
-        bulk_g2s(smem_u32(x), xg, (uint32_t)V * 4u, bar);
+        bulk_g2s(smem_u32(x_of(row)), a.scores + row * V, (uint32_t)V * 4u, bar);
+    };
+    if (tid == 0 && bulk) {
+        for (int k = 0; k < nbuf; ++k) {
+            mbar_init(smem_u32(&full[k]), 1);
+            slot_row[k] = -1;
+        }
+        fence_mbar_init();
     }
-    const int n = a.n_live[r];
-    const int base = a.row_ptr[rb];
-    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
-    const float cum = a.cum[row];
-    if (b == 0 && tid == 0) {   // the pick kernel counts from 0
-        a.surv_cnt[r] = 0;
-        a.ticket[r] = 0;
-    }
-    const bool live = b < n;
-    // the row's entries, up to 4 per thread per batch: tokens first
-    constexpr int U = 4;
-    const int n_e = max(0, end - beg);
-    int tk[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int j = tid + u * kRowThreads;
-        tk[u] = (live && j < n_e) ? a.cols[beg + j] : -1;
-    }
-    if (stage && !bulk)
-        for (int i = tid; i < V; i += kRowThreads) x[i] = xg[i];
-    __syncthreads();
-    if (bulk && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
-    float lse = 0.f;
-    if (stage && live) lse = block_lse(x, V, red_f, a.status);
-    uint64_t *keys = a.keys + (int64_t)r * a.key_cap - base;   // keys[e] for CSR entry e
-    const int64_t kend = (int64_t)base + a.key_cap;
-    uint64_t best = kNoKey;
-    for (int j0 = 0; j0 < n_e; j0 += U * kRowThreads) {
-        if (j0 > 0) {
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int j = j0 + tid + u * kRowThreads;
-                tk[u] = (live && j < n_e) ? a.cols[beg + j] : -1;
+    // Every load of a row's work happens per window, ahead of the rows: a global
+    // load issued behind the bulk traffic waits microseconds.  The first window's
+    // loads even go out before the first bulk copies.
+    for (int64_t w0 = r0; w0 < r1;) {
+        // ---- window metadata: one round trip
+        const int64_t wmax = min(r1, w0 + kRowsWin);
+        for (int64_t row = w0 + tid; row <= wmax; row += kRowsThreads) {
+            rp[row - w0] = a.row_ptr[row];
+            if (row < wmax) {
+                cum_w[row - w0] = a.cum[row];
+                nl_w[row - w0] = a.n_live[row / BW];
+                base_w[row - w0] = a.row_ptr[row / BW * BW];
             }
         }
-        float lv[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int j = j0 + tid + u * kRowThreads;
-            const bool ok = live && j < n_e && tk[u] >= 0 && tk[u] < V;
-            if (live && j < n_e && !ok) set_status(a.status, XGR_DEV_MASK);
-            lv[u] = ok ? (stage ? x[tk[u]] : xg[tk[u]]) : 0.f;
+        __syncthreads();
+        // rows whose entries fit the token area (at least one row)
+        if (tid == 0) {
+            int64_t w1 = w0 + 1;
+            while (w1 < wmax && rp[w1 + 1 - w0] - rp[0] <= kRowsTok) ++w1;
+            win_end = (int)(w1 - w0);
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int j = j0 + tid + u * kRowThreads;
-            if (j >= n_e) continue;
-            uint64_t key = kNoKey;
-            if (live && tk[u] >= 0 && tk[u] < V) {
-                float lp = lv[u];
-                if (a.logits) lp -= lse;
-                uint64_t k2;
-                if (make_key(cum, lp, b, tk[u], V, a.status, k2)) key = k2;
+        __syncthreads();
+        const int64_t w1 = w0 + win_end;
+        const int t0 = rp[0], nt = min(rp[w1 - w0] - t0, kRowsTok);
+        // ---- the window's tokens (one contiguous range), then log-prob scores
+        for (int j = tid; j < nt; j += kRowsThreads) {
+            const int t = a.cols[t0 + j];
+            tok[j] = t;
+            if (!stage) {
+                // entry j's row: the last window row whose first entry is <= j
+                int l = 0, h = (int)(w1 - w0);
+                while (h - l > 1) {
+                    const int m = (l + h) >> 1;
+                    if (rp[m] - t0 <= j) l = m; else h = m;
+                }
+                const int64_t row = w0 + l;
+                val[j] = (t >= 0 && t < V) ? a.scores[row * V + t] : 0.f;
             }
-            const int64_t e = (int64_t)beg + j;
-            if (e >= base && e < kend) keys[e] = key;
-            best = key < best ? key : best;
         }
-    }
-    best = block_min_u64(best, red_k);
-    if (tid == 0) {
-        a.best[row] = best;
-        a.row_lse[row] = lse;
+        __syncthreads();
+        if (w0 == r0 && tid == 0 && bulk)
+            for (int64_t row = r0; row < min(r1, r0 + nbuf); ++row) issue(row);
+        // ---- the window's rows: group g (256 threads, named barrier 1 + g) takes
+        // rows w0 + g, w0 + g + 4, ...; when it is done with a row it starts the
+        // copy of the row nbuf places later into the same slot
+        const Group grp{1 + tid / kRowsGroup, kRowsGroup, tid % kRowsGroup};
+        const int gi = tid / kRowsGroup;
+        for (int64_t row = w0 + gi; row < w1; row += kRowsGroups) {
+            const int r = (int)(row / BW), b = (int)(row % BW);
+            const int i = (int)(row - w0);
+            const bool live = b < nl_w[i];
+            if (b == 0 && grp.t == 0) {   // the pick kernel counts from 0
+                a.surv_cnt[r] = 0;
+                a.ticket[r] = 0;
+            }
+            const float *xg = a.scores + row * V;
+            float *x = x_of(row);
+            if (stage && !bulk) {   // unaligned rows: plain loads into the slot
+                for (int t = grp.t; t < V; t += kRowsGroup) x[t] = xg[t];
+                grp.sync();
+            }
+            if (bulk) {
+                // a slot serves rows nbuf apart, taken by different groups: wait until
+                // this row's copy is the one in flight, then for its bytes
+                const int k = (int)((row - r0) % nbuf);
+                bool ok = false;
+                for (uint32_t it = 0; it < kSpinLimit && !ok; ++it)
+                    ok = reinterpret_cast<volatile int *>(slot_row)[k] == (int)(row - r0);
+                if (!ok || !mbar_wait(smem_u32(&full[k]), (int)((row - r0) / nbuf) & 1, nullptr))
+                    set_status(a.status, XGR_DEV_TIMEOUT);
+            }
+            float lse = 0.f;
+            if (stage && live) lse = group_lse(x, V, red_f + 36 * gi, a.status, grp);
+            const int beg = rp[i], end = rp[i + 1], n_e = max(0, end - beg);
+            uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
+            const int base = base_w[i];
+            const float cum = cum_w[i];
+            uint64_t best = kNoKey;
+            for (int j = grp.t; j < n_e; j += kRowsGroup) {
+                const int e = beg + j, ew = e - t0;   // entry, its place in the window's tokens
+                const bool staged = ew >= 0 && ew < nt;
+                uint64_t key = kNoKey;
+                if (live) {
+                    const int t = staged ? tok[ew] : a.cols[e];
+                    if (t < 0 || t >= V) {
+                        set_status(a.status, XGR_DEV_MASK);
+                    } else {
+                        float lp = stage ? x[t] : (staged ? val[ew] : xg[t]);
+                        if (a.logits) lp -= lse;
+                        uint64_t k2;
+                        if (make_key(cum, lp, b, t, V, a.status, k2)) key = k2;
+                    }
+                }
+                if (e >= base && (int64_t)(e - base) < a.key_cap) keys[e - base] = key;
+                best = key < best ? key : best;
+            }
+            best = group_min_u64(best, red_k + 8 * gi, grp);   // (its barriers end every read of the slot)
+            if (grp.t == 0) {
+                a.best[row] = best;
+                a.row_lse[row] = lse;
+                if (bulk && row + nbuf < r1) issue(row + nbuf);
+            }
+        }
+        w0 = w1;
+        __syncthreads();   // the window's shared metadata is reused
     }
 }
 
@@ -782,10 +988,16 @@ __global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs
     if (fits) {
         // every winner survived tau; T >= BW whenever tau cuts anything
         want = min(BW, T);
-        if (in_smem) {
-            const ListCand<false> cand{sk};
-            if (want < T) radix_select(cand, T, want, hist, sc, prefix, mask);
-            collect(cand, T, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
+        if (in_smem) {   // the survivors' keys in registers, 8 per thread
+            static_assert(kSmemSurv == 8 * kPickThreads, "survivors per thread");
+            uint64_t kr[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = tid + u * kPickThreads;
+                kr[u] = i < T ? sk[i] : kNoKey;
+            }
+            if (want < T) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask);
+            collect_regs(kr, prefix, mask, BW, [&](int u) { return se[tid + u * kPickThreads]; }, f);
         } else if (T <= a.surv_cap) {
             const ListCand<true> cand{sk_g};
             if (want < T) radix_select(cand, T, want, hist, sc, prefix, mask);
@@ -797,6 +1009,115 @@ __global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs
         }
     } else {
         // the key buffer overflowed: exact selection over every candidate
+        ReqCand cand;
+        cand.x = a.scores + rb * dm.V;
+        cand.cols = a.cols + base;
+        cand.rp = f.rp;
+        cand.cum = cum_s;
+        cand.lse = lse_s;
+        cand.status = a.status;
+        cand.n = n;
+        cand.logits = a.logits;
+        cand.V = dm.V;
+        const int total = f.rp[n];
+        want = min(BW, total);
+        if (want < total) radix_select(cand, total, want, hist, sc, prefix, mask);
+        collect(cand, total, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    }
+    __syncthreads();
+    finish_request(a, r, min(*f.cnt, want), f);
+}
+
+// ---- requests of few CSR entries: one CTA each, every key in registers
+
+constexpr int kPickOneThreads = 1024;
+constexpr int kPickOneKpt = 16;          // keys per thread in registers
+constexpr int kPickOneTail = 16384;      // further keys in shared memory
+constexpr int kPickOneMax = kPickOneKpt * kPickOneThreads + kPickOneTail;
+
+size_t pick_one_smem(const Dims &dm) {
+    return (size_t)kPickOneTail * 8 + finish_bytes(dm.BW, dm.BW, dm.S, 0) + al16((size_t)dm.BW * 8);
+}
+
+// One CTA per request: the request's keys go straight into registers and a
+// shared-memory tail (no threshold pass, no survivor buffer), then the exact
+// radix select, ordering, outputs and rewiring.  Requests with more entries
+// select from the key buffer in global memory (or, past the buffer, from the
+// scores), exactly as the multi-CTA pick does.
+__global__ void __launch_bounds__(kPickOneThreads, 1) select_pick_one_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int hist[256];
+    __shared__ int sc[4];
+    __shared__ int red_i[32];
+    __shared__ uint64_t red_k[32];
+    const Dims dm = a.dims;
+    const int BW = dm.BW, r = blockIdx.x, tid = threadIdx.x;
+    const int64_t rb = (int64_t)r * BW;
+    uint64_t *tail = reinterpret_cast<uint64_t *>(smem);
+    uint8_t *fin = smem + (size_t)kPickOneTail * 8;
+    const FinishSmem f = carve_finish(fin, BW, BW, dm.S, 0);
+    float *cum_s = reinterpret_cast<float *>(fin + finish_bytes(BW, BW, dm.S, 0));
+    float *lse_s = cum_s + BW;
+    const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
+    constexpr int kReg = kPickOneKpt * kPickOneThreads;
+    // every load below is independent of the others: one round trip
+    const int n = a.n_live[r];
+    const int base = a.row_ptr[rb];
+    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;   // dead rows' entries hold kNoKey
+    uint64_t kr[kPickOneKpt];
+#pragma unroll
+    for (int u = 0; u < kPickOneKpt; ++u) {
+        const int64_t e = tid + u * kPickOneThreads;
+        kr[u] = e < a.key_cap ? __ldcg(keys + e) : kNoKey;
+    }
+    if (tid == 0) *f.cnt = 0;
+    for (int b = tid; b <= BW; b += kPickOneThreads) f.rp[b] = a.row_ptr[rb + b] - base;
+    if (a.rewire) stage_rows(a, rb, BW, f);
+    const bool in_smem = E <= a.key_cap && E <= kPickOneMax;
+    const int n_tail = in_smem && E > kReg ? (int)(E - kReg) : 0;
+    for (int i = tid; i < n_tail; i += kPickOneThreads) tail[i] = __ldcg(keys + kReg + i);
+    if (E > a.key_cap)
+        for (int b = tid; b < n; b += kPickOneThreads) {
+            cum_s[b] = a.cum[rb + b];
+            lse_s[b] = a.logits ? a.row_lse[rb + b] : 0.f;
+        }
+    __syncthreads();
+    if (a.rewire) stage_children(a, n, f);
+    uint64_t prefix = ~0ull, mask = 0;
+    int want;
+    if (in_smem) {
+        int c = 0;
+#pragma unroll
+        for (int u = 0; u < kPickOneKpt; ++u) {
+            if (tid + u * kPickOneThreads >= E) kr[u] = kNoKey;
+            c += kr[u] != kNoKey;
+        }
+        for (int i = tid; i < n_tail; i += kPickOneThreads) c += tail[i] != kNoKey;
+        const int T = block_sum_int(c, red_i);   // (its barriers also publish the staging)
+        want = min(BW, T);
+        if (want < T) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask, tail, n_tail);
+        collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kPickOneThreads; }, f);
+        for (int i = tid; i < n_tail; i += kPickOneThreads) {
+            const uint64_t key = tail[i];
+            if (key != kNoKey && (key & mask) <= prefix) {
+                const int pos = atomicAdd(f.cnt, 1);
+                if (pos < BW) {
+                    f.win_k[pos] = key;
+                    f.win_e[pos] = kReg + i;
+                }
+            }
+        }
+    } else if (E <= a.key_cap) {
+        __syncthreads();
+        const KeyCand cand{keys, kNoKey};
+        int c = 0;
+        for (int64_t e = tid; e < E; e += kPickOneThreads) c += __ldcg(keys + e) != kNoKey;
+        const int T = block_sum_int(c, red_i);
+        want = min(BW, T);
+        if (want < T) radix_select(cand, E, want, hist, sc, prefix, mask);
+        collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    } else {
+        __syncthreads();
         ReqCand cand;
         cand.x = a.scores + rb * dm.V;
         cand.cols = a.cols + base;
@@ -867,12 +1188,25 @@ cudaError_t launch_beam_select(const SelectArgs &a_in, cudaStream_t s) {
         return cudaGetLastError();
     }
     {
-        const size_t smem = a.logits ? dense_x_bytes(dm.V) : 0;
+        // one persistent CTA per SM, as many row slots as shared memory holds
+        const size_t xb = a.logits ? dense_x_bytes(dm.V) : 0, fixed = rows_fixed_bytes(a.logits);
+        const int nbuf = a.logits ? (int)std::min<size_t>(kRowsMaxBuf, ((210u << 10) - fixed) / xb) : 1;
+        if (nbuf < 1) return cudaErrorInvalidValue;
+        const size_t smem = nbuf * xb + fixed;
         cudaError_t e = ensure_smem(select_rows_kernel, smem);
         if (e != cudaSuccess) return e;
-        select_rows_kernel<<<dm.B * dm.BW, kRowThreads, smem, s>>>(a);
+        const int64_t rows = (int64_t)dm.B * dm.BW;
+        const int grid = (int)std::min<int64_t>(rows, a.num_sms > 0 ? a.num_sms : 148);
+        select_rows_kernel<<<grid, kRowsThreads, smem, s>>>(a, nbuf);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+    }
+    if (std::min<int64_t>(a.max_entries, a.key_cap) <= kPickOneMax) {
+        const size_t smem = pick_one_smem(dm);
+        cudaError_t e = ensure_smem(select_pick_one_kernel, smem);
+        if (e != cudaSuccess) return e;
+        select_pick_one_kernel<<<dm.B, kPickOneThreads, smem, s>>>(a);
+        return cudaGetLastError();
     }
     int64_t parts = (std::min<int64_t>(a.max_entries, a.key_cap) + kPickKeys - 1) / kPickKeys;
     a.pick_parts = (int)std::max<int64_t>(1, std::min<int64_t>(parts, kMaxPickParts));

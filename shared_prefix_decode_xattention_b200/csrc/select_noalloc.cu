@@ -109,6 +109,10 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     a.row_ptr = d_row_ptr;
     a.cols = d_cols;
     a.max_entries = key_cap;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&a.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return XGR_ERR_CUDA;
     select_scratch_carve(sc + kStatusBytes, n_requests, beam_width, key_cap, surv_cap, a);
     a.parent = d_parent;
     a.token = d_token;

@@ -695,6 +695,7 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.row_ptr = mask->row_ptr;
     a.cols = mask->cols;
     a.max_entries = step == 0 ? c->cfg.vocab : (int64_t)c->cfg.beam_width * c->level_fanout[step];
+    a.num_sms = c->num_sms;
     select_scratch_carve(c->at<uint8_t>(c->L.select_scratch), c->cfg.max_requests,
                          c->cfg.beam_width, c->L.key_cap, c->L.surv_cap, a);
     a.parent = d_parent;
