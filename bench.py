@@ -226,6 +226,21 @@ def decode_required_bytes(w, logits_mode, nnz):
     return total
 
 
+def measured_traffic(call: str):
+    """DRAM bytes per launch of a call, from the committed ncu summary
+    (profiles/traffic.json), or None when any of the call's kernel sources has
+    changed since the counters were taken (their SHA-256 no longer matches)."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[call]
+        for rel, sha in rec["sources"].items():
+            if hashlib.sha256(open(os.path.join(ROOT, rel), "rb").read()).hexdigest() != sha:
+                return None
+        return rec["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def graph_kernel_nodes(g) -> int:
     """Kernel nodes of a captured CUDA graph: the library kernels one decode launches."""
     from cuda.bindings import runtime as rt
@@ -453,14 +468,15 @@ def run_gpu(args, w):
         achieved = att_flops / att_avg / 1e12
         roof = {"kernel": "xgr_decode_step (staged attention, steps >= 1)", "bound": "tensor",
                 "achieved": achieved, "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
-                "peak_source": f"bf16_tflops burst {src}", "traffic": None,
+                "peak_source": f"bf16_tflops burst {src}",
+                "traffic": measured_traffic("xgr_decode_step"),
                 "algorithmic_per_launch": att_flops, "launch_ms": att_avg * 1e3,
                 "hbm_gbs_required_bytes": att_bytes / att_avg / 1e9}
     else:
         achieved = sel_bytes / sel_avg / 1e9
         roof = {"kernel": "xgr_beam_select (steps >= 1)", "bound": "hbm", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_source": f"hbm_gbs {src}", "traffic": None,
+                "peak_source": f"hbm_gbs {src}", "traffic": measured_traffic("xgr_beam_select"),
                 "algorithmic_per_launch": sel_bytes, "launch_ms": sel_avg * 1e3}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
