@@ -197,6 +197,17 @@ def algorithmic(w, s, logits_mode, nnz_step):
     return att_bytes, att_flops, sel_bytes
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest value over all ranks (one all-reduce; the value itself with one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def decode_required_bytes(w, logits_mode, nnz):
     """Bytes one decode must move at least: per step, every prompt and suffix
     K/V once, each live beam's earlier Unshared k/v, this step's k/v (read and
@@ -276,6 +287,8 @@ def run_gpu(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device(dev))
 
+    # weak scaling: rank r decodes its own B requests (shard r of the batch)
+    w = workloads.shard_of(w, rank)
     items = workloads.items(w)
     logits_mode = args.scores == "logits"
     flags = xgr.XGR_SCORES_LOGITS if logits_mode else xgr.XGR_SCORES_LOGPROB
@@ -390,11 +403,7 @@ def run_gpu(args, w):
     if world > 1:
         dist.barrier()
     clocks = clk.stop() if clk else None
-    total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), dev)
     n_live = nout.cpu().numpy()
     cands = candidates_per_decode(w) * args.steps * world
     value = cands / (total_ms / 1e3)
@@ -438,11 +447,7 @@ def run_gpu(args, w):
             g_e2e.replay()
             e_e[i].record()
         torch.cuda.synchronize()
-        e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e))
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)), dev)
         e2e = {"value": cands / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
         del g_e2e

@@ -88,89 +88,96 @@ __global__ void __launch_bounds__(kWarps * 32) attn_merge_kernel(MergeArgs a) {
     copy_lane<D>(kn, a.pool_k + s * pool_step + pool_beam + ((int64_t)b * dm.Hkv + g) * D, lane);
     copy_lane<D>(vn, a.pool_v + s * pool_step + pool_beam + ((int64_t)b * dm.Hkv + g) * D, lane);
 
+    // Every load below that does not depend on another goes out at once (the
+    // beam's ancestry slots, then all its k and v rows, and the partials four
+    // slots at a time), so the warp waits a few round trips, not one per token
+    // and per partial.
     float q[G][N];
 #pragma unroll
     for (int hg = 0; hg < G; ++hg) load_lane<D>(a.q + (gid0 + hg) * D, lane, q[hg]);
+    int slot[kMaxSteps];
+#pragma unroll
+    for (int i = 0; i < kMaxSteps; ++i) slot[i] = i < s ? a.st.anc[beam_row * dm.S + i] : b;
 
     // ---- Unshared stage: the beam's own tokens of steps 0..s
     const float scale_log2 = kLog2e * rsqrtf((float)D);
-    float sc[G][kMaxSteps];
-    int n_tok = 0;
-    for (int i = 0; i <= s; ++i) {
-        const __nv_bfloat16 *kp;
-        if (i == s) {
-            kp = kn;
-        } else {
-            const int slot = a.st.anc[beam_row * dm.S + i];
-            if (slot < 0 || slot >= dm.BW) {   // corrupt ancestry: record, skip the token
-                if (lane == 0) set_status(a.st.status, XGR_DEV_INDEX);
+    float kf[kMaxSteps][N], vf[kMaxSteps][N];
+    bool tok_ok[kMaxSteps];
 #pragma unroll
-                for (int hg = 0; hg < G; ++hg) sc[hg][i] = -INFINITY;
-                continue;
-            }
-            kp = a.pool_k + i * pool_step + pool_beam + ((int64_t)slot * dm.Hkv + g) * D;
+    for (int i = 0; i < kMaxSteps; ++i) {
+        tok_ok[i] = i <= s && slot[i] >= 0 && slot[i] < dm.BW;
+        if (i <= s && !tok_ok[i] && lane == 0) set_status(a.st.status, XGR_DEV_INDEX);   // corrupt ancestry
+        const int64_t off = i * pool_step + pool_beam + ((int64_t)slot[i] * dm.Hkv + g) * D;
+        const __nv_bfloat16 *kp = i == s ? kn : a.pool_k + off;
+        const __nv_bfloat16 *vp = i == s ? vn : a.pool_v + off;
+#pragma unroll
+        for (int e = 0; e < N; ++e) kf[i][e] = vf[i][e] = 0.f;
+        if (tok_ok[i]) {
+            load_lane<D>(kp, lane, kf[i]);
+            load_lane<D>(vp, lane, vf[i]);
         }
-        float kf[N];
-        load_lane<D>(kp, lane, kf);
-#pragma unroll
-        for (int hg = 0; hg < G; ++hg) {
-            float t = 0.f;
-#pragma unroll
-            for (int e = 0; e < N; ++e) t += q[hg][e] * kf[e];
-            sc[hg][i] = warp_sum(t) * scale_log2;
-        }
-        ++n_tok;
     }
     float m[G], l[G], o[G][N];
 #pragma unroll
     for (int hg = 0; hg < G; ++hg) {
+        float sc[kMaxSteps];
         m[hg] = -INFINITY;
-        for (int i = 0; i <= s; ++i) m[hg] = fmaxf(m[hg], sc[hg][i]);
+#pragma unroll
+        for (int i = 0; i < kMaxSteps; ++i) {
+            float t = 0.f;
+#pragma unroll
+            for (int e = 0; e < N; ++e) t += q[hg][e] * kf[i][e];
+            sc[i] = tok_ok[i] ? warp_sum(t) * scale_log2 : -INFINITY;
+            m[hg] = fmaxf(m[hg], sc[i]);
+        }
         l[hg] = 0.f;
 #pragma unroll
         for (int e = 0; e < N; ++e) o[hg][e] = 0.f;
-    }
-    for (int i = 0; i <= s; ++i) {
-        const __nv_bfloat16 *vp;
-        if (i == s) {
-            vp = vn;
-        } else {
-            const int slot = a.st.anc[beam_row * dm.S + i];
-            if (slot < 0 || slot >= dm.BW) continue;
-            vp = a.pool_v + i * pool_step + pool_beam + ((int64_t)slot * dm.Hkv + g) * D;
-        }
-        float vf[N];
-        load_lane<D>(vp, lane, vf);
 #pragma unroll
-        for (int hg = 0; hg < G; ++hg) {
-            const float p = exp2f(sc[hg][i] - m[hg]);
+        for (int i = 0; i < kMaxSteps; ++i) {
+            if (!tok_ok[i]) continue;
+            const float p = exp2f(sc[i] - m[hg]);
             l[hg] += p;
 #pragma unroll
-            for (int e = 0; e < N; ++e) o[hg][e] += p * vf[e];
+            for (int e = 0; e < N; ++e) o[hg][e] += p * vf[i][e];
         }
     }
-    (void)n_tok;
 
-    // ---- Merging stage: fold in every Shared-stage partial (online softmax)
-    for (int p = 0; p < n_slots; ++p) {
+    // ---- Merging stage: fold in every Shared-stage partial (online softmax),
+    // loading four slots at a time
+    for (int p0 = 0; p0 < n_slots; p0 += 4) {
+        float2 ml[4][G];
+        float po[4][G][N];
 #pragma unroll
-        for (int hg = 0; hg < G; ++hg) {
-            const int64_t prow = (int64_t)p * a.part.rows + gid0 + hg;
-            const float2 ml = a.part.ml[prow];
-            float po[N];
-            if constexpr (N == 4) {
-                const float4 t = *reinterpret_cast<const float4 *>(a.part.o + prow * D + lane * 4);
-                po[0] = t.x; po[1] = t.y; po[2] = t.z; po[3] = t.w;
-            } else {
-                const float2 t = *reinterpret_cast<const float2 *>(a.part.o + prow * D + lane * 2);
-                po[0] = t.x; po[1] = t.y;
+        for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int hg = 0; hg < G; ++hg) {
+                const int64_t prow = (int64_t)(p0 + u) * a.part.rows + gid0 + hg;
+                const bool in = p0 + u < n_slots;
+                ml[u][hg] = in ? a.part.ml[prow] : make_float2(-INFINITY, 0.f);
+                if constexpr (N == 4) {
+                    const float4 t = in ? *reinterpret_cast<const float4 *>(a.part.o + prow * D + lane * 4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    po[u][hg][0] = t.x; po[u][hg][1] = t.y; po[u][hg][2] = t.z; po[u][hg][3] = t.w;
+                } else {
+                    const float2 t = in ? *reinterpret_cast<const float2 *>(a.part.o + prow * D + lane * 2)
+                                        : make_float2(0.f, 0.f);
+                    po[u][hg][0] = t.x; po[u][hg][1] = t.y;
+                }
             }
-            const float m_new = fmaxf(m[hg], ml.x);
-            const float a1 = exp2f(m[hg] - m_new), a2 = exp2f(ml.x - m_new);
-            l[hg] = l[hg] * a1 + ml.y * a2;
+        }
 #pragma unroll
-            for (int e = 0; e < N; ++e) o[hg][e] = o[hg][e] * a1 + po[e] * a2;
-            m[hg] = m_new;
+        for (int u = 0; u < 4; ++u) {
+            if (p0 + u >= n_slots) break;
+#pragma unroll
+            for (int hg = 0; hg < G; ++hg) {
+                const float m_new = fmaxf(m[hg], ml[u][hg].x);
+                const float a1 = exp2f(m[hg] - m_new), a2 = exp2f(ml[u][hg].x - m_new);
+                l[hg] = l[hg] * a1 + ml[u][hg].y * a2;
+#pragma unroll
+                for (int e = 0; e < N; ++e) o[hg][e] = o[hg][e] * a1 + po[u][hg][e] * a2;
+                m[hg] = m_new;
+            }
         }
     }
 

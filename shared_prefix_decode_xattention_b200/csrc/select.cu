@@ -275,13 +275,17 @@ __device__ void radix_select(const Cand &cand, int64_t E, int want, int *hist, i
 }
 
 // The same over keys held in registers (KPT per thread, kNoKey for none) plus
-// an optional tail of n_tail keys in shared memory.  The digits start at the
-// highest bit where the smallest and largest key differ (the bits above are
-// common to all keys), so the first histogram already spreads the keys over
-// many bins and plain shared-memory atomics do not pile onto one counter.
-// red: 32 u64 of shared memory.
+// an optional tail of n_tail keys in shared memory, with 11-bit digits (2048
+// bins, bucket found by a block-wide scan: half the passes of 8-bit digits).
+// The digits start at the highest bit where the smallest and largest key
+// differ (the bits above are common to all keys), so the first histogram
+// already spreads the keys over many bins and the shared-memory atomics do not
+// pile onto a few counters.  hist: kWideBins ints; scan_w: 32 ints; red: 32
+// u64 of shared memory.
+constexpr int kWideBits = 11, kWideBins = 1 << kWideBits;
+
 template <int KPT>
-__device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist, int *sc,
+__device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist, int *sc, int *scan_w,
                                   uint64_t *red, uint64_t &prefix, uint64_t &mask,
                                   const uint64_t *tail = nullptr, int n_tail = 0) {
     uint64_t lo = kNoKey, hi = 0;
@@ -304,15 +308,15 @@ __device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist,
         mask = ~0ull;
         return;
     }
-    // digits of 8 bits from the highest differing bit down (the last may be narrower)
     int pos = 64 - __clzll((long long)diff);   // bits [pos, 64) are common to every key
     mask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
     prefix = lo & mask;
     int k_rem = want;
+    const int bpt = kWideBins / blockDim.x;   // bins per thread in the bucket scan (1, 2 or 4)
     while (pos > 0) {
-        const int shift = pos > 8 ? pos - 8 : 0, width = pos - shift;
+        const int shift = pos > kWideBits ? pos - kWideBits : 0, width = pos - shift;
         const uint64_t dmask = (1ull << width) - 1ull;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        for (int i = threadIdx.x; i < kWideBins; i += blockDim.x) hist[i] = 0;
         __syncthreads();
 #pragma unroll
         for (int u = 0; u < KPT; ++u)
@@ -322,7 +326,32 @@ __device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist,
             if (key != kNoKey && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
         }
         __syncthreads();
-        if (radix_bucket(hist, sc, shift, width, k_rem, prefix, mask)) break;
+        // the bin holding the k_rem-th key: thread t scans bins [t*bpt, t*bpt + bpt)
+        int h[4] = {0, 0, 0, 0}, sum = 0;
+        for (int j = 0; j < bpt; ++j) {
+            h[j] = hist[threadIdx.x * bpt + j];
+            sum += h[j];
+        }
+        int total;
+        int acc = block_exclusive_scan_int(sum, scan_w, &total);
+        if (acc < k_rem && acc + sum >= k_rem) {
+            for (int j = 0; j < bpt; ++j) {
+                if (acc + h[j] >= k_rem) {
+                    sc[0] = threadIdx.x * bpt + j;
+                    sc[1] = h[j] - (k_rem - acc);   // 0 <=> the whole bucket is taken
+                    sc[2] = k_rem - acc;
+                    break;
+                }
+                acc += h[j];
+            }
+        }
+        __syncthreads();
+        const int d = sc[0], surplus = sc[1];
+        k_rem = sc[2];
+        prefix |= (uint64_t)d << shift;
+        mask |= dmask << shift;
+        __syncthreads();
+        if (surplus == 0) break;
         pos = shift;
     }
 }
@@ -629,6 +658,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectAr
     __shared__ int red_i[32];
     __shared__ uint64_t red_k[32];
     __shared__ int hist[256];
+    __shared__ int whist[kWideBins];
     __shared__ int sc[4];
     const Dims dm = a.dims;
     const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32;
@@ -708,7 +738,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectAr
             uint64_t key = kNoKey;
             kr[u] = (t < E && cand(t, key)) ? key : kNoKey;
         }
-        if (want < total) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask);
+        if (want < total) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask);
         collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kDenseThreads; }, f);
     } else {
         if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
@@ -898,6 +928,8 @@ __global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs
     __shared__ int sc[4];
     __shared__ int last;
     __shared__ int scan_w[32];
+    __shared__ int red_i[32];
+    __shared__ int whist[kWideBins];
     __shared__ int slice_base;
     const Dims dm = a.dims;
     const int BW = dm.BW, P = a.pick_parts;
@@ -996,7 +1028,7 @@ __global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs
                 const int i = tid + u * kPickThreads;
                 kr[u] = i < T ? sk[i] : kNoKey;
             }
-            if (want < T) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask);
+            if (want < T) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask);
             collect_regs(kr, prefix, mask, BW, [&](int u) { return se[tid + u * kPickThreads]; }, f);
         } else if (T <= a.surv_cap) {
             const ListCand<true> cand{sk_g};
@@ -1050,6 +1082,7 @@ __global__ void __launch_bounds__(kPickOneThreads, 1) select_pick_one_kernel(Sel
     __shared__ int sc[4];
     __shared__ int red_i[32];
     __shared__ uint64_t red_k[32];
+    __shared__ int whist[kWideBins];
     const Dims dm = a.dims;
     const int BW = dm.BW, r = blockIdx.x, tid = threadIdx.x;
     const int64_t rb = (int64_t)r * BW;
@@ -1095,7 +1128,7 @@ __global__ void __launch_bounds__(kPickOneThreads, 1) select_pick_one_kernel(Sel
         for (int i = tid; i < n_tail; i += kPickOneThreads) c += tail[i] != kNoKey;
         const int T = block_sum_int(c, red_i);   // (its barriers also publish the staging)
         want = min(BW, T);
-        if (want < T) radix_select_regs(kr, want, hist, sc, red_k, prefix, mask, tail, n_tail);
+        if (want < T) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask, tail, n_tail);
         collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kPickOneThreads; }, f);
         for (int i = tid; i < n_tail; i += kPickOneThreads) {
             const uint64_t key = tail[i];
@@ -1137,9 +1170,11 @@ __global__ void __launch_bounds__(kPickOneThreads, 1) select_pick_one_kernel(Sel
     finish_request(a, r, min(*f.cnt, want), f);
 }
 
+// opt in to the dynamic shared memory a launch needs: without it static plus
+// dynamic shared memory may not pass 48 KB
 template <class K>
 cudaError_t ensure_smem(K kernel, size_t bytes) {
-    if (bytes <= 48 * 1024) return cudaSuccess;
+    if (bytes == 0) return cudaSuccess;
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
@@ -1176,7 +1211,17 @@ void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, int64_t
     a.surv_cap = surv_cap;
 }
 
-cudaError_t launch_beam_select(const SelectArgs &a_in, cudaStream_t s) {
+static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t s);
+
+cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s) {
+    const cudaError_t e = launch_beam_select_impl(a, s);
+    if (e != cudaSuccess)
+        debug_log("beam select (B=%d BW=%d V=%d dense=%d): launch failed: %s", a.dims.B, a.dims.BW,
+                  a.dims.V, a.dense, cudaGetErrorString(e));
+    return e;
+}
+
+static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t s) {
     SelectArgs a = a_in;
     const Dims &dm = a.dims;
     if (dm.BW > 1024 || dm.V > kSelectMaxVocab || dm.V < 1) return cudaErrorInvalidValue;
@@ -1201,7 +1246,8 @@ cudaError_t launch_beam_select(const SelectArgs &a_in, cudaStream_t s) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    if (std::min<int64_t>(a.max_entries, a.key_cap) <= kPickOneMax) {
+    // the one-CTA pick when the pool fits its registers and its shared memory fits the SM
+    if (std::min<int64_t>(a.max_entries, a.key_cap) <= kPickOneMax && pick_one_smem(dm) <= (200u << 10)) {
         const size_t smem = pick_one_smem(dm);
         cudaError_t e = ensure_smem(select_pick_one_kernel, smem);
         if (e != cudaSuccess) return e;

@@ -59,6 +59,7 @@ class Workload:
     logits_std: float = 2.0     # "N(0,2)" read as standard deviation 2
     groups: int = 0             # >0: requests share prefixes in this many groups
     suffix: tuple = (0, 0)      # per-request unshared suffix length range (inclusive)
+    shard: int = 0              # which B-request slice of a larger batch (one per GPU)
 
     @property
     def G(self) -> int:
@@ -104,8 +105,14 @@ def small(w: Workload, **kw) -> Workload:
     return dataclasses.replace(w, **kw)
 
 
-def _seed(w: Workload, tid: int, extra: int = 0) -> int:
-    return 1000 * w.wid + tid + 100_000 * extra
+def shard_of(w: Workload, shard: int) -> Workload:
+    """Requests shard*B .. shard*B + B-1 of a batch split over GPUs: the same shapes
+    and the same global item set, their own prompts, queries and scores."""
+    return dataclasses.replace(w, shard=shard)
+
+
+def _seed(w: Workload, tid: int, extra: int = 0, per_shard: bool = True) -> int:
+    return 1000 * w.wid + tid + 100_000 * extra + (10_000_000 * w.shard if per_shard else 0)
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -120,7 +127,7 @@ def items(w: Workload) -> np.ndarray:
     Duplicates are rejected and redrawn; the result keeps first-draw order.
     Returns int32 [n_items][S].
     """
-    rng = np.random.default_rng(_seed(w, _T_ITEMS))
+    rng = np.random.default_rng(_seed(w, _T_ITEMS, per_shard=False))   # one global item set
     n, L, V = w.n_items, w.S, w.V
     if n > V ** L:
         raise ValueError("more distinct items requested than tuples exist")
