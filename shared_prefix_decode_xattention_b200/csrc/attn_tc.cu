@@ -12,19 +12,21 @@
 //
 // One CTA per work item (kv head, 128-row tile, key range):
 //   warp 0      TMA producer: Q, then K and V chunks of 128 keys (two 64-column
-//               128-byte-swizzled boxes each) on separate two-stage rings;
+//               128-byte-swizzled boxes each) on separate three-stage rings;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_j = Q K_j^T into TMEM buffer j % 2, O_{j%2} += P_j V_j;
+//               S_j = Q K_j^T into TMEM buffer j % 2, O_{j%2} += P_j V_j with
+//               P_j read from tensor memory;
 //   warps 2-9   two softmax warpgroups; warpgroup h owns the chunks j with
 //               j % 2 == h, one query row per thread: it reads S_j from TMEM,
 //               keeps the running max and sum of its own accumulator O_h (lazy
 //               rescaling: O_h is rescaled only when the max grows by more than
-//               2^8), and writes P_j (bf16) into its own shared-memory buffer in
-//               the canonical 128-byte-swizzled K-major layout.  The two
-//               warpgroups never wait for each other inside the loop, so one's
-//               exponentials overlap the other's row maxima and TMEM traffic;
-//               at the end they swap (m, l) and merge O_0 and O_1 into the
-//               partial (O, m, l) or, for a request's only segment, the output.
+//               2^8), and writes P_j (bf16 pairs) over the first half of S_j's
+//               TMEM buffer, so no shared memory goes to P and the K and V rings
+//               are three deep.  The two warpgroups never wait for each other
+//               inside the loop, so one's exponentials overlap the other's row
+//               maxima and TMEM traffic; at the end they swap (m, l) and merge
+//               O_0 and O_1 into the partial (O, m, l) or, for a request's only
+//               segment, the output.
 // In a request's only KV segment ("final" items) the Unshared and Merging
 // stages run here too: before the loop the softmax threads gather the beam's
 // own tokens (direct indices into the token-granular pool), seed O_0 and its
@@ -50,25 +52,28 @@ constexpr int kKStages = 2;                  // K chunks in flight
 constexpr int kVStages = 2;                  // V chunks in flight
 constexpr uint32_t kHalf = 16384;            // one 128-row x 64-column bf16 sub-tile
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 bf16
+constexpr uint32_t kUBytes = 65536;          // U area: the Unshared stage's staged rows
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
-constexpr uint32_t kOffP = kOffV + kVStages * kTile;   // P of warpgroup 0, then of warpgroup 1
-constexpr uint32_t kOffBar = kOffP + 2 * kTile;
+constexpr uint32_t kOffU = kOffV + kVStages * kTile;
+constexpr uint32_t kOffBar = kOffU + kUBytes;
 constexpr uint32_t kOffMisc = kOffBar + 256;  // TMEM address, abort flag
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = 232448;       // the sm_100 per-block maximum
 constexpr uint32_t kSmemSpare = kSmemBytes - kSmemUsed;   // room to realign the window
-constexpr uint32_t kTmemCols = 512;          // S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512)
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_j (bf16, two
+// per column) overwrites the first 64 columns of S_j's buffer once S_j is read
+constexpr uint32_t kTmemCols = 512;
 
 // barrier slots (8 bytes each) after kOffBar; SFULL, PFULL, PVDONE and XCH have one
 // slot per warpgroup
-enum { B_KFULL = 0, B_KEMPTY = 2, B_VFULL = 4, B_VEMPTY = 6, B_SFULL = 8, B_PFULL = 10,
-       B_PVDONE = 12, B_QFULL = 14, B_DONE = 15, B_XCH = 16, B_PRO = 18, B_SFREE = 19,
-       B_COUNT = 21 };
-// B_SFREE: a warpgroup has read all of S_j (its TMEM buffer may take S_{j+2});
-// B_DONE: every MMA has completed; B_XCH: the warpgroups' (m, l) exchange;
-// B_PRO: the Unshared prologue's loads have returned
+enum { B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
+       B_VEMPTY = B_VFULL + kVStages, B_SFULL = B_VEMPTY + kVStages, B_PFULL = B_SFULL + 2,
+       B_PVDONE = B_PFULL + 2, B_QFULL = B_PVDONE + 2, B_DONE = B_QFULL + 1, B_XCH = B_DONE + 1,
+       B_COUNT = B_XCH + 2 };
+// B_PVDONE: P_j V_j has completed (S_j's TMEM buffer, which held P_j, may take
+// S_{j+2}); B_DONE: every MMA has completed; B_XCH: the warpgroups' (m, l) exchange
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -113,6 +118,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t 
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// the same with A in tensor memory (rows in lanes, two bf16 per 32-bit column)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -167,6 +183,33 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
+// wait for this thread's TMEM loads; v (their destination) is tied to the wait,
+// so no use of it can be scheduled before
+__device__ __forceinline__ void tmem_wait_ld_into(float *v) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+                   "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]),
+                   "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]),
+                   "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]),
+                   "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]),
+                   "+f"(v[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -185,6 +228,12 @@ __device__ __forceinline__ float ex2(float x) {   // 2^x, one MUFU op; tiny resu
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// 16-byte global -> shared copy that bypasses the registers (and L1)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -212,10 +261,8 @@ __device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it,
 }
 
 // 10 warps: the register file is split over the 4 schedulers (16K registers each) and 3 of
-// the 10 warps share one, so a thread may use at most 168 registers
-// NT: the most Unshared tokens (step + 1) the prologue handles; one instance per
-// step range keeps the unrolled prologue (and the instruction footprint) small
-template <int NT>
+// the 10 warps share one, so a thread may use at most 168 registers.  One instance
+// serves every step (the code is warm in the caches after the first launch).
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const __grid_constant__ CUtensorMap tmq, TcArgs a) {
@@ -269,11 +316,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 mbar_init(bar(B_PFULL + h), kGroupThreads);
                 mbar_init(bar(B_PVDONE + h), 1);
                 mbar_init(bar(B_XCH + h), kGroupThreads);
-                mbar_init(bar(B_SFREE + h), kGroupThreads);
             }
             mbar_init(bar(B_QFULL), q_tma ? 1 : kSoftmaxThreads);
             mbar_init(bar(B_DONE), 1);
-            mbar_init(bar(B_PRO), kSoftmaxThreads);
             *abort_flag = 0;
             fence_mbar_init();
         }
@@ -286,12 +331,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_3d(sb + kOffQ, &tmq, 0, it.g * G, z, bar(B_QFULL));
             tma_load_3d(sb + kOffQ + kHalf, &tmq, 64, it.g * G, z, bar(B_QFULL));
         }
-        // In final items only Q and the first K chunk go out now: the rest of the
-        // K/V fill waits until the Unshared prologue's scattered loads have
-        // returned, so that those do not queue behind megabytes of streaming.
         if (lane == 0)
-            for (int j = 0; j < min(nchunks, final_item ? 1 : kKStages); ++j) issue_k(j);
-        if (lane == 1 && !final_item)
+            for (int j = 0; j < min(nchunks, kKStages); ++j) issue_k(j);
+        if (lane == 1)
             for (int j = 0; j < min(nchunks, kVStages); ++j) issue_v(j);
     }
     if (warp == 1) {
@@ -327,9 +369,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producers
         if (lane == 0) {
-            int n_issued = min(nchunks, final_item ? 1 : kKStages);
-            if (final_item && n_issued < min(nchunks, kKStages) && mbar_wait(bar(B_PRO), 0, abort))
-                for (; n_issued < min(nchunks, kKStages); ++n_issued) issue_k(n_issued);
+            int n_issued = min(nchunks, kKStages);
             for (int j = kKStages; j < nchunks && n_issued == j; ++j) {
                 if (!mbar_wait(bar(B_KEMPTY + j % kKStages), ((j / kKStages) - 1) & 1, abort)) break;
                 issue_k(j);
@@ -339,9 +379,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int j = max(0, n_issued - kKStages); j < n_issued; ++j)
                     mbar_wait(bar(B_KFULL + j % kKStages), (j / kKStages) & 1, nullptr);
         } else if (lane == 1) {
-            int n_issued = final_item ? 0 : min(nchunks, kVStages);
-            if (final_item && nchunks > 0 && mbar_wait(bar(B_PRO), 0, abort))
-                for (; n_issued < min(nchunks, kVStages); ++n_issued) issue_v(n_issued);
+            int n_issued = min(nchunks, kVStages);
             for (int j = kVStages; j < nchunks && n_issued == j; ++j) {
                 if (!mbar_wait(bar(B_VEMPTY + j % kVStages), ((j / kVStages) - 1) & 1, abort)) break;
                 issue_v(j);
@@ -360,9 +398,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
-            auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T
+            auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T (waits for K_j unless it has landed)
                 const int st = j % kKStages;
-                if (!mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) return false;
+                if (j < 2 && !mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) return false;
                 fence_after_sync();
                 const uint32_t kq = sb + kOffQ, kk = sb + kOffK + st * kTile;
 #pragma unroll
@@ -376,28 +414,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 return true;
             };
             bool ok = mbar_wait(bar(B_QFULL), 0, abort);
-            for (int j = 0; ok && j < min(nchunks, 2); ++j) ok = issue_s(j);
-            for (int j = 0; ok && j < nchunks; ++j) {   // S_{j+2}, then O_h += P_j V_j
-                const int h = j & 1, sv = j % kVStages;
-                if (j + 2 < nchunks) {
-                    if (!mbar_wait(bar(B_SFREE + h), (j >> 1) & 1, abort)) break;
-                    if (!issue_s(j + 2)) break;
+            int ns = 0;   // the next S to issue
+            for (; ok && ns < min(nchunks, 2); ++ns) ok = issue_s(ns);
+            // Then whichever is ready first: S_ns (P_{ns-2} V_{ns-2}, which read its
+            // TMEM buffer, complete and K_ns landed) or O_h += P_j V_j (P_j written,
+            // V_j landed).  Every phase polled here is at most one behind the
+            // barrier's current one, so the parity tests are exact.
+            uint32_t idle = 0;
+            for (int j = 0; ok && j < nchunks;) {
+                bool progress = false;
+                if (ns < nchunks && mbar_test(bar(B_PVDONE + (ns & 1)), ((ns - 2) >> 1) & 1) &&
+                    mbar_test(bar(B_KFULL + ns % kKStages), (ns / kKStages) & 1)) {
+                    issue_s(ns++);
+                    progress = true;
                 }
-                if (!mbar_wait(bar(B_PFULL + h), (j >> 1) & 1, abort)) break;
-                if (!mbar_wait(bar(B_VFULL + sv), (j / kVStages) & 1, abort)) break;
+                const int h = j & 1, sv = j % kVStages;
+                if (!(mbar_test(bar(B_PFULL + h), (j >> 1) & 1) &&
+                      mbar_test(bar(B_VFULL + sv), (j / kVStages) & 1))) {
+                    if (progress) {
+                        idle = 0;
+                    } else if (++idle >= kSpinLimit) {
+                        *abort = 1;
+                        ok = false;
+                    } else if ((idle & 255) == 0 && *abort) {
+                        ok = false;
+                    }
+                    continue;
+                }
+                idle = 0;
                 fence_after_sync();
-                const uint32_t kp = sb + kOffP + (uint32_t)h * kTile, kv = sb + kOffV + sv * kTile;
+                const uint32_t kv = sb + kOffV + sv * kTile;
                 // O_0 starts from the Unshared stage in final items
                 const bool acc0 = j >= 2 || (j == 0 && final_item);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t offp = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                    umma_bf16(tmem + 256u + (uint32_t)h * 128u, umma_desc(kp + offp, 16, 1024),
-                              umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
-                              (k > 0 || acc0) ? 1u : 0u);
-                }
+                for (int k = 0; k < 8; ++k)   // P_j: 16 keys = 8 TMEM columns per MMA
+                    umma_bf16_ts(tmem + 256u + (uint32_t)h * 128u, tmem + (uint32_t)h * 128u + 8u * k,
+                                 umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
+                                 (k > 0 || acc0) ? 1u : 0u);
                 umma_commit(bar(B_PVDONE + h));
                 umma_commit(bar(B_VEMPTY + sv));
+                ++j;
             }
             // arrives once every MMA issued above has completed (TMEM final / free)
             umma_commit(bar(B_DONE));
@@ -407,7 +463,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ------------------------------------------------------------ softmax
         // Warpgroup `half` owns the chunks j with j % 2 == half, whole rows: thread
         // `row` reads TMEM lane `row` of S buffer `half`, keeps the running max and
-        // sum of accumulator O_half and writes row `row` of P buffer `half`.  The
+        // sum of accumulator O_half and writes row `row` of P_j over it.  The
         // two warpgroups never wait for each other inside the loop; their
         // (m, l, O) are merged at the end.  In the Unshared prologue thread
         // (row, half) handles head-dim columns [64*half, 64*half + 64).
@@ -425,134 +481,127 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t col0 = (uint32_t)(64 * half);
         float m_used = -INFINITY, l = 0.f;   // running max / sum of O_half
         const Dims dm = a.dims;
-        const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
-        const int64_t kvo = (beam_row * dm.Hkv + it.g) * 128;
-        const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
-        const int64_t pool_req = (int64_t)ri.r * dm.BW * dm.Hkv * 128;
-        const int s_now = a.step;
-        const int n_tok = s_now + 1;
-        // the beam's ancestry slots are read together with n_live, while Q is in flight
-        int slot[NT];
-        if (final_item) {
-#pragma unroll
-            for (int i = 0; i < NT; ++i)
-                slot[i] = (ri.valid && i < s_now) ? a.st.anc[beam_row * dm.S + i] : ri.b;
-        }
         const bool live = ri.valid && ri.b < a.n_live[ri.r];
-        float sc[NT];   // scaled scores of the beam's own tokens (final items)
         if (final_item) {
             // ---- Unshared stage first (the item covers its requests' only KV
-            // segment): the beam's own tokens of steps 0..s, read through its
-            // direct indices, seed the online softmax -- their max, their sum (half
-            // 0) and their weighted values in the TMEM O accumulator -- so the
-            // main loop merges the two stages as it goes.  Row hg = 0 of each beam
-            // also appends this step's k/v (already in registers) at Unshared slot
-            // (s, b).
-            const bool appender = live && ri.hg == 0;
-            const __nv_bfloat16 *kp[NT], *vp[NT];
+            // segment): each beam's own tokens of steps 0..s, read through its
+            // direct indices (ancestry slots) into the token-granular pool, seed
+            // the online softmax -- their max, their sum (half 0) and their
+            // weighted values in the TMEM accumulator O_0 -- so the main loop
+            // merges the two stages as it goes.  The rows of the tile's beams are
+            // staged in the U area by cp.async: one round trip for the slots, one
+            // per batch of (beams, tokens) that fits, whatever the step.  Thread
+            // (row, half) computes the full score of its row and the weighted
+            // values of its 64 head-dim columns.
+            const int G = dm.G, ts = tid - 64;
+            const int s_now = a.step, n_tok = s_now + 1;
+            const int lb0 = it.row_begin / G;
+            const int nbeam = (it.row_begin + it.n_rows - 1) / G - lb0 + 1;   // beams in the tile
+            const int lb = (it.row_begin + row) / G - lb0;                     // this row's beam
+            constexpr int kTabW = kMaxSteps + 1;   // per beam: slot of each token, then r * BW + b
+            int *tab = reinterpret_cast<int *>(base + kOffU);
+            const uint32_t tab_bytes = ((uint32_t)nbeam * kTabW * 4u + 127u) & ~127u;
+            // [tokens][beams][k | v][128] bf16, kStgRow bytes per (token, beam): the 16-byte
+            // pad puts the beams one warp reads at once in different banks
+            constexpr uint32_t kStgRow = 528;
+            uint8_t *stg = base + kOffU + tab_bytes;
+            const int nbg = min(nbeam, (int)((kUBytes - tab_bytes) / kStgRow));   // beams per batch
+            const int tb = max(1, (int)((kUBytes - tab_bytes) / ((uint32_t)nbg * kStgRow)));   // tokens per batch
+            // 1. the tile's first row of each beam reads the beam's slots (one round trip)
+            if (ri.valid && (ri.hg == 0 || row == 0) && half == 0) {
+                const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
+                int sl[kMaxSteps];
 #pragma unroll
-            for (int i = 0; i < NT; ++i) {
-                kp[i] = vp[i] = nullptr;
-                if (!live || i >= n_tok) continue;
-                if (slot[i] < 0 || slot[i] >= dm.BW) {
-                    set_status(a.status, XGR_DEV_INDEX);
-                    continue;
-                }
-                if (i == s_now) {
-                    kp[i] = a.k_new + kvo;
-                    vp[i] = a.v_new + kvo;
-                } else {
-                    const int64_t o2 = i * pool_step + pool_req + ((int64_t)slot[i] * dm.Hkv + it.g) * 128;
-                    kp[i] = a.pool_k + o2;
-                    vp[i] = a.pool_v + o2;
-                }
-                if (i >= 2) asm volatile("prefetch.global.L2 [%0];" ::"l"(kp[i] + col0));
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(vp[i] + col0));
-            }
-            __nv_bfloat16 *const k_app = a.pool_k + s_now * pool_step + kvo + col0;
-            __nv_bfloat16 *const v_app = a.pool_v + s_now * pool_step + kvo + col0;
-            // the first two k rows load while Q is still in flight
-            uint4 k0[8], k1[8];
+                for (int i = 0; i < kMaxSteps; ++i)
+                    sl[i] = (live && i < s_now) ? a.st.anc[beam_row * dm.S + i] : -1;
+                int *t = tab + lb * kTabW;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                k0[c] = kp[0] ? reinterpret_cast<const uint4 *>(kp[0] + col0)[c] : make_uint4(0, 0, 0, 0);
-                k1[c] = (1 < n_tok && kp[1]) ? reinterpret_cast<const uint4 *>(kp[1] + col0)[c]
-                                             : make_uint4(0, 0, 0, 0);
+                for (int i = 0; i < kMaxSteps; ++i) {
+                    if (i >= s_now) break;
+                    if (live && (sl[i] < 0 || sl[i] >= dm.BW)) set_status(a.status, XGR_DEV_INDEX);
+                    t[i] = (sl[i] >= 0 && sl[i] < dm.BW) ? sl[i] : -1;
+                }
+                t[s_now] = live ? ri.b : -1;
+                t[kMaxSteps] = (int)beam_row;
             }
-            if (q_tma)   // the prologue reads Q from shared memory
+            if (q_tma)   // the scores read Q from shared memory
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort));
-            float *xd = reinterpret_cast<float *>(base + kOffP);   // [2 halves][NT][128]
-#pragma unroll
-            for (int i = 0; i < NT; i += 2) {
-                if (i >= n_tok) break;
-                if (i > 0) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        k0[c] = kp[i] ? reinterpret_cast<const uint4 *>(kp[i] + col0)[c] : make_uint4(0, 0, 0, 0);
-                        k1[c] = (i + 1 < n_tok && kp[i + 1])
-                                    ? reinterpret_cast<const uint4 *>(kp[i + 1] + col0)[c]
-                                    : make_uint4(0, 0, 0, 0);
-                    }
-                }
-                if (appender && i == s_now) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(k_app)[c] = k0[c];
-                }
-                if (appender && i + 1 == s_now) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(k_app)[c] = k1[c];
-                }
-                float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {   // q (bf16, swizzled K-major) read 8 columns at a time
-                    float qf[8], f0[8], f1[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)), qf);
-                    unpack8(k0[c], f0);
-                    unpack8(k1[c], f1);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        acc0 = fmaf(qf[e], f0[e], acc0);
-                        acc1 = fmaf(qf[e], f1[e], acc1);
-                    }
-                }
-                xd[(half * NT + i) * 128 + row] = acc0;
-                if (i + 1 < n_tok) xd[(half * NT + i + 1) * 128 + row] = acc1;
-            }
             named_sync(1, kSoftmaxThreads);
-            float m_u = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < NT; ++i) {
-                sc[i] = (i < n_tok && kp[i]) ? (xd[i * 128 + row] + xd[(NT + i) * 128 + row]) * cscale
-                                             : -INFINITY;
-                m_u = fmaxf(m_u, sc[i]);
-            }
-            named_sync(1, kSoftmaxThreads);   // the exchange area is reused by P afterwards
-            float l_u = 0.f;
-            float o[64];
+            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+            const int64_t kvo = ((int64_t)(ri.r * dm.BW + ri.b) * dm.Hkv + it.g) * 128;
+            float m_u = -INFINITY, l_u = 0.f, o[64];
 #pragma unroll
             for (int e = 0; e < 64; ++e) o[e] = 0.f;
+            // 2. batches: stage the k and v rows of (beams, tokens), then fold them in
+            for (int gb = 0; gb < nbeam; gb += nbg) {
+                const int ngb = min(nbg, nbeam - gb);
+                for (int i0 = 0; i0 < n_tok; i0 += tb) {
+                    const int ntb = min(tb, n_tok - i0);
+                    const int units = ngb * ntb * 32;   // 16-byte pieces: 16 of k and 16 of v per row pair
+                    for (int u = ts; u < units; u += kSoftmaxThreads) {
+                        const int c = u & 15, kind = (u >> 4) & 1, bt = u >> 5;
+                        const int bl = bt % ngb, ti = bt / ngb, i = i0 + ti;
+                        const int *t = tab + (gb + bl) * kTabW;
+                        const int sl = t[i];
+                        if (sl < 0) continue;
+                        const int64_t brow = t[kMaxSteps];
+                        const int64_t src_row = i == s_now ? brow
+                                                           : (brow - brow % dm.BW + sl) + (int64_t)i * a.Bcap * dm.BW;
+                        const __nv_bfloat16 *src =
+                            (i == s_now ? (kind ? a.v_new : a.k_new) : (kind ? a.pool_v : a.pool_k)) +
+                            (src_row * dm.Hkv + it.g) * 128 + c * 8;
+                        cp_async16(smem_u32(stg + (uint32_t)(ti * ngb + bl) * kStgRow + kind * 256u + c * 16), src);
+                    }
+                    cp_async_wait_all();
+                    named_sync(1, kSoftmaxThreads);
+                    if (live && lb >= gb && lb < gb + ngb) {
+#pragma unroll 1
+                        for (int ti = 0; ti < ntb; ++ti) {
+                            const int i = i0 + ti;
+                            if (tab[lb * kTabW + i] < 0) continue;
+                            const uint8_t *kr = stg + (uint32_t)(ti * ngb + lb - gb) * kStgRow;
+                            const uint8_t *vr = kr + 256;
+                            float acc = 0.f;
+#pragma unroll 4
+                            for (int c = 0; c < 16; ++c) {
+                                float qf[8], kf[8];
+                                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, c)), qf);
+                                unpack8(*reinterpret_cast<const uint4 *>(kr + c * 16), kf);
 #pragma unroll
-            for (int i = 0; i < NT; ++i) {
-                if (i >= n_tok || sc[i] == -INFINITY) continue;
-                const float pw = ex2(sc[i] - m_u);
-                l_u += pw;
-                uint4 vv[8];
+                                for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
+                            }
+                            const float sc = acc * cscale;
+                            if (sc > m_u) {   // online softmax over the beam's tokens
+                                const float al = ex2(m_u - sc);
+                                l_u *= al;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) vv[c] = reinterpret_cast<const uint4 *>(vp[i] + col0)[c];
-                if (appender && i == s_now) {
+                                for (int e = 0; e < 64; ++e) o[e] *= al;
+                                m_u = sc;
+                            }
+                            const float pw = ex2(sc - m_u);
+                            l_u += pw;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(v_app)[c] = vv[c];
-                }
+                            for (int c = 0; c < 8; ++c) {
+                                float vf[8];
+                                unpack8(*reinterpret_cast<const uint4 *>(vr + col0 * 2 + c * 16), vf);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float vf[8];
-                    unpack8(vv[c], vf);
+                                for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw, vf[e], o[8 * c + e]);
+                            }
+                            if (i == s_now && ri.hg == 0) {   // append this step's k / v at slot (s, b)
+                                uint4 *ka = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + kvo + col0);
+                                uint4 *va = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + kvo + col0);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw, vf[e], o[8 * c + e]);
+                                for (int c = 0; c < 8; ++c) {
+                                    ka[c] = *reinterpret_cast<const uint4 *>(kr + col0 * 2 + c * 16);
+                                    va[c] = *reinterpret_cast<const uint4 *>(vr + col0 * 2 + c * 16);
+                                }
+                            }
+                        }
+                    }
+                    if (gb + nbg < nbeam || i0 + tb < n_tok) named_sync(1, kSoftmaxThreads);   // restage
                 }
             }
-            mbar_arrive(bar(B_PRO));   // the scattered loads are in: the K/V fill may start
-            // the Unshared stage seeds the O accumulator, the running max and (half 0) sum
+            // the Unshared stage seeds O_0 (both halves' columns), the running max and (half 0) sum
             tmem_st32(tmem + lane_base + 256 + col0, o);
             tmem_st32(tmem + lane_base + 256 + col0 + 32, o + 32);
             tmem_wait_st();
@@ -561,21 +610,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l = l_u;
             }
         }
+        if (final_item && a.nb == 1 && dm.BW > 1) {
+            // One live beam per request (step 0): while the first scores are in
+            // flight, write O = 0 and LSE = -inf for beams 1 .. BW-1 in this kv
+            // head's query heads, for every request whose rows start in this tile.
+            const int G = dm.G, ts = tid - 64;
+            const int m_lo = (it.row_begin + G - 1) / G;
+            const int m_hi = (it.row_begin + it.n_rows + G - 1) / G;
+            for (int m = m_lo; m < m_hi; ++m) {
+                const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + m];
+                const int64_t row1 = ((int64_t)r * dm.BW + 1) * dm.Hq + it.g * G;   // beam 1, head g*G
+                const int units = (dm.BW - 1) * G * 16;   // 16-byte pieces
+                for (int u = ts; u < units; u += kSoftmaxThreads) {
+                    const int bb = u / (G * 16), hg = (u / 16) % G;
+                    reinterpret_cast<uint4 *>(a.out + (row1 + (int64_t)bb * dm.Hq + hg) * 128)[u % 16] =
+                        make_uint4(0, 0, 0, 0);
+                }
+                for (int u = ts; u < (dm.BW - 1) * G; u += kSoftmaxThreads)
+                    a.lse[row1 + (int64_t)(u / G) * dm.Hq + u % G] = -INFINITY;
+            }
+        }
         const uint32_t s_col = (uint32_t)half * 128u;          // S buffer of this warpgroup
         const uint32_t o_col = 256u + (uint32_t)half * 128u;   // its O accumulator
-        uint8_t *pb = base + kOffP + (uint32_t)half * kTile;   // its P buffer
         for (int j = half, jj = 0; ok && j < nchunks; j += 2, ++jj) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + half), jj & 1, abort));
             if (!ok) break;
             fence_after_sync();
             const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
-            // the chunk's 128 scores in one TMEM read; S_j's buffer is then free for S_{j+2}
+            // the chunk's 128 scores in one TMEM read (P_j then overwrites them)
             float sv[128];
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) tmem_ld32(tmem + lane_base + s_col + 32 * q2, sv + 32 * q2);
             tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(bar(B_SFREE + half));
             if (nvalid < kBlockN) {   // the range's last chunk: keys past its end do not count
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
@@ -595,29 +661,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 rescale = jj > 0 || (half == 0 && final_item);   // O_half already holds data
                 m_used = mx;
             }
-            // P V of this warpgroup's previous chunk has read P_half and written O_half
-            if (jj > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_PVDONE + half), (jj - 1) & 1, abort));
-                if (!ok) break;
-            }
-            // exponentials, row sum and P (bf16), 8 columns (16 bytes) at a time
+            // (S_j was issued after P_{j-2} V_{j-2} completed: O_half is current and
+            // this TMEM buffer no longer holds P_{j-2})
+            // exponentials, row sum and P (bf16 pairs) into the first 64 columns of
+            // the S buffer, in four rolled pieces of 32 scores re-read from TMEM (a
+            // small loop body): piece q's 16 P columns land on scores already read
             const float neg_m = -m_used;
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+#pragma unroll 1
+            for (int q2 = 0; q2 < 4; ++q2) {
+                float v[32], pw[16];
+                tmem_ld32(tmem + lane_base + s_col + 32 * q2, v);
+                tmem_wait_ld_into(v);
+                const int nv = nvalid - 32 * q2;   // keys of the piece inside the range
+                if (nv < 32) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint32_t w4[4];
+                    for (int e = 0; e < 32; ++e)
+                        if (e >= nv) v[e] = -INFINITY;
+                }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2(fmaf(sv[8 * c + 2 * e], cscale, neg_m));
-                    const float p1 = ex2(fmaf(sv[8 * c + 2 * e + 1], cscale, neg_m));
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(v[2 * e], cscale, neg_m));
+                    const float p1 = ex2(fmaf(v[2 * e + 1], cscale, neg_m));
                     sp[(2 * e) & 7] += p0;
                     sp[(2 * e + 1) & 7] += p1;
                     __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    w4[e] = *reinterpret_cast<uint32_t *>(&h2);
+                    pw[e] = __uint_as_float(*reinterpret_cast<uint32_t *>(&h2));
                 }
-                *reinterpret_cast<uint4 *>(pb + sw128_off(row, c)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                tmem_st16(tmem + lane_base + s_col + 16 * q2, pw);
             }
             if (__any_sync(0xffffffffu, rescale)) {   // O_half *= alpha before P_j V_j adds in
                 fence_after_sync();
@@ -634,7 +707,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_wait_st();
             }
             l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
-            fence_async_smem();
+            tmem_wait_st();   // P_j (and a rescaled O_half) in TMEM before the MMA warp reads them
             fence_before_sync();
             mbar_arrive(bar(B_PFULL + half));
         }
@@ -644,7 +717,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             fence_after_sync();
             // the warpgroups swap (m, l); thread (row, half) then merges head-dim
             // columns [64*half, 64*half + 64) of O_0 and O_1
-            float2 *xl = reinterpret_cast<float2 *>(base + kOffP);   // [2][128]
+            float2 *xl = reinterpret_cast<float2 *>(base + kOffV);   // [2][128]; V is consumed
             xl[half * 128 + row] = make_float2(m_used, l);
             mbar_arrive(bar(B_XCH + half));
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH + (half ^ 1)), 0, abort));
@@ -757,17 +830,16 @@ cudaError_t make_q_tensor_map(CUtensorMap *map, const void *q, int64_t beam_rows
 
 namespace {
 
-template <int NT>
-cudaError_t launch_nt(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+cudaError_t launch_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
                       const TcArgs &a, int n_items, cudaStream_t st) {
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<NT>,
+        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_tc_kernel<NT>);
+        e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
         if (e != cudaSuccess) return e;
         if (fa.maxThreadsPerBlock < kTcThreads) {
             debug_log("attn_tc: %d registers/thread allow only %d threads per block", fa.numRegs,
@@ -776,7 +848,7 @@ cudaError_t launch_nt(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUte
         }
         attr = true;
     }
-    attn_tc_kernel<NT><<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
+    attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
     return cudaGetLastError();
 }
 
@@ -785,11 +857,8 @@ cudaError_t launch_nt(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUte
 cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
                            const TcArgs &a, int n_items, cudaStream_t st) {
     if (n_items <= 0) return cudaSuccess;
-    const int n_tok = a.step + 1;   // Unshared tokens of a beam at this step
-    if (n_tok <= 2) return launch_nt<2>(tmk, tmv, tmq, a, n_items, st);
-    if (n_tok <= 4) return launch_nt<4>(tmk, tmv, tmq, a, n_items, st);
-    if (n_tok <= kMaxSteps) return launch_nt<kMaxSteps>(tmk, tmv, tmq, a, n_items, st);
-    return cudaErrorInvalidValue;
+    if (a.step + 1 > kMaxSteps) return cudaErrorInvalidValue;   // Unshared tokens of a beam
+    return launch_tc(tmk, tmv, tmq, a, n_items, st);
 }
 
 }  // namespace xgr

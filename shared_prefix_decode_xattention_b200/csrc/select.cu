@@ -155,33 +155,68 @@ __device__ __forceinline__ Group whole_block() { return Group{0, (int)blockDim.x
 // log-sum-exp of the values x[i], i < n, in shared memory, over a group: the
 // row max first, then the sum of exponentials, each reduced without
 // branches; reports NaN.  red: 33 floats of shared memory for the group.
+// log-sum-exp of x[0..n) (shared memory) over a group, in one pass: each thread
+// keeps its own (max, sum of 2^((x - max) log2 e)) over blocks of 16 values
+// (16-byte loads when x is 16-byte aligned), rescaling its sum when its max
+// grows; the pairs are then combined across the group.  red holds 2 floats per
+// warp of the group.
+__device__ __forceinline__ void lse_pair_merge(float &m, float &s, float m2, float s2) {
+    const float M = fmaxf(m, m2);
+    if (M == -INFINITY) return;   // both empty
+    s = (m == -INFINITY ? 0.f : s * ex2f((m - M) * kLog2e)) +
+        (m2 == -INFINITY ? 0.f : s2 * ex2f((m2 - M) * kLog2e));
+    m = M;
+}
 __device__ float group_lse(const float *x, int n, float *red, int32_t *status, const Group &g) {
     const int lane = g.t % 32, w = g.t / 32, nw = g.n / 32;
-    float m = -INFINITY;
+    float m = -INFINITY, s = 0.f;
     bool nan = false;
-    for (int i = g.t; i < n; i += g.n) {
-        const float v = x[i];
-        nan |= isnan(v);
-        m = fmaxf(m, v);
+    auto fold = [&](const float *v, int k) {   // k values already in registers
+        float mv = -INFINITY;
+        for (int e = 0; e < k; ++e) {
+            nan |= isnan(v[e]);
+            mv = fmaxf(mv, v[e]);
+        }
+        if (mv > m) {
+            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
+            m = mv;
+        }
+        if (m != -INFINITY) {
+            const float mk = m * kLog2e;
+            for (int e = 0; e < k; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
+        }
+    };
+    const int n4 = (reinterpret_cast<uintptr_t>(x) & 15) == 0 ? n / 4 : 0;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x);
+    for (int b = 0; b < n4; b += 4 * g.n) {
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = b + k * g.n + g.t;
+            const float4 q = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            v[4 * k] = q.x;
+            v[4 * k + 1] = q.y;
+            v[4 * k + 2] = q.z;
+            v[4 * k + 3] = q.w;
+        }
+        fold(v, 16);
     }
+    for (int i = 4 * n4 + g.t; i < n; i += g.n) fold(x + i, 1);
     if (nan) set_status(status, XGR_DEV_NAN);
-    m = warp_max(m);
-    if (lane == 0) red[w] = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_pair_merge(m, s, m2, s2);
+    }
+    if (lane == 0) {
+        red[2 * w] = m;
+        red[2 * w + 1] = s;
+    }
     g.sync();
     m = red[0];
-    for (int k = 1; k < nw; ++k) m = fmaxf(m, red[k]);
+    s = red[1];
+    for (int k = 1; k < nw; ++k) lse_pair_merge(m, s, red[2 * k], red[2 * k + 1]);
     g.sync();   // red is reused
-    float s = 0.f;
-    if (m != -INFINITY) {
-        const float mk = m * kLog2e;
-        for (int i = g.t; i < n; i += g.n) s += ex2f(fmaf(x[i], kLog2e, -mk));
-    }
-    s = warp_sum(s);
-    if (lane == 0) red[w] = s;
-    g.sync();
-    s = red[0];
-    for (int k = 1; k < nw; ++k) s += red[k];
-    g.sync();
     return m + logf(s);
 }
 __device__ float block_lse(const float *x, int n, float *red, int32_t *status) {
@@ -802,16 +837,21 @@ __global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs
         mbar_expect_tx(bar, (uint32_t)V * 4u);
         bulk_g2s(smem_u32(x_of(row)), a.scores + row * V, (uint32_t)V * 4u, bar);
     };
-    if (tid == 0 && bulk) {
+    // The last thread (it has no window metadata to load while the windows hold
+    // far fewer rows than threads) sets up the slots and starts the first rows'
+    // bulk copies at once; the other threads meanwhile load the first window.
+    constexpr int kIssuer = kRowsThreads - 1;
+    static_assert(kRowsWin < kIssuer, "the issuing thread loads no window metadata");
+    if (tid == kIssuer && bulk) {
         for (int k = 0; k < nbuf; ++k) {
             mbar_init(smem_u32(&full[k]), 1);
             slot_row[k] = -1;
         }
         fence_mbar_init();
+        for (int64_t row = r0; row < min(r1, r0 + nbuf); ++row) issue(row);
     }
-    // Every load of a row's work happens per window, ahead of the rows: a global
-    // load issued behind the bulk traffic waits microseconds.  The first window's
-    // loads even go out before the first bulk copies.
+    // Every other load of a row's work happens per window, ahead of the rows: a
+    // global load issued behind the bulk traffic waits microseconds.
     for (int64_t w0 = r0; w0 < r1;) {
         // ---- window metadata: one round trip
         const int64_t wmax = min(r1, w0 + kRowsWin);
@@ -849,8 +889,6 @@ __global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs
             }
         }
         __syncthreads();
-        if (w0 == r0 && tid == 0 && bulk)
-            for (int64_t row = r0; row < min(r1, r0 + nbuf); ++row) issue(row);
         // ---- the window's rows: group g (256 threads, named barrier 1 + g) takes
         // rows w0 + g, w0 + g + 4, ...; when it is done with a row it starts the
         // copy of the row nbuf places later into the same slot

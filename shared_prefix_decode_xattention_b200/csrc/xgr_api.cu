@@ -16,6 +16,9 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMinChunk = 256;     // fewest keys per split-K work item
+// the separate merge kernel that split items need, in key units of the
+// tensor-core loop (one more dependent launch plus a few round trips)
+constexpr double kMergeKeys = 768.0;
 constexpr int64_t kSurvCap = 65536;   // selection survivors per request (more: exact path over the keys)
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
@@ -205,6 +208,13 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > 0; };
     // split factor per kind: the fewest waves x keys per item (+ a fixed
     // per-item overhead in key units), over the resident CTAs of the GPU
+    // A tensor-core segment left whole finishes its requests itself; splitting
+    // it adds the merge kernel, unless some segment needs that kernel anyway.
+    bool merge_anyway = false;
+    for (auto &sg : segs) {
+        if (!is_tc(sg)) merge_anyway = true;
+        for (int r : sg.members) merge_anyway |= nseg[r] > 1;
+    }
     auto pick_split = [&](bool tc) {
         int64_t base = 0, keys = 0, nseg_k = 0;
         for (auto &sg : segs) {
@@ -218,12 +228,13 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         const double L = (double)keys / nseg_k;
         const int64_t cap = tc ? c->num_sms : 2ll * c->num_sms;
         const double over = tc ? 384.0 : 128.0;
+        const double merge = (tc && !merge_anyway) ? kMergeKeys : 0.0;
         int64_t best = 1;
         double best_cost = 1e300;
         for (int64_t f = 1; f <= c->L.slots; ++f) {
             if (f > 1 && L / f < kMinChunk) break;
             const double waves = (double)((base * f + cap - 1) / cap);
-            const double cost = waves * (L / f + over);
+            const double cost = waves * (L / f + over) + (f > 1 ? merge : 0.0);
             if (cost < best_cost * 0.999) {
                 best_cost = cost;
                 best = f;
@@ -600,9 +611,9 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
             return XGR_ERR_CUDA;
         }
     }
-    // the merge kernel also writes the rows of dead beams; at step 0 only beam 0
-    // of each request is covered by Shared-stage work items
-    if (c->n_unfused[which] == 0 && (which == 1 || c->cfg.beam_width == 1)) {
+    // every request finished by the tensor-core kernel (which also writes the
+    // rows of beams that are not live): no merge launch
+    if (c->n_unfused[which] == 0) {
         if (c->cfg.vocab == 0) c->cur_step = step + 1;
         return XGR_OK;
     }
