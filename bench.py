@@ -63,11 +63,49 @@ def candidates_per_decode(w):
 # ---------------------------------------------------------------- clocks
 
 class Clocks:
+    """SM clock and clock-event reasons sampled while the timed region runs:
+    NVML polled from a background thread every half millisecond (the timed
+    region can be a few milliseconds), else nvidia-smi every 200 ms.  Only
+    reads the GPU's state."""
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("sw_power_cap", 0x4))
     FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
+        import threading
+        self.sm, self.mx, self.reasons = [], 0.0, set()
+        self.p = self.t = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            self.stop_ev = threading.Event()
+
+            def poll():
+                while not self.stop_ev.is_set():
+                    try:
+                        self.sm.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                        bits = get_reasons(h) if get_reasons else 0
+                        for n, b in self.REASONS:
+                            if bits & b:
+                                self.reasons.add(n)
+                    except Exception:
+                        return
+                    self.stop_ev.wait(0.0005)
+
+            self.t = threading.Thread(target=poll, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.t = None
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
@@ -77,31 +115,36 @@ class Clocks:
             self.p = None
 
     def stop(self):
-        if self.p is None:
-            return None
-        self.p.terminate()
-        try:
-            self.p.wait(timeout=5)
-        except Exception:
-            self.p.kill()
-        self.f.flush()
-        rows = [l.strip().split(", ") for l in open(self.f.name) if l.strip()]
-        os.unlink(self.f.name)
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        if self.t is not None:
+            self.stop_ev.set()
+            self.t.join(timeout=5)
+            sm = self.sm
+        elif self.p is not None:
+            self.p.terminate()
             try:
-                sm.append(float(r[0]))
-                mx = max(mx, float(r[1]))
-                for n, v in zip(names, r[3:7]):
-                    if v.strip().lower() == "active":
-                        reasons.add(n)
-            except (ValueError, IndexError):
-                continue
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+            self.f.flush()
+            rows = [l.strip().split(", ") for l in open(self.f.name) if l.strip()]
+            os.unlink(self.f.name)
+            sm = []
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for r in rows:
+                try:
+                    sm.append(float(r[0]))
+                    self.mx = max(self.mx, float(r[1]))
+                    for n, v in zip(names, r[3:7]):
+                        if v.strip().lower() == "active":
+                            self.reasons.add(n)
+                except (ValueError, IndexError):
+                    continue
+        else:
+            return None
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.mx,
+                "reasons": sorted(self.reasons), "samples": len(sm)}
 
 
 # ---------------------------------------------------------------- CPU oracle

@@ -501,12 +501,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr int kTabW = kMaxSteps + 1;   // per beam: slot of each token, then r * BW + b
             int *tab = reinterpret_cast<int *>(base + kOffU);
             const uint32_t tab_bytes = ((uint32_t)nbeam * kTabW * 4u + 127u) & ~127u;
-            // [tokens][beams][k | v][128] bf16, kStgRow bytes per (token, beam): the 16-byte
-            // pad puts the beams one warp reads at once in different banks
+            // then the two halves' partial dots [2][kMaxSteps][128] (fp32), then the staged
+            // rows [tokens][beams][k | v][128] (bf16), kStgRow bytes per (token, beam): the
+            // 16-byte pad puts the beams one warp reads at once in different banks
             constexpr uint32_t kStgRow = 528;
-            uint8_t *stg = base + kOffU + tab_bytes;
-            const int nbg = min(nbeam, (int)((kUBytes - tab_bytes) / kStgRow));   // beams per batch
-            const int tb = max(1, (int)((kUBytes - tab_bytes) / ((uint32_t)nbg * kStgRow)));   // tokens per batch
+            constexpr uint32_t kXdBytes = 2u * kMaxSteps * 128u * 4u;
+            float *xd = reinterpret_cast<float *>(base + kOffU + tab_bytes);
+            uint8_t *stg = base + kOffU + tab_bytes + kXdBytes;
+            const uint32_t room = kUBytes - tab_bytes - kXdBytes;
+            const int nbg = min(nbeam, (int)(room / kStgRow));   // beams per batch
+            const int tb = max(1, (int)(room / ((uint32_t)nbg * kStgRow)));   // tokens per batch
             // 1. the tile's first row of each beam reads the beam's slots (one round trip)
             if (ri.valid && (ri.hg == 0 || row == 0) && half == 0) {
                 const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
@@ -554,23 +558,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     cp_async_wait_all();
                     named_sync(1, kSoftmaxThreads);
-                    if (live && lb >= gb && lb < gb + ngb) {
+                    const bool mine = live && lb >= gb && lb < gb + ngb;
+                    if (mine) {   // partial dots over this thread's 64 head-dim columns
+#pragma unroll 1
+                        for (int ti = 0; ti < ntb; ++ti) {
+                            const uint8_t *kr = stg + (uint32_t)(ti * ngb + lb - gb) * kStgRow + col0 * 2;
+                            float acc = 0.f;
+#pragma unroll 4
+                            for (int c = 0; c < 8; ++c) {
+                                float qf[8], kf[8];
+                                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)),
+                                        qf);
+                                unpack8(*reinterpret_cast<const uint4 *>(kr + c * 16), kf);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
+                            }
+                            xd[(half * kMaxSteps + ti) * 128 + row] = acc;
+                        }
+                    }
+                    named_sync(1, kSoftmaxThreads);
+                    if (mine) {
 #pragma unroll 1
                         for (int ti = 0; ti < ntb; ++ti) {
                             const int i = i0 + ti;
                             if (tab[lb * kTabW + i] < 0) continue;
                             const uint8_t *kr = stg + (uint32_t)(ti * ngb + lb - gb) * kStgRow;
                             const uint8_t *vr = kr + 256;
-                            float acc = 0.f;
-#pragma unroll 4
-                            for (int c = 0; c < 16; ++c) {
-                                float qf[8], kf[8];
-                                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, c)), qf);
-                                unpack8(*reinterpret_cast<const uint4 *>(kr + c * 16), kf);
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
-                            }
-                            const float sc = acc * cscale;
+                            const float sc = (xd[ti * 128 + row] + xd[(kMaxSteps + ti) * 128 + row]) * cscale;
                             if (sc > m_u) {   // online softmax over the beam's tokens
                                 const float al = ex2(m_u - sc);
                                 l_u *= al;
