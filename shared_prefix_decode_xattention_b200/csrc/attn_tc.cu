@@ -281,6 +281,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     const WorkItem it = a.items[blockIdx.x];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    if (it.flags & 4) {   // zero-fill item: these CTAs run beside the attention on idle SMs
+        const int64_t row0 = ((int64_t)it.r0 * a.dims.BW + it.row_begin) * a.dims.Hq;   // first query row
+        const int64_t n = (int64_t)it.n_rows * a.dims.Hq;
+        uint4 *o = reinterpret_cast<uint4 *>(a.out + row0 * 128);
+        for (int64_t u = tid; u < n * 16; u += kTcThreads) o[u] = make_uint4(0, 0, 0, 0);
+        for (int64_t u = tid; u < n; u += kTcThreads) a.lse[row0 + u] = -INFINITY;
+        return;
+    }
     const int n_keys = it.key_end - it.key_begin;
     const int nchunks = (n_keys + kBlockN - 1) / kBlockN;
     const bool final_item = (it.flags & 1) != 0;
@@ -622,26 +630,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (live && half == 0) {   // O_0 holds the Unshared stage
                 m_used = m_u;
                 l = l_u;
-            }
-        }
-        if (final_item && a.nb == 1 && dm.BW > 1) {
-            // One live beam per request (step 0): while the first scores are in
-            // flight, write O = 0 and LSE = -inf for beams 1 .. BW-1 in this kv
-            // head's query heads, for every request whose rows start in this tile.
-            const int G = dm.G, ts = tid - 64;
-            const int m_lo = (it.row_begin + G - 1) / G;
-            const int m_hi = (it.row_begin + it.n_rows + G - 1) / G;
-            for (int m = m_lo; m < m_hi; ++m) {
-                const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + m];
-                const int64_t row1 = ((int64_t)r * dm.BW + 1) * dm.Hq + it.g * G;   // beam 1, head g*G
-                const int units = (dm.BW - 1) * G * 16;   // 16-byte pieces
-                for (int u = ts; u < units; u += kSoftmaxThreads) {
-                    const int bb = u / (G * 16), hg = (u / 16) % G;
-                    reinterpret_cast<uint4 *>(a.out + (row1 + (int64_t)bb * dm.Hq + hg) * 128)[u % 16] =
-                        make_uint4(0, 0, 0, 0);
-                }
-                for (int u = ts; u < (dm.BW - 1) * G; u += kSoftmaxThreads)
-                    a.lse[row1 + (int64_t)(u / G) * dm.Hq + u % G] = -INFINITY;
             }
         }
         const uint32_t s_col = (uint32_t)half * 128u;          // S buffer of this warpgroup

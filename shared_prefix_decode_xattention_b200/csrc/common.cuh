@@ -61,7 +61,10 @@ struct WorkItem {
     int32_t slot;        // partial slot this item writes for its rows
     int32_t flags;       // bit 0: final -- the item covers its requests' only KV segment
                          // whole, so it also runs the Unshared and Merging stages;
-                         // bit 1: its query rows form one TMA box (a single request)
+                         // bit 1: its query rows form one TMA box (a single request);
+                         // bit 2: zero fill -- no attention: O = 0 and LSE = -inf for
+                         // beams [row_begin, row_begin + n_rows) of request r0, every
+                         // query head (beams not live yet at step 0)
     int32_t r0;          // the item's first member request
     int32_t pad;
 };

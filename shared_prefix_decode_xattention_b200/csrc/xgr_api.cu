@@ -292,13 +292,36 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
                 }
         for (int r : sg.members) nslots[r] = (int32_t)(slot0 + splits);
     }
-    std::vector<WorkItem> items(items_small);
-    items.insert(items.end(), items_tc.begin(), items_tc.end());
     int unfused = 0;
     for (int r = 0; r < B; ++r) {
         if (fused[r]) nslots[r] = -1;   // the merge kernel skips this request
         else ++unfused;
     }
+    // One live beam per request (plan 0): when the tensor-core items finish every
+    // request, zero-fill items in the same launch write the other beams' rows on
+    // the SMs the attention leaves idle, so no merge kernel runs.
+    bool dead_rows = nb == cf.beam_width;   // plan 1: the items' tiles cover every beam
+    if (!dead_rows && unfused == 0 && !items_tc.empty()) {
+        const int64_t dead = (int64_t)B * (cf.beam_width - 1);
+        const int64_t idle = std::max<int64_t>(1, (int64_t)c->num_sms - (int64_t)items_tc.size() - B);
+        const int zb = (int)std::max<int64_t>(8, (dead + idle - 1) / idle);   // beams per zero item
+        const int64_t n_zero = (int64_t)B * ((cf.beam_width - 1 + zb - 1) / zb);
+        if ((int64_t)(items_small.size() + items_tc.size()) + n_zero <= c->L.item_cap) {
+            for (int r = 0; r < B; ++r)
+                for (int b0 = 1; b0 < cf.beam_width; b0 += zb) {
+                    WorkItem it{};
+                    it.r0 = r;
+                    it.row_begin = b0;
+                    it.n_rows = std::min(zb, cf.beam_width - b0);
+                    it.flags = 4;
+                    items_tc.push_back(it);
+                }
+            dead_rows = true;
+        }
+    }
+    if (!dead_rows && unfused == 0) unfused = 1;   // the merge kernel writes the dead rows
+    std::vector<WorkItem> items(items_small);
+    items.insert(items.end(), items_tc.begin(), items_tc.end());
     if ((int64_t)items.size() > c->L.item_cap || (int64_t)members.size() > c->L.member_cap)
         return XGR_ERR_CAPACITY;
     if (!items.empty() &&

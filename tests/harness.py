@@ -68,8 +68,9 @@ class GpuRun:
 
     def step(self, s, q, kn, vn, scores=None, flags=xgr.XGR_SCORES_LOGPROB) -> StepOut:
         w = self.w
-        out = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=self.device)
-        lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=self.device)
+        # NaN sentinels: every row the call must write (dead beams' zeros included) is checked
+        out = torch.full((w.B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=self.device)
+        lse = torch.full((w.B, w.BW, w.Hq), float("nan"), dtype=torch.float32, device=self.device)
         self.sess.decode_step(s, q, kn, vn, out, lse)
         if not w.V:
             return StepOut(out, lse, None)

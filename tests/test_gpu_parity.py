@@ -128,6 +128,19 @@ def test_ragged_prompts_and_split_k():
     decode_and_compare(w2, max_partials=6)
 
 
+def test_unshared_staging_in_batches():
+    """The tensor-core kernel stages each beam's own k/v rows in a 64 KB area;
+    when a tile's beams x tokens exceed it, it works in batches.  G = 1 (128
+    beams in a 128-row tile: two batches of beams, one token each) and G = 2 over
+    six steps (64 beams, one token per batch)."""
+    w = workloads.small(workloads.WORKLOADS[1], wid=105, B=2, prompt=(300, 300), BW=128, K=128,
+                        S=3, Hq=4, Hkv=4, D=128, V=256, n_items=20000)
+    decode_and_compare(w, beams_per_step=16)
+    w2 = workloads.small(workloads.WORKLOADS[1], wid=106, B=2, prompt=(200, 200), BW=64, K=64,
+                         S=6, Hq=4, Hkv=2, D=128, V=64, n_items=30000)
+    decode_and_compare(w2, beams_per_step=16)
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
