@@ -791,11 +791,11 @@ __global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectAr
 // -- in another (log-prob mode: then the tokens' scores), all into shared
 // memory.  In logits mode the score rows stream through nbuf slots by bulk
 // copies issued nbuf rows ahead, so the HBM traffic overlaps the work on
-// earlier rows.  Four groups of warps work on four rows at a time.  Per row:
+// earlier rows.  Eight groups of four warps work on eight rows at a time.  Per row:
 // the log-sum-exp (logits), each entry's key beside its CSR position, the
 // row's best key.
 constexpr int kRowsThreads = 1024;
-constexpr int kRowsGroups = 4;                       // rows in work at once
+constexpr int kRowsGroups = 8;   // rows in work at once (more, smaller groups measured faster)
 constexpr int kRowsGroup = kRowsThreads / kRowsGroups;
 constexpr int kRowsMaxBuf = 8;
 constexpr int kRowsWin = 256;     // rows per metadata window
@@ -809,8 +809,9 @@ __global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t full[kRowsMaxBuf];
     __shared__ int slot_row[kRowsMaxBuf];   // the row (index in the block) whose copy a slot holds
-    __shared__ float red_f[36 * kRowsGroups];
-    __shared__ uint64_t red_k[8 * kRowsGroups];
+    constexpr int kGroupWarps = kRowsGroup / 32;
+    __shared__ float red_f[2 * kGroupWarps * kRowsGroups];   // per group: (m, s) of each warp
+    __shared__ uint64_t red_k[kGroupWarps * kRowsGroups];   // per group: each warp's min
     __shared__ int win_end;
     const Dims dm = a.dims;
     const int V = dm.V, BW = dm.BW, tid = threadIdx.x;
@@ -919,7 +920,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs
                     set_status(a.status, XGR_DEV_TIMEOUT);
             }
             float lse = 0.f;
-            if (stage && live) lse = group_lse(x, V, red_f + 36 * gi, a.status, grp);
+            if (stage && live) lse = group_lse(x, V, red_f + 2 * kGroupWarps * gi, a.status, grp);
             const int beg = rp[i], end = rp[i + 1], n_e = max(0, end - beg);
             uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
             const int base = base_w[i];
@@ -943,7 +944,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs
                 if (e >= base && (int64_t)(e - base) < a.key_cap) keys[e - base] = key;
                 best = key < best ? key : best;
             }
-            best = group_min_u64(best, red_k + 8 * gi, grp);   // (its barriers end every read of the slot)
+            best = group_min_u64(best, red_k + kGroupWarps * gi, grp);   // (its barriers end every read of the slot)
             if (grp.t == 0) {
                 a.best[row] = best;
                 a.row_lse[row] = lse;
