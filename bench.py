@@ -280,15 +280,24 @@ def decode_required_bytes(w, logits_mode, nnz):
     return total
 
 
+def code_sha(path: str) -> str:
+    """SHA-256 of a CUDA/C++ source with its comments and whitespace removed:
+    the code the counters were taken on, unchanged by edits of comments."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"//[^\n]*|/\*.*?\*/", " ", text, flags=re.S)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
+
+
 def measured_traffic(call: str):
     """DRAM bytes per launch of a call, from the committed ncu summary
-    (profiles/traffic.json), or None when any of the call's kernel sources has
-    changed since the counters were taken (their SHA-256 no longer matches)."""
-    import hashlib
+    (profiles/traffic.json), or None when the code of any of the call's kernel
+    sources has changed since the counters were taken (code_sha differs)."""
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[call]
         for rel, sha in rec["sources"].items():
-            if hashlib.sha256(open(os.path.join(ROOT, rel), "rb").read()).hexdigest() != sha:
+            if code_sha(os.path.join(ROOT, rel)) != sha:
                 return None
         return rec["dram_bytes_per_launch"]
     except (OSError, KeyError, ValueError):

@@ -12,7 +12,7 @@
 //
 // One CTA per work item (kv head, 128-row tile, key range):
 //   warp 0      TMA producer: Q, then K and V chunks of 128 keys (two 64-column
-//               128-byte-swizzled boxes each) on separate three-stage rings;
+//               128-byte-swizzled boxes each) on separate two-stage rings;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
 //               S_j = Q K_j^T into TMEM buffer j % 2, O_{j%2} += P_j V_j with
 //               P_j read from tensor memory;
@@ -21,16 +21,18 @@
 //               keeps the running max and sum of its own accumulator O_h (lazy
 //               rescaling: O_h is rescaled only when the max grows by more than
 //               2^8), and writes P_j (bf16 pairs) over the first half of S_j's
-//               TMEM buffer, so no shared memory goes to P and the K and V rings
-//               are three deep.  The two warpgroups never wait for each other
+//               TMEM buffer, so no shared memory goes to P (it holds the
+//               Unshared staging area instead).  The two warpgroups never wait for each other
 //               inside the loop, so one's exponentials overlap the other's row
 //               maxima and TMEM traffic; at the end they swap (m, l) and merge
 //               O_0 and O_1 into the partial (O, m, l) or, for a request's only
 //               segment, the output.
 // In a request's only KV segment ("final" items) the Unshared and Merging
-// stages run here too: before the loop the softmax threads gather the beam's
-// own tokens (direct indices into the token-granular pool), seed O_0 and its
-// (m, l) with them, and append this step's k / v to the pool.
+// stages run here too: before the loop the softmax threads read the beams'
+// ancestry slots, stage the beams' own k / v rows (direct indices into the
+// token-granular pool) by cp.async, seed O_0 and its (m, l) with them, and
+// append this step's k / v to the pool.  Zero-fill items (step 0) only write
+// the rows of the beams that are not live yet.
 // Every wait on an mbarrier is bounded; on time-out the CTA records
 // XGR_DEV_TIMEOUT in the status word and unwinds (no trap, no hang).
 #include <cuda.h>

@@ -19,19 +19,23 @@
 // score, then lower parent beam, then lower token), so every comparison is an
 // exact integer comparison and ties resolve identically everywhere.
 //
-// Two shapes of work:
-//  * dense mask (one live beam per request): select_dense_kernel, one CTA per
-//    request, stages the beam's score row in shared memory with one bulk copy,
-//    takes its log-sum-exp (logits) and selects the best BW tokens there; the
-//    keys are recomputed from shared memory in every radix pass.
-//  * sparse (CSR) masks: select_rows_kernel, one CTA per beam row, stages the
-//    row (logits mode) with one bulk copy while it reads the row's CSR
-//    entries, and writes each entry's key beside its CSR position plus the
-//    row's best key; select_pick_kernel, a few CTAs per request, reduces tau
+// Kernels:
+//  * dense mask (one live beam per request, step 0): select_dense_kernel, one
+//    CTA per request, stages the beam's score row with one bulk copy, takes its
+//    log-sum-exp (logits), computes every token's key once into registers and
+//    radix-selects the best BW there.
+//  * sparse (CSR) masks: select_rows_kernel, one persistent 1024-thread CTA per
+//    SM over a contiguous block of beam rows: the rows' metadata and CSR tokens
+//    in two round trips, the score rows (logits mode) through bulk-copy slots,
+//    eight 128-thread groups on eight rows at a time; per row the log-sum-exp,
+//    each entry's key beside its CSR position and the row's best key.  Then one
+//    of two picks: select_pick_one_kernel (one CTA per request, when the
+//    request's pool fits its registers and shared memory) radix-selects the
+//    pool directly; select_pick_kernel (a few CTAs per request) reduces tau
 //    from the best keys, filters its slices of the request's keys and appends
-//    the survivors; the last CTA of the request to finish (an atomic ticket
-//    that the rows kernel resets) runs the exact selection, the ordering, the
-//    outputs and the rewiring.
+//    the survivors, and the request's last CTA to finish (an atomic ticket the
+//    rows kernel resets) selects among them.  Both end in finish_request: the
+//    ordering, the outputs and the rewiring.
 #include <algorithm>
 
 #include "async.cuh"
