@@ -141,6 +141,16 @@ def test_unshared_staging_in_batches():
     decode_and_compare(w2, beams_per_step=16)
 
 
+def test_shared_prefix_groups_with_beams():
+    """Beam search over requests that share prompts in groups: one KV segment
+    with several member requests per 128-row tile (Q staged by the threads, not
+    one TMA box; the staged Unshared rows of two requests in one tile) and, at
+    step 0, the zero fill of every member's beams that are not live yet."""
+    w = workloads.small(workloads.WORKLOADS[2], wid=107, B=4, groups=2, prompt=(600, 600), BW=16,
+                        K=16, S=3, Hq=8, Hkv=2, D=128, V=512, n_items=20000)
+    decode_and_compare(w)
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
