@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--scores", default="logits", choices=["logits", "logprob"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bw512", action="store_true",
+                    help="skip the BW = 512 attention figure (second half of the metric)")
     return ap.parse_args()
 
 
@@ -238,6 +240,85 @@ def algorithmic(w, s, logits_mode, nnz_step):
     att_flops = 4.0 * B * BW * Hq * D * (P + s + 1)
     sel_bytes = (B * BW * V * 4 if logits_mode else nnz_step * 4) + nnz_step * 4 + B * BW * 16
     return att_bytes, att_flops, sel_bytes
+
+
+def attention_bw512(dev, hbm, tf, src, reps=5):
+    """The metric's second half, "attention HBM GB/s vs peak (BW=512)": the staged
+    attention of the 512x512 candidate pool (gr-decode-pool-512x512: 32 requests,
+    4096-token prompts, 512 beams, Hq 32 / Hkv 8) at step 1, with the step's mask
+    built beside it as in the decode.  One graph of the phase, replayed with the
+    L2 flushed before each replay (the phase rewrites the same outputs and the
+    same Unshared slots, so every replay does the same work); required bytes
+    (shared KV once per request, the beams' Unshared tokens, this step's k/v
+    read and appended, q, O, LSE) per median replay time."""
+    import torch
+    import workloads
+    from shared_prefix_decode_xattention_b200 import xgr
+    from shared_prefix_decode_xattention_b200.session import Session, config_for
+    w = workloads.WORKLOADS[3]
+    items = workloads.items(w)
+    sess = Session(config_for(w), dev)
+    sess.build_trie(items)
+    for r in range(w.B):
+        k, v = workloads.shared_kv(w, w.shared_id(r), dev)
+        sess.prefill(r, w.shared_id(r), k, v)
+    del k, v
+    qkv = [workloads.step_qkv(w, s, dev) for s in range(2)]
+    out = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=dev)
+    par = torch.empty((w.B, w.BW), dtype=torch.int32, device=dev)
+    tok = torch.empty_like(par)
+    cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
+    nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
+    cur = torch.cuda.current_stream
+    side = torch.cuda.Stream(device=dev)
+    sess.begin(w.B, cur())
+    sc0 = workloads.step_logits(w, 0, dev)
+    m0 = sess.build_mask(0, cur())
+    sess.decode_step(0, *qkv[0], out, lse, cur())
+    sess.beam_select(0, sc0, xgr.XGR_SCORES_LOGITS, m0, par, tok, cum, nout, cur())
+    torch.cuda.synchronize()
+    del sc0
+    keep = []
+
+    def phase():
+        side.wait_stream(cur())
+        with torch.cuda.stream(side):
+            keep.append(sess.build_mask(1, side))
+        sess.decode_step(1, *qkv[1], out, lse, cur())
+        cur().wait_stream(side)
+
+    phase()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        phase()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        flush.zero_()
+        g.replay()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    status = sess.device_status()
+    del g
+    sess.close()
+    ms = statistics.median(ts)
+    att_bytes, att_flops, _ = algorithmic(w, 1, True, 0)
+    gbs = att_bytes / (ms / 1e3) / 1e9
+    tfl = att_flops / (ms / 1e3) / 1e12
+    return {"workload": f"{w.name}: B={w.B}, prompt {w.prompt[0]} tokens, BW={w.BW}, "
+                        f"Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, step 1 (mask built beside it)",
+            "ms": ms, "required_bytes": att_bytes, "achieved_gbs": gbs, "peak_gbs": hbm,
+            "frac": gbs / hbm, "tflops": tfl, "tensor_peak_tflops": tf, "tensor_frac": tfl / tf,
+            "peak_source": src, "l2": "flushed before each of the timed replays",
+            "device_status": status}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -557,6 +638,10 @@ def run_gpu(args, w):
         line["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, items, args.scores)
+    if world == 1 and not args.no_bw512:
+        del g_decode, g_phase
+        g_decode = g_phase = None
+        line["attention_bw512"] = attention_bw512(dev, hbm, tf, src)
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_decode, g_phase
