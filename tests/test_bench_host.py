@@ -1,0 +1,27 @@
+"""Host-side logic of bench.py (no GPU): the source hash that ties the counters
+in profiles/traffic.json to the code they were taken on, and the byte / flop
+model of the attention."""
+import bench
+import workloads
+
+def test_code_hash_ignores_comments_and_whitespace(tmp_path):
+    a = tmp_path / "a.cu"
+    a.write_text("int f(int x) {  // twice\n    return 2 * x;\n}\n/* done */\n")
+    b = tmp_path / "b.cu"
+    b.write_text("// a comment of its own\nint f(int x) {\n  return 2 * x; }\n")
+    c = tmp_path / "c.cu"
+    c.write_text("int f(int x) {\n    return 3 * x;\n}\n")
+    assert bench.code_sha(str(a)) == bench.code_sha(str(b))
+    assert bench.code_sha(str(a)) != bench.code_sha(str(c))
+
+
+def test_attention_byte_and_flop_model_of_the_512_pool():
+    # workload 3 at step 1: shared K/V once per request, the beams' earlier
+    # Unshared tokens, this step's k/v read and appended, q and O, LSE
+    w = workloads.WORKLOADS[3]
+    att_bytes, att_flops, _ = bench.algorithmic(w, 1, True, 0)
+    B, BW, Hq, Hkv, D, P = w.B, w.BW, w.Hq, w.Hkv, w.D, w.prompt[0]
+    expect = (2 * B * Hkv * P * D * 2 + 2 * B * BW * Hkv * D * 2 + 2 * B * BW * Hkv * D * 4
+              + 2 * B * BW * Hq * D * 2 + B * BW * Hq * 4)
+    assert att_bytes == expect
+    assert att_flops == 4.0 * B * BW * Hq * D * (P + 2)
