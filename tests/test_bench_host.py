@@ -4,6 +4,7 @@ model of the attention."""
 import bench
 import workloads
 
+
 def test_code_hash_ignores_comments_and_whitespace(tmp_path):
     a = tmp_path / "a.cu"
     a.write_text("int f(int x) {  // twice\n    return 2 * x;\n}\n/* done */\n")
