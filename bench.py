@@ -638,13 +638,11 @@ def run_gpu(args, w):
         line["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, items, args.scores)
+    del g_decode, g_phase   # released before the next workload's session
     if world == 1 and not args.no_bw512:
-        del g_decode, g_phase
-        g_decode = g_phase = None
         line["attention_bw512"] = attention_bw512(dev, hbm, tf, src)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_decode, g_phase
     sess.close()
     if world > 1:
         dist.barrier()

@@ -634,8 +634,8 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
             return XGR_ERR_CUDA;
         }
     }
-    // every request finished by the tensor-core kernel (which also writes the
-    // rows of beams that are not live): no merge launch
+    // every request finished by the tensor-core launch (its items cover every
+    // beam's rows, the not-yet-live ones at step 0 by zero-fill items): no merge
     if (c->n_unfused[which] == 0) {
         if (c->cfg.vocab == 0) c->cur_step = step + 1;
         return XGR_OK;
