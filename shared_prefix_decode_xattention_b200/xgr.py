@@ -9,6 +9,7 @@ library raises at once -- there is no fallback.
 from __future__ import annotations
 
 import ctypes
+import glob
 import os
 import re
 from typing import Optional
@@ -82,10 +83,12 @@ _lib = None
 
 
 def declared_functions() -> list:
-    """Names of the entry points include/xgr.h declares."""
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:xgr_status|const char \*|[a-z_]+)\s*\*?\s*(xgr_\w+)\s*\(",
-                                 text, flags=re.M)))
+    """Names of the entry points the headers in include/ declare."""
+    names = set()
+    for h in sorted(glob.glob(os.path.join(os.path.dirname(HEADER), "*.h"))):
+        names |= set(re.findall(r"^\s*(?:xgr_status|const char \*|[a-z_]+)\s*\*?\s*(xgr_\w+)\s*\(",
+                                open(h).read(), flags=re.M))
+    return sorted(names)
 
 
 def lib():
@@ -112,6 +115,17 @@ def lib():
         "xgr_get_sequences": [P, P, P],
         "xgr_device_status": [P, P, ctypes.POINTER(i32)],
         "xgr_beam_topk_noalloc": [i32, i32, i32, i32, P, i32, P, P, P, P, P, P, P, P, P, P],
+        # host-side batch former (include/xgr_sched.h)
+        "xgr_cht_create": [i32, ctypes.POINTER(P)],
+        "xgr_cht_destroy": [P],
+        "xgr_cht_insert": [P, i64, P, i64],
+        "xgr_cht_remove": [P, i64],
+        "xgr_cht_find_best": [P, ctypes.POINTER(i64), ctypes.POINTER(i32), ctypes.POINTER(i32),
+                              ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "xgr_cht_add_to_batch": [P, i64],
+        "xgr_cht_dispatch": [P, P, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "xgr_cht_counts": [P, ctypes.POINTER(i32), ctypes.POINTER(i32)],
+        "xgr_cht_form_batches": [P, i32, i32, P, i64, P, P, i32, ctypes.POINTER(i32)],
     }
     for name, args in sig.items():
         f = getattr(L, name)
