@@ -17,19 +17,23 @@ def _lib():
 
 
 # Chunks of 2 tokens.  A = [1 2|3 4|5 6], B = [1 2|3 4|7 8], C = [9 9|1 2],
-# D = [1 2|3 4|5 6|7] (3 full chunks), E = [1 2|8 8], inserted A..E.
-# max_batch 10, min_shared 1: A seeds (tip 3).  Missing: B 1, C 2, D 0, E 1 ->
-# D (depth 3).  Then B (1, older than E; depth 2, tip 2) -> E (depth
-# min(2, 1) = 1) -> C would leave depth 0 < 1: dispatch [A D B E] sharing 1
-# chunk; then C alone (its own 2 chunks).
+# D = [1 2|3 4|5 6|7] (3 full chunks), E = [1 2|8 8], F = [1 2|3 4|7 8|9 9],
+# inserted A..F.  Shared leading chunks: A-B 2, A-D 3, A-E 1, A-F 2, B-D 2,
+# B-E 1, B-F 3, D-E 1, D-F 2, E-F 1, C-anything 0.
+# max_batch 10, min_shared 1: A seeds (tip 3).  Missing: B 1, C 2, D 0, E 1,
+# F 2 -> D (depth 3).  B (1, older than E; depth 2, tip 2).  Now E 1 and F 1
+# (F's coverage comes from B, 3 chunks) -> E, older (depth min(2, 1) = 1).
+# Then F 1 against C 2 -> F (depth min(1, 2) = 1).  C would leave depth 0:
+# dispatch [A D B E F] sharing 1; then C alone (its own 2 chunks).
 # min_shared 2: A, D, B as before; E would leave depth 1 < 2: dispatch [A D B]
-# sharing 2; C seeds (E shares nothing with C: depth 0): [C] 2; [E] 2.
+# sharing 2.  C seeds; E (missing 2) would leave depth 0: [C] 2.  E seeds; F
+# (missing 3) would leave depth 1: [E] 2.  [F] 4.
 HAND = {"A": [1, 2, 3, 4, 5, 6], "B": [1, 2, 3, 4, 7, 8], "C": [9, 9, 1, 2],
-        "D": [1, 2, 3, 4, 5, 6, 7], "E": [1, 2, 8, 8]}
-IDS = {k: i + 1 for i, k in enumerate("ABCDE")}
+        "D": [1, 2, 3, 4, 5, 6, 7], "E": [1, 2, 8, 8], "F": [1, 2, 3, 4, 7, 8, 9, 9]}
+IDS = {k: i + 1 for i, k in enumerate("ABCDEF")}
 HAND_EXPECT = {
-    1: [(["A", "D", "B", "E"], 1), (["C"], 2)],
-    2: [(["A", "D", "B"], 2), (["C"], 2), (["E"], 2)],
+    1: [(["A", "D", "B", "E", "F"], 1), (["C"], 2)],
+    2: [(["A", "D", "B"], 2), (["C"], 2), (["E"], 2), (["F"], 4)],
 }
 
 
@@ -41,7 +45,7 @@ def _named(batches):
 @pytest.mark.parametrize("min_shared", [1, 2])
 def test_oracle_hand_example(min_shared):
     o = BatchFormerOracle(2)
-    for k in "ABCDE":
+    for k in "ABCDEF":
         o.insert(IDS[k], HAND[k])
     assert _named(o.form_batches(10, min_shared)) == HAND_EXPECT[min_shared]
 
@@ -49,7 +53,7 @@ def test_oracle_hand_example(min_shared):
 @pytest.mark.parametrize("min_shared", [1, 2])
 def test_tree_hand_example(min_shared):
     t = ChunkedHashTree(2)
-    for k in "ABCDE":
+    for k in "ABCDEF":
         t.insert(IDS[k], HAND[k])
     assert _named(t.form_batches(10, min_shared)) == HAND_EXPECT[min_shared]
 
@@ -57,7 +61,7 @@ def test_tree_hand_example(min_shared):
 def test_hand_example_step_by_step():
     """find_best's (missing, depth_after, delta, w) on the example, both sides."""
     o, t = BatchFormerOracle(2), ChunkedHashTree(2)
-    for k in "ABCDE":
+    for k in "ABCDEF":
         o.insert(IDS[k], HAND[k])
         t.insert(IDS[k], HAND[k])
     # empty batch: the oldest (A) seeds; it keeps its 3 chunks; D also holds
@@ -69,9 +73,9 @@ def test_hand_example_step_by_step():
     assert o.find_best() == t.find_best() == (IDS["D"], 0, 3, 0, 0)
     for side in (o, t):
         side.add(IDS["D"])
-    # B: missing 1, depth 2 (delta 1); A and D are in the batch, no waiting
-    # request shares B's first 2 chunks
-    assert o.find_best() == t.find_best() == (IDS["B"], 1, 2, 1, 0)
+    # B: missing 1, depth 2 (delta 1); of the waiting requests F shares B's
+    # first 2 chunks, so w = 1
+    assert o.find_best() == t.find_best() == (IDS["B"], 1, 2, 1, 1)
 
 
 def _family_workload(rng, n_req, n_fam, chunk, vocab=50):
@@ -194,3 +198,67 @@ def test_long_running_tree_compacts_and_stays_exact():
             o.insert(i, r)
             t.insert(i, r)
         assert t.form_batches(6, 1) == o.form_batches(6, 1), f"round {rnd}"
+
+
+def _hand_outcomes(oracle_cls):
+    """Everything the hand example pins: both formations and the step-by-step
+    find_best values."""
+    res = []
+    for ms in (1, 2):
+        o = oracle_cls(2)
+        for k in "ABCDEF":
+            o.insert(IDS[k], HAND[k])
+        res.append(_named(o.form_batches(10, ms)))
+    o = oracle_cls(2)
+    for k in "ABCDEF":
+        o.insert(IDS[k], HAND[k])
+    steps = [o.find_best()]
+    o.add(IDS["A"])
+    steps.append(o.find_best())
+    o.add(IDS["D"])
+    steps.append(o.find_best())
+    return res, steps
+
+
+def _mutant(name):
+    """A copy of the oracle with one plausible mistake planted."""
+    class M(BatchFormerOracle):
+        pass
+    if name == "newest first on ties":
+        def find_best(self):
+            w0 = list(self.waiting)
+            self.waiting = w0[::-1]
+            try:
+                return BatchFormerOracle.find_best(self)
+            finally:
+                self.waiting = w0
+        M.find_best = find_best
+    elif name == "coverage by the least-sharing member":
+        M.missing = lambda self, r: (self.chunks(r) if not self.batch
+                                     else self.chunks(r) - min(self.shared(r, m) for m in self.batch))
+    elif name == "tip as the deepest member":
+        M.tip = lambda self: (0 if not self.batch else
+                              max(self.shared(m, self.batch[0]) if m != self.batch[0]
+                                  else self.chunks(m) for m in self.batch))
+    elif name == "stop at equality":
+        def form_batches(self, max_batch, min_shared_chunks):
+            return BatchFormerOracle.form_batches(self, max_batch, min_shared_chunks + 1)
+        M.form_batches = form_batches
+    elif name == "partial chunk counted":
+        M.chunks = lambda self, r: -(-len(self.tokens[r]) // self.C)
+    elif name == "w counts the candidate":
+        def find_best(self):
+            b = BatchFormerOracle.find_best(self)
+            return None if b is None else b[:4] + (b[4] + (1 if b[2] > 0 else 0),)
+        M.find_best = find_best
+    return M
+
+
+@pytest.mark.parametrize("name", ["newest first on ties", "coverage by the least-sharing member",
+                                  "tip as the deepest member", "stop at equality",
+                                  "partial chunk counted", "w counts the candidate"])
+def test_planted_mistakes_fail_the_hand_pins(name):
+    good = ([HAND_EXPECT[1], HAND_EXPECT[2]],
+            [(IDS["A"], 3, 3, 0, 1), (IDS["D"], 0, 3, 0, 0), (IDS["B"], 1, 2, 1, 1)])
+    assert _hand_outcomes(BatchFormerOracle) == good
+    assert _hand_outcomes(_mutant(name)) != good, name
