@@ -236,7 +236,11 @@ xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_co
  * may set a kernel attribute, so make that first call before any stream capture.
  * All calls share the array: calls that overlap on the GPU race and must be
  * serialised by the caller.  NaN scores and out-of-range mask tokens are
- * skipped, as in the context path, but not reported.  Host-side argument
+ * skipped, as in the context path, but not reported: the kernels set bits in
+ * a status word inside the static array that this call neither clears nor
+ * reads (use the context path and xgr_device_status to diagnose such inputs).
+ * The tensor arguments must be device memory of the stated element types;
+ * the call cannot check that.  Host-side argument
  * errors return XGR_ERR_ARG / XGR_ERR_SHAPE; nothing is enqueued then. */
 xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_width, int32_t top_k,
                                  int32_t vocab, const float *d_scores, int32_t flags,

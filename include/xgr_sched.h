@@ -36,13 +36,17 @@
  *    depth_after - 1 is the batch's (the page's count of requests sharing the
  *    new depth; 0 when depth_after is 0).
  *  - Stopping policy (xgr_cht_form_batches): the page's learned policies need
- *    live traffic and are not built; the static rule here adds the best
- *    request while the batch holds fewer than max_batch requests and
- *    depth_after >= min_shared_chunks, and dispatches otherwise.
+ *    live traffic and are not built; the static rule here adds, while the
+ *    batch holds fewer than max_batch requests, the best waiting request among
+ *    those whose depth_after >= min_shared_chunks (smallest missing count,
+ *    then the earliest inserted), and dispatches when none qualifies.  A
+ *    request that shares too little with the batch (a short or unrelated
+ *    prompt: few chunks, so a small missing count) is passed over, not allowed
+ *    to end the batch while requests sharing its prefix still wait.
  *
  * Conventions: host memory only, no CUDA calls; a handle is not thread-safe
- * (one caller at a time); request ids are any int64 unique among live
- * requests.  Every call returns an xgr_status (XGR_OK = 0); XGR_ERR_ARG for a
+ * (one caller at a time); request ids are non-negative int64s unique among
+ * live requests (a negative id is XGR_ERR_ARG: -1 reports "none waiting").  Every call returns an xgr_status (XGR_OK = 0); XGR_ERR_ARG for a
  * null handle or pointer, an unknown or duplicate id, or max_batch < 1;
  * XGR_ERR_STATE for a request in the wrong state (adding or removing one that
  * is not waiting); XGR_ERR_SHAPE for a negative length or a chunk size < 1.

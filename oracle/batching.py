@@ -14,7 +14,8 @@ the loss of shared prefix depth (delta) and the number of waiting requests
 that share the new depth (w), and adds the request or dispatches the batch.
 The readings of what the page leaves open (full chunks only, the
 earliest-inserted request seeding a batch and breaking ties, depth measured
-against the first member, the static stopping rule) are the ones stated in the
+against the first member, the static policy that adds the best request whose
+depth stays at or above a floor and passes over the others) are the ones stated in the
 library's header, restated here in terms of tokens.
 
 Parity status: pinned by tests/test_sched_cht.py (a hand-derived example).
@@ -89,6 +90,20 @@ class BatchFormerOracle:
                     w += 1
         return r, miss, d, delta, w
 
+    def depth_after(self, r: int) -> int:
+        """Chunks the batch would still share with r added: min(tip, shared with the first member)."""
+        return min(self.tip(), self.shared(r, self.batch[0]))
+
+    def best_passing(self, floor: int) -> Optional[int]:
+        """The static policy's choice: among the waiting requests whose depth_after
+        reaches the floor, the one with the smallest missing count, then the
+        earliest inserted; None when none qualifies."""
+        order = {q: i for i, q in enumerate(self.waiting)}
+        ok = [q for q in self.waiting if self.depth_after(q) >= floor]
+        if not ok:
+            return None
+        return min(ok, key=lambda q: (self.missing(q), order[q]))
+
     def add(self, r: int) -> None:
         self.waiting.remove(r)
         self.batch.append(r)
@@ -107,9 +122,9 @@ class BatchFormerOracle:
         while self.waiting:
             self.add(self.find_best()[0])   # the earliest-inserted request seeds the batch
             while len(self.batch) < max_batch:
-                best = self.find_best()
-                if best is None or best[2] < min_shared_chunks:
+                r = self.best_passing(min_shared_chunks)
+                if r is None:
                     break
-                self.add(best[0])
+                self.add(r)
             res.append(self.dispatch())
         return res

@@ -95,6 +95,33 @@ struct xgr_cht {
         }
         return -1;
     }
+    // The best waiting request whose depth_after reaches `floor` (smallest missing
+    // count, then the earliest inserted), or -1.  Entries that fail the floor are
+    // set aside while the heap is searched and pushed back afterwards, so a
+    // request that shares nothing with the batch (a short or unrelated prompt,
+    // whose missing count is small) does not end the batch while requests that
+    // share its prefix still wait.
+    int32_t best_passing(int32_t floor) {
+        if (n_waiting == 0 || batch.empty()) return -1;
+        std::vector<Entry> aside;
+        int32_t found = -1;
+        while (!by_missing.empty()) {
+            const Entry e = by_missing.top();
+            const int32_t i = std::get<2>(e);
+            if (reqs[i].state != kWaiting || reqs[i].missing != std::get<0>(e)) {
+                by_missing.pop();   // stale
+                continue;
+            }
+            if (shared_with_tip(reqs[i]) >= floor) {
+                found = i;
+                break;
+            }
+            aside.push_back(e);
+            by_missing.pop();
+        }
+        for (const Entry &e : aside) by_missing.push(e);
+        return found;
+    }
     void add(int32_t i) {
         Req &r = reqs[i];
         const int32_t from = covered(r);
@@ -178,7 +205,7 @@ xgr_status xgr_cht_destroy(xgr_cht *t) {
 }
 
 xgr_status xgr_cht_insert(xgr_cht *t, int64_t request_id, const int32_t *h_tokens, int64_t n_tokens) {
-    if (!t || (n_tokens > 0 && !h_tokens)) return XGR_ERR_ARG;
+    if (!t || (n_tokens > 0 && !h_tokens) || request_id < 0) return XGR_ERR_ARG;
     if (n_tokens < 0) return XGR_ERR_SHAPE;
     if (t->live.count(request_id)) return XGR_ERR_ARG;
     Req r;
@@ -276,7 +303,7 @@ xgr_status xgr_cht_form_batches(xgr_cht *t, int32_t max_batch, int32_t min_share
     int32_t nb = 0;
     auto close = [&]() {
         h_shared[nb] = t->tip;
-        const int32_t k = t->dispatch(h_ids + at, (int32_t)(cap_ids - at));
+        const int32_t k = t->dispatch(h_ids + at, (int32_t)std::min<int64_t>(cap_ids - at, INT32_MAX));
         h_sizes[nb++] = k;
         at += k;
     };
@@ -284,8 +311,8 @@ xgr_status xgr_cht_form_batches(xgr_cht *t, int32_t max_batch, int32_t min_share
     while (t->n_waiting > 0) {
         t->add(t->best());   // the oldest waiting request seeds the batch
         while ((int32_t)t->batch.size() < max_batch) {
-            const int32_t i = t->best();
-            if (i < 0 || t->shared_with_tip(t->reqs[i]) < min_shared_chunks) break;
+            const int32_t i = t->best_passing(min_shared_chunks);
+            if (i < 0) break;
             t->add(i);
         }
         close();

@@ -33,6 +33,7 @@ XGR_DEV_NAN = 1
 XGR_DEV_INDEX = 2
 XGR_DEV_MASK = 4
 XGR_DEV_CAPACITY = 8
+XGR_DEV_TIMEOUT = 16
 
 XGR_SCORES_LOGPROB = 0
 XGR_SCORES_LOGITS = 1
@@ -233,7 +234,26 @@ def xgr_device_status(ctx: int, stream=None) -> int:
 def xgr_beam_topk_noalloc(n_requests: int, beam_width: int, top_k: int, vocab: int, scores,
                           flags: int, cum, n_live, bits, row_ptr, cols, parent, token, cum_out,
                           n_out, stream=None) -> None:
-    """Masked top-K without a context or any allocation (see include/xgr.h)."""
+    """Masked top-K without a context or any allocation (see include/xgr.h).
+
+    Tensor arguments must be contiguous CUDA tensors of the types the header
+    states (the call itself cannot see a host pointer or a wrong element size,
+    and it reports no device status): scores, cum, cum_out fp32; n_live,
+    row_ptr, cols, parent, token, n_out int32; bits int32 or uint32.  Integer
+    addresses are passed through unchecked."""
+    import torch
+    want = {"scores": (scores, (torch.float32,)), "cum": (cum, (torch.float32,)),
+            "n_live": (n_live, (torch.int32,)), "bits": (bits, (torch.int32, torch.uint32)),
+            "row_ptr": (row_ptr, (torch.int32,)), "cols": (cols, (torch.int32,)),
+            "parent": (parent, (torch.int32,)), "token": (token, (torch.int32,)),
+            "cum_out": (cum_out, (torch.float32,)), "n_out": (n_out, (torch.int32,))}
+    for name, (t, dtypes) in want.items():
+        if t is None or isinstance(t, int):
+            continue
+        if not (t.is_cuda and t.is_contiguous() and t.dtype in dtypes):
+            raise XgrError(f"xgr_beam_topk_noalloc({name}: {t.dtype}, "
+                           f"{'cuda' if t.is_cuda else 'host'}, "
+                           f"{'contiguous' if t.is_contiguous() else 'strided'})", XGR_ERR_ARG)
     _check("xgr_beam_topk_noalloc", lib().xgr_beam_topk_noalloc(
         n_requests, beam_width, top_k, vocab, _ptr(scores), flags, _ptr(cum), _ptr(n_live),
         _ptr(bits), _ptr(row_ptr), _ptr(cols), _ptr(parent), _ptr(token), _ptr(cum_out),

@@ -180,6 +180,14 @@ def compare_select_tie_aware(so: StepOut, r: int, dec, scores_r: np.ndarray, mas
     pr, tk, cm, n, _ = oracle.select_logits(dec.cum, scores_r, row_ptr, cols, dec.BW, dec.n_live)
     assert so.n_out[r] == n, what
     gp, gt = so.parent[r][:n], so.token[r][:n]
+    # every choice is a distinct candidate of the oracle's mask for this step
+    assert len(set(zip(gp.tolist(), gt.tolist()))) == n, f"{what}: a (parent, token) repeats"
+    for p_, t_ in zip(gp.tolist(), gt.tolist()):
+        assert 0 <= p_ < dec.n_live, f"{what}: parent {p_} not live"
+        row = cols[row_ptr[p_]:row_ptr[p_ + 1]] if s else cols
+        assert t_ in set(row.tolist()), f"{what}: token {t_} not valid for parent {p_}"
+    dead = so.parent[r][n:]
+    assert np.all(dead == -1) and np.all(so.token[r][n:] == -1), f"{what}: dead slots"
     gk = oracle.logits_keys(dec.cum, scores_r, list(zip(gp.tolist(), gt.tolist())))
     # the GPU's k-th choice has the oracle's k-th best score up to near-ties
     assert np.all(np.abs(np.sort(gk)[::-1] - cm[:n]) <= TIE_EPS), f"{what}: selection differs"

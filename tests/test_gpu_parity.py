@@ -102,6 +102,18 @@ def test_workload3_sampled():
     decode_and_compare(workloads.WORKLOADS[3], requests=[0, 13, 22, 31], beams_per_step=12)
 
 
+def test_workload3_logits_sampled():
+    """Logits mode at the 512x512 pool: row log-sum-exp over V = 8192 and pools
+    above 32K entries (the multi-CTA threshold pick)."""
+    decode_and_compare(workloads.WORKLOADS[3], mode="logits", requests=[3, 30], beams_per_step=8)
+
+
+def test_workload5_logits_sampled():
+    """Logits mode over V = 16384 with ragged long prompts and four steps."""
+    decode_and_compare(workloads.WORKLOADS[5], mode="logits", requests=[7, 100],
+                       beams_per_step=6)
+
+
 def test_workload4_homogeneous():
     decode_and_compare(workloads.WORKLOADS[4])
 

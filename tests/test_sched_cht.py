@@ -25,15 +25,15 @@ def _lib():
 # (F's coverage comes from B, 3 chunks) -> E, older (depth min(2, 1) = 1).
 # Then F 1 against C 2 -> F (depth min(1, 2) = 1).  C would leave depth 0:
 # dispatch [A D B E F] sharing 1; then C alone (its own 2 chunks).
-# min_shared 2: A, D, B as before; E would leave depth 1 < 2: dispatch [A D B]
-# sharing 2.  C seeds; E (missing 2) would leave depth 0: [C] 2.  E seeds; F
-# (missing 3) would leave depth 1: [E] 2.  [F] 4.
+# min_shared 2: A, D, B as before (tip 2); E (missing 1) would leave depth 1 < 2
+# and is passed over; F (missing 1, younger) keeps depth 2: [A D B F] sharing 2.
+# C seeds; E (missing 2) would leave depth 0: [C] 2.  E seeds alone: [E] 2.
 HAND = {"A": [1, 2, 3, 4, 5, 6], "B": [1, 2, 3, 4, 7, 8], "C": [9, 9, 1, 2],
         "D": [1, 2, 3, 4, 5, 6, 7], "E": [1, 2, 8, 8], "F": [1, 2, 3, 4, 7, 8, 9, 9]}
 IDS = {k: i + 1 for i, k in enumerate("ABCDEF")}
 HAND_EXPECT = {
     1: [(["A", "D", "B", "E", "F"], 1), (["C"], 2)],
-    2: [(["A", "D", "B"], 2), (["C"], 2), (["E"], 2), (["F"], 4)],
+    2: [(["A", "D", "B", "F"], 2), (["C"], 2), (["E"], 2)],
 }
 
 
@@ -78,6 +78,62 @@ def test_hand_example_step_by_step():
     assert o.find_best() == t.find_best() == (IDS["B"], 1, 2, 1, 1)
 
 
+# A request sharing nothing with the batch (Z: shorter than a chunk, so it
+# misses no chunk at all) arrives between requests that share A's whole
+# prompt.  Chunks of 4; A = 32 tokens (8 chunks), Z = 2 tokens (0 chunks),
+# B and C = A's tokens + 8 of their own (10 chunks); inserted A, Z, B, C;
+# max_batch 16, min_shared 1.  A seeds (tip 8).  Z ranks first by missing
+# count (0) but would leave depth 0 < 1: passed over.  B (missing 2, depth 8,
+# older than C) joins, then C (missing 2: its first 8 chunks are covered).
+# Only Z is left and it fails the floor: dispatch [A B C] sharing 8, then [Z]
+# sharing 0 (it has no full chunk).
+SHORT = {"A": list(range(32)), "Z": [100, 101], "B": list(range(32)) + list(range(40, 48)),
+         "C": list(range(32)) + list(range(50, 58))}
+SHORT_IDS = {"A": 10, "Z": 11, "B": 12, "C": 13}
+SHORT_EXPECT = [(["A", "B", "C"], 8), (["Z"], 0)]
+
+
+# Coverage counts the member sharing the MOST with a candidate.  Chunks of 1;
+# P = [1 2 3], Q = [1 2 9], X = [1 2 3 4], W = [1 5], inserted P, Q, X, W;
+# max_batch 10, min_shared 1.  P seeds (tip 3): Q, X and W all miss one chunk
+# -> Q, the oldest (tip 2).  X now misses 4 - max(3 with P, 2 with Q) = 1 and
+# W misses 1: X, older, joins (depth 2), then W (depth 1).  [P Q X W] sharing 1.
+MAXCOV = {"P": [1, 2, 3], "Q": [1, 2, 9], "X": [1, 2, 3, 4], "W": [1, 5]}
+MAXCOV_IDS = {"P": 20, "Q": 21, "X": 22, "W": 23}
+MAXCOV_EXPECT = [(["P", "Q", "X", "W"], 1)]
+
+
+def _maxcov_named(batches):
+    inv = {v: k for k, v in MAXCOV_IDS.items()}
+    return [([inv[i] for i in ids], sh) for ids, sh in batches]
+
+
+def test_coverage_by_the_most_sharing_member():
+    for side in (BatchFormerOracle(1), ChunkedHashTree(1)):
+        for k in "PQXW":
+            side.insert(MAXCOV_IDS[k], MAXCOV[k])
+        assert _maxcov_named(side.form_batches(10, 1)) == MAXCOV_EXPECT, type(side).__name__
+
+
+def _short_named(batches):
+    inv = {v: k for k, v in SHORT_IDS.items()}
+    return [([inv[i] for i in ids], sh) for ids, sh in batches]
+
+
+def test_short_prompt_does_not_end_a_batch():
+    for side in (BatchFormerOracle(4), ChunkedHashTree(4)):
+        for k in "AZBC":
+            side.insert(SHORT_IDS[k], SHORT[k])
+        assert _short_named(side.form_batches(16, 1)) == SHORT_EXPECT, type(side).__name__
+
+
+def test_negative_request_id_is_rejected():
+    t = ChunkedHashTree(2)
+    with pytest.raises(xgr.XgrError) as e:
+        t.insert(-1, [1, 2, 3])
+    assert e.value.status == xgr.XGR_ERR_ARG
+
+
 def _family_workload(rng, n_req, n_fam, chunk, vocab=50):
     """Requests from a few prompt families: a family prefix, then a private
     random tail; some share longer sub-prefixes, some are shorter than a chunk."""
@@ -99,7 +155,7 @@ def test_tree_matches_oracle_on_random_families(seed):
     max_batch = [1, 3, 8, 1000][seed % 4]
     min_shared = [0, 1, 2][seed % 3]
     o, t = BatchFormerOracle(chunk), ChunkedHashTree(chunk)
-    ids = rng.permutation(10_000)[:len(reqs)] - 5000   # arbitrary, some negative
+    ids = rng.permutation(10_000)[:len(reqs)]   # arbitrary non-negative ids
     for i, r in zip(ids, reqs):
         o.insert(int(i), r)
         t.insert(int(i), r)
@@ -201,9 +257,17 @@ def test_long_running_tree_compacts_and_stays_exact():
 
 
 def _hand_outcomes(oracle_cls):
-    """Everything the hand example pins: both formations and the step-by-step
-    find_best values."""
+    """Everything the hand examples pin: both formations, the short-prompt
+    formation and the step-by-step find_best values."""
     res = []
+    o = oracle_cls(4)
+    for k in "AZBC":
+        o.insert(SHORT_IDS[k], SHORT[k])
+    res.append(_short_named(o.form_batches(16, 1)))
+    o = oracle_cls(1)
+    for k in "PQXW":
+        o.insert(MAXCOV_IDS[k], MAXCOV[k])
+    res.append(_maxcov_named(o.form_batches(10, 1)))
     for ms in (1, 2):
         o = oracle_cls(2)
         for k in "ABCDEF":
@@ -240,6 +304,19 @@ def _mutant(name):
         M.tip = lambda self: (0 if not self.batch else
                               max(self.shared(m, self.batch[0]) if m != self.batch[0]
                                   else self.chunks(m) for m in self.batch))
+    elif name == "dispatch when the best request fails the floor":
+        def form_batches(self, max_batch, min_shared_chunks):
+            res = []
+            while self.waiting:
+                self.add(self.find_best()[0])
+                while len(self.batch) < max_batch:
+                    best = self.find_best()
+                    if best is None or best[2] < min_shared_chunks:
+                        break
+                    self.add(best[0])
+                res.append(self.dispatch())
+            return res
+        M.form_batches = form_batches
     elif name == "stop at equality":
         def form_batches(self, max_batch, min_shared_chunks):
             return BatchFormerOracle.form_batches(self, max_batch, min_shared_chunks + 1)
@@ -255,10 +332,11 @@ def _mutant(name):
 
 
 @pytest.mark.parametrize("name", ["newest first on ties", "coverage by the least-sharing member",
+                                  "dispatch when the best request fails the floor",
                                   "tip as the deepest member", "stop at equality",
                                   "partial chunk counted", "w counts the candidate"])
 def test_planted_mistakes_fail_the_hand_pins(name):
-    good = ([HAND_EXPECT[1], HAND_EXPECT[2]],
+    good = ([SHORT_EXPECT, MAXCOV_EXPECT, HAND_EXPECT[1], HAND_EXPECT[2]],
             [(IDS["A"], 3, 3, 0, 1), (IDS["D"], 0, 3, 0, 0), (IDS["B"], 1, 2, 1, 1)])
     assert _hand_outcomes(BatchFormerOracle) == good
     assert _hand_outcomes(_mutant(name)) != good, name
