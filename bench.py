@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bw512", action="store_true",
                     help="skip the BW = 512 attention figure (second half of the metric)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the prefix-batch and long-history workload figures")
     return ap.parse_args()
 
 
@@ -181,8 +183,11 @@ def oracle_decode_sample(w, items, sorted_items, requests, scores_mode):
 
 
 def cpu_baseline(w, items, scores_mode, budget_s=20.0):
+    """The oracle on the host cores: whole decodes of requests 0, 1, ... until
+    about budget_s/2 of all-core time, then the same requests with one thread."""
     import oracle
     si = oracle.SortedItems(items, w.V)
+    cores = oracle.num_threads()
     secs, cands = oracle_decode_sample(w, items, si, [0], scores_mode)
     reqs = [0]
     r = 1
@@ -192,9 +197,18 @@ def cpu_baseline(w, items, scores_mode, budget_s=20.0):
         cands += c
         reqs.append(r)
         r += 1
-    return {"value": cands / secs, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+    single = None
+    try:
+        oracle.set_num_threads(1)
+        t1, c1 = oracle_decode_sample(w, items, si, reqs[:1], scores_mode)
+        single = {"value": c1 / t1, "cores": 1,
+                  "sample": f"full {w.S}-step decode of request 0 ({c1} candidates in {t1:.2f} s)"}
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": cands / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"full {w.S}-step decode of {len(reqs)} of {w.B} requests "
-                      f"({cands} candidates in {secs:.2f} s)"}
+                      f"({cands} candidates in {secs:.2f} s)",
+            "single_thread": single}
 
 
 def run_reference(args, w):
@@ -208,8 +222,8 @@ def run_reference(args, w):
     for _ in range(args.warmup):
         oracle_decode_sample(w, items, si, [0], args.scores)
     secs, cands = 0.0, 0
-    for i in range(args.steps):
-        t, c = oracle_decode_sample(w, items, si, [i % w.B], args.scores)
+    for i in range(args.steps):   # each step: the whole batch, as the GPU arm
+        t, c = oracle_decode_sample(w, items, si, list(range(w.B)), args.scores)
         secs += t
         cands += c
     value = cands / secs
@@ -220,7 +234,7 @@ def run_reference(args, w):
             "impl": "reference", "config": workload_config(w, args.scores),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle",
-                             "sample": f"each step: full {w.S}-step decode of one request"},
+                             "sample": f"each step: full {w.S}-step decode of all {w.B} requests"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -319,6 +333,186 @@ def attention_bw512(dev, hbm, tf, src, reps=5):
             "frac": gbs / hbm, "tflops": tfl, "tensor_peak_tflops": tf, "tensor_frac": tfl / tf,
             "peak_source": src, "l2": "flushed before each of the timed replays",
             "device_status": status}
+
+
+def _timed_graph(fn, dev, reps=5, warm=3):
+    """Median device time (ms) of one CUDA graph of fn, replayed with the L2
+    flushed (a 256 MiB write) before every replay."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warm):
+        flush.zero_()
+        g.replay()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    del g
+    return statistics.median(ts)
+
+
+def prefix_batches(dev, hbm, tf, src):
+    """Feather's comparison (Feather page, "Results": prefix-homogeneous batches
+    against heterogeneous ones), kernel side: the staged attention of the
+    prefix-shared workload (64 requests, beam 1, 8192-token prefixes shared in 4
+    groups of 16, private suffixes of 256-2048 tokens) against the same request
+    lengths with 64 distinct prefixes.  One decode step each, replayed as a graph
+    with the L2 flushed; required bytes = every prefix and suffix K/V once, q, O,
+    LSE, this step's k/v read and appended."""
+    import torch
+    import workloads
+    from shared_prefix_decode_xattention_b200 import xgr
+    from shared_prefix_decode_xattention_b200.session import Session, config_for
+    out = {}
+    for kind, w in (("homogeneous", workloads.WORKLOADS[4]),
+                    ("heterogeneous", workloads.heterogeneous(workloads.WORKLOADS[4]))):
+        sess = Session(config_for(w), dev)
+        for sid in range(w.n_shared):
+            members = [r for r in range(w.B) if w.shared_id(r) == sid]
+            k, v = workloads.shared_kv(w, sid, dev)
+            sess.prefill(members[0], sid, k, v)
+            for r in members[1:]:
+                sess.link(r, sid)
+            del k, v
+        for r in range(w.B):
+            k, v = workloads.suffix_kv(w, r, dev)
+            sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+            del k, v
+        q, kn, vn = workloads.step_qkv(w, 0, dev)
+        o = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=dev)
+        sess.begin(w.B)
+        cur = torch.cuda.current_stream
+
+        def step():
+            sess.begin(w.B, cur())
+            sess.decode_step(0, q, kn, vn, o, lse, cur())
+
+        ms = _timed_graph(step, dev)
+        status = sess.device_status()
+        sess.close()
+        kv_tok = int(workloads.prompt_lengths(w).sum()) + int(workloads.suffix_lengths(w).sum())
+        req = (2 * w.Hkv * w.D * 2 * kv_tok + 2 * w.B * w.Hkv * w.D * 2 * 2
+               + 2 * w.B * w.Hq * w.D * 2 + w.B * w.Hq * 4)
+        gbs = req / (ms / 1e3) / 1e9
+        keys = sum(int(workloads.prompt_lengths(w)[w.shared_id(r)]) + int(workloads.suffix_lengths(w)[r]) + 1
+                   for r in range(w.B))
+        tfl = 4.0 * w.Hq * w.D * keys / (ms / 1e3) / 1e12
+        out[kind] = {"ms": ms, "required_bytes": req, "achieved_gbs": gbs, "frac": gbs / hbm,
+                     "tflops": tfl, "device_status": status}
+    out["time_ratio_heterogeneous_over_homogeneous"] = (out["heterogeneous"]["ms"]
+                                                         / out["homogeneous"]["ms"])
+    out["context"] = ("Feather reports about 2x throughput for homogeneous batches with unmodified "
+                      "kernels on A100 / RTX 6000 Ada (Feather page, Results)")
+    out["peak_gbs"] = hbm
+    out["peak_source"] = src
+    out["workload"] = ("prefix-shared-llm-decode: 64 requests, beam 1, 8192-token prefixes in 4 groups "
+                       "of 16 (heterogeneous: 64 distinct), suffixes 256-2048, Hq=32, Hkv=8, D=128")
+    return out
+
+
+def long_history(dev, hbm, tf, src, reps=3):
+    """The long-history ragged workload (128 requests, prompts of 2048-16384
+    tokens, 256 beams, Hq 32 / Hkv 4, D 128, V 16384, logits) at step 1: the
+    staged attention (its mask built beside it) and the selection, each timed
+    between events around its own graph, after a graph that replays the decode
+    up to that step; the L2 is flushed before every repetition."""
+    import torch
+    import workloads
+    from shared_prefix_decode_xattention_b200 import xgr
+    from shared_prefix_decode_xattention_b200.session import Session, config_for
+    w = workloads.WORKLOADS[5]
+    items = workloads.items(w)
+    sess = Session(config_for(w), dev)
+    sess.build_trie(items)
+    del items
+    for r in range(w.B):
+        k, v = workloads.shared_kv(w, w.shared_id(r), dev)
+        sess.prefill(r, w.shared_id(r), k, v)
+        del k, v
+    qkv = [workloads.step_qkv(w, s, dev) for s in range(2)]
+    sc = [workloads.step_logits(w, s, dev) for s in range(2)]
+    o = torch.empty((w.B, w.BW, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.BW, w.Hq), dtype=torch.float32, device=dev)
+    par = torch.empty((w.B, w.BW), dtype=torch.int32, device=dev)
+    tok = torch.empty_like(par)
+    cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
+    nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
+    cur = torch.cuda.current_stream
+    side = torch.cuda.Stream(device=dev)
+    masks = {}
+    F = xgr.XGR_SCORES_LOGITS
+
+    def head():
+        sess.begin(w.B, cur())
+        masks[0] = sess.build_mask(0, cur())
+        sess.decode_step(0, *qkv[0], o, lse, cur())
+        sess.beam_select(0, sc[0], F, masks[0], par, tok, cum, nout, cur())
+
+    def att():
+        side.wait_stream(cur())
+        with torch.cuda.stream(side):
+            masks[1] = sess.build_mask(1, side)
+        sess.decode_step(1, *qkv[1], o, lse, cur())
+        cur().wait_stream(side)
+
+    def sel():
+        sess.beam_select(1, sc[1], F, masks[1], par, tok, cum, nout, cur())
+
+    head()
+    att()
+    torch.cuda.synchronize()
+    nnz = sess.mask_entries(masks[1])
+    sel()
+    torch.cuda.synchronize()
+    graphs = []
+    for fn in (head, att, sel):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs.append(g)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    att_ms, sel_ms = [], []
+    for i in range(reps + 1):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        graphs[0].replay()
+        ev[0].record()
+        graphs[1].replay()
+        ev[1].record()
+        graphs[2].replay()
+        ev[2].record()
+        torch.cuda.synchronize()
+        if i:
+            att_ms.append(ev[0].elapsed_time(ev[1]))
+            sel_ms.append(ev[1].elapsed_time(ev[2]))
+    status = sess.device_status()
+    del graphs
+    sess.close()
+    att_bytes, att_flops, sel_bytes = algorithmic(w, 1, True, nnz)
+    am, sm = statistics.median(att_ms), statistics.median(sel_ms)
+    return {"workload": f"{w.name}: B={w.B}, prompts {w.prompt[0]}-{w.prompt[1]} tokens, BW={w.BW}, "
+                        f"Hq={w.Hq}, Hkv={w.Hkv}, D={w.D}, V={w.V}, step 1, logits",
+            "attention_ms": am, "attention_required_bytes": att_bytes,
+            "attention_gbs": att_bytes / (am / 1e3) / 1e9,
+            "attention_hbm_frac": att_bytes / (am / 1e3) / 1e9 / hbm,
+            "attention_tflops": att_flops / (am / 1e3) / 1e12,
+            "attention_tensor_frac": att_flops / (am / 1e3) / 1e12 / tf,
+            "select_ms": sm, "select_required_bytes": sel_bytes,
+            "select_gbs": sel_bytes / (sm / 1e3) / 1e9,
+            "select_hbm_frac": sel_bytes / (sm / 1e3) / 1e9 / hbm,
+            "csr_entries_step1": nnz, "peak_gbs": hbm, "tensor_peak_tflops": tf,
+            "peak_source": src, "l2": "flushed before each repetition", "device_status": status}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -621,8 +815,8 @@ def run_gpu(args, w):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_config(w, args.scores), global_batch=w.B * world,
-                           parallelism=f"dp{world}" if world > 1 else "single"),
+            "config": workload_config(w, args.scores),
+            "global_batch": w.B * world, "parallelism": f"dp{world}" if world > 1 else "single",
             "roofline": roof,
             "step_breakdown_ms": {"attention_with_mask_step_ge1": att_avg * 1e3,
                                   "select_step_ge1": sel_avg * 1e3},
@@ -641,6 +835,20 @@ def run_gpu(args, w):
     del g_decode, g_phase   # released before the next workload's session
     if world == 1 and not args.no_bw512:
         line["attention_bw512"] = attention_bw512(dev, hbm, tf, src)
+    if world == 1 and not args.no_extra:
+        line["prefix_batches"] = prefix_batches(dev, hbm, tf, src)
+        line["long_history"] = long_history(dev, hbm, tf, src)
+    # the Shared stage's tensor throughput per workload (the stage is a dense
+    # contraction; its tensor fraction is what bounds it at 128+ beams)
+    tfr = {"gr-decode-pool-128x128 (step >= 1, with the Unshared and Merging stages)":
+           att_flops / att_avg / 1e12 / tf}
+    if "attention_bw512" in line:
+        tfr["gr-decode-pool-512x512 (step 1)"] = line["attention_bw512"]["tensor_frac"]
+    if "long_history" in line:
+        tfr["long-history-ragged-gr-decode (step 1)"] = line["long_history"]["attention_tensor_frac"]
+    if "prefix_batches" in line:
+        tfr["prefix-shared-llm-decode homogeneous"] = line["prefix_batches"]["homogeneous"]["tflops"] / tf
+    line["shared_stage_tensor_frac"] = tfr
     if rank == 0:
         print(json.dumps(line), flush=True)
     sess.close()

@@ -28,11 +28,18 @@
 //               O_0 and O_1 into the partial (O, m, l) or, for a request's only
 //               segment, the output.
 // In a request's only KV segment ("final" items) the Unshared and Merging
-// stages run here too: before the loop the softmax threads read the beams'
-// ancestry slots, stage the beams' own k / v rows (direct indices into the
-// token-granular pool) by cp.async, seed O_0 and its (m, l) with them, and
-// append this step's k / v to the pool.  Zero-fill items (step 0) only write
-// the rows of the beams that are not live yet.
+// stages run here too.  The Unshared stage is one more key chunk of the same
+// loop (or a few, when the tile's beams x tokens pass 128): lanes 2-31 of the
+// producer warp gather the tile's beams' own k / v rows of steps 0..s (direct
+// indices into the token-granular pool; this step's from k_new / v_new) into
+// the U area at kernel start, so the gather overlaps the Shared loop, and
+// append this step's k / v to the pool.  Row u of that chunk is token u % T of
+// the tile's beam u / T (T = s + 1 tokens per beam): the chunk is block-
+// diagonal, and each query row keeps only its own beam's valid tokens (the
+// rest of the chunk's scores are masked to -inf before the exponentials).
+// The online softmax then merges the Shared and Unshared stages as it goes.
+// Zero-fill items (step 0) only write the rows of the beams that are not live
+// yet.
 // Every wait on an mbarrier is bounded; on time-out the CTA records
 // XGR_DEV_TIMEOUT in the status word and unwinds (no trap, no hang).
 #include <cuda.h>
@@ -54,7 +61,8 @@ constexpr int kKStages = 2;                  // K chunks in flight
 constexpr int kVStages = 2;                  // V chunks in flight
 constexpr uint32_t kHalf = 16384;            // one 128-row x 64-column bf16 sub-tile
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 bf16
-constexpr uint32_t kUBytes = 65536;          // U area: the Unshared stage's staged rows
+constexpr uint32_t kUBytes = 65536;          // U area: the Unshared chunk's K and V tiles
+constexpr int kGatherLanes = 30;             // producer-warp lanes 2..31 gather the Unshared rows
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
@@ -73,9 +81,11 @@ constexpr uint32_t kTmemCols = 512;
 enum { B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
        B_VEMPTY = B_VFULL + kVStages, B_SFULL = B_VEMPTY + kVStages, B_PFULL = B_SFULL + 2,
        B_PVDONE = B_PFULL + 2, B_QFULL = B_PVDONE + 2, B_DONE = B_QFULL + 1, B_XCH = B_DONE + 1,
-       B_COUNT = B_XCH + 2 };
+       B_UFULL = B_XCH + 2, B_UEMPTY = B_UFULL + 1, B_COUNT = B_UEMPTY + 1 };
 // B_PVDONE: P_j V_j has completed (S_j's TMEM buffer, which held P_j, may take
-// S_{j+2}); B_DONE: every MMA has completed; B_XCH: the warpgroups' (m, l) exchange
+// S_{j+2}); B_DONE: every MMA has completed; B_XCH: the warpgroups' (m, l) exchange;
+// B_UFULL: an Unshared chunk is gathered into the U area; B_UEMPTY: its MMAs have
+// completed (the U area may take the next one)
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -237,9 +247,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // query row `row` of a work item -> (request, beam, query head, global row, live)
 struct RowInfo {
@@ -292,8 +299,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return;
     }
     const int n_keys = it.key_end - it.key_begin;
-    const int nchunks = (n_keys + kBlockN - 1) / kBlockN;
+    const int nchunks = (n_keys + kBlockN - 1) / kBlockN;   // Shared-stage chunks
     const bool final_item = (it.flags & 1) != 0;
+    // Unshared chunks (final items): the tile's beams x (s + 1) tokens, 128 rows each
+    const int T = a.step + 1;
+    const int lb0 = it.row_begin / a.dims.G;
+    const int nbeam = (it.row_begin + it.n_rows - 1) / a.dims.G - lb0 + 1;
+    const int n_u = final_item ? (nbeam * T + kBlockN - 1) / kBlockN : 0;
+    const int nall = nchunks + n_u;
     const bool q_tma = (it.flags & 2) != 0;   // the Q tile is one TMA box
     volatile int *abort = abort_flag;
     const int y0 = it.g * (int)a.kv_tokens + it.kv_off + it.key_begin;
@@ -329,6 +342,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             mbar_init(bar(B_QFULL), q_tma ? 1 : kSoftmaxThreads);
             mbar_init(bar(B_DONE), 1);
+            mbar_init(bar(B_UFULL), kGatherLanes);
+            mbar_init(bar(B_UEMPTY), 1);
             *abort_flag = 0;
             fence_mbar_init();
         }
@@ -398,6 +413,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (*abort)
                 for (int j = max(0, n_issued - kVStages); j < n_issued; ++j)
                     mbar_wait(bar(B_VFULL + j % kVStages), (j / kVStages) & 1, nullptr);
+        } else if (n_u > 0) {
+            // ---- Unshared stage: gather the tile's beams' own k / v rows of steps
+            // 0..s into the U area, one 128-row chunk at a time (row u: token u % T
+            // of tile beam u / T), in the canonical swizzled layout; rows of dead
+            // beams, bad slots and the tail are zero.  This step's rows are also
+            // appended to the pool at slot (s, b).
+            const int gl = lane - 2;
+            const Dims dm = a.dims;
+            const int s_now = a.step;
+            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+            for (int q = 0; q < n_u; ++q) {
+                if (q > 0 && !mbar_wait(bar(B_UEMPTY), (q - 1) & 1, abort)) break;
+                for (int u = gl; u < kBlockN; u += kGatherLanes) {
+                    const int ug = kBlockN * q + u, lb = ug / T, i = ug % T;
+                    const __nv_bfloat16 *sk = nullptr, *sv = nullptr;
+                    if (lb < nbeam) {
+                        const int lbs = lb0 + lb;   // beam index within the segment's rows / G
+                        const int member = lbs / a.nb, b = lbs % a.nb;
+                        const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + member];
+                        const int64_t brow = (int64_t)r * dm.BW + b;
+                        if (b < a.n_live[r]) {
+                            if (i == s_now) {
+                                sk = a.k_new + (brow * dm.Hkv + it.g) * 128;
+                                sv = a.v_new + (brow * dm.Hkv + it.g) * 128;
+                            } else {
+                                const int sl = a.st.anc[brow * dm.S + i];
+                                if (sl >= 0 && sl < dm.BW) {
+                                    const int64_t prow = (brow - b + sl) * dm.Hkv + it.g;
+                                    sk = a.pool_k + i * pool_step + prow * 128;
+                                    sv = a.pool_v + i * pool_step + prow * 128;
+                                }
+                            }
+                        }
+                    }
+                    const uint32_t dk = sb + kOffU, dv = sb + kOffU + kTile;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (sk) {
+                            cp_async16(dk + sw128_off(u, c), sk + 8 * c);
+                            cp_async16(dv + sw128_off(u, c), sv + 8 * c);
+                        } else {
+                            *reinterpret_cast<uint4 *>(base + kOffU + sw128_off(u, c)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(base + kOffU + kTile + sw128_off(u, c)) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                cp_async_wait_all();
+                // this step's k / v of the gathered live beams -> pool slot (s, b)
+                for (int u = gl; u < kBlockN; u += kGatherLanes) {
+                    const int ug = kBlockN * q + u, lb = ug / T, i = ug % T;
+                    if (lb >= nbeam || i != s_now) continue;
+                    const int lbs = lb0 + lb, member = lbs / a.nb, b = lbs % a.nb;
+                    const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + member];
+                    if (b >= a.n_live[r]) continue;
+                    const int64_t orow = ((int64_t)r * dm.BW + b) * dm.Hkv + it.g;
+                    uint4 *pk = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + orow * 128);
+                    uint4 *pv = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + orow * 128);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        pk[c] = *reinterpret_cast<const uint4 *>(base + kOffU + sw128_off(u, c));
+                        pv[c] = *reinterpret_cast<const uint4 *>(base + kOffU + kTile + sw128_off(u, c));
+                    }
+                }
+                fence_async_smem();   // the gathered rows are visible to the tensor cores
+                mbar_arrive(bar(B_UFULL));
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -408,11 +490,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
             constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
-            auto issue_s = [&](int j) -> bool {   // S_j = Q K_j^T (waits for K_j unless it has landed)
-                const int st = j % kKStages;
-                if (j < 2 && !mbar_wait(bar(B_KFULL + st), (j / kKStages) & 1, abort)) return false;
+            // chunk j < nchunks: a Shared chunk in the K / V rings; j >= nchunks: an
+            // Unshared chunk in the U area (its K and V land together on B_UFULL)
+            auto k_ready = [&](int j, bool block) -> bool {
+                const uint32_t b = j < nchunks ? bar(B_KFULL + j % kKStages) : bar(B_UFULL);
+                const uint32_t ph = j < nchunks ? (j / kKStages) & 1 : (j - nchunks) & 1;
+                return block ? mbar_wait(b, ph, abort) : mbar_test(b, ph);
+            };
+            auto issue_s = [&](int j) {   // S_j = Q K_j^T into TMEM buffer j % 2
                 fence_after_sync();
-                const uint32_t kq = sb + kOffQ, kk = sb + kOffK + st * kTile;
+                const uint32_t kq = sb + kOffQ;
+                const uint32_t kk = j < nchunks ? sb + kOffK + (j % kKStages) * kTile : sb + kOffU;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
@@ -420,27 +508,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                               umma_desc(kk + off, 16, 1024), idS, k > 0);
                 }
                 umma_commit(bar(B_SFULL + (j & 1)));
-                umma_commit(bar(B_KEMPTY + st));
-                return true;
+                if (j < nchunks) umma_commit(bar(B_KEMPTY + j % kKStages));
             };
             bool ok = mbar_wait(bar(B_QFULL), 0, abort);
             int ns = 0;   // the next S to issue
-            for (; ok && ns < min(nchunks, 2); ++ns) ok = issue_s(ns);
+            for (; ok && ns < min(nall, 2); ++ns) {
+                ok = k_ready(ns, true);
+                if (ok) issue_s(ns);
+            }
             // Then whichever is ready first: S_ns (P_{ns-2} V_{ns-2}, which read its
             // TMEM buffer, complete and K_ns landed) or O_h += P_j V_j (P_j written,
             // V_j landed).  Every phase polled here is at most one behind the
             // barrier's current one, so the parity tests are exact.
             uint32_t idle = 0;
-            for (int j = 0; ok && j < nchunks;) {
+            for (int j = 0; ok && j < nall;) {
                 bool progress = false;
-                if (ns < nchunks && mbar_test(bar(B_PVDONE + (ns & 1)), ((ns - 2) >> 1) & 1) &&
-                    mbar_test(bar(B_KFULL + ns % kKStages), (ns / kKStages) & 1)) {
+                if (ns < nall && mbar_test(bar(B_PVDONE + (ns & 1)), ((ns - 2) >> 1) & 1) &&
+                    k_ready(ns, false)) {
                     issue_s(ns++);
                     progress = true;
                 }
                 const int h = j & 1, sv = j % kVStages;
-                if (!(mbar_test(bar(B_PFULL + h), (j >> 1) & 1) &&
-                      mbar_test(bar(B_VFULL + sv), (j / kVStages) & 1))) {
+                const bool v_ready = j < nchunks ? mbar_test(bar(B_VFULL + sv), (j / kVStages) & 1)
+                                                 : mbar_test(bar(B_UFULL), (j - nchunks) & 1);
+                if (!(mbar_test(bar(B_PFULL + h), (j >> 1) & 1) && v_ready)) {
                     if (progress) {
                         idle = 0;
                     } else if (++idle >= kSpinLimit) {
@@ -453,16 +544,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 idle = 0;
                 fence_after_sync();
-                const uint32_t kv = sb + kOffV + sv * kTile;
-                // O_0 starts from the Unshared stage in final items
-                const bool acc0 = j >= 2 || (j == 0 && final_item);
+                const uint32_t kv = j < nchunks ? sb + kOffV + sv * kTile : sb + kOffU + kTile;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)   // P_j: 16 keys = 8 TMEM columns per MMA
                     umma_bf16_ts(tmem + 256u + (uint32_t)h * 128u, tmem + (uint32_t)h * 128u + 8u * k,
                                  umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024), idPV,
-                                 (k > 0 || acc0) ? 1u : 0u);
+                                 (k > 0 || j >= 2) ? 1u : 0u);
                 umma_commit(bar(B_PVDONE + h));
-                umma_commit(bar(B_VEMPTY + sv));
+                umma_commit(j < nchunks ? bar(B_VEMPTY + sv) : bar(B_UEMPTY));
                 ++j;
             }
             // arrives once every MMA issued above has completed (TMEM final / free)
@@ -475,8 +564,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // `row` reads TMEM lane `row` of S buffer `half`, keeps the running max and
         // sum of accumulator O_half and writes row `row` of P_j over it.  The
         // two warpgroups never wait for each other inside the loop; their
-        // (m, l, O) are merged at the end.  In the Unshared prologue thread
-        // (row, half) handles head-dim columns [64*half, 64*half + 64).
+        // (m, l, O) are merged at the end, where thread (row, half) handles
+        // head-dim columns [64*half, 64*half + 64).
         const int half = (warp - 2) >> 2;
         const int row = 32 * (warp & 3) + lane;
         bool ok = true;
@@ -492,161 +581,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float m_used = -INFINITY, l = 0.f;   // running max / sum of O_half
         const Dims dm = a.dims;
         const bool live = ri.valid && ri.b < a.n_live[ri.r];
-        if (final_item) {
-            // ---- Unshared stage first (the item covers its requests' only KV
-            // segment): each beam's own tokens of steps 0..s, read through its
-            // direct indices (ancestry slots) into the token-granular pool, seed
-            // the online softmax -- their max, their sum (half 0) and their
-            // weighted values in the TMEM accumulator O_0 -- so the main loop
-            // merges the two stages as it goes.  The rows of the tile's beams are
-            // staged in the U area by cp.async: one round trip for the slots, one
-            // per batch of (beams, tokens) that fits, whatever the step.  Thread
-            // (row, half) computes the full score of its row and the weighted
-            // values of its 64 head-dim columns.
-            const int G = dm.G, ts = tid - 64;
-            const int s_now = a.step, n_tok = s_now + 1;
-            const int lb0 = it.row_begin / G;
-            const int nbeam = (it.row_begin + it.n_rows - 1) / G - lb0 + 1;   // beams in the tile
-            const int lb = (it.row_begin + row) / G - lb0;                     // this row's beam
-            constexpr int kTabW = kMaxSteps + 1;   // per beam: slot of each token, then r * BW + b
-            int *tab = reinterpret_cast<int *>(base + kOffU);
-            const uint32_t tab_bytes = ((uint32_t)nbeam * kTabW * 4u + 127u) & ~127u;
-            // then the two halves' partial dots [2][kMaxSteps][128] (fp32), then the staged
-            // rows [tokens][beams][k | v][128] (bf16), kStgRow bytes per (token, beam): the
-            // 16-byte pad puts the beams one warp reads at once in different banks
-            constexpr uint32_t kStgRow = 528;
-            constexpr uint32_t kXdBytes = 2u * kMaxSteps * 128u * 4u;
-            float *xd = reinterpret_cast<float *>(base + kOffU + tab_bytes);
-            uint8_t *stg = base + kOffU + tab_bytes + kXdBytes;
-            const uint32_t room = kUBytes - tab_bytes - kXdBytes;
-            const int nbg = min(nbeam, (int)(room / kStgRow));   // beams per batch
-            const int tb = max(1, (int)(room / ((uint32_t)nbg * kStgRow)));   // tokens per batch
-            // 1. the tile's first row of each beam reads the beam's slots (one round trip)
-            if (ri.valid && (ri.hg == 0 || row == 0) && half == 0) {
-                const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
-                int sl[kMaxSteps];
-#pragma unroll
-                for (int i = 0; i < kMaxSteps; ++i)
-                    sl[i] = (live && i < s_now) ? a.st.anc[beam_row * dm.S + i] : -1;
-                int *t = tab + lb * kTabW;
-#pragma unroll
-                for (int i = 0; i < kMaxSteps; ++i) {
-                    if (i >= s_now) break;
-                    if (live && (sl[i] < 0 || sl[i] >= dm.BW)) set_status(a.status, XGR_DEV_INDEX);
-                    t[i] = (sl[i] >= 0 && sl[i] < dm.BW) ? sl[i] : -1;
-                }
-                t[s_now] = live ? ri.b : -1;
-                t[kMaxSteps] = (int)beam_row;
-            }
-            if (q_tma)   // the scores read Q from shared memory
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(B_QFULL), 0, abort));
-            named_sync(1, kSoftmaxThreads);
-            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
-            const int64_t kvo = ((int64_t)(ri.r * dm.BW + ri.b) * dm.Hkv + it.g) * 128;
-            float m_u = -INFINITY, l_u = 0.f, o[64];
-#pragma unroll
-            for (int e = 0; e < 64; ++e) o[e] = 0.f;
-            // 2. batches: stage the k and v rows of (beams, tokens), then fold them in
-            for (int gb = 0; gb < nbeam; gb += nbg) {
-                const int ngb = min(nbg, nbeam - gb);
-                for (int i0 = 0; i0 < n_tok; i0 += tb) {
-                    const int ntb = min(tb, n_tok - i0);
-                    const int units = ngb * ntb * 32;   // 16-byte pieces: 16 of k and 16 of v per row pair
-                    for (int u = ts; u < units; u += kSoftmaxThreads) {
-                        const int c = u & 15, kind = (u >> 4) & 1, bt = u >> 5;
-                        const int bl = bt % ngb, ti = bt / ngb, i = i0 + ti;
-                        const int *t = tab + (gb + bl) * kTabW;
-                        const int sl = t[i];
-                        if (sl < 0) continue;
-                        const int64_t brow = t[kMaxSteps];
-                        const int64_t src_row = i == s_now ? brow
-                                                           : (brow - brow % dm.BW + sl) + (int64_t)i * a.Bcap * dm.BW;
-                        const __nv_bfloat16 *src =
-                            (i == s_now ? (kind ? a.v_new : a.k_new) : (kind ? a.pool_v : a.pool_k)) +
-                            (src_row * dm.Hkv + it.g) * 128 + c * 8;
-                        cp_async16(smem_u32(stg + (uint32_t)(ti * ngb + bl) * kStgRow + kind * 256u + c * 16), src);
-                    }
-                    cp_async_wait_all();
-                    named_sync(1, kSoftmaxThreads);
-                    const bool mine = live && lb >= gb && lb < gb + ngb;
-                    if (mine) {   // partial dots over this thread's 64 head-dim columns
-#pragma unroll 1
-                        for (int ti = 0; ti < ntb; ++ti) {
-                            const uint8_t *kr = stg + (uint32_t)(ti * ngb + lb - gb) * kStgRow + col0 * 2;
-                            float acc = 0.f;
-#pragma unroll 4
-                            for (int c = 0; c < 8; ++c) {
-                                float qf[8], kf[8];
-                                unpack8(*reinterpret_cast<const uint4 *>(base + kOffQ + sw128_off(row, 8 * half + c)),
-                                        qf);
-                                unpack8(*reinterpret_cast<const uint4 *>(kr + c * 16), kf);
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) acc = fmaf(qf[e], kf[e], acc);
-                            }
-                            xd[(half * kMaxSteps + ti) * 128 + row] = acc;
-                        }
-                    }
-                    named_sync(1, kSoftmaxThreads);
-                    if (mine) {
-#pragma unroll 1
-                        for (int ti = 0; ti < ntb; ++ti) {
-                            const int i = i0 + ti;
-                            if (tab[lb * kTabW + i] < 0) continue;
-                            const uint8_t *kr = stg + (uint32_t)(ti * ngb + lb - gb) * kStgRow;
-                            const uint8_t *vr = kr + 256;
-                            const float sc = (xd[ti * 128 + row] + xd[(kMaxSteps + ti) * 128 + row]) * cscale;
-                            if (sc > m_u) {   // online softmax over the beam's tokens
-                                const float al = ex2(m_u - sc);
-                                l_u *= al;
-#pragma unroll
-                                for (int e = 0; e < 64; ++e) o[e] *= al;
-                                m_u = sc;
-                            }
-                            const float pw = ex2(sc - m_u);
-                            l_u += pw;
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                float vf[8];
-                                unpack8(*reinterpret_cast<const uint4 *>(vr + col0 * 2 + c * 16), vf);
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) o[8 * c + e] = fmaf(pw, vf[e], o[8 * c + e]);
-                            }
-                            if (i == s_now && ri.hg == 0) {   // append this step's k / v at slot (s, b)
-                                uint4 *ka = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + kvo + col0);
-                                uint4 *va = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + kvo + col0);
-#pragma unroll
-                                for (int c = 0; c < 8; ++c) {
-                                    ka[c] = *reinterpret_cast<const uint4 *>(kr + col0 * 2 + c * 16);
-                                    va[c] = *reinterpret_cast<const uint4 *>(vr + col0 * 2 + c * 16);
-                                }
-                            }
-                        }
-                    }
-                    if (gb + nbg < nbeam || i0 + tb < n_tok) named_sync(1, kSoftmaxThreads);   // restage
-                }
-            }
-            // the Unshared stage seeds O_0 (both halves' columns), the running max and (half 0) sum
-            tmem_st32(tmem + lane_base + 256 + col0, o);
-            tmem_st32(tmem + lane_base + 256 + col0 + 32, o + 32);
-            tmem_wait_st();
-            if (live && half == 0) {   // O_0 holds the Unshared stage
-                m_used = m_u;
-                l = l_u;
+        // Unshared chunks: this row keeps columns [u_lo, u_lo + T) of the block-
+        // diagonal U rows -- its beam's tokens -- where the token's slot is valid
+        // (bit i of vmask; this step's own token when the beam is live)
+        uint32_t vmask = 0;
+        const int u_lo = ((it.row_begin + row) / dm.G - lb0) * T;
+        if (final_item && live) {
+            const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
+            vmask = 1u << a.step;
+            for (int i = 0; i < a.step; ++i) {
+                const int sl = a.st.anc[beam_row * dm.S + i];
+                if (sl >= 0 && sl < dm.BW) vmask |= 1u << i;
+                else if (ri.hg == 0 && half == 0) set_status(a.status, XGR_DEV_INDEX);
             }
         }
         const uint32_t s_col = (uint32_t)half * 128u;          // S buffer of this warpgroup
         const uint32_t o_col = 256u + (uint32_t)half * 128u;   // its O accumulator
-        for (int j = half, jj = 0; ok && j < nchunks; j += 2, ++jj) {
+        for (int j = half, jj = 0; ok && j < nall; j += 2, ++jj) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + half), jj & 1, abort));
             if (!ok) break;
             fence_after_sync();
             const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
+            const bool is_u = j >= nchunks;            // an Unshared chunk
+            const int c0 = u_lo - kBlockN * (j - nchunks);   // (is_u) the row's first column in it
+            auto u_out = [&](int c) {   // column c of an Unshared chunk is not this row's
+                const int t = c - c0;
+                return !(t >= 0 && t < T && ((vmask >> t) & 1u));
+            };
             // the chunk's 128 scores in one TMEM read (P_j then overwrites them)
             float sv[128];
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) tmem_ld32(tmem + lane_base + s_col + 32 * q2, sv + 32 * q2);
             tmem_wait_ld();
-            if (nvalid < kBlockN) {   // the range's last chunk: keys past its end do not count
+            if (is_u) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (u_out(c)) sv[c] = -INFINITY;
+            } else if (nvalid < kBlockN) {   // the range's last chunk: keys past its end do not count
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= nvalid) sv[c] = -INFINITY;
@@ -662,7 +633,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             bool rescale = false;
             if (mx > m_used + 8.f) {   // lazy rescaling: keep the old max unless it grew by 2^8
                 alpha = ex2(m_used - mx);
-                rescale = jj > 0 || (half == 0 && final_item);   // O_half already holds data
+                rescale = jj > 0;   // O_half already holds data
                 m_used = mx;
             }
             // (S_j was issued after P_{j-2} V_{j-2} completed: O_half is current and
@@ -680,7 +651,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tmem_ld32(tmem + lane_base + s_col + 32 * q2, v);
                 tmem_wait_ld_into(v);
                 const int nv = nvalid - 32 * q2;   // keys of the piece inside the range
-                if (nv < 32) {
+                if (is_u) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (u_out(32 * q2 + e)) v[e] = -INFINITY;
+                } else if (nv < 32) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (e >= nv) v[e] = -INFINITY;

@@ -71,8 +71,9 @@ cudaError_t launch_attn_merge(const MergeArgs &a, cudaStream_t st);
 
 // Beam state reset of xgr_begin.
 // mask_sync: the mask builder's look-back words [Bcap] and ticket, zeroed here
+// sel_ticket: the selection's tickets [Bcap], zeroed here
 cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync,
-                         cudaStream_t s);
+                         uint32_t *sel_ticket, cudaStream_t s);
 
 // Sparse masks of steps >= 1: one CSR row per beam.
 struct MaskArgs {
@@ -105,19 +106,18 @@ struct SelectArgs {
     const uint32_t *bits;
     const int32_t *row_ptr;
     const int32_t *cols;
-    int64_t max_entries;        // expected largest CSR entry count of one request (sizes the pick grid)
     // scratch (select_scratch_carve)
-    float *row_lse;             // [B][BW]
-    uint64_t *best;             // [B][BW] each beam's best candidate key
-    int32_t *surv_cnt;          // [B] survivors appended
-    uint32_t *ticket;           // [B] pick CTAs done (reset by the rows kernel)
+    float *row_lse;             // [B][BW] each live row's log-sum-exp (logits mode)
+    int32_t *row_cnt;           // [B][BW] valid candidates of each row
+    uint64_t *head_k;           // [B][BW][m] each beam's m best keys, ascending (kNoKey pads)
+    int32_t *head_e;            // [B][BW][m] their CSR entries (relative to the request)
+    int head_m;                 // m
+    uint32_t *ticket;           // [B] CTAs of the request done; the last resets it to 0
     uint64_t *keys;             // [B][key_cap] key of each CSR entry (relative to the request)
     int64_t key_cap;
-    uint64_t *surv_key;         // [B][surv_cap] candidates at or above the threshold
-    int32_t *surv_e;            // [B][surv_cap] their entry
-    int64_t surv_cap;
-    int pick_parts;             // set by the launcher
-    int num_sms;                // SMs of the device (sizes the persistent row kernel)
+    int sp_parts;               // set by the launcher: CTAs per request of the sparse kernel
+    int sp_rows;                //   and the beams each of them takes
+    int num_sms;                // SMs of the device
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
     float *cum_out;
@@ -125,14 +125,17 @@ struct SelectArgs {
 };
 // Largest vocabulary of the selection: a score row is staged whole in shared memory.
 constexpr int kSelectMaxVocab = 32768;
-// Scratch of the selection for B requests of BW beams: row_lse and best per
-// beam row, surv_cnt and ticket per request, keys [B][key_cap] (a request's
-// CSR entries beyond key_cap take the exact fallback over the scores) and the
-// survivor buffer [B][surv_cap] (more survivors: exact selection over the keys).
-// Everything in it is written by the same call before it is read.
-size_t select_scratch_bytes(int B, int BW, int64_t key_cap, int64_t surv_cap);
-void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, int64_t surv_cap,
-                          SelectArgs &a);
+// Scratch of the selection for B requests of BW beams: per beam row its
+// log-sum-exp, valid-candidate count and head (its m best keys and their
+// entries), a ticket per request, and the key buffer [B][key_cap] (a request
+// whose CSR entries exceed key_cap takes the exact fallback over the scores).
+// Everything read is written by the same call first, except the tickets,
+// which must be zero before a call (xgr_begin zeroes them, each call leaves
+// them zero).
+int select_head_m(int BW);
+size_t select_scratch_bytes(int B, int BW, int64_t key_cap);
+size_t select_ticket_offset(int B, int BW);   // byte offset of the tickets in the scratch
+void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectArgs &a);
 cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
 
 cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);

@@ -6,11 +6,11 @@
 //      come only from the valid-item vocabulary -- a dense bitset of first
 //      tokens at step 0, sparse rows (each beam's sorted trie children) later.
 //      "Early sort termination": the page orders each beam's candidates and
-//      cuts every list at a global min-heap threshold.  Here the threshold tau
-//      is the worst of the live beams' best keys: with all BW beams live these
-//      are BW real candidates, so every one of the BW winners ranks at or
-//      above tau, and only the candidates at or above it ("survivors") reach
-//      the exact selection.
+//      cuts every list at a global min-heap threshold.  Here each beam's list
+//      is ordered as far as its head (its m best keys), the threshold tau is
+//      the BW-th best of all heads (BW real candidates rank at or above it, so
+//      every winner does), and only the candidates at or above it
+//      ("survivors") reach the exact selection.
 //  2.1 "In-place updates": the beam state (ancestry slots, trie node, token
 //      history, cumulative score) is rewritten in place; every row a new beam
 //      reads is staged in shared memory before any row is written.
@@ -22,20 +22,19 @@
 // Kernels:
 //  * dense mask (one live beam per request, step 0): select_dense_kernel, one
 //    CTA per request, stages the beam's score row with one bulk copy, takes its
-//    log-sum-exp (logits), computes every token's key once into registers and
-//    radix-selects the best BW there.
-//  * sparse (CSR) masks: select_rows_kernel, one persistent 1024-thread CTA per
-//    SM over a contiguous block of beam rows: the rows' metadata and CSR tokens
-//    in two round trips, the score rows (logits mode) through bulk-copy slots,
-//    eight 128-thread groups on eight rows at a time; per row the log-sum-exp,
-//    each entry's key beside its CSR position and the row's best key.  Then one
-//    of two picks: select_pick_one_kernel (one CTA per request, when the
-//    request's pool fits its registers and shared memory) radix-selects the
-//    pool directly; select_pick_kernel (a few CTAs per request) reduces tau
-//    from the best keys, filters its slices of the request's keys and appends
-//    the survivors, and the request's last CTA to finish (an atomic ticket the
-//    rows kernel resets) selects among them.  Both end in finish_request: the
-//    ordering, the outputs and the rewiring.
+//    log-sum-exp (logits), cuts the row into slices with a head each (their m
+//    best keys, in order), and selects the best BW among the survivors of the
+//    heads' threshold, as the sparse kernel does.
+//  * sparse (CSR) masks: select_sparse_kernel, one launch per step.  Each
+//    request gets several CTAs; a warp takes one beam row at a time: its
+//    log-sum-exp (logits), the key of each of its CSR entries, and its head --
+//    the beam's m best keys in order (the page's ordered per-beam candidate
+//    list, cut at m).  The request's last CTA to finish (an atomic ticket)
+//    takes tau = the BW-th best head key (at least BW real candidates rank at
+//    or above it, so every winner does), gathers the survivors at or above tau
+//    -- the head keys, and the further keys of beams whose whole head
+//    survived -- and radix-selects the BW best of them.  It ends in
+//    finish_request: the ordering, the outputs and the rewiring.
 #include <algorithm>
 
 #include "async.cuh"
@@ -46,11 +45,6 @@ namespace xgr {
 
 namespace {
 
-constexpr int kDenseThreads = 1024;
-constexpr int kPickThreads = 512;
-constexpr int kPickKeys = 4096;    // keys one pick CTA filters per slice (8 per thread)
-constexpr int kSmemSurv = 4096;    // survivors selected in shared memory
-constexpr int kMaxPickParts = 16;
 
 __device__ __forceinline__ float ex2f(float x) {
     float y;
@@ -145,25 +139,8 @@ __device__ int block_exclusive_scan_int(int v, int *warp_tot, int *total) {
     return before + incl - v;
 }
 
-// A set of threads that reduce together: the whole block (barrier 0) or a
-// group of warps with its own named barrier.
-struct Group {
-    int bar, n, t;   // barrier id (0: __syncthreads), threads, this thread's index in the group
-    __device__ __forceinline__ void sync() const {
-        if (bar == 0) __syncthreads();
-        else asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(n) : "memory");
-    }
-};
-__device__ __forceinline__ Group whole_block() { return Group{0, (int)blockDim.x, (int)threadIdx.x}; }
-
-// log-sum-exp of the values x[i], i < n, in shared memory, over a group: the
-// row max first, then the sum of exponentials, each reduced without
-// branches; reports NaN.  red: 33 floats of shared memory for the group.
-// log-sum-exp of x[0..n) (shared memory) over a group, in one pass: each thread
-// keeps its own (max, sum of 2^((x - max) log2 e)) over blocks of 16 values
-// (16-byte loads when x is 16-byte aligned), rescaling its sum when its max
-// grows; the pairs are then combined across the group.  red holds 2 floats per
-// warp of the group.
+// (m, s) <- the pair that stands for both (m, s) and (m2, s2), where each pair
+// is a maximum m and a sum s of exp(x - m) over some values (natural units)
 __device__ __forceinline__ void lse_pair_merge(float &m, float &s, float m2, float s2) {
     const float M = fmaxf(m, m2);
     if (M == -INFINITY) return;   // both empty
@@ -171,72 +148,6 @@ __device__ __forceinline__ void lse_pair_merge(float &m, float &s, float m2, flo
         (m2 == -INFINITY ? 0.f : s2 * ex2f((m2 - M) * kLog2e));
     m = M;
 }
-__device__ float group_lse(const float *x, int n, float *red, int32_t *status, const Group &g) {
-    const int lane = g.t % 32, w = g.t / 32, nw = g.n / 32;
-    float m = -INFINITY, s = 0.f;
-    bool nan = false;
-    auto fold = [&](const float *v, int k) {   // k values already in registers
-        float mv = -INFINITY;
-        for (int e = 0; e < k; ++e) {
-            nan |= isnan(v[e]);
-            mv = fmaxf(mv, v[e]);
-        }
-        if (mv > m) {
-            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
-            m = mv;
-        }
-        if (m != -INFINITY) {
-            const float mk = m * kLog2e;
-            for (int e = 0; e < k; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
-        }
-    };
-    const int n4 = (reinterpret_cast<uintptr_t>(x) & 15) == 0 ? n / 4 : 0;
-    const float4 *x4 = reinterpret_cast<const float4 *>(x);
-    for (int b = 0; b < n4; b += 4 * g.n) {
-        float v[16];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = b + k * g.n + g.t;
-            const float4 q = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-            v[4 * k] = q.x;
-            v[4 * k + 1] = q.y;
-            v[4 * k + 2] = q.z;
-            v[4 * k + 3] = q.w;
-        }
-        fold(v, 16);
-    }
-    for (int i = 4 * n4 + g.t; i < n; i += g.n) fold(x + i, 1);
-    if (nan) set_status(status, XGR_DEV_NAN);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_pair_merge(m, s, m2, s2);
-    }
-    if (lane == 0) {
-        red[2 * w] = m;
-        red[2 * w + 1] = s;
-    }
-    g.sync();
-    m = red[0];
-    s = red[1];
-    for (int k = 1; k < nw; ++k) lse_pair_merge(m, s, red[2 * k], red[2 * k + 1]);
-    g.sync();   // red is reused
-    return m + logf(s);
-}
-__device__ float block_lse(const float *x, int n, float *red, int32_t *status) {
-    return group_lse(x, n, red, status, whole_block());
-}
-__device__ uint64_t group_min_u64(uint64_t v, uint64_t *red, const Group &g) {
-    const int lane = g.t % 32, w = g.t / 32, nw = g.n / 32;
-    v = warp_min_u64(v);
-    if (lane == 0) red[w] = v;
-    g.sync();
-    v = red[0];
-    for (int k = 1; k < nw; ++k) v = red[k] < v ? red[k] : v;
-    g.sync();
-    return v;
-}
-
 // One radix pass's bucket search over the digit of `width` bits at `shift`:
 // the bin holding the k_rem-th key, by a one-warp scan of the 256-bin
 // histogram.  Returns whether the digit is resolved exactly (the bin's keys are
@@ -310,88 +221,6 @@ __device__ void radix_select(const Cand &cand, int64_t E, int want, int *hist, i
         }
         __syncthreads();
         if (radix_bucket(hist, sc, shift, 8, k_rem, prefix, mask)) break;
-    }
-}
-
-// The same over keys held in registers (KPT per thread, kNoKey for none) plus
-// an optional tail of n_tail keys in shared memory, with 11-bit digits (2048
-// bins, bucket found by a block-wide scan: half the passes of 8-bit digits).
-// The digits start at the highest bit where the smallest and largest key
-// differ (the bits above are common to all keys), so the first histogram
-// already spreads the keys over many bins and the shared-memory atomics do not
-// pile onto a few counters.  hist: kWideBins ints; scan_w: 32 ints; red: 32
-// u64 of shared memory.
-constexpr int kWideBits = 11, kWideBins = 1 << kWideBits;
-
-template <int KPT>
-__device__ void radix_select_regs(const uint64_t (&k)[KPT], int want, int *hist, int *sc, int *scan_w,
-                                  uint64_t *red, uint64_t &prefix, uint64_t &mask,
-                                  const uint64_t *tail = nullptr, int n_tail = 0) {
-    uint64_t lo = kNoKey, hi = 0;
-#pragma unroll
-    for (int u = 0; u < KPT; ++u)
-        if (k[u] != kNoKey) {
-            lo = k[u] < lo ? k[u] : lo;
-            hi = k[u] > hi ? k[u] : hi;
-        }
-    for (int i = threadIdx.x; i < n_tail; i += blockDim.x)
-        if (tail[i] != kNoKey) {
-            lo = tail[i] < lo ? tail[i] : lo;
-            hi = tail[i] > hi ? tail[i] : hi;
-        }
-    lo = block_min_u64(lo, red);
-    hi = block_max_u64(hi, red);
-    const uint64_t diff = lo ^ hi;
-    if (diff == 0) {   // one distinct key (keys are unique: one candidate)
-        prefix = lo;
-        mask = ~0ull;
-        return;
-    }
-    int pos = 64 - __clzll((long long)diff);   // bits [pos, 64) are common to every key
-    mask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
-    prefix = lo & mask;
-    int k_rem = want;
-    const int bpt = kWideBins / blockDim.x;   // bins per thread in the bucket scan (1, 2 or 4)
-    while (pos > 0) {
-        const int shift = pos > kWideBits ? pos - kWideBits : 0, width = pos - shift;
-        const uint64_t dmask = (1ull << width) - 1ull;
-        for (int i = threadIdx.x; i < kWideBins; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int u = 0; u < KPT; ++u)
-            if (k[u] != kNoKey && (k[u] & mask) == prefix) atomicAdd(&hist[(k[u] >> shift) & dmask], 1);
-        for (int i = threadIdx.x; i < n_tail; i += blockDim.x) {
-            const uint64_t key = tail[i];
-            if (key != kNoKey && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
-        }
-        __syncthreads();
-        // the bin holding the k_rem-th key: thread t scans bins [t*bpt, t*bpt + bpt)
-        int h[4] = {0, 0, 0, 0}, sum = 0;
-        for (int j = 0; j < bpt; ++j) {
-            h[j] = hist[threadIdx.x * bpt + j];
-            sum += h[j];
-        }
-        int total;
-        int acc = block_exclusive_scan_int(sum, scan_w, &total);
-        if (acc < k_rem && acc + sum >= k_rem) {
-            for (int j = 0; j < bpt; ++j) {
-                if (acc + h[j] >= k_rem) {
-                    sc[0] = threadIdx.x * bpt + j;
-                    sc[1] = h[j] - (k_rem - acc);   // 0 <=> the whole bucket is taken
-                    sc[2] = k_rem - acc;
-                    break;
-                }
-                acc += h[j];
-            }
-        }
-        __syncthreads();
-        const int d = sc[0], surplus = sc[1];
-        k_rem = sc[2];
-        prefix |= (uint64_t)d << shift;
-        mask |= dmask << shift;
-        __syncthreads();
-        if (surplus == 0) break;
-        pos = shift;
     }
 }
 
@@ -556,22 +385,6 @@ __device__ void collect(const Cand &cand, int64_t E, uint64_t prefix, uint64_t m
     }
 }
 
-// the same for keys held in registers (KPT per thread; entry(u) names key u's entry)
-template <int KPT, class Entry>
-__device__ void collect_regs(const uint64_t (&k)[KPT], uint64_t prefix, uint64_t mask, int BW,
-                             const Entry &entry, const FinishSmem &f) {
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) {
-        if (k[u] != kNoKey && (k[u] & mask) <= prefix) {
-            const int pos = atomicAdd(f.cnt, 1);
-            if (pos < BW) {
-                f.win_k[pos] = k[u];
-                f.win_e[pos] = entry(u);
-            }
-        }
-    }
-}
-
 // Rank the n_win winners (unique keys; a winner's rank is its number of better
 // winners, counted by one warp per winner), write the outputs in rank order
 // and, when a.rewire, rewrite the request's beam state in place.  The caller
@@ -584,7 +397,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
     const int s = a.step;
     // sparse rewiring: each winner's trie child and the check of its token load
     // while the winners are ranked (winners i = threadIdx.x + u * blockDim.x)
-    constexpr int kWinPerThread = 2;   // BW <= 1024 <= 2 * blockDim.x
+    constexpr int kWinPerThread = 4;   // BW <= 1024 <= 4 * blockDim.x (blockDim.x >= 256)
     int child_c[kWinPerThread], child_t[kWinPerThread];
 #pragma unroll
     for (int u = 0; u < kWinPerThread; ++u) {
@@ -681,533 +494,642 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
     }
 }
 
+// ------------------------------------------------------------------ sparse steps
+
+// One launch per sparse step.  Request r gets sp_parts CTAs of kSpThreads
+// threads; CTA `part` takes beams [part*R, part*R + R) (R = sp_rows), one warp
+// per beam at a time, so no reduction spans more than one warp.  Per beam:
+//  * logits mode: the row's log-sum-exp over the full vocabulary, streamed
+//    from HBM in 16-byte loads with the next batch in flight while the current
+//    one is folded (online max / sum of exponentials per lane, then across
+//    the warp);
+//  * the key of every CSR entry (its score read back, an L2 hit in logits
+//    mode), written to the request's key buffer;
+//  * the beam's head: its m best keys with their entries, ascending (the
+//    page's per-beam ordered candidate list, cut at m).
+// Then each CTA takes a ticket; the last of the request's CTAs to arrive
+// selects for the whole request (select_request), so no second launch and no
+// grid-wide wait is needed.
+constexpr int kSpThreads = 256;
+constexpr int kSpWarps = kSpThreads / 32;
+constexpr int kSpKpc = 8;   // CSR entries per lane in one pass of the key loop
+constexpr int kLseU = 8;    // float4 per lane in one batch of the row stream
+
+__device__ __forceinline__ float4 ld_stream4(const float4 *p) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// natural-log log-sum-exp of x[0..V), by one warp (every lane gets it); a NaN
+// anywhere in the row sets XGR_DEV_NAN
+__device__ float warp_row_lse(const float *x, int V, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    float m = -INFINITY, s = 0.f;
+    bool nan = false;
+    auto fold = [&](const float *v, int k) {
+        float mv = -INFINITY;
+        for (int e = 0; e < k; ++e) {
+            nan |= v[e] != v[e];
+            mv = fmaxf(mv, v[e]);
+        }
+        if (mv > m) {
+            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
+            m = mv;
+        }
+        if (m != -INFINITY) {
+            const float mk = m * kLog2e;
+            for (int e = 0; e < k; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
+        }
+    };
+    if ((V & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+        const float4 *x4 = reinterpret_cast<const float4 *>(x);
+        const int n4 = V >> 2;
+        constexpr int kStep = 32 * kLseU;
+        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        float4 cur[kLseU];
+#pragma unroll
+        for (int u = 0; u < kLseU; ++u) {
+            const int i = u * 32 + lane;
+            cur[u] = i < n4 ? ld_stream4(x4 + i) : ninf;
+        }
+        for (int b0 = 0; b0 < n4; b0 += kStep) {
+            float4 nxt[kLseU];
+#pragma unroll
+            for (int u = 0; u < kLseU; ++u) {   // the next batch is in flight while this one folds
+                const int i = b0 + kStep + u * 32 + lane;
+                nxt[u] = i < n4 ? ld_stream4(x4 + i) : ninf;
+            }
+            float v[4 * kLseU];
+#pragma unroll
+            for (int u = 0; u < kLseU; ++u) {
+                v[4 * u] = cur[u].x;
+                v[4 * u + 1] = cur[u].y;
+                v[4 * u + 2] = cur[u].z;
+                v[4 * u + 3] = cur[u].w;
+            }
+            fold(v, 4 * kLseU);
+#pragma unroll
+            for (int u = 0; u < kLseU; ++u) cur[u] = nxt[u];
+        }
+    } else {
+        for (int i = lane; i < V; i += 32) fold(x + i, 1);
+    }
+    if (__any_sync(0xffffffffu, nan)) {
+        if (lane == 0) set_status(status, XGR_DEV_NAN);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_pair_merge(m, s, m2, s2);
+    }
+    return m + logf(s);
+}
+
+// Merges the keys c[] of every lane (entries ce[]) into the warp's running
+// head: afterwards lanes 0..m-1 hold the m smallest keys seen so far, in
+// ascending order (kNoKey pads), with their entries.  Keys are unique.  m
+// rounds of a warp minimum; c[] is consumed.
+template <int KPC>
+__device__ __forceinline__ void warp_head_merge(uint64_t (&c)[KPC], const int (&ce)[KPC], uint64_t &run,
+                                                int &run_e, int m) {
+    const int lane = threadIdx.x & 31;
+    uint64_t nrun = kNoKey;
+    int nrun_e = -1;
+    for (int i = 0; i < m; ++i) {
+        uint64_t lm = run;
+        int le = run_e, slot = KPC;
+#pragma unroll
+        for (int u = 0; u < KPC; ++u)
+            if (c[u] < lm) {
+                lm = c[u];
+                le = ce[u];
+                slot = u;
+            }
+        const uint64_t wm = warp_min_u64(lm);
+        if (wm == kNoKey) break;   // (uniform across the warp)
+        const int owner = __ffs(__ballot_sync(0xffffffffu, lm == wm)) - 1;   // keys are unique
+        const int we = __shfl_sync(0xffffffffu, le, owner);
+        if (lane == owner) {
+            if (slot == KPC) run = kNoKey;
+#pragma unroll
+            for (int u = 0; u < KPC; ++u)
+                if (u == slot) c[u] = kNoKey;
+        }
+        if (lane == i) {
+            nrun = wm;
+            nrun_e = we;
+        }
+    }
+    run = nrun;
+    run_e = nrun_e;
+}
+
+// Phase 1 of one beam row, by one warp: keys of its CSR entries into the key
+// buffer, its head (m best keys and entries, lanes 0..m-1) and its count of
+// valid candidates.
+__device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int base, uint64_t *keys) {
+    const int lane = threadIdx.x & 31;
+    const Dims dm = a.dims;
+    const int V = dm.V, m = a.head_m;
+    const int64_t row = (int64_t)r * dm.BW + b;
+    const bool live = b < n_live;
+    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
+    const float cum = a.cum[row];
+    const float *x = a.scores + row * V;
+    float lse = 0.f;
+    if (a.logits && live) lse = warp_row_lse(x, V, a.status);
+    const int n_e = max(0, end - beg);
+    uint64_t run = kNoKey;   // lane i < m: the i-th best key of the row so far
+    int run_e = -1;
+    int n_valid = 0;
+    for (int j0 = 0; j0 < n_e; j0 += 32 * kSpKpc) {
+        uint64_t c[kSpKpc];
+        int ce[kSpKpc];
+        int tk[kSpKpc];
+#pragma unroll
+        for (int u = 0; u < kSpKpc; ++u) {   // the entries' tokens (one round trip) ...
+            const int j = j0 + u * 32 + lane;
+            tk[u] = (j < n_e && live) ? a.cols[beg + j] : -1;
+        }
+        float sv[kSpKpc];
+#pragma unroll
+        for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (another)
+            sv[u] = (tk[u] >= 0 && tk[u] < V) ? __ldg(x + tk[u]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < kSpKpc; ++u) {
+            const int j = j0 + u * 32 + lane;
+            c[u] = kNoKey;
+            ce[u] = -1;
+            if (j >= n_e) continue;
+            const int e = beg + j;
+            uint64_t key = kNoKey;
+            if (live) {
+                if (tk[u] < 0 || tk[u] >= V) {
+                    set_status(a.status, XGR_DEV_MASK);
+                } else {
+                    const float lp = a.logits ? sv[u] - lse : sv[u];
+                    uint64_t k2;
+                    if (make_key(cum, lp, b, tk[u], V, a.status, k2)) key = k2;
+                }
+            }
+            if (e >= base && (int64_t)(e - base) < a.key_cap) keys[e - base] = key;
+            c[u] = key;
+            ce[u] = e - base;
+            n_valid += key != kNoKey;
+        }
+        warp_head_merge(c, ce, run, run_e, m);
+    }
+    n_valid = warp_sum_int(n_valid);
+    if (lane < m) {
+        a.head_k[row * m + lane] = run;
+        a.head_e[row * m + lane] = run_e;
+    }
+    if (lane == 0) {
+        a.row_cnt[row] = n_valid;
+        a.row_lse[row] = lse;
+    }
+}
+
+// exact radix select over the keys k[0..n) in shared memory (unique keys;
+// kNoKey entries are not candidates), by a block of kSpThreads threads, with
+// 8-bit digits starting at the highest bit where the smallest and largest key
+// differ.  On return exactly `want` keys satisfy (key & mask) <= prefix
+// (0 < want <= number of candidates).  hist: 256 ints; scan_w: 32 ints; red:
+// 32 u64; sc: 3 ints of shared memory.
+__device__ void smem_radix_select(const uint64_t *k, int n, int want, int *hist, int *scan_w,
+                                  uint64_t *red, int *sc, uint64_t &prefix, uint64_t &mask) {
+    const int tid = threadIdx.x;
+    uint64_t lo = kNoKey, hi = 0;
+    for (int i = tid; i < n; i += kSpThreads) {
+        const uint64_t key = k[i];
+        if (key == kNoKey) continue;
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+    }
+    lo = block_min_u64(lo, red);
+    hi = block_max_u64(hi, red);
+    const uint64_t diff = lo ^ hi;
+    if (diff == 0) {
+        prefix = lo;
+        mask = ~0ull;
+        return;
+    }
+    int pos = 64 - __clzll((long long)diff);
+    mask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
+    prefix = lo & mask;
+    int k_rem = want;
+    while (pos > 0) {
+        const int shift = pos > 8 ? pos - 8 : 0, width = pos - shift;
+        const uint64_t dmask = (1ull << width) - 1ull;
+        hist[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += kSpThreads) {
+            const uint64_t key = k[i];
+            if (key != kNoKey && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
+        }
+        __syncthreads();
+        const int h = hist[tid];
+        int total;
+        const int acc = block_exclusive_scan_int(h, scan_w, &total);
+        if (acc < k_rem && acc + h >= k_rem) {
+            sc[0] = tid;
+            sc[1] = h - (k_rem - acc);   // 0 <=> the whole bin is taken
+            sc[2] = k_rem - acc;
+        }
+        __syncthreads();
+        const int d = sc[0], surplus = sc[1];
+        k_rem = sc[2];
+        prefix |= (uint64_t)d << shift;
+        mask |= dmask << shift;
+        __syncthreads();
+        if (surplus == 0) break;
+        pos = shift;
+    }
+}
+
+__host__ __device__ inline int sparse_cand_cap(int BW, int m) { return BW * m; }
+__host__ __device__ inline int sparse_surv_cap(int BW) { return BW >= 1024 ? 4096 : (BW >= 256 ? 4 * BW : 1024); }
+
+size_t sparse_smem(const Dims &dm, int m) {
+    const int cc = sparse_cand_cap(dm.BW, m), scap = sparse_surv_cap(dm.BW);
+    return al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) + al16((size_t)scap * 4) +
+           al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) +
+           finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
+}
+
+// Phase 2, by the request's last CTA.  tau = the BW-th best of the beams'
+// heads: at least BW real candidates rank at or above it, so every winner
+// does.  Survivors = the head keys at or above tau, plus, for a beam whose
+// whole head survived and that has more entries than its head holds, its
+// further keys at or above tau from the key buffer.  Then the exact radix
+// select of the BW best survivors, the ordering, the outputs and the
+// rewiring.  Exact fallbacks: survivors beyond the shared-memory buffer select
+// from the key buffer; a request with more CSR entries than the key buffer
+// holds selects from the scores.
+__device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *hist, int *scan_w,
+                               uint64_t *red_k, int *sc, int *red_i) {
+    const Dims dm = a.dims;
+    const int BW = dm.BW, m = a.head_m, tid = threadIdx.x;
+    const int64_t rb = (int64_t)r * BW;
+    const int cc = sparse_cand_cap(BW, m), scap = sparse_surv_cap(BW);
+    uint8_t *p = smem;
+    uint64_t *hk = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)cc * 8);
+    int *he = reinterpret_cast<int *>(p);
+    p += al16((size_t)cc * 4);
+    uint64_t *sk = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)scap * 8);
+    int *se = reinterpret_cast<int *>(p);
+    p += al16((size_t)scap * 4);
+    int *sat = reinterpret_cast<int *>(p);   // beams whose further keys must be read
+    p += al16((size_t)(BW + 1) * 4);
+    float *cum_s = reinterpret_cast<float *>(p);
+    p += al16((size_t)BW * 4);
+    float *lse_s = reinterpret_cast<float *>(p);
+    p += al16((size_t)BW * 4);
+    const FinishSmem f = carve_finish(p, BW, BW, dm.S, 0);
+    int *cnts = reinterpret_cast<int *>(p + finish_bytes(BW, BW, dm.S, 0));   // [0] survivors, [1] saturated
+
+    // every load below is independent of the others: one round trip
+    const int n = min(max(a.n_live[r], 0), BW);
+    const int base = a.row_ptr[rb];
+    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;
+    for (int i = tid; i < BW * m; i += kSpThreads) {
+        const int b = i / m;
+        hk[i] = b < n ? __ldcg(a.head_k + rb * m + i) : kNoKey;
+        he[i] = __ldcg(a.head_e + rb * m + i);
+    }
+    int c = 0;
+    for (int b = tid; b < BW; b += kSpThreads) c += b < n ? __ldcg(a.row_cnt + rb + b) : 0;
+    for (int b = tid; b <= BW; b += kSpThreads) f.rp[b] = a.row_ptr[rb + b] - base;
+    if (a.rewire) stage_rows(a, rb, n, f);
+    if (E > a.key_cap)
+        for (int b = tid; b < n; b += kSpThreads) {
+            cum_s[b] = a.cum[rb + b];
+            lse_s[b] = a.logits ? __ldcg(a.row_lse + rb + b) : 0.f;
+        }
+    if (tid == 0) {
+        *f.cnt = 0;
+        cnts[0] = 0;
+        cnts[1] = 0;
+    }
+    const int total = block_sum_int(c, red_i);   // valid candidates of the request (+ a barrier)
+    if (a.rewire) stage_children(a, n, f);
+    const int want = min(BW, total);
+    uint64_t prefix = ~0ull, mask = 0;
+    const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
+    if (E > a.key_cap) {
+        // the key buffer overflowed: exact selection over every candidate
+        __syncthreads();
+        ReqCand cand;
+        cand.x = a.scores + rb * dm.V;
+        cand.cols = a.cols + base;
+        cand.rp = f.rp;
+        cand.cum = cum_s;
+        cand.lse = lse_s;
+        cand.status = a.status;
+        cand.n = n;
+        cand.logits = a.logits;
+        cand.V = dm.V;
+        if (want > 0 && want < total) radix_select(cand, f.rp[n], want, hist, sc, prefix, mask);
+        collect(cand, f.rp[n], prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+    } else if (want > 0) {
+        // tau from the heads (every head key is a real candidate)
+        int c0 = 0;
+        for (int i = tid; i < BW * m; i += kSpThreads) c0 += hk[i] != kNoKey;
+        const int in_heads = block_sum_int(c0, red_i);
+        uint64_t tau = kNoKey;
+        if (total > BW && in_heads >= BW) {
+            uint64_t tp, tm;
+            smem_radix_select(hk, BW * m, BW, hist, scan_w, red_k, sc, tp, tm);
+            uint64_t t = 0;
+            for (int i = tid; i < BW * m; i += kSpThreads)
+                if (hk[i] != kNoKey && (hk[i] & tm) <= tp) t = hk[i] > t ? hk[i] : t;
+            tau = block_max_u64(t, red_k);
+        }
+        // survivors from the heads; beams whose whole head survived and that have
+        // more entries go on the saturated list
+        for (int i = tid; i < BW * m; i += kSpThreads) {
+            const uint64_t key = hk[i];
+            if (key == kNoKey || key > tau) continue;
+            const int pos = atomicAdd(&cnts[0], 1);
+            if (pos < scap) {
+                sk[pos] = key;
+                se[pos] = he[i];
+            }
+            const int b = i / m;
+            if (i % m == m - 1 && f.rp[b + 1] - f.rp[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
+        }
+        __syncthreads();
+        const int n_sat = cnts[1];
+        for (int q = 0; q < n_sat; ++q) {   // their keys beyond the head (worse than its last)
+            const int b = sat[q];
+            const uint64_t last = hk[b * m + m - 1];
+            for (int e = max(f.rp[b], 0) + tid; e < (int)min((int64_t)f.rp[b + 1], E); e += kSpThreads) {
+                const uint64_t key = __ldcg(keys + e);
+                if (key == kNoKey || key > tau || key <= last) continue;
+                const int pos = atomicAdd(&cnts[0], 1);
+                if (pos < scap) {
+                    sk[pos] = key;
+                    se[pos] = e;
+                }
+            }
+        }
+        __syncthreads();
+        const int ns = cnts[0];
+        if (ns <= scap) {
+            if (want < ns) smem_radix_select(sk, ns, want, hist, scan_w, red_k, sc, prefix, mask);
+            collect(ListCand<false>{sk}, ns, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
+        } else {   // more survivors than the buffer: exact selection over the key buffer
+            const KeyCand cand{keys, tau};
+            radix_select(cand, E, want, hist, sc, prefix, mask);
+            collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+        }
+    }
+    __syncthreads();
+    finish_request(a, r, min(*f.cnt, want), f);
+}
+
+__global__ void __launch_bounds__(kSpThreads) select_sparse_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int hist[256];
+    __shared__ int scan_w[32];
+    __shared__ int red_i[32];
+    __shared__ uint64_t red_k[32];
+    __shared__ int sc[4];
+    __shared__ int last;
+    const Dims dm = a.dims;
+    const int C = a.sp_parts, R = a.sp_rows;
+    const int r = blockIdx.x / C, part = blockIdx.x % C;
+    const int warp = threadIdx.x / 32;
+    const int64_t rb = (int64_t)r * dm.BW;
+    const int n_live = min(max(a.n_live[r], 0), dm.BW);
+    const int base = a.row_ptr[rb];
+    uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
+    const int b1 = min(dm.BW, part * R + R);
+    for (int b = part * R + warp; b < b1; b += kSpWarps) sparse_row(a, r, b, n_live, base, keys);
+    // the request's last CTA to arrive selects
+    __threadfence();   // this thread's keys and head are visible before the ticket
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&a.ticket[r], 1u) == (unsigned)(C - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    select_request(a, r, smem, hist, scan_w, red_k, sc, red_i);
+    if (threadIdx.x == 0) a.ticket[r] = 0;   // zero again for the next call
+}
+
 // ------------------------------------------------------------------ dense step
 
+// The first step: one live beam per request and the dense bitset of valid
+// first tokens.  One CTA of kSpThreads per request: the beam's score row is
+// staged by one bulk copy; its log-sum-exp from per-warp partials; then the
+// row is cut into slices of Z tokens, and a warp takes the key of every valid
+// token of a slice and the slice's head (its m best keys, in order).  tau =
+// the BW-th best head key; the survivors -- head keys at or above tau, plus
+// the further keys of slices whose whole head survived, recomputed from the
+// staged row -- go through the exact radix select, then finish_request.
+// Z is chosen so that the heads hold at least 2*BW keys where the row allows.
+__host__ __device__ inline int dense_slice(int V, int BW, int m) {
+    const int64_t z = ((int64_t)V * m / (2 * (int64_t)BW)) / 32 * 32;
+    return (int)(z < 32 ? 32 : (z > 256 ? 256 : z));
+}
+__host__ __device__ inline int dense_heads(int V, int BW, int m) {
+    const int z = dense_slice(V, BW, m);
+    return (V + z - 1) / z * m;
+}
+__host__ __device__ inline int dense_surv_cap(int BW) { return BW >= 512 ? 4 * BW : 2048; }
 __host__ __device__ inline size_t dense_x_bytes(int V) { return al16((size_t)V * 4); }
 __host__ __device__ inline size_t dense_bits_bytes(int V) { return al16((size_t)((V + 31) / 32) * 4); }
 
-size_t dense_smem(const Dims &dm) {
-    return dense_x_bytes(dm.V) + dense_bits_bytes(dm.V) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32);
+size_t dense_smem(const Dims &dm, int m) {
+    const int nh = dense_heads(dm.V, dm.BW, m), scap = dense_surv_cap(dm.BW);
+    return dense_x_bytes(dm.V) + dense_bits_bytes(dm.V) + al16((size_t)nh * 8) + al16((size_t)nh * 4) +
+           al16((size_t)scap * 8) + al16((size_t)scap * 4) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32) +
+           64;
 }
 
-__global__ void __launch_bounds__(kDenseThreads, 1) select_dense_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bar_mem;
-    __shared__ float red_f[72];
+    __shared__ float red_f[2 * kSpWarps];
     __shared__ int red_i[32];
+    __shared__ int scan_w[32];
     __shared__ uint64_t red_k[32];
     __shared__ int hist[256];
-    __shared__ int whist[kWideBins];
     __shared__ int sc[4];
+    __shared__ int cnts[2];
     const Dims dm = a.dims;
-    const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32;
-    const int r = blockIdx.x, tid = threadIdx.x;
+    const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32, m = a.head_m;
+    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rb = (int64_t)r * BW;
-    float *x = reinterpret_cast<float *>(smem);
-    uint32_t *bits = reinterpret_cast<uint32_t *>(smem + dense_x_bytes(V));
-    const FinishSmem f = carve_finish(smem + dense_x_bytes(V) + dense_bits_bytes(V), BW, 1, dm.S, nw);
+    const int Z = dense_slice(V, BW, m), n_sl = (V + Z - 1) / Z, nh = n_sl * m;
+    const int scap = dense_surv_cap(BW);
+    uint8_t *p = smem;
+    float *x = reinterpret_cast<float *>(p);
+    p += dense_x_bytes(V);
+    uint32_t *bits = reinterpret_cast<uint32_t *>(p);
+    p += dense_bits_bytes(V);
+    uint64_t *hk = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)nh * 8);
+    int *he = reinterpret_cast<int *>(p);
+    p += al16((size_t)nh * 4);
+    uint64_t *sk = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)scap * 8);
+    int *se = reinterpret_cast<int *>(p);
+    p += al16((size_t)scap * 4);
+    const FinishSmem f = carve_finish(p, BW, 1, dm.S, nw);
     const float *xg = a.scores + rb * V;   // beam 0 of request r
     const uint32_t bar = smem_u32(&bar_mem);
     const bool bulk = (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
+    const int n = min(max(a.n_live[r], 0), 1);
     if (tid == 0) {
         *f.cnt = 0;
-        if (bulk) {
+        cnts[0] = 0;
+        cnts[1] = 0;
+        if (bulk && n > 0) {
             mbar_init(bar, 1);
             fence_mbar_init();
             mbar_expect_tx(bar, (uint32_t)V * 4u);
             bulk_g2s(smem_u32(x), xg, (uint32_t)V * 4u, bar);
         }
     }
-    const int n = min(a.n_live[r], 1);
     const float cum = a.cum[rb];
-    for (int w = tid; w < nw; w += blockDim.x) bits[w] = a.bits[w];
+    // the mask with the tokens past V cleared; the valid-candidate count
+    int c = 0;
+    for (int w = tid; w < nw; w += kSpThreads) {
+        const uint32_t v = a.bits[w] & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u);
+        bits[w] = v;
+        c += __popc(v);
+    }
     if (a.rewire) {
         stage_rows(a, rb, n, f);
-        // root children: bitset and exclusive prefix popcounts (trie order = token order)
         if (a.trie.root_bits) {
-            int c = 0;
-            for (int w = tid; w < nw; w += blockDim.x) {   // nw <= blockDim.x (V <= 32768)
-                const uint32_t v = a.trie.root_bits[w];
-                f.root[w] = v;
-                c = __popc(v);
-            }
-            // block exclusive scan of one count per thread
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (tid % 32 >= o) incl += t;
-            }
-            if (tid % 32 == 31) red_i[tid / 32] = incl;
-            __syncthreads();
-            if (tid < 32) {
-                const int wv = red_i[tid];
-                int wi = wv;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int t = __shfl_up_sync(0xffffffffu, wi, o);
-                    if (tid >= o) wi += t;
+            // root children: bitset and exclusive prefix popcounts (trie order =
+            // token order); thread t owns words [t*wpt, t*wpt + wpt)
+            const int wpt = (nw + kSpThreads - 1) / kSpThreads;
+            int cw = 0;
+            for (int k = 0; k < wpt; ++k) {
+                const int w = tid * wpt + k;
+                if (w < nw) {
+                    const uint32_t v = a.trie.root_bits[w];
+                    f.root[w] = v;
+                    cw += __popc(v);
                 }
-                red_i[tid] = wi - wv;
             }
-            __syncthreads();
-            if (tid < nw) f.root[nw + tid] = (uint32_t)(red_i[tid / 32] + incl - c);
-            __syncthreads();
+            int tot;
+            int pre = block_exclusive_scan_int(cw, scan_w, &tot);
+            for (int k = 0; k < wpt; ++k) {
+                const int w = tid * wpt + k;
+                if (w < nw) {
+                    f.root[nw + w] = (uint32_t)pre;
+                    pre += __popc(f.root[w]);
+                }
+            }
         }
     }
-    if (!bulk)
-        for (int i = tid; i < V; i += blockDim.x) x[i] = xg[i];
-    __syncthreads();
-    if (bulk && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
-    float lse = 0.f;
-    if (a.logits && n > 0) lse = block_lse(x, V, red_f, a.status);
-    int c = 0;   // candidates: mask bits below V
-    for (int w = tid; w < nw; w += blockDim.x)
-        c += __popc(bits[w] & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u));
-    const int total = n > 0 ? block_sum_int(c, red_i) : 0;
+    if (!bulk && n > 0)
+        for (int i = tid; i < V; i += kSpThreads) x[i] = xg[i];
+    const int total = n > 0 ? block_sum_int(c, red_i) : 0;   // (+ a barrier)
+    if (bulk && n > 0 && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
     const int want = min(BW, total);
+    float lse = 0.f;
+    if (a.logits && want > 0) {   // per-warp (max, sum) over a slice, then combined
+        const int per = (V + kSpWarps - 1) / kSpWarps;
+        float mw = -INFINITY, sw = 0.f;
+        bool nan = false;
+        for (int i = warp * per + lane; i < min(V, warp * per + per); i += 32) {
+            const float v = x[i];
+            nan |= v != v;
+            lse_pair_merge(mw, sw, v, 1.f);
+        }
+        if (__any_sync(0xffffffffu, nan) && lane == 0) set_status(a.status, XGR_DEV_NAN);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mw, o), s2 = __shfl_xor_sync(0xffffffffu, sw, o);
+            lse_pair_merge(mw, sw, m2, s2);
+        }
+        if (lane == 0) {
+            red_f[2 * warp] = mw;
+            red_f[2 * warp + 1] = sw;
+        }
+        __syncthreads();
+        float M = red_f[0], Ssum = red_f[1];
+        for (int k = 1; k < kSpWarps; ++k) lse_pair_merge(M, Ssum, red_f[2 * k], red_f[2 * k + 1]);
+        lse = M + logf(Ssum);
+    }
     DenseCand cand{x, bits, cum, lse, V, a.logits, a.status};
-    const int64_t E = n > 0 ? V : 0;
     uint64_t prefix = ~0ull, mask = 0;
-    if (V <= 8 * kDenseThreads) {   // every key computed once, held in registers
-        uint64_t kr[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = tid + u * kDenseThreads;
-            uint64_t key = kNoKey;
-            kr[u] = (t < E && cand(t, key)) ? key : kNoKey;
-        }
-        if (want < total) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask);
-        collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kDenseThreads; }, f);
-    } else {
-        if (want < total) radix_select(cand, E, want, hist, sc, prefix, mask);
-        collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
-    }
-    __syncthreads();
-    finish_request(a, r, min(*f.cnt, want), f);
-}
-
-// ------------------------------------------------------------------ sparse steps
-
-// One persistent CTA per SM takes a contiguous block of beam rows.  It reads
-// the metadata of a window of its rows (row pointers, cumulative scores, live
-// counts) in one round trip and the window's CSR tokens -- one contiguous range
-// -- in another (log-prob mode: then the tokens' scores), all into shared
-// memory.  In logits mode the score rows stream through nbuf slots by bulk
-// copies issued nbuf rows ahead, so the HBM traffic overlaps the work on
-// earlier rows.  Eight groups of four warps work on eight rows at a time.  Per row:
-// the log-sum-exp (logits), each entry's key beside its CSR position, the
-// row's best key.
-constexpr int kRowsThreads = 1024;
-constexpr int kRowsGroups = 8;   // rows in work at once (more, smaller groups measured faster)
-constexpr int kRowsGroup = kRowsThreads / kRowsGroups;
-constexpr int kRowsMaxBuf = 8;
-constexpr int kRowsWin = 256;     // rows per metadata window
-constexpr int kRowsTok = 8192;    // CSR entries staged per window (a longer row reads the rest in place)
-
-__host__ __device__ inline size_t rows_fixed_bytes(bool logits) {
-    return (size_t)kRowsTok * 4 * (logits ? 1 : 2) + (size_t)(kRowsWin + 1) * 4 + (size_t)kRowsWin * 12;
-}
-
-__global__ void __launch_bounds__(kRowsThreads, 1) select_rows_kernel(SelectArgs a, int nbuf) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t full[kRowsMaxBuf];
-    __shared__ int slot_row[kRowsMaxBuf];   // the row (index in the block) whose copy a slot holds
-    constexpr int kGroupWarps = kRowsGroup / 32;
-    __shared__ float red_f[2 * kGroupWarps * kRowsGroups];   // per group: (m, s) of each warp
-    __shared__ uint64_t red_k[kGroupWarps * kRowsGroups];   // per group: each warp's min
-    __shared__ int win_end;
-    const Dims dm = a.dims;
-    const int V = dm.V, BW = dm.BW, tid = threadIdx.x;
-    const int64_t n_rows = (int64_t)dm.B * BW;
-    const int64_t per = (n_rows + gridDim.x - 1) / gridDim.x;
-    const int64_t r0 = (int64_t)blockIdx.x * per, r1 = min(n_rows, r0 + per);
-    const bool stage = a.logits;   // logits: whole rows (their log-sum-exp)
-    const bool bulk = stage && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0;
-    const size_t xb = stage ? al16((size_t)V * 4) : 0;
-    uint8_t *p = smem + nbuf * xb;
-    int *tok = reinterpret_cast<int *>(p);
-    p += (size_t)kRowsTok * 4;
-    float *val = reinterpret_cast<float *>(p);   // log-prob mode only
-    if (!stage) p += (size_t)kRowsTok * 4;
-    int *rp = reinterpret_cast<int *>(p);        // [kRowsWin + 1]
-    p += (size_t)(kRowsWin + 1) * 4;
-    float *cum_w = reinterpret_cast<float *>(p);  // [kRowsWin]
-    int *nl_w = reinterpret_cast<int *>(cum_w + kRowsWin);   // [kRowsWin] live beams of the row's request
-    int *base_w = nl_w + kRowsWin;                           // [kRowsWin] first entry of the row's request
-    auto x_of = [&](int64_t row) { return reinterpret_cast<float *>(smem + ((row - r0) % nbuf) * xb); };
-    auto issue = [&](int64_t row) {   // one thread: the bulk copy of a row into its slot
-        const uint32_t bar = smem_u32(&full[(row - r0) % nbuf]);
-        reinterpret_cast<volatile int *>(slot_row)[(row - r0) % nbuf] = (int)(row - r0);
-        mbar_expect_tx(bar, (uint32_t)V * 4u);
-        bulk_g2s(smem_u32(x_of(row)), a.scores + row * V, (uint32_t)V * 4u, bar);
-    };
-    // The last thread (it has no window metadata to load while the windows hold
-    // far fewer rows than threads) sets up the slots and starts the first rows'
-    // bulk copies at once; the other threads meanwhile load the first window.
-    constexpr int kIssuer = kRowsThreads - 1;
-    static_assert(kRowsWin < kIssuer, "the issuing thread loads no window metadata");
-    if (tid == kIssuer && bulk) {
-        for (int k = 0; k < nbuf; ++k) {
-            mbar_init(smem_u32(&full[k]), 1);
-            slot_row[k] = -1;
-        }
-        fence_mbar_init();
-        for (int64_t row = r0; row < min(r1, r0 + nbuf); ++row) issue(row);
-    }
-    // Every other load of a row's work happens per window, ahead of the rows: a
-    // global load issued behind the bulk traffic waits microseconds.
-    for (int64_t w0 = r0; w0 < r1;) {
-        // ---- window metadata: one round trip
-        const int64_t wmax = min(r1, w0 + kRowsWin);
-        for (int64_t row = w0 + tid; row <= wmax; row += kRowsThreads) {
-            rp[row - w0] = a.row_ptr[row];
-            if (row < wmax) {
-                cum_w[row - w0] = a.cum[row];
-                nl_w[row - w0] = a.n_live[row / BW];
-                base_w[row - w0] = a.row_ptr[row / BW * BW];
-            }
-        }
-        __syncthreads();
-        // rows whose entries fit the token area (at least one row)
-        if (tid == 0) {
-            int64_t w1 = w0 + 1;
-            while (w1 < wmax && rp[w1 + 1 - w0] - rp[0] <= kRowsTok) ++w1;
-            win_end = (int)(w1 - w0);
-        }
-        __syncthreads();
-        const int64_t w1 = w0 + win_end;
-        const int t0 = rp[0], nt = min(rp[w1 - w0] - t0, kRowsTok);
-        // ---- the window's tokens (one contiguous range), then log-prob scores
-        for (int j = tid; j < nt; j += kRowsThreads) {
-            const int t = a.cols[t0 + j];
-            tok[j] = t;
-            if (!stage) {
-                // entry j's row: the last window row whose first entry is <= j
-                int l = 0, h = (int)(w1 - w0);
-                while (h - l > 1) {
-                    const int m = (l + h) >> 1;
-                    if (rp[m] - t0 <= j) l = m; else h = m;
-                }
-                const int64_t row = w0 + l;
-                val[j] = (t >= 0 && t < V) ? a.scores[row * V + t] : 0.f;
-            }
-        }
-        __syncthreads();
-        // ---- the window's rows: group g (256 threads, named barrier 1 + g) takes
-        // rows w0 + g, w0 + g + 4, ...; when it is done with a row it starts the
-        // copy of the row nbuf places later into the same slot
-        const Group grp{1 + tid / kRowsGroup, kRowsGroup, tid % kRowsGroup};
-        const int gi = tid / kRowsGroup;
-        for (int64_t row = w0 + gi; row < w1; row += kRowsGroups) {
-            const int r = (int)(row / BW), b = (int)(row % BW);
-            const int i = (int)(row - w0);
-            const bool live = b < nl_w[i];
-            if (b == 0 && grp.t == 0) {   // the pick kernel counts from 0
-                a.surv_cnt[r] = 0;
-                a.ticket[r] = 0;
-            }
-            const float *xg = a.scores + row * V;
-            float *x = x_of(row);
-            if (stage && !bulk) {   // unaligned rows: plain loads into the slot
-                for (int t = grp.t; t < V; t += kRowsGroup) x[t] = xg[t];
-                grp.sync();
-            }
-            if (bulk) {
-                // a slot serves rows nbuf apart, taken by different groups: wait until
-                // this row's copy is the one in flight, then for its bytes
-                const int k = (int)((row - r0) % nbuf);
-                bool ok = false;
-                for (uint32_t it = 0; it < kSpinLimit && !ok; ++it)
-                    ok = reinterpret_cast<volatile int *>(slot_row)[k] == (int)(row - r0);
-                if (!ok || !mbar_wait(smem_u32(&full[k]), (int)((row - r0) / nbuf) & 1, nullptr))
-                    set_status(a.status, XGR_DEV_TIMEOUT);
-            }
-            float lse = 0.f;
-            if (stage && live) lse = group_lse(x, V, red_f + 2 * kGroupWarps * gi, a.status, grp);
-            const int beg = rp[i], end = rp[i + 1], n_e = max(0, end - beg);
-            uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-            const int base = base_w[i];
-            const float cum = cum_w[i];
-            uint64_t best = kNoKey;
-            for (int j = grp.t; j < n_e; j += kRowsGroup) {
-                const int e = beg + j, ew = e - t0;   // entry, its place in the window's tokens
-                const bool staged = ew >= 0 && ew < nt;
-                uint64_t key = kNoKey;
-                if (live) {
-                    const int t = staged ? tok[ew] : a.cols[e];
-                    if (t < 0 || t >= V) {
-                        set_status(a.status, XGR_DEV_MASK);
-                    } else {
-                        float lp = stage ? x[t] : (staged ? val[ew] : xg[t]);
-                        if (a.logits) lp -= lse;
-                        uint64_t k2;
-                        if (make_key(cum, lp, b, t, V, a.status, k2)) key = k2;
-                    }
-                }
-                if (e >= base && (int64_t)(e - base) < a.key_cap) keys[e - base] = key;
-                best = key < best ? key : best;
-            }
-            best = group_min_u64(best, red_k + kGroupWarps * gi, grp);   // (its barriers end every read of the slot)
-            if (grp.t == 0) {
-                a.best[row] = best;
-                a.row_lse[row] = lse;
-                if (bulk && row + nbuf < r1) issue(row + nbuf);
-            }
-        }
-        w0 = w1;
-        __syncthreads();   // the window's shared metadata is reused
-    }
-}
-
-size_t pick_smem(const Dims &dm) {
-    return (size_t)kSmemSurv * 12 + finish_bytes(dm.BW, dm.BW, dm.S, 0) + al16((size_t)dm.BW * 8);
-}
-
-__global__ void __launch_bounds__(kPickThreads, 1) select_pick_kernel(SelectArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t red_k[32];
-    __shared__ int hist[256];
-    __shared__ int sc[4];
-    __shared__ int last;
-    __shared__ int scan_w[32];
-    __shared__ int red_i[32];
-    __shared__ int whist[kWideBins];
-    __shared__ int slice_base;
-    const Dims dm = a.dims;
-    const int BW = dm.BW, P = a.pick_parts;
-    const int r = blockIdx.x / P, part = blockIdx.x % P;
-    const int tid = threadIdx.x;
-    const int64_t rb = (int64_t)r * BW;
-    const int n = a.n_live[r];
-    const int base = a.row_ptr[rb];
-    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;   // dead rows' entries hold kNoKey
-    // tau: the worst of the live beams' best keys, when all BW beams are live
-    uint64_t worst = 0;
-    for (int b = tid; b < BW; b += kPickThreads) {
-        const uint64_t k = a.best[rb + b];
-        if (b < n) worst = k > worst ? k : worst;
-    }
-    worst = block_max_u64(worst, red_k);
-    const uint64_t tau = n == BW ? worst : kNoKey;
-    const bool fits = E <= a.key_cap;
-    const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-    uint64_t *sk_g = a.surv_key + (int64_t)r * a.surv_cap;
-    int32_t *se_g = a.surv_e + (int64_t)r * a.surv_cap;
-    if (fits) {
-        // survivors of each slice: a block scan of the per-thread counts, one
-        // atomic per slice for the slice's place in the request's buffer
-        constexpr int U = kPickKeys / kPickThreads;
-        for (int64_t s0 = (int64_t)part * kPickKeys; s0 < E; s0 += (int64_t)P * kPickKeys) {
-            uint64_t k[U];
-            int c = 0;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int64_t e = s0 + tid + u * kPickThreads;
-                k[u] = e < E ? __ldcg(keys + e) : kNoKey;
-                c += k[u] != kNoKey && k[u] <= tau;
-            }
-            int n_slice;
-            int pos = block_exclusive_scan_int(c, scan_w, &n_slice);
-            if (tid == 0) slice_base = n_slice ? atomicAdd(&a.surv_cnt[r], n_slice) : 0;
-            __syncthreads();
-            pos += slice_base;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (k[u] == kNoKey || k[u] > tau) continue;
-                if (pos < a.surv_cap) {
-                    sk_g[pos] = k[u];
-                    se_g[pos] = (int32_t)(s0 + tid + u * kPickThreads);
-                }
-                ++pos;
-            }
-            __syncthreads();   // slice_base is reused
-        }
-    }
-    // the last CTA of the request to finish its slices takes the selection
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last = atomicAdd(&a.ticket[r], 1u) == (unsigned)(P - 1);
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-
-    uint64_t *sk = reinterpret_cast<uint64_t *>(smem);
-    int *se = reinterpret_cast<int *>(smem + (size_t)kSmemSurv * 8);
-    uint8_t *fin = smem + (size_t)kSmemSurv * 12;
-    const FinishSmem f = carve_finish(fin, BW, BW, dm.S, 0);
-    float *cum_s = reinterpret_cast<float *>(fin + finish_bytes(BW, BW, dm.S, 0));
-    float *lse_s = cum_s + BW;
-    const int T = __ldcg(&a.surv_cnt[r]);
-    if (tid == 0) *f.cnt = 0;
-    for (int b = tid; b <= n; b += kPickThreads) f.rp[b] = a.row_ptr[rb + b] - base;
-    if (a.rewire) stage_rows(a, rb, n, f);
-    if (!fits)
-        for (int b = tid; b < n; b += kPickThreads) {
-            cum_s[b] = a.cum[rb + b];
-            lse_s[b] = a.logits ? a.row_lse[rb + b] : 0.f;
-        }
-    __syncthreads();
-    // the survivors and the parents' child ranges load together
-    const bool in_smem = fits && T <= kSmemSurv;
-    if (in_smem) {
-        for (int i = tid; i < T; i += kPickThreads) {
-            sk[i] = __ldcg(sk_g + i);
-            se[i] = __ldcg(se_g + i);
-        }
-    }
-    if (a.rewire) stage_children(a, n, f);
-    __syncthreads();
-    uint64_t prefix = ~0ull, mask = 0;
-    int want;
-    if (fits) {
-        // every winner survived tau; T >= BW whenever tau cuts anything
-        want = min(BW, T);
-        if (in_smem) {   // the survivors' keys in registers, 8 per thread
-            static_assert(kSmemSurv == 8 * kPickThreads, "survivors per thread");
-            uint64_t kr[8];
+    if (want > 0) {
+        // keys and heads: warp w takes slices w, w + 8, ...
+        for (int sl = warp; sl < n_sl; sl += kSpWarps) {
+            uint64_t ck[8];
+            int cke[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int i = tid + u * kPickThreads;
-                kr[u] = i < T ? sk[i] : kNoKey;
+                const int t = sl * Z + u * 32 + lane;
+                uint64_t key = kNoKey;
+                if (u * 32 < Z && t < V) cand(t, key);
+                ck[u] = key;
+                cke[u] = t;
             }
-            if (want < T) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask);
-            collect_regs(kr, prefix, mask, BW, [&](int u) { return se[tid + u * kPickThreads]; }, f);
-        } else if (T <= a.surv_cap) {
-            const ListCand<true> cand{sk_g};
-            if (want < T) radix_select(cand, T, want, hist, sc, prefix, mask);
-            collect(cand, T, prefix, mask, BW, [&](int64_t i) { return __ldcg(se_g + i); }, f);
-        } else {
-            const KeyCand cand{keys, tau};
-            if (want < T) radix_select(cand, E, want, hist, sc, prefix, mask);
-            collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+            uint64_t run = kNoKey;
+            int run_e = -1;
+            warp_head_merge(ck, cke, run, run_e, m);
+            if (lane < m) {
+                hk[sl * m + lane] = run;
+                he[sl * m + lane] = run_e;
+            }
         }
-    } else {
-        // the key buffer overflowed: exact selection over every candidate
-        ReqCand cand;
-        cand.x = a.scores + rb * dm.V;
-        cand.cols = a.cols + base;
-        cand.rp = f.rp;
-        cand.cum = cum_s;
-        cand.lse = lse_s;
-        cand.status = a.status;
-        cand.n = n;
-        cand.logits = a.logits;
-        cand.V = dm.V;
-        const int total = f.rp[n];
-        want = min(BW, total);
-        if (want < total) radix_select(cand, total, want, hist, sc, prefix, mask);
-        collect(cand, total, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
-    }
-    __syncthreads();
-    finish_request(a, r, min(*f.cnt, want), f);
-}
-
-// ---- requests of few CSR entries: one CTA each, every key in registers
-
-constexpr int kPickOneThreads = 1024;
-constexpr int kPickOneKpt = 16;          // keys per thread in registers
-constexpr int kPickOneTail = 16384;      // further keys in shared memory
-constexpr int kPickOneMax = kPickOneKpt * kPickOneThreads + kPickOneTail;
-
-size_t pick_one_smem(const Dims &dm) {
-    return (size_t)kPickOneTail * 8 + finish_bytes(dm.BW, dm.BW, dm.S, 0) + al16((size_t)dm.BW * 8);
-}
-
-// One CTA per request: the request's keys go straight into registers and a
-// shared-memory tail (no threshold pass, no survivor buffer), then the exact
-// radix select, ordering, outputs and rewiring.  Requests with more entries
-// select from the key buffer in global memory (or, past the buffer, from the
-// scores), exactly as the multi-CTA pick does.
-__global__ void __launch_bounds__(kPickOneThreads, 1) select_pick_one_kernel(SelectArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int hist[256];
-    __shared__ int sc[4];
-    __shared__ int red_i[32];
-    __shared__ uint64_t red_k[32];
-    __shared__ int whist[kWideBins];
-    const Dims dm = a.dims;
-    const int BW = dm.BW, r = blockIdx.x, tid = threadIdx.x;
-    const int64_t rb = (int64_t)r * BW;
-    uint64_t *tail = reinterpret_cast<uint64_t *>(smem);
-    uint8_t *fin = smem + (size_t)kPickOneTail * 8;
-    const FinishSmem f = carve_finish(fin, BW, BW, dm.S, 0);
-    float *cum_s = reinterpret_cast<float *>(fin + finish_bytes(BW, BW, dm.S, 0));
-    float *lse_s = cum_s + BW;
-    const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-    constexpr int kReg = kPickOneKpt * kPickOneThreads;
-    // every load below is independent of the others: one round trip
-    const int n = a.n_live[r];
-    const int base = a.row_ptr[rb];
-    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;   // dead rows' entries hold kNoKey
-    uint64_t kr[kPickOneKpt];
-#pragma unroll
-    for (int u = 0; u < kPickOneKpt; ++u) {
-        const int64_t e = tid + u * kPickOneThreads;
-        kr[u] = e < a.key_cap ? __ldcg(keys + e) : kNoKey;
-    }
-    if (tid == 0) *f.cnt = 0;
-    for (int b = tid; b <= BW; b += kPickOneThreads) f.rp[b] = a.row_ptr[rb + b] - base;
-    if (a.rewire) stage_rows(a, rb, BW, f);
-    const bool in_smem = E <= a.key_cap && E <= kPickOneMax;
-    const int n_tail = in_smem && E > kReg ? (int)(E - kReg) : 0;
-    for (int i = tid; i < n_tail; i += kPickOneThreads) tail[i] = __ldcg(keys + kReg + i);
-    if (E > a.key_cap)
-        for (int b = tid; b < n; b += kPickOneThreads) {
-            cum_s[b] = a.cum[rb + b];
-            lse_s[b] = a.logits ? a.row_lse[rb + b] : 0.f;
+        __syncthreads();
+        int c0 = 0;
+        for (int i = tid; i < nh; i += kSpThreads) c0 += hk[i] != kNoKey;
+        const int in_heads = block_sum_int(c0, red_i);
+        uint64_t tau = kNoKey;
+        if (total > BW && in_heads >= BW) {
+            uint64_t tp, tm;
+            smem_radix_select(hk, nh, BW, hist, scan_w, red_k, sc, tp, tm);
+            uint64_t t = 0;
+            for (int i = tid; i < nh; i += kSpThreads)
+                if (hk[i] != kNoKey && (hk[i] & tm) <= tp) t = hk[i] > t ? hk[i] : t;
+            tau = block_max_u64(t, red_k);
         }
-    __syncthreads();
-    if (a.rewire) stage_children(a, n, f);
-    uint64_t prefix = ~0ull, mask = 0;
-    int want;
-    if (in_smem) {
-        int c = 0;
-#pragma unroll
-        for (int u = 0; u < kPickOneKpt; ++u) {
-            if (tid + u * kPickOneThreads >= E) kr[u] = kNoKey;
-            c += kr[u] != kNoKey;
+        // survivors: heads at or above tau, then the further keys of the slices
+        // whose whole head survived (recomputed from the staged row)
+        for (int i = tid; i < nh; i += kSpThreads) {
+            const uint64_t key = hk[i];
+            if (key == kNoKey || key > tau) continue;
+            const int pos = atomicAdd(&cnts[0], 1);
+            if (pos < scap) {
+                sk[pos] = key;
+                se[pos] = he[i];
+            }
         }
-        for (int i = tid; i < n_tail; i += kPickOneThreads) c += tail[i] != kNoKey;
-        const int T = block_sum_int(c, red_i);   // (its barriers also publish the staging)
-        want = min(BW, T);
-        if (want < T) radix_select_regs(kr, want, whist, sc, red_i, red_k, prefix, mask, tail, n_tail);
-        collect_regs(kr, prefix, mask, BW, [&](int u) { return tid + u * kPickOneThreads; }, f);
-        for (int i = tid; i < n_tail; i += kPickOneThreads) {
-            const uint64_t key = tail[i];
-            if (key != kNoKey && (key & mask) <= prefix) {
-                const int pos = atomicAdd(f.cnt, 1);
-                if (pos < BW) {
-                    f.win_k[pos] = key;
-                    f.win_e[pos] = kReg + i;
+        for (int sl = warp; sl < n_sl; sl += kSpWarps) {
+            const uint64_t last = hk[sl * m + m - 1];
+            if (last == kNoKey || last > tau) continue;   // (uniform across the warp)
+            for (int t = sl * Z + lane; t < min(V, sl * Z + Z); t += 32) {
+                uint64_t key;
+                if (!cand(t, key) || key > tau || key <= last) continue;
+                const int pos = atomicAdd(&cnts[0], 1);
+                if (pos < scap) {
+                    sk[pos] = key;
+                    se[pos] = t;
                 }
             }
         }
-    } else if (E <= a.key_cap) {
         __syncthreads();
-        const KeyCand cand{keys, kNoKey};
-        int c = 0;
-        for (int64_t e = tid; e < E; e += kPickOneThreads) c += __ldcg(keys + e) != kNoKey;
-        const int T = block_sum_int(c, red_i);
-        want = min(BW, T);
-        if (want < T) radix_select(cand, E, want, hist, sc, prefix, mask);
-        collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
-    } else {
-        __syncthreads();
-        ReqCand cand;
-        cand.x = a.scores + rb * dm.V;
-        cand.cols = a.cols + base;
-        cand.rp = f.rp;
-        cand.cum = cum_s;
-        cand.lse = lse_s;
-        cand.status = a.status;
-        cand.n = n;
-        cand.logits = a.logits;
-        cand.V = dm.V;
-        const int total = f.rp[n];
-        want = min(BW, total);
-        if (want < total) radix_select(cand, total, want, hist, sc, prefix, mask);
-        collect(cand, total, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+        const int ns = cnts[0];
+        if (ns <= scap) {
+            if (want < ns) smem_radix_select(sk, ns, want, hist, scan_w, red_k, sc, prefix, mask);
+            collect(ListCand<false>{sk}, ns, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
+        } else {   // more survivors than the buffer: exact selection over every token
+            radix_select(cand, V, want, hist, sc, prefix, mask);
+            collect(cand, V, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
+        }
     }
     __syncthreads();
     finish_request(a, r, min(*f.cnt, want), f);
@@ -1227,31 +1149,33 @@ cudaError_t ensure_smem(K kernel, size_t bytes) {
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t select_scratch_bytes(int B, int BW, int64_t key_cap, int64_t surv_cap) {
-    const size_t rows = (size_t)B * BW;
-    return al256(rows * 4) + al256(rows * 8) + al256((size_t)B * 4) + al256((size_t)B * 4) +
-           al256((size_t)B * key_cap * 8) + al256((size_t)B * surv_cap * 8) +
-           al256((size_t)B * surv_cap * 4);
+int select_head_m(int BW) { return BW >= 1024 ? 4 : 8; }
+
+size_t select_ticket_offset(int B, int BW) {
+    const size_t rows = (size_t)B * BW, m = (size_t)select_head_m(BW);
+    return al256(rows * 4) + al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4);
 }
 
-void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, int64_t surv_cap,
-                          SelectArgs &a) {
+size_t select_scratch_bytes(int B, int BW, int64_t key_cap) {
+    return select_ticket_offset(B, BW) + al256((size_t)B * 4) + al256((size_t)B * key_cap * 8);
+}
+
+void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectArgs &a) {
     const size_t rows = (size_t)B * BW;
+    const int m = select_head_m(BW);
     a.row_lse = reinterpret_cast<float *>(base);
     base += al256(rows * 4);
-    a.best = reinterpret_cast<uint64_t *>(base);
-    base += al256(rows * 8);
-    a.surv_cnt = reinterpret_cast<int32_t *>(base);
-    base += al256((size_t)B * 4);
+    a.row_cnt = reinterpret_cast<int32_t *>(base);
+    base += al256(rows * 4);
+    a.head_k = reinterpret_cast<uint64_t *>(base);
+    base += al256(rows * m * 8);
+    a.head_e = reinterpret_cast<int32_t *>(base);
+    base += al256(rows * m * 4);
     a.ticket = reinterpret_cast<uint32_t *>(base);
     base += al256((size_t)B * 4);
     a.keys = reinterpret_cast<uint64_t *>(base);
-    base += al256((size_t)B * key_cap * 8);
-    a.surv_key = reinterpret_cast<uint64_t *>(base);
-    base += al256((size_t)B * surv_cap * 8);
-    a.surv_e = reinterpret_cast<int32_t *>(base);
     a.key_cap = key_cap;
-    a.surv_cap = surv_cap;
+    a.head_m = m;
 }
 
 static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t s);
@@ -1269,40 +1193,25 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
     const Dims &dm = a.dims;
     if (dm.BW > 1024 || dm.V > kSelectMaxVocab || dm.V < 1) return cudaErrorInvalidValue;
     if (a.dense) {
-        const size_t smem = dense_smem(dm);
+        if (a.head_m < 1 || a.head_m > 32) return cudaErrorInvalidValue;
+        const size_t smem = dense_smem(dm, a.head_m);
         cudaError_t e = ensure_smem(select_dense_kernel, smem);
         if (e != cudaSuccess) return e;
-        select_dense_kernel<<<dm.B, kDenseThreads, smem, s>>>(a);
+        select_dense_kernel<<<dm.B, kSpThreads, smem, s>>>(a);
         return cudaGetLastError();
     }
-    {
-        // one persistent CTA per SM, as many row slots as shared memory holds
-        const size_t xb = a.logits ? dense_x_bytes(dm.V) : 0, fixed = rows_fixed_bytes(a.logits);
-        const int nbuf = a.logits ? (int)std::min<size_t>(kRowsMaxBuf, ((210u << 10) - fixed) / xb) : 1;
-        if (nbuf < 1) return cudaErrorInvalidValue;
-        const size_t smem = nbuf * xb + fixed;
-        cudaError_t e = ensure_smem(select_rows_kernel, smem);
-        if (e != cudaSuccess) return e;
-        const int64_t rows = (int64_t)dm.B * dm.BW;
-        const int grid = (int)std::min<int64_t>(rows, a.num_sms > 0 ? a.num_sms : 148);
-        select_rows_kernel<<<grid, kRowsThreads, smem, s>>>(a, nbuf);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    // the one-CTA pick when the pool fits its registers and its shared memory fits the SM
-    if (std::min<int64_t>(a.max_entries, a.key_cap) <= kPickOneMax && pick_one_smem(dm) <= (200u << 10)) {
-        const size_t smem = pick_one_smem(dm);
-        cudaError_t e = ensure_smem(select_pick_one_kernel, smem);
-        if (e != cudaSuccess) return e;
-        select_pick_one_kernel<<<dm.B, kPickOneThreads, smem, s>>>(a);
-        return cudaGetLastError();
-    }
-    int64_t parts = (std::min<int64_t>(a.max_entries, a.key_cap) + kPickKeys - 1) / kPickKeys;
-    a.pick_parts = (int)std::max<int64_t>(1, std::min<int64_t>(parts, kMaxPickParts));
-    const size_t smem = pick_smem(dm);
-    cudaError_t e = ensure_smem(select_pick_kernel, smem);
+    // sparse: one launch, sp_parts CTAs per request (a beam per warp at a time;
+    // fewer CTAs when only the masked entries' log-probs are read)
+    const int R = std::min(dm.BW, a.logits ? kSpWarps : 4 * kSpWarps);
+    a.sp_rows = R;
+    a.sp_parts = (dm.BW + R - 1) / R;
+    if (a.head_m < 1 || a.head_m > 32) return cudaErrorInvalidValue;
+    const size_t smem = sparse_smem(dm, a.head_m);
+    cudaError_t e = ensure_smem(select_sparse_kernel, smem);
     if (e != cudaSuccess) return e;
-    select_pick_kernel<<<dm.B * a.pick_parts, kPickThreads, smem, s>>>(a);
+    const int64_t grid = (int64_t)dm.B * a.sp_parts;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    select_sparse_kernel<<<(int)grid, kSpThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 

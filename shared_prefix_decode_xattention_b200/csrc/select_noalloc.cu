@@ -11,8 +11,9 @@
 // beam counts and the mask, and gets parent / token / cum / n_out back.
 //
 // It runs the very same selection kernels as xgr_beam_select (without the
-// rewiring).  Their scratch (each beam's row log-sum-exp and best key, and each
-// request's key and survivor buffers) lives in one file-scope device array of
+// rewiring).  Their scratch (each beam's row log-sum-exp, candidate count and
+// head of best keys, each request's ticket and key buffer) lives in one
+// file-scope device array of
 // kScratchBytes; every GPU that loads the library holds that array until the
 // process exits.  All
 // calls share it, so calls that overlap on the GPU (two streams, two threads)
@@ -83,14 +84,13 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
         return XGR_ERR_SHAPE;
     if (vocab > kSelectMaxVocab) return XGR_ERR_UNIMPLEMENTED;
     // what the fixed array leaves after the per-row scratch goes to the key
-    // buffer (8 bytes a CSR entry) and the survivors (12 bytes, half as many)
-    const size_t fixed = kStatusBytes + select_scratch_bytes(n_requests, beam_width, 0, 0) + 1024;
+    // buffer (8 bytes a CSR entry)
+    const size_t fixed = kStatusBytes + select_scratch_bytes(n_requests, beam_width, 0) + 1024;
     if (fixed >= kScratchBytes) return XGR_ERR_CAPACITY;
-    const int64_t key_cap = (int64_t)((kScratchBytes - fixed) / ((size_t)n_requests * 14)) & ~31ll;
-    const int64_t surv_cap = key_cap / 2;
+    const int64_t key_cap = (int64_t)((kScratchBytes - fixed) / ((size_t)n_requests * 8)) & ~31ll;
     const int64_t need = std::max<int64_t>({(int64_t)vocab, 8ll * beam_width, 4096});
     if (key_cap < need ||
-        kStatusBytes + select_scratch_bytes(n_requests, beam_width, key_cap, surv_cap) > kScratchBytes)
+        kStatusBytes + select_scratch_bytes(n_requests, beam_width, key_cap) > kScratchBytes)
         return XGR_ERR_CAPACITY;   // beyond the fixed 8 MiB scratch
     void *scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return XGR_ERR_CUDA;
@@ -108,12 +108,14 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     a.bits = d_bits;
     a.row_ptr = d_row_ptr;
     a.cols = d_cols;
-    a.max_entries = key_cap;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&a.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return XGR_ERR_CUDA;
-    select_scratch_carve(sc + kStatusBytes, n_requests, beam_width, key_cap, surv_cap, a);
+    select_scratch_carve(sc + kStatusBytes, n_requests, beam_width, key_cap, a);
+    // the tickets must start at zero (each call also leaves them at zero)
+    if (!dense && cudaMemsetAsync(a.ticket, 0, (size_t)n_requests * 4, (cudaStream_t)stream) != cudaSuccess)
+        return XGR_ERR_CUDA;
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum_out;

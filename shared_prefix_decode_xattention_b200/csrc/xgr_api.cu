@@ -19,7 +19,6 @@ constexpr int kMinChunk = 256;     // fewest keys per split-K work item
 // the separate merge kernel that split items need, in key units of the
 // tensor-core loop (one more dependent launch plus a few round trips)
 constexpr double kMergeKeys = 768.0;
-constexpr int64_t kSurvCap = 65536;   // selection survivors per request (more: exact path over the keys)
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -51,7 +50,7 @@ struct Layout {
     size_t mask_row_ptr, mask_cols, mask_sync;
     int64_t mask_cap;
     size_t select_scratch;
-    int64_t key_cap, surv_cap;   // selection keys / survivors per request
+    int64_t key_cap;             // selection keys per request
     size_t part_o, part_ml;
     int slots;
     size_t plan_items[2], plan_members[2], plan_nslots[2];
@@ -88,14 +87,13 @@ void make_layout(const xgr_config &c, Layout &L) {
         L.mask_sync = take(8 * (B + 1));   // look-back words, then the two ticket words
         L.mask_cols = take(4 * L.mask_cap);
         L.key_cap = BW * (int64_t)fanout_cap(c);
-        L.surv_cap = std::min<int64_t>(L.key_cap, kSurvCap);
-        L.select_scratch = take(select_scratch_bytes((int)B, (int)BW, L.key_cap, L.surv_cap));
+        L.select_scratch = take(select_scratch_bytes((int)B, (int)BW, L.key_cap));
     } else {
         L.trie_level_cap = 0;
         L.trie_ptr = L.trie_tok = L.root_bits = L.mask_row_ptr = L.mask_cols = L.mask_sync = 0;
         L.select_scratch = 0;
         L.mask_cap = 0;
-        L.key_cap = L.surv_cap = 0;
+        L.key_cap = 0;
     }
     L.slots = partial_slots(c);
     L.part_o = take(4 * (size_t)L.slots * partial_rows(c) * D);
@@ -201,11 +199,13 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     for (auto &sg : segs)
         for (int r : sg.members) nseg[r]++;
 
-    // kind of every segment: tensor-core tiles of 128 rows whenever D = 128
-    // (few rows waste tensor work but the stage then streams K/V at HBM speed),
-    // else the small-row kernel
+    // kind of every segment: tensor-core tiles of 128 rows when D = 128 and the
+    // segment has more rows than one small-row item holds; else the small-row
+    // kernel, split over the keys (a few query rows -- one beam at step 0, one
+    // request's suffix -- make the stage a K/V stream, which many short CTAs
+    // read faster than a few long tensor-core loops)
     auto rows_of = [&](const Seg &sg) { return (int64_t)sg.members.size() * nb * G; };
-    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > 0; };
+    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > kSmallRows; };
     // split factor per kind: the fewest waves x keys per item (+ a fixed
     // per-item overhead in key units), over the resident CTAs of the GPU
     // A tensor-core segment left whole finishes its requests itself; splitting
@@ -564,8 +564,13 @@ xgr_status xgr_begin(xgr_ctx *c, int32_t n_requests, xgr_stream_t stream) {
         c->planned_B = n_requests;
     }
     c->dims.B = n_requests;
+    uint32_t *sel_ticket =
+        c->cfg.vocab > 0 ? reinterpret_cast<uint32_t *>(
+                               c->at<uint8_t>(c->L.select_scratch) +
+                               select_ticket_offset(c->cfg.max_requests, c->cfg.beam_width))
+                         : nullptr;
     if (launch_begin(c->st, c->dims, c->cfg.max_requests, c->cfg.vocab == 0,
-                     c->cfg.vocab > 0 ? c->at<uint64_t>(c->L.mask_sync) : nullptr,
+                     c->cfg.vocab > 0 ? c->at<uint64_t>(c->L.mask_sync) : nullptr, sel_ticket,
                      (cudaStream_t)stream) != cudaSuccess)
         return XGR_ERR_CUDA;
     c->begun = true;
@@ -728,10 +733,9 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.bits = mask->bits;
     a.row_ptr = mask->row_ptr;
     a.cols = mask->cols;
-    a.max_entries = step == 0 ? c->cfg.vocab : (int64_t)c->cfg.beam_width * c->level_fanout[step];
     a.num_sms = c->num_sms;
     select_scratch_carve(c->at<uint8_t>(c->L.select_scratch), c->cfg.max_requests,
-                         c->cfg.beam_width, c->L.key_cap, c->L.surv_cap, a);
+                         c->cfg.beam_width, c->L.key_cap, a);
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum;

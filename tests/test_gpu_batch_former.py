@@ -1,0 +1,77 @@
+"""GPU: batches formed by the Chunked Hash Tree feed the staged attention.
+
+Feather page ("Requests of the same feather must flock together"),
+"Methodology", 1. Chunked Hash Tree, and "Results": prefix-homogeneous batches
+are the ones whose shared prefix is read once for all members.  Here the 64
+requests of the prefix-shared workload (4 prompt families of 16, 8192-token
+family prefixes, private suffixes of 256-2048 tokens) arrive in a shuffled
+order; the tree forms the batches; each batch becomes one shared KV segment
+(its first member's prefix, as deep as the batch shares it) that every member
+links to, with the rest of each prompt loaded as the member's private suffix;
+one decode step runs through the C ABI and every request's attention is
+compared with the oracle over that request's own full prompt.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from harness import compare_attention, u16
+from shared_prefix_decode_xattention_b200 import xgr
+from shared_prefix_decode_xattention_b200.sched import ChunkedHashTree
+from shared_prefix_decode_xattention_b200.session import Session, config_for
+
+pytestmark = pytest.mark.gpu
+
+CHUNK = 256
+
+
+def _prompt_tokens(w):
+    """Token ids of every request's prompt: its family's prefix, then its own suffix."""
+    rng = np.random.default_rng(4242)
+    lens = workloads.prompt_lengths(w)
+    fam = [rng.integers(0, 32000, size=int(lens[g])) for g in range(w.n_shared)]
+    suf = workloads.suffix_lengths(w)
+    return [np.concatenate([fam[w.shared_id(r)], rng.integers(0, 32000, size=int(suf[r]))])
+            for r in range(w.B)]
+
+
+def test_tree_batches_feed_the_attention():
+    w = workloads.WORKLOADS[4]
+    toks = _prompt_tokens(w)
+    tree = ChunkedHashTree(CHUNK)
+    for r in np.random.default_rng(7).permutation(w.B):   # interleaved arrivals
+        tree.insert(int(r), toks[r])
+    batches = tree.form_batches(w.B // w.groups, 1)
+    # the four families come back whole, each sharing its full prefix
+    assert sorted(sorted(m) for m, _ in batches) == [
+        list(range(g * 16, g * 16 + 16)) for g in range(w.groups)]
+    assert all(sh * CHUNK == int(workloads.prompt_lengths(w)[0]) for _, sh in batches)
+
+    sess = Session(config_for(w), "cuda")
+    for sid, (members, shared_chunks) in enumerate(batches):
+        depth = shared_chunks * CHUNK
+        k, v = workloads.shared_kv(w, w.shared_id(members[0]), "cuda")   # the first member's prefix
+        sess.prefill(members[0], sid, k[:, :depth].contiguous(), v[:, :depth].contiguous())
+        for r in members[1:]:
+            sess.link(r, sid)
+    for r in range(w.B):
+        k, v = workloads.suffix_kv(w, r, "cuda")
+        sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+    sess.begin(w.B)
+    q, kn, vn = workloads.step_qkv(w, 0, "cuda")
+    out = torch.full((w.B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((w.B, w.BW, w.Hq), float("nan"), dtype=torch.float32, device="cuda")
+    sess.decode_step(0, q, kn, vn, out, lse)
+    torch.cuda.synchronize()
+    qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
+    for r in range(w.B):
+        ks, vs = workloads.shared_kv(w, w.shared_id(r), "cpu")
+        kx, vx = workloads.suffix_kv(w, r, "cpu")
+        dec = oracle.BeamDecode(None, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V)
+        dec.begin(u16(ks), u16(vs), u16(kx), u16(vx))
+        o_ref, l_ref = dec.attention(0, qc[r], knc[r], vnc[r])
+        compare_attention(out[r], lse[r], o_ref, l_ref, np.ones(w.BW, bool), f"request {r}")
+    assert sess.device_status() == 0
+    sess.close()
