@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bw512", action="store_true",
                     help="skip the BW = 512 attention figure (second half of the metric)")
+    ap.add_argument("--groups", type=int, default=1,
+                    help="request groups decoded on their own streams inside the one graph")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the prefix-batch and long-history workload figures")
     return ap.parse_args()
@@ -619,11 +621,24 @@ def run_gpu(args, w):
     items = workloads.items(w)
     logits_mode = args.scores == "logits"
     flags = xgr.XGR_SCORES_LOGITS if logits_mode else xgr.XGR_SCORES_LOGPROB
-    sess = Session(config_for(w), dev)
-    sess.build_trie(items)
-    for r in range(w.B):
-        k, v = workloads.shared_kv(w, w.shared_id(r), dev)
-        sess.prefill(r, w.shared_id(r), k, v)
+    # Request groups: the batch split into G contexts whose decodes run on G
+    # streams of one graph (requests are independent; one group's selection
+    # overlaps another's attention -- the multi-stream batching of the xGR
+    # page's xSchedule, applied to the hot path).  G = 1: one context.
+    G = max(1, min(args.groups, w.B))
+    while w.B % G:
+        G -= 1
+    Bg = w.B // G
+    wg = workloads.small(w, B=Bg)   # the shape of one group's context
+    sessions = []
+    for g in range(G):
+        sg = Session(config_for(wg), dev)
+        sg.build_trie(items)
+        for i in range(Bg):
+            r = g * Bg + i
+            k, v = workloads.shared_kv(w, w.shared_id(r), dev)
+            sg.prefill(i, i, k, v)
+        sessions.append(sg)
     del k, v
     inputs = []
     for s in range(w.S):
@@ -637,48 +652,68 @@ def run_gpu(args, w):
     cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
     nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    sess.begin(w.B)   # plan once (setup)
+    for sg in sessions:
+        sg.begin(Bg)   # plan once (setup)
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
     cur = torch.cuda.current_stream
+    streams = [torch.cuda.Stream(device=dev) for _ in range(G)]
+    sl = lambda g: slice(g * Bg, (g + 1) * Bg)
 
     # One decode = phases: [begin + step 0] then, for s >= 1, [attention s] and
     # [mask + selection s].  Each phase is enqueued on the current stream (the
-    # capture stream while a CUDA graph is recorded); with `host`, the step's
-    # inputs come from pinned host memory and its outputs go back to it.
-    # The valid-path mask of step s depends only on the beam state the previous
-    # selection left, so it is built on a side stream while the attention runs.
-    side = torch.cuda.Stream(device=dev)
-    masks = [None] * w.S
+    # capture stream while a CUDA graph is recorded), forked into one stream
+    # per request group and joined again; with `host`, the step's inputs come
+    # from pinned host memory and its outputs go back to it.  The masks are
+    # views (xgr_build_mask enqueues nothing).
+    masks = [[None] * w.S for _ in range(G)]
 
-    def enqueue_att(s, inp, host):
+    def fork(body):
+        top = cur()
+        for g in range(G):
+            streams[g].wait_stream(top)
+            with torch.cuda.stream(streams[g]):
+                body(g, streams[g])
+        for g in range(G):
+            top.wait_stream(streams[g])
+
+    def att_g(g, st, s, inp, host):
         q, kn, vn, sc = inp[s]
-        side.wait_stream(cur())
-        with torch.cuda.stream(side):
-            masks[s] = sess.build_mask(s, side)
+        masks[g][s] = sessions[g].build_mask(s, st)
         if host is not None:
             for d, h in zip(inp[s], host[s]):
-                d.copy_(h, non_blocking=True)
-        sess.decode_step(s, q, kn, vn, out, lse, cur())
-        cur().wait_stream(side)
+                d[sl(g)].copy_(h[sl(g)], non_blocking=True)
+        sessions[g].decode_step(s, q[sl(g)], kn[sl(g)], vn[sl(g)], out[sl(g)], lse[sl(g)], st)
 
-    def enqueue_sel(s, inp, host):
-        sess.beam_select(s, inp[s][3], flags, masks[s], par, tok, cum, nout, cur())
+    def sel_g(g, st, s, inp, host):
+        sessions[g].beam_select(s, inp[s][3][sl(g)], flags, masks[g][s], par[sl(g)], tok[sl(g)],
+                                cum[sl(g)], nout[sl(g)], st)
         if host is not None:
             for h, d in zip(host[w.S + s], (par, tok, cum, nout)):
-                h.copy_(d, non_blocking=True)
+                h[sl(g)].copy_(d[sl(g)], non_blocking=True)
+
+    def enqueue_att(s, inp, host):
+        fork(lambda g, st: att_g(g, st, s, inp, host))
+
+    def enqueue_sel(s, inp, host):
+        fork(lambda g, st: sel_g(g, st, s, inp, host))
+
+    def head_g(g, st, inp, host):
+        sessions[g].begin(Bg, st)
+        att_g(g, st, 0, inp, host)
+        sel_g(g, st, 0, inp, host)
 
     def enqueue_head(inp, host):
-        sess.begin(w.B, cur())
-        enqueue_att(0, inp, host)
-        enqueue_sel(0, inp, host)
+        fork(lambda g, st: head_g(g, st, inp, host))
 
     def enqueue_decode(inp=inputs, host=None):
-        enqueue_head(inp, host)
-        for s in range(1, w.S):
-            enqueue_att(s, inp, host)
-            enqueue_sel(s, inp, host)
+        def chain(g, st):   # a group's whole decode on its own stream
+            head_g(g, st, inp, host)
+            for s in range(1, w.S):
+                att_g(g, st, s, inp, host)
+                sel_g(g, st, s, inp, host)
+        fork(chain)
 
     def capture(fn, keep=False):
         g = torch.cuda.CUDAGraph(keep_graph=keep)
@@ -691,17 +726,19 @@ def run_gpu(args, w):
     for _ in range(max(args.warmup, 3)):   # eager warm-up (plans, attributes)
         enqueue_decode()
     torch.cuda.synchronize()
-    # CSR entries of every step (one eager decode, read back after each mask)
-    nnz = []
-    sess.begin(w.B, cur())
+    # valid (row, token) entries of every step (one eager decode, summed over groups)
+    nnz = [0] * w.S
+    for g in range(G):
+        sessions[g].begin(Bg, cur())
     for s in range(w.S):
         enqueue_att(s, inputs, None)
-        m = masks[s]
         torch.cuda.synchronize()
-        nnz.append(sess.mask_entries(m) if m.kind == xgr.XGR_MASK_CSR else 0)
+        for g in range(G):
+            m = masks[g][s]
+            nnz[s] += sessions[g].mask_entries(m) if m.kind != xgr.XGR_MASK_DENSE else 0
         enqueue_sel(s, inputs, None)
     torch.cuda.synchronize()
-    if sess.device_status() != 0:
+    if any(sg.device_status() != 0 for sg in sessions):
         raise RuntimeError("device status set during warm-up")
     # the graph-based execution of the pages' system level: a whole decode is one graph
     g_decode = capture(lambda: enqueue_decode(), keep=True)
@@ -779,7 +816,9 @@ def run_gpu(args, w):
                "d2h_bytes_per_step": d2h}
         del g_e2e
 
-    status = sess.device_status()
+    status = 0
+    for sg in sessions:
+        status |= sg.device_status()
 
     # ---- roofline of the dominant call (attention vs selection at steps >= 1)
     peaks = {}
@@ -824,6 +863,7 @@ def run_gpu(args, w):
                            "peak_gbs": hbm, "frac": dec_gbs / hbm,
                            "note": "whole decode (all steps, every kernel) against the copy "
                                    f"bandwidth {src}"},
+            "request_groups": G,
             "gpu_launches": launches_per_decode * args.steps,
             "device_status": status, "n_live_last": int(n_live.min()) if n_live.size else 0}
     if e2e:
@@ -851,7 +891,8 @@ def run_gpu(args, w):
     line["shared_stage_tensor_frac"] = tfr
     if rank == 0:
         print(json.dumps(line), flush=True)
-    sess.close()
+    for sg in sessions:
+        sg.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -93,7 +93,14 @@ enum {
     XGR_KV_SUFFIX = 1           /* a request's private prefix continuation (beam width 1 use) */
 };
 
-enum { XGR_MASK_DENSE = 0, XGR_MASK_CSR = 1 };
+/* Mask kinds (xGR 2.2 "Hybrid dense/sparse storage": dense, pre-generated
+ * masks for the first steps, sparse masks updated in place afterwards). */
+enum {
+    XGR_MASK_DENSE = 0,         /* step 0: one bitset shared by every live beam */
+    XGR_MASK_CSR = 1,           /* explicit CSR rows (xgr_mask_to_csr, or a caller's) */
+    XGR_MASK_NODE_BITS = 2,     /* a pre-generated bitset per trie node, picked by each row's node */
+    XGR_MASK_TRIE_ROWS = 3      /* each row = the sorted children of its trie node (no copy) */
+};
 
 typedef struct {
     int32_t max_requests;   /* B: requests per batch */
@@ -112,10 +119,21 @@ typedef struct {
 } xgr_config;
 
 /* A mask as produced by xgr_build_mask: views into the workspace, valid until
- * the next xgr_build_mask.  Dense: bits[w] bit j set <=> token 32w+j valid
- * (shared by every live beam of step 0).  CSR: the valid next tokens of row
- * r*BW+b are cols[row_ptr[row] .. row_ptr[row+1]), ascending; row_ptr lives
- * on the device, so nnz = row_ptr[n_rows] is known to kernels only. */
+ * the next selection (which rewires the trie nodes the row views read).
+ *  DENSE:      bits[w] bit j set <=> token 32w+j valid (every live beam of
+ *              step 0); n_words = ceil(V/32).
+ *  CSR:        the valid next tokens of row r*BW+b are cols[row_ptr[row] ..
+ *              row_ptr[row+1]), ascending (device arrays; nnz = row_ptr[n_rows]).
+ *  NODE_BITS:  row `row` may take token t iff bit t of the bitset
+ *              bits + row_node[row] * n_words is set; the table holds one
+ *              bitset per node of trie level `step`, pre-generated by
+ *              xgr_build_trie.
+ *  TRIE_ROWS:  row `row`'s valid tokens are cols[node_ptr[nd] ..
+ *              node_ptr[nd+1]) with nd = row_node[row] (ascending): the trie
+ *              level's own child lists, nothing copied.
+ * row_node is the context's per-beam trie node, which the selection rewires in
+ * place; rows of dead beams hold -1 and are empty.  row_stride bounds the
+ * valid tokens of one row (the level's largest child count). */
 typedef struct {
     int32_t kind;
     int32_t step;
@@ -125,6 +143,10 @@ typedef struct {
     const int32_t *row_ptr;
     const int32_t *cols;
     int64_t cols_capacity;
+    const int32_t *row_node;
+    const int32_t *node_ptr;
+    int32_t n_nodes;
+    int32_t row_stride;
 } xgr_mask;
 
 /* Bytes of device workspace a context with this config needs (256-byte
@@ -179,18 +201,31 @@ xgr_status xgr_begin(xgr_ctx *ctx, int32_t n_requests, xgr_stream_t stream);
 xgr_status xgr_decode_step(xgr_ctx *ctx, int32_t step, const void *d_q, const void *d_k_new,
                            const void *d_v_new, void *d_out, float *d_lse, xgr_stream_t stream);
 
-/* Valid-path mask of step `step` (xGR 2.2 "Hybrid dense/sparse storage"):
- * step 0 returns the pre-generated dense bitset (no kernel); later steps
- * write one CSR row per beam (the sorted valid next tokens of its trie node).
- * Fills *out with views into the workspace. */
+/* Valid-path mask of step `step` (xGR 2.2 "Hybrid dense/sparse storage").
+ * Enqueues nothing: every kind is a view of pre-built tables and of the beam
+ * state.  Step 0: DENSE (the root's bitset).  Step 1: NODE_BITS when
+ * xgr_build_trie pre-generated that level's per-node bitsets (levels with many
+ * valid tokens per node, whose table fits the workspace), else TRIE_ROWS.
+ * Later steps: TRIE_ROWS -- each beam's row follows its trie node, which the
+ * selection updates in place.  Fills *out. */
 xgr_status xgr_build_mask(xgr_ctx *ctx, int32_t step, xgr_mask *out, xgr_stream_t stream);
+
+/* Writes the mask of a step >= 1 (any kind, as returned by xgr_build_mask for
+ * the current step) as explicit CSR rows: d_row_ptr int32 [n_rows+1],
+ * d_cols int32 [cols_capacity] (device, caller-owned).  One kernel on
+ * `stream`.  Rows past cols_capacity are cut and XGR_DEV_CAPACITY is set in
+ * the device status word.  For callers that want the rows themselves (a
+ * check, or the CSR input of xgr_beam_topk_noalloc). */
+xgr_status xgr_mask_to_csr(xgr_ctx *ctx, const xgr_mask *mask, int32_t *d_row_ptr, int32_t *d_cols,
+                           int64_t cols_capacity, xgr_stream_t stream);
 
 /* Masked top-K beam selection with in-place rewiring (xGR 2.2 "Early sort
  * termination", 2.1 "In-place updates").  Vocabularies up to 32768 tokens
  * (xgr_create returns XGR_ERR_UNIMPLEMENTED above):
  *   d_scores fp32 [B][BW][V]  log-probs or logits (flags); rows of dead beams
  *                             are not read
- *   mask                      as returned by xgr_build_mask for this step
+ *   mask                      as returned by xgr_build_mask for this step (or
+ *                             its rows written by xgr_mask_to_csr, kind CSR)
  *   d_parent, d_token int32 [B][BW], d_cum fp32 [B][BW], d_n_out int32 [B]:
  *     the new beams in rank order (slot = rank): higher score first, then
  *     lower parent, then lower token.  Score = fp32(cum[parent] + lp).

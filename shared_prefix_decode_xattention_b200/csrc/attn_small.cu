@@ -9,7 +9,8 @@
 // CTA handles one work item (a kv head, <= 16 rows, a key range) and writes
 // one partial (O unnormalised, m, l) per row.  The rows are few, so the kernel
 // is bound by streaming K/V from HBM; keys are staged through shared memory
-// with 16-byte loads, 128 keys per tile.
+// by 16-byte cp.async copies (a whole tile in flight), 128 keys per tile.
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,14 +94,14 @@ __global__ void __launch_bounds__(kThreads) attn_small_kernel(SmallArgs a) {
     for (int kb = it.key_begin; kb < it.key_end; kb += kTileKeys) {
         const int nk = min(kTileKeys, it.key_end - kb);
         __syncthreads();   // previous tile fully consumed
+        // the tile's K and V rows, every 16-byte piece in flight at once
         for (int idx = tid; idx < nk * (D / 8); idx += kThreads) {
             const int j = idx / (D / 8), c = idx % (D / 8);
             const int64_t src = (head_row0 + kb + j) * D + c * 8;
-            *reinterpret_cast<uint4 *>(&sm.k[j * kRow + c * 8]) =
-                *reinterpret_cast<const uint4 *>(a.kstore + src);
-            *reinterpret_cast<uint4 *>(&sm.v[j * kRow + c * 8]) =
-                *reinterpret_cast<const uint4 *>(a.vstore + src);
+            cp_async16(smem_u32(&sm.k[j * kRow + c * 8]), a.kstore + src);
+            cp_async16(smem_u32(&sm.v[j * kRow + c * 8]), a.vstore + src);
         }
+        cp_async_wait_all();
         __syncthreads();
 
         // scores: thread tid <-> key j of the tile, all rows

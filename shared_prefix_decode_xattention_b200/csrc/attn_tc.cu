@@ -16,6 +16,7 @@
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
 //               S_j = Q K_j^T into TMEM buffer j % 2, O_{j%2} += P_j V_j with
 //               P_j read from tensor memory;
+//   warp 10     gathers the Unshared chunks (see below);
 //   warps 2-9   two softmax warpgroups; warpgroup h owns the chunks j with
 //               j % 2 == h, one query row per thread: it reads S_j from TMEM,
 //               keeps the running max and sum of its own accumulator O_h (lazy
@@ -29,8 +30,8 @@
 //               segment, the output.
 // In a request's only KV segment ("final" items) the Unshared and Merging
 // stages run here too.  The Unshared stage is one more key chunk of the same
-// loop (or a few, when the tile's beams x tokens pass 128): lanes 2-31 of the
-// producer warp gather the tile's beams' own k / v rows of steps 0..s (direct
+// loop (or a few, when the tile's beams x tokens pass 128): a gather warp
+// collects the tile's beams' own k / v rows of steps 0..s (direct
 // indices into the token-granular pool; this step's from k_new / v_new) into
 // the U area at kernel start, so the gather overlaps the Shared loop, and
 // append this step's k / v to the pool.  Row u of that chunk is token u % T of
@@ -53,7 +54,8 @@ namespace xgr {
 
 namespace {
 
-constexpr int kTcThreads = 320;              // producer warp, MMA warp, 2 softmax warpgroups
+constexpr int kTcThreads = 352;              // producer warp, MMA warp, 2 softmax warpgroups, gather warp
+constexpr int kGatherWarp = 10;              // gathers the Unshared chunks (and appends this step's k / v)
 constexpr int kSoftmaxThreads = 256;
 constexpr int kGroupThreads = 128;           // one softmax warpgroup: one query row per thread
 constexpr int kBlockN = 128;                 // keys per chunk
@@ -62,7 +64,7 @@ constexpr int kVStages = 2;                  // V chunks in flight
 constexpr uint32_t kHalf = 16384;            // one 128-row x 64-column bf16 sub-tile
 constexpr uint32_t kTile = 2 * kHalf;        // 128 x 128 bf16
 constexpr uint32_t kUBytes = 65536;          // U area: the Unshared chunk's K and V tiles
-constexpr int kGatherLanes = 30;             // producer-warp lanes 2..31 gather the Unshared rows
+constexpr int kGatherLanes = 32;             // the gather warp's lanes
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
@@ -156,9 +158,6 @@ __device__ __forceinline__ void fence_after_sync() {
 __device__ __forceinline__ void fence_before_sync() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     uint32_t r[32];
@@ -241,11 +240,6 @@ __device__ __forceinline__ float ex2(float x) {   // 2^x, one MUFU op; tiny resu
     return y;
 }
 
-// 16-byte global -> shared copy that bypasses the registers (and L1)
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 
 // query row `row` of a work item -> (request, beam, query head, global row, live)
@@ -269,8 +263,8 @@ __device__ __forceinline__ RowInfo row_info(const TcArgs &a, const WorkItem &it,
     return ri;
 }
 
-// 10 warps: the register file is split over the 4 schedulers (16K registers each) and 3 of
-// the 10 warps share one, so a thread may use at most 168 registers.  One instance
+// 11 warps: the register file is split over the 4 schedulers (16K registers each) and 3
+// warps share each of three of them, so a thread may use at most 168 registers.  One instance
 // serves every step (the code is warm in the caches after the first launch).
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -370,7 +364,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // softmax threads stage the Q tile meanwhile: 16 consecutive threads read one
     // 256-byte row (coalesced) and write it in the swizzled K-major layout
-    if (warp >= 2 && !q_tma) {
+    if (warp >= 2 && warp < kGatherWarp && !q_tma) {
         const int ts = tid - 64;
         uint4 qv[8];
 #pragma unroll
@@ -413,73 +407,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (*abort)
                 for (int j = max(0, n_issued - kVStages); j < n_issued; ++j)
                     mbar_wait(bar(B_VFULL + j % kVStages), (j / kVStages) & 1, nullptr);
-        } else if (n_u > 0) {
-            // ---- Unshared stage: gather the tile's beams' own k / v rows of steps
-            // 0..s into the U area, one 128-row chunk at a time (row u: token u % T
-            // of tile beam u / T), in the canonical swizzled layout; rows of dead
-            // beams, bad slots and the tail are zero.  This step's rows are also
-            // appended to the pool at slot (s, b).
-            const int gl = lane - 2;
-            const Dims dm = a.dims;
-            const int s_now = a.step;
-            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
-            for (int q = 0; q < n_u; ++q) {
-                if (q > 0 && !mbar_wait(bar(B_UEMPTY), (q - 1) & 1, abort)) break;
-                for (int u = gl; u < kBlockN; u += kGatherLanes) {
-                    const int ug = kBlockN * q + u, lb = ug / T, i = ug % T;
-                    const __nv_bfloat16 *sk = nullptr, *sv = nullptr;
-                    if (lb < nbeam) {
-                        const int lbs = lb0 + lb;   // beam index within the segment's rows / G
-                        const int member = lbs / a.nb, b = lbs % a.nb;
-                        const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + member];
-                        const int64_t brow = (int64_t)r * dm.BW + b;
-                        if (b < a.n_live[r]) {
-                            if (i == s_now) {
-                                sk = a.k_new + (brow * dm.Hkv + it.g) * 128;
-                                sv = a.v_new + (brow * dm.Hkv + it.g) * 128;
-                            } else {
-                                const int sl = a.st.anc[brow * dm.S + i];
-                                if (sl >= 0 && sl < dm.BW) {
-                                    const int64_t prow = (brow - b + sl) * dm.Hkv + it.g;
-                                    sk = a.pool_k + i * pool_step + prow * 128;
-                                    sv = a.pool_v + i * pool_step + prow * 128;
-                                }
-                            }
-                        }
-                    }
-                    const uint32_t dk = sb + kOffU, dv = sb + kOffU + kTile;
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        if (sk) {
-                            cp_async16(dk + sw128_off(u, c), sk + 8 * c);
-                            cp_async16(dv + sw128_off(u, c), sv + 8 * c);
-                        } else {
-                            *reinterpret_cast<uint4 *>(base + kOffU + sw128_off(u, c)) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4 *>(base + kOffU + kTile + sw128_off(u, c)) =
-                                make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                }
-                cp_async_wait_all();
-                // this step's k / v of the gathered live beams -> pool slot (s, b)
-                for (int u = gl; u < kBlockN; u += kGatherLanes) {
-                    const int ug = kBlockN * q + u, lb = ug / T, i = ug % T;
-                    if (lb >= nbeam || i != s_now) continue;
-                    const int lbs = lb0 + lb, member = lbs / a.nb, b = lbs % a.nb;
-                    const int r = it.n_members == 1 ? it.r0 : a.members[it.member_off + member];
-                    if (b >= a.n_live[r]) continue;
-                    const int64_t orow = ((int64_t)r * dm.BW + b) * dm.Hkv + it.g;
-                    uint4 *pk = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + orow * 128);
-                    uint4 *pv = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + orow * 128);
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        pk[c] = *reinterpret_cast<const uint4 *>(base + kOffU + sw128_off(u, c));
-                        pv[c] = *reinterpret_cast<const uint4 *>(base + kOffU + kTile + sw128_off(u, c));
-                    }
-                }
-                fence_async_smem();   // the gathered rows are visible to the tensor cores
-                mbar_arrive(bar(B_UFULL));
-            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -558,7 +485,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             umma_commit(bar(B_DONE));
             if (*abort) mbar_wait(bar(B_DONE), 0, nullptr);
         }
-    } else {
+    } else if (warp < kGatherWarp) {
         // ------------------------------------------------------------ softmax
         // Warpgroup `half` owns the chunks j with j % 2 == half, whole rows: thread
         // `row` reads TMEM lane `row` of S buffer `half`, keeps the running max and
@@ -752,6 +679,92 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         a.lse[ri.gid] = live ? (M + __log2f(l_row)) * kLn2 : -INFINITY;
                     }
                 }
+            }
+        }
+    } else if (n_u > 0) {
+        // ------------------------------------------------------------ gather
+        {
+            // ---- Unshared stage: gather the tile's beams' own k / v rows of steps
+            // 0..s into the U area, one 128-row chunk at a time (row u: token u % T
+            // of tile beam u / T), in the canonical swizzled layout; rows of dead
+            // beams, bad slots and the tail are zero.  This step's rows are also
+            // appended to the pool at slot (s, b).
+            const int gl = lane;
+            const Dims dm = a.dims;
+            const int s_now = a.step;
+            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+            for (int q = 0; q < n_u; ++q) {
+                if (q > 0 && !mbar_wait(bar(B_UEMPTY), (q - 1) & 1, abort)) break;
+                // this lane's rows u = gl + k * kGatherLanes: their request and beam,
+                // then every index they need, then the copies -- each stage's loads
+                // all in flight together
+                constexpr int kRowsPerLane = (kBlockN + kGatherLanes - 1) / kGatherLanes;
+                int rr[kRowsPerLane], bb[kRowsPerLane], ii[kRowsPerLane];
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes, ug = kBlockN * q + u, lb = ug / T;
+                    ii[k] = ug % T;
+                    rr[k] = -1;
+                    bb[k] = -1;
+                    if (u < kBlockN && lb < nbeam) {
+                        const int lbs = lb0 + lb;   // beam index within the segment's rows / G
+                        bb[k] = lbs % a.nb;
+                        rr[k] = it.n_members == 1 ? it.r0 : a.members[it.member_off + lbs / a.nb];
+                    }
+                }
+                int nl[kRowsPerLane], sl[kRowsPerLane];
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    nl[k] = rr[k] >= 0 ? a.n_live[rr[k]] : 0;
+                    sl[k] = (rr[k] >= 0 && ii[k] < s_now)
+                                ? a.st.anc[((int64_t)rr[k] * dm.BW + bb[k]) * dm.S + ii[k]] : -1;
+                }
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes;
+                    if (u >= kBlockN) continue;
+                    const __nv_bfloat16 *sk = nullptr, *sv = nullptr;
+                    if (rr[k] >= 0 && bb[k] < nl[k]) {
+                        const int64_t brow = (int64_t)rr[k] * dm.BW + bb[k];
+                        if (ii[k] == s_now) {
+                            sk = a.k_new + (brow * dm.Hkv + it.g) * 128;
+                            sv = a.v_new + (brow * dm.Hkv + it.g) * 128;
+                        } else if (sl[k] >= 0 && sl[k] < dm.BW) {
+                            const int64_t prow = (brow - bb[k] + sl[k]) * dm.Hkv + it.g;
+                            sk = a.pool_k + ii[k] * pool_step + prow * 128;
+                            sv = a.pool_v + ii[k] * pool_step + prow * 128;
+                        }
+                    }
+                    const uint32_t dk = sb + kOffU, dv = sb + kOffU + kTile;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (sk) {
+                            cp_async16(dk + sw128_off(u, c), sk + 8 * c);
+                            cp_async16(dv + sw128_off(u, c), sv + 8 * c);
+                        } else {
+                            *reinterpret_cast<uint4 *>(base + kOffU + sw128_off(u, c)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(base + kOffU + kTile + sw128_off(u, c)) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                cp_async_wait_all();
+                // this step's k / v of the gathered live beams -> pool slot (s, b)
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes;
+                    if (u >= kBlockN || rr[k] < 0 || ii[k] != s_now || bb[k] >= nl[k]) continue;
+                    const int64_t orow = ((int64_t)rr[k] * dm.BW + bb[k]) * dm.Hkv + it.g;
+                    uint4 *pk = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + orow * 128);
+                    uint4 *pv = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + orow * 128);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        pk[c] = *reinterpret_cast<const uint4 *>(base + kOffU + sw128_off(u, c));
+                        pv[c] = *reinterpret_cast<const uint4 *>(base + kOffU + kTile + sw128_off(u, c));
+                    }
+                }
+                fence_async_smem();   // the gathered rows are visible to the tensor cores
+                mbar_arrive(bar(B_UFULL));
             }
         }
     }

@@ -104,11 +104,24 @@ struct SelectArgs {
     const float *scores;        // [B][BW][V]
     int dense;                  // mask kind (dense: only beam 0 of each request is read)
     const uint32_t *bits;
+    // sparse steps: mask_kind XGR_MASK_CSR (row_ptr, cols), XGR_MASK_TRIE_ROWS
+    // (row_node, node_ptr, node_tok) or XGR_MASK_NODE_BITS (row_node, node_ptr,
+    // node_bits with n_words words per node)
+    int mask_kind;
     const int32_t *row_ptr;
     const int32_t *cols;
+    const int32_t *row_node;    // [B*BW] trie node of each row
+    const int32_t *node_ptr;    // [n_nodes+1] child range of each node of the level
+    const int32_t *node_tok;    // the level's child tokens
+    const uint32_t *node_bits;  // [n_nodes][n_words]
+    int32_t n_nodes;
+    int32_t n_words;
+    int32_t row_stride;         // most valid tokens of one row (TRIE_ROWS / NODE_BITS entry stride)
     // scratch (select_scratch_carve)
     float *row_lse;             // [B][BW] each live row's log-sum-exp (logits mode)
     int32_t *row_cnt;           // [B][BW] valid candidates of each row
+    int32_t *row_len;           // [B][BW] mask entries of each row
+    int32_t *row_cb;            // [B][BW] first trie child of each row's node (-1: none)
     uint64_t *head_k;           // [B][BW][m] each beam's m best keys, ascending (kNoKey pads)
     int32_t *head_e;            // [B][BW][m] their CSR entries (relative to the request)
     int head_m;                 // m
@@ -116,7 +129,8 @@ struct SelectArgs {
     uint64_t *keys;             // [B][key_cap] key of each CSR entry (relative to the request)
     int64_t key_cap;
     int sp_parts;               // set by the launcher: CTAs per request of the sparse kernel
-    int sp_rows;                //   and the beams each of them takes
+    int sp_rows;                //   and the beams each of them takes (<= 8: one per warp)
+    int sp_slots;               //   and its shared-memory slots for logits rows (0: none)
     int num_sms;                // SMs of the device
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
@@ -126,9 +140,11 @@ struct SelectArgs {
 // Largest vocabulary of the selection: a score row is staged whole in shared memory.
 constexpr int kSelectMaxVocab = 32768;
 // Scratch of the selection for B requests of BW beams: per beam row its
-// log-sum-exp, valid-candidate count and head (its m best keys and their
-// entries), a ticket per request, and the key buffer [B][key_cap] (a request
-// whose CSR entries exceed key_cap takes the exact fallback over the scores).
+// log-sum-exp, valid-candidate count, entry count, first trie child and head
+// (its m best keys and their entries), a ticket per request, and the key
+// buffer [B][key_cap] (CSR masks: entry e of the request at e - row_ptr[r*BW];
+// node masks: entry j of beam b at b * row_stride + j; a request whose CSR
+// entries exceed key_cap takes the exact fallback over the scores).
 // Everything read is written by the same call first, except the tickets,
 // which must be zero before a call (xgr_begin zeroes them, each call leaves
 // them zero).

@@ -22,9 +22,8 @@
 // Kernels:
 //  * dense mask (one live beam per request, step 0): select_dense_kernel, one
 //    CTA per request, stages the beam's score row with one bulk copy, takes its
-//    log-sum-exp (logits), cuts the row into slices with a head each (their m
-//    best keys, in order), and selects the best BW among the survivors of the
-//    heads' threshold, as the sparse kernel does.
+//    log-sum-exp (logits); tau = the BW-th best of the threads' best keys, and
+//    the survivors at or above it are ranked by counting.
 //  * sparse (CSR) masks: select_sparse_kernel, one launch per step.  Each
 //    request gets several CTAs; a warp takes one beam row at a time: its
 //    log-sum-exp (logits), the key of each of its CSR entries, and its head --
@@ -253,11 +252,18 @@ struct ListCand {
     }
 };
 
-// the request's key buffer, restricted to the survivors of tau
+// the request's key buffer, restricted to the survivors of tau; with a row
+// stride (node masks) only the first rl[b] slots of row b hold keys
 struct KeyCand {
     const uint64_t *k;
     uint64_t tau;
+    const int *rp, *rl;   // shared memory
+    int stride, n;        // stride 0: CSR numbering (every entry written)
     __device__ bool operator()(int64_t e, uint64_t &key) const {
+        if (stride) {
+            const int b = (int)(e / stride), j = (int)(e % stride);
+            if (b >= n || j >= rl[b]) return false;
+        }
         key = __ldcg(k + e);
         return key != kNoKey && key <= tau;
     }
@@ -304,11 +310,12 @@ struct FinishSmem {
     uint64_t *win_k;   // [BW] winners (unordered)
     int *win_e;        // [BW] their entry: CSR entry relative to the request (sparse) or token
     int *rank;         // [BW]
-    int *rp;           // [BW+1] sparse: entry offset of each live beam
+    int *rp;           // [BW+1] sparse: first entry of each beam's row (relative to the request)
     int *st_node;      // [n_stage] staged old rows (rewiring)
     int *st_anc;       // [n_stage*S]
     int *st_seq;       // [n_stage*S]
     int *cb, *ce;      // [n_stage] sparse: child range of each staged row's trie node
+    int *rl;           // [n_stage] sparse: mask entries of each row
     uint32_t *root;    // dense: [nw] root-children bitset, [nw] prefix popcounts
     int *cnt;          // winners appended
 };
@@ -318,7 +325,7 @@ __host__ __device__ inline size_t al16(size_t x) { return (x + 15) & ~(size_t)15
 // n_stage: old rows staged for the rewiring (the live beams: BW, or 1 for a dense step)
 __host__ __device__ inline size_t finish_bytes(int BW, int n_stage, int S, int nw_root) {
     return al16((size_t)BW * 8) + 2 * al16((size_t)BW * 4) + al16((size_t)(BW + 1) * 4) +
-           3 * al16((size_t)n_stage * 4) + 2 * al16((size_t)n_stage * S * 4) + al16((size_t)nw_root * 8) +
+           4 * al16((size_t)n_stage * 4) + 2 * al16((size_t)n_stage * S * 4) + al16((size_t)nw_root * 8) +
            16;
 }
 
@@ -342,6 +349,8 @@ __device__ FinishSmem carve_finish(uint8_t *p, int BW, int n_stage, int S, int n
     p += al16((size_t)n_stage * 4);
     f.ce = reinterpret_cast<int *>(p);
     p += al16((size_t)n_stage * 4);
+    f.rl = reinterpret_cast<int *>(p);
+    p += al16((size_t)n_stage * 4);
     f.root = reinterpret_cast<uint32_t *>(p);
     p += al16((size_t)nw_root * 8);
     f.cnt = reinterpret_cast<int *>(p);
@@ -356,17 +365,6 @@ __device__ void stage_rows(const SelectArgs &a, int64_t rb, int n, const FinishS
         f.st_seq[i] = a.st.seq[rb * S + i];
     }
     for (int b = threadIdx.x; b < n; b += blockDim.x) f.st_node[b] = a.st.node[rb + b];
-}
-
-// child range of every staged row's trie node (sparse steps; after stage_rows)
-__device__ void stage_children(const SelectArgs &a, int n, const FinishSmem &f) {
-    const int s = a.step;
-    for (int b = threadIdx.x; b < n; b += blockDim.x) {
-        const int node = f.st_node[b];
-        const bool ok = s < a.trie.levels && node >= 0 && node < a.trie.n_nodes[s];
-        f.cb[b] = ok ? a.trie.ptr[s][node] : -1;
-        f.ce[b] = ok ? a.trie.ptr[s][node + 1] : -1;
-    }
 }
 
 // append the winners among the candidates [0, E) of `cand` ((key & mask) <= prefix)
@@ -389,7 +387,8 @@ __device__ void collect(const Cand &cand, int64_t E, uint64_t prefix, uint64_t m
 // winners, counted by one warp per winner), write the outputs in rank order
 // and, when a.rewire, rewrite the request's beam state in place.  The caller
 // has staged the old rows (stage_rows) and rp / root.
-__device__ void finish_request(const SelectArgs &a, int r, int n_win, const FinishSmem &f) {
+__device__ void finish_request(const SelectArgs &a, int r, int n_win, const FinishSmem &f,
+                               bool in_rank_order = false) {
     const Dims dm = a.dims;
     const int BW = dm.BW, S = dm.S, V = dm.V;
     const int64_t rb = (int64_t)r * BW;
@@ -414,12 +413,16 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
             child_t[u] = a.trie.tok[s][c];
         }
     }
-    for (int i = warp; i < n_win; i += nwarps) {
-        const uint64_t k = f.win_k[i];
-        int c = 0;
-        for (int j = lane; j < n_win; j += 32) c += f.win_k[j] < k;
-        c = warp_sum_int(c);
-        if (lane == 0) f.rank[i] = c;
+    if (in_rank_order) {   // the winners already sit at their ranks
+        for (int i = threadIdx.x; i < n_win; i += blockDim.x) f.rank[i] = i;
+    } else {
+        for (int i = warp; i < n_win; i += nwarps) {
+            const uint64_t k = f.win_k[i];
+            int c = 0;
+            for (int j = lane; j < n_win; j += 32) c += f.win_k[j] < k;
+            c = warp_sum_int(c);
+            if (lane == 0) f.rank[i] = c;
+        }
     }
 #pragma unroll
     for (int u = 0; u < kWinPerThread; ++u) {   // the checked child of winner i, in rank
@@ -513,7 +516,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
 constexpr int kSpThreads = 256;
 constexpr int kSpWarps = kSpThreads / 32;
 constexpr int kSpKpc = 8;   // CSR entries per lane in one pass of the key loop
-constexpr int kLseU = 8;    // float4 per lane in one batch of the row stream
+constexpr int kLseU = 16;   // float4 per lane in one batch of the row stream (8 KB per warp)
 
 __device__ __forceinline__ float4 ld_stream4(const float4 *p) {
     float4 v;
@@ -627,21 +630,138 @@ __device__ __forceinline__ void warp_head_merge(uint64_t (&c)[KPC], const int (&
     run_e = nrun_e;
 }
 
-// Phase 1 of one beam row, by one warp: keys of its CSR entries into the key
-// buffer, its head (m best keys and entries, lanes 0..m-1) and its count of
-// valid candidates.
-__device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int base, uint64_t *keys) {
+// the same over a row staged in shared memory (16-byte aligned, V % 4 == 0)
+__device__ float warp_row_lse_smem(const float *x, int V, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x);
+    const int n4 = V >> 2;
+    float m = -INFINITY, s = 0.f;
+    bool nan = false;
+    for (int b0 = 0; b0 < n4; b0 += 32 * 4) {   // 16 values per lane per pass
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = b0 + u * 32 + lane;
+            const float4 q = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            v[4 * u] = q.x;
+            v[4 * u + 1] = q.y;
+            v[4 * u + 2] = q.z;
+            v[4 * u + 3] = q.w;
+        }
+        float mv = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            nan |= v[e] != v[e];
+            mv = fmaxf(mv, v[e]);
+        }
+        if (mv > m) {
+            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
+            m = mv;
+        }
+        if (m != -INFINITY) {
+            const float mk = m * kLog2e;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
+        }
+    }
+    if (__any_sync(0xffffffffu, nan)) {
+        if (lane == 0) set_status(status, XGR_DEV_NAN);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_pair_merge(m, s, m2, s2);
+    }
+    return m + logf(s);
+}
+
+// The valid tokens of a NODE_BITS row, compacted into wtok[0..) in token
+// order (the node's children in trie order) by one warp; returns their count.
+__device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int cap) {
+    const int lane = threadIdx.x & 31;
+    int cnt = 0;
+    for (int w0 = 0; w0 < nw; w0 += 32 * 8) {
+        uint32_t wv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {   // up to 256 words in flight per pass
+            const int w = w0 + u * 32 + lane;
+            wv[u] = w < nw ? __ldg(wb + w) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c = __popc(wv[u]);
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            int pos = cnt + incl - c;
+            uint32_t v = wv[u];
+            const int tbase = 32 * (w0 + u * 32 + lane);
+            while (v) {
+                const int bit = __ffs(v) - 1;
+                v &= v - 1;
+                if (pos < cap) wtok[pos] = tbase + bit;
+                ++pos;
+            }
+            cnt += __shfl_sync(0xffffffffu, incl, 31);
+        }
+    }
+    __syncwarp();
+    return cnt;
+}
+
+// Phase 1 of one beam row, by one warp: keys of its mask entries into the key
+// buffer, its head (m best keys and entries, lanes 0..m-1), its count of valid
+// candidates, its entry count and the first trie child of its node.  The
+// row's tokens come from the CSR rows, from its node's children in the trie
+// level (TRIE_ROWS), or from its node's pre-generated bitset (NODE_BITS,
+// compacted into wtok).
+__device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int base, uint64_t *keys,
+                           int *wtok, const float *xs) {
     const int lane = threadIdx.x & 31;
     const Dims dm = a.dims;
-    const int V = dm.V, m = a.head_m;
+    const int V = dm.V, m = a.head_m, s = a.step;
     const int64_t row = (int64_t)r * dm.BW + b;
     const bool live = b < n_live;
-    const int beg = a.row_ptr[row], end = a.row_ptr[row + 1];
     const float cum = a.cum[row];
     const float *x = a.scores + row * V;
+    // the first loads of the row's tokens go out before the row stream; the
+    // rest (its tokens, the node's first child) follow its log-sum-exp
+    const bool csr = a.mask_kind == XGR_MASK_CSR;
+    const int beg = csr ? a.row_ptr[row] : 0, end = csr ? a.row_ptr[row + 1] : 0;
+    const int node = (csr ? (a.rewire && live) : live) ? (csr ? a.st.node[row] : a.row_node[row]) : -1;
     float lse = 0.f;
-    if (a.logits && live) lse = warp_row_lse(x, V, a.status);
-    const int n_e = max(0, end - beg);
+    if (a.logits && live) lse = xs ? warp_row_lse_smem(xs, V, a.status) : warp_row_lse(x, V, a.status);
+    // the row's tokens (tokp[0..n_e)), their entry base and the node's first child
+    const int32_t *tokp = nullptr;
+    int n_e = 0, cb = -1;
+    int64_t ebase;
+    if (csr) {
+        tokp = a.cols + beg;
+        n_e = max(0, end - beg);
+        ebase = beg - base;
+        if (s < a.trie.levels && node >= 0 && node < a.trie.n_nodes[s]) cb = a.trie.ptr[s][node];
+    } else {
+        ebase = (int64_t)b * a.row_stride;
+        if (node >= 0 && node < a.n_nodes) {
+            const int lo = a.node_ptr[node], hi = a.node_ptr[node + 1];
+            cb = lo;
+            n_e = min(max(0, hi - lo), a.row_stride);
+            if (a.mask_kind == XGR_MASK_TRIE_ROWS) {
+                tokp = a.node_tok + lo;
+            } else {
+                const int nb = warp_bits_to_tokens(a.node_bits + (int64_t)node * a.n_words, a.n_words, wtok,
+                                                   a.row_stride);
+                if (nb != hi - lo && lane == 0) set_status(a.status, XGR_DEV_MASK);   // table and trie disagree
+                n_e = min(nb, a.row_stride);
+                tokp = wtok;
+            }
+        } else if (live && lane == 0) {
+            set_status(a.status, XGR_DEV_INDEX);
+        }
+    }
     uint64_t run = kNoKey;   // lane i < m: the i-th best key of the row so far
     int run_e = -1;
     int n_valid = 0;
@@ -652,19 +772,19 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
 #pragma unroll
         for (int u = 0; u < kSpKpc; ++u) {   // the entries' tokens (one round trip) ...
             const int j = j0 + u * 32 + lane;
-            tk[u] = (j < n_e && live) ? a.cols[beg + j] : -1;
+            tk[u] = (j < n_e && live) ? tokp[j] : -1;
         }
         float sv[kSpKpc];
 #pragma unroll
-        for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (another)
-            sv[u] = (tk[u] >= 0 && tk[u] < V) ? __ldg(x + tk[u]) : 0.f;
+        for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (staged, or another)
+            sv[u] = (tk[u] >= 0 && tk[u] < V) ? (xs ? xs[tk[u]] : __ldg(x + tk[u])) : 0.f;
 #pragma unroll
         for (int u = 0; u < kSpKpc; ++u) {
             const int j = j0 + u * 32 + lane;
             c[u] = kNoKey;
             ce[u] = -1;
             if (j >= n_e) continue;
-            const int e = beg + j;
+            const int64_t e = ebase + j;   // the entry, relative to the request
             uint64_t key = kNoKey;
             if (live) {
                 if (tk[u] < 0 || tk[u] >= V) {
@@ -675,9 +795,9 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
                     if (make_key(cum, lp, b, tk[u], V, a.status, k2)) key = k2;
                 }
             }
-            if (e >= base && (int64_t)(e - base) < a.key_cap) keys[e - base] = key;
+            if (e >= 0 && e < a.key_cap) keys[e] = key;
             c[u] = key;
-            ce[u] = e - base;
+            ce[u] = (int)e;
             n_valid += key != kNoKey;
         }
         warp_head_merge(c, ce, run, run_e, m);
@@ -690,20 +810,24 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
     if (lane == 0) {
         a.row_cnt[row] = n_valid;
         a.row_lse[row] = lse;
+        a.row_len[row] = n_e;
+        a.row_cb[row] = cb;
     }
 }
 
 // exact radix select over the keys k[0..n) in shared memory (unique keys;
-// kNoKey entries are not candidates), by a block of kSpThreads threads, with
-// 8-bit digits starting at the highest bit where the smallest and largest key
-// differ.  On return exactly `want` keys satisfy (key & mask) <= prefix
-// (0 < want <= number of candidates).  hist: 256 ints; scan_w: 32 ints; red:
-// 32 u64; sc: 3 ints of shared memory.
+// kNoKey entries are not candidates), by the whole block (blockDim a multiple
+// of 256, at most 2048), with 11-bit digits starting at the highest bit where
+// the smallest and largest key differ (so the first digit already spreads the
+// keys).  On return exactly `want` keys satisfy (key & mask) <= prefix
+// (0 < want <= number of candidates).  hist: kRadixBins ints; scan_w: 32 ints;
+// red: 32 u64; sc: 3 ints of shared memory.
+constexpr int kRadixBits = 11, kRadixBins = 1 << kRadixBits;
 __device__ void smem_radix_select(const uint64_t *k, int n, int want, int *hist, int *scan_w,
                                   uint64_t *red, int *sc, uint64_t &prefix, uint64_t &mask) {
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, nt = blockDim.x;
     uint64_t lo = kNoKey, hi = 0;
-    for (int i = tid; i < n; i += kSpThreads) {
+    for (int i = tid; i < n; i += nt) {
         const uint64_t key = k[i];
         if (key == kNoKey) continue;
         lo = key < lo ? key : lo;
@@ -721,23 +845,39 @@ __device__ void smem_radix_select(const uint64_t *k, int n, int want, int *hist,
     mask = pos == 64 ? 0ull : ~((1ull << pos) - 1ull);
     prefix = lo & mask;
     int k_rem = want;
+    const int bpt = kRadixBins / nt;   // bins per thread in the bucket search (8, 4 or 2)
     while (pos > 0) {
-        const int shift = pos > 8 ? pos - 8 : 0, width = pos - shift;
+        const int shift = pos > kRadixBits ? pos - kRadixBits : 0, width = pos - shift;
         const uint64_t dmask = (1ull << width) - 1ull;
-        hist[tid] = 0;
+        for (int i = tid; i < kRadixBins; i += nt) hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kSpThreads) {
+        for (int i = tid; i < n; i += nt) {
             const uint64_t key = k[i];
             if (key != kNoKey && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
         }
         __syncthreads();
-        const int h = hist[tid];
+        int h[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            h[j] = j < bpt ? hist[tid * bpt + j] : 0;
+            sum += h[j];
+        }
         int total;
-        const int acc = block_exclusive_scan_int(h, scan_w, &total);
-        if (acc < k_rem && acc + h >= k_rem) {
-            sc[0] = tid;
-            sc[1] = h - (k_rem - acc);   // 0 <=> the whole bin is taken
-            sc[2] = k_rem - acc;
+        int acc = block_exclusive_scan_int(sum, scan_w, &total);
+        if (acc < k_rem && acc + sum >= k_rem) {
+            bool found = false;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (found || j >= bpt) continue;
+                if (acc + h[j] >= k_rem) {
+                    sc[0] = tid * bpt + j;
+                    sc[1] = h[j] - (k_rem - acc);   // 0 <=> the whole bin is taken
+                    sc[2] = k_rem - acc;
+                    found = true;
+                } else {
+                    acc += h[j];
+                }
+            }
         }
         __syncthreads();
         const int d = sc[0], surplus = sc[1];
@@ -750,14 +890,42 @@ __device__ void smem_radix_select(const uint64_t *k, int n, int want, int *hist,
     }
 }
 
+// The largest key of k[0..n) that the radix select kept ((key & mask) <= prefix).
+__device__ uint64_t selected_max(const uint64_t *k, int n, uint64_t prefix, uint64_t mask, uint64_t *red) {
+    uint64_t t = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        if (k[i] != kNoKey && (k[i] & mask) <= prefix) t = k[i] > t ? k[i] : t;
+    return block_max_u64(t, red);
+}
+
+// The `want` best of the survivors sk[0..ns) (unique keys, ns >= want), placed
+// in rank order: a survivor's rank is its number of better survivors (every
+// thread counts for its own survivors over the whole list -- broadcast reads,
+// no barrier in between), so the winners land at f.win_k[rank] directly.
+constexpr int kRankDirect = 512;   // most survivors ranked by counting
+__device__ void place_by_rank(const uint64_t *sk, const int *se, int ns, int want, const FinishSmem &f) {
+    for (int i = threadIdx.x; i < ns; i += blockDim.x) {
+        const uint64_t x = sk[i];
+        int c = 0;
+        for (int j = 0; j < ns; ++j) c += sk[j] < x;
+        if (c < want) {
+            f.win_k[c] = x;
+            f.win_e[c] = se[i];
+        }
+    }
+}
+
 __host__ __device__ inline int sparse_cand_cap(int BW, int m) { return BW * m; }
 __host__ __device__ inline int sparse_surv_cap(int BW) { return BW >= 1024 ? 4096 : (BW >= 256 ? 4 * BW : 1024); }
 
-size_t sparse_smem(const Dims &dm, int m) {
+size_t sparse_smem(const Dims &dm, int m, int node_bits_stride, int slots) {
     const int cc = sparse_cand_cap(dm.BW, m), scap = sparse_surv_cap(dm.BW);
-    return al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) + al16((size_t)scap * 4) +
-           al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) +
-           finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
+    const size_t pick = al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) +
+                        al16((size_t)scap * 4) + al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) +
+                        finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
+    // phase 1: the staged rows, then the per-warp token lists
+    const size_t rows = slots * al16((size_t)dm.V * 4) + (size_t)kSpWarps * node_bits_stride * 4;
+    return pick > rows ? pick : rows;
 }
 
 // Phase 2, by the request's last CTA.  tau = the BW-th best of the beams'
@@ -793,18 +961,28 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
     const FinishSmem f = carve_finish(p, BW, BW, dm.S, 0);
     int *cnts = reinterpret_cast<int *>(p + finish_bytes(BW, BW, dm.S, 0));   // [0] survivors, [1] saturated
 
-    // every load below is independent of the others: one round trip
+    // every load below is independent of the others: one round trip.  Entry
+    // numbering of the key buffer: CSR rows as in the mask; node masks row b
+    // at b * row_stride.
+    const bool csr = a.mask_kind == XGR_MASK_CSR;
     const int n = min(max(a.n_live[r], 0), BW);
-    const int base = a.row_ptr[rb];
-    const int64_t E = (int64_t)a.row_ptr[rb + BW] - base;
+    const int base = csr ? a.row_ptr[rb] : 0;
+    const int64_t E = csr ? (int64_t)a.row_ptr[rb + BW] - base : (int64_t)BW * a.row_stride;
     for (int i = tid; i < BW * m; i += kSpThreads) {
         const int b = i / m;
         hk[i] = b < n ? __ldcg(a.head_k + rb * m + i) : kNoKey;
         he[i] = __ldcg(a.head_e + rb * m + i);
     }
     int c = 0;
-    for (int b = tid; b < BW; b += kSpThreads) c += b < n ? __ldcg(a.row_cnt + rb + b) : 0;
-    for (int b = tid; b <= BW; b += kSpThreads) f.rp[b] = a.row_ptr[rb + b] - base;
+    for (int b = tid; b < BW; b += kSpThreads) {
+        c += b < n ? __ldcg(a.row_cnt + rb + b) : 0;
+        const int len = b < n ? __ldcg(a.row_len + rb + b) : 0, cb = __ldcg(a.row_cb + rb + b);
+        f.rl[b] = len;
+        f.cb[b] = b < n ? cb : -1;
+        f.ce[b] = (b < n && cb >= 0) ? cb + len : -1;
+    }
+    for (int b = tid; b <= BW; b += kSpThreads)
+        f.rp[b] = csr ? a.row_ptr[rb + b] - base : b * a.row_stride;
     if (a.rewire) stage_rows(a, rb, n, f);
     if (E > a.key_cap)
         for (int b = tid; b < n; b += kSpThreads) {
@@ -817,11 +995,11 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
         cnts[1] = 0;
     }
     const int total = block_sum_int(c, red_i);   // valid candidates of the request (+ a barrier)
-    if (a.rewire) stage_children(a, n, f);
     const int want = min(BW, total);
     uint64_t prefix = ~0ull, mask = 0;
+    bool ranked = false;   // the winners were placed in rank order
     const uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-    if (E > a.key_cap) {
+    if (csr && E > a.key_cap) {
         // the key buffer overflowed: exact selection over every candidate
         __syncthreads();
         ReqCand cand;
@@ -845,10 +1023,7 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
         if (total > BW && in_heads >= BW) {
             uint64_t tp, tm;
             smem_radix_select(hk, BW * m, BW, hist, scan_w, red_k, sc, tp, tm);
-            uint64_t t = 0;
-            for (int i = tid; i < BW * m; i += kSpThreads)
-                if (hk[i] != kNoKey && (hk[i] & tm) <= tp) t = hk[i] > t ? hk[i] : t;
-            tau = block_max_u64(t, red_k);
+            tau = selected_max(hk, BW * m, tp, tm, red_k);
         }
         // survivors from the heads; beams whose whole head survived and that have
         // more entries go on the saturated list
@@ -861,14 +1036,15 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
                 se[pos] = he[i];
             }
             const int b = i / m;
-            if (i % m == m - 1 && f.rp[b + 1] - f.rp[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
+            if (i % m == m - 1 && f.rl[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
         }
         __syncthreads();
         const int n_sat = cnts[1];
         for (int q = 0; q < n_sat; ++q) {   // their keys beyond the head (worse than its last)
             const int b = sat[q];
             const uint64_t last = hk[b * m + m - 1];
-            for (int e = max(f.rp[b], 0) + tid; e < (int)min((int64_t)f.rp[b + 1], E); e += kSpThreads) {
+            const int e1 = (int)min((int64_t)f.rp[b] + f.rl[b], E);
+            for (int e = max(f.rp[b], 0) + tid; e < e1; e += kSpThreads) {
                 const uint64_t key = __ldcg(keys + e);
                 if (key == kNoKey || key > tau || key <= last) continue;
                 const int pos = atomicAdd(&cnts[0], 1);
@@ -880,22 +1056,26 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
         }
         __syncthreads();
         const int ns = cnts[0];
-        if (ns <= scap) {
+        if (ns <= kRankDirect) {   // few survivors: each one's rank by counting
+            place_by_rank(sk, se, ns, want, f);
+            ranked = true;
+        } else if (ns <= scap) {
             if (want < ns) smem_radix_select(sk, ns, want, hist, scan_w, red_k, sc, prefix, mask);
             collect(ListCand<false>{sk}, ns, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
         } else {   // more survivors than the buffer: exact selection over the key buffer
-            const KeyCand cand{keys, tau};
+            const KeyCand cand{keys, tau, f.rp, f.rl, csr ? 0 : a.row_stride, n};
             radix_select(cand, E, want, hist, sc, prefix, mask);
             collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
         }
     }
     __syncthreads();
-    finish_request(a, r, min(*f.cnt, want), f);
+    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked);
 }
 
 __global__ void __launch_bounds__(kSpThreads) select_sparse_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int hist[256];
+    __shared__ uint64_t full_bar[kSpWarps];
+    __shared__ int hist[kRadixBins];
     __shared__ int scan_w[32];
     __shared__ int red_i[32];
     __shared__ uint64_t red_k[32];
@@ -907,10 +1087,41 @@ __global__ void __launch_bounds__(kSpThreads) select_sparse_kernel(SelectArgs a)
     const int warp = threadIdx.x / 32;
     const int64_t rb = (int64_t)r * dm.BW;
     const int n_live = min(max(a.n_live[r], 0), dm.BW);
-    const int base = a.row_ptr[rb];
+    const int base = a.mask_kind == XGR_MASK_CSR ? a.row_ptr[rb] : 0;
     uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-    const int b1 = min(dm.BW, part * R + R);
-    for (int b = part * R + warp; b < b1; b += kSpWarps) sparse_row(a, r, b, n_live, base, keys);
+    const int b0 = part * R, b1 = min(dm.BW, part * R + R);
+    // short logits rows (every warp's fits beside the others') are staged by
+    // the TMA engine, one slot and one landing barrier per warp; longer ones
+    // stream through registers
+    const int ns = a.sp_slots;   // 0 or R
+    const size_t xb = al16((size_t)dm.V * 4);
+    float *xslot = reinterpret_cast<float *>(smem);
+    int *wtok = reinterpret_cast<int *>(smem + ns * xb) + (size_t)warp * a.row_stride;   // NODE_BITS rows
+    if (ns > 0) {
+        if (threadIdx.x == 0) {
+            for (int w = 0; w < ns; ++w) mbar_init(smem_u32(&full_bar[w]), 1);
+            fence_mbar_init();
+            for (int w = 0; w < min(ns, b1 - b0); ++w) {
+                if (b0 + w >= n_live) continue;   // dead rows are not read
+                mbar_expect_tx(smem_u32(&full_bar[w]), (uint32_t)dm.V * 4u);
+                bulk_g2s(smem_u32(xslot + (size_t)w * (xb / 4)), a.scores + (rb + b0 + w) * dm.V,
+                         (uint32_t)dm.V * 4u, smem_u32(&full_bar[w]));
+            }
+        }
+        __syncthreads();
+    }
+    const int b = b0 + warp;
+    if (b < b1) {
+        const float *xs = nullptr;
+        if (ns > 0 && b < n_live) {
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[warp]), 0, nullptr))) {
+                if ((threadIdx.x & 31) == 0) set_status(a.status, XGR_DEV_TIMEOUT);
+            } else {
+                xs = xslot + (size_t)warp * (xb / 4);
+            }
+        }
+        sparse_row(a, r, b, n_live, base, keys, wtok, xs);
+    }
     // the request's last CTA to arrive selects
     __threadfence();   // this thread's keys and head are visible before the ticket
     __syncthreads();
@@ -925,58 +1136,47 @@ __global__ void __launch_bounds__(kSpThreads) select_sparse_kernel(SelectArgs a)
 // ------------------------------------------------------------------ dense step
 
 // The first step: one live beam per request and the dense bitset of valid
-// first tokens.  One CTA of kSpThreads per request: the beam's score row is
-// staged by one bulk copy; its log-sum-exp from per-warp partials; then the
-// row is cut into slices of Z tokens, and a warp takes the key of every valid
-// token of a slice and the slice's head (its m best keys, in order).  tau =
-// the BW-th best head key; the survivors -- head keys at or above tau, plus
-// the further keys of slices whose whole head survived, recomputed from the
-// staged row -- go through the exact radix select, then finish_request.
-// Z is chosen so that the heads hold at least 2*BW keys where the row allows.
-__host__ __device__ inline int dense_slice(int V, int BW, int m) {
-    const int64_t z = ((int64_t)V * m / (2 * (int64_t)BW)) / 32 * 32;
-    return (int)(z < 32 ? 32 : (z > 256 ? 256 : z));
-}
-__host__ __device__ inline int dense_heads(int V, int BW, int m) {
-    const int z = dense_slice(V, BW, m);
-    return (V + z - 1) / z * m;
-}
+// first tokens.  One CTA of kDnThreads per request: the beam's score row is
+// staged by one bulk copy; its log-sum-exp from per-warp partials; every
+// thread takes the keys of its tokens t = tid + kDnThreads * u and keeps their
+// minimum -- kDnThreads real candidates at most; tau = the BW-th best of
+// these (so at least BW candidates rank at or above it); the survivors at or
+// above tau (each thread recomputes its keys from the staged row) are ranked
+// by counting, then finish_request.
+constexpr int kDnThreads = 512;
 __host__ __device__ inline int dense_surv_cap(int BW) { return BW >= 512 ? 4 * BW : 2048; }
 __host__ __device__ inline size_t dense_x_bytes(int V) { return al16((size_t)V * 4); }
 __host__ __device__ inline size_t dense_bits_bytes(int V) { return al16((size_t)((V + 31) / 32) * 4); }
 
-size_t dense_smem(const Dims &dm, int m) {
-    const int nh = dense_heads(dm.V, dm.BW, m), scap = dense_surv_cap(dm.BW);
-    return dense_x_bytes(dm.V) + dense_bits_bytes(dm.V) + al16((size_t)nh * 8) + al16((size_t)nh * 4) +
-           al16((size_t)scap * 8) + al16((size_t)scap * 4) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32) +
-           64;
+size_t dense_smem(const Dims &dm) {
+    const int scap = dense_surv_cap(dm.BW);
+    return dense_x_bytes(dm.V) + dense_bits_bytes(dm.V) + al16((size_t)kDnThreads * 8) +
+           al16((size_t)scap * 8) + al16((size_t)scap * 4) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32) + 64;
 }
 
-__global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bar_mem;
-    __shared__ float red_f[2 * kSpWarps];
+    __shared__ float red_f[2 * (kDnThreads / 32)];
     __shared__ int red_i[32];
     __shared__ int scan_w[32];
     __shared__ uint64_t red_k[32];
-    __shared__ int hist[256];
+    __shared__ int hist[kRadixBins];
     __shared__ int sc[4];
-    __shared__ int cnts[2];
+    __shared__ int cnts[1];
+    constexpr int kWarps = kDnThreads / 32;
     const Dims dm = a.dims;
-    const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32, m = a.head_m;
+    const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32;
     const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rb = (int64_t)r * BW;
-    const int Z = dense_slice(V, BW, m), n_sl = (V + Z - 1) / Z, nh = n_sl * m;
     const int scap = dense_surv_cap(BW);
     uint8_t *p = smem;
     float *x = reinterpret_cast<float *>(p);
     p += dense_x_bytes(V);
     uint32_t *bits = reinterpret_cast<uint32_t *>(p);
     p += dense_bits_bytes(V);
-    uint64_t *hk = reinterpret_cast<uint64_t *>(p);
-    p += al16((size_t)nh * 8);
-    int *he = reinterpret_cast<int *>(p);
-    p += al16((size_t)nh * 4);
+    uint64_t *mins = reinterpret_cast<uint64_t *>(p);
+    p += al16((size_t)kDnThreads * 8);
     uint64_t *sk = reinterpret_cast<uint64_t *>(p);
     p += al16((size_t)scap * 8);
     int *se = reinterpret_cast<int *>(p);
@@ -989,7 +1189,6 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
     if (tid == 0) {
         *f.cnt = 0;
         cnts[0] = 0;
-        cnts[1] = 0;
         if (bulk && n > 0) {
             mbar_init(bar, 1);
             fence_mbar_init();
@@ -1000,7 +1199,7 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
     const float cum = a.cum[rb];
     // the mask with the tokens past V cleared; the valid-candidate count
     int c = 0;
-    for (int w = tid; w < nw; w += kSpThreads) {
+    for (int w = tid; w < nw; w += kDnThreads) {
         const uint32_t v = a.bits[w] & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u);
         bits[w] = v;
         c += __popc(v);
@@ -1010,7 +1209,7 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
         if (a.trie.root_bits) {
             // root children: bitset and exclusive prefix popcounts (trie order =
             // token order); thread t owns words [t*wpt, t*wpt + wpt)
-            const int wpt = (nw + kSpThreads - 1) / kSpThreads;
+            const int wpt = (nw + kDnThreads - 1) / kDnThreads;
             int cw = 0;
             for (int k = 0; k < wpt; ++k) {
                 const int w = tid * wpt + k;
@@ -1032,19 +1231,23 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
         }
     }
     if (!bulk && n > 0)
-        for (int i = tid; i < V; i += kSpThreads) x[i] = xg[i];
+        for (int i = tid; i < V; i += kDnThreads) x[i] = xg[i];
     const int total = n > 0 ? block_sum_int(c, red_i) : 0;   // (+ a barrier)
     if (bulk && n > 0 && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
     const int want = min(BW, total);
     float lse = 0.f;
     if (a.logits && want > 0) {   // per-warp (max, sum) over a slice, then combined
-        const int per = (V + kSpWarps - 1) / kSpWarps;
+        const int per = (V + kWarps - 1) / kWarps;
         float mw = -INFINITY, sw = 0.f;
         bool nan = false;
         for (int i = warp * per + lane; i < min(V, warp * per + per); i += 32) {
             const float v = x[i];
             nan |= v != v;
-            lse_pair_merge(mw, sw, v, 1.f);
+            if (v > mw) {
+                sw = mw == -INFINITY ? 0.f : sw * ex2f((mw - v) * kLog2e);
+                mw = v;
+            }
+            if (mw != -INFINITY) sw += ex2f((v - mw) * kLog2e);
         }
         if (__any_sync(0xffffffffu, nan) && lane == 0) set_status(a.status, XGR_DEV_NAN);
 #pragma unroll
@@ -1058,72 +1261,43 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
         }
         __syncthreads();
         float M = red_f[0], Ssum = red_f[1];
-        for (int k = 1; k < kSpWarps; ++k) lse_pair_merge(M, Ssum, red_f[2 * k], red_f[2 * k + 1]);
+        for (int k = 1; k < kWarps; ++k) lse_pair_merge(M, Ssum, red_f[2 * k], red_f[2 * k + 1]);
         lse = M + logf(Ssum);
     }
     DenseCand cand{x, bits, cum, lse, V, a.logits, a.status};
     uint64_t prefix = ~0ull, mask = 0;
+    bool ranked = false;
     if (want > 0) {
-        // keys and heads: warp w takes slices w, w + 8, ...
-        for (int sl = warp; sl < n_sl; sl += kSpWarps) {
-            uint64_t ck[8];
-            int cke[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = sl * Z + u * 32 + lane;
-                uint64_t key = kNoKey;
-                if (u * 32 < Z && t < V) cand(t, key);
-                ck[u] = key;
-                cke[u] = t;
-            }
-            uint64_t run = kNoKey;
-            int run_e = -1;
-            warp_head_merge(ck, cke, run, run_e, m);
-            if (lane < m) {
-                hk[sl * m + lane] = run;
-                he[sl * m + lane] = run_e;
-            }
+        // each thread's best key: real candidates for the threshold
+        uint64_t mn = kNoKey;
+        for (int t = tid; t < V; t += kDnThreads) {
+            uint64_t key = kNoKey;
+            if (cand(t, key) && key < mn) mn = key;
         }
-        __syncthreads();
-        int c0 = 0;
-        for (int i = tid; i < nh; i += kSpThreads) c0 += hk[i] != kNoKey;
-        const int in_heads = block_sum_int(c0, red_i);
+        mins[tid] = mn;
+        const int n_min = block_sum_int(mn != kNoKey ? 1 : 0, red_i);   // (+ a barrier)
         uint64_t tau = kNoKey;
-        if (total > BW && in_heads >= BW) {
+        if (total > BW && n_min >= BW) {
             uint64_t tp, tm;
-            smem_radix_select(hk, nh, BW, hist, scan_w, red_k, sc, tp, tm);
-            uint64_t t = 0;
-            for (int i = tid; i < nh; i += kSpThreads)
-                if (hk[i] != kNoKey && (hk[i] & tm) <= tp) t = hk[i] > t ? hk[i] : t;
-            tau = block_max_u64(t, red_k);
+            smem_radix_select(mins, kDnThreads, BW, hist, scan_w, red_k, sc, tp, tm);
+            tau = selected_max(mins, kDnThreads, tp, tm, red_k);
         }
-        // survivors: heads at or above tau, then the further keys of the slices
-        // whose whole head survived (recomputed from the staged row)
-        for (int i = tid; i < nh; i += kSpThreads) {
-            const uint64_t key = hk[i];
-            if (key == kNoKey || key > tau) continue;
+        // survivors: every key at or above tau, recomputed from the staged row
+        for (int t = tid; t < V; t += kDnThreads) {
+            uint64_t key;
+            if (!cand(t, key) || key > tau) continue;
             const int pos = atomicAdd(&cnts[0], 1);
             if (pos < scap) {
                 sk[pos] = key;
-                se[pos] = he[i];
-            }
-        }
-        for (int sl = warp; sl < n_sl; sl += kSpWarps) {
-            const uint64_t last = hk[sl * m + m - 1];
-            if (last == kNoKey || last > tau) continue;   // (uniform across the warp)
-            for (int t = sl * Z + lane; t < min(V, sl * Z + Z); t += 32) {
-                uint64_t key;
-                if (!cand(t, key) || key > tau || key <= last) continue;
-                const int pos = atomicAdd(&cnts[0], 1);
-                if (pos < scap) {
-                    sk[pos] = key;
-                    se[pos] = t;
-                }
+                se[pos] = t;
             }
         }
         __syncthreads();
         const int ns = cnts[0];
-        if (ns <= scap) {
+        if (ns <= kRankDirect) {
+            place_by_rank(sk, se, ns, want, f);
+            ranked = true;
+        } else if (ns <= scap) {
             if (want < ns) smem_radix_select(sk, ns, want, hist, scan_w, red_k, sc, prefix, mask);
             collect(ListCand<false>{sk}, ns, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
         } else {   // more survivors than the buffer: exact selection over every token
@@ -1132,7 +1306,7 @@ __global__ void __launch_bounds__(kSpThreads) select_dense_kernel(SelectArgs a) 
         }
     }
     __syncthreads();
-    finish_request(a, r, min(*f.cnt, want), f);
+    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked);
 }
 
 // opt in to the dynamic shared memory a launch needs: without it static plus
@@ -1153,7 +1327,7 @@ int select_head_m(int BW) { return BW >= 1024 ? 4 : 8; }
 
 size_t select_ticket_offset(int B, int BW) {
     const size_t rows = (size_t)B * BW, m = (size_t)select_head_m(BW);
-    return al256(rows * 4) + al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4);
+    return 4 * al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4);
 }
 
 size_t select_scratch_bytes(int B, int BW, int64_t key_cap) {
@@ -1166,6 +1340,10 @@ void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectA
     a.row_lse = reinterpret_cast<float *>(base);
     base += al256(rows * 4);
     a.row_cnt = reinterpret_cast<int32_t *>(base);
+    base += al256(rows * 4);
+    a.row_len = reinterpret_cast<int32_t *>(base);
+    base += al256(rows * 4);
+    a.row_cb = reinterpret_cast<int32_t *>(base);
     base += al256(rows * 4);
     a.head_k = reinterpret_cast<uint64_t *>(base);
     base += al256(rows * m * 8);
@@ -1193,20 +1371,32 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
     const Dims &dm = a.dims;
     if (dm.BW > 1024 || dm.V > kSelectMaxVocab || dm.V < 1) return cudaErrorInvalidValue;
     if (a.dense) {
-        if (a.head_m < 1 || a.head_m > 32) return cudaErrorInvalidValue;
-        const size_t smem = dense_smem(dm, a.head_m);
+        const size_t smem = dense_smem(dm);
         cudaError_t e = ensure_smem(select_dense_kernel, smem);
         if (e != cudaSuccess) return e;
-        select_dense_kernel<<<dm.B, kSpThreads, smem, s>>>(a);
+        select_dense_kernel<<<dm.B, kDnThreads, smem, s>>>(a);
         return cudaGetLastError();
     }
-    // sparse: one launch, sp_parts CTAs per request (a beam per warp at a time;
-    // fewer CTAs when only the masked entries' log-probs are read)
-    const int R = std::min(dm.BW, a.logits ? kSpWarps : 4 * kSpWarps);
+    // sparse: one launch, sp_parts CTAs per request of R beams, one per warp
+    const int R = std::min(dm.BW, kSpWarps);
     a.sp_rows = R;
     a.sp_parts = (dm.BW + R - 1) / R;
     if (a.head_m < 1 || a.head_m > 32) return cudaErrorInvalidValue;
-    const size_t smem = sparse_smem(dm, a.head_m);
+    if (a.mask_kind != XGR_MASK_CSR && a.mask_kind != XGR_MASK_TRIE_ROWS && a.mask_kind != XGR_MASK_NODE_BITS)
+        return cudaErrorInvalidValue;
+    if (a.mask_kind != XGR_MASK_CSR && (int64_t)dm.BW * a.row_stride > a.key_cap) return cudaErrorInvalidValue;
+    const int wt = a.mask_kind == XGR_MASK_NODE_BITS ? a.row_stride : 0;
+    // logits rows through the TMA engine: as many slots of a row as fit beside
+    // the token lists (each CTA takes R <= 8 rows, one per warp)
+    a.sp_slots = 0;
+    if (a.logits && (dm.V & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0) {
+        const size_t room = (200u << 10) - (size_t)kSpWarps * wt * 4;
+        // only when every warp gets a slot of its own: a slot handed from warp to
+        // warp would leave the later rows waiting for the earlier ones
+        if (room / al16((size_t)dm.V * 4) >= (size_t)R) a.sp_slots = R;
+    }
+    const size_t smem = sparse_smem(dm, a.head_m, wt, a.sp_slots);
+    if (smem > (220u << 10)) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(select_sparse_kernel, smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)dm.B * a.sp_parts;

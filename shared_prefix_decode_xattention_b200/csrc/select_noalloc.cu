@@ -105,6 +105,7 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     a.logits = flags == XGR_SCORES_LOGITS;
     a.scores = d_scores;
     a.dense = dense;
+    a.mask_kind = dense ? XGR_MASK_DENSE : XGR_MASK_CSR;
     a.bits = d_bits;
     a.row_ptr = d_row_ptr;
     a.cols = d_cols;

@@ -15,6 +15,12 @@ using namespace xgr;
 namespace {
 
 constexpr size_t kAlign = 256;
+// the largest pre-generated table of per-node bitsets (dense masks of step 1)
+constexpr size_t kNodeBitsMax = size_t(256) << 20;
+// a level takes dense masks when its nodes have at least V / 256 children on
+// average (many candidates per beam) and at most kNodeBitsStride children each
+// (the selection compacts a row's bits into a per-warp list of that size)
+constexpr int kNodeBitsStride = 2048;
 constexpr int kMinChunk = 256;     // fewest keys per split-K work item
 // the separate merge kernel that split items need, in key units of the
 // tensor-core loop (one more dependent launch plus a few round trips)
@@ -45,10 +51,10 @@ int64_t plan_item_cap(const xgr_config &c) {
 struct Layout {
     size_t status, n_live, cum, node, anc, seq;
     size_t kstore, vstore, pool_k, pool_v;
-    size_t trie_ptr, trie_tok, root_bits;
+    size_t trie_ptr, trie_tok, root_bits, node_bits;
+    size_t node_bits_bytes;    // room for the pre-generated per-node bitsets of level 1
     int64_t trie_level_cap;    // ints per level in each of trie_ptr / trie_tok
-    size_t mask_row_ptr, mask_cols, mask_sync;
-    int64_t mask_cap;
+    size_t mask_sync;
     size_t select_scratch;
     int64_t key_cap;             // selection keys per request
     size_t part_o, part_ml;
@@ -82,17 +88,20 @@ void make_layout(const xgr_config &c, Layout &L) {
         L.trie_ptr = take(4 * S * L.trie_level_cap);
         L.trie_tok = take(4 * S * L.trie_level_cap);
         L.root_bits = take(4 * ((c.vocab + 31) / 32));
-        L.mask_cap = B * BW * (int64_t)fanout_cap(c);
-        L.mask_row_ptr = take(4 * (B * BW + 1));
+        // level 1 has at most min(V, items) nodes; its dense table is kept only
+        // when it fits kNodeBitsMax
+        const size_t nb = (size_t)std::min<int64_t>(c.vocab, c.max_items) * (size_t)((c.vocab + 31) / 32) * 4;
+        L.node_bits_bytes = (c.steps >= 2 && nb <= kNodeBitsMax) ? nb : 0;
+        L.node_bits = L.node_bits_bytes ? take(L.node_bits_bytes) : 0;
+
         L.mask_sync = take(8 * (B + 1));   // look-back words, then the two ticket words
-        L.mask_cols = take(4 * L.mask_cap);
         L.key_cap = BW * (int64_t)fanout_cap(c);
         L.select_scratch = take(select_scratch_bytes((int)B, (int)BW, L.key_cap));
     } else {
         L.trie_level_cap = 0;
-        L.trie_ptr = L.trie_tok = L.root_bits = L.mask_row_ptr = L.mask_cols = L.mask_sync = 0;
+        L.trie_ptr = L.trie_tok = L.root_bits = L.mask_sync = 0;
+        L.node_bits = L.node_bits_bytes = 0;
         L.select_scratch = 0;
-        L.mask_cap = 0;
         L.key_cap = 0;
     }
     L.slots = partial_slots(c);
@@ -145,6 +154,7 @@ struct xgr_ctx {
     TrieView trie;
     bool has_trie = false;
     int level_fanout[kMaxSteps] = {};   // most children of one node of each trie level
+    bool level_bits[kMaxSteps] = {};    // the level's per-node bitsets are pre-generated
     // prompt KV store bookkeeping (host)
     int64_t kv_used = 0;
     std::vector<int64_t> sid_off, sid_len;
@@ -199,13 +209,11 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
     for (auto &sg : segs)
         for (int r : sg.members) nseg[r]++;
 
-    // kind of every segment: tensor-core tiles of 128 rows when D = 128 and the
-    // segment has more rows than one small-row item holds; else the small-row
-    // kernel, split over the keys (a few query rows -- one beam at step 0, one
-    // request's suffix -- make the stage a K/V stream, which many short CTAs
-    // read faster than a few long tensor-core loops)
+    // kind of every segment: tensor-core tiles of 128 rows whenever D = 128
+    // (few rows waste tensor work, but the loop still streams K/V faster than
+    // the small-row kernel's scalar dot products), else the small-row kernel
     auto rows_of = [&](const Seg &sg) { return (int64_t)sg.members.size() * nb * G; };
-    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > kSmallRows; };
+    auto is_tc = [&](const Seg &sg) { return c->has_tc && rows_of(sg) > 0; };
     // split factor per kind: the fewest waves x keys per item (+ a fixed
     // per-item overhead in key units), over the resident CTAs of the GPU
     // A tensor-core segment left whole finishes its requests itself; splitting
@@ -484,7 +492,23 @@ xgr_status xgr_build_trie(xgr_ctx *c, const int32_t *h_items, int64_t n_items, i
         tv.ptr[l] = dptr;
         tv.tok[l] = dtok;
         c->level_fanout[l] = max_children;
+        c->level_bits[l] = false;
         tv.n_nodes[l + 1] = (int32_t)tok.size();
+        // xGR 2.2 "Hybrid dense/sparse storage": dense, pre-generated masks for
+        // the first steps -- here level 1 (step 1) when its nodes have many
+        // children: one bitset of valid next tokens per node
+        const int n_nodes_l = (int)ptr.size() - 1;
+        const size_t nwv = (size_t)((cf.vocab + 31) / 32);
+        if (l == 1 && c->L.node_bits_bytes >= (size_t)n_nodes_l * nwv * 4 &&
+            max_children <= kNodeBitsStride && (int64_t)tok.size() * 256 >= (int64_t)n_nodes_l * cf.vocab) {
+            std::vector<uint32_t> tb((size_t)n_nodes_l * nwv, 0u);
+            for (int nd = 0; nd < n_nodes_l; ++nd)
+                for (int e = ptr[nd]; e < ptr[nd + 1]; ++e) tb[(size_t)nd * nwv + (tok[e] >> 5)] |= 1u << (tok[e] & 31);
+            if (cudaMemcpy(c->at<uint32_t>(c->L.node_bits), tb.data(), tb.size() * 4, cudaMemcpyHostToDevice) !=
+                cudaSuccess)
+                return XGR_ERR_CUDA;
+            c->level_bits[l] = true;
+        }
         if (l == 0) {
             std::vector<uint32_t> bits((cf.vocab + 31) / 32, 0u);
             for (int32_t t : tok) bits[t >> 5] |= 1u << (t & 31);
@@ -671,36 +695,52 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
 }
 
 xgr_status xgr_build_mask(xgr_ctx *c, int32_t step, xgr_mask *out, xgr_stream_t stream) {
+    (void)stream;   // every kind is a view: nothing is enqueued
     if (!c || !out) return XGR_ERR_ARG;
     if (!c->has_trie || !c->begun || step != c->cur_step || step >= c->cfg.steps)
         return XGR_ERR_STATE;
     std::memset(out, 0, sizeof(*out));
     out->step = step;
     out->n_rows = c->dims.B * c->dims.BW;
+    out->n_words = (c->cfg.vocab + 31) / 32;
     if (step == 0) {
         out->kind = XGR_MASK_DENSE;
         out->bits = c->trie.root_bits;
-        out->n_words = (c->cfg.vocab + 31) / 32;
         return XGR_OK;
     }
+    out->kind = c->level_bits[step] ? XGR_MASK_NODE_BITS : XGR_MASK_TRIE_ROWS;
+    out->bits = c->level_bits[step] ? c->at<uint32_t>(c->L.node_bits) : nullptr;
+    out->row_node = c->st.node;
+    out->node_ptr = c->trie.ptr[step];
+    out->cols = c->trie.tok[step];
+    out->cols_capacity = c->trie.n_nodes[step + 1];
+    out->n_nodes = c->trie.n_nodes[step];
+    out->row_stride = std::max(1, c->level_fanout[step]);
+    return XGR_OK;
+}
+
+xgr_status xgr_mask_to_csr(xgr_ctx *c, const xgr_mask *mask, int32_t *d_row_ptr, int32_t *d_cols,
+                           int64_t cols_capacity, xgr_stream_t stream) {
+    if (!c || !mask || !aligned16(d_row_ptr) || !aligned16(d_cols) || cols_capacity < 1) return XGR_ERR_ARG;
+    if (mask->kind != XGR_MASK_NODE_BITS && mask->kind != XGR_MASK_TRIE_ROWS) return XGR_ERR_ARG;
+    if (!c->has_trie || !c->begun || mask->step != c->cur_step || mask->step < 1 ||
+        mask->step >= c->cfg.steps)
+        return XGR_ERR_STATE;
+    const int step = mask->step;
     MaskArgs ma;
     ma.st = c->st;
     ma.trie = c->trie;
     ma.dims = c->dims;
     ma.step = step;
-    ma.row_ptr = c->at<int32_t>(c->L.mask_row_ptr);
-    ma.cols = c->at<int32_t>(c->L.mask_cols);
-    ma.cap = c->L.mask_cap;
+    ma.row_ptr = d_row_ptr;
+    ma.cols = d_cols;
+    ma.cap = cols_capacity;
     ma.flags = c->at<uint64_t>(c->L.mask_sync);
     ma.ticket = reinterpret_cast<uint32_t *>(ma.flags + c->cfg.max_requests);
     // CTAs per request sharing the copy: about 16K entries each
     const int64_t entries = (int64_t)c->cfg.beam_width * c->level_fanout[step];
     const int parts = (int)std::min<int64_t>(16, std::max<int64_t>(1, (entries + 16383) / 16384));
     if (launch_build_mask(ma, parts, (cudaStream_t)stream) != cudaSuccess) return XGR_ERR_CUDA;
-    out->kind = XGR_MASK_CSR;
-    out->row_ptr = ma.row_ptr;
-    out->cols = ma.cols;
-    out->cols_capacity = ma.cap;
     return XGR_OK;
 }
 
@@ -715,9 +755,23 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     if (!c->has_trie || !c->begun || step != c->cur_step || step >= c->cfg.steps)
         return XGR_ERR_STATE;
     if (mask->step != step) return XGR_ERR_STATE;
-    if (step == 0 ? (mask->kind != XGR_MASK_DENSE || !mask->bits)
-                  : (mask->kind != XGR_MASK_CSR || !mask->row_ptr || !mask->cols))
+    if (step == 0) {
+        if (mask->kind != XGR_MASK_DENSE || !mask->bits) return XGR_ERR_ARG;
+    } else if (mask->kind == XGR_MASK_CSR) {
+        if (!mask->row_ptr || !mask->cols) return XGR_ERR_ARG;
+    } else if (mask->kind == XGR_MASK_TRIE_ROWS || mask->kind == XGR_MASK_NODE_BITS) {
+        // node views of this context's own trie level and beam state only
+        if (mask->row_node != c->st.node || mask->node_ptr != c->trie.ptr[step] ||
+            mask->cols != c->trie.tok[step] || mask->n_nodes != c->trie.n_nodes[step] ||
+            mask->row_stride != std::max(1, c->level_fanout[step]))
+            return XGR_ERR_ARG;
+        if (mask->kind == XGR_MASK_NODE_BITS &&
+            (!c->level_bits[step] || mask->bits != c->at<uint32_t>(c->L.node_bits) ||
+             mask->n_words != (c->cfg.vocab + 31) / 32))
+            return XGR_ERR_ARG;
+    } else {
         return XGR_ERR_ARG;
+    }
     SelectArgs a;
     a.cum = c->st.cum;
     a.n_live = c->st.n_live;
@@ -731,8 +785,16 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.scores = d_scores;
     a.dense = step == 0;
     a.bits = mask->bits;
+    a.mask_kind = mask->kind;
     a.row_ptr = mask->row_ptr;
     a.cols = mask->cols;
+    a.row_node = mask->row_node;
+    a.node_ptr = mask->node_ptr;
+    a.node_tok = mask->cols;
+    a.node_bits = mask->kind == XGR_MASK_NODE_BITS ? mask->bits : nullptr;
+    a.n_nodes = mask->n_nodes;
+    a.n_words = mask->n_words;
+    a.row_stride = mask->row_stride;
     a.num_sms = c->num_sms;
     select_scratch_carve(c->at<uint8_t>(c->L.select_scratch), c->cfg.max_requests,
                          c->cfg.beam_width, c->L.key_cap, a);

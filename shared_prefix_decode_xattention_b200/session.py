@@ -56,12 +56,23 @@ class Session:
     def build_mask(self, step, stream=None) -> xgr.xgr_mask:
         return xgr.xgr_build_mask(self.ctx, step, stream)
 
-    def mask_entries(self, mask: xgr.xgr_mask) -> int:
-        """CSR entries of a mask built in this workspace (reads row_ptr[n_rows]; synchronises)."""
+    def mask_csr(self, mask: xgr.xgr_mask, stream=None):
+        """The rows of a step >= 1 mask as CSR device tensors (row_ptr int32
+        [n_rows+1], cols int32 [cap]; the valid length is row_ptr[-1])."""
         import torch
-        off = mask.row_ptr + 4 * mask.n_rows - self.workspace.data_ptr()
-        assert 0 <= off and off + 4 <= self.nbytes
-        return int(self.workspace[off:off + 4].view(torch.int32).item())
+        dev = self.workspace.device
+        cap = max(1, mask.n_rows * max(1, mask.row_stride))
+        row_ptr = torch.empty(mask.n_rows + 1, dtype=torch.int32, device=dev)
+        cols = torch.empty(cap, dtype=torch.int32, device=dev)
+        xgr.xgr_mask_to_csr(self.ctx, mask, row_ptr, cols, cap, stream)
+        return row_ptr, cols
+
+    def mask_entries(self, mask: xgr.xgr_mask) -> int:
+        """Valid (row, token) entries of a step >= 1 mask (synchronises)."""
+        import torch
+        row_ptr, _ = self.mask_csr(mask)
+        torch.cuda.synchronize()
+        return int(row_ptr[-1].item())
 
     def beam_select(self, step, scores, flags, mask, parent, token, cum, n_out, stream=None):
         xgr.xgr_beam_select(self.ctx, step, scores, flags, mask, parent, token, cum, n_out, stream)

@@ -41,6 +41,8 @@ XGR_KV_SHARED = 0
 XGR_KV_SUFFIX = 1
 XGR_MASK_DENSE = 0
 XGR_MASK_CSR = 1
+XGR_MASK_NODE_BITS = 2
+XGR_MASK_TRIE_ROWS = 3
 
 
 class XgrError(RuntimeError):
@@ -77,6 +79,10 @@ class xgr_mask(ctypes.Structure):
         ("row_ptr", ctypes.c_void_p),
         ("cols", ctypes.c_void_p),
         ("cols_capacity", ctypes.c_int64),
+        ("row_node", ctypes.c_void_p),
+        ("node_ptr", ctypes.c_void_p),
+        ("n_nodes", ctypes.c_int32),
+        ("row_stride", ctypes.c_int32),
     ]
 
 
@@ -112,6 +118,7 @@ def lib():
         "xgr_begin": [P, i32, P],
         "xgr_decode_step": [P, i32, P, P, P, P, P, P],
         "xgr_build_mask": [P, i32, ctypes.POINTER(xgr_mask), P],
+        "xgr_mask_to_csr": [P, ctypes.POINTER(xgr_mask), P, P, i64, P],
         "xgr_beam_select": [P, i32, P, i32, ctypes.POINTER(xgr_mask), P, P, P, P, P],
         "xgr_get_sequences": [P, P, P],
         "xgr_device_status": [P, P, ctypes.POINTER(i32)],
@@ -209,6 +216,11 @@ def xgr_build_mask(ctx: int, step: int, stream=None) -> xgr_mask:
     m = xgr_mask()
     _check("xgr_build_mask", lib().xgr_build_mask(ctx, step, ctypes.byref(m), _stream(stream)))
     return m
+
+
+def xgr_mask_to_csr(ctx: int, mask: xgr_mask, row_ptr, cols, cols_capacity: int, stream=None) -> None:
+    _check("xgr_mask_to_csr", lib().xgr_mask_to_csr(ctx, ctypes.byref(mask), _ptr(row_ptr), _ptr(cols),
+                                                    cols_capacity, _stream(stream)))
 
 
 def xgr_beam_select(ctx: int, step: int, scores, flags: int, mask: xgr_mask, parent, token, cum,

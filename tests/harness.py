@@ -65,6 +65,7 @@ class GpuRun:
                 self.kv[("x", r)] = (k, v)
                 self.sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
         self.sess.begin(w.B)
+        self.kinds = []   # the mask kind of every sparse step
 
     def step(self, s, q, kn, vn, scores=None, flags=xgr.XGR_SCORES_LOGPROB) -> StepOut:
         w = self.w
@@ -81,15 +82,15 @@ class GpuRun:
             _copy_dev(bits, m.bits, m.n_words * 4, self.sess)
             mask = ("dense", bits.cpu().numpy().view(np.uint32).copy())
         else:
-            n_rows = m.n_rows
-            rp = torch.empty(n_rows + 1, dtype=torch.int32, device=self.device)
-            _copy_dev(rp, m.row_ptr, (n_rows + 1) * 4, self.sess)
+            assert m.kind in (xgr.XGR_MASK_NODE_BITS, xgr.XGR_MASK_TRIE_ROWS), m.kind
+            self.kinds.append(m.kind)
+            rp, cols = self.sess.mask_csr(m)   # the rows the selection reads, written out
+            torch.cuda.synchronize()
             rpn = rp.cpu().numpy()
             nnz = int(rpn[-1])
-            cols = torch.empty(max(nnz, 1), dtype=torch.int32, device=self.device)
-            if nnz:
-                _copy_dev(cols, m.cols, nnz * 4, self.sess)
             mask = ("csr", (rpn.astype(np.int64), cols.cpu().numpy()[:nnz].copy()))
+            if m.kind == xgr.XGR_MASK_NODE_BITS:
+                _check_node_bits(m, mask[1], w.V, self.sess)
         parent = torch.empty((w.B, w.BW), dtype=torch.int32, device=self.device)
         token = torch.empty_like(parent)
         cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=self.device)
@@ -108,6 +109,28 @@ class GpuRun:
 
     def status(self) -> int:
         return self.sess.device_status()
+
+
+def _check_node_bits(m, csr, V: int, sess: Session):
+    """The pre-generated bitset of every row's node holds exactly that row's
+    valid tokens (the CSR rows, themselves compared with the oracle)."""
+    nodes = torch.empty(m.n_rows, dtype=torch.int32, device=sess.workspace.device)
+    _copy_dev(nodes, m.row_node, m.n_rows * 4, sess)
+    off = m.bits - sess.workspace.data_ptr()
+    nbytes = m.n_nodes * m.n_words * 4
+    assert 0 <= off and off + nbytes <= sess.nbytes
+    table = sess.workspace[off:off + nbytes].view(torch.int32).view(m.n_nodes, m.n_words)
+    nd = nodes.cpu().numpy()
+    rows = np.nonzero(nd >= 0)[0]
+    got = table[torch.as_tensor(nd[rows]).long().to(table.device)].cpu().numpy().view(np.uint8)
+    dense = np.unpackbits(got, axis=1, bitorder="little")[:, :V].astype(bool)
+    rp, cols = csr
+    want = np.zeros_like(dense)
+    for i, row in enumerate(rows):
+        want[i, cols[rp[row]:rp[row + 1]]] = True
+    assert np.array_equal(dense, want), "a node's pre-generated bitset differs from its valid tokens"
+    for row in np.nonzero(nd < 0)[0]:
+        assert rp[row + 1] == rp[row], "a row without a node has tokens"
 
 
 def _copy_dev(dst: torch.Tensor, src_ptr: int, nbytes: int, sess: Session):

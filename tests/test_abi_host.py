@@ -30,6 +30,15 @@ def _cfg(**kw):
     return xgr.make_config(**base)
 
 
+def test_mask_struct_matches_the_header(L):
+    """xgr_mask as ctypes lays it out: the field order and the 72 bytes of the
+    C struct (natural alignment on x86-64)."""
+    names = [f[0] for f in xgr.xgr_mask._fields_]
+    assert names == ["kind", "step", "bits", "n_words", "n_rows", "row_ptr", "cols",
+                     "cols_capacity", "row_node", "node_ptr", "n_nodes", "row_stride"]
+    assert ctypes.sizeof(xgr.xgr_mask) == 72
+
+
 def test_workspace_bytes_for_a_valid_config(L):
     n = xgr.xgr_workspace_bytes(_cfg())
     assert n % 256 == 0 and n > 8192 * 4 * 128 * 2 * 2
@@ -59,6 +68,7 @@ def test_null_arguments(L):
     m = xgr.xgr_mask()
     assert L.xgr_beam_select(None, 0, None, 0, ctypes.byref(m), None, None, None, None,
                              None) == xgr.XGR_ERR_ARG
+    assert L.xgr_mask_to_csr(None, ctypes.byref(m), None, None, 1, None) == xgr.XGR_ERR_ARG
     assert xgr.xgr_status_string(xgr.XGR_ERR_CAPACITY).startswith("capacity")
 
 

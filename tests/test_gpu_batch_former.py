@@ -49,16 +49,19 @@ def test_tree_batches_feed_the_attention():
         list(range(g * 16, g * 16 + 16)) for g in range(w.groups)]
     assert all(sh * CHUNK == int(workloads.prompt_lengths(w)[0]) for _, sh in batches)
 
+    # the families' prefix K/V and the requests' suffix K/V (drawn once on the
+    # device; the oracle reads the same tensors)
+    fam_kv = {g: workloads.shared_kv(w, g, "cuda") for g in range(w.groups)}
+    suf_kv = {r: workloads.suffix_kv(w, r, "cuda") for r in range(w.B)}
     sess = Session(config_for(w), "cuda")
     for sid, (members, shared_chunks) in enumerate(batches):
         depth = shared_chunks * CHUNK
-        k, v = workloads.shared_kv(w, w.shared_id(members[0]), "cuda")   # the first member's prefix
+        k, v = fam_kv[w.shared_id(members[0])]   # the batch's prefix: its first member's
         sess.prefill(members[0], sid, k[:, :depth].contiguous(), v[:, :depth].contiguous())
         for r in members[1:]:
             sess.link(r, sid)
     for r in range(w.B):
-        k, v = workloads.suffix_kv(w, r, "cuda")
-        sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+        sess.prefill(r, 0, *suf_kv[r], kind=xgr.XGR_KV_SUFFIX)
     sess.begin(w.B)
     q, kn, vn = workloads.step_qkv(w, 0, "cuda")
     out = torch.full((w.B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -67,8 +70,8 @@ def test_tree_batches_feed_the_attention():
     torch.cuda.synchronize()
     qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
     for r in range(w.B):
-        ks, vs = workloads.shared_kv(w, w.shared_id(r), "cpu")
-        kx, vx = workloads.suffix_kv(w, r, "cpu")
+        ks, vs = fam_kv[w.shared_id(r)]   # the request's own full prompt
+        kx, vx = suf_kv[r]
         dec = oracle.BeamDecode(None, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V)
         dec.begin(u16(ks), u16(vs), u16(kx), u16(vx))
         o_ref, l_ref = dec.attention(0, qc[r], knc[r], vnc[r])

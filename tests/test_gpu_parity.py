@@ -78,7 +78,7 @@ def decode_and_compare(w, mode="logprob", requests=None, beams_per_step=None, it
                 assert tuple(seq[r, b].tolist()) in item_set
     assert run.status() == 0
     run.sess.close()
-    return worst
+    return worst, run.kinds
 
 
 def test_workload1_logprob_full():
@@ -90,7 +90,11 @@ def test_workload1_logits_tie_aware():
 
 
 def test_workload2_logprob_full():
-    decode_and_compare(workloads.WORKLOADS[2])
+    _, kinds = decode_and_compare(workloads.WORKLOADS[2])
+    # xGR 2.2 "Hybrid dense/sparse storage": step 1 (about 122 valid tokens per
+    # beam out of 8192) takes the pre-generated per-node bitsets, step 2 (about
+    # one) the trie rows that the rewiring updates in place
+    assert kinds == [xgr.XGR_MASK_NODE_BITS, xgr.XGR_MASK_TRIE_ROWS]
 
 
 def test_workload2_logits_sampled():
@@ -103,8 +107,9 @@ def test_workload3_sampled():
 
 
 def test_workload3_logits_sampled():
-    """Logits mode at the 512x512 pool: row log-sum-exp over V = 8192 and pools
-    above 32K entries (the multi-CTA threshold pick)."""
+    """Logits mode at the 512x512 pool: row log-sum-exp over V = 8192, about 475
+    valid tokens per beam at step 1 (beams whose whole head survives the
+    threshold, so their further keys are read)."""
     decode_and_compare(workloads.WORKLOADS[3], mode="logits", requests=[3, 30], beams_per_step=8)
 
 
@@ -141,10 +146,11 @@ def test_ragged_prompts_and_split_k():
 
 
 def test_unshared_staging_in_batches():
-    """The tensor-core kernel stages each beam's own k/v rows in a 64 KB area;
-    when a tile's beams x tokens exceed it, it works in batches.  G = 1 (128
-    beams in a 128-row tile: two batches of beams, one token each) and G = 2 over
-    six steps (64 beams, one token per batch)."""
+    """The tensor-core kernel gathers each tile's beams' own k/v rows into
+    128-row Unshared chunks; when the tile's beams x tokens pass 128 it runs
+    several chunks through the same U area.  G = 1 (128 beams in a 128-row
+    tile: up to three chunks at step 2) and G = 2 over six steps (64 beams, up
+    to three chunks)."""
     w = workloads.small(workloads.WORKLOADS[1], wid=105, B=2, prompt=(300, 300), BW=128, K=128,
                         S=3, Hq=4, Hkv=4, D=128, V=256, n_items=20000)
     decode_and_compare(w, beams_per_step=16)

@@ -59,11 +59,13 @@ def test_noalloc_matches_context_select(wid, flags):
                 torch.empty((B, BW), dtype=torch.float32, device=dev),
                 torch.empty((B,), dtype=torch.int32, device=dev)]
         got = [torch.full_like(t, 7) for t in want]
-        run.sess.beam_select(s, scores, flags, m, *want)
         dense = m.kind == xgr.XGR_MASK_DENSE
+        rp = cols = None
+        if not dense:   # the same rows as explicit CSR, the form this call takes
+            rp, cols = run.sess.mask_csr(m)
+        run.sess.beam_select(s, scores, flags, m, *want)
         xgr.xgr_beam_topk_noalloc(B, BW, w.K, w.V, scores, flags, cum, n_live,
-                                  m.bits if dense else None, None if dense else m.row_ptr,
-                                  None if dense else m.cols, *got)
+                                  m.bits if dense else None, rp, cols, *got)
         torch.cuda.synchronize()
         for a, b in zip(want, got):
             assert torch.equal(a.view(torch.int32), b.view(torch.int32)), f"step {s}"
