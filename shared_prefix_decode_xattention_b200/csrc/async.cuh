@@ -78,6 +78,27 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// closes this thread's current group of cp.async copies
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most N of this thread's committed groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the kernel before it in the
+// stream is still running; griddep_wait() returns once that kernel has
+// completed and its memory operations are visible (at once when the launch
+// had no such attribute).  griddep_launch_dependents() lets the next kernel in
+// the stream start early.  A kernel calls it after its own griddep_wait() (so
+// whatever an early-started kernel reads before its own wait was written by
+// kernels that had completed already), unless its only dependent reads no
+// global memory before its wait.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // orders this thread's generic-proxy shared-memory accesses before later
 // async-proxy ones (bulk copies, tensor-core operand reads)

@@ -13,6 +13,7 @@
 // k/v of the beam's step+1 tokens (16-byte vector loads, one 2*D-byte vector
 // per token), then fold in the Shared-stage partials and write O (bf16) and
 // LSE (fp32, natural log).
+#include "async.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -60,6 +61,8 @@ __global__ void __launch_bounds__(kWarps * 32) attn_merge_kernel(MergeArgs a) {
     const int lane = threadIdx.x % 32;
     const int64_t wid = (int64_t)blockIdx.x * kWarps + threadIdx.x / 32;
     const int64_t n_units = (int64_t)dm.B * dm.BW * dm.Hkv;
+    griddep_wait();   // the partials come from the attention kernels before
+    griddep_launch_dependents();
     if (wid >= n_units) return;
     const int g = (int)(wid % dm.Hkv);
     const int b = (int)((wid / dm.Hkv) % dm.BW);
@@ -207,13 +210,12 @@ cudaError_t launch_d(const MergeArgs &a, cudaStream_t st) {
     const int blocks = (int)((units + kWarps - 1) / kWarps);
     if (blocks == 0) return cudaSuccess;
     switch (a.dims.G) {
-        case 1: attn_merge_kernel<D, 1><<<blocks, kWarps * 32, 0, st>>>(a); break;
-        case 2: attn_merge_kernel<D, 2><<<blocks, kWarps * 32, 0, st>>>(a); break;
-        case 4: attn_merge_kernel<D, 4><<<blocks, kWarps * 32, 0, st>>>(a); break;
-        case 8: attn_merge_kernel<D, 8><<<blocks, kWarps * 32, 0, st>>>(a); break;
+        case 1: return launch_pdl(attn_merge_kernel<D, 1>, dim3(blocks), dim3(kWarps * 32), 0, st, a);
+        case 2: return launch_pdl(attn_merge_kernel<D, 2>, dim3(blocks), dim3(kWarps * 32), 0, st, a);
+        case 4: return launch_pdl(attn_merge_kernel<D, 4>, dim3(blocks), dim3(kWarps * 32), 0, st, a);
+        case 8: return launch_pdl(attn_merge_kernel<D, 8>, dim3(blocks), dim3(kWarps * 32), 0, st, a);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

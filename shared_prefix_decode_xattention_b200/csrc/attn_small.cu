@@ -41,7 +41,9 @@ __global__ void __launch_bounds__(kThreads) attn_small_kernel(SmallArgs a) {
     constexpr int kRowGroups = kThreads / D;           // threads per dim
     constexpr int kRowsPerThread = kSmallRows / kRowGroups;
 
-    const WorkItem it = a.items[blockIdx.x];
+    const WorkItem it = a.items[blockIdx.x];   // (the plan is written before any decode kernel)
+    griddep_wait();
+    griddep_launch_dependents();
     const int tid = threadIdx.x;
     const Dims dm = a.dims;
     const int G = dm.G;
@@ -202,8 +204,7 @@ cudaError_t launch_small_impl(const SmallArgs &a, int n_items, cudaStream_t st) 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    attn_small_kernel<D><<<n_items, kThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(attn_small_kernel<D>, dim3(n_items), dim3(kThreads), smem, st, a);
 }
 
 }  // namespace

@@ -285,6 +285,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const WorkItem it = a.items[blockIdx.x];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     if (it.flags & 4) {   // zero-fill item: these CTAs run beside the attention on idle SMs
+        griddep_wait();
+        griddep_launch_dependents();
         const int64_t row0 = ((int64_t)it.r0 * a.dims.BW + it.row_begin) * a.dims.Hq;   // first query row
         const int64_t n = (int64_t)it.n_rows * a.dims.Hq;
         uint4 *o = reinterpret_cast<uint4 *>(a.out + row0 * 128);
@@ -342,14 +344,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             fence_mbar_init();
         }
         __syncwarp();
-        // Q and the first chunks start streaming before the block-wide setup barrier
-        if (lane == 0 && q_tma) {
-            const int G = a.dims.G;
-            const int z = it.r0 * a.dims.BW + it.row_begin / G;
-            mbar_expect_tx(bar(B_QFULL), kTile);
-            tma_load_3d(sb + kOffQ, &tmq, 0, it.g * G, z, bar(B_QFULL));
-            tma_load_3d(sb + kOffQ + kHalf, &tmq, 64, it.g * G, z, bar(B_QFULL));
-        }
+        // The prompt's first K / V chunks stream in while the kernel before this
+        // one finishes: the prompt (and suffix) KV store is written only by the
+        // prefill copies, which completed before any decode kernel started.
         if (lane == 0)
             for (int j = 0; j < min(nchunks, kKStages); ++j) issue_k(j);
         if (lane == 1)
@@ -361,6 +358,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // Everything above touches only this CTA's shared and tensor memory, the
+    // plan (written before any decode kernel) and the prompt KV store; from
+    // here on the kernel reads what the kernels before it wrote (the beam
+    // state, this step's inputs).
+    griddep_wait();
+    griddep_launch_dependents();
+    if (warp == 0 && lane == 0 && q_tma) {   // Q streams in before the block-wide setup barrier
+        const int G = a.dims.G;
+        const int z = it.r0 * a.dims.BW + it.row_begin / G;
+        mbar_expect_tx(bar(B_QFULL), kTile);
+        tma_load_3d(sb + kOffQ, &tmq, 0, it.g * G, z, bar(B_QFULL));
+        tma_load_3d(sb + kOffQ + kHalf, &tmq, 64, it.g * G, z, bar(B_QFULL));
     }
     // softmax threads stage the Q tile meanwhile: 16 consecutive threads read one
     // 256-byte row (coalesced) and write it in the swizzled K-major layout
@@ -840,8 +850,7 @@ cudaError_t launch_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUte
         }
         attr = true;
     }
-    attn_tc_kernel<<<n_items, kTcThreads, kSmemBytes, st>>>(tmk, tmv, tmq, a);
-    return cudaGetLastError();
+    return launch_pdl(attn_tc_kernel, dim3(n_items), dim3(kTcThreads), kSmemBytes, st, tmk, tmv, tmq, a);
 }
 
 }  // namespace

@@ -22,11 +22,9 @@ namespace {
 // score 0.  Without a vocabulary (attention only) every beam is an
 // independent live sequence whose Unshared token of step i sits at slot
 // (i, b).
-__global__ void begin_kernel(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync,
-                             uint32_t *sel_ticket) {
+__global__ void begin_kernel(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (mask_sync && idx <= Bcap) mask_sync[idx] = 0;   // mask look-back words and ticket
-    if (sel_ticket && idx < Bcap) sel_ticket[idx] = 0;  // the selection's tickets
     if (idx >= (int64_t)Bcap * dm.BW) return;
     const int r = (int)(idx / dm.BW), b = (int)(idx % dm.BW);
     const bool live = all_live || b == 0;
@@ -217,9 +215,9 @@ __global__ void get_sequences_kernel(BeamState st, Dims dm, int32_t *seq) {
 }  // namespace
 
 cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync,
-                         uint32_t *sel_ticket, cudaStream_t s) {
+                         cudaStream_t s) {
     const int64_t n = (int64_t)Bcap * dm.BW + 1;
-    begin_kernel<<<(int)((n + 255) / 256), 256, 0, s>>>(st, dm, Bcap, all_live, mask_sync, sel_ticket);
+    begin_kernel<<<(int)((n + 255) / 256), 256, 0, s>>>(st, dm, Bcap, all_live, mask_sync);
     return cudaGetLastError();
 }
 

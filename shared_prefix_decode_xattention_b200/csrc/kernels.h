@@ -73,7 +73,7 @@ cudaError_t launch_attn_merge(const MergeArgs &a, cudaStream_t st);
 // mask_sync: the mask builder's look-back words [Bcap] and ticket, zeroed here
 // sel_ticket: the selection's tickets [Bcap], zeroed here
 cudaError_t launch_begin(BeamState st, Dims dm, int Bcap, int all_live, uint64_t *mask_sync,
-                         uint32_t *sel_ticket, cudaStream_t s);
+                         cudaStream_t s);
 
 // Sparse masks of steps >= 1: one CSR row per beam.
 struct MaskArgs {
@@ -125,12 +125,12 @@ struct SelectArgs {
     uint64_t *head_k;           // [B][BW][m] each beam's m best keys, ascending (kNoKey pads)
     int32_t *head_e;            // [B][BW][m] their CSR entries (relative to the request)
     int head_m;                 // m
-    uint32_t *ticket;           // [B] CTAs of the request done; the last resets it to 0
     uint64_t *keys;             // [B][key_cap] key of each CSR entry (relative to the request)
     int64_t key_cap;
+    int prep_early;             // the kernel before writes no beam state: the mask lookups may
+                                //   run before the programmatic-launch wait
     int sp_parts;               // set by the launcher: CTAs per request of the sparse kernel
     int sp_rows;                //   and the beams each of them takes (<= 8: one per warp)
-    int sp_slots;               //   and its shared-memory slots for logits rows (0: none)
     int num_sms;                // SMs of the device
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;
@@ -150,10 +150,29 @@ constexpr int kSelectMaxVocab = 32768;
 // them zero).
 int select_head_m(int BW);
 size_t select_scratch_bytes(int B, int BW, int64_t key_cap);
-size_t select_ticket_offset(int B, int BW);   // byte offset of the tickets in the scratch
 void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectArgs &a);
 cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
 
 cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);
+
+// Launches `kernel` on `s` with programmatic stream serialization: the
+// kernel may start while the previous kernel in the stream is still running,
+// so it must call griddep_wait() before it reads or writes anything that
+// kernel (or an earlier one) produces or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
 
 }  // namespace xgr

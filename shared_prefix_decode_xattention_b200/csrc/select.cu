@@ -22,18 +22,23 @@
 // Kernels:
 //  * dense mask (one live beam per request, step 0): select_dense_kernel, one
 //    CTA per request, stages the beam's score row with one bulk copy, takes its
-//    log-sum-exp (logits); tau = the BW-th best of the threads' best keys, and
-//    the survivors at or above it are ranked by counting.
-//  * sparse (CSR) masks: select_sparse_kernel, one launch per step.  Each
-//    request gets several CTAs; a warp takes one beam row at a time: its
-//    log-sum-exp (logits), the key of each of its CSR entries, and its head --
-//    the beam's m best keys in order (the page's ordered per-beam candidate
-//    list, cut at m).  The request's last CTA to finish (an atomic ticket)
-//    takes tau = the BW-th best head key (at least BW real candidates rank at
-//    or above it, so every winner does), gathers the survivors at or above tau
-//    -- the head keys, and the further keys of beams whose whole head
-//    survived -- and radix-selects the BW best of them.  It ends in
-//    finish_request: the ordering, the outputs and the rewiring.
+//    log-sum-exp (logits); the cut comes from the threads' best keys (at
+//    least BW real candidates lie at or before it), and the survivors are
+//    ranked by counting.
+//  * sparse masks (steps >= 1): two launches.  select_rows_kernel gives each
+//    beam row a warp: its log-sum-exp (logits), the key of each of its mask
+//    entries, and its head -- the beam's m best keys in order (the page's
+//    ordered per-beam candidate list, cut at m).  select_pick_kernel (one CTA
+//    per request) cuts at the heads (at least BW real candidates lie at or
+//    before the cut, so every winner survives), gathers the survivors -- the
+//    head keys, and the further keys of beams whose whole head survived --
+//    and ranks them.  Both end in finish_request: the ordering, the outputs
+//    and the rewiring.
+//  Every kernel is launched as a programmatic dependent of the kernel before
+//  it; the one-CTA-per-request kernels run a dry pass of their own code on
+//  synthetic shared-memory data before they wait for that kernel, so the
+//  instruction fetches of code that runs once per launch are not on the
+//  critical path.
 #include <algorithm>
 
 #include "async.cuh"
@@ -82,6 +87,11 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
     return v;
 }
 __device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
@@ -252,22 +262,7 @@ struct ListCand {
     }
 };
 
-// the request's key buffer, restricted to the survivors of tau; with a row
-// stride (node masks) only the first rl[b] slots of row b hold keys
-struct KeyCand {
-    const uint64_t *k;
-    uint64_t tau;
-    const int *rp, *rl;   // shared memory
-    int stride, n;        // stride 0: CSR numbering (every entry written)
-    __device__ bool operator()(int64_t e, uint64_t &key) const {
-        if (stride) {
-            const int b = (int)(e / stride), j = (int)(e % stride);
-            if (b >= n || j >= rl[b]) return false;
-        }
-        key = __ldcg(k + e);
-        return key != kNoKey && key <= tau;
-    }
-};
+
 
 // every CSR entry of the request's live beams, keys recomputed from the scores
 // (rp = per-beam entry offsets relative to the request's first entry)
@@ -387,8 +382,10 @@ __device__ void collect(const Cand &cand, int64_t E, uint64_t prefix, uint64_t m
 // winners, counted by one warp per winner), write the outputs in rank order
 // and, when a.rewire, rewrite the request's beam state in place.  The caller
 // has staged the old rows (stage_rows) and rp / root.
+// dry: the same instructions with every global load and store turned off (a
+// warm-up pass over synthetic shared-memory data)
 __device__ void finish_request(const SelectArgs &a, int r, int n_win, const FinishSmem &f,
-                               bool in_rank_order = false) {
+                               bool in_rank_order, bool dry) {
     const Dims dm = a.dims;
     const int BW = dm.BW, S = dm.S, V = dm.V;
     const int64_t rb = (int64_t)r * BW;
@@ -403,7 +400,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
         const int i = threadIdx.x + u * blockDim.x;
         child_c[u] = -1;
         child_t[u] = -1;
-        if (!a.rewire || a.dense || i >= n_win) continue;
+        if (!a.rewire || a.dense || i >= n_win || dry) continue;
         const uint32_t lo = (uint32_t)f.win_k[i];
         const int p = (int)(lo / (uint32_t)V);
         if (f.cb[p] < 0) continue;
@@ -431,6 +428,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
             f.win_e[i] = (child_c[u] >= 0 && child_t[u] == (int)((uint32_t)f.win_k[i] % (uint32_t)V)) ? child_c[u] : -1;
     }
     __syncthreads();   // every rank is written
+    const bool wr = !dry;   // (predicated stores: a dry pass fetches the same code)
     for (int i = threadIdx.x; i < BW; i += blockDim.x) {
         if (i < n_win) {
             const int nb = f.rank[i];
@@ -439,9 +437,11 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
             const uint32_t lo = (uint32_t)key;
             const int p = (int)(lo / (uint32_t)V), t = (int)(lo % (uint32_t)V);
             const float sc = desc_bits_to_score((uint32_t)(key >> 32));
-            a.parent[o] = p;
-            a.token[o] = t;
-            a.cum_out[o] = sc;
+            if (wr) {
+                a.parent[o] = p;
+                a.token[o] = t;
+                a.cum_out[o] = sc;
+            }
             if (!a.rewire) continue;
             for (int j = 0; j < S; ++j) {
                 int av = -1, sv = -1;
@@ -454,8 +454,10 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
                 } else if (j == s + 1) {
                     av = nb;   // the new beam's token of step s+1 will sit at slot (s+1, nb)
                 }
-                a.st.anc[o * S + j] = av;
-                a.st.seq[o * S + j] = sv;
+                if (wr) {
+                    a.st.anc[o * S + j] = av;
+                    a.st.seq[o * S + j] = sv;
+                }
             }
             // the trie child of the parent's node through token t
             int child = -1;
@@ -466,7 +468,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
                     const int nw = (V + 31) / 32;
                     const uint32_t w = f.root[t >> 5], bit = 1u << (t & 31);
                     if (w & bit) child = (int)f.root[nw + (t >> 5)] + __popc(w & (bit - 1u));
-                } else {
+                } else if (wr) {
                     child = find_child(a.trie, s, node, t);
                 }
             } else {
@@ -474,10 +476,12 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
                 // the entry index located the child (checked above)
                 child = f.win_e[i];
             }
-            if (child < 0) set_status(a.status, XGR_DEV_MASK);
-            a.st.node[o] = child;
-            a.st.cum[o] = sc;
-        } else {
+            if (wr) {
+                if (child < 0) set_status(a.status, XGR_DEV_MASK);
+                a.st.node[o] = child;
+                a.st.cum[o] = sc;
+            }
+        } else if (wr) {
             const int64_t o = rb + i;
             a.parent[o] = -1;
             a.token[o] = -1;
@@ -491,7 +495,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
             a.st.cum[o] = -INFINITY;
         }
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && wr) {
         a.n_out[r] = n_win;
         if (a.rewire) a.st.n_live[r] = n_win;
     }
@@ -499,96 +503,166 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
 
 // ------------------------------------------------------------------ sparse steps
 
-// One launch per sparse step.  Request r gets sp_parts CTAs of kSpThreads
+// Phase 1 (select_rows_kernel): request r gets sp_parts CTAs of kSpThreads
 // threads; CTA `part` takes beams [part*R, part*R + R) (R = sp_rows), one warp
-// per beam at a time, so no reduction spans more than one warp.  Per beam:
+// per beam, so no reduction spans more than one warp.  Per beam:
 //  * logits mode: the row's log-sum-exp over the full vocabulary, streamed
-//    from HBM in 16-byte loads with the next batch in flight while the current
-//    one is folded (online max / sum of exponentials per lane, then across
-//    the warp);
-//  * the key of every CSR entry (its score read back, an L2 hit in logits
-//    mode), written to the request's key buffer;
+//    from HBM through a ring of bulk copies (online max / sum of exponentials
+//    per lane, then across the warp), while the mask lookups and the first
+//    entries' scores are fetched;
+//  * the key of every mask entry, written to the request's key buffer;
 //  * the beam's head: its m best keys with their entries, ascending (the
 //    page's per-beam ordered candidate list, cut at m).
-// Then each CTA takes a ticket; the last of the request's CTAs to arrive
-// selects for the whole request (select_request), so no second launch and no
-// grid-wide wait is needed.
+// Phase 2 (select_pick_kernel) selects for the whole request from the heads.
 constexpr int kSpThreads = 256;
 constexpr int kSpWarps = kSpThreads / 32;
-constexpr int kSpKpc = 8;   // CSR entries per lane in one pass of the key loop
-constexpr int kLseU = 16;   // float4 per lane in one batch of the row stream (8 KB per warp)
+constexpr int kSpKpc = 8;             // CSR entries per lane in one pass of the key loop
+constexpr int kRingStageBytes = 4096;  // one stage of a warp's row stream
+constexpr int kRingStages = 5;         // stages of a warp's ring, all in flight but the one folding
+constexpr int kWtokCap = 1024;         // NODE_BITS tokens listed beside the ring before the stream
+constexpr size_t kRingWarpBytes = (size_t)kRingStages * kRingStageBytes + kWtokCap * 4;   // 24 KB
 
-__device__ __forceinline__ float4 ld_stream4(const float4 *p) {
-    float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p));
-    return v;
+// max that returns NaN when either operand is NaN
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
 }
 
-// natural-log log-sum-exp of x[0..V), by one warp (every lane gets it); a NaN
-// anywhere in the row sets XGR_DEV_NAN
-__device__ float warp_row_lse(const float *x, int V, int32_t *status) {
-    const int lane = threadIdx.x & 31;
-    float m = -INFINITY, s = 0.f;
-    bool nan = false;
-    auto fold = [&](const float *v, int k) {
-        float mv = -INFINITY;
-        for (int e = 0; e < k; ++e) {
-            nan |= v[e] != v[e];
-            mv = fmaxf(mv, v[e]);
-        }
-        if (mv > m) {
-            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
-            m = mv;
-        }
-        if (m != -INFINITY) {
-            const float mk = m * kLog2e;
-            for (int e = 0; e < k; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
-        }
-    };
-    if ((V & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0) {
-        const float4 *x4 = reinterpret_cast<const float4 *>(x);
-        const int n4 = V >> 2;
-        constexpr int kStep = 32 * kLseU;
-        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        float4 cur[kLseU];
+// Folds 32 values into a lane's running (max m, sum s of 2^((v - m) log2 e)):
+// the values' maximum over eight independent chains, s rescaled when the
+// maximum grows, then the exponentials into eight independent partial sums.
+// A NaN value turns s into NaN (reported by the caller through the row's
+// log-sum-exp).
+__device__ __forceinline__ void lse_fold32(const float (&v)[32], float &m, float &s) {
+    float mx[8];
 #pragma unroll
-        for (int u = 0; u < kLseU; ++u) {
-            const int i = u * 32 + lane;
-            cur[u] = i < n4 ? ld_stream4(x4 + i) : ninf;
-        }
-        for (int b0 = 0; b0 < n4; b0 += kStep) {
-            float4 nxt[kLseU];
+    for (int e = 0; e < 8; ++e) mx[e] = v[e];
 #pragma unroll
-            for (int u = 0; u < kLseU; ++u) {   // the next batch is in flight while this one folds
-                const int i = b0 + kStep + u * 32 + lane;
-                nxt[u] = i < n4 ? ld_stream4(x4 + i) : ninf;
-            }
-            float v[4 * kLseU];
-#pragma unroll
-            for (int u = 0; u < kLseU; ++u) {
-                v[4 * u] = cur[u].x;
-                v[4 * u + 1] = cur[u].y;
-                v[4 * u + 2] = cur[u].z;
-                v[4 * u + 3] = cur[u].w;
-            }
-            fold(v, 4 * kLseU);
-#pragma unroll
-            for (int u = 0; u < kLseU; ++u) cur[u] = nxt[u];
-        }
-    } else {
-        for (int i = lane; i < V; i += 32) fold(x + i, 1);
+    for (int e = 8; e < 32; ++e) mx[e & 7] = max_nan(mx[e & 7], v[e]);
+    const float bm = max_nan(max_nan(max_nan(mx[0], mx[1]), max_nan(mx[2], mx[3])),
+                             max_nan(max_nan(mx[4], mx[5]), max_nan(mx[6], mx[7])));
+    if (!(bm <= m)) {   // the maximum grew (or a NaN arrived)
+        s = m == -INFINITY ? 0.f : s * ex2f((m - bm) * kLog2e);
+        m = bm;
     }
-    if (__any_sync(0xffffffffu, nan)) {
-        if (lane == 0) set_status(status, XGR_DEV_NAN);
+    if (m != -INFINITY) {
+        const float mk = m * kLog2e;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = ex2f(fmaf(v[e], kLog2e, -mk));
+#pragma unroll
+        for (int e = 8; e < 32; ++e) acc[e & 7] += ex2f(fmaf(v[e], kLog2e, -mk));
+        s += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     }
+}
+
+__device__ __forceinline__ float warp_lse_merge(float m, float s) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
         lse_pair_merge(m, s, m2, s2);
     }
     return m + logf(s);
+}
+
+// A warp's score-row stream: the row's bytes go through the warp's ring of
+// kRingStages shared-memory stages by bulk copies (the TMA engine), issued
+// by lane 0 and landing on one mbarrier per stage; all stages but the one the
+// lanes fold are in flight.  The same warp issues, waits for and refills each
+// stage in order, so a stage's barrier is never more than one phase ahead of
+// its waiter (parity = use count & 1).  Needs the row 16-byte aligned and a
+// multiple of 16 bytes long.
+struct RowStream {
+    const uint8_t *src;
+    int bytes, nst;
+    float4 *ring;     // the warp's stages
+    uint32_t bar0;    // its kRingStages barriers (8 bytes apart)
+    __device__ void issue(int st) const {   // lane 0
+        if (st >= nst) return;
+        const int slot = st % kRingStages, off = st * kRingStageBytes;
+        const uint32_t n = (uint32_t)min(kRingStageBytes, bytes - off);
+        const uint32_t bar = bar0 + 8u * (uint32_t)slot;
+        mbar_expect_tx(bar, n);
+        bulk_g2s(smem_u32(ring) + (uint32_t)(slot * kRingStageBytes), src + off, n, bar);
+    }
+};
+
+// starts the stream: the first kRingStages stages go out (barriers initialised
+// by lane 0 here, before any lane waits on them)
+__device__ RowStream row_stream_start(const float *x, int V, float4 *ring, uint64_t *bars) {
+    RowStream rs;
+    rs.src = reinterpret_cast<const uint8_t *>(x);
+    rs.bytes = V * 4;
+    rs.nst = (rs.bytes + kRingStageBytes - 1) / kRingStageBytes;
+    rs.ring = ring;
+    rs.bar0 = smem_u32(bars);
+    if ((threadIdx.x & 31) == 0) {
+        for (int i = 0; i < kRingStages; ++i) mbar_init(rs.bar0 + 8u * (uint32_t)i, 1);
+        fence_mbar_init();
+        for (int st = 0; st < min(rs.nst, kRingStages); ++st) rs.issue(st);
+    }
+    __syncwarp();
+    return rs;
+}
+
+// Natural-log log-sum-exp of the streamed row by its warp (every lane gets it;
+// NaN when the row holds a NaN).  Each stage is folded by all lanes, then
+// refilled with the stage kRingStages ahead.  A stage that never lands (a
+// bounded wait runs out) sets XGR_DEV_TIMEOUT; the copies still in flight are
+// waited for (bounded) before the ring is given back.
+__device__ float row_stream_lse(const RowStream &rs, int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    float m = -INFINITY, s = 0.f;
+    int st = 0;
+    for (; st < rs.nst; ++st) {
+        const int slot = st % kRingStages;
+        const uint32_t bar = rs.bar0 + 8u * (uint32_t)slot;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)(st / kRingStages) & 1u, nullptr))) break;
+        const float4 *src = rs.ring + slot * (kRingStageBytes / 16);
+        const int n4 = min(kRingStageBytes, rs.bytes - st * kRingStageBytes) / 16;
+        float v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = u * 32 + lane;
+            const float4 q = i < n4 ? src[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            v[4 * u] = q.x;
+            v[4 * u + 1] = q.y;
+            v[4 * u + 2] = q.z;
+            v[4 * u + 3] = q.w;
+        }
+        lse_fold32(v, m, s);
+        __syncwarp();   // every lane has read the stage
+        if (lane == 0 && st + kRingStages < rs.nst) {
+            fence_async_smem();   // those reads before the bulk copy's writes
+            rs.issue(st + kRingStages);
+        }
+    }
+    if (st < rs.nst) {   // timed out: let the issued copies land before the ring is reused
+        if (lane == 0) {
+            set_status(status, XGR_DEV_TIMEOUT);
+            for (int q = st; q < min(rs.nst, st + kRingStages); ++q)
+                mbar_wait(rs.bar0 + 8u * (uint32_t)(q % kRingStages), (uint32_t)(q / kRingStages) & 1u, nullptr);
+        }
+        __syncwarp();
+    }
+    return warp_lse_merge(m, s);
+}
+
+// the same for rows the ring cannot take (V % 4 != 0 or unaligned): plain loads
+__device__ float warp_row_lse_plain(const float *x, int V) {
+    const int lane = threadIdx.x & 31;
+    float m = -INFINITY, s = 0.f;
+    for (int i0 = 0; i0 < V; i0 += 32 * 32) {
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int i = i0 + e * 32 + lane;
+            v[e] = i < V ? __ldg(x + i) : -INFINITY;
+        }
+        lse_fold32(v, m, s);
+    }
+    return warp_lse_merge(m, s);
 }
 
 // Merges the keys c[] of every lane (entries ce[]) into the warp's running
@@ -630,54 +704,11 @@ __device__ __forceinline__ void warp_head_merge(uint64_t (&c)[KPC], const int (&
     run_e = nrun_e;
 }
 
-// the same over a row staged in shared memory (16-byte aligned, V % 4 == 0)
-__device__ float warp_row_lse_smem(const float *x, int V, int32_t *status) {
-    const int lane = threadIdx.x & 31;
-    const float4 *x4 = reinterpret_cast<const float4 *>(x);
-    const int n4 = V >> 2;
-    float m = -INFINITY, s = 0.f;
-    bool nan = false;
-    for (int b0 = 0; b0 < n4; b0 += 32 * 4) {   // 16 values per lane per pass
-        float v[16];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = b0 + u * 32 + lane;
-            const float4 q = i < n4 ? x4[i] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-            v[4 * u] = q.x;
-            v[4 * u + 1] = q.y;
-            v[4 * u + 2] = q.z;
-            v[4 * u + 3] = q.w;
-        }
-        float mv = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            nan |= v[e] != v[e];
-            mv = fmaxf(mv, v[e]);
-        }
-        if (mv > m) {
-            s = m == -INFINITY ? 0.f : s * ex2f((m - mv) * kLog2e);
-            m = mv;
-        }
-        if (m != -INFINITY) {
-            const float mk = m * kLog2e;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) s += ex2f(fmaf(v[e], kLog2e, -mk));
-        }
-    }
-    if (__any_sync(0xffffffffu, nan)) {
-        if (lane == 0) set_status(status, XGR_DEV_NAN);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_pair_merge(m, s, m2, s2);
-    }
-    return m + logf(s);
-}
-
 // The valid tokens of a NODE_BITS row, compacted into wtok[0..) in token
 // order (the node's children in trie order) by one warp; returns their count.
-__device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int cap) {
+// first: the first pass's words, when the caller loaded them already.
+__device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int cap,
+                                   const uint32_t *first = nullptr) {
     const int lane = threadIdx.x & 31;
     int cnt = 0;
     for (int w0 = 0; w0 < nw; w0 += 32 * 8) {
@@ -685,7 +716,7 @@ __device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int ca
 #pragma unroll
         for (int u = 0; u < 8; ++u) {   // up to 256 words in flight per pass
             const int w = w0 + u * 32 + lane;
-            wv[u] = w < nw ? __ldg(wb + w) : 0u;
+            wv[u] = (w0 == 0 && first) ? first[u] : w < nw ? __ldg(wb + w) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -717,51 +748,109 @@ __device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int ca
 // candidates, its entry count and the first trie child of its node.  The
 // row's tokens come from the CSR rows, from its node's children in the trie
 // level (TRIE_ROWS), or from its node's pre-generated bitset (NODE_BITS,
-// compacted into wtok).
-__device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int base, uint64_t *keys,
-                           int *wtok, const float *xs) {
+// listed in the warp's token area).
+//
+// row_prep runs before the kernel waits for the kernel before it: it reads
+// only the beam state, which the previous selection wrote (that kernel had
+// completed before the one before this kernel started), and the mask tables.
+// row_run follows the wait: in logits mode the row streams through the warp's
+// ring for its log-sum-exp while the first pass's scores are fetched.  area:
+// the warp's kRingWarpBytes of shared memory (16-byte aligned); bars: its
+// kRingStages mbarriers.
+struct RowPrep {
+    bool live;
+    float cum;
+    int node, n_e, cb, nb_full;
+    int64_t ebase;
+    const int32_t *tokp;
+    int tk0[kSpKpc];   // the first pass's tokens (lane j: entries j, j + 32, ...)
+};
+
+__device__ RowPrep row_prep(const SelectArgs &a, int r, int b, int n_live, int base, uint8_t *area) {
     const int lane = threadIdx.x & 31;
     const Dims dm = a.dims;
-    const int V = dm.V, m = a.head_m, s = a.step;
+    const int s = a.step;
     const int64_t row = (int64_t)r * dm.BW + b;
-    const bool live = b < n_live;
-    const float cum = a.cum[row];
-    const float *x = a.scores + row * V;
-    // the first loads of the row's tokens go out before the row stream; the
-    // rest (its tokens, the node's first child) follow its log-sum-exp
+    int *wtok = reinterpret_cast<int *>(area + (size_t)kRingStages * kRingStageBytes);
+    RowPrep p;
+    p.live = b < n_live;
+    p.cum = a.cum[row];
     const bool csr = a.mask_kind == XGR_MASK_CSR;
     const int beg = csr ? a.row_ptr[row] : 0, end = csr ? a.row_ptr[row + 1] : 0;
-    const int node = (csr ? (a.rewire && live) : live) ? (csr ? a.st.node[row] : a.row_node[row]) : -1;
-    float lse = 0.f;
-    if (a.logits && live) lse = xs ? warp_row_lse_smem(xs, V, a.status) : warp_row_lse(x, V, a.status);
-    // the row's tokens (tokp[0..n_e)), their entry base and the node's first child
-    const int32_t *tokp = nullptr;
-    int n_e = 0, cb = -1;
-    int64_t ebase;
+    p.node = (csr ? (a.rewire && p.live) : p.live) ? (csr ? a.st.node[row] : a.row_node[row]) : -1;
+    p.tokp = nullptr;
+    p.n_e = 0;
+    p.cb = -1;
+    p.nb_full = 0;
     if (csr) {
-        tokp = a.cols + beg;
-        n_e = max(0, end - beg);
-        ebase = beg - base;
-        if (s < a.trie.levels && node >= 0 && node < a.trie.n_nodes[s]) cb = a.trie.ptr[s][node];
+        p.tokp = a.cols + beg;
+        p.n_e = max(0, end - beg);
+        p.ebase = beg - base;
+        if (s < a.trie.levels && p.node >= 0 && p.node < a.trie.n_nodes[s]) p.cb = a.trie.ptr[s][p.node];
     } else {
-        ebase = (int64_t)b * a.row_stride;
-        if (node >= 0 && node < a.n_nodes) {
-            const int lo = a.node_ptr[node], hi = a.node_ptr[node + 1];
-            cb = lo;
-            n_e = min(max(0, hi - lo), a.row_stride);
+        p.ebase = (int64_t)b * a.row_stride;
+        if (p.node >= 0 && p.node < a.n_nodes) {
+            const uint32_t *wb = a.node_bits + (int64_t)p.node * a.n_words;
+            uint32_t first[8];   // the bitset's first words load beside the child range
+            if (a.mask_kind == XGR_MASK_NODE_BITS)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int w = u * 32 + lane;
+                    first[u] = w < a.n_words ? __ldg(wb + w) : 0u;
+                }
+            const int lo = a.node_ptr[p.node], hi = a.node_ptr[p.node + 1];
+            p.cb = lo;
+            p.n_e = min(max(0, hi - lo), a.row_stride);
             if (a.mask_kind == XGR_MASK_TRIE_ROWS) {
-                tokp = a.node_tok + lo;
+                p.tokp = a.node_tok + lo;
             } else {
-                const int nb = warp_bits_to_tokens(a.node_bits + (int64_t)node * a.n_words, a.n_words, wtok,
-                                                   a.row_stride);
-                if (nb != hi - lo && lane == 0) set_status(a.status, XGR_DEV_MASK);   // table and trie disagree
-                n_e = min(nb, a.row_stride);
-                tokp = wtok;
+                p.nb_full = warp_bits_to_tokens(wb, a.n_words, wtok, kWtokCap, first);
+                if (p.nb_full != hi - lo && lane == 0) set_status(a.status, XGR_DEV_MASK);   // table and trie disagree
+                p.n_e = min(p.nb_full, a.row_stride);
+                p.tokp = wtok;
             }
-        } else if (live && lane == 0) {
+        } else if (p.live && lane == 0) {
             set_status(a.status, XGR_DEV_INDEX);
         }
     }
+#pragma unroll
+    for (int u = 0; u < kSpKpc; ++u) {
+        const int j = u * 32 + lane;
+        p.tk0[u] = (j < p.n_e && p.live) ? p.tokp[j] : -1;
+    }
+    return p;
+}
+
+__device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uint64_t *keys, uint8_t *area,
+                        uint64_t *bars) {
+    const int lane = threadIdx.x & 31;
+    const Dims dm = a.dims;
+    const int V = dm.V, m = a.head_m;
+    const int64_t row = (int64_t)r * dm.BW + b;
+    const bool live = p.live;
+    const float *x = a.scores + row * V;
+    float4 *ring = reinterpret_cast<float4 *>(area);
+    const bool stream = a.logits && live && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+    RowStream rs{};
+    if (stream) rs = row_stream_start(x, V, ring, bars);
+    // the first pass's scores go out before the stream is folded
+    float sv0[kSpKpc];
+#pragma unroll
+    for (int u = 0; u < kSpKpc; ++u) sv0[u] = (p.tk0[u] >= 0 && p.tk0[u] < V) ? __ldg(x + p.tk0[u]) : 0.f;
+    float lse = 0.f;
+    if (a.logits && live) {
+        lse = stream ? row_stream_lse(rs, a.status) : warp_row_lse_plain(x, V);
+        if (lse != lse && lane == 0) set_status(a.status, XGR_DEV_NAN);
+    }
+    const int32_t *tokp = p.tokp;
+    if (p.nb_full > kWtokCap) {
+        // a node with more children than the token area holds: list them all in
+        // the ring, which the stream has given back
+        int *wtok = reinterpret_cast<int *>(area);
+        warp_bits_to_tokens(a.node_bits + (int64_t)p.node * a.n_words, a.n_words, wtok, a.row_stride);
+        tokp = wtok;
+    }
+    const int n_e = p.n_e;
     uint64_t run = kNoKey;   // lane i < m: the i-th best key of the row so far
     int run_e = -1;
     int n_valid = 0;
@@ -769,22 +858,30 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
         uint64_t c[kSpKpc];
         int ce[kSpKpc];
         int tk[kSpKpc];
-#pragma unroll
-        for (int u = 0; u < kSpKpc; ++u) {   // the entries' tokens (one round trip) ...
-            const int j = j0 + u * 32 + lane;
-            tk[u] = (j < n_e && live) ? tokp[j] : -1;
-        }
         float sv[kSpKpc];
+        if (j0 == 0) {
 #pragma unroll
-        for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (staged, or another)
-            sv[u] = (tk[u] >= 0 && tk[u] < V) ? (xs ? xs[tk[u]] : __ldg(x + tk[u])) : 0.f;
+            for (int u = 0; u < kSpKpc; ++u) {
+                tk[u] = p.tk0[u];
+                sv[u] = sv0[u];
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < kSpKpc; ++u) {   // the entries' tokens (one round trip) ...
+                const int j = j0 + u * 32 + lane;
+                tk[u] = (j < n_e && live) ? tokp[j] : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (another)
+                sv[u] = (tk[u] >= 0 && tk[u] < V) ? __ldg(x + tk[u]) : 0.f;
+        }
 #pragma unroll
         for (int u = 0; u < kSpKpc; ++u) {
             const int j = j0 + u * 32 + lane;
             c[u] = kNoKey;
             ce[u] = -1;
             if (j >= n_e) continue;
-            const int64_t e = ebase + j;   // the entry, relative to the request
+            const int64_t e = p.ebase + j;   // the entry, relative to the request
             uint64_t key = kNoKey;
             if (live) {
                 if (tk[u] < 0 || tk[u] >= V) {
@@ -792,7 +889,7 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
                 } else {
                     const float lp = a.logits ? sv[u] - lse : sv[u];
                     uint64_t k2;
-                    if (make_key(cum, lp, b, tk[u], V, a.status, k2)) key = k2;
+                    if (make_key(p.cum, lp, b, tk[u], V, a.status, k2)) key = k2;
                 }
             }
             if (e >= 0 && e < a.key_cap) keys[e] = key;
@@ -811,7 +908,7 @@ __device__ void sparse_row(const SelectArgs &a, int r, int b, int n_live, int ba
         a.row_cnt[row] = n_valid;
         a.row_lse[row] = lse;
         a.row_len[row] = n_e;
-        a.row_cb[row] = cb;
+        a.row_cb[row] = p.cb;
     }
 }
 
@@ -898,6 +995,149 @@ __device__ uint64_t selected_max(const uint64_t *k, int n, uint64_t prefix, uint
     return block_max_u64(t, red);
 }
 
+// ---- the threshold cut
+//
+// The survivors of a cut are the candidates that can still be among the
+// `want` best.  A binned cut maps every key's score word (key >> 32, which
+// orders like the key) onto kCutBins linear bins between the smallest and
+// largest score word of a reference set of real candidates (the beams' heads,
+// or the threads' best keys), and finds the smallest bin B* such that at
+// least `want` reference keys lie in bins <= B*.  The mapping is monotone in
+// the key, so the `want` best reference keys -- and with them the `want` best
+// candidates overall -- all lie in bins <= B*: "bin <= B*" keeps every winner,
+// and needs one histogram pass instead of a radix select.  When every
+// reference key has the same score word the cut falls back to the exact
+// BW-th best reference key (tau); with fewer than `want` reference keys
+// everything survives.
+constexpr int kCutBins = 2048;
+struct Cut {
+    int mode;        // 0: everything survives; 1: binned; 2: key <= tau
+    uint32_t lo;     // binned: the smallest score word
+    float scale;     // binned: bins per score-word unit
+    int bstar;       // binned: the last surviving bin
+    uint64_t tau;    // mode 2
+    __device__ __forceinline__ int bin(uint64_t key) const {
+        const uint32_t d = (uint32_t)(key >> 32) - lo;
+        return min(kCutBins - 1, (int)((float)d * scale));
+    }
+    __device__ __forceinline__ bool keep(uint64_t key) const {
+        if (key == kNoKey) return false;
+        return mode == 0 ? true : mode == 1 ? bin(key) <= bstar : key <= tau;
+    }
+};
+
+// the request's key buffer, restricted to the survivors of the cut; with a
+// row stride (node masks) only the first rl[b] slots of row b hold keys
+struct KeyCand {
+    const uint64_t *k;
+    Cut cut;
+    const int *rp, *rl;   // shared memory
+    int stride, n;        // stride 0: CSR numbering (every entry written)
+    __device__ bool operator()(int64_t e, uint64_t &key) const {
+        if (stride) {
+            const int b = (int)(e / stride), j = (int)(e % stride);
+            if (b >= n || j >= rl[b]) return false;
+        }
+        key = __ldcg(k + e);
+        return cut.keep(key);
+    }
+};
+
+// The cut over the reference keys k[0..n) (kNoKey entries are not keys), by
+// the whole block (blockDim a multiple of 32, kCutBins a multiple of it).
+// hist: kCutBins ints; red32: 64 words; scan_w: 32 ints; sc: 4 ints; red_k: 32
+// u64 (exact fallback).
+__device__ Cut make_cut(const uint64_t *k, int n, int want, int *hist, uint32_t *red32, int *scan_w, int *sc,
+                        uint64_t *red_k) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    Cut c{0, 0, 0.f, 0, kNoKey};
+    for (int i = tid; i < kCutBins; i += nt) hist[i] = 0;
+    uint32_t lo = ~0u, hi = 0;
+    int cnt = 0;
+    for (int i = tid; i < n; i += nt) {
+        const uint64_t key = k[i];
+        if (key == kNoKey) continue;
+        const uint32_t w = (uint32_t)(key >> 32);
+        lo = min(lo, w);
+        hi = max(hi, w);
+        ++cnt;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    }
+    if (lane == 0) {
+        red32[warp] = lo;
+        red32[32 + warp] = hi;
+        scan_w[warp] = cnt;
+    }
+    __syncthreads();
+    lo = ~0u;
+    hi = 0;
+    cnt = 0;
+    for (int w = 0; w < nw; ++w) {
+        lo = min(lo, red32[w]);
+        hi = max(hi, red32[32 + w]);
+        cnt += scan_w[w];
+    }
+    __syncthreads();   // red32 / scan_w are read before anyone reuses them
+    if (cnt < want || want <= 0) return c;   // everything survives
+    if (lo == hi) {   // one score word: the exact BW-th best key
+        uint64_t tp, tm;
+        smem_radix_select(k, n, want, hist, scan_w, red_k, sc, tp, tm);
+        c.mode = 2;
+        c.tau = selected_max(k, n, tp, tm, red_k);
+        return c;
+    }
+    c.mode = 1;
+    c.lo = lo;
+    c.scale = (float)kCutBins / ((float)(hi - lo) + 1.f);
+    for (int i = tid; i < n; i += nt) {
+        const uint64_t key = k[i];
+        if (key != kNoKey) atomicAdd(&hist[c.bin(key)], 1);
+    }
+    __syncthreads();
+    // the bin where the running count reaches `want`: each thread scans its
+    // kCutBins / nt consecutive bins
+    const int bpt = kCutBins / nt;
+    int sum = 0;
+    for (int j = 0; j < bpt; ++j) sum += hist[tid * bpt + j];
+    int total;
+    int acc = block_exclusive_scan_int(sum, scan_w, &total);
+    if (acc < want && acc + sum >= want) {
+        for (int j = 0; j < bpt; ++j) {
+            acc += hist[tid * bpt + j];
+            if (acc >= want) {
+                sc[0] = tid * bpt + j;
+                break;
+            }
+        }
+    }
+    __syncthreads();
+    c.bstar = sc[0];
+    __syncthreads();   // sc is read before anyone reuses it
+    return c;
+}
+
+// Global -> shared copy of `bytes` (a multiple of 4) through L2 only (the
+// source may have been written by other CTAs of this launch): 16-byte
+// cp.async copies when both ends are 16-byte aligned, else 4-byte loads.  The
+// caller waits (cp_async_wait_all, then a barrier).
+__device__ void stage_l2(void *dst, const void *src, int bytes) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    int i4 = 0;
+    if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) & 15) == 0) {
+        const int n16 = bytes >> 4;
+        for (int i = tid; i < n16; i += nt)
+            cp_async16(smem_u32(static_cast<uint8_t *>(dst) + 16 * i), static_cast<const uint8_t *>(src) + 16 * i);
+        i4 = n16 * 4;
+    }
+    for (int i = i4 + tid; i < (bytes >> 2); i += nt)
+        static_cast<int *>(dst)[i] = __ldcg(static_cast<const int *>(src) + i);
+}
+
 // The `want` best of the survivors sk[0..ns) (unique keys, ns >= want), placed
 // in rank order: a survivor's rank is its number of better survivors (every
 // thread counts for its own survivors over the whole list -- broadcast reads,
@@ -918,29 +1158,32 @@ __device__ void place_by_rank(const uint64_t *sk, const int *se, int ns, int wan
 __host__ __device__ inline int sparse_cand_cap(int BW, int m) { return BW * m; }
 __host__ __device__ inline int sparse_surv_cap(int BW) { return BW >= 1024 ? 4096 : (BW >= 256 ? 4 * BW : 1024); }
 
-size_t sparse_smem(const Dims &dm, int m, int node_bits_stride, int slots) {
+size_t sparse_pick_smem(const Dims &dm, int m) {
     const int cc = sparse_cand_cap(dm.BW, m), scap = sparse_surv_cap(dm.BW);
-    const size_t pick = al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) +
-                        al16((size_t)scap * 4) + al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) +
-                        finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
-    // phase 1: the staged rows, then the per-warp token lists
-    const size_t rows = slots * al16((size_t)dm.V * 4) + (size_t)kSpWarps * node_bits_stride * 4;
-    return pick > rows ? pick : rows;
+    return al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) + al16((size_t)scap * 4) +
+           al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) + finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
 }
+// phase 1: one ring per warp (the row stream and the NODE_BITS token list)
+constexpr size_t kRowsSmem = (size_t)kSpWarps * kRingWarpBytes;
 
-// Phase 2, by the request's last CTA.  tau = the BW-th best of the beams'
-// heads: at least BW real candidates rank at or above it, so every winner
-// does.  Survivors = the head keys at or above tau, plus, for a beam whose
-// whole head survived and that has more entries than its head holds, its
-// further keys at or above tau from the key buffer.  Then the exact radix
-// select of the BW best survivors, the ordering, the outputs and the
-// rewiring.  Exact fallbacks: survivors beyond the shared-memory buffer select
-// from the key buffer; a request with more CSR entries than the key buffer
-// holds selects from the scores.
-__device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *hist, int *scan_w,
-                               uint64_t *red_k, int *sc, int *red_i) {
+// Phase 2, by the request's last CTA.  The cut comes from the beams' heads
+// (every head key is a real candidate, so at least BW real candidates lie at
+// or before it and every winner survives).  Survivors = the head keys that
+// the cut keeps, plus, for a beam whose whole head survived and that has more
+// entries than its head holds, its further keys that the cut keeps (from the
+// key buffer, one warp per such beam).  The survivors are ranked by counting
+// (or radix-selected when there are many), then finish_request writes the
+// outputs and the rewiring.  Exact fallbacks: survivors beyond the
+// shared-memory buffer select from the key buffer; a request with more CSR
+// entries than the key buffer holds selects from the scores.
+// dry: a warm-up pass -- a synthetic request in shared memory (BW x m
+// distinct head keys, no beam saturated, no trie) through the same code, with
+// no global memory access.
+__device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n, uint8_t *smem, int *hist,
+                                               int *scan_w, uint64_t *red_k, int *sc, int *red_i, uint32_t *red32,
+                                               bool dry) {
     const Dims dm = a.dims;
-    const int BW = dm.BW, m = a.head_m, tid = threadIdx.x;
+    const int BW = dm.BW, m = a.head_m, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t rb = (int64_t)r * BW;
     const int cc = sparse_cand_cap(BW, m), scap = sparse_surv_cap(BW);
     uint8_t *p = smem;
@@ -961,40 +1204,70 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
     const FinishSmem f = carve_finish(p, BW, BW, dm.S, 0);
     int *cnts = reinterpret_cast<int *>(p + finish_bytes(BW, BW, dm.S, 0));   // [0] survivors, [1] saturated
 
-    // every load below is independent of the others: one round trip.  Entry
-    // numbering of the key buffer: CSR rows as in the mask; node masks row b
-    // at b * row_stride.
-    const bool csr = a.mask_kind == XGR_MASK_CSR;
-    const int n = min(max(a.n_live[r], 0), BW);
-    const int base = csr ? a.row_ptr[rb] : 0;
-    const int64_t E = csr ? (int64_t)a.row_ptr[rb + BW] - base : (int64_t)BW * a.row_stride;
-    for (int i = tid; i < BW * m; i += kSpThreads) {
-        const int b = i / m;
-        hk[i] = b < n ? __ldcg(a.head_k + rb * m + i) : kNoKey;
-        he[i] = __ldcg(a.head_e + rb * m + i);
-    }
-    int c = 0;
-    for (int b = tid; b < BW; b += kSpThreads) {
-        c += b < n ? __ldcg(a.row_cnt + rb + b) : 0;
-        const int len = b < n ? __ldcg(a.row_len + rb + b) : 0, cb = __ldcg(a.row_cb + rb + b);
-        f.rl[b] = len;
-        f.cb[b] = b < n ? cb : -1;
-        f.ce[b] = (b < n && cb >= 0) ? cb + len : -1;
-    }
-    for (int b = tid; b <= BW; b += kSpThreads)
-        f.rp[b] = csr ? a.row_ptr[rb + b] - base : b * a.row_stride;
-    if (a.rewire) stage_rows(a, rb, n, f);
-    if (E > a.key_cap)
-        for (int b = tid; b < n; b += kSpThreads) {
-            cum_s[b] = a.cum[rb + b];
-            lse_s[b] = a.logits ? __ldcg(a.row_lse + rb + b) : 0.f;
+    // Everything this CTA reads from phase 1 and the beam state, in one round
+    // trip: the heads, each beam's entry count and first trie child, the CSR
+    // row offsets and the old beam rows (rewiring) stream into shared memory
+    // by cp.async while each thread loads its beams' candidate counts.  (n,
+    // the live beams, is the count phase 1 read: dead beams' heads hold no
+    // keys.)
+    const bool csr = a.mask_kind == XGR_MASK_CSR && !dry;
+    const int mshift = __ffs(m) - 1;   // m is a power of two
+    int base = 0, c = 0;
+    int64_t E = (int64_t)BW * (dry ? m : a.row_stride);
+    if (dry) {
+        n = BW;
+        for (int i = tid; i < BW * m; i += kSpThreads) {
+            const uint32_t h = 0xC1000000u + (((uint32_t)i * 2654435761u) >> 10);
+            hk[i] = ((uint64_t)h << 32) | (uint32_t)((i >> mshift) * dm.V + (i & (m - 1)) % dm.V);
+            he[i] = i;
         }
+        for (int b = tid; b < BW; b += kSpThreads) {
+            f.rl[b] = m;
+            f.cb[b] = -1;
+            f.rp[b] = b * m;
+        }
+        if (tid == 0) f.rp[BW] = BW * m;
+        c = tid == 0 ? BW * m : 0;
+    } else {
+        stage_l2(hk, a.head_k + rb * m, BW * m * 8);
+        stage_l2(he, a.head_e + rb * m, BW * m * 4);
+        stage_l2(f.rl, a.row_len + rb, BW * 4);
+        stage_l2(f.cb, a.row_cb + rb, BW * 4);
+        if (csr) stage_l2(f.rp, a.row_ptr + rb, (BW + 1) * 4);
+        if (a.rewire) {
+            stage_l2(f.st_anc, a.st.anc + rb * dm.S, BW * dm.S * 4);
+            stage_l2(f.st_seq, a.st.seq + rb * dm.S, BW * dm.S * 4);
+            stage_l2(f.st_node, a.st.node + rb, BW * 4);
+        }
+        if (csr) {
+            base = a.row_ptr[rb];
+            E = (int64_t)a.row_ptr[rb + BW] - base;
+        }
+        for (int b = tid; b < n; b += kSpThreads) c += __ldcg(a.row_cnt + rb + b);
+    }
     if (tid == 0) {
         *f.cnt = 0;
         cnts[0] = 0;
         cnts[1] = 0;
     }
-    const int total = block_sum_int(c, red_i);   // valid candidates of the request (+ a barrier)
+    cp_async_wait_all();
+    const int total = block_sum_int(c, red_i);   // valid candidates of the request (+ barriers)
+    // per beam: entries relative to the request, the trie child range
+    for (int b = tid; b < BW; b += kSpThreads) {
+        const bool lv = b < n;
+        const int len = lv ? f.rl[b] : 0, cb = lv ? f.cb[b] : -1;
+        f.rl[b] = len;
+        f.cb[b] = cb;
+        f.ce[b] = cb >= 0 ? cb + len : -1;
+        if (!dry) f.rp[b] = csr ? f.rp[b] - base : b * a.row_stride;
+    }
+    if (tid == 0 && !dry) f.rp[BW] = csr ? f.rp[BW] - base : BW * a.row_stride;
+    if (csr && E > a.key_cap)
+        for (int b = tid; b < n; b += kSpThreads) {
+            cum_s[b] = a.cum[rb + b];
+            lse_s[b] = a.logits ? __ldcg(a.row_lse + rb + b) : 0.f;
+        }
+    __syncthreads();
     const int want = min(BW, total);
     uint64_t prefix = ~0ull, mask = 0;
     bool ranked = false;   // the winners were placed in rank order
@@ -1015,40 +1288,44 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
         if (want > 0 && want < total) radix_select(cand, f.rp[n], want, hist, sc, prefix, mask);
         collect(cand, f.rp[n], prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
     } else if (want > 0) {
-        // tau from the heads (every head key is a real candidate)
-        int c0 = 0;
-        for (int i = tid; i < BW * m; i += kSpThreads) c0 += hk[i] != kNoKey;
-        const int in_heads = block_sum_int(c0, red_i);
-        uint64_t tau = kNoKey;
-        if (total > BW && in_heads >= BW) {
-            uint64_t tp, tm;
-            smem_radix_select(hk, BW * m, BW, hist, scan_w, red_k, sc, tp, tm);
-            tau = selected_max(hk, BW * m, tp, tm, red_k);
-        }
-        // survivors from the heads; beams whose whole head survived and that have
-        // more entries go on the saturated list
-        for (int i = tid; i < BW * m; i += kSpThreads) {
-            const uint64_t key = hk[i];
-            if (key == kNoKey || key > tau) continue;
-            const int pos = atomicAdd(&cnts[0], 1);
+        const Cut cut = total > BW ? make_cut(hk, BW * m, BW, hist, red32, scan_w, sc, red_k) : Cut{0, 0, 0.f, 0, kNoKey};
+        // survivors from the heads (one shared-memory atomic per warp); beams
+        // whose whole head survived and that have more entries go on the
+        // saturated list
+        const unsigned lt = (1u << lane) - 1u;
+        for (int i0 = 0; i0 < BW * m; i0 += kSpThreads) {
+            const int i = i0 + tid;
+            const uint64_t key = i < BW * m ? hk[i] : kNoKey;
+            const bool keep = cut.keep(key);
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            int pos0 = 0;
+            if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            if (!keep) continue;
+            const int pos = pos0 + __popc(bal & lt);
             if (pos < scap) {
                 sk[pos] = key;
                 se[pos] = he[i];
             }
-            const int b = i / m;
-            if (i % m == m - 1 && f.rl[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
+            const int b = i >> mshift;
+            if ((i & (m - 1)) == m - 1 && f.rl[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
         }
         __syncthreads();
         const int n_sat = cnts[1];
-        for (int q = 0; q < n_sat; ++q) {   // their keys beyond the head (worse than its last)
+        for (int q = warp; q < n_sat; q += kSpWarps) {   // their keys beyond the head (worse than its last)
             const int b = sat[q];
             const uint64_t last = hk[b * m + m - 1];
-            const int e1 = (int)min((int64_t)f.rp[b] + f.rl[b], E);
-            for (int e = max(f.rp[b], 0) + tid; e < e1; e += kSpThreads) {
-                const uint64_t key = __ldcg(keys + e);
-                if (key == kNoKey || key > tau || key <= last) continue;
-                const int pos = atomicAdd(&cnts[0], 1);
-                if (pos < scap) {
+            const int e0 = max(f.rp[b], 0), e1 = (int)min((int64_t)f.rp[b] + f.rl[b], E);
+            for (int j0 = e0; j0 < e1; j0 += 32) {
+                const int e = j0 + lane;
+                const uint64_t key = e < e1 ? __ldcg(keys + e) : kNoKey;
+                const bool keep = key > last && cut.keep(key);
+                const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                int pos0 = 0;
+                if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
+                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                const int pos = pos0 + __popc(bal & lt);
+                if (keep && pos < scap) {
                     sk[pos] = key;
                     se[pos] = e;
                 }
@@ -1063,74 +1340,74 @@ __device__ void select_request(const SelectArgs &a, int r, uint8_t *smem, int *h
             if (want < ns) smem_radix_select(sk, ns, want, hist, scan_w, red_k, sc, prefix, mask);
             collect(ListCand<false>{sk}, ns, prefix, mask, BW, [&](int64_t i) { return se[i]; }, f);
         } else {   // more survivors than the buffer: exact selection over the key buffer
-            const KeyCand cand{keys, tau, f.rp, f.rl, csr ? 0 : a.row_stride, n};
+            const KeyCand cand{keys, cut, f.rp, f.rl, csr ? 0 : a.row_stride, n};
             radix_select(cand, E, want, hist, sc, prefix, mask);
             collect(cand, E, prefix, mask, BW, [](int64_t e) { return (int)e; }, f);
         }
     }
     __syncthreads();
-    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked);
+    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked, dry);
 }
 
-__global__ void __launch_bounds__(kSpThreads) select_sparse_kernel(SelectArgs a) {
+// Phase 1: sp_parts CTAs per request of sp_rows beams, one warp per beam.
+__global__ void __launch_bounds__(kSpThreads, 1) select_rows_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t full_bar[kSpWarps];
-    __shared__ int hist[kRadixBins];
-    __shared__ int scan_w[32];
-    __shared__ int red_i[32];
-    __shared__ uint64_t red_k[32];
-    __shared__ int sc[4];
-    __shared__ int last;
+    __shared__ uint64_t ring_bar[kSpWarps][kRingStages];
     const Dims dm = a.dims;
     const int C = a.sp_parts, R = a.sp_rows;
     const int r = blockIdx.x / C, part = blockIdx.x % C;
     const int warp = threadIdx.x / 32;
     const int64_t rb = (int64_t)r * dm.BW;
-    const int n_live = min(max(a.n_live[r], 0), dm.BW);
-    const int base = a.mask_kind == XGR_MASK_CSR ? a.row_ptr[rb] : 0;
-    uint64_t *keys = a.keys + (int64_t)r * a.key_cap;
-    const int b0 = part * R, b1 = min(dm.BW, part * R + R);
-    // short logits rows (every warp's fits beside the others') are staged by
-    // the TMA engine, one slot and one landing barrier per warp; longer ones
-    // stream through registers
-    const int ns = a.sp_slots;   // 0 or R
-    const size_t xb = al16((size_t)dm.V * 4);
-    float *xslot = reinterpret_cast<float *>(smem);
-    int *wtok = reinterpret_cast<int *>(smem + ns * xb) + (size_t)warp * a.row_stride;   // NODE_BITS rows
-    if (ns > 0) {
-        if (threadIdx.x == 0) {
-            for (int w = 0; w < ns; ++w) mbar_init(smem_u32(&full_bar[w]), 1);
-            fence_mbar_init();
-            for (int w = 0; w < min(ns, b1 - b0); ++w) {
-                if (b0 + w >= n_live) continue;   // dead rows are not read
-                mbar_expect_tx(smem_u32(&full_bar[w]), (uint32_t)dm.V * 4u);
-                bulk_g2s(smem_u32(xslot + (size_t)w * (xb / 4)), a.scores + (rb + b0 + w) * dm.V,
-                         (uint32_t)dm.V * 4u, smem_u32(&full_bar[w]));
-            }
+    const int b = part * R + warp;
+    const bool has_row = warp < R && b < dm.BW;
+    uint8_t *area = smem + (size_t)warp * kRingWarpBytes;
+    // the mask lookups (beam state and tables only) go before the wait when
+    // the kernel before writes no beam state (the scores always follow it)
+    RowPrep p;
+    auto prep = [&]() {
+        const int n_live = min(max(a.n_live[r], 0), dm.BW);
+        const int base = a.mask_kind == XGR_MASK_CSR ? a.row_ptr[rb] : 0;
+        if (has_row) p = row_prep(a, r, b, n_live, base, area);
+    };
+    // The pick kernel (the only kernel launched after this one) may start at
+    // once: before its own wait it touches no global memory, so this kernel
+    // lets it in before its own wait, and the pick's warm-up overlaps phase 1.
+    griddep_launch_dependents();
+    if (a.prep_early) prep();
+    griddep_wait();
+    if (!a.prep_early) prep();
+    if (has_row) row_run(a, r, b, p, a.keys + (int64_t)r * a.key_cap, area, ring_bar[warp]);
+}
+
+// Phase 2: one CTA per request.  It starts while the rows kernel runs (on the
+// SMs that kernel leaves free) and first takes a dry pass of the whole pick
+// over synthetic shared-memory data: the pick's code runs once per launch on
+// whichever SM holds the CTA, and fetching it cold costs more than the pick
+// itself, so the dry pass hides that behind phase 1.  Then it waits for the
+// rows kernel and selects for real.
+__global__ void __launch_bounds__(kSpThreads, 1) select_pick_kernel(const __grid_constant__ SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int hist[kRadixBins];
+    __shared__ int scan_w[32];
+    __shared__ int red_i[32];
+    __shared__ uint32_t red32[64];
+    __shared__ uint64_t red_k[32];
+    __shared__ int sc[4];
+    const int r = blockIdx.x;
+    // Two passes through one inlined copy of the pick (a rolled loop, so the
+    // dry pass fetches the very instructions the real one runs): the dry pass
+    // before the wait, then the real one.
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        int n_live = 0;
+        if (pass == 1) {
+            griddep_wait();   // phase 1 of every request has completed
+            griddep_launch_dependents();
+            n_live = min(max(a.n_live[r], 0), a.dims.BW);
         }
-        __syncthreads();
+        select_request(a, r, n_live, smem, hist, scan_w, red_k, sc, red_i, red32, pass == 0);
+        __syncthreads();   // the pass's shared memory is free again
     }
-    const int b = b0 + warp;
-    if (b < b1) {
-        const float *xs = nullptr;
-        if (ns > 0 && b < n_live) {
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[warp]), 0, nullptr))) {
-                if ((threadIdx.x & 31) == 0) set_status(a.status, XGR_DEV_TIMEOUT);
-            } else {
-                xs = xslot + (size_t)warp * (xb / 4);
-            }
-        }
-        sparse_row(a, r, b, n_live, base, keys, wtok, xs);
-    }
-    // the request's last CTA to arrive selects
-    __threadfence();   // this thread's keys and head are visible before the ticket
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(&a.ticket[r], 1u) == (unsigned)(C - 1);
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    select_request(a, r, smem, hist, scan_w, red_k, sc, red_i);
-    if (threadIdx.x == 0) a.ticket[r] = 0;   // zero again for the next call
 }
 
 // ------------------------------------------------------------------ dense step
@@ -1154,16 +1431,26 @@ size_t dense_smem(const Dims &dm) {
            al16((size_t)scap * 8) + al16((size_t)scap * 4) + finish_bytes(dm.BW, 1, dm.S, (dm.V + 31) / 32) + 64;
 }
 
-__global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t bar_mem;
-    __shared__ float red_f[2 * (kDnThreads / 32)];
-    __shared__ int red_i[32];
-    __shared__ int scan_w[32];
-    __shared__ uint64_t red_k[32];
-    __shared__ int hist[kRadixBins];
-    __shared__ int sc[4];
-    __shared__ int cnts[1];
+struct DenseShared {
+    uint64_t bar;
+    float red_f[kDnThreads / 32];
+    int red_i[32];
+    int scan_w[32];
+    uint32_t red32[64];
+    uint64_t red_k[32];
+    int hist[kRadixBins];
+    int sc[4];
+    int cnts[1];
+};
+
+// One request's first step.  dry: a warm-up pass -- a synthetic score row,
+// mask and root in shared memory through the same code, with no global
+// memory access.
+__device__ __forceinline__ void dense_select(const SelectArgs &a, uint8_t *smem, DenseShared &sh, bool dry) {
+    float *red_f = sh.red_f;
+    int *red_i = sh.red_i, *scan_w = sh.scan_w, *hist = sh.hist, *sc = sh.sc, *cnts = sh.cnts;
+    uint32_t *red32 = sh.red32;
+    uint64_t *red_k = sh.red_k;
     constexpr int kWarps = kDnThreads / 32;
     const Dims dm = a.dims;
     const int V = dm.V, BW = dm.BW, nw = (V + 31) / 32;
@@ -1183,9 +1470,9 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) 
     p += al16((size_t)scap * 4);
     const FinishSmem f = carve_finish(p, BW, 1, dm.S, nw);
     const float *xg = a.scores + rb * V;   // beam 0 of request r
-    const uint32_t bar = smem_u32(&bar_mem);
-    const bool bulk = (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
-    const int n = min(max(a.n_live[r], 0), 1);
+    const uint32_t bar = smem_u32(&sh.bar);
+    const bool bulk = !dry && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
+    const int n = dry ? 1 : min(max(a.n_live[r], 0), 1);
     if (tid == 0) {
         *f.cnt = 0;
         cnts[0] = 0;
@@ -1196,16 +1483,16 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) 
             bulk_g2s(smem_u32(x), xg, (uint32_t)V * 4u, bar);
         }
     }
-    const float cum = a.cum[rb];
+    const float cum = dry ? 0.f : a.cum[rb];
     // the mask with the tokens past V cleared; the valid-candidate count
     int c = 0;
     for (int w = tid; w < nw; w += kDnThreads) {
-        const uint32_t v = a.bits[w] & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u);
+        const uint32_t v = (dry ? ~0u : a.bits[w]) & (32 * w + 32 <= V ? ~0u : (1u << (V & 31)) - 1u);
         bits[w] = v;
         c += __popc(v);
     }
     if (a.rewire) {
-        stage_rows(a, rb, n, f);
+        if (!dry) stage_rows(a, rb, n, f);
         if (a.trie.root_bits) {
             // root children: bitset and exclusive prefix popcounts (trie order =
             // token order); thread t owns words [t*wpt, t*wpt + wpt)
@@ -1214,7 +1501,7 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) 
             for (int k = 0; k < wpt; ++k) {
                 const int w = tid * wpt + k;
                 if (w < nw) {
-                    const uint32_t v = a.trie.root_bits[w];
+                    const uint32_t v = dry ? ~0u : a.trie.root_bits[w];
                     f.root[w] = v;
                     cw += __popc(v);
                 }
@@ -1230,64 +1517,88 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) 
             }
         }
     }
-    if (!bulk && n > 0)
+    if (dry) {
+        for (int i = tid; i < V; i += kDnThreads) x[i] = -1e-3f * (float)(((uint32_t)i * 2654435761u) >> 16);
+        if (a.rewire)
+            for (int i = tid; i < dm.S; i += kDnThreads) {
+                f.st_anc[i] = 0;
+                f.st_seq[i] = 0;
+            }
+        if (tid == 0) f.st_node[0] = 0;
+    } else if (!bulk && n > 0) {
         for (int i = tid; i < V; i += kDnThreads) x[i] = xg[i];
+    }
     const int total = n > 0 ? block_sum_int(c, red_i) : 0;   // (+ a barrier)
     if (bulk && n > 0 && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
     const int want = min(BW, total);
     float lse = 0.f;
-    if (a.logits && want > 0) {   // per-warp (max, sum) over a slice, then combined
-        const int per = (V + kWarps - 1) / kWarps;
-        float mw = -INFINITY, sw = 0.f;
-        bool nan = false;
-        for (int i = warp * per + lane; i < min(V, warp * per + per); i += 32) {
-            const float v = x[i];
-            nan |= v != v;
-            if (v > mw) {
-                sw = mw == -INFINITY ? 0.f : sw * ex2f((mw - v) * kLog2e);
-                mw = v;
-            }
-            if (mw != -INFINITY) sw += ex2f((v - mw) * kLog2e);
-        }
-        if (__any_sync(0xffffffffu, nan) && lane == 0) set_status(a.status, XGR_DEV_NAN);
+    if (a.logits && want > 0) {
+        // thread t folds tokens t + kDnThreads * u: the maximum over four
+        // independent chains (NaN-propagating), then the sum of exponentials
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int i = tid; i < V; i += 4 * kDnThreads) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, mw, o), s2 = __shfl_xor_sync(0xffffffffu, sw, o);
-            lse_pair_merge(mw, sw, m2, s2);
+            for (int u = 0; u < 4; ++u) {
+                const int t = i + u * kDnThreads;
+                if (t < V) mx[u] = max_nan(mx[u], x[t]);
+            }
         }
-        if (lane == 0) {
-            red_f[2 * warp] = mw;
-            red_f[2 * warp + 1] = sw;
-        }
+        float mv = max_nan(max_nan(mx[0], mx[1]), max_nan(mx[2], mx[3]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mv = max_nan(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+        if (lane == 0) red_f[warp] = mv;
         __syncthreads();
-        float M = red_f[0], Ssum = red_f[1];
-        for (int k = 1; k < kWarps; ++k) lse_pair_merge(M, Ssum, red_f[2 * k], red_f[2 * k + 1]);
-        lse = M + logf(Ssum);
+        float M = red_f[0];
+        for (int k = 1; k < kWarps; ++k) M = max_nan(M, red_f[k]);
+        __syncthreads();   // red_f is read before it takes the sums
+        float sv = 0.f;
+        if (M != -INFINITY) {
+            const float mk = M * kLog2e;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int i = tid; i < V; i += 4 * kDnThreads) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int t = i + u * kDnThreads;
+                    if (t < V) acc[u] += ex2f(fmaf(x[t], kLog2e, -mk));
+                }
+            }
+            sv = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        }
+        sv = warp_sum_f(sv);
+        if (lane == 0) red_f[warp] = sv;
+        __syncthreads();
+        float S = 0.f;
+        for (int k = 0; k < kWarps; ++k) S += red_f[k];
+        lse = M + logf(S);
+        if (lse != lse && tid == 0) set_status(a.status, XGR_DEV_NAN);
     }
     DenseCand cand{x, bits, cum, lse, V, a.logits, a.status};
     uint64_t prefix = ~0ull, mask = 0;
     bool ranked = false;
     if (want > 0) {
-        // each thread's best key: real candidates for the threshold
+        // each thread's best key: real candidates for the cut
         uint64_t mn = kNoKey;
         for (int t = tid; t < V; t += kDnThreads) {
             uint64_t key = kNoKey;
             if (cand(t, key) && key < mn) mn = key;
         }
         mins[tid] = mn;
-        const int n_min = block_sum_int(mn != kNoKey ? 1 : 0, red_i);   // (+ a barrier)
-        uint64_t tau = kNoKey;
-        if (total > BW && n_min >= BW) {
-            uint64_t tp, tm;
-            smem_radix_select(mins, kDnThreads, BW, hist, scan_w, red_k, sc, tp, tm);
-            tau = selected_max(mins, kDnThreads, tp, tm, red_k);
-        }
-        // survivors: every key at or above tau, recomputed from the staged row
-        for (int t = tid; t < V; t += kDnThreads) {
-            uint64_t key;
-            if (!cand(t, key) || key > tau) continue;
-            const int pos = atomicAdd(&cnts[0], 1);
-            if (pos < scap) {
+        __syncthreads();
+        const Cut cut = total > BW ? make_cut(mins, kDnThreads, BW, hist, red32, scan_w, sc, red_k)
+                                   : Cut{0, 0, 0.f, 0, kNoKey};
+        // survivors: every key the cut keeps, recomputed from the staged row
+        // (one shared-memory atomic per warp and pass)
+        const unsigned lt = (1u << lane) - 1u;
+        for (int t0 = 0; t0 < V; t0 += kDnThreads) {
+            const int t = t0 + tid;
+            uint64_t key = kNoKey;
+            const bool keep = t < V && cand(t, key) && cut.keep(key);
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            int pos0 = 0;
+            if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            const int pos = pos0 + __popc(bal & lt);
+            if (keep && pos < scap) {
                 sk[pos] = key;
                 se[pos] = t;
             }
@@ -1306,7 +1617,25 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(SelectArgs a) 
         }
     }
     __syncthreads();
-    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked);
+    finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked, dry);
+}
+
+// The first step's kernel: one CTA per request.  It starts while the kernel
+// before it runs and takes a dry pass first (the code is cold on its SM),
+// then waits for that kernel and selects.
+__global__ void __launch_bounds__(kDnThreads) select_dense_kernel(const __grid_constant__ SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ DenseShared sh;
+    // a dry pass, then the real one, through one inlined copy (a rolled loop)
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1) {
+            griddep_wait();   // the scores and the beam state come from earlier kernels
+            griddep_launch_dependents();
+        }
+        dense_select(a, smem, sh, pass == 0);
+        __syncthreads();   // the pass's shared memory is free again
+    }
 }
 
 // opt in to the dynamic shared memory a launch needs: without it static plus
@@ -1325,13 +1654,9 @@ static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int select_head_m(int BW) { return BW >= 1024 ? 4 : 8; }
 
-size_t select_ticket_offset(int B, int BW) {
-    const size_t rows = (size_t)B * BW, m = (size_t)select_head_m(BW);
-    return 4 * al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4);
-}
-
 size_t select_scratch_bytes(int B, int BW, int64_t key_cap) {
-    return select_ticket_offset(B, BW) + al256((size_t)B * 4) + al256((size_t)B * key_cap * 8);
+    const size_t rows = (size_t)B * BW, m = (size_t)select_head_m(BW);
+    return 4 * al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4) + al256((size_t)B * key_cap * 8);
 }
 
 void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectArgs &a) {
@@ -1349,8 +1674,6 @@ void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectA
     base += al256(rows * m * 8);
     a.head_e = reinterpret_cast<int32_t *>(base);
     base += al256(rows * m * 4);
-    a.ticket = reinterpret_cast<uint32_t *>(base);
-    base += al256((size_t)B * 4);
     a.keys = reinterpret_cast<uint64_t *>(base);
     a.key_cap = key_cap;
     a.head_m = m;
@@ -1374,35 +1697,28 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
         const size_t smem = dense_smem(dm);
         cudaError_t e = ensure_smem(select_dense_kernel, smem);
         if (e != cudaSuccess) return e;
-        select_dense_kernel<<<dm.B, kDnThreads, smem, s>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(select_dense_kernel, dim3(dm.B), dim3(kDnThreads), smem, s, a);
     }
     // sparse: one launch, sp_parts CTAs per request of R beams, one per warp
     const int R = std::min(dm.BW, kSpWarps);
     a.sp_rows = R;
     a.sp_parts = (dm.BW + R - 1) / R;
-    if (a.head_m < 1 || a.head_m > 32) return cudaErrorInvalidValue;
+    if (a.head_m < 1 || a.head_m > 32 || (a.head_m & (a.head_m - 1))) return cudaErrorInvalidValue;
     if (a.mask_kind != XGR_MASK_CSR && a.mask_kind != XGR_MASK_TRIE_ROWS && a.mask_kind != XGR_MASK_NODE_BITS)
         return cudaErrorInvalidValue;
     if (a.mask_kind != XGR_MASK_CSR && (int64_t)dm.BW * a.row_stride > a.key_cap) return cudaErrorInvalidValue;
-    const int wt = a.mask_kind == XGR_MASK_NODE_BITS ? a.row_stride : 0;
-    // logits rows through the TMA engine: as many slots of a row as fit beside
-    // the token lists (each CTA takes R <= 8 rows, one per warp)
-    a.sp_slots = 0;
-    if (a.logits && (dm.V & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15) == 0) {
-        const size_t room = (200u << 10) - (size_t)kSpWarps * wt * 4;
-        // only when every warp gets a slot of its own: a slot handed from warp to
-        // warp would leave the later rows waiting for the earlier ones
-        if (room / al16((size_t)dm.V * 4) >= (size_t)R) a.sp_slots = R;
-    }
-    const size_t smem = sparse_smem(dm, a.head_m, wt, a.sp_slots);
-    if (smem > (220u << 10)) return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem(select_sparse_kernel, smem);
+    // a NODE_BITS row's token list takes its warp's ring once the row is streamed
+    if (a.mask_kind == XGR_MASK_NODE_BITS && (size_t)a.row_stride * 4 > kRingWarpBytes) return cudaErrorInvalidValue;
+    const size_t pick_smem = sparse_pick_smem(dm, a.head_m);
+    if (pick_smem > (220u << 10)) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_smem(select_rows_kernel, kRowsSmem);
+    if (e == cudaSuccess) e = ensure_smem(select_pick_kernel, pick_smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)dm.B * a.sp_parts;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    select_sparse_kernel<<<(int)grid, kSpThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    e = launch_pdl(select_rows_kernel, dim3((unsigned)grid), dim3(kSpThreads), kRowsSmem, s, a);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(select_pick_kernel, dim3(dm.B), dim3(kSpThreads), pick_smem, s, a);
 }
 
 }  // namespace xgr

@@ -105,6 +105,7 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
     a.logits = flags == XGR_SCORES_LOGITS;
     a.scores = d_scores;
     a.dense = dense;
+    a.prep_early = 0;   // nothing is known about the kernel before
     a.mask_kind = dense ? XGR_MASK_DENSE : XGR_MASK_CSR;
     a.bits = d_bits;
     a.row_ptr = d_row_ptr;
@@ -114,9 +115,6 @@ extern "C" xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_wid
         cudaDeviceGetAttribute(&a.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return XGR_ERR_CUDA;
     select_scratch_carve(sc + kStatusBytes, n_requests, beam_width, key_cap, a);
-    // the tickets must start at zero (each call also leaves them at zero)
-    if (!dense && cudaMemsetAsync(a.ticket, 0, (size_t)n_requests * 4, (cudaStream_t)stream) != cudaSuccess)
-        return XGR_ERR_CUDA;
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum_out;

@@ -167,6 +167,13 @@ struct xgr_ctx {
     int n_unfused[2] = {0, 0};   // requests the merge kernel still has to finish
     bool has_tc = false;       // tensor-core Shared stage available (D = 128, tensor maps built)
     CUtensorMap tmk, tmv;
+    CUtensorMap tmq;             // Q tensor map of the last decode step, re-encoded when q or B changes
+    const void *tmq_ptr = nullptr;
+    int64_t tmq_rows = -1;
+    // the last beam-state-writing or attention launch of this context: the
+    // attention of step attn_step on attn_stream (-1: something else)
+    int attn_step = -1;
+    cudaStream_t attn_stream = nullptr;
     // decode state
     bool begun = false;
     int cur_step = 0;
@@ -588,17 +595,13 @@ xgr_status xgr_begin(xgr_ctx *c, int32_t n_requests, xgr_stream_t stream) {
         c->planned_B = n_requests;
     }
     c->dims.B = n_requests;
-    uint32_t *sel_ticket =
-        c->cfg.vocab > 0 ? reinterpret_cast<uint32_t *>(
-                               c->at<uint8_t>(c->L.select_scratch) +
-                               select_ticket_offset(c->cfg.max_requests, c->cfg.beam_width))
-                         : nullptr;
     if (launch_begin(c->st, c->dims, c->cfg.max_requests, c->cfg.vocab == 0,
-                     c->cfg.vocab > 0 ? c->at<uint64_t>(c->L.mask_sync) : nullptr, sel_ticket,
-                     (cudaStream_t)stream) != cudaSuccess)
+                     c->cfg.vocab > 0 ? c->at<uint64_t>(c->L.mask_sync) : nullptr, (cudaStream_t)stream) !=
+        cudaSuccess)
         return XGR_ERR_CUDA;
     c->begun = true;
     c->cur_step = 0;
+    c->attn_step = -1;
     return XGR_OK;
 }
 
@@ -651,13 +654,17 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
         ta.step = step;
         // Q tiles of single-request items are one TMA box: D x (query heads of
         // one kv head) x (128 / G beams) over q viewed as [B*BW][Hq][D]
-        CUtensorMap tmq;
-        if (make_q_tensor_map(&tmq, d_q, (int64_t)c->dims.B * c->cfg.beam_width, c->cfg.n_q_heads,
-                              c->dims.G) != cudaSuccess) {
-            debug_log("decode_step: q tensor map failed");
-            return XGR_ERR_CUDA;
+        const int64_t q_rows = (int64_t)c->dims.B * c->cfg.beam_width;
+        if (c->tmq_ptr != d_q || c->tmq_rows != q_rows) {
+            if (make_q_tensor_map(&c->tmq, d_q, q_rows, c->cfg.n_q_heads, c->dims.G) != cudaSuccess) {
+                c->tmq_ptr = nullptr;
+                debug_log("decode_step: q tensor map failed");
+                return XGR_ERR_CUDA;
+            }
+            c->tmq_ptr = d_q;
+            c->tmq_rows = q_rows;
         }
-        const cudaError_t e = launch_attn_tc(c->tmk, c->tmv, tmq, ta, c->n_tc[which], s);
+        const cudaError_t e = launch_attn_tc(c->tmk, c->tmv, c->tmq, ta, c->n_tc[which], s);
         if (e != cudaSuccess) {
             debug_log("decode_step: tensor-core launch failed: %s", cudaGetErrorString(e));
             return XGR_ERR_CUDA;
@@ -667,6 +674,8 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
     // beam's rows, the not-yet-live ones at step 0 by zero-fill items): no merge
     if (c->n_unfused[which] == 0) {
         if (c->cfg.vocab == 0) c->cur_step = step + 1;
+        c->attn_step = step;
+        c->attn_stream = s;
         return XGR_OK;
     }
     MergeArgs ma;
@@ -691,6 +700,8 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
         }
     }
     if (c->cfg.vocab == 0) c->cur_step = step + 1;   // attention-only: no selection step
+    c->attn_step = step;
+    c->attn_stream = s;
     return XGR_OK;
 }
 
@@ -796,12 +807,16 @@ xgr_status xgr_beam_select(xgr_ctx *c, int32_t step, const float *d_scores, int3
     a.n_words = mask->n_words;
     a.row_stride = mask->row_stride;
     a.num_sms = c->num_sms;
+    // right after this step's attention on the same stream, the kernel before
+    // the selection wrote no beam state (the attention reads it only)
+    a.prep_early = c->attn_step == step && c->attn_stream == (cudaStream_t)stream;
     select_scratch_carve(c->at<uint8_t>(c->L.select_scratch), c->cfg.max_requests,
                          c->cfg.beam_width, c->L.key_cap, a);
     a.parent = d_parent;
     a.token = d_token;
     a.cum_out = d_cum;
     a.n_out = d_n_out;
+    c->attn_step = -1;
     if (launch_beam_select(a, (cudaStream_t)stream) != cudaSuccess) return XGR_ERR_CUDA;
     c->cur_step = step + 1;
     return XGR_OK;
