@@ -541,23 +541,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
             const bool is_u = j >= nchunks;            // an Unshared chunk
             const int c0 = u_lo - kBlockN * (j - nchunks);   // (is_u) the row's first column in it
-            auto u_out = [&](int c) {   // column c of an Unshared chunk is not this row's
-                const int t = c - c0;
-                return !(t >= 0 && t < T && ((vmask >> t) & 1u));
+            // Masked chunks (an Unshared chunk: only this row's own tokens count;
+            // the range's last chunk: keys past its end do not) keep the
+            // columns of a 32-bit mask per 32-column piece
+            const bool masked = is_u || nvalid < kBlockN;
+            auto piece_mask = [&](int q2) -> uint32_t {
+                if (is_u) {   // the row's valid tokens (vmask) start at column c0
+                    const int off = c0 - 32 * q2;
+                    return off >= 32 || off <= -32 ? 0u : off >= 0 ? vmask << off : vmask >> -off;
+                }
+                const int nv = nvalid - 32 * q2;
+                return nv >= 32 ? ~0u : nv <= 0 ? 0u : (1u << nv) - 1u;
             };
             // the chunk's 128 scores in one TMEM read (P_j then overwrites them)
             float sv[128];
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) tmem_ld32(tmem + lane_base + s_col + 32 * q2, sv + 32 * q2);
             tmem_wait_ld();
-            if (is_u) {
+            if (masked) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (u_out(c)) sv[c] = -INFINITY;
-            } else if (nvalid < kBlockN) {   // the range's last chunk: keys past its end do not count
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const uint32_t pm = piece_mask(q2);
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= nvalid) sv[c] = -INFINITY;
+                    for (int e = 0; e < 32; ++e)
+                        if (!((pm >> e) & 1u)) sv[32 * q2 + e] = -INFINITY;
+                }
             }
             float mxp[8];
 #pragma unroll
@@ -587,15 +595,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float v[32], pw[16];
                 tmem_ld32(tmem + lane_base + s_col + 32 * q2, v);
                 tmem_wait_ld_into(v);
-                const int nv = nvalid - 32 * q2;   // keys of the piece inside the range
-                if (is_u) {
+                if (masked) {
+                    const uint32_t pm = piece_mask(q2);
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        if (u_out(32 * q2 + e)) v[e] = -INFINITY;
-                } else if (nv < 32) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (e >= nv) v[e] = -INFINITY;
+                        if (!((pm >> e) & 1u)) v[e] = -INFINITY;
                 }
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {

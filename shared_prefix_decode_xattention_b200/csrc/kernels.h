@@ -124,6 +124,7 @@ struct SelectArgs {
     int32_t *row_cb;            // [B][BW] first trie child of each row's node (-1: none)
     uint64_t *head_k;           // [B][BW][m] each beam's m best keys, ascending (kNoKey pads)
     int32_t *head_e;            // [B][BW][m] their CSR entries (relative to the request)
+    uint64_t *head_next;        // [B][BW] each row's (m+1)-th best key (kNoKey: none)
     int head_m;                 // m
     uint64_t *keys;             // [B][key_cap] key of each CSR entry (relative to the request)
     int64_t key_cap;

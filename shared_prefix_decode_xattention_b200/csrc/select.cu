@@ -897,12 +897,14 @@ __device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uin
             ce[u] = (int)e;
             n_valid += key != kNoKey;
         }
-        warp_head_merge(c, ce, run, run_e, m);
+        warp_head_merge(c, ce, run, run_e, m + 1);
     }
     n_valid = warp_sum_int(n_valid);
     if (lane < m) {
         a.head_k[row * m + lane] = run;
         a.head_e[row * m + lane] = run_e;
+    } else if (lane == m) {
+        a.head_next[row] = run;   // the best key beyond the head
     }
     if (lane == 0) {
         a.row_cnt[row] = n_valid;
@@ -1146,8 +1148,12 @@ constexpr int kRankDirect = 512;   // most survivors ranked by counting
 __device__ void place_by_rank(const uint64_t *sk, const int *se, int ns, int want, const FinishSmem &f) {
     for (int i = threadIdx.x; i < ns; i += blockDim.x) {
         const uint64_t x = sk[i];
-        int c = 0;
-        for (int j = 0; j < ns; ++j) c += sk[j] < x;
+        int c = 0, j = 0;
+        for (; j + 8 <= ns; j += 8) {   // eight broadcast reads in flight
+#pragma unroll
+            for (int u = 0; u < 8; ++u) c += sk[j + u] < x;
+        }
+        for (; j < ns; ++j) c += sk[j] < x;
         if (c < want) {
             f.win_k[c] = x;
             f.win_e[c] = se[i];
@@ -1161,7 +1167,8 @@ __host__ __device__ inline int sparse_surv_cap(int BW) { return BW >= 1024 ? 409
 size_t sparse_pick_smem(const Dims &dm, int m) {
     const int cc = sparse_cand_cap(dm.BW, m), scap = sparse_surv_cap(dm.BW);
     return al16((size_t)cc * 8) + al16((size_t)cc * 4) + al16((size_t)scap * 8) + al16((size_t)scap * 4) +
-           al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) + finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
+           al16((size_t)(dm.BW + 1) * 4) + 2 * al16((size_t)dm.BW * 4) + al16((size_t)dm.BW * 8) +
+           finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
 }
 // phase 1: one ring per warp (the row stream and the NODE_BITS token list)
 constexpr size_t kRowsSmem = (size_t)kSpWarps * kRingWarpBytes;
@@ -1201,6 +1208,8 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
     p += al16((size_t)BW * 4);
     float *lse_s = reinterpret_cast<float *>(p);
     p += al16((size_t)BW * 4);
+    uint64_t *hnext = reinterpret_cast<uint64_t *>(p);   // each beam's best key beyond its head
+    p += al16((size_t)BW * 8);
     const FinishSmem f = carve_finish(p, BW, BW, dm.S, 0);
     int *cnts = reinterpret_cast<int *>(p + finish_bytes(BW, BW, dm.S, 0));   // [0] survivors, [1] saturated
 
@@ -1225,6 +1234,7 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
             f.rl[b] = m;
             f.cb[b] = -1;
             f.rp[b] = b * m;
+            hnext[b] = kNoKey;
         }
         if (tid == 0) f.rp[BW] = BW * m;
         c = tid == 0 ? BW * m : 0;
@@ -1233,6 +1243,7 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
         stage_l2(he, a.head_e + rb * m, BW * m * 4);
         stage_l2(f.rl, a.row_len + rb, BW * 4);
         stage_l2(f.cb, a.row_cb + rb, BW * 4);
+        stage_l2(hnext, a.head_next + rb, BW * 8);
         if (csr) stage_l2(f.rp, a.row_ptr + rb, (BW + 1) * 4);
         if (a.rewire) {
             stage_l2(f.st_anc, a.st.anc + rb * dm.S, BW * dm.S * 4);
@@ -1307,8 +1318,10 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
                 sk[pos] = key;
                 se[pos] = he[i];
             }
+            // (a beam whose best key beyond the head fails the cut has no
+            // further survivors: its further keys are worse still)
             const int b = i >> mshift;
-            if ((i & (m - 1)) == m - 1 && f.rl[b] > m) sat[atomicAdd(&cnts[1], 1)] = b;
+            if ((i & (m - 1)) == m - 1 && f.rl[b] > m && cut.keep(hnext[b])) sat[atomicAdd(&cnts[1], 1)] = b;
         }
         __syncthreads();
         const int n_sat = cnts[1];
@@ -1576,35 +1589,66 @@ __device__ __forceinline__ void dense_select(const SelectArgs &a, uint8_t *smem,
     uint64_t prefix = ~0ull, mask = 0;
     bool ranked = false;
     if (want > 0) {
-        // each thread's best key: real candidates for the cut
+        // each thread's best key: real candidates for the cut (four tokens in
+        // flight per pass)
         uint64_t mn = kNoKey;
-        for (int t = tid; t < V; t += kDnThreads) {
-            uint64_t key = kNoKey;
-            if (cand(t, key) && key < mn) mn = key;
+        for (int t0 = tid; t0 < V; t0 += 4 * kDnThreads) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + u * kDnThreads;
+                uint64_t key = kNoKey;
+                if (t < V && cand(t, key) && key < mn) mn = key;
+            }
         }
         mins[tid] = mn;
         __syncthreads();
         const Cut cut = total > BW ? make_cut(mins, kDnThreads, BW, hist, red32, scan_w, sc, red_k)
                                    : Cut{0, 0, 0.f, 0, kNoKey};
-        // survivors: every key the cut keeps, recomputed from the staged row
-        // (one shared-memory atomic per warp and pass)
-        const unsigned lt = (1u << lane) - 1u;
-        for (int t0 = 0; t0 < V; t0 += kDnThreads) {
-            const int t = t0 + tid;
-            uint64_t key = kNoKey;
-            const bool keep = t < V && cand(t, key) && cut.keep(key);
-            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-            int pos0 = 0;
-            if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
-            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-            const int pos = pos0 + __popc(bal & lt);
-            if (keep && pos < scap) {
-                sk[pos] = key;
-                se[pos] = t;
+        // survivors: every key the cut keeps, recomputed from the staged row --
+        // each thread counts its own, one block scan places them, then each
+        // thread writes its own (no atomics)
+        // (the first kKeep of a thread's survivors wait in registers)
+        constexpr int kKeep = 4;
+        uint64_t kk[kKeep];
+        int kt[kKeep];
+        int mine = 0;
+        for (int t0 = tid; t0 < V; t0 += 4 * kDnThreads) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + u * kDnThreads;
+                uint64_t key;
+                if (t < V && cand(t, key) && cut.keep(key)) {
+#pragma unroll
+                    for (int q = 0; q < kKeep; ++q)
+                        if (q == mine) {
+                            kk[q] = key;
+                            kt[q] = t;
+                        }
+                    ++mine;
+                }
+            }
+        }
+        int ns;
+        int pos = block_exclusive_scan_int(mine, scan_w, &ns);
+        if (mine <= kKeep) {
+#pragma unroll
+            for (int q = 0; q < kKeep; ++q)
+                if (q < mine && pos + q < scap) {
+                    sk[pos + q] = kk[q];
+                    se[pos + q] = kt[q];
+                }
+        } else {
+            for (int t = tid; t < V; t += kDnThreads) {
+                uint64_t key;
+                if (!cand(t, key) || !cut.keep(key)) continue;
+                if (pos < scap) {
+                    sk[pos] = key;
+                    se[pos] = t;
+                }
+                ++pos;
             }
         }
         __syncthreads();
-        const int ns = cnts[0];
         if (ns <= kRankDirect) {
             place_by_rank(sk, se, ns, want, f);
             ranked = true;
@@ -1656,7 +1700,8 @@ int select_head_m(int BW) { return BW >= 1024 ? 4 : 8; }
 
 size_t select_scratch_bytes(int B, int BW, int64_t key_cap) {
     const size_t rows = (size_t)B * BW, m = (size_t)select_head_m(BW);
-    return 4 * al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4) + al256((size_t)B * key_cap * 8);
+    return 4 * al256(rows * 4) + al256(rows * m * 8) + al256(rows * m * 4) + al256(rows * 8) +
+           al256((size_t)B * key_cap * 8);
 }
 
 void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectArgs &a) {
@@ -1674,6 +1719,8 @@ void select_scratch_carve(uint8_t *base, int B, int BW, int64_t key_cap, SelectA
     base += al256(rows * m * 8);
     a.head_e = reinterpret_cast<int32_t *>(base);
     base += al256(rows * m * 4);
+    a.head_next = reinterpret_cast<uint64_t *>(base);
+    base += al256(rows * 8);
     a.keys = reinterpret_cast<uint64_t *>(base);
     a.key_cap = key_cap;
     a.head_m = m;
@@ -1703,7 +1750,7 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
     const int R = std::min(dm.BW, kSpWarps);
     a.sp_rows = R;
     a.sp_parts = (dm.BW + R - 1) / R;
-    if (a.head_m < 1 || a.head_m > 32 || (a.head_m & (a.head_m - 1))) return cudaErrorInvalidValue;
+    if (a.head_m < 1 || a.head_m > 16 || (a.head_m & (a.head_m - 1))) return cudaErrorInvalidValue;   // (m + 1 lanes merge)
     if (a.mask_kind != XGR_MASK_CSR && a.mask_kind != XGR_MASK_TRIE_ROWS && a.mask_kind != XGR_MASK_NODE_BITS)
         return cudaErrorInvalidValue;
     if (a.mask_kind != XGR_MASK_CSR && (int64_t)dm.BW * a.row_stride > a.key_cap) return cudaErrorInvalidValue;
