@@ -584,27 +584,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // (S_j was issued after P_{j-2} V_{j-2} completed: O_half is current and
             // this TMEM buffer no longer holds P_{j-2})
             // exponentials, row sum and P (bf16 pairs) into the first 64 columns of
-            // the S buffer, in four rolled pieces of 32 scores re-read from TMEM (a
-            // small loop body): piece q's 16 P columns land on scores already read
+            // the S buffer, from the scores already in registers (masked ones are
+            // -inf): piece q's 16 P columns land on scores already read
             const float neg_m = -m_used;
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-#pragma unroll 1
-            for (int q2 = 0; q2 < 4; ++q2) {
-                float v[32], pw[16];
-                tmem_ld32(tmem + lane_base + s_col + 32 * q2, v);
-                tmem_wait_ld_into(v);
-                if (masked) {
-                    const uint32_t pm = piece_mask(q2);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (!((pm >> e) & 1u)) v[e] = -INFINITY;
-                }
+            for (int q2 = 0; q2 < 4; ++q2) {
+                float pw[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(v[2 * e], cscale, neg_m));
-                    const float p1 = ex2(fmaf(v[2 * e + 1], cscale, neg_m));
+                    const float p0 = ex2(fmaf(sv[32 * q2 + 2 * e], cscale, neg_m));
+                    const float p1 = ex2(fmaf(sv[32 * q2 + 2 * e + 1], cscale, neg_m));
                     sp[(2 * e) & 7] += p0;
                     sp[(2 * e + 1) & 7] += p1;
                     __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
