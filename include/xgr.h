@@ -201,6 +201,29 @@ xgr_status xgr_begin(xgr_ctx *ctx, int32_t n_requests, xgr_stream_t stream);
 xgr_status xgr_decode_step(xgr_ctx *ctx, int32_t step, const void *d_q, const void *d_k_new,
                            const void *d_v_new, void *d_out, float *d_lse, xgr_stream_t stream);
 
+/* Per-beam comparison path -- a baseline, not the product path.  xGR page, 1
+ * "Problem definition": serving systems built around PagedAttention treat
+ * each beam as an independent sequence, so every beam reloads the shared
+ * prompt KV, and forking beams copies KV blocks; 4 "Kernel efficiency"
+ * compares the staged kernel with that baseline.  Same contract as
+ * xgr_decode_step (same arguments and outputs, equal within rounding), but
+ * computed that way: each beam streams its request's whole prompt (+ suffix)
+ * from the KV store itself, and its generated tokens live in a private block
+ * of 16 tokens that a new beam copies whole from its parent (its ancestry slot
+ * of the previous step) before appending this step's k / v.  The context's
+ * Unshared pool is neither read nor written.
+ *   d_blocks: caller-owned device memory of xgr_per_beam_bytes bytes (16-byte
+ *             aligned) kept for the whole decode, the first call of which is
+ *             step 0 (its blocks of the previous step are the parents').
+ * head_dim 128 and at most 8 query heads per kv head (else
+ * XGR_ERR_UNIMPLEMENTED); blocks_bytes below the size: XGR_ERR_CAPACITY.  Two
+ * kernels on `stream`; advances the current step only for a context without
+ * a vocabulary, like xgr_decode_step. */
+xgr_status xgr_per_beam_bytes(const xgr_ctx *ctx, size_t *bytes);
+xgr_status xgr_decode_step_per_beam(xgr_ctx *ctx, int32_t step, const void *d_q, const void *d_k_new,
+                                    const void *d_v_new, void *d_out, float *d_lse, void *d_blocks,
+                                    size_t blocks_bytes, xgr_stream_t stream);
+
 /* Valid-path mask of step `step` (xGR 2.2 "Hybrid dense/sparse storage").
  * Enqueues nothing: every kind is a view of pre-built tables and of the beam
  * state.  Step 0: DENSE (the root's bitset).  Step 1: NODE_BITS when

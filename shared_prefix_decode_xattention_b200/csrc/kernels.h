@@ -156,6 +156,29 @@ cudaError_t launch_beam_select(const SelectArgs &a, cudaStream_t s);
 
 cudaError_t launch_get_sequences(BeamState st, Dims dm, int32_t *seq, cudaStream_t s);
 
+// ---- the per-beam comparison path (attn_per_beam.cu)
+constexpr int kPerBeamBlock = 16;   // tokens of a beam's private block (>= kMaxSteps)
+struct PerBeamArgs {
+    const __nv_bfloat16 *q;        // [B][BW][Hq][D]
+    const __nv_bfloat16 *k_new;    // [B][BW][Hkv][D]
+    const __nv_bfloat16 *v_new;
+    const __nv_bfloat16 *kstore;   // [Hkv][kv_tokens][D]
+    const __nv_bfloat16 *vstore;
+    __nv_bfloat16 *blk_k;          // [2][Bcap][BW][Hkv][kPerBeamBlock][D] (step parity first)
+    __nv_bfloat16 *blk_v;
+    __nv_bfloat16 *out;            // [B][BW][Hq][D]
+    float *lse;                    // [B][BW][Hq]
+    const int32_t *req_seg;        // [B][4]: prompt offset, length, suffix offset, length
+    const int32_t *n_live;         // [B]
+    BeamState st;
+    int32_t *status;
+    Dims dims;
+    int Bcap, step;
+    int64_t kv_tokens;
+};
+cudaError_t launch_per_beam(const PerBeamArgs &a, cudaStream_t st);
+size_t per_beam_block_bytes(int Bcap, int BW, int Hkv, int D);
+
 // Launches `kernel` on `s` with programmatic stream serialization: the
 // kernel may start while the previous kernel in the stream is still running,
 // so it must call griddep_wait() before it reads or writes anything that

@@ -60,6 +60,7 @@ struct Layout {
     size_t part_o, part_ml;
     int slots;
     size_t plan_items[2], plan_members[2], plan_nslots[2];
+    size_t req_seg;              // [B][4] each request's prompt and suffix ranges (per-beam path)
     int64_t item_cap, member_cap;
     size_t total;
 };
@@ -114,6 +115,7 @@ void make_layout(const xgr_config &c, Layout &L) {
         L.plan_members[p] = take(4 * L.member_cap);
         L.plan_nslots[p] = take(4 * B);
     }
+    L.req_seg = take(16 * B);
     L.total = off;
 }
 
@@ -591,6 +593,18 @@ xgr_status xgr_begin(xgr_ctx *c, int32_t n_requests, xgr_stream_t stream) {
             const xgr_status e = build_plan(c, p, n_requests);
             if (e) return e;
         }
+        // each request's KV ranges, for the per-beam comparison path
+        std::vector<int32_t> seg(4 * (size_t)n_requests);
+        for (int r = 0; r < n_requests; ++r) {
+            const int sid = c->req_sid[r];
+            seg[4 * r] = sid >= 0 ? (int32_t)c->sid_off[sid] : 0;
+            seg[4 * r + 1] = sid >= 0 ? (int32_t)c->sid_len[sid] : 0;
+            seg[4 * r + 2] = (int32_t)c->suf_off[r];
+            seg[4 * r + 3] = (int32_t)c->suf_len[r];
+        }
+        if (cudaMemcpy(c->at<int32_t>(c->L.req_seg), seg.data(), seg.size() * 4, cudaMemcpyHostToDevice) !=
+            cudaSuccess)
+            return XGR_ERR_CUDA;
         c->plan_dirty = false;
         c->planned_B = n_requests;
     }
@@ -699,6 +713,51 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
             return XGR_ERR_CUDA;
         }
     }
+    if (c->cfg.vocab == 0) c->cur_step = step + 1;   // attention-only: no selection step
+    c->attn_step = step;
+    c->attn_stream = s;
+    return XGR_OK;
+}
+
+xgr_status xgr_per_beam_bytes(const xgr_ctx *c, size_t *bytes) {
+    if (!c || !bytes) return XGR_ERR_ARG;
+    *bytes = per_beam_block_bytes(c->cfg.max_requests, c->cfg.beam_width, c->cfg.n_kv_heads, c->cfg.head_dim);
+    return XGR_OK;
+}
+
+xgr_status xgr_decode_step_per_beam(xgr_ctx *c, int32_t step, const void *d_q, const void *d_k_new,
+                                    const void *d_v_new, void *d_out, float *d_lse, void *d_blocks,
+                                    size_t blocks_bytes, xgr_stream_t stream) {
+    if (!c) return XGR_ERR_ARG;
+    if (!aligned16(d_q) || !aligned16(d_k_new) || !aligned16(d_v_new) || !aligned16(d_out) ||
+        !aligned16(d_lse) || !aligned16(d_blocks))
+        return XGR_ERR_ARG;
+    if (!c->begun || step != c->cur_step || step >= c->cfg.steps) return XGR_ERR_STATE;
+    if (c->cfg.head_dim != 128 || c->dims.G > 8 || (c->dims.G & (c->dims.G - 1)) || step + 1 > kPerBeamBlock)
+        return XGR_ERR_UNIMPLEMENTED;
+    const size_t need = per_beam_block_bytes(c->cfg.max_requests, c->cfg.beam_width, c->cfg.n_kv_heads,
+                                             c->cfg.head_dim);
+    if (blocks_bytes < need) return XGR_ERR_CAPACITY;
+    const cudaStream_t s = (cudaStream_t)stream;
+    PerBeamArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(d_q);
+    a.k_new = static_cast<const __nv_bfloat16 *>(d_k_new);
+    a.v_new = static_cast<const __nv_bfloat16 *>(d_v_new);
+    a.kstore = c->at<__nv_bfloat16>(c->L.kstore);
+    a.vstore = c->at<__nv_bfloat16>(c->L.vstore);
+    a.blk_k = static_cast<__nv_bfloat16 *>(d_blocks);
+    a.blk_v = a.blk_k + need / 4;   // (need / 2 bytes of K blocks, then V)
+    a.out = static_cast<__nv_bfloat16 *>(d_out);
+    a.lse = d_lse;
+    a.req_seg = c->at<int32_t>(c->L.req_seg);
+    a.n_live = c->st.n_live;
+    a.st = c->st;
+    a.status = c->st.status;
+    a.dims = c->dims;
+    a.Bcap = c->cfg.max_requests;
+    a.step = step;
+    a.kv_tokens = c->cfg.kv_tokens;
+    if (launch_per_beam(a, s) != cudaSuccess) return XGR_ERR_CUDA;
     if (c->cfg.vocab == 0) c->cur_step = step + 1;   // attention-only: no selection step
     c->attn_step = step;
     c->attn_stream = s;

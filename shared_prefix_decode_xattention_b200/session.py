@@ -53,6 +53,15 @@ class Session:
     def decode_step(self, step, q, k_new, v_new, out, lse, stream=None):
         xgr.xgr_decode_step(self.ctx, step, q, k_new, v_new, out, lse, stream)
 
+    def decode_step_per_beam(self, step, q, k_new, v_new, out, lse, stream=None):
+        """The per-beam comparison path (its private blocks allocated on first use)."""
+        import torch
+        if getattr(self, "_pb_blocks", None) is None:
+            n = xgr.xgr_per_beam_bytes(self.ctx)
+            self._pb_blocks = torch.zeros(n, dtype=torch.uint8, device=self.workspace.device)
+        xgr.xgr_decode_step_per_beam(self.ctx, step, q, k_new, v_new, out, lse, self._pb_blocks,
+                                     self._pb_blocks.numel(), stream)
+
     def build_mask(self, step, stream=None) -> xgr.xgr_mask:
         return xgr.xgr_build_mask(self.ctx, step, stream)
 

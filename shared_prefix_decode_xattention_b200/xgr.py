@@ -117,6 +117,8 @@ def lib():
         "xgr_reset_kv": [P],
         "xgr_begin": [P, i32, P],
         "xgr_decode_step": [P, i32, P, P, P, P, P, P],
+        "xgr_per_beam_bytes": [P, ctypes.POINTER(ctypes.c_size_t)],
+        "xgr_decode_step_per_beam": [P, i32, P, P, P, P, P, P, ctypes.c_size_t, P],
         "xgr_build_mask": [P, i32, ctypes.POINTER(xgr_mask), P],
         "xgr_mask_to_csr": [P, ctypes.POINTER(xgr_mask), P, P, i64, P],
         "xgr_beam_select": [P, i32, P, i32, ctypes.POINTER(xgr_mask), P, P, P, P, P],
@@ -210,6 +212,19 @@ def xgr_begin(ctx: int, n_requests: int, stream=None) -> None:
 def xgr_decode_step(ctx: int, step: int, q, k_new, v_new, out, lse, stream=None) -> None:
     _check("xgr_decode_step", lib().xgr_decode_step(ctx, step, _ptr(q), _ptr(k_new), _ptr(v_new),
                                                     _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def xgr_per_beam_bytes(ctx: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("xgr_per_beam_bytes", lib().xgr_per_beam_bytes(ctx, ctypes.byref(n)))
+    return n.value
+
+
+def xgr_decode_step_per_beam(ctx: int, step: int, q, k_new, v_new, out, lse, blocks, nbytes: int,
+                             stream=None) -> None:
+    _check("xgr_decode_step_per_beam",
+           lib().xgr_decode_step_per_beam(ctx, step, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                          _ptr(lse), _ptr(blocks), nbytes, _stream(stream)))
 
 
 def xgr_build_mask(ctx: int, step: int, stream=None) -> xgr_mask:

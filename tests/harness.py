@@ -44,8 +44,9 @@ class StepOut:
 class GpuRun:
     """One decode of workload w on cuda:0 through the C ABI."""
 
-    def __init__(self, w, items=None, device="cuda", max_partials=0):
+    def __init__(self, w, items=None, device="cuda", max_partials=0, per_beam=False):
         self.w, self.device = w, device
+        self.per_beam = per_beam   # attention by the per-beam comparison path
         self.sess = Session(config_for(w, max_partials=max_partials), device)
         if w.V:
             self.sess.build_trie(items)
@@ -72,7 +73,10 @@ class GpuRun:
         # NaN sentinels: every row the call must write (dead beams' zeros included) is checked
         out = torch.full((w.B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=self.device)
         lse = torch.full((w.B, w.BW, w.Hq), float("nan"), dtype=torch.float32, device=self.device)
-        self.sess.decode_step(s, q, kn, vn, out, lse)
+        if self.per_beam:
+            self.sess.decode_step_per_beam(s, q, kn, vn, out, lse)
+        else:
+            self.sess.decode_step(s, q, kn, vn, out, lse)
         if not w.V:
             return StepOut(out, lse, None)
         m = self.sess.build_mask(s)

@@ -27,10 +27,10 @@ def _sample_beams(n_live, k, seed):
 
 
 def decode_and_compare(w, mode="logprob", requests=None, beams_per_step=None, items=None,
-                       max_partials=0, scores_fn=None):
+                       max_partials=0, scores_fn=None, per_beam=False):
     items = workloads.items(w) if items is None else items
     si = oracle.SortedItems(items, w.V) if w.V else None
-    run = GpuRun(w, items, max_partials=max_partials)
+    run = GpuRun(w, items, max_partials=max_partials, per_beam=per_beam)
     reqs = list(range(w.B)) if requests is None else list(requests)
     decs = {r: oracle_request(w, si, run, r, mode) for r in reqs}
     flags = xgr.XGR_SCORES_LOGPROB if mode == "logprob" else xgr.XGR_SCORES_LOGITS
