@@ -705,7 +705,9 @@ def run_gpu(args, w):
     par = torch.empty((w.B, w.BW), dtype=torch.int32, device=dev)
     tok = torch.empty_like(par)
     cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=dev)
-    nout = torch.empty((w.B,), dtype=torch.int32, device=dev)
+    # one n_out per group (the call wants 16-byte aligned outputs; a group's
+    # slice of one [B] array is not when B / G is not a multiple of 4)
+    nout_g = [torch.empty((Bg,), dtype=torch.int32, device=dev) for _ in range(G)]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for sg in sessions:
         sg.begin(Bg)   # plan once (setup)
@@ -743,10 +745,11 @@ def run_gpu(args, w):
 
     def sel_g(g, st, s, inp, host):
         sessions[g].beam_select(s, inp[s][3][sl(g)], flags, masks[g][s], par[sl(g)], tok[sl(g)],
-                                cum[sl(g)], nout[sl(g)], st)
+                                cum[sl(g)], nout_g[g], st)
         if host is not None:
-            for h, d in zip(host[w.S + s], (par, tok, cum, nout)):
+            for h, d in zip(host[w.S + s], (par, tok, cum)):
                 h[sl(g)].copy_(d[sl(g)], non_blocking=True)
+            host[w.S + s][3][sl(g)].copy_(nout_g[g], non_blocking=True)
 
     def enqueue_att(s, inp, host):
         fork(lambda g, st: att_g(g, st, s, inp, host))
@@ -823,7 +826,7 @@ def run_gpu(args, w):
         dist.barrier()
     clocks = clk.stop() if clk else None
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), dev)
-    n_live = nout.cpu().numpy()
+    n_live = torch.cat(nout_g).cpu().numpy()
     cands = candidates_per_decode(w) * args.steps * world
     value = cands / (total_ms / 1e3)
 
@@ -850,7 +853,8 @@ def run_gpu(args, w):
             host.append(hs)
             h2d += sum(t.numel() * t.element_size() for t in hs)
         for s in range(w.S):
-            hs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (par, tok, cum, nout)]
+            hs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (par, tok, cum)]
+            hs.append(torch.empty((w.B,), dtype=torch.int32).pin_memory())
             host.append(hs)
             d2h += sum(t.numel() * t.element_size() for t in hs)
         dev_in = [tuple(torch.empty_like(t) for t in inputs[s]) for s in range(w.S)]
