@@ -131,7 +131,7 @@ struct SelectArgs {
     int prep_early;             // the kernel before writes no beam state: the mask lookups may
                                 //   run before the programmatic-launch wait
     int sp_parts;               // set by the launcher: CTAs per request of the sparse kernel
-    int sp_rows;                //   and the beams each of them takes (<= 8: one per warp)
+    int sp_rows;                //   and the beams each of them takes (one per warp)
     int num_sms;                // SMs of the device
     int32_t *parent;            // outputs [B][BW]
     int32_t *token;

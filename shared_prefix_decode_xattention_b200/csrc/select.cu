@@ -503,7 +503,7 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
 
 // ------------------------------------------------------------------ sparse steps
 
-// Phase 1 (select_rows_kernel): request r gets sp_parts CTAs of kSpThreads
+// Phase 1 (select_rows_kernel): request r gets sp_parts CTAs of 32 * sp_rows
 // threads; CTA `part` takes beams [part*R, part*R + R) (R = sp_rows), one warp
 // per beam, so no reduction spans more than one warp.  Per beam:
 //  * logits mode: the row's log-sum-exp over the full vocabulary, streamed
@@ -514,13 +514,19 @@ __device__ void finish_request(const SelectArgs &a, int r, int n_win, const Fini
 //  * the beam's head: its m best keys with their entries, ascending (the
 //    page's per-beam ordered candidate list, cut at m).
 // Phase 2 (select_pick_kernel) selects for the whole request from the heads.
-constexpr int kSpThreads = 256;
+constexpr int kSpThreads = 256;   // the pick kernel's CTA
 constexpr int kSpWarps = kSpThreads / 32;
+// The rows kernel's CTA takes kRowWarpsWide beam rows with five-stage rings
+// (one CTA per SM) when the grid fits one wave, else kRowWarpsNarrow rows with
+// three-stage rings (three CTAs per SM: more rows stream at once, and one
+// CTA's keys and head merge overlap the others' streams).
+constexpr int kRowWarpsWide = 8, kRingWide = 5;
+constexpr int kRowWarpsNarrow = 4, kRingNarrow = 3;
 constexpr int kSpKpc = 8;             // CSR entries per lane in one pass of the key loop
 constexpr int kRingStageBytes = 4096;  // one stage of a warp's row stream
-constexpr int kRingStages = 5;         // stages of a warp's ring, all in flight but the one folding
 constexpr int kWtokCap = 1024;         // NODE_BITS tokens listed beside the ring before the stream
-constexpr size_t kRingWarpBytes = (size_t)kRingStages * kRingStageBytes + kWtokCap * 4;   // 24 KB
+// a warp's area: its ring of `ring` stages, then its token list
+__host__ __device__ inline size_t ring_warp_bytes(int ring) { return (size_t)ring * kRingStageBytes + kWtokCap * 4; }
 
 // max that returns NaN when either operand is NaN
 __device__ __forceinline__ float max_nan(float a, float b) {
@@ -567,40 +573,42 @@ __device__ __forceinline__ float warp_lse_merge(float m, float s) {
 }
 
 // A warp's score-row stream: the row's bytes go through the warp's ring of
-// kRingStages shared-memory stages by bulk copies (the TMA engine), issued
+// RING shared-memory stages by bulk copies (the TMA engine), issued
 // by lane 0 and landing on one mbarrier per stage; all stages but the one the
 // lanes fold are in flight.  The same warp issues, waits for and refills each
 // stage in order, so a stage's barrier is never more than one phase ahead of
 // its waiter (parity = use count & 1).  Needs the row 16-byte aligned and a
 // multiple of 16 bytes long.
+template <int RING>
 struct RowStream {
     const uint8_t *src;
     int bytes, nst;
-    float4 *ring;     // the warp's stages
-    uint32_t bar0;    // its kRingStages barriers (8 bytes apart)
+    float4 *stages;   // the warp's stage area
+    uint32_t bar0;    // its RING barriers (8 bytes apart)
     __device__ void issue(int st) const {   // lane 0
         if (st >= nst) return;
-        const int slot = st % kRingStages, off = st * kRingStageBytes;
+        const int slot = st % RING, off = st * kRingStageBytes;
         const uint32_t n = (uint32_t)min(kRingStageBytes, bytes - off);
         const uint32_t bar = bar0 + 8u * (uint32_t)slot;
         mbar_expect_tx(bar, n);
-        bulk_g2s(smem_u32(ring) + (uint32_t)(slot * kRingStageBytes), src + off, n, bar);
+        bulk_g2s(smem_u32(stages) + (uint32_t)(slot * kRingStageBytes), src + off, n, bar);
     }
 };
 
-// starts the stream: the first kRingStages stages go out (barriers initialised
+// starts the stream: the first RING stages go out (barriers initialised
 // by lane 0 here, before any lane waits on them)
-__device__ RowStream row_stream_start(const float *x, int V, float4 *ring, uint64_t *bars) {
-    RowStream rs;
+template <int RING>
+__device__ RowStream<RING> row_stream_start(const float *x, int V, float4 *ring_area, uint64_t *bars) {
+    RowStream<RING> rs;
     rs.src = reinterpret_cast<const uint8_t *>(x);
     rs.bytes = V * 4;
     rs.nst = (rs.bytes + kRingStageBytes - 1) / kRingStageBytes;
-    rs.ring = ring;
+    rs.stages = ring_area;
     rs.bar0 = smem_u32(bars);
     if ((threadIdx.x & 31) == 0) {
-        for (int i = 0; i < kRingStages; ++i) mbar_init(rs.bar0 + 8u * (uint32_t)i, 1);
+        for (int i = 0; i < RING; ++i) mbar_init(rs.bar0 + 8u * (uint32_t)i, 1);
         fence_mbar_init();
-        for (int st = 0; st < min(rs.nst, kRingStages); ++st) rs.issue(st);
+        for (int st = 0; st < min(rs.nst, RING); ++st) rs.issue(st);
     }
     __syncwarp();
     return rs;
@@ -608,18 +616,19 @@ __device__ RowStream row_stream_start(const float *x, int V, float4 *ring, uint6
 
 // Natural-log log-sum-exp of the streamed row by its warp (every lane gets it;
 // NaN when the row holds a NaN).  Each stage is folded by all lanes, then
-// refilled with the stage kRingStages ahead.  A stage that never lands (a
+// refilled with the stage RING ahead.  A stage that never lands (a
 // bounded wait runs out) sets XGR_DEV_TIMEOUT; the copies still in flight are
 // waited for (bounded) before the ring is given back.
-__device__ float row_stream_lse(const RowStream &rs, int32_t *status) {
+template <int RING>
+__device__ float row_stream_lse(const RowStream<RING> &rs, int32_t *status) {
     const int lane = threadIdx.x & 31;
     float m = -INFINITY, s = 0.f;
     int st = 0;
     for (; st < rs.nst; ++st) {
-        const int slot = st % kRingStages;
+        const int slot = st % RING;
         const uint32_t bar = rs.bar0 + 8u * (uint32_t)slot;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)(st / kRingStages) & 1u, nullptr))) break;
-        const float4 *src = rs.ring + slot * (kRingStageBytes / 16);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar, (uint32_t)(st / RING) & 1u, nullptr))) break;
+        const float4 *src = rs.stages + slot * (kRingStageBytes / 16);
         const int n4 = min(kRingStageBytes, rs.bytes - st * kRingStageBytes) / 16;
         float v[32];
 #pragma unroll
@@ -633,16 +642,16 @@ __device__ float row_stream_lse(const RowStream &rs, int32_t *status) {
         }
         lse_fold32(v, m, s);
         __syncwarp();   // every lane has read the stage
-        if (lane == 0 && st + kRingStages < rs.nst) {
+        if (lane == 0 && st + RING < rs.nst) {
             fence_async_smem();   // those reads before the bulk copy's writes
-            rs.issue(st + kRingStages);
+            rs.issue(st + RING);
         }
     }
     if (st < rs.nst) {   // timed out: let the issued copies land before the ring is reused
         if (lane == 0) {
             set_status(status, XGR_DEV_TIMEOUT);
-            for (int q = st; q < min(rs.nst, st + kRingStages); ++q)
-                mbar_wait(rs.bar0 + 8u * (uint32_t)(q % kRingStages), (uint32_t)(q / kRingStages) & 1u, nullptr);
+            for (int q = st; q < min(rs.nst, st + RING); ++q)
+                mbar_wait(rs.bar0 + 8u * (uint32_t)(q % RING), (uint32_t)(q / RING) & 1u, nullptr);
         }
         __syncwarp();
     }
@@ -755,8 +764,8 @@ __device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int ca
 // completed before the one before this kernel started), and the mask tables.
 // row_run follows the wait: in logits mode the row streams through the warp's
 // ring for its log-sum-exp while the first pass's scores are fetched.  area:
-// the warp's kRingWarpBytes of shared memory (16-byte aligned); bars: its
-// kRingStages mbarriers.
+// the warp's ring_warp_bytes(RING) of shared memory (16-byte aligned);
+// bars: its RING mbarriers.
 struct RowPrep {
     bool live;
     float cum;
@@ -766,12 +775,13 @@ struct RowPrep {
     int tk0[kSpKpc];   // the first pass's tokens (lane j: entries j, j + 32, ...)
 };
 
+template <int RING>
 __device__ RowPrep row_prep(const SelectArgs &a, int r, int b, int n_live, int base, uint8_t *area) {
     const int lane = threadIdx.x & 31;
     const Dims dm = a.dims;
     const int s = a.step;
     const int64_t row = (int64_t)r * dm.BW + b;
-    int *wtok = reinterpret_cast<int *>(area + (size_t)kRingStages * kRingStageBytes);
+    int *wtok = reinterpret_cast<int *>(area + (size_t)RING * kRingStageBytes);
     RowPrep p;
     p.live = b < n_live;
     p.cum = a.cum[row];
@@ -821,6 +831,7 @@ __device__ RowPrep row_prep(const SelectArgs &a, int r, int b, int n_live, int b
     return p;
 }
 
+template <int RING>
 __device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uint64_t *keys, uint8_t *area,
                         uint64_t *bars) {
     const int lane = threadIdx.x & 31;
@@ -831,8 +842,8 @@ __device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uin
     const float *x = a.scores + row * V;
     float4 *ring = reinterpret_cast<float4 *>(area);
     const bool stream = a.logits && live && (V & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
-    RowStream rs{};
-    if (stream) rs = row_stream_start(x, V, ring, bars);
+    RowStream<RING> rs{};
+    if (stream) rs = row_stream_start<RING>(x, V, ring, bars);
     // the first pass's scores go out before the stream is folded
     float sv0[kSpKpc];
 #pragma unroll
@@ -1171,7 +1182,6 @@ size_t sparse_pick_smem(const Dims &dm, int m) {
            finish_bytes(dm.BW, dm.BW, dm.S, 0) + 64;
 }
 // phase 1: one ring per warp (the row stream and the NODE_BITS token list)
-constexpr size_t kRowsSmem = (size_t)kSpWarps * kRingWarpBytes;
 
 // Phase 2, by the request's last CTA.  The cut comes from the beams' heads
 // (every head key is a real candidate, so at least BW real candidates lie at
@@ -1362,10 +1372,12 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
     finish_request(a, r, ranked ? want : min(*f.cnt, want), f, ranked, dry);
 }
 
-// Phase 1: sp_parts CTAs per request of sp_rows beams, one warp per beam.
-__global__ void __launch_bounds__(kSpThreads, 1) select_rows_kernel(SelectArgs a) {
+// Phase 1: sp_parts CTAs per request of sp_rows (<= W) beams, one warp per
+// beam, each with a ring of RING stages.
+template <int W, int kMinBlocks, int RING>
+__global__ void __launch_bounds__(W * 32, kMinBlocks) select_rows_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t ring_bar[kSpWarps][kRingStages];
+    __shared__ uint64_t ring_bar[W][RING];
     const Dims dm = a.dims;
     const int C = a.sp_parts, R = a.sp_rows;
     const int r = blockIdx.x / C, part = blockIdx.x % C;
@@ -1373,14 +1385,14 @@ __global__ void __launch_bounds__(kSpThreads, 1) select_rows_kernel(SelectArgs a
     const int64_t rb = (int64_t)r * dm.BW;
     const int b = part * R + warp;
     const bool has_row = warp < R && b < dm.BW;
-    uint8_t *area = smem + (size_t)warp * kRingWarpBytes;
+    uint8_t *area = smem + (size_t)warp * ring_warp_bytes(RING);
     // the mask lookups (beam state and tables only) go before the wait when
     // the kernel before writes no beam state (the scores always follow it)
     RowPrep p;
     auto prep = [&]() {
         const int n_live = min(max(a.n_live[r], 0), dm.BW);
         const int base = a.mask_kind == XGR_MASK_CSR ? a.row_ptr[rb] : 0;
-        if (has_row) p = row_prep(a, r, b, n_live, base, area);
+        if (has_row) p = row_prep<RING>(a, r, b, n_live, base, area);
     };
     // The pick kernel (the only kernel launched after this one) may start at
     // once: before its own wait it touches no global memory, so this kernel
@@ -1389,7 +1401,7 @@ __global__ void __launch_bounds__(kSpThreads, 1) select_rows_kernel(SelectArgs a
     if (a.prep_early) prep();
     griddep_wait();
     if (!a.prep_early) prep();
-    if (has_row) row_run(a, r, b, p, a.keys + (int64_t)r * a.key_cap, area, ring_bar[warp]);
+    if (has_row) row_run<RING>(a, r, b, p, a.keys + (int64_t)r * a.key_cap, area, ring_bar[warp]);
 }
 
 // Phase 2: one CTA per request.  It starts while the rows kernel runs (on the
@@ -1746,24 +1758,35 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
         if (e != cudaSuccess) return e;
         return launch_pdl(select_dense_kernel, dim3(dm.B), dim3(kDnThreads), smem, s, a);
     }
-    // sparse: one launch, sp_parts CTAs per request of R beams, one per warp
-    const int R = std::min(dm.BW, kSpWarps);
+    // sparse: the rows kernel (sp_parts CTAs per request of R beams, one per
+    // warp), then the pick kernel (one CTA per request)
+    // A NODE_BITS row's token list takes its warp's whole area once the row is
+    // streamed, so a long row takes the wide shape's deeper ring.
+    const int sms = a.num_sms > 0 ? a.num_sms : 148;
+    const bool wide = (int64_t)dm.B * ((dm.BW + kRowWarpsWide - 1) / kRowWarpsWide) <= sms ||
+                      (size_t)a.row_stride * 4 > ring_warp_bytes(kRingNarrow);
+    const int R = std::min(dm.BW, wide ? kRowWarpsWide : kRowWarpsNarrow);
     a.sp_rows = R;
     a.sp_parts = (dm.BW + R - 1) / R;
     if (a.head_m < 1 || a.head_m > 16 || (a.head_m & (a.head_m - 1))) return cudaErrorInvalidValue;   // (m + 1 lanes merge)
     if (a.mask_kind != XGR_MASK_CSR && a.mask_kind != XGR_MASK_TRIE_ROWS && a.mask_kind != XGR_MASK_NODE_BITS)
         return cudaErrorInvalidValue;
     if (a.mask_kind != XGR_MASK_CSR && (int64_t)dm.BW * a.row_stride > a.key_cap) return cudaErrorInvalidValue;
-    // a NODE_BITS row's token list takes its warp's ring once the row is streamed
-    if (a.mask_kind == XGR_MASK_NODE_BITS && (size_t)a.row_stride * 4 > kRingWarpBytes) return cudaErrorInvalidValue;
-    const size_t pick_smem = sparse_pick_smem(dm, a.head_m);
-    if (pick_smem > (220u << 10)) return cudaErrorInvalidValue;
-    cudaError_t e = ensure_smem(select_rows_kernel, kRowsSmem);
-    if (e == cudaSuccess) e = ensure_smem(select_pick_kernel, pick_smem);
-    if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)dm.B * a.sp_parts;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    e = launch_pdl(select_rows_kernel, dim3((unsigned)grid), dim3(kSpThreads), kRowsSmem, s, a);
+    const int ring = wide ? kRingWide : kRingNarrow;
+    if (a.mask_kind == XGR_MASK_NODE_BITS && (size_t)a.row_stride * 4 > ring_warp_bytes(ring))
+        return cudaErrorInvalidValue;
+    const size_t rows_smem = (size_t)R * ring_warp_bytes(ring);
+    const size_t pick_smem = sparse_pick_smem(dm, a.head_m);
+    if (pick_smem > (220u << 10)) return cudaErrorInvalidValue;
+    auto *rows_kernel = wide ? select_rows_kernel<kRowWarpsWide, 1, kRingWide>
+                             : select_rows_kernel<kRowWarpsNarrow, 3, kRingNarrow>;
+    cudaError_t e = ensure_smem(rows_kernel, rows_smem);
+    if (e == cudaSuccess) e = ensure_smem(select_pick_kernel, pick_smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(rows_kernel, dim3((unsigned)grid), dim3((wide ? kRowWarpsWide : kRowWarpsNarrow) * 32), rows_smem,
+                   s, a);
     if (e != cudaSuccess) return e;
     return launch_pdl(select_pick_kernel, dim3(dm.B), dim3(kSpThreads), pick_smem, s, a);
 }
