@@ -240,7 +240,22 @@ __device__ __forceinline__ float ex2(float x) {   // 2^x, one MUFU op; tiny resu
     return y;
 }
 
-
+// Packed fp32 pair a * b + c (one instruction for two lanes of arithmetic on
+// sm_100), each element rounded as the scalar fmaf rounds it.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 // query row `row` of a work item -> (request, beam, query head, global row, live)
 struct RowInfo {
@@ -567,13 +582,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         if (!((pm >> e) & 1u)) sv[32 * q2 + e] = -INFINITY;
                 }
             }
+            // row maximum: eight chains of three-input maxima
             float mxp[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mxp[e] = sv[e];
+            for (int e = 0; e < 8; ++e) mxp[e] = fmaxf(sv[e], sv[8 + e]);
 #pragma unroll
-            for (int c = 8; c < 128; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], sv[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                                   fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * cscale;
+            for (int c = 16; c < 128; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mxp[e] = fmax3(mxp[e], sv[c + e], sv[c + 8 + e]);
+            const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]),
+                                   fmaxf(mxp[6], mxp[7])) * cscale;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_used + 8.f) {   // lazy rescaling: keep the old max unless it grew by 2^8
@@ -586,7 +604,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // exponentials, row sum and P (bf16 pairs) into the first 64 columns of
             // the S buffer, from the scores already in registers (masked ones are
             // -inf): piece q's 16 P columns land on scores already read
-            const float neg_m = -m_used;
+            // x = s * scale - m in packed pairs; sums in eight chains
+            const float2 sc2 = make_float2(cscale, cscale), nm2 = make_float2(-m_used, -m_used);
             float sp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) sp[e] = 0.f;
@@ -595,11 +614,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float pw[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(sv[32 * q2 + 2 * e], cscale, neg_m));
-                    const float p1 = ex2(fmaf(sv[32 * q2 + 2 * e + 1], cscale, neg_m));
-                    sp[(2 * e) & 7] += p0;
-                    sp[(2 * e + 1) & 7] += p1;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    const float2 x = ffma2(make_float2(sv[32 * q2 + 2 * e], sv[32 * q2 + 2 * e + 1]), sc2, nm2);
+                    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    sp[(2 * e) & 7] += p.x;
+                    sp[(2 * e + 1) & 7] += p.y;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p.x, p.y);
                     pw[e] = __uint_as_float(*reinterpret_cast<uint32_t *>(&h2));
                 }
                 tmem_st16(tmem + lane_base + s_col + 16 * q2, pw);
