@@ -636,22 +636,6 @@ def measured_traffic(call: str):
         return None
 
 
-def graph_kernel_nodes(g) -> int:
-    """Kernel nodes of a captured CUDA graph: the library kernels one decode launches."""
-    from cuda.bindings import runtime as rt
-    graph = rt.cudaGraph_t(init_value=int(g.raw_cuda_graph()))
-    err, _, n = rt.cudaGraphGetNodes(graph, 0)
-    assert err == rt.cudaError_t.cudaSuccess, err
-    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
-    assert err == rt.cudaError_t.cudaSuccess, err
-    count = 0
-    for nd in nodes[:n]:
-        err, kind = rt.cudaGraphNodeGetType(nd)
-        assert err == rt.cudaError_t.cudaSuccess, err
-        count += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
-    return count
-
-
 def run_gpu(args, w):
     import numpy as np
     import torch
@@ -798,16 +782,23 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     if any(sg.device_status() != 0 for sg in sessions):
         raise RuntimeError("device status set during warm-up")
-    # the graph-based execution of the pages' system level: a whole decode is one graph
-    g_decode = capture(lambda: enqueue_decode(), keep=True)
-    launches_per_decode = graph_kernel_nodes(g_decode)
+    # the graph-based execution of the pages' system level: a whole decode is one
+    # graph, built by the library (xgr_decode_graph_create), each request group's
+    # chain on its own stream
+    decode_graph = xgr.xgr_decode_graph_create(
+        [dict(ctx=sessions[g].ctx, n_requests=Bg, score_flags=flags,
+              q=[inputs[s][0][sl(g)] for s in range(w.S)], k_new=[inputs[s][1][sl(g)] for s in range(w.S)],
+              v_new=[inputs[s][2][sl(g)] for s in range(w.S)], scores=[inputs[s][3][sl(g)] for s in range(w.S)],
+              out=out[sl(g)], lse=lse[sl(g)], parent=par[sl(g)], token=tok[sl(g)], cum=cum[sl(g)],
+              n_out=nout_g[g]) for g in range(G)], w.S)
+    launches_per_decode = xgr.xgr_decode_graph_kernels(decode_graph)
     g_phase = [capture(lambda: enqueue_head(inputs, None))]
     for s in range(1, w.S):
         g_phase.append(capture(lambda s=s: enqueue_att(s, inputs, None)))
         g_phase.append(capture(lambda s=s: enqueue_sel(s, inputs, None)))
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
-        g_decode.replay()
+        xgr.xgr_decode_graph_launch(decode_graph, cur())
     torch.cuda.synchronize()
 
     # ---- timed region: K whole-decode graph replays, L2 flushed before each
@@ -819,7 +810,7 @@ def run_gpu(args, w):
     for i in range(args.steps):
         flush.zero_()
         starts[i].record()
-        g_decode.replay()
+        xgr.xgr_decode_graph_launch(decode_graph, cur())
         ends[i].record()
     torch.cuda.synchronize()
     if world > 1:
@@ -936,7 +927,8 @@ def run_gpu(args, w):
         line["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, items, args.scores)
-    del g_decode, g_phase   # released before the next workload's session
+    xgr.xgr_decode_graph_destroy(decode_graph)
+    del g_phase   # released before the next workload's session
     if world == 1 and not args.no_bw512:
         line["attention_bw512"] = attention_bw512(dev, hbm, tf, src)
     if world == 1 and not args.no_extra:

@@ -307,6 +307,63 @@ xgr_status xgr_beam_topk_noalloc(int32_t n_requests, int32_t beam_width, int32_t
                                  const int32_t *d_cols, int32_t *d_parent, int32_t *d_token,
                                  float *d_cum_out, int32_t *d_n_out, xgr_stream_t stream);
 
+/* ---------------------------------------------------------------- whole-decode graph
+ * xGR page, 2.3 xSchedule: "Graph-based execution" (a decode's device work is
+ * captured in a static graph and dispatched in one go) and "Dynamic batching
+ * and multi-stream" (independent request groups on their own streams).  One
+ * graph runs a whole decode of n_groups request groups, each with its own
+ * context: per group, xgr_begin, then for s = 0 .. steps-1 xgr_build_mask,
+ * xgr_decode_step and xgr_beam_select -- on a stream of its own, forked from
+ * and joined back to the stream the graph is launched on, so one group's
+ * attention may run beside another group's selection (inside a group every
+ * kernel follows the one before through a programmatic dependent launch).
+ *
+ * A group (all device pointers caller-owned and fixed for the graph's life):
+ *   ctx          its context: trie built, the requests' KV prefilled; no two
+ *                groups may share one
+ *   n_requests   xgr_begin's n_requests
+ *   score_flags  XGR_SCORES_LOGPROB or XGR_SCORES_LOGITS
+ *   d_q, d_k_new, d_v_new, d_scores: HOST arrays of `steps` device pointers,
+ *                step s's inputs as xgr_decode_step / xgr_beam_select take
+ *                them (read at creation only; the pointers are baked in)
+ *   d_out, d_lse, d_parent, d_token, d_cum, d_n_out: the step outputs,
+ *                rewritten every step (the last step's remain)
+ * Creation runs the decode once eagerly (planning, launch attributes and
+ * tensor maps are set up then; its results are left in the output buffers),
+ * then captures and instantiates it; every launch re-runs it from xgr_begin on
+ * the inputs' current contents.  Host-side errors of any of the calls above
+ * are returned as they are; XGR_ERR_ARG for a NULL or repeated context, NULL
+ * pointer arrays, n_groups outside [1, 64] or steps < 1.  Each context's host
+ * state afterwards is that of a finished decode (xgr_get_sequences works; a
+ * new decode through the calls above starts with xgr_begin). */
+typedef struct {
+    xgr_ctx *ctx;
+    int32_t n_requests;
+    int32_t score_flags;
+    const void *const *d_q;
+    const void *const *d_k_new;
+    const void *const *d_v_new;
+    const float *const *d_scores;
+    void *d_out;
+    float *d_lse;
+    int32_t *d_parent;
+    int32_t *d_token;
+    float *d_cum;
+    int32_t *d_n_out;
+} xgr_decode_group;
+
+typedef struct xgr_decode_graph xgr_decode_graph;
+
+xgr_status xgr_decode_graph_create(const xgr_decode_group *groups, int32_t n_groups, int32_t steps,
+                                   xgr_decode_graph **out);
+/* Enqueues the whole decode on `stream` (one graph launch). */
+xgr_status xgr_decode_graph_launch(xgr_decode_graph *graph, xgr_stream_t stream);
+/* Kernel launches of one decode (the graph's kernel nodes). */
+xgr_status xgr_decode_graph_kernels(const xgr_decode_graph *graph, int32_t *n_kernels);
+/* Frees the graph (not the contexts or buffers); the caller makes sure no
+ * launch of it is still running. */
+xgr_status xgr_decode_graph_destroy(xgr_decode_graph *graph);
+
 #ifdef __cplusplus
 }
 #endif

@@ -86,6 +86,24 @@ class xgr_mask(ctypes.Structure):
     ]
 
 
+class xgr_decode_group(ctypes.Structure):
+    _fields_ = [
+        ("ctx", ctypes.c_void_p),
+        ("n_requests", ctypes.c_int32),
+        ("score_flags", ctypes.c_int32),
+        ("d_q", ctypes.POINTER(ctypes.c_void_p)),
+        ("d_k_new", ctypes.POINTER(ctypes.c_void_p)),
+        ("d_v_new", ctypes.POINTER(ctypes.c_void_p)),
+        ("d_scores", ctypes.POINTER(ctypes.c_void_p)),
+        ("d_out", ctypes.c_void_p),
+        ("d_lse", ctypes.c_void_p),
+        ("d_parent", ctypes.c_void_p),
+        ("d_token", ctypes.c_void_p),
+        ("d_cum", ctypes.c_void_p),
+        ("d_n_out", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -125,6 +143,10 @@ def lib():
         "xgr_get_sequences": [P, P, P],
         "xgr_device_status": [P, P, ctypes.POINTER(i32)],
         "xgr_beam_topk_noalloc": [i32, i32, i32, i32, P, i32, P, P, P, P, P, P, P, P, P, P],
+        "xgr_decode_graph_create": [ctypes.POINTER(xgr_decode_group), i32, i32, ctypes.POINTER(P)],
+        "xgr_decode_graph_launch": [P, P],
+        "xgr_decode_graph_kernels": [P, ctypes.POINTER(i32)],
+        "xgr_decode_graph_destroy": [P],
         # host-side batch former (include/xgr_sched.h)
         "xgr_cht_create": [i32, ctypes.POINTER(P)],
         "xgr_cht_destroy": [P],
@@ -285,6 +307,44 @@ def xgr_beam_topk_noalloc(n_requests: int, beam_width: int, top_k: int, vocab: i
         n_requests, beam_width, top_k, vocab, _ptr(scores), flags, _ptr(cum), _ptr(n_live),
         _ptr(bits), _ptr(row_ptr), _ptr(cols), _ptr(parent), _ptr(token), _ptr(cum_out),
         _ptr(n_out), _stream(stream)))
+
+
+def xgr_decode_graph_create(groups, steps: int) -> int:
+    """The whole-decode graph of include/xgr.h.  `groups`: one dict per request
+    group with keys ctx, n_requests, score_flags, q, k_new, v_new, scores
+    (sequences of `steps` device buffers) and out, lse, parent, token, cum,
+    n_out (device buffers).  Returns the graph handle."""
+    n = len(groups)
+    arr = (xgr_decode_group * max(n, 1))()
+    keep = []
+    for i, g in enumerate(groups):
+        x = arr[i]
+        x.ctx = g["ctx"]
+        x.n_requests = g["n_requests"]
+        x.score_flags = g["score_flags"]
+        for field in ("q", "k_new", "v_new", "scores"):
+            ptrs = (ctypes.c_void_p * max(1, len(g[field])))(*[_ptr(t) for t in g[field]])
+            keep.append(ptrs)
+            setattr(x, "d_" + field, ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p)))
+        for field in ("out", "lse", "parent", "token", "cum", "n_out"):
+            setattr(x, "d_" + field, _ptr(g[field]))
+    h = ctypes.c_void_p(0)
+    _check("xgr_decode_graph_create", lib().xgr_decode_graph_create(arr, n, steps, ctypes.byref(h)))
+    return h.value
+
+
+def xgr_decode_graph_launch(graph: int, stream=None) -> None:
+    _check("xgr_decode_graph_launch", lib().xgr_decode_graph_launch(graph, _stream(stream)))
+
+
+def xgr_decode_graph_kernels(graph: int) -> int:
+    n = ctypes.c_int32(0)
+    _check("xgr_decode_graph_kernels", lib().xgr_decode_graph_kernels(graph, ctypes.byref(n)))
+    return n.value
+
+
+def xgr_decode_graph_destroy(graph: int) -> None:
+    _check("xgr_decode_graph_destroy", lib().xgr_decode_graph_destroy(graph))
 
 
 def make_config(**kw) -> xgr_config:

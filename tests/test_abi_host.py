@@ -85,3 +85,39 @@ def test_create_without_a_device_fails_cleanly(L):
     h = ctypes.c_void_p(0)
     n = xgr.xgr_workspace_bytes(cfg)
     assert L.xgr_create(ctypes.byref(cfg), 1 << 20, n, ctypes.byref(h)) == xgr.XGR_ERR_CUDA
+
+
+def test_decode_group_struct_matches_the_header(L):
+    """xgr_decode_group as ctypes lays it out: 13 fields, 96 bytes (natural
+    alignment on x86-64: the pointer after the three 32-bit fields is padded to
+    offset 24)."""
+    names = [f[0] for f in xgr.xgr_decode_group._fields_]
+    assert names == ["ctx", "n_requests", "score_flags", "d_q", "d_k_new", "d_v_new", "d_scores",
+                     "d_out", "d_lse", "d_parent", "d_token", "d_cum", "d_n_out"]
+    assert xgr.xgr_decode_group.d_q.offset == 16
+    assert ctypes.sizeof(xgr.xgr_decode_group) == 96
+
+
+def test_decode_graph_rejects_bad_arguments_before_any_device_work(L):
+    h = ctypes.c_void_p(0)
+    arr = (xgr.xgr_decode_group * 2)()
+    assert L.xgr_decode_graph_create(None, 1, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_create(arr, 1, 3, None) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_create(arr, 1, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG   # NULL ctx
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the checks come first
+    ptrs = (ctypes.c_void_p * 3)(1 << 20, 1 << 21, 1 << 22)
+    for g in arr:
+        g.ctx = fake
+        for f in ("d_q", "d_k_new", "d_v_new", "d_scores"):
+            setattr(g, f, ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p)))
+    assert L.xgr_decode_graph_create(arr, 2, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG   # shared ctx
+    assert L.xgr_decode_graph_create(arr, 0, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_create(arr, 65, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_create(arr, 1, 0, ctypes.byref(h)) == xgr.XGR_ERR_ARG
+    arr[0].d_scores = None
+    assert L.xgr_decode_graph_create(arr, 1, 3, ctypes.byref(h)) == xgr.XGR_ERR_ARG
+    assert h.value is None
+    n = ctypes.c_int32(0)
+    assert L.xgr_decode_graph_launch(None, None) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_kernels(None, ctypes.byref(n)) == xgr.XGR_ERR_ARG
+    assert L.xgr_decode_graph_destroy(None) == xgr.XGR_ERR_ARG
