@@ -1273,6 +1273,10 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
     }
     cp_async_wait_all();
     const int total = block_sum_int(c, red_i);   // valid candidates of the request (+ barriers)
+    // the staged rows have landed: the kernel after this one (the next step's
+    // attention, whose prologue prefetches the prompt K/V) may start; any
+    // earlier, that traffic queued ahead of these loads
+    if (!dry) griddep_launch_dependents();
     // per beam: entries relative to the request, the trie child range
     for (int b = tid; b < BW; b += kSpThreads) {
         const bool lv = b < n;
@@ -1427,7 +1431,6 @@ __global__ void __launch_bounds__(kSpThreads, 1) select_pick_kernel(const __grid
         int n_live = 0;
         if (pass == 1) {
             griddep_wait();   // phase 1 of every request has completed
-            griddep_launch_dependents();
             n_live = min(max(a.n_live[r], 0), a.dims.BW);
         }
         select_request(a, r, n_live, smem, hist, scan_w, red_k, sc, red_i, red32, pass == 0);
@@ -1555,6 +1558,10 @@ __device__ __forceinline__ void dense_select(const SelectArgs &a, uint8_t *smem,
     }
     const int total = n > 0 ? block_sum_int(c, red_i) : 0;   // (+ a barrier)
     if (bulk && n > 0 && !mbar_wait(bar, 0, nullptr)) set_status(a.status, XGR_DEV_TIMEOUT);
+    // the kernel after this one (the next step's attention) may start now: its
+    // prologue prefetches the prompt K/V, and started any earlier that traffic
+    // would queue ahead of this row's load
+    if (!dry) griddep_launch_dependents();
     const int want = min(BW, total);
     float lse = 0.f;
     if (a.logits && want > 0) {
@@ -1687,7 +1694,6 @@ __global__ void __launch_bounds__(kDnThreads) select_dense_kernel(const __grid_c
     for (int pass = 0; pass < 2; ++pass) {
         if (pass == 1) {
             griddep_wait();   // the scores and the beam state come from earlier kernels
-            griddep_launch_dependents();
         }
         dense_select(a, smem, sh, pass == 0);
         __syncthreads();   // the pass's shared memory is free again
