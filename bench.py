@@ -185,8 +185,9 @@ def oracle_decode_sample(w, items, sorted_items, requests, scores_mode):
 
 
 def cpu_baseline(w, items, scores_mode, budget_s=20.0):
-    """The oracle on the host cores: whole decodes of requests 0, 1, ... until
-    about budget_s/2 of all-core time, then the same requests with one thread."""
+    """The oracle on the host cores: whole decodes of requests 0, 1, ... (then
+    of the whole batch again) until about budget_s/2 of all-core time, then
+    request 0 with one thread."""
     import oracle
     si = oracle.SortedItems(items, w.V)
     cores = oracle.num_threads()
@@ -199,6 +200,12 @@ def cpu_baseline(w, items, scores_mode, budget_s=20.0):
         cands += c
         reqs.append(r)
         r += 1
+    rounds = 1
+    while secs < budget_s / 2:                      # the whole batch fits: repeat it
+        t, c = oracle_decode_sample(w, items, si, reqs, scores_mode)
+        secs += t
+        cands += c
+        rounds += 1
     single = None
     try:
         oracle.set_num_threads(1)
@@ -208,8 +215,9 @@ def cpu_baseline(w, items, scores_mode, budget_s=20.0):
     finally:
         oracle.set_num_threads(cores)
     return {"value": cands / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"full {w.S}-step decode of {len(reqs)} of {w.B} requests "
-                      f"({cands} candidates in {secs:.2f} s)",
+            "sample": f"full {w.S}-step decode of {len(reqs)} of {w.B} requests"
+                      + (f", {rounds} times" if rounds > 1 else "")
+                      + f" ({cands} candidates in {secs:.2f} s)",
             "single_thread": single}
 
 
