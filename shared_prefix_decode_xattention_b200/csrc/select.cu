@@ -1343,18 +1343,26 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
             const int b = sat[q];
             const uint64_t last = hk[b * m + m - 1];
             const int e0 = max(f.rp[b], 0), e1 = (int)min((int64_t)f.rp[b] + f.rl[b], E);
-            for (int j0 = e0; j0 < e1; j0 += 32) {
-                const int e = j0 + lane;
-                const uint64_t key = e < e1 ? __ldcg(keys + e) : kNoKey;
-                const bool keep = key > last && cut.keep(key);
-                const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                int pos0 = 0;
-                if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
-                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                const int pos = pos0 + __popc(bal & lt);
-                if (keep && pos < scap) {
-                    sk[pos] = key;
-                    se[pos] = e;
+            for (int j0 = e0; j0 < e1; j0 += 128) {   // four loads per lane in flight
+                uint64_t kq[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = j0 + 32 * u + lane;
+                    kq[u] = e < e1 ? __ldcg(keys + e) : kNoKey;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = j0 + 32 * u + lane;
+                    const bool keep = kq[u] > last && cut.keep(kq[u]);
+                    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                    int pos0 = 0;
+                    if (lane == 0 && bal) pos0 = atomicAdd(&cnts[0], __popc(bal));
+                    pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                    const int pos = pos0 + __popc(bal & lt);
+                    if (keep && pos < scap) {
+                        sk[pos] = kq[u];
+                        se[pos] = e;
+                    }
                 }
             }
         }
