@@ -2,8 +2,8 @@
 several request groups, each with its own context and stream, captured once
 and launched as one graph.  Its results must be those of the same decode
 issued call by call -- bit for bit, the kernels being the same -- on every
-launch, for one group and for two groups of the 128-beam workload (whose
-eager decode the parity tests compare with the oracle)."""
+launch, for one, two and four groups of the 128-beam workload (whose eager
+decode the parity tests compare with the oracle), in both score modes."""
 import pytest
 import torch
 
@@ -16,7 +16,8 @@ def _groups(w, G, dev, flags):
     Bg = w.B // G
     wg = workloads.small(w, B=Bg)
     items = workloads.items(w)
-    inputs = [workloads.step_qkv(w, s, dev) + (workloads.step_logits(w, s, dev),) for s in range(w.S)]
+    gen = workloads.step_logits if flags == xgr.XGR_SCORES_LOGITS else workloads.step_logprobs
+    inputs = [workloads.step_qkv(w, s, dev) + (gen(w, s, dev),) for s in range(w.S)]
     groups = []
     for g in range(G):
         sess = Session(config_for(wg), dev)
@@ -63,10 +64,11 @@ def _same(a, b):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("G", [1, 2])
-def test_decode_graph_equals_the_eager_decode(G):
+@pytest.mark.parametrize("G,flags", [(1, xgr.XGR_SCORES_LOGITS), (2, xgr.XGR_SCORES_LOGITS),
+                                     (4, xgr.XGR_SCORES_LOGPROB)])
+def test_decode_graph_equals_the_eager_decode(G, flags):
     w = workloads.WORKLOADS[2]
-    groups = _groups(w, G, "cuda", xgr.XGR_SCORES_LOGITS)
+    groups = _groups(w, G, "cuda", flags)
     want = [_eager(w, g) for g in groups]
     graph = xgr.xgr_decode_graph_create(groups, w.S)
     try:
