@@ -805,6 +805,593 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
+
+// ---------------------------------------------------------------- one-O variant
+// For short items (a few key chunks each) both softmax warpgroups add into one O:
+// that frees TMEM for a third S buffer, so S_{j+3} waits for P_j V_j, issued a
+// whole chunk earlier, and the tensor pipe does not drain between chunks.  A row
+// then has one reference maximum (shared memory), raised lazily -- only when a
+// chunk's max passes it by more than 2^8 -- by the warpgroup that sees that
+// chunk; the other warpgroup takes the new reference (B_DEC) before its next
+// chunk's P, and O is rescaled between the two products.  Long items keep
+// attn_tc_kernel, whose warpgroups never wait for each other.
+namespace one_o {
+
+constexpr uint32_t kOffMref = kOffMisc + 16;  // [128] each row's reference maximum (log2 units)
+constexpr uint32_t kSmemUsed = kOffMref + 512;
+constexpr uint32_t kSmemSpare = kSmemBytes - kSmemUsed;   // room to realign the window
+// TMEM columns: S0 [0,128) S1 [128,256) S2 [256,384) O [384,512); S_j goes to
+// buffer j % 3, and P_j (bf16, two per column) overwrites its first 64 columns
+// once S_j is read.
+constexpr int kSBufs = 3;
+constexpr uint32_t kOCol = 384;
+// P_j written and P_j V_j complete: barriers j % 4.  (With three S buffers a
+// warpgroup may finish chunk j+2 before P_j V_j is issued -- S_{j+2} waits only
+// for P_{j-1} V_{j-1} -- but not chunk j+4, whose S waits for P_{j+1} V_{j+1};
+// and P_{j+4} V_{j+4} cannot complete before S_{j+4}, issued once P_{j+1} V_{j+1}
+// was seen complete: four barriers of each keep every phase polled at most one
+// behind the barrier's current one, so the parity tests are exact.)
+constexpr int kPBars = 4;
+// S_j complete: barrier j % 6, so that each barrier serves one warpgroup and
+// its phases are consumed in order without relying on commit order
+constexpr int kSBars = 6;
+
+// barrier slots (8 bytes each) after kOffBar
+enum { B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_VFULL = B_KEMPTY + kKStages,
+       B_VEMPTY = B_VFULL + kVStages, B_SFULL = B_VEMPTY + kVStages, B_PFULL = B_SFULL + kSBars,
+       B_PVDONE = B_PFULL + kPBars, B_QFULL = B_PVDONE + kPBars, B_DONE = B_QFULL + 1, B_XCH = B_DONE + 1,
+       B_UFULL = B_XCH + 2, B_UEMPTY = B_UFULL + 1, B_DEC = B_UEMPTY + 1, B_COUNT = B_DEC + 2 };
+// B_SFULL: one per chunk index mod 6; B_PFULL, B_PVDONE: one per chunk index
+// mod 4; B_DEC: one per chunk parity (= warpgroup).  B_PVDONE: P_j V_j has completed (O holds every product up to
+// chunk j; S_j's buffer, which held P_j, may take S_{j+3}); B_DEC: chunk j's
+// warpgroup has settled the rows' reference maxima for chunk j (the other
+// warpgroup reads them for chunk j+1); B_DONE: every MMA has completed; B_XCH: the warpgroups' l exchange;
+// B_UFULL: an Unshared chunk is gathered into the U area; B_UEMPTY: its MMAs have
+// completed (the U area may take the next one)
+static_assert(B_COUNT * 8 <= 256, "barrier area");
+
+// The one-O variant (same warps, shared memory and registers as attn_tc_kernel).
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_one_o_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                   const __grid_constant__ CUtensorMap tmq, TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad > kSmemSpare) {   // the dynamic window is expected 1024-aligned; never trap
+        if (threadIdx.x == 0) set_status(a.status, XGR_DEV_TIMEOUT);
+        return;
+    }
+    uint8_t *base = smem_raw + pad;
+    const uint32_t sb = smem_u32(base);
+    const uint32_t bar0 = sb + kOffBar;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(base + kOffMisc);
+    int *abort_flag = reinterpret_cast<int *>(base + kOffMisc + 4);
+
+    const WorkItem it = a.items[blockIdx.x];
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    if (it.flags & 4) {   // zero-fill item: these CTAs run beside the attention on idle SMs
+        griddep_wait();
+        griddep_launch_dependents();
+        const int64_t row0 = ((int64_t)it.r0 * a.dims.BW + it.row_begin) * a.dims.Hq;   // first query row
+        const int64_t n = (int64_t)it.n_rows * a.dims.Hq;
+        uint4 *o = reinterpret_cast<uint4 *>(a.out + row0 * 128);
+        for (int64_t u = tid; u < n * 16; u += kTcThreads) o[u] = make_uint4(0, 0, 0, 0);
+        for (int64_t u = tid; u < n; u += kTcThreads) a.lse[row0 + u] = -INFINITY;
+        return;
+    }
+    const int n_keys = it.key_end - it.key_begin;
+    const int nchunks = (n_keys + kBlockN - 1) / kBlockN;   // Shared-stage chunks
+    const bool final_item = (it.flags & 1) != 0;
+    // Unshared chunks (final items): the tile's beams x (s + 1) tokens, 128 rows each
+    const int T = a.step + 1;
+    const int lb0 = it.row_begin / a.dims.G;
+    const int nbeam = (it.row_begin + it.n_rows - 1) / a.dims.G - lb0 + 1;
+    const int n_u = final_item ? (nbeam * T + kBlockN - 1) / kBlockN : 0;
+    const int nall = nchunks + n_u;
+    const bool q_tma = (it.flags & 2) != 0;   // the Q tile is one TMA box
+    volatile int *abort = abort_flag;
+    const int y0 = it.g * (int)a.kv_tokens + it.kv_off + it.key_begin;
+    // producer lanes: lane 0 streams K chunks, lane 1 V chunks, each on its own ring
+    auto issue_k = [&](int j) {
+        const int st = j % kKStages;
+        mbar_expect_tx(bar(B_KFULL + st), kTile);
+        tma_load_2d(sb + kOffK + st * kTile, &tmk, 0, y0 + j * kBlockN, bar(B_KFULL + st));
+        tma_load_2d(sb + kOffK + st * kTile + kHalf, &tmk, 64, y0 + j * kBlockN, bar(B_KFULL + st));
+    };
+    auto issue_v = [&](int j) {
+        const int st = j % kVStages;
+        mbar_expect_tx(bar(B_VFULL + st), kTile);
+        tma_load_2d(sb + kOffV + st * kTile, &tmv, 0, y0 + j * kBlockN, bar(B_VFULL + st));
+        tma_load_2d(sb + kOffV + st * kTile + kHalf, &tmv, 64, y0 + j * kBlockN, bar(B_VFULL + st));
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < kKStages; ++s) {
+                mbar_init(bar(B_KFULL + s), 1);
+                mbar_init(bar(B_KEMPTY + s), 1);
+            }
+            for (int s = 0; s < kVStages; ++s) {
+                mbar_init(bar(B_VFULL + s), 1);
+                mbar_init(bar(B_VEMPTY + s), 1);
+            }
+            for (int h = 0; h < kPBars; ++h) {
+                mbar_init(bar(B_PFULL + h), kGroupThreads);
+                mbar_init(bar(B_PVDONE + h), 1);
+            }
+            for (int h = 0; h < 2; ++h) {
+                mbar_init(bar(B_XCH + h), kGroupThreads);
+                mbar_init(bar(B_DEC + h), kGroupThreads);
+            }
+            for (int b = 0; b < kSBars; ++b) mbar_init(bar(B_SFULL + b), 1);
+            mbar_init(bar(B_QFULL), q_tma ? 1 : kSoftmaxThreads);
+            mbar_init(bar(B_DONE), 1);
+            mbar_init(bar(B_UFULL), kGatherLanes);
+            mbar_init(bar(B_UEMPTY), 1);
+            *abort_flag = 0;
+            fence_mbar_init();
+        }
+        __syncwarp();
+        // The prompt's first K / V chunks stream in while the kernel before this
+        // one finishes: the prompt (and suffix) KV store is written only by the
+        // prefill copies, which completed before any decode kernel started.
+        if (lane == 0)
+            for (int j = 0; j < min(nchunks, kKStages); ++j) issue_k(j);
+        if (lane == 1)
+            for (int j = 0; j < min(nchunks, kVStages); ++j) issue_v(j);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_holder)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // Everything above touches only this CTA's shared and tensor memory, the
+    // plan (written before any decode kernel) and the prompt KV store; from
+    // here on the kernel reads what the kernels before it wrote (the beam
+    // state, this step's inputs).
+    griddep_wait();
+    griddep_launch_dependents();
+    if (warp == 0 && lane == 0 && q_tma) {   // Q streams in before the block-wide setup barrier
+        const int G = a.dims.G;
+        const int z = it.r0 * a.dims.BW + it.row_begin / G;
+        mbar_expect_tx(bar(B_QFULL), kTile);
+        tma_load_3d(sb + kOffQ, &tmq, 0, it.g * G, z, bar(B_QFULL));
+        tma_load_3d(sb + kOffQ + kHalf, &tmq, 64, it.g * G, z, bar(B_QFULL));
+    }
+    // softmax threads stage the Q tile meanwhile: 16 consecutive threads read one
+    // 256-byte row (coalesced) and write it in the swizzled K-major layout
+    if (warp >= 2 && warp < kGatherWarp && !q_tma) {
+        const int ts = tid - 64;
+        uint4 qv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = ts + kSoftmaxThreads * k;
+            const RowInfo qi = row_info(a, it, idx >> 4);
+            qv[k] = qi.valid ? reinterpret_cast<const uint4 *>(a.q + qi.gid * 128)[idx & 15]
+                             : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int idx = ts + kSoftmaxThreads * k;
+            *reinterpret_cast<uint4 *>(base + kOffQ + sw128_off(idx >> 4, idx & 15)) = qv[k];
+        }
+    }
+    if (warp >= 2 && warp < 6) reinterpret_cast<float *>(base + kOffMref)[tid - 64] = -INFINITY;
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producers
+        if (lane == 0) {
+            int n_issued = min(nchunks, kKStages);
+            for (int j = kKStages; j < nchunks && n_issued == j; ++j) {
+                if (!mbar_wait(bar(B_KEMPTY + j % kKStages), ((j / kKStages) - 1) & 1, abort)) break;
+                issue_k(j);
+                ++n_issued;
+            }
+            if (*abort)   // let the copies in flight land before the CTA exits
+                for (int j = max(0, n_issued - kKStages); j < n_issued; ++j)
+                    mbar_wait(bar(B_KFULL + j % kKStages), (j / kKStages) & 1, nullptr);
+        } else if (lane == 1) {
+            int n_issued = min(nchunks, kVStages);
+            for (int j = kVStages; j < nchunks && n_issued == j; ++j) {
+                if (!mbar_wait(bar(B_VEMPTY + j % kVStages), ((j / kVStages) - 1) & 1, abort)) break;
+                issue_v(j);
+                ++n_issued;
+            }
+            if (*abort)
+                for (int j = max(0, n_issued - kVStages); j < n_issued; ++j)
+                    mbar_wait(bar(B_VFULL + j % kVStages), (j / kVStages) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // Chunk j belongs to warpgroup h = j % 2: S_j goes to TMEM buffer j % 3,
+        // P_j is read from that buffer, and every P_j V_j accumulates into O in
+        // chunk order.  Order of issue: S_0 .. S_2, then whichever is ready:
+        // S_ns (P_{ns-3} V_{ns-3}, which read its buffer, complete and K_ns
+        // landed) or P_j V_j (P_j written, V_j landed).
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
+            // chunk j < nchunks: a Shared chunk in the K / V rings; j >= nchunks: an
+            // Unshared chunk in the U area (its K and V land together on B_UFULL)
+            auto k_ready = [&](int j, bool block) -> bool {
+                const uint32_t b = j < nchunks ? bar(B_KFULL + j % kKStages) : bar(B_UFULL);
+                const uint32_t ph = j < nchunks ? (j / kKStages) & 1 : (j - nchunks) & 1;
+                return block ? mbar_wait(b, ph, abort) : mbar_test(b, ph);
+            };
+            auto issue_s = [&](int j) {   // S_j = Q K_j^T into TMEM buffer j % 3
+                fence_after_sync();
+                const uint32_t kq = sb + kOffQ;
+                const uint32_t kk = j < nchunks ? sb + kOffK + (j % kKStages) * kTile : sb + kOffU;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
+                    umma_bf16(tmem + (uint32_t)(j % kSBufs) * 128u, umma_desc(kq + off, 16, 1024),
+                              umma_desc(kk + off, 16, 1024), idS, k > 0);
+                }
+                umma_commit(bar(B_SFULL + j % kSBars));
+                if (j < nchunks) umma_commit(bar(B_KEMPTY + j % kKStages));
+            };
+            bool ok = mbar_wait(bar(B_QFULL), 0, abort);
+            int ns = 0;   // the next S to issue
+            for (; ok && ns < min(nall, kSBufs); ++ns) {
+                ok = k_ready(ns, true);
+                if (ok) issue_s(ns);
+            }
+            uint32_t idle = 0;
+            for (int j = 0; ok && j < nall;) {
+                bool progress = false;
+                if (ns < nall && mbar_test(bar(B_PVDONE + (ns - kSBufs) % kPBars), ((ns - kSBufs) / kPBars) & 1) &&
+                    k_ready(ns, false)) {
+                    issue_s(ns++);
+                    progress = true;
+                }
+                const int sv = j % kVStages;
+                const bool v_ready = j < nchunks ? mbar_test(bar(B_VFULL + sv), (j / kVStages) & 1)
+                                                 : mbar_test(bar(B_UFULL), (j - nchunks) & 1);
+                if (!(mbar_test(bar(B_PFULL + j % kPBars), (j / kPBars) & 1) && v_ready)) {
+                    if (progress) {
+                        idle = 0;
+                    } else if (++idle >= kSpinLimit) {
+                        *abort = 1;
+                        ok = false;
+                    } else if ((idle & 255) == 0 && *abort) {
+                        ok = false;
+                    }
+                    continue;
+                }
+                idle = 0;
+                fence_after_sync();
+                const uint32_t kv = j < nchunks ? sb + kOffV + sv * kTile : sb + kOffU + kTile;
+                const uint32_t pcol = (uint32_t)(j % kSBufs) * 128u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)   // P_j: 16 keys = 8 TMEM columns per MMA
+                    umma_bf16_ts(tmem + kOCol, tmem + pcol + 8u * k, umma_desc(kv + (uint32_t)k * 2048u, kHalf, 1024),
+                                 idPV, (k > 0 || j > 0) ? 1u : 0u);
+                umma_commit(bar(B_PVDONE + j % kPBars));
+                umma_commit(j < nchunks ? bar(B_VEMPTY + sv) : bar(B_UEMPTY));
+                ++j;
+            }
+            // arrives once every MMA issued above has completed (TMEM final / free)
+            umma_commit(bar(B_DONE));
+            if (*abort) mbar_wait(bar(B_DONE), 0, nullptr);
+        }
+    } else if (warp < kGatherWarp) {
+        // ------------------------------------------------------------ softmax
+        // Warpgroup `half` owns the chunks j with j % 2 == half, whole rows: thread
+        // `row` reads TMEM lane `row` of S_j's buffer and writes row `row` of P_j
+        // over it.  Both warpgroups' P_j V_j add into the one O, so each row has
+        // one reference maximum (shared memory), raised lazily -- only when a
+        // chunk's max passes it by 2^8 -- by the warpgroup that sees the chunk;
+        // the other warpgroup waits for that decision (B_DEC) before its next
+        // chunk's P, and O is rescaled between P_{j-1} V_{j-1} and P_j V_j.
+        // Each warpgroup keeps its own row sum l relative to the reference it
+        // last used; at the end the two sums meet, and thread (row, half)
+        // handles head-dim columns [64*half, 64*half + 64).
+        const int half = (warp - 2) >> 2;
+        const int row = 32 * (warp & 3) + lane;
+        bool ok = true;
+        if (!q_tma) {
+            fence_async_smem();
+            mbar_arrive(bar(B_QFULL));
+        }
+
+        const RowInfo ri = row_info(a, it, row);
+        const float cscale = kLog2e * rsqrtf(128.f);
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t col0 = (uint32_t)(64 * half);
+        float my_ref = -INFINITY, l = 0.f;   // the reference l is relative to; this warpgroup's row sum
+        float *mref = reinterpret_cast<float *>(base + kOffMref);   // [128] the rows' shared references
+        const Dims dm = a.dims;
+        const bool live = ri.valid && ri.b < a.n_live[ri.r];
+        // Unshared chunks: this row keeps columns [u_lo, u_lo + T) of the block-
+        // diagonal U rows -- its beam's tokens -- where the token's slot is valid
+        // (bit i of vmask; this step's own token when the beam is live)
+        uint32_t vmask = 0;
+        const int u_lo = ((it.row_begin + row) / dm.G - lb0) * T;
+        if (final_item && live) {
+            const int64_t beam_row = (int64_t)ri.r * dm.BW + ri.b;
+            vmask = 1u << a.step;
+            for (int i = 0; i < a.step; ++i) {
+                const int sl = a.st.anc[beam_row * dm.S + i];
+                if (sl >= 0 && sl < dm.BW) vmask |= 1u << i;
+                else if (ri.hg == 0 && half == 0) set_status(a.status, XGR_DEV_INDEX);
+            }
+        }
+        for (int j = half; ok && j < nall; j += 2) {
+            const uint32_t s_col = (uint32_t)(j % kSBufs) * 128u;   // S_j's buffer
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + j % kSBars), (j / kSBars) & 1, abort));
+            if (!ok) break;
+            fence_after_sync();
+            const int nvalid = n_keys - j * kBlockN;   // keys of the chunk inside the range
+            const bool is_u = j >= nchunks;            // an Unshared chunk
+            const int c0 = u_lo - kBlockN * (j - nchunks);   // (is_u) the row's first column in it
+            // Masked chunks (an Unshared chunk: only this row's own tokens count;
+            // the range's last chunk: keys past its end do not) keep the
+            // columns of a 32-bit mask per 32-column piece
+            const bool masked = is_u || nvalid < kBlockN;
+            auto piece_mask = [&](int q2) -> uint32_t {
+                if (is_u) {   // the row's valid tokens (vmask) start at column c0
+                    const int off = c0 - 32 * q2;
+                    return off >= 32 || off <= -32 ? 0u : off >= 0 ? vmask << off : vmask >> -off;
+                }
+                const int nv = nvalid - 32 * q2;
+                return nv >= 32 ? ~0u : nv <= 0 ? 0u : (1u << nv) - 1u;
+            };
+            // the chunk's 128 scores in one TMEM read (P_j then overwrites them)
+            float sv[128];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) tmem_ld32(tmem + lane_base + s_col + 32 * q2, sv + 32 * q2);
+            tmem_wait_ld();
+            if (masked) {
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const uint32_t pm = piece_mask(q2);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((pm >> e) & 1u)) sv[32 * q2 + e] = -INFINITY;
+                }
+            }
+            // row maximum: eight chains of three-input maxima
+            float mxp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxp[e] = fmaxf(sv[e], sv[8 + e]);
+#pragma unroll
+            for (int c = 16; c < 128; c += 16)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mxp[e] = fmax3(mxp[e], sv[c + e], sv[c + 8 + e]);
+            const float mx = fmax3(fmax3(mxp[0], mxp[1], mxp[2]), fmax3(mxp[3], mxp[4], mxp[5]),
+                                   fmaxf(mxp[6], mxp[7])) * cscale;
+            // the rows' references as chunk j-1's warpgroup left them
+            if (j > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DEC + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort));
+            if (!ok) break;
+            const float ref = mref[row];
+            if (ref != my_ref) {   // raised by the other warpgroup: l follows (l is 0 while my_ref is -inf)
+                l *= ex2(my_ref - ref);
+                my_ref = ref;
+            }
+            const bool grow = mx > my_ref + 8.f;   // lazy: a new reference only when the max grew by 2^8
+            const float alpha = grow ? ex2(my_ref - mx) : 1.f;
+            if (grow) {
+                my_ref = mx;
+                mref[row] = mx;
+            }
+            mbar_arrive(bar(B_DEC + (j & 1)));   // (releases the reference for chunk j+1)
+            // exponentials, row sum and P (bf16 pairs) into the first 64 columns of
+            // the S buffer, from the scores already in registers (masked ones are
+            // -inf; a row masked in every chunk so far has a -inf reference and P 0):
+            // piece q's 16 P columns land on scores already read
+            const float nm = my_ref == -INFINITY ? 0.f : -my_ref;
+            // x = s * scale - m in packed pairs; sums in eight chains
+            const float2 sc2 = make_float2(cscale, cscale), nm2 = make_float2(nm, nm);
+            float sp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                float pw[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float2 x = ffma2(make_float2(sv[32 * q2 + 2 * e], sv[32 * q2 + 2 * e + 1]), sc2, nm2);
+                    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    sp[(2 * e) & 7] += p.x;
+                    sp[(2 * e + 1) & 7] += p.y;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p.x, p.y);
+                    pw[e] = __uint_as_float(*reinterpret_cast<uint32_t *>(&h2));
+                }
+                tmem_st16(tmem + lane_base + s_col + 16 * q2, pw);
+            }
+            if (__any_sync(0xffffffffu, grow && j > 0)) {
+                // O *= alpha on the rows whose reference rose, once every product
+                // of the old reference (up to P_{j-1} V_{j-1}) is in O and before
+                // P_j V_j adds in
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(bar(B_PVDONE + (j - 1) % kPBars), ((j - 1) / kPBars) & 1, abort));
+                if (!ok) break;
+                fence_after_sync();
+                const float f = grow ? alpha : 1.f;
+#pragma unroll 1
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + q2 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= f;
+                    tmem_st32(tmem + lane_base + kOCol + q2 * 32, o);
+                }
+            }
+            l = l * alpha + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
+            tmem_wait_st();   // P_j (and a rescaled O) in TMEM before the MMA warp reads them
+            fence_before_sync();
+            mbar_arrive(bar(B_PFULL + j % kPBars));
+        }
+        // every MMA done: O is final, the S buffers free
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, abort));
+        if (ok) {
+            fence_after_sync();
+            // the warpgroups swap (reference, l): the larger reference is the row's
+            // last, the one O is relative to; thread (row, half) then writes
+            // head-dim columns [64*half, 64*half + 64) of O
+            float2 *xl = reinterpret_cast<float2 *>(base + kOffV);   // [2][128]; V is consumed
+            xl[half * 128 + row] = make_float2(my_ref, l);
+            mbar_arrive(bar(B_XCH + half));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_XCH + (half ^ 1)), 0, abort));
+            const float2 other = xl[(half ^ 1) * 128 + row];
+            const float m0 = half == 0 ? my_ref : other.x, l0 = half == 0 ? l : other.y;
+            const float m1 = half == 0 ? other.x : my_ref, l1 = half == 0 ? other.y : l;
+            const float M = fmaxf(m0, m1);
+            // a sum relative to a -inf reference is 0 (no chunk of the row had a key)
+            const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+            const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+            const float l_row = l0 * f0 + l1 * f1;
+            if (ok) {
+#pragma unroll 1
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_base + kOCol + col0 + 32 * q2, o);
+                    tmem_wait_ld();
+                    const uint32_t c0 = col0 + 32 * q2;
+                    if (!final_item) {
+                        if (live) {
+                            float *dst = a.part.o + ((int64_t)it.slot * a.part.rows + ri.gid) * 128 + c0;
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4 *>(dst + e) =
+                                    make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+                        }
+                    } else if (ri.valid) {
+                        // final: O / l in bf16; dead rows 0
+                        const float inv = live ? 1.f / l_row : 0.f;
+                        uint4 *dst = reinterpret_cast<uint4 *>(a.out + ri.gid * 128 + c0);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float v0 = live ? o[8 * c + 2 * e] * inv : 0.f;
+                                const float v1 = live ? o[8 * c + 2 * e + 1] * inv : 0.f;
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                                w4[e] = *reinterpret_cast<uint32_t *>(&h2);
+                            }
+                            dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    }
+                }
+                if (half == 0) {
+                    if (!final_item) {
+                        if (live) a.part.ml[(int64_t)it.slot * a.part.rows + ri.gid] = make_float2(M, l_row);
+                    } else if (ri.valid) {   // LSE = m + log2(l) in natural log; dead rows -inf
+                        a.lse[ri.gid] = live ? (M + __log2f(l_row)) * kLn2 : -INFINITY;
+                    }
+                }
+            }
+        }
+    } else if (n_u > 0) {
+        // ------------------------------------------------------------ gather
+        {
+            // ---- Unshared stage: gather the tile's beams' own k / v rows of steps
+            // 0..s into the U area, one 128-row chunk at a time (row u: token u % T
+            // of tile beam u / T), in the canonical swizzled layout; rows of dead
+            // beams, bad slots and the tail are zero.  This step's rows are also
+            // appended to the pool at slot (s, b).
+            const int gl = lane;
+            const Dims dm = a.dims;
+            const int s_now = a.step;
+            const int64_t pool_step = (int64_t)a.Bcap * dm.BW * dm.Hkv * 128;
+            for (int q = 0; q < n_u; ++q) {
+                if (q > 0 && !mbar_wait(bar(B_UEMPTY), (q - 1) & 1, abort)) break;
+                // this lane's rows u = gl + k * kGatherLanes: their request and beam,
+                // then every index they need, then the copies -- each stage's loads
+                // all in flight together
+                constexpr int kRowsPerLane = (kBlockN + kGatherLanes - 1) / kGatherLanes;
+                int rr[kRowsPerLane], bb[kRowsPerLane], ii[kRowsPerLane];
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes, ug = kBlockN * q + u, lb = ug / T;
+                    ii[k] = ug % T;
+                    rr[k] = -1;
+                    bb[k] = -1;
+                    if (u < kBlockN && lb < nbeam) {
+                        const int lbs = lb0 + lb;   // beam index within the segment's rows / G
+                        bb[k] = lbs % a.nb;
+                        rr[k] = it.n_members == 1 ? it.r0 : a.members[it.member_off + lbs / a.nb];
+                    }
+                }
+                int nl[kRowsPerLane], sl[kRowsPerLane];
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    nl[k] = rr[k] >= 0 ? a.n_live[rr[k]] : 0;
+                    sl[k] = (rr[k] >= 0 && ii[k] < s_now)
+                                ? a.st.anc[((int64_t)rr[k] * dm.BW + bb[k]) * dm.S + ii[k]] : -1;
+                }
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes;
+                    if (u >= kBlockN) continue;
+                    const __nv_bfloat16 *sk = nullptr, *sv = nullptr;
+                    if (rr[k] >= 0 && bb[k] < nl[k]) {
+                        const int64_t brow = (int64_t)rr[k] * dm.BW + bb[k];
+                        if (ii[k] == s_now) {
+                            sk = a.k_new + (brow * dm.Hkv + it.g) * 128;
+                            sv = a.v_new + (brow * dm.Hkv + it.g) * 128;
+                        } else if (sl[k] >= 0 && sl[k] < dm.BW) {
+                            const int64_t prow = (brow - bb[k] + sl[k]) * dm.Hkv + it.g;
+                            sk = a.pool_k + ii[k] * pool_step + prow * 128;
+                            sv = a.pool_v + ii[k] * pool_step + prow * 128;
+                        }
+                    }
+                    const uint32_t dk = sb + kOffU, dv = sb + kOffU + kTile;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        if (sk) {
+                            cp_async16(dk + sw128_off(u, c), sk + 8 * c);
+                            cp_async16(dv + sw128_off(u, c), sv + 8 * c);
+                        } else {
+                            *reinterpret_cast<uint4 *>(base + kOffU + sw128_off(u, c)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(base + kOffU + kTile + sw128_off(u, c)) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                cp_async_wait_all();
+                // this step's k / v of the gathered live beams -> pool slot (s, b)
+#pragma unroll
+                for (int k = 0; k < kRowsPerLane; ++k) {
+                    const int u = gl + k * kGatherLanes;
+                    if (u >= kBlockN || rr[k] < 0 || ii[k] != s_now || bb[k] >= nl[k]) continue;
+                    const int64_t orow = ((int64_t)rr[k] * dm.BW + bb[k]) * dm.Hkv + it.g;
+                    uint4 *pk = reinterpret_cast<uint4 *>(a.pool_k + s_now * pool_step + orow * 128);
+                    uint4 *pv = reinterpret_cast<uint4 *>(a.pool_v + s_now * pool_step + orow * 128);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        pk[c] = *reinterpret_cast<const uint4 *>(base + kOffU + sw128_off(u, c));
+                        pv[c] = *reinterpret_cast<const uint4 *>(base + kOffU + kTile + sw128_off(u, c));
+                    }
+                }
+                fence_async_smem();   // the gathered rows are visible to the tensor cores
+                mbar_arrive(bar(B_UFULL));
+            }
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    if (*abort && tid == 0) set_status(a.status, XGR_DEV_TIMEOUT);
+    if (warp == 1) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace one_o
+
 }  // namespace
 
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -847,16 +1434,14 @@ cudaError_t make_q_tensor_map(CUtensorMap *map, const void *q, int64_t beam_rows
 
 namespace {
 
-cudaError_t launch_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
+template <class K>
+cudaError_t launch_tc(K kernel, bool &attr, const CUtensorMap &tmk, const CUtensorMap &tmv, const CUtensorMap &tmq,
                       const TcArgs &a, int n_items, cudaStream_t st) {
-    static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
+        e = cudaFuncGetAttributes(&fa, kernel);
         if (e != cudaSuccess) return e;
         if (fa.maxThreadsPerBlock < kTcThreads) {
             debug_log("attn_tc: %d registers/thread allow only %d threads per block", fa.numRegs,
@@ -865,7 +1450,7 @@ cudaError_t launch_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const CUte
         }
         attr = true;
     }
-    return launch_pdl(attn_tc_kernel, dim3(n_items), dim3(kTcThreads), kSmemBytes, st, tmk, tmv, tmq, a);
+    return launch_pdl(kernel, dim3(n_items), dim3(kTcThreads), kSmemBytes, st, tmk, tmv, tmq, a);
 }
 
 }  // namespace
@@ -874,7 +1459,9 @@ cudaError_t launch_attn_tc(const CUtensorMap &tmk, const CUtensorMap &tmv, const
                            const TcArgs &a, int n_items, cudaStream_t st) {
     if (n_items <= 0) return cudaSuccess;
     if (a.step + 1 > kMaxSteps) return cudaErrorInvalidValue;   // Unshared tokens of a beam
-    return launch_tc(tmk, tmv, tmq, a, n_items, st);
+    static bool attr_two = false, attr_one = false;
+    return a.shared_o ? launch_tc(one_o::attn_tc_one_o_kernel, attr_one, tmk, tmv, tmq, a, n_items, st)
+                      : launch_tc(attn_tc_kernel, attr_two, tmk, tmv, tmq, a, n_items, st);
 }
 
 }  // namespace xgr

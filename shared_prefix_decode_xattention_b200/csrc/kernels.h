@@ -43,6 +43,8 @@ struct TcArgs {
     BeamState st;
     int Bcap;
     int step;
+    int shared_o;                  // one O for both softmax warpgroups and three S buffers (the
+                                   //   launch's items are short), else an O per warpgroup
 };
 // 2-D tensor map over a [rows][128] bf16 store, 64 x 128 boxes, 128-byte swizzle.
 cudaError_t make_kv_tensor_map(CUtensorMap *map, const void *base, int64_t rows);

@@ -25,6 +25,9 @@ constexpr int kMinChunk = 256;     // fewest keys per split-K work item
 // the separate merge kernel that split items need, in key units of the
 // tensor-core loop (one more dependent launch plus a few round trips)
 constexpr double kMergeKeys = 768.0;
+// most key chunks per tensor-core item (on average over a launch) for the
+// one-O variant of the kernel
+constexpr int64_t kSharedOChunks = 12;
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -167,6 +170,7 @@ struct xgr_ctx {
     int n_small[2] = {0, 0};   // small-row work items of each plan (then n_tc[] tensor-core ones)
     int n_tc[2] = {0, 0};
     int n_unfused[2] = {0, 0};   // requests the merge kernel still has to finish
+    int tc_shared[2] = {0, 0};   // the tensor-core launch takes the one-O variant (short items)
     bool has_tc = false;       // tensor-core Shared stage available (D = 128, tensor maps built)
     CUtensorMap tmk, tmv;
     CUtensorMap tmq;             // Q tensor map of the last decode step, re-encoded when q or B changes
@@ -354,6 +358,20 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         return XGR_ERR_CUDA;
     c->n_small[which] = (int)items_small.size();
     c->n_tc[which] = (int)items_tc.size();
+    // Short items (few key chunks each) run the one-O variant of the
+    // tensor-core kernel (three S buffers: the tensor pipe does not drain
+    // between chunks); long ones keep an O per softmax warpgroup, whose
+    // warpgroups never wait for each other (measured: 8-chunk items faster
+    // with one O, 16- to 128-chunk items slower).
+    {
+        int64_t chunks = 0, n = 0;
+        for (const WorkItem &it : items_tc)
+            if (!(it.flags & 4)) {
+                chunks += (it.key_end - it.key_begin + 127) / 128;
+                ++n;
+            }
+        c->tc_shared[which] = n > 0 && chunks <= kSharedOChunks * n;
+    }
     c->n_unfused[which] = unfused;
     return XGR_OK;
 }
@@ -666,6 +684,7 @@ xgr_status xgr_decode_step(xgr_ctx *c, int32_t step, const void *d_q, const void
         ta.st = c->st;
         ta.Bcap = c->cfg.max_requests;
         ta.step = step;
+        ta.shared_o = c->tc_shared[which];
         // Q tiles of single-request items are one TMA box: D x (query heads of
         // one kv head) x (128 / G beams) over q viewed as [B*BW][Hq][D]
         const int64_t q_rows = (int64_t)c->dims.B * c->cfg.beam_width;
