@@ -486,6 +486,89 @@ def prefix_batches(dev, hbm, tf, src):
     return out
 
 
+def batch_formation(dev, src, batch=16, chunk=256):
+    """Feather's batching on the kernel side (Feather page, "Methodology", 1.
+    Chunked Hash Tree, and "Results"): the 64 requests of the prefix-shared
+    workload (4 prompt families of 16; 8192-token family prefixes, private
+    suffixes of 256-2048 tokens) arrive in a shuffled order.  The batches the
+    tree forms from their token ids are timed against batches of 16 consecutive
+    arrivals.  A batch is one context: each family it holds is one shared KV
+    segment (loaded once, linked by the batch's other members of that family),
+    each request adds its suffix; one decode step per batch, one graph each,
+    the L2 flushed before each; the figure is the sum over the batches."""
+    import numpy as np
+    import torch
+    import workloads
+    from shared_prefix_decode_xattention_b200 import xgr
+    from shared_prefix_decode_xattention_b200.sched import ChunkedHashTree
+    from shared_prefix_decode_xattention_b200.session import Session
+    w = workloads.WORKLOADS[4]
+    lens, suf = workloads.prompt_lengths(w), workloads.suffix_lengths(w)
+    rng = np.random.default_rng(4242)
+    fam = [rng.integers(0, 32000, size=int(lens[g])) for g in range(w.n_shared)]
+    toks = [np.concatenate([fam[w.shared_id(r)], rng.integers(0, 32000, size=int(suf[r]))])
+            for r in range(w.B)]
+    arrivals = [int(r) for r in np.random.default_rng(7).permutation(w.B)]
+    tree = ChunkedHashTree(chunk)
+    for r in arrivals:
+        tree.insert(r, toks[r])
+    formed = tree.form_batches(batch, 1)
+    tree.close()
+    for members, shared in formed:   # each batch shares its family's whole prefix
+        if shared * chunk != int(lens[w.shared_id(members[0])]):
+            raise RuntimeError("the tree's batches do not share their whole prefix")
+    batchings = (("tree", [list(m) for m, _ in formed]),
+                 ("arrival_order", [arrivals[i:i + batch] for i in range(0, w.B, batch)]))
+    q, kn, vn = workloads.step_qkv(w, 0, dev)
+    fam_kv = {g: workloads.shared_kv(w, g, dev) for g in range(w.n_shared)}
+    cur = torch.cuda.current_stream
+    out = {}
+    for kind, batches in batchings:
+        ms = 0.0
+        n_prefix = 0
+        status = 0
+        for members in batches:
+            n = len(members)
+            fams = sorted({w.shared_id(r) for r in members})
+            kv_tokens = sum(int(lens[g]) for g in fams) + sum(int(suf[r]) for r in members)
+            cfg = xgr.make_config(max_requests=n, max_shared=len(fams), kv_tokens=kv_tokens,
+                                  beam_width=1, top_k=1, steps=1, n_q_heads=w.Hq, n_kv_heads=w.Hkv,
+                                  head_dim=w.D, vocab=0, max_items=0, max_fanout=0, max_partials=0)
+            sess = Session(cfg, dev)
+            for sid, g in enumerate(fams):
+                idx = [i for i, r in enumerate(members) if w.shared_id(r) == g]
+                sess.prefill(idx[0], sid, *fam_kv[g])
+                for i in idx[1:]:
+                    sess.link(i, sid)
+            for i, r in enumerate(members):
+                k, v = workloads.suffix_kv(w, r, dev)
+                sess.prefill(i, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+            sel = torch.tensor(members, device=dev)
+            qb, knb, vnb = q[sel].contiguous(), kn[sel].contiguous(), vn[sel].contiguous()
+            o = torch.empty((n, 1, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+            lse = torch.empty((n, 1, w.Hq), dtype=torch.float32, device=dev)
+            sess.begin(n)
+
+            def step():
+                sess.begin(n, cur())
+                sess.decode_step(0, qb, knb, vnb, o, lse, cur())
+
+            ms += _timed_graph(step, dev)
+            status |= sess.device_status()
+            sess.close()
+            n_prefix += len(fams)
+        prefix_bytes = n_prefix * 2 * w.Hkv * int(lens[0]) * w.D * 2
+        out[kind] = {"ms": ms, "batches": len(batches), "prefix_segments": n_prefix,
+                     "prefix_bytes_read": prefix_bytes, "device_status": status}
+    out["time_ratio_arrival_over_tree"] = out["arrival_order"]["ms"] / out["tree"]["ms"]
+    out["workload"] = ("prefix-shared-llm-decode: 64 requests in a shuffled arrival order, batches of 16: "
+                       "Chunked Hash Tree (256-token chunks) against consecutive arrivals")
+    out["context"] = ("Feather reports about 2x throughput for homogeneous batches (Feather page, Results); "
+                      "here arrival-order batches still share a prefix among their members of one family")
+    out["peak_source"] = src
+    return out
+
+
 def long_history(dev, hbm, tf, src, reps=3):
     """The long-history ragged workload (128 requests, prompts of 2048-16384
     tokens, 256 beams, Hq 32 / Hkv 4, D 128, V 16384, logits) at step 1: the
@@ -944,6 +1027,7 @@ def run_gpu(args, w):
     if world == 1 and not args.no_extra:
         line["per_beam_baseline"] = per_beam_baseline(dev, hbm, src)
         line["prefix_batches"] = prefix_batches(dev, hbm, tf, src)
+        line["batch_formation"] = batch_formation(dev, src)
         line["long_history"] = long_history(dev, hbm, tf, src)
     # the Shared stage's tensor throughput per workload (the stage is a dense
     # contraction; its tensor fraction is what bounds it at 128+ beams)

@@ -25,8 +25,8 @@ constexpr int kMinChunk = 256;     // fewest keys per split-K work item
 // the separate merge kernel that split items need, in key units of the
 // tensor-core loop (one more dependent launch plus a few round trips)
 constexpr double kMergeKeys = 768.0;
-// most key chunks per tensor-core item (on average over a launch) for the
-// one-O variant of the kernel
+// most key chunks of any tensor-core item of a launch that runs the one-O
+// variant of the kernel
 constexpr int64_t kSharedOChunks = 12;
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
@@ -264,6 +264,29 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         return best;
     };
     const int64_t f_tc = pick_split(true), f_small = pick_split(false);
+    // Segments of very different lengths (a shared prefix beside its members'
+    // private suffixes): the common split, sized by the average segment, leaves
+    // the long ones as the launch's tail.  Where the merge kernel runs anyway, a
+    // tensor-core segment longer than twice t_keys -- the average key load per
+    // SM, or the common split's range when larger -- is split into items of at
+    // most t_keys keys (measured on the prefix-shared workload: batches of one
+    // 8192-token prefix and 16 suffixes 0.393 -> 0.225 ms per four; segments
+    // only 1.4 x t_keys long measured slower split).
+    int64_t t_keys = 0;
+    if (merge_anyway) {
+        int64_t work = 0, keys = 0, n = 0;
+        for (auto &sg : segs) {
+            if (!is_tc(sg)) continue;
+            work += (rows_of(sg) + kTcRows - 1) / kTcRows * cf.n_kv_heads * sg.len;
+            keys += sg.len;
+            ++n;
+        }
+        if (n) {
+            const int64_t per_sm = (work + c->num_sms - 1) / c->num_sms;
+            const int64_t common = (keys / n + f_tc - 1) / f_tc;
+            t_keys = (std::max<int64_t>({per_sm, common, kMinChunk}) + 127) / 128 * 128;
+        }
+    }
 
     std::vector<WorkItem> items_small, items_tc;
     std::vector<int32_t> members;
@@ -277,8 +300,10 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         int max_seg = 1;
         for (int r : sg.members) max_seg = std::max(max_seg, nseg[r]);
         const int64_t slot_cap = std::max(1, c->L.slots / max_seg);
-        int64_t splits = std::min<int64_t>({tc ? f_tc : f_small, slot_cap,
-                                            (sg.len + kMinChunk - 1) / kMinChunk});
+        const bool long_seg = tc && t_keys > 0 && sg.len > 2 * t_keys;
+        const int64_t want = long_seg ? std::max<int64_t>(f_tc, (sg.len + t_keys - 1) / t_keys)
+                                      : (tc ? f_tc : f_small);
+        int64_t splits = std::min<int64_t>({want, slot_cap, (sg.len + kMinChunk - 1) / kMinChunk});
         splits = std::max<int64_t>(1, splits);
         int64_t chunk = (sg.len + splits - 1) / splits;
         chunk = (chunk + 127) / 128 * 128;
@@ -358,19 +383,19 @@ xgr_status build_plan(xgr_ctx *c, int which, int B) {
         return XGR_ERR_CUDA;
     c->n_small[which] = (int)items_small.size();
     c->n_tc[which] = (int)items_tc.size();
-    // Short items (few key chunks each) run the one-O variant of the
-    // tensor-core kernel (three S buffers: the tensor pipe does not drain
-    // between chunks); long ones keep an O per softmax warpgroup, whose
-    // warpgroups never wait for each other (measured: 8-chunk items faster
-    // with one O, 16- to 128-chunk items slower).
+    // Launches of short items only (few key chunks each) run the one-O variant
+    // of the tensor-core kernel (three S buffers: the tensor pipe does not
+    // drain between chunks); a launch with any long item keeps an O per
+    // softmax warpgroup, whose warpgroups never wait for each other (measured:
+    // 8-chunk items faster with one O, 16- to 128-chunk items slower).
     {
-        int64_t chunks = 0, n = 0;
+        int64_t longest = 0, n = 0;
         for (const WorkItem &it : items_tc)
             if (!(it.flags & 4)) {
-                chunks += (it.key_end - it.key_begin + 127) / 128;
+                longest = std::max<int64_t>(longest, (it.key_end - it.key_begin + 127) / 128);
                 ++n;
             }
-        c->tc_shared[which] = n > 0 && chunks <= kSharedOChunks * n;
+        c->tc_shared[which] = n > 0 && longest <= kSharedOChunks;
     }
     c->n_unfused[which] = unfused;
     return XGR_OK;
