@@ -169,6 +169,18 @@ def test_shared_prefix_groups_with_beams():
     decode_and_compare(w)
 
 
+def test_largest_beam_width_and_vocabulary():
+    """The configuration's limits: BW = K = 1024 (each beam's ordered head
+    shrinks to 4 keys; the pick's survivor buffer is at its largest) over a
+    32768-token vocabulary (the largest the selection takes: its dense first
+    step stages the whole row), in both score modes; attention on a sample of
+    beams."""
+    w = workloads.small(workloads.WORKLOADS[1], wid=108, B=2, prompt=(256, 256), BW=1024, K=1024,
+                        S=3, Hq=4, Hkv=1, D=128, V=32768, n_items=200000)
+    decode_and_compare(w, beams_per_step=16)
+    decode_and_compare(w, mode="logits", beams_per_step=16)
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
