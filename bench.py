@@ -342,6 +342,8 @@ def attention_bw512(dev, hbm, tf, src, reps=5):
             "ms": ms, "required_bytes": att_bytes, "achieved_gbs": gbs, "peak_gbs": hbm,
             "frac": gbs / hbm, "tflops": tfl, "tensor_peak_tflops": tf, "tensor_frac": tfl / tf,
             "peak_source": src, "l2": "flushed before each of the timed replays",
+            "kernel": attention_kernel(w),
+            "traffic": measured_traffic(attention_kernel(w), w.name),
             "device_status": status}
 
 
@@ -713,18 +715,31 @@ def code_sha(path: str) -> str:
     return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
 
 
-def measured_traffic(call: str):
-    """DRAM bytes per launch of a call, from the committed ncu summary
-    (profiles/traffic.json), or None when the code of any of the call's kernel
-    sources has changed since the counters were taken (code_sha differs)."""
+def measured_traffic(call: str, workload: str):
+    """DRAM bytes per launch of a call on a workload, from the committed ncu
+    summary (profiles/traffic.json), or None when there is no capture of that
+    call on that workload or the code of any of the call's kernel sources has
+    changed since the counters were taken (code_sha differs)."""
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[call]
+        if rec.get("workload_name") != workload:
+            return None
         for rel, sha in rec["sources"].items():
             if code_sha(os.path.join(ROOT, rel)) != sha:
                 return None
         return rec["dram_bytes_per_launch"]
     except (OSError, KeyError, ValueError):
         return None
+
+
+def attention_kernel(w):
+    """The attention kernel the work plan runs at steps >= 1 for a workload of
+    single-request segments: the tensor-core one (D = 128), in its one-O
+    variant when no item passes 12 key chunks, else the small-row kernel with
+    the merge."""
+    if w.D != 128:
+        return "attn_small_kernel + attn_merge_kernel"
+    return "attn_tc_one_o_kernel" if -(-w.prompt[1] // 128) <= 12 else "attn_tc_kernel"
 
 
 def run_gpu(args, w):
@@ -978,14 +993,15 @@ def run_gpu(args, w):
     sel_avg = statistics.mean(sel_ms) / 1e3
     # the dominant kernel (largest share of the decode in the ncu launch list,
     # profiles/launches_*.md): the tensor-core attention, one launch per step --
-    # for this workload's short items (8 prompt chunks + 1) the one-O variant
+    # for short items (workload 2: 8 prompt chunks + 1) the one-O variant
     # attn_tc_one_o_kernel -- timed by its phase graph (the attention of a step
     # is that one launch)
     achieved = att_flops / att_avg / 1e12
-    roof = {"kernel": "attn_tc_one_o_kernel (xgr_decode_step, steps >= 1)", "bound": "tensor",
+    att_kernel = attention_kernel(w)
+    roof = {"kernel": f"{att_kernel} (xgr_decode_step, steps >= 1)", "bound": "tensor",
             "achieved": achieved, "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
             "peak_source": f"bf16_tflops burst {src}",
-            "traffic": measured_traffic("attn_tc_one_o_kernel"),
+            "traffic": measured_traffic(att_kernel, w.name),
             "algorithmic_per_launch": att_flops, "launch_ms": att_avg * 1e3,
             "hbm_gbs_required_bytes": att_bytes / att_avg / 1e9,
             "hbm_frac_required_bytes": att_bytes / att_avg / 1e9 / hbm}
@@ -995,7 +1011,7 @@ def run_gpu(args, w):
                    "bound": "hbm", "achieved": sel_gbs, "peak": hbm, "unit": "GB/s",
                    "frac": sel_gbs / hbm, "algorithmic_per_call": sel_bytes,
                    "call_ms": sel_avg * 1e3,
-                   "traffic_rows_kernel": measured_traffic("select_rows_kernel")}
+                   "traffic_rows_kernel": measured_traffic("select_rows_kernel", w.name)}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -1031,8 +1047,7 @@ def run_gpu(args, w):
         line["long_history"] = long_history(dev, hbm, tf, src)
     # the Shared stage's tensor throughput per workload (the stage is a dense
     # contraction; its tensor fraction is what bounds it at 128+ beams)
-    tfr = {"gr-decode-pool-128x128 (step >= 1, with the Unshared and Merging stages)":
-           att_flops / att_avg / 1e12 / tf}
+    tfr = {f"{w.name} (step >= 1, with the Unshared and Merging stages)": att_flops / att_avg / 1e12 / tf}
     if "attention_bw512" in line:
         tfr["gr-decode-pool-512x512 (step 1)"] = line["attention_bw512"]["tensor_frac"]
     if "long_history" in line:
