@@ -283,12 +283,13 @@ xgr_status xgr_device_status(xgr_ctx *ctx, xgr_stream_t stream, int32_t *host_co
  * xgr_beam_select does (same order, same tie-break, same bits).
  * Allocation: none.  Its scratch is one static device array of 8 MiB per GPU
  * (held by every GPU that loads the library until the process exits).  After
- * about 12 bytes per beam row, the rest is shared by the requests as a key
- * buffer (8 bytes per CSR entry) plus a survivor buffer (12 bytes per entry,
- * half as many); a call returns XGR_ERR_CAPACITY unless every request gets
- * room for max(V, 8*BW, 4096) entries (e.g. 8 requests x 128 beams over
- * V = 8192 get about 74000).  A request with more CSR entries than its share
- * is still selected exactly, on a slower path.  V above 32768 returns
+ * 120 bytes per beam row (its log-sum-exp, counts, ordered head of 8 best
+ * keys with their entries and its next key; 4 keys from BW = 1024 on), the
+ * rest is shared by the requests as key buffers (8 bytes per CSR entry); a
+ * call returns XGR_ERR_CAPACITY unless every request gets room for
+ * max(V, 8*BW, 4096) entries (e.g. 8 requests x 128 beams get about 129000
+ * each).  A request with more CSR entries than its share is still selected
+ * exactly, from the scores, on a slower path.  V above 32768 returns
  * XGR_ERR_UNIMPLEMENTED (a score row is staged whole in shared memory).
  * The first call on a device looks the array up (cudaGetSymbolAddress) and
  * may set a kernel attribute, so make that first call before any stream capture.
