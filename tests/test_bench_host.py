@@ -26,3 +26,24 @@ def test_attention_byte_and_flop_model_of_the_512_pool():
               + 2 * B * BW * Hq * D * 2 + B * BW * Hq * 4)
     assert att_bytes == expect
     assert att_flops == 4.0 * B * BW * Hq * D * (P + 2)
+
+
+def test_attention_kernel_named_per_workload():
+    # short items (workload 2: 8 prompt chunks) run the one-O variant, long
+    # ones (32 or more chunks) the two-accumulator kernel, D = 64 the small-row
+    # kernel with the merge
+    assert bench.attention_kernel(workloads.WORKLOADS[2]) == "attn_tc_one_o_kernel"
+    assert bench.attention_kernel(workloads.WORKLOADS[3]) == "attn_tc_kernel"
+    assert bench.attention_kernel(workloads.WORKLOADS[5]) == "attn_tc_kernel"
+    assert bench.attention_kernel(workloads.WORKLOADS[1]).startswith("attn_small_kernel")
+
+
+def test_traffic_is_reported_only_for_the_workload_it_was_taken_on():
+    # the committed counters belong to one workload each; another workload's
+    # line (or a kernel with no capture) reports none
+    w2, w3 = workloads.WORKLOADS[2].name, workloads.WORKLOADS[3].name
+    one_o = bench.measured_traffic("attn_tc_one_o_kernel", w2)
+    assert one_o is None or one_o > 0
+    assert bench.measured_traffic("attn_tc_one_o_kernel", w3) is None
+    assert bench.measured_traffic("attn_tc_kernel", w2) is None
+    assert bench.measured_traffic("no_such_kernel", w2) is None
