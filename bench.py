@@ -732,6 +732,26 @@ def measured_traffic(call: str, workload: str):
         return None
 
 
+def _pct(xs, q):
+    """The q-th percentile of sorted values (nearest rank)."""
+    if not xs:
+        return None
+    return xs[min(len(xs) - 1, max(0, int(round(q / 100 * (len(xs) - 1)))))]
+
+
+def secondary_rates(w, items, nnz, ms):
+    """The step's other throughputs: valid (beam, token) candidates scored per
+    second (step 0: one live beam per request against the distinct first
+    tokens; later steps: the mask's measured entries) and vocabulary entries
+    scored per second (live beams x V; logits mode reads every one)."""
+    import numpy as np
+    first = int(np.unique(items[:, 0]).size) * w.B
+    valid = first + sum(nnz[1:])
+    scored = sum(w.B * (1 if s == 0 else w.BW) * w.V for s in range(w.S))
+    return {"valid_candidates_per_s": valid / (ms / 1e3), "tokens_scored_per_s": scored / (ms / 1e3),
+            "valid_candidates_per_decode": valid, "tokens_scored_per_decode": scored}
+
+
 def attention_kernel(w):
     """The attention kernel the work plan runs at steps >= 1 for a workload of
     single-request segments: the tensor-core one (D = 128), in its one-O
@@ -922,7 +942,8 @@ def run_gpu(args, w):
     if world > 1:
         dist.barrier()
     clocks = clk.stop() if clk else None
-    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), dev)
+    step_ms = sorted(a.elapsed_time(b) for a, b in zip(starts, ends))
+    total_ms = max_over_ranks(sum(step_ms), dev)
     n_live = torch.cat(nout_g).cpu().numpy()
     cands = candidates_per_decode(w) * args.steps * world
     value = cands / (total_ms / 1e3)
@@ -1027,6 +1048,10 @@ def run_gpu(args, w):
                            "peak_gbs": hbm, "frac": dec_gbs / hbm,
                            "note": "whole decode (all steps, every kernel) against the copy "
                                    f"bandwidth {src}"},
+            "step_ms_percentiles": {"p10": _pct(step_ms, 10), "p50": _pct(step_ms, 50),
+                                    "p90": _pct(step_ms, 90), "replays": len(step_ms),
+                                    "note": "this rank's timed replays"},
+            "secondary_rates": secondary_rates(w, items, nnz, total_ms / args.steps),
             "request_groups": G,
             "gpu_launches": launches_per_decode * args.steps,
             "device_status": status, "n_live_last": int(n_live.min()) if n_live.size else 0}

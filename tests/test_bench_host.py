@@ -47,3 +47,17 @@ def test_traffic_is_reported_only_for_the_workload_it_was_taken_on():
     assert bench.measured_traffic("attn_tc_one_o_kernel", w3) is None
     assert bench.measured_traffic("attn_tc_kernel", w2) is None
     assert bench.measured_traffic("no_such_kernel", w2) is None
+
+
+def test_step_percentiles_and_secondary_rates():
+    xs = [float(i) for i in range(1, 11)]
+    assert bench._pct(xs, 10) == 2.0 and bench._pct(xs, 90) == 9.0 and bench._pct([3.0], 50) == 3.0
+    # workload 2 over 1 ms: step 0 scores the distinct first tokens of one beam
+    # per request, later steps the mask's entries; every live row reads V logits
+    w = workloads.WORKLOADS[2]
+    import numpy as np
+    items = np.array([[1, 2, 3], [1, 5, 6], [7, 2, 3]], dtype=np.int32)
+    r = bench.secondary_rates(w, items, [0, 100, 20], 1.0)
+    assert r["valid_candidates_per_decode"] == 2 * w.B + 120
+    assert r["tokens_scored_per_decode"] == w.B * w.V * (1 + 2 * w.BW)
+    assert r["valid_candidates_per_s"] == r["valid_candidates_per_decode"] * 1e3
