@@ -78,3 +78,52 @@ def test_tree_batches_feed_the_attention():
         compare_attention(out[r], lse[r], o_ref, l_ref, np.ones(w.BW, bool), f"request {r}")
     assert sess.device_status() == 0
     sess.close()
+
+
+def test_tree_batches_as_separate_contexts():
+    """The launch configuration the bench times for the tree's batches: each
+    batch of 16 requests is a context of its own, holding one shared 8192-token
+    prefix beside 16 private suffixes, so the work plan splits the prefix into
+    several key ranges (it is more than twice the average key load per SM)
+    and the merge kernel folds them with each suffix.  Every request's
+    attention is compared with the oracle over its own full prompt."""
+    w = workloads.WORKLOADS[4]
+    toks = _prompt_tokens(w)
+    tree = ChunkedHashTree(CHUNK)
+    for r in np.random.default_rng(7).permutation(w.B):
+        tree.insert(int(r), toks[r])
+    batches = tree.form_batches(w.B // w.groups, 1)
+    tree.close()
+    lens, suf = workloads.prompt_lengths(w), workloads.suffix_lengths(w)
+    q, kn, vn = workloads.step_qkv(w, 0, "cuda")
+    qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
+    for members, shared_chunks in batches:
+        fam = w.shared_id(members[0])
+        assert shared_chunks * CHUNK == int(lens[fam])
+        n = len(members)
+        cfg = xgr.make_config(max_requests=n, max_shared=1,
+                              kv_tokens=int(lens[fam]) + sum(int(suf[r]) for r in members),
+                              beam_width=1, top_k=1, steps=1, n_q_heads=w.Hq, n_kv_heads=w.Hkv,
+                              head_dim=w.D, vocab=0, max_items=0, max_fanout=0, max_partials=0)
+        sess = Session(cfg, "cuda")
+        ks, vs = workloads.shared_kv(w, fam, "cuda")
+        sess.prefill(0, 0, ks, vs)
+        for i in range(1, n):
+            sess.link(i, 0)
+        suf_kv = {r: workloads.suffix_kv(w, r, "cuda") for r in members}
+        for i, r in enumerate(members):
+            sess.prefill(i, 0, *suf_kv[r], kind=xgr.XGR_KV_SUFFIX)
+        sel = torch.tensor(members, device="cuda")
+        out = torch.full((n, 1, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        lse = torch.full((n, 1, w.Hq), float("nan"), dtype=torch.float32, device="cuda")
+        sess.begin(n)
+        sess.decode_step(0, q[sel].contiguous(), kn[sel].contiguous(), vn[sel].contiguous(), out, lse)
+        torch.cuda.synchronize()
+        assert sess.device_status() == 0
+        for i, r in enumerate(members):
+            kx, vx = suf_kv[r]
+            dec = oracle.BeamDecode(None, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V)
+            dec.begin(u16(ks), u16(vs), u16(kx), u16(vx))
+            o_ref, l_ref = dec.attention(0, qc[r], knc[r], vnc[r])
+            compare_attention(out[i], lse[i], o_ref, l_ref, np.ones(w.BW, bool), f"request {r}")
+        sess.close()
