@@ -80,36 +80,47 @@ def test_tree_batches_feed_the_attention():
     sess.close()
 
 
-def test_tree_batches_as_separate_contexts():
-    """The launch configuration the bench times for the tree's batches: each
-    batch of 16 requests is a context of its own, holding one shared 8192-token
-    prefix beside 16 private suffixes, so the work plan splits the prefix into
+@pytest.mark.parametrize("batching", ["tree", "arrival_order"])
+def test_batches_as_separate_contexts(batching):
+    """The launch configurations the bench times: each batch of 16 requests is
+    a context of its own.  A tree batch holds one shared 8192-token prefix
+    beside 16 private suffixes, so the work plan splits the prefix into
     several key ranges (it is more than twice the average key load per SM)
-    and the merge kernel folds them with each suffix.  Every request's
-    attention is compared with the oracle over its own full prompt."""
+    and the merge kernel folds them with each suffix; a batch of consecutive
+    arrivals holds the four families' prefixes, each linked by its own
+    members.  Every request's attention is compared with the oracle over its
+    own full prompt."""
     w = workloads.WORKLOADS[4]
     toks = _prompt_tokens(w)
-    tree = ChunkedHashTree(CHUNK)
-    for r in np.random.default_rng(7).permutation(w.B):
-        tree.insert(int(r), toks[r])
-    batches = tree.form_batches(w.B // w.groups, 1)
-    tree.close()
+    arrivals = [int(r) for r in np.random.default_rng(7).permutation(w.B)]
     lens, suf = workloads.prompt_lengths(w), workloads.suffix_lengths(w)
+    if batching == "tree":
+        tree = ChunkedHashTree(CHUNK)
+        for r in arrivals:
+            tree.insert(r, toks[r])
+        formed = tree.form_batches(w.B // w.groups, 1)
+        tree.close()
+        for members, shared_chunks in formed:
+            assert shared_chunks * CHUNK == int(lens[w.shared_id(members[0])])
+        batches = [list(m) for m, _ in formed]
+    else:
+        batches = [arrivals[i:i + 16] for i in range(0, w.B, 16)]
     q, kn, vn = workloads.step_qkv(w, 0, "cuda")
     qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
-    for members, shared_chunks in batches:
-        fam = w.shared_id(members[0])
-        assert shared_chunks * CHUNK == int(lens[fam])
+    fam_kv = {g: workloads.shared_kv(w, g, "cuda") for g in range(w.groups)}
+    for members in batches:
         n = len(members)
-        cfg = xgr.make_config(max_requests=n, max_shared=1,
-                              kv_tokens=int(lens[fam]) + sum(int(suf[r]) for r in members),
+        fams = sorted({w.shared_id(r) for r in members})
+        cfg = xgr.make_config(max_requests=n, max_shared=len(fams),
+                              kv_tokens=sum(int(lens[g]) for g in fams) + sum(int(suf[r]) for r in members),
                               beam_width=1, top_k=1, steps=1, n_q_heads=w.Hq, n_kv_heads=w.Hkv,
                               head_dim=w.D, vocab=0, max_items=0, max_fanout=0, max_partials=0)
         sess = Session(cfg, "cuda")
-        ks, vs = workloads.shared_kv(w, fam, "cuda")
-        sess.prefill(0, 0, ks, vs)
-        for i in range(1, n):
-            sess.link(i, 0)
+        for sid, g in enumerate(fams):
+            idx = [i for i, r in enumerate(members) if w.shared_id(r) == g]
+            sess.prefill(idx[0], sid, *fam_kv[g])
+            for i in idx[1:]:
+                sess.link(i, sid)
         suf_kv = {r: workloads.suffix_kv(w, r, "cuda") for r in members}
         for i, r in enumerate(members):
             sess.prefill(i, 0, *suf_kv[r], kind=xgr.XGR_KV_SUFFIX)
@@ -121,6 +132,7 @@ def test_tree_batches_as_separate_contexts():
         torch.cuda.synchronize()
         assert sess.device_status() == 0
         for i, r in enumerate(members):
+            ks, vs = fam_kv[w.shared_id(r)]
             kx, vx = suf_kv[r]
             dec = oracle.BeamDecode(None, w.BW, w.K, w.S, w.Hq, w.Hkv, w.D, w.V)
             dec.begin(u16(ks), u16(vs), u16(kx), u16(vx))
