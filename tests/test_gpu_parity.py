@@ -181,6 +181,17 @@ def test_largest_beam_width_and_vocabulary():
     decode_and_compare(w, mode="logits", beams_per_step=16)
 
 
+def test_longest_items():
+    """Eight-token items, the most decode steps a context takes: at the last
+    step every beam attends to eight Unshared tokens through its ancestry (16
+    beams x 8 tokens fill one 128-row Unshared chunk at G = 2), in both score
+    modes."""
+    w = workloads.small(workloads.WORKLOADS[1], wid=109, B=2, prompt=(300, 300), BW=16, K=16,
+                        S=8, Hq=4, Hkv=2, D=128, V=64, n_items=5000)
+    decode_and_compare(w)
+    decode_and_compare(w, mode="logits")
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
