@@ -44,10 +44,12 @@ class StepOut:
 class GpuRun:
     """One decode of workload w on cuda:0 through the C ABI."""
 
-    def __init__(self, w, items=None, device="cuda", max_partials=0, per_beam=False):
+    def __init__(self, w, items=None, device="cuda", max_partials=0, per_beam=False, capacity=None):
         self.w, self.device = w, device
         self.per_beam = per_beam   # attention by the per-beam comparison path
-        self.sess = Session(config_for(w, max_partials=max_partials), device)
+        # capacity: a context sized for more requests than the decode runs
+        cw = w if capacity is None else workloads.small(w, B=capacity)
+        self.sess = Session(config_for(cw, max_partials=max_partials), device)
         if w.V:
             self.sess.build_trie(items)
         self.kv = {}

@@ -27,10 +27,10 @@ def _sample_beams(n_live, k, seed):
 
 
 def decode_and_compare(w, mode="logprob", requests=None, beams_per_step=None, items=None,
-                       max_partials=0, scores_fn=None, per_beam=False):
+                       max_partials=0, scores_fn=None, per_beam=False, capacity=None):
     items = workloads.items(w) if items is None else items
     si = oracle.SortedItems(items, w.V) if w.V else None
-    run = GpuRun(w, items, max_partials=max_partials, per_beam=per_beam)
+    run = GpuRun(w, items, max_partials=max_partials, per_beam=per_beam, capacity=capacity)
     reqs = list(range(w.B)) if requests is None else list(requests)
     decs = {r: oracle_request(w, si, run, r, mode) for r in reqs}
     flags = xgr.XGR_SCORES_LOGPROB if mode == "logprob" else xgr.XGR_SCORES_LOGITS
@@ -190,6 +190,15 @@ def test_longest_items():
                         S=8, Hq=4, Hkv=2, D=128, V=64, n_items=5000)
     decode_and_compare(w)
     decode_and_compare(w, mode="logits")
+
+
+def test_fewer_requests_than_the_context_holds():
+    """A context sized for 8 requests decoding a batch of 3: the beam state and
+    the Unshared pool keep the capacity's strides while the work plan, the
+    masks and the selection cover the 3 requests of this decode."""
+    w = workloads.small(workloads.WORKLOADS[2], wid=110, B=3, prompt=(500, 500), n_items=200000)
+    decode_and_compare(w, capacity=8, beams_per_step=16)
+    decode_and_compare(w, mode="logits", capacity=8, beams_per_step=16)
 
 
 def test_fewer_candidates_than_beams():
