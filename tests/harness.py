@@ -67,14 +67,20 @@ class GpuRun:
                 k, v = workloads.suffix_kv(w, r, device)
                 self.kv[("x", r)] = (k, v)
                 self.sess.prefill(r, 0, k, v, kind=xgr.XGR_KV_SUFFIX)
+        self.n = w.B      # requests of the current decode
         self.sess.begin(w.B)
         self.kinds = []   # the mask kind of every sparse step
 
+    def restart(self, n: int):
+        """A new decode of the context's first n requests (xgr_begin(n))."""
+        self.n = n
+        self.sess.begin(n)
+
     def step(self, s, q, kn, vn, scores=None, flags=xgr.XGR_SCORES_LOGPROB) -> StepOut:
-        w = self.w
+        w, B = self.w, self.n
         # NaN sentinels: every row the call must write (dead beams' zeros included) is checked
-        out = torch.full((w.B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=self.device)
-        lse = torch.full((w.B, w.BW, w.Hq), float("nan"), dtype=torch.float32, device=self.device)
+        out = torch.full((B, w.BW, w.Hq, w.D), float("nan"), dtype=torch.bfloat16, device=self.device)
+        lse = torch.full((B, w.BW, w.Hq), float("nan"), dtype=torch.float32, device=self.device)
         if self.per_beam:
             self.sess.decode_step_per_beam(s, q, kn, vn, out, lse)
         else:
@@ -97,10 +103,10 @@ class GpuRun:
             mask = ("csr", (rpn.astype(np.int64), cols.cpu().numpy()[:nnz].copy()))
             if m.kind == xgr.XGR_MASK_NODE_BITS:
                 _check_node_bits(m, mask[1], w.V, self.sess)
-        parent = torch.empty((w.B, w.BW), dtype=torch.int32, device=self.device)
+        parent = torch.empty((B, w.BW), dtype=torch.int32, device=self.device)
         token = torch.empty_like(parent)
-        cum = torch.empty((w.B, w.BW), dtype=torch.float32, device=self.device)
-        n_out = torch.empty((w.B,), dtype=torch.int32, device=self.device)
+        cum = torch.empty((B, w.BW), dtype=torch.float32, device=self.device)
+        n_out = torch.empty((B,), dtype=torch.int32, device=self.device)
         self.sess.beam_select(s, scores, flags, m, parent, token, cum, n_out)
         torch.cuda.synchronize()
         return StepOut(out, lse, mask, parent.cpu().numpy(), token.cpu().numpy(),
@@ -108,7 +114,7 @@ class GpuRun:
 
     def sequences(self) -> np.ndarray:
         w = self.w
-        seq = torch.empty((w.B, w.BW, w.S), dtype=torch.int32, device=self.device)
+        seq = torch.empty((self.n, w.BW, w.S), dtype=torch.int32, device=self.device)
         self.sess.sequences(seq)
         torch.cuda.synchronize()
         return seq.cpu().numpy()

@@ -201,6 +201,42 @@ def test_fewer_requests_than_the_context_holds():
     decode_and_compare(w, mode="logits", capacity=8, beams_per_step=16)
 
 
+def test_context_reused_across_batch_sizes():
+    """One context decodes its first 3 requests, then all 8, then 3 again:
+    every xgr_begin re-plans for its batch and resets the beam state, so each
+    decode matches the oracle (log-prob mode, selections and final sequences
+    bit-exact) whatever the decodes before it left in the workspace."""
+    w = workloads.small(workloads.WORKLOADS[2], wid=112, B=8, prompt=(400, 400), n_items=200000)
+    items = workloads.items(w)
+    si = oracle.SortedItems(items, w.V)
+    run = GpuRun(w, items)
+    inputs = [(*workloads.step_qkv(w, s, "cuda"), workloads.step_logprobs(w, s, "cuda"))
+              for s in range(w.S)]
+    for n in (3, 8, 3):
+        run.restart(n)
+        decs = {r: oracle_request(w, si, run, r) for r in sorted({0, n - 1})}
+        for s in range(w.S):
+            q, kn, vn, lp = (t[:n].contiguous() for t in inputs[s])
+            so = run.step(s, q, kn, vn, lp)
+            qc, knc, vnc, sc = q.cpu(), kn.cpu(), vn.cpu(), lp.cpu().numpy()
+            for r, dec in decs.items():
+                what = f"batch of {n}, step {s}, request {r}"
+                beams = _sample_beams(dec.n_live, 8, 1000 * s + r)
+                o_ref, l_ref = dec.attention(s, qc[r], knc[r], vnc[r], beams)
+                ids = np.arange(w.BW) if beams is None else beams
+                idx = torch.as_tensor(ids).long()
+                compare_attention(so.out[r][idx], so.lse[r][idx], o_ref, l_ref, ids < dec.n_live, what)
+                om = dec.mask(s)
+                compare_mask(so.mask, om, r, w.BW, what)
+                p, t, c, cnt = dec.select(s, sc[r], om)
+                compare_select_exact(so, r, p, t, c, cnt, what)
+        seq = run.sequences()
+        for r, dec in decs.items():
+            assert np.array_equal(seq[r], dec.paths), f"batch of {n}: sequences of request {r}"
+    assert run.status() == 0
+    run.sess.close()
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
