@@ -224,7 +224,11 @@ def compare_select_tie_aware(so: StepOut, r: int, dec, scores_r: np.ndarray, mas
     dead = so.parent[r][n:]
     assert np.all(dead == -1) and np.all(so.token[r][n:] == -1), f"{what}: dead slots"
     gk = oracle.logits_keys(dec.cum, scores_r, list(zip(gp.tolist(), gt.tolist())))
+    # -inf is an ordinary (lowest) score: two -inf keys are equal, not NaN apart
+    def close(x, y):
+        with np.errstate(invalid="ignore"):
+            return (x == y) | (np.abs(x - y) <= TIE_EPS)
     # the GPU's k-th choice has the oracle's k-th best score up to near-ties
-    assert np.all(np.abs(np.sort(gk)[::-1] - cm[:n]) <= TIE_EPS), f"{what}: selection differs"
-    assert np.all(np.abs(so.cum[r][:n].astype(np.float64) - gk) <= TIE_EPS), f"{what}: cum"
+    assert np.all(close(np.sort(gk)[::-1], cm[:n])), f"{what}: selection differs"
+    assert np.all(close(so.cum[r][:n].astype(np.float64), gk)), f"{what}: cum"
     return gp, gt, n

@@ -237,6 +237,25 @@ def test_context_reused_across_batch_sizes():
     run.sess.close()
 
 
+def test_logits_of_large_magnitude_and_minus_inf():
+    """Logits mode on rows whose unshifted exponentials overflow fp32: logits of
+    spread 20 around 100 (kept below a few hundred so that one fp32 ulp of the
+    row's log-sum-exp stays under the 1e-4 tie tolerance), and every seventh
+    token at -inf (a score that ranks last; it adds nothing to a row's
+    log-sum-exp).  The tiny workload in full, and two requests of the 128-beam
+    pool (its streamed rows and dense first step)."""
+    def extreme(w):
+        def fn(s):
+            x = workloads.step_logits(w, s, "cuda") * 10.0 + 100.0
+            x[..., ::7] = float("-inf")
+            return x
+        return fn
+    w1 = workloads.WORKLOADS[1]
+    decode_and_compare(w1, mode="logits", scores_fn=extreme(w1))
+    w2 = workloads.WORKLOADS[2]
+    decode_and_compare(w2, mode="logits", requests=[1, 6], beams_per_step=8, scores_fn=extreme(w2))
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
