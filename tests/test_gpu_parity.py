@@ -256,6 +256,21 @@ def test_logits_of_large_magnitude_and_minus_inf():
     decode_and_compare(w2, mode="logits", requests=[1, 6], beams_per_step=8, scores_fn=extreme(w2))
 
 
+def test_logprob_minus_inf_scores():
+    """Log-prob mode with every fifth token at -inf (a token the model rules
+    out): such candidates rank after every finite one and among themselves by
+    parent, then token; selections bit-exact.  Two requests of the 128-beam
+    pool, where late steps have about one valid token per beam, so -inf
+    candidates are among the winners."""
+    w = workloads.WORKLOADS[2]
+
+    def fn(s):
+        x = workloads.step_logprobs(w, s, "cuda")
+        x[..., ::5] = float("-inf")
+        return x
+    decode_and_compare(w, requests=[2, 7], beams_per_step=8, scores_fn=fn)
+
+
 def test_fewer_candidates_than_beams():
     """A vocabulary of 3 items: at most 3 live beams of 8, the rest dead."""
     w = workloads.small(workloads.WORKLOADS[1], wid=103, BW=8, K=8, n_items=3)
