@@ -35,11 +35,19 @@ def test_noalloc_rejects_bad_arguments_on_the_host():
     assert L.xgr_beam_topk_noalloc(*bad) == xgr.XGR_ERR_ARG
 
 
+# the configuration's limits: 1024 beams over a 32768-token vocabulary (each
+# beam's head holds 4 keys; the dense step stages the whole row)
+_LIMITS = dict(wid=108, B=2, prompt=(256, 256), BW=1024, K=1024, S=3, Hq=4, Hkv=1, D=128,
+               V=32768, n_items=200000)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("wid,flags", [(1, xgr.XGR_SCORES_LOGPROB), (2, xgr.XGR_SCORES_LOGITS)])
+@pytest.mark.parametrize("wid,flags", [(1, xgr.XGR_SCORES_LOGPROB), (2, xgr.XGR_SCORES_LOGITS),
+                                       ("limits", xgr.XGR_SCORES_LOGPROB)])
 def test_noalloc_matches_context_select(wid, flags):
     from harness import GpuRun
-    w = workloads.WORKLOADS[wid]
+    w = (workloads.small(workloads.WORKLOADS[1], **_LIMITS) if wid == "limits"
+         else workloads.WORKLOADS[wid])
     run = GpuRun(w, workloads.items(w))
     B, BW = w.B, w.BW
     dev = "cuda"
