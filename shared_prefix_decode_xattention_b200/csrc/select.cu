@@ -676,12 +676,50 @@ __device__ float warp_row_lse_plain(const float *x, int V) {
 
 // Merges the keys c[] of every lane (entries ce[]) into the warp's running
 // head: afterwards lanes 0..m-1 hold the m smallest keys seen so far, in
-// ascending order (kNoKey pads), with their entries.  Keys are unique.  m
-// rounds of a warp minimum; c[] is consumed.
+// ascending order (kNoKey pads), with their entries.  Keys are unique.
+// Only keys below the head's m-th key can enter it.  When at most
+// kHeadInsertMax of them do (a sparse row, or a long row's later pass once
+// its head is full), each is inserted into the lane-distributed sorted head
+// (its rank by one ballot, the lanes above shifted up by one); otherwise m
+// rounds of a warp minimum.  c[] is consumed.
+constexpr int kHeadInsertMax = 32;
 template <int KPC>
 __device__ __forceinline__ void warp_head_merge(uint64_t (&c)[KPC], const int (&ce)[KPC], uint64_t &run,
                                                 int &run_e, int m) {
     const int lane = threadIdx.x & 31;
+    uint64_t bound = __shfl_sync(0xffffffffu, run, m - 1);   // the head's m-th key (kNoKey: not full)
+    int q = 0;
+#pragma unroll
+    for (int u = 0; u < KPC; ++u) q += c[u] < bound;
+    const int entering = __reduce_add_sync(0xffffffffu, q);
+    if (entering == 0) return;
+    if (entering <= kHeadInsertMax) {
+#pragma unroll
+        for (int u = 0; u < KPC; ++u) {
+            // a key at or above the bound now cannot enter later: the bound only falls
+            unsigned who = __ballot_sync(0xffffffffu, c[u] < bound);
+            while (who) {
+                const int src = __ffs(who) - 1;
+                who &= who - 1;
+                const uint64_t x = __shfl_sync(0xffffffffu, c[u], src);
+                const int xe = __shfl_sync(0xffffffffu, ce[u], src);
+                if (x >= bound) continue;   // (uniform) passed by keys inserted meanwhile
+                const int pos = __popc(__ballot_sync(0xffffffffu, lane < m && run < x));
+                const uint64_t up = __shfl_up_sync(0xffffffffu, run, 1);
+                const int up_e = __shfl_up_sync(0xffffffffu, run_e, 1);
+                if (lane > pos && lane < m) {
+                    run = up;
+                    run_e = up_e;
+                }
+                if (lane == pos) {
+                    run = x;
+                    run_e = xe;
+                }
+                bound = __shfl_sync(0xffffffffu, run, m - 1);
+            }
+        }
+        return;
+    }
     uint64_t nrun = kNoKey;
     int nrun_e = -1;
     for (int i = 0; i < m; ++i) {
