@@ -1109,12 +1109,9 @@ __device__ Cut make_cut(const uint64_t *k, int n, int want, int *hist, uint32_t 
         hi = max(hi, w);
         ++cnt;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
     if (lane == 0) {
         red32[warp] = lo;
         red32[32 + warp] = hi;
