@@ -518,7 +518,13 @@ constexpr int kSpWarps = kSpThreads / 32;
 // CTA's keys and head merge overlap the others' streams).
 constexpr int kRowWarpsWide = 8, kRingWide = 5;
 constexpr int kRowWarpsNarrow = 4, kRingNarrow = 3;
-constexpr int kSpKpc = 8;             // CSR entries per lane in one pass of the key loop
+constexpr int kSpKpc = 8;             // CSR entries per lane in one pass of the key loop (many-wave shape)
+// the one-wave shape's rows (small batches, where each row's latency is the
+// launch's) take half as many a pass: cheaper merge rounds over a short row;
+// a longer row's later passes go through the insertion path (measured: the
+// 128-beam decode 0.4-1.0 us faster; 4 for the many-wave shape's long rows
+// cost the 512-beam selection 2.5%)
+constexpr int kSpKpcWide = 4;
 constexpr int kRingStageBytes = 4096;  // one stage of a warp's row stream
 constexpr int kWtokCap = 1024;         // NODE_BITS tokens listed beside the ring before the stream
 // a warp's area: its ring of `ring` stages, then its token list
@@ -800,23 +806,24 @@ __device__ int warp_bits_to_tokens(const uint32_t *wb, int nw, int *wtok, int ca
 // ring for its log-sum-exp while the first pass's scores are fetched.  area:
 // the warp's ring_warp_bytes(RING) of shared memory (16-byte aligned);
 // bars: its RING mbarriers.
+template <int KPC>
 struct RowPrep {
     bool live;
     float cum;
     int node, n_e, cb, nb_full;
     int64_t ebase;
     const int32_t *tokp;
-    int tk0[kSpKpc];   // the first pass's tokens (lane j: entries j, j + 32, ...)
+    int tk0[KPC];   // the first pass's tokens (lane j: entries j, j + 32, ...)
 };
 
-template <int RING>
-__device__ RowPrep row_prep(const SelectArgs &a, int r, int b, int n_live, int base, uint8_t *area) {
+template <int RING, int KPC>
+__device__ RowPrep<KPC> row_prep(const SelectArgs &a, int r, int b, int n_live, int base, uint8_t *area) {
     const int lane = threadIdx.x & 31;
     const Dims dm = a.dims;
     const int s = a.step;
     const int64_t row = (int64_t)r * dm.BW + b;
     int *wtok = reinterpret_cast<int *>(area + (size_t)RING * kRingStageBytes);
-    RowPrep p;
+    RowPrep<KPC> p;
     p.live = b < n_live;
     p.cum = a.cum[row];
     const bool csr = a.mask_kind == XGR_MASK_CSR;
@@ -858,15 +865,15 @@ __device__ RowPrep row_prep(const SelectArgs &a, int r, int b, int n_live, int b
         }
     }
 #pragma unroll
-    for (int u = 0; u < kSpKpc; ++u) {
+    for (int u = 0; u < KPC; ++u) {
         const int j = u * 32 + lane;
         p.tk0[u] = (j < p.n_e && p.live) ? p.tokp[j] : -1;
     }
     return p;
 }
 
-template <int RING>
-__device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uint64_t *keys, uint8_t *area,
+template <int RING, int KPC>
+__device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep<KPC> &p, uint64_t *keys, uint8_t *area,
                         uint64_t *bars) {
     const int lane = threadIdx.x & 31;
     const Dims dm = a.dims;
@@ -879,9 +886,9 @@ __device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uin
     RowStream<RING> rs{};
     if (stream) rs = row_stream_start<RING>(x, V, ring, bars);
     // the first pass's scores go out before the stream is folded
-    float sv0[kSpKpc];
+    float sv0[KPC];
 #pragma unroll
-    for (int u = 0; u < kSpKpc; ++u) sv0[u] = (p.tk0[u] >= 0 && p.tk0[u] < V) ? __ldg(x + p.tk0[u]) : 0.f;
+    for (int u = 0; u < KPC; ++u) sv0[u] = (p.tk0[u] >= 0 && p.tk0[u] < V) ? __ldg(x + p.tk0[u]) : 0.f;
     float lse = 0.f;
     if (a.logits && live) {
         lse = stream ? row_stream_lse(rs, a.status) : warp_row_lse_plain(x, V);
@@ -899,29 +906,29 @@ __device__ void row_run(const SelectArgs &a, int r, int b, const RowPrep &p, uin
     uint64_t run = kNoKey;   // lane i < m: the i-th best key of the row so far
     int run_e = -1;
     int n_valid = 0;
-    for (int j0 = 0; j0 < n_e; j0 += 32 * kSpKpc) {
-        uint64_t c[kSpKpc];
-        int ce[kSpKpc];
-        int tk[kSpKpc];
-        float sv[kSpKpc];
+    for (int j0 = 0; j0 < n_e; j0 += 32 * KPC) {
+        uint64_t c[KPC];
+        int ce[KPC];
+        int tk[KPC];
+        float sv[KPC];
         if (j0 == 0) {
 #pragma unroll
-            for (int u = 0; u < kSpKpc; ++u) {
+            for (int u = 0; u < KPC; ++u) {
                 tk[u] = p.tk0[u];
                 sv[u] = sv0[u];
             }
         } else {
 #pragma unroll
-            for (int u = 0; u < kSpKpc; ++u) {   // the entries' tokens (one round trip) ...
+            for (int u = 0; u < KPC; ++u) {   // the entries' tokens (one round trip) ...
                 const int j = j0 + u * 32 + lane;
                 tk[u] = (j < n_e && live) ? tokp[j] : -1;
             }
 #pragma unroll
-            for (int u = 0; u < kSpKpc; ++u)     // ... then their scores (another)
+            for (int u = 0; u < KPC; ++u)     // ... then their scores (another)
                 sv[u] = (tk[u] >= 0 && tk[u] < V) ? __ldg(x + tk[u]) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < kSpKpc; ++u) {
+        for (int u = 0; u < KPC; ++u) {
             const int j = j0 + u * 32 + lane;
             c[u] = kNoKey;
             ce[u] = -1;
@@ -1417,7 +1424,7 @@ __device__ __forceinline__ void select_request(const SelectArgs &a, int r, int n
 
 // Phase 1: sp_parts CTAs per request of sp_rows (<= W) beams, one warp per
 // beam, each with a ring of RING stages.
-template <int W, int kMinBlocks, int RING>
+template <int W, int kMinBlocks, int RING, int KPC>
 __global__ void __launch_bounds__(W * 32, kMinBlocks) select_rows_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t ring_bar[W][RING];
@@ -1431,11 +1438,11 @@ __global__ void __launch_bounds__(W * 32, kMinBlocks) select_rows_kernel(SelectA
     uint8_t *area = smem + (size_t)warp * ring_warp_bytes(RING);
     // the mask lookups (beam state and tables only) go before the wait when
     // the kernel before writes no beam state (the scores always follow it)
-    RowPrep p;
+    RowPrep<KPC> p;
     auto prep = [&]() {
         const int n_live = min(max(a.n_live[r], 0), dm.BW);
         const int base = a.mask_kind == XGR_MASK_CSR ? a.row_ptr[rb] : 0;
-        if (has_row) p = row_prep<RING>(a, r, b, n_live, base, area);
+        if (has_row) p = row_prep<RING, KPC>(a, r, b, n_live, base, area);
     };
     // The pick kernel (the only kernel launched after this one) may start at
     // once: before its own wait it touches no global memory, so this kernel
@@ -1444,7 +1451,7 @@ __global__ void __launch_bounds__(W * 32, kMinBlocks) select_rows_kernel(SelectA
     if (a.prep_early) prep();
     griddep_wait();
     if (!a.prep_early) prep();
-    if (has_row) row_run<RING>(a, r, b, p, a.keys + (int64_t)r * a.key_cap, area, ring_bar[warp]);
+    if (has_row) row_run<RING, KPC>(a, r, b, p, a.keys + (int64_t)r * a.key_cap, area, ring_bar[warp]);
 }
 
 // Phase 2: one CTA per request.  It starts while the rows kernel runs (on the
@@ -1825,8 +1832,8 @@ static cudaError_t launch_beam_select_impl(const SelectArgs &a_in, cudaStream_t 
     const size_t rows_smem = (size_t)R * ring_warp_bytes(ring);
     const size_t pick_smem = sparse_pick_smem(dm, a.head_m);
     if (pick_smem > (220u << 10)) return cudaErrorInvalidValue;
-    auto *rows_kernel = wide ? select_rows_kernel<kRowWarpsWide, 1, kRingWide>
-                             : select_rows_kernel<kRowWarpsNarrow, 3, kRingNarrow>;
+    auto *rows_kernel = wide ? select_rows_kernel<kRowWarpsWide, 1, kRingWide, kSpKpcWide>
+                             : select_rows_kernel<kRowWarpsNarrow, 3, kRingNarrow, kSpKpc>;
     cudaError_t e = ensure_smem(rows_kernel, rows_smem);
     if (e == cudaSuccess) e = ensure_smem(select_pick_kernel, pick_smem);
     if (e != cudaSuccess) return e;
